@@ -1,0 +1,255 @@
+"""CPU oracle of the MoE layer. TEST INFRASTRUCTURE ONLY.
+
+Only tests/, the package's smoke check and the benchmark's CPU-baseline leg
+import this module. The product path (the CUDA library and its binding) never
+imports it. The arithmetic lives in moe_oracle.c (plain C, explicit loops).
+This file compiles that source with gcc and marshals numpy arrays to it.
+
+Every function returns numpy arrays and takes host arrays only:
+  bf16 tensors as uint16 bit patterns, fp32 as float32, indices as int32.
+ctypes releases the GIL during each call, so `moe_forward_tokens` can spread
+per-token work over host threads. Each token is independent, so the results
+do not depend on the thread count.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+from concurrent.futures import ThreadPoolExecutor
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB_DIR = os.path.join(_HERE, "_build")
+_LIB = os.path.join(_LIB_DIR, "libmoe_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile moe_oracle.c into oracle/_build/libmoe_oracle.so (gcc, -O2,
+    no fast-math, no FMA contraction)."""
+    os.makedirs(_LIB_DIR, exist_ok=True)
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-ffp-contract=off",
+                               "-fno-fast-math", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            i64, i32, f32 = ctypes.c_int64, ctypes.c_int, ctypes.c_float
+            lib.oracle_round_bf16.argtypes = [ctypes.c_double]
+            lib.oracle_round_bf16.restype = ctypes.c_uint16
+            lib.oracle_router_topk.argtypes = [P, i64, i32, i32, i32, i32, f32, P, P, P, P, P, P]
+            lib.oracle_router_topk.restype = i32
+            lib.oracle_dispatch.argtypes = [P, i64, i32, i32, P, P, P]
+            lib.oracle_dispatch.restype = i32
+            lib.oracle_gather_rows.argtypes = [P, i32, P, i64, P]
+            lib.oracle_gather_rows.restype = None
+            lib.oracle_expert_mlp.argtypes = [P, i64, i32, i32, P, P, i32, P, P, P, P]
+            lib.oracle_expert_mlp.restype = None
+            lib.oracle_grouped_mlp.argtypes = [P, P, i32, i32, i32, P, P, i32, P]
+            lib.oracle_grouped_mlp.restype = None
+            lib.oracle_combine.argtypes = [P, P, P, i64, i32, i32, P, P]
+            lib.oracle_combine.restype = None
+            lib.oracle_moe_forward_tokens.argtypes = [P, P, i32, i32, i32, i32, i32, i32, f32, P,
+                                                      P, P, P, P, i32, P, i64, P]
+            lib.oracle_moe_forward_tokens.restype = i32
+            lib.oracle_moe_backward.argtypes = [P, i64, i32, i32, i32, i32, P, P, P, P, P, i32,
+                                                i32, P, i64, P, P, P, P]
+            lib.oracle_moe_backward.restype = i32
+            _lib = lib
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return None if a is None else np.ascontiguousarray(a, dtype=dtype)
+
+
+def bf16_bits(t) -> np.ndarray:
+    """A torch bf16 tensor (any device) -> uint16 numpy array of its bits."""
+    import torch
+    return t.detach().to("cpu").contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def bits_to_float(b: np.ndarray) -> np.ndarray:
+    """uint16 bf16 bit patterns -> float64 values."""
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def round_bf16(v: float) -> int:
+    return int(_load().oracle_round_bf16(float(v)))
+
+
+def router_topk(logits, k, score=0, renormalize=True, scaling=1.0, expert_bias=None,
+                with_map=True):
+    lib = _load()
+    logits = _c(logits, np.float32)
+    T, E = logits.shape
+    idx = np.zeros((T, k), np.int32)
+    prob = np.zeros((T, k), np.float32)
+    rmap = np.zeros((T, E), np.uint8) if with_map else None
+    counts = np.zeros(E, np.int32)
+    offsets = np.zeros(E + 1, np.int32)
+    rc = lib.oracle_router_topk(_p(logits), T, E, k, score, int(renormalize), scaling,
+                                _p(_c(expert_bias, np.float32)), _p(idx), _p(prob), _p(rmap),
+                                _p(counts), _p(offsets))
+    if rc:
+        raise ValueError(f"oracle_router_topk rejected its arguments ({rc})")
+    return dict(topk_idx=idx, topk_prob=prob, routing_map=rmap, counts=counts, offsets=offsets)
+
+
+def dispatch(topk_idx, offsets, E):
+    lib = _load()
+    topk_idx = _c(topk_idx, np.int32)
+    offsets = _c(offsets, np.int32)
+    T, k = topk_idx.shape
+    A = int(offsets[E])
+    sorted_token = np.full(A, -1, np.int32)
+    row_of = np.full((T, k), -1, np.int32)
+    rc = lib.oracle_dispatch(_p(topk_idx), T, k, E, _p(offsets), _p(sorted_token), _p(row_of))
+    if rc:
+        raise ValueError(f"oracle_dispatch: invalid routing ({rc})")
+    return sorted_token, row_of
+
+
+def gather_rows(x_bits, sorted_token):
+    lib = _load()
+    x_bits = _c(x_bits, np.uint16)
+    sorted_token = _c(sorted_token, np.int32)
+    H = x_bits.shape[1]
+    out = np.zeros((sorted_token.shape[0], H), np.uint16)
+    lib.oracle_gather_rows(_p(x_bits), H, _p(sorted_token), sorted_token.shape[0], _p(out))
+    return out
+
+
+def expert_mlp(x_bits, w_gu_bits, w_d_bits, round_h=True, want_intermediates=False):
+    """One expert on rows x_bits [n,H]; w_gu_bits [H,2I], w_d_bits [I,H]."""
+    lib = _load()
+    x_bits = _c(x_bits, np.uint16)
+    w_gu_bits = _c(w_gu_bits, np.uint16)
+    w_d_bits = _c(w_d_bits, np.uint16)
+    n, H = x_bits.shape
+    I = w_d_bits.shape[0]
+    y = np.zeros((n, H), np.float64)
+    g = u = h = None
+    if want_intermediates:
+        g, u, h = (np.zeros((n, I), np.float64) for _ in range(3))
+    lib.oracle_expert_mlp(_p(x_bits), n, H, I, _p(w_gu_bits), _p(w_d_bits), int(round_h),
+                          _p(y), _p(g), _p(u), _p(h))
+    return (y, g, u, h) if want_intermediates else y
+
+
+def grouped_mlp(x_perm_bits, offsets, w_gu_bits, w_d_bits, round_h=True):
+    lib = _load()
+    x_perm_bits = _c(x_perm_bits, np.uint16)
+    offsets = _c(offsets, np.int32)
+    w_gu_bits = _c(w_gu_bits, np.uint16)
+    w_d_bits = _c(w_d_bits, np.uint16)
+    E, H, I2 = w_gu_bits.shape
+    y = np.zeros((x_perm_bits.shape[0], H), np.float64)
+    lib.oracle_grouped_mlp(_p(x_perm_bits), _p(offsets), E, H, I2 // 2, _p(w_gu_bits),
+                           _p(w_d_bits), int(round_h), _p(y))
+    return y
+
+
+def combine(y_perm, row_of, probs=None, shared=None):
+    lib = _load()
+    y_perm = _c(y_perm, np.float64)
+    row_of = _c(row_of, np.int32)
+    T, k = row_of.shape
+    H = y_perm.shape[1]
+    out = np.zeros((T, H), np.float64)
+    lib.oracle_combine(_p(y_perm), _p(row_of), _p(_c(probs, np.float32)), T, k, H,
+                       _p(_c(shared, np.float64)), _p(out))
+    return out
+
+
+def _chunks(tokens, threads):
+    tokens = np.asarray(tokens, np.int64)
+    n = max(1, min(threads, len(tokens)))
+    return [c for c in np.array_split(tokens, n) if len(c)]
+
+
+def moe_forward_tokens(x_bits, logits, w_gu_bits, w_d_bits, k, tokens=None, score=0,
+                       renormalize=True, scaling=1.0, expert_bias=None, shared_gu_bits=None,
+                       shared_d_bits=None, round_h=True, threads=None):
+    """The layer by its plain definition for the listed tokens (default: all);
+    rows of the result are in list order (float64 [n, H])."""
+    lib = _load()
+    x_bits = _c(x_bits, np.uint16)
+    logits = _c(logits, np.float32)
+    w_gu_bits = _c(w_gu_bits, np.uint16)
+    w_d_bits = _c(w_d_bits, np.uint16)
+    shared_gu_bits = _c(shared_gu_bits, np.uint16)
+    shared_d_bits = _c(shared_d_bits, np.uint16)
+    expert_bias = _c(expert_bias, np.float32)
+    T, H = x_bits.shape
+    E, _, I2 = w_gu_bits.shape
+    if tokens is None:
+        tokens = np.arange(T, dtype=np.int64)
+    tokens = np.asarray(tokens, np.int64)
+    out = np.zeros((len(tokens), H), np.float64)
+    threads = threads or os.cpu_count() or 1
+
+    def run(chunk_and_start):
+        chunk, start = chunk_and_start
+        o = np.zeros((len(chunk), H), np.float64)
+        rc = lib.oracle_moe_forward_tokens(_p(x_bits), _p(logits), H, I2 // 2, E, k, score,
+                                           int(renormalize), scaling, _p(expert_bias),
+                                           _p(w_gu_bits), _p(w_d_bits), _p(shared_gu_bits),
+                                           _p(shared_d_bits), int(round_h), _p(chunk), len(chunk),
+                                           _p(o))
+        if rc:
+            raise ValueError(f"oracle_moe_forward_tokens failed ({rc})")
+        out[start:start + len(chunk)] = o
+
+    chunks = _chunks(tokens, threads)
+    starts = np.cumsum([0] + [len(c) for c in chunks[:-1]])
+    with ThreadPoolExecutor(max_workers=len(chunks)) as ex:
+        list(ex.map(run, zip(chunks, starts)))
+    return out
+
+
+def moe_backward(x_bits, topk_idx, topk_prob, w_gu_bits, w_d_bits, dout_bits, round_h=True,
+                 only_expert=-1, tokens=None, want=("dx", "dw_gate_up", "dw_down", "dprob")):
+    """Gradients of the layer for a given routing (see moe_oracle.c)."""
+    lib = _load()
+    x_bits = _c(x_bits, np.uint16)
+    topk_idx = _c(topk_idx, np.int32)
+    topk_prob = _c(topk_prob, np.float32)
+    w_gu_bits = _c(w_gu_bits, np.uint16)
+    w_d_bits = _c(w_d_bits, np.uint16)
+    dout_bits = _c(dout_bits, np.uint16)
+    T, H = x_bits.shape
+    E, _, I2 = w_gu_bits.shape
+    I = I2 // 2
+    k = topk_idx.shape[1]
+    tl = None if tokens is None else np.asarray(tokens, np.int64)
+    nt = T if tl is None else len(tl)
+    dx = np.zeros((nt, H)) if "dx" in want else None
+    ne = 1 if only_expert >= 0 else E
+    dwgu = np.zeros((ne, H, I2)) if "dw_gate_up" in want else None
+    dwd = np.zeros((ne, I, H)) if "dw_down" in want else None
+    dprob = np.zeros((nt, k)) if "dprob" in want else None
+    rc = lib.oracle_moe_backward(_p(x_bits), T, H, I, E, k, _p(topk_idx), _p(topk_prob),
+                                 _p(w_gu_bits), _p(w_d_bits), _p(dout_bits), int(round_h),
+                                 only_expert, _p(tl), 0 if tl is None else len(tl),
+                                 _p(dx), _p(dwgu), _p(dwd), _p(dprob))
+    if rc:
+        raise ValueError(f"oracle_moe_backward failed ({rc})")
+    return dict(dx=dx, dw_gate_up=dwgu, dw_down=dwd, dprob=dprob)

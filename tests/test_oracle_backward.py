@@ -1,0 +1,137 @@
+"""Pins of the oracle's backward: fp64 finite differences of the oracle's own
+forward, and torch autograd of the layer restated with torch primitives.
+
+Transformer Engine "Mixture of Experts", Example (every stage is
+differentiable). The routing weights are inputs, so their gradient is
+<dout, expert output>.
+"""
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import workloads as wl
+
+
+def setup(T=5, H=16, I=8, E=3, k=2, seed=0):
+    w = wl.WORKLOADS["tiny"].scaled(T=T, H=H, I=I, E=E, k=k, seed=seed)
+    d = wl.make_inputs(w, with_dout=True)
+    return w, d
+
+
+def loss(oracle_lib, w, x, logits_unused, wgu, wd, idx, prob, dout):
+    """L = <dout, out> with out = sum_j p_j MLP_{e_j}(x_t), via the oracle's
+    forward pieces (round_h off, so L is smooth)."""
+    out = np.zeros((w.T, w.H))
+    for t in range(w.T):
+        for j in range(w.k):
+            e = idx[t, j]
+            y = oracle_lib.expert_mlp(x[t:t + 1], wgu[e], wd[e], round_h=False)
+            out[t] += float(prob[t, j]) * y[0]
+    return float((oracle_lib.bits_to_float(dout) * out).sum())
+
+
+def richardson(f, delta):
+    """Central difference with one Richardson step: error O(delta^4)."""
+    d1 = (f(delta) - f(-delta)) / (2 * delta)
+    d2 = (f(2 * delta) - f(-2 * delta)) / (4 * delta)
+    return (4 * d1 - d2) / 3
+
+
+def test_backward_matches_finite_differences(oracle_lib):
+    w, d = setup()
+    bits = oracle_lib.bf16_bits
+    x, wgu, wd, dout = bits(d["x"]), bits(d["w_gate_up"]), bits(d["w_down"]), bits(d["dout"])
+    r = oracle_lib.router_topk(d["logits"].numpy(), w.k)
+    idx, prob = r["topk_idx"], r["topk_prob"]
+    rng = np.random.default_rng(1)
+    c = 0.5          # a perturbed bf16 coordinate is set to c; c +- delta, c +- 2 delta are exact
+    delta = 2.0 ** -6
+
+    def with_value(arr, pos, v):
+        a = arr.copy()
+        a[pos] = oracle_lib.round_bf16(v)
+        assert oracle_lib.bits_to_float(a[pos]) == v
+        return a
+
+    checked = 0
+    for name in ("x", "w_gate_up", "w_down"):
+        base = {"x": x, "w_gate_up": wgu, "w_down": wd}[name]
+        for _ in range(12):
+            pos = tuple(int(rng.integers(0, s)) for s in base.shape)
+            arrs = {"x": x, "w_gate_up": wgu, "w_down": wd}
+            arrs[name] = with_value(base, pos, c)
+            g = oracle_lib.moe_backward(arrs["x"], idx, prob, arrs["w_gate_up"], arrs["w_down"],
+                                        dout, round_h=False)
+            analytic = {"x": g["dx"], "w_gate_up": g["dw_gate_up"], "w_down": g["dw_down"]}[name][pos]
+
+            def f(dl):
+                a2 = dict(arrs)
+                a2[name] = with_value(base, pos, c + dl)
+                return loss(oracle_lib, w, a2["x"], None, a2["w_gate_up"], a2["w_down"], idx, prob, dout)
+            numeric = richardson(f, delta)
+            assert abs(numeric - analytic) <= 1e-6 + 1e-5 * abs(analytic), (name, pos, numeric, analytic)
+            checked += 1
+    # routing weights: fp32 inputs
+    g = oracle_lib.moe_backward(x, idx, prob, wgu, wd, dout, round_h=False)
+    for t in range(w.T):
+        for j in range(w.k):
+            def f(dl):
+                p2 = prob.astype(np.float64).copy()
+                p2[t, j] += dl
+                out = 0.0
+                y = oracle_lib.expert_mlp(x[t:t + 1], wgu[idx[t, j]], wd[idx[t, j]], round_h=False)
+                return float((oracle_lib.bits_to_float(dout[t]) * y[0]).sum() * p2[t, j])
+            numeric = richardson(f, 1e-3)
+            assert abs(numeric - g["dprob"][t, j]) <= 1e-9 + 1e-9 * abs(numeric)
+            checked += 1
+    assert checked == 36 + w.T * w.k
+
+
+@pytest.mark.parametrize("round_h", [False, True])
+def test_backward_matches_torch_autograd(oracle_lib, round_h):
+    w, d = setup(T=24, H=32, I=24, E=5, k=2, seed=3)
+    bits = oracle_lib.bf16_bits
+    r = oracle_lib.router_topk(d["logits"].numpy(), w.k)
+    idx = torch.from_numpy(r["topk_idx"].astype(np.int64))
+    prob = torch.from_numpy(r["topk_prob"]).double().requires_grad_(True)
+    x = d["x"].double().requires_grad_(True)
+    wgu = d["w_gate_up"].double().requires_grad_(True)
+    wd = d["w_down"].double().requires_grad_(True)
+    I = w.I
+    out = torch.zeros(w.T, w.H, dtype=torch.float64)
+    for t in range(w.T):
+        for j in range(w.k):
+            e = int(idx[t, j])
+            h = F.silu(x[t] @ wgu[e][:, :I]) * (x[t] @ wgu[e][:, I:])
+            if round_h:      # straight-through rounding: value rounded, gradient identity
+                h = h + (h.detach().float().to(torch.bfloat16).double() - h.detach())
+            out[t] = out[t] + prob[t, j] * (h @ wd[e])
+    (out * d["dout"].double()).sum().backward()
+    g = oracle_lib.moe_backward(bits(d["x"]), r["topk_idx"], r["topk_prob"], bits(d["w_gate_up"]),
+                                bits(d["w_down"]), bits(d["dout"]), round_h=round_h)
+    np.testing.assert_allclose(g["dx"], x.grad.numpy(), rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(g["dw_gate_up"], wgu.grad.numpy(), rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(g["dw_down"], wd.grad.numpy(), rtol=1e-9, atol=1e-11)
+    np.testing.assert_allclose(g["dprob"], prob.grad.numpy(), rtol=1e-9, atol=1e-11)
+
+
+def test_backward_empty_expert_and_expert_filter(oracle_lib):
+    w, d = setup(T=10, H=16, I=8, E=4, k=1, seed=4)
+    logits = d["logits"].numpy().copy()
+    logits[:, 1] = -1e4
+    r = oracle_lib.router_topk(logits, 1)
+    assert r["counts"][1] == 0
+    bits = oracle_lib.bf16_bits
+    args = (bits(d["x"]), r["topk_idx"], r["topk_prob"], bits(d["w_gate_up"]), bits(d["w_down"]),
+            bits(d["dout"]))
+    g = oracle_lib.moe_backward(*args)
+    assert np.all(g["dw_gate_up"][1] == 0) and np.all(g["dw_down"][1] == 0)
+    for e in range(4):
+        ge = oracle_lib.moe_backward(*args, only_expert=e, want=("dw_gate_up", "dw_down"))
+        np.testing.assert_array_equal(ge["dw_gate_up"][0], g["dw_gate_up"][e])
+        np.testing.assert_array_equal(ge["dw_down"][0], g["dw_down"][e])
+    toks = [7, 2, 9]
+    gt = oracle_lib.moe_backward(*args, tokens=toks, want=("dx", "dprob"))
+    np.testing.assert_array_equal(gt["dx"], g["dx"][toks])
+    np.testing.assert_array_equal(gt["dprob"], g["dprob"][toks])
