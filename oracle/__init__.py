@@ -137,7 +137,7 @@ def gather_rows(x_bits, sorted_token):
     return out
 
 
-def expert_mlp(x_bits, w_gu_bits, w_d_bits, round_h=True, want_intermediates=False):
+def expert_mlp(x_bits, w_gu_bits, w_d_bits, round_bf16=True, want_intermediates=False):
     """One expert on rows x_bits [n,H]; w_gu_bits [H,2I], w_d_bits [I,H]."""
     lib = _load()
     x_bits = _c(x_bits, np.uint16)
@@ -149,12 +149,12 @@ def expert_mlp(x_bits, w_gu_bits, w_d_bits, round_h=True, want_intermediates=Fal
     g = u = h = None
     if want_intermediates:
         g, u, h = (np.zeros((n, I), np.float64) for _ in range(3))
-    lib.oracle_expert_mlp(_p(x_bits), n, H, I, _p(w_gu_bits), _p(w_d_bits), int(round_h),
+    lib.oracle_expert_mlp(_p(x_bits), n, H, I, _p(w_gu_bits), _p(w_d_bits), int(round_bf16),
                           _p(y), _p(g), _p(u), _p(h))
     return (y, g, u, h) if want_intermediates else y
 
 
-def grouped_mlp(x_perm_bits, offsets, w_gu_bits, w_d_bits, round_h=True):
+def grouped_mlp(x_perm_bits, offsets, w_gu_bits, w_d_bits, round_bf16=True):
     lib = _load()
     x_perm_bits = _c(x_perm_bits, np.uint16)
     offsets = _c(offsets, np.int32)
@@ -163,7 +163,7 @@ def grouped_mlp(x_perm_bits, offsets, w_gu_bits, w_d_bits, round_h=True):
     E, H, I2 = w_gu_bits.shape
     y = np.zeros((x_perm_bits.shape[0], H), np.float64)
     lib.oracle_grouped_mlp(_p(x_perm_bits), _p(offsets), E, H, I2 // 2, _p(w_gu_bits),
-                           _p(w_d_bits), int(round_h), _p(y))
+                           _p(w_d_bits), int(round_bf16), _p(y))
     return y
 
 
@@ -187,7 +187,7 @@ def _chunks(tokens, threads):
 
 def moe_forward_tokens(x_bits, logits, w_gu_bits, w_d_bits, k, tokens=None, score=0,
                        renormalize=True, scaling=1.0, expert_bias=None, shared_gu_bits=None,
-                       shared_d_bits=None, round_h=True, threads=None):
+                       shared_d_bits=None, round_bf16=True, threads=None):
     """The layer by its plain definition for the listed tokens (default: all);
     rows of the result are in list order (float64 [n, H])."""
     lib = _load()
@@ -212,7 +212,7 @@ def moe_forward_tokens(x_bits, logits, w_gu_bits, w_d_bits, k, tokens=None, scor
         rc = lib.oracle_moe_forward_tokens(_p(x_bits), _p(logits), H, I2 // 2, E, k, score,
                                            int(renormalize), scaling, _p(expert_bias),
                                            _p(w_gu_bits), _p(w_d_bits), _p(shared_gu_bits),
-                                           _p(shared_d_bits), int(round_h), _p(chunk), len(chunk),
+                                           _p(shared_d_bits), int(round_bf16), _p(chunk), len(chunk),
                                            _p(o))
         if rc:
             raise ValueError(f"oracle_moe_forward_tokens failed ({rc})")
@@ -225,7 +225,7 @@ def moe_forward_tokens(x_bits, logits, w_gu_bits, w_d_bits, k, tokens=None, scor
     return out
 
 
-def moe_backward(x_bits, topk_idx, topk_prob, w_gu_bits, w_d_bits, dout_bits, round_h=True,
+def moe_backward(x_bits, topk_idx, topk_prob, w_gu_bits, w_d_bits, dout_bits, round_bf16=True,
                  only_expert=-1, tokens=None, want=("dx", "dw_gate_up", "dw_down", "dprob")):
     """Gradients of the layer for a given routing (see moe_oracle.c)."""
     lib = _load()
@@ -247,7 +247,7 @@ def moe_backward(x_bits, topk_idx, topk_prob, w_gu_bits, w_d_bits, dout_bits, ro
     dwd = np.zeros((ne, I, H)) if "dw_down" in want else None
     dprob = np.zeros((nt, k)) if "dprob" in want else None
     rc = lib.oracle_moe_backward(_p(x_bits), T, H, I, E, k, _p(topk_idx), _p(topk_prob),
-                                 _p(w_gu_bits), _p(w_d_bits), _p(dout_bits), int(round_h),
+                                 _p(w_gu_bits), _p(w_d_bits), _p(dout_bits), int(round_bf16),
                                  only_expert, _p(tl), 0 if tl is None else len(tl),
                                  _p(dx), _p(dwgu), _p(dwd), _p(dprob))
     if rc:

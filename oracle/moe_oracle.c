@@ -22,9 +22,13 @@
  *  - Router: fp32 throughout. [TE] Router says all internal math runs in FP32.
  *  - Expert MLP, combine and backward: fp64 accumulation. The pages do not fix
  *    it. The bf16 inputs are exact in fp64.
- *  - The SwiGLU intermediate h is rounded to bf16 when round_h != 0. This is
- *    the reading that FC2 reads a bf16 intermediate from memory ([TE] Grouped
- *    MLP). round_h = 0 keeps it exact; finite-difference checks use that.
+ *  - With round_bf16 != 0, the two tensors that the pages' bf16 pipeline
+ *    stores are rounded to bf16: the SwiGLU intermediate h, because FC2 reads
+ *    it from memory ([TE] Grouped MLP), and the expert output y, because FC2
+ *    is a bf16 grouped linear whose output token combine merges with fp32
+ *    weights ([TE] Grouped GEMM and Token combine; [TT] _grouped_mm returns
+ *    bf16; [MIX] the loop's F.linear output). round_bf16 = 0 keeps both exact;
+ *    the finite-difference checks use that.
  *
  * Pins. Each function is checked in tests/ against something other than
  * itself: brute-force sorts, invariants, closed forms, a special case that
@@ -232,13 +236,13 @@ static double silu(double g) { return g / (1.0 + exp(-g)); }
  * are the first and second halves of the FC1 output. [TT] GroupedExperts:
  * silu(x w1) * (x w3), times w2.
  *   g = x . Wgu[:, 0:I]    u = x . Wgu[:, I:2I]    (Wgu is [H, 2I], row-major)
- *   h = silu(g) * u        (rounded to bf16 when round_h)
- *   y = h . Wd             (Wd is [I, H], row-major)
+ *   h = silu(g) * u        (rounded to bf16 when round_bf16)
+ *   y = h . Wd             (Wd is [I, H], row-major; rounded to bf16 when round_bf16)
  * Accumulation is fp64, in ascending index order. g, u, h are optional
  * outputs.
  */
 void oracle_expert_mlp(const uint16_t* x, int64_t n, int H, int I,
-                       const uint16_t* w_gate_up, const uint16_t* w_down, int round_h,
+                       const uint16_t* w_gate_up, const uint16_t* w_down, int round_bf16,
                        double* y, double* g_out, double* u_out, double* h_out)
 {
     double* g = (double*)malloc(sizeof(double) * (size_t)I);
@@ -257,7 +261,7 @@ void oracle_expert_mlp(const uint16_t* x, int64_t n, int H, int I,
         }
         for (int i = 0; i < I; i++) {
             double v = silu(g[i]) * u[i];
-            h[i] = round_h ? bf16_to_double(double_to_bf16(v)) : v;
+            h[i] = round_bf16 ? bf16_to_double(double_to_bf16(v)) : v;
         }
         double* yr = y + r * H;
         for (int c = 0; c < H; c++) yr[c] = 0.0;
@@ -265,6 +269,8 @@ void oracle_expert_mlp(const uint16_t* x, int64_t n, int H, int I,
             const uint16_t* wrow = w_down + (int64_t)i * H;
             for (int c = 0; c < H; c++) yr[c] += h[i] * bf16_to_double(wrow[c]);
         }
+        if (round_bf16)
+            for (int c = 0; c < H; c++) yr[c] = bf16_to_double(double_to_bf16(yr[c]));
         if (g_out) memcpy(g_out + r * I, g, sizeof(double) * (size_t)I);
         if (u_out) memcpy(u_out + r * I, u, sizeof(double) * (size_t)I);
         if (h_out) memcpy(h_out + r * I, h, sizeof(double) * (size_t)I);
@@ -280,7 +286,7 @@ void oracle_expert_mlp(const uint16_t* x, int64_t n, int H, int I,
  * block is skipped.
  */
 void oracle_grouped_mlp(const uint16_t* x_perm, const int32_t* offsets, int E, int H, int I,
-                        const uint16_t* w_gate_up, const uint16_t* w_down, int round_h,
+                        const uint16_t* w_gate_up, const uint16_t* w_down, int round_bf16,
                         double* y_perm)
 {
     for (int e = 0; e < E; e++) {
@@ -288,7 +294,7 @@ void oracle_grouped_mlp(const uint16_t* x_perm, const int32_t* offsets, int E, i
         if (n <= 0) continue;
         oracle_expert_mlp(x_perm + r0 * H, n, H, I,
                           w_gate_up + (int64_t)e * H * 2 * I, w_down + (int64_t)e * I * H,
-                          round_h, y_perm + r0 * H, NULL, NULL, NULL);
+                          round_bf16, y_perm + r0 * H, NULL, NULL, NULL);
     }
 }
 
@@ -329,7 +335,7 @@ int oracle_moe_forward_tokens(const uint16_t* x, const float* logits, int H, int
                               int score_fn, int renormalize, float scaling, const float* expert_bias,
                               const uint16_t* w_gate_up, const uint16_t* w_down,
                               const uint16_t* shared_gate_up, const uint16_t* shared_down,
-                              int round_h, const int64_t* token_list, int64_t n_tokens, double* out)
+                              int round_bf16, const int64_t* token_list, int64_t n_tokens, double* out)
 {
     int32_t* idx = (int32_t*)malloc(sizeof(int32_t) * (size_t)k);
     float* p = (float*)malloc(sizeof(float) * (size_t)k);
@@ -343,7 +349,7 @@ int oracle_moe_forward_tokens(const uint16_t* x, const float* logits, int H, int
                                 expert_bias, idx, p, NULL, cnt, off);
         double* o = out + n * H;
         if (shared_gate_up) {
-            oracle_expert_mlp(x + t * H, 1, H, I, shared_gate_up, shared_down, round_h, o,
+            oracle_expert_mlp(x + t * H, 1, H, I, shared_gate_up, shared_down, round_bf16, o,
                               NULL, NULL, NULL);
         } else {
             for (int c = 0; c < H; c++) o[c] = 0.0;
@@ -351,7 +357,7 @@ int oracle_moe_forward_tokens(const uint16_t* x, const float* logits, int H, int
         for (int j = 0; j < k; j++) {
             int e = idx[j];
             oracle_expert_mlp(x + t * H, 1, H, I, w_gate_up + (int64_t)e * H * 2 * I,
-                              w_down + (int64_t)e * I * H, round_h, y, NULL, NULL, NULL);
+                              w_down + (int64_t)e * I * H, round_bf16, y, NULL, NULL, NULL);
             for (int c = 0; c < H; c++) o[c] += (double)p[j] * y[c];
         }
     }
@@ -367,7 +373,7 @@ int oracle_moe_forward_tokens(const uint16_t* x, const float* logits, int H, int
  * routing (topk_idx, topk_prob) and upstream gradient dout. It is the chain
  * rule applied to the forward above. [TE] Example: every stage is
  * differentiable. The routing weights are an input here, so nothing flows into
- * the logits. The bf16 rounding of h is treated as the identity.
+ * the logits. The bf16 rounding of h and y is treated as the identity.
  * Per assignment (t, j) with e = topk_idx[t,j] and p = topk_prob[t,j]:
  *   y = MLP_e(x_t);           dprob[t,j] = <dout_t, y>
  *   dy = p * dout_t;          dWd[e]   += h^T dy
@@ -386,7 +392,7 @@ int oracle_moe_forward_tokens(const uint16_t* x, const float* logits, int H, int
 int oracle_moe_backward(const uint16_t* x, int64_t T, int H, int I, int E, int k,
                         const int32_t* topk_idx, const float* topk_prob,
                         const uint16_t* w_gate_up, const uint16_t* w_down, const uint16_t* dout,
-                        int round_h, int only_expert, const int64_t* token_list, int64_t n_tokens,
+                        int round_bf16, int only_expert, const int64_t* token_list, int64_t n_tokens,
                         double* dx, double* dw_gate_up, double* dw_down, double* dprob)
 {
     int64_t nt = token_list ? n_tokens : T;
@@ -414,7 +420,7 @@ int oracle_moe_backward(const uint16_t* x, int64_t T, int H, int I, int E, int k
             double p = (double)topk_prob[t * k + j];
             const uint16_t* wgu = w_gate_up + (int64_t)e * H * 2 * I;
             const uint16_t* wd = w_down + (int64_t)e * I * H;
-            oracle_expert_mlp(xt, 1, H, I, wgu, wd, round_h, y, g, u, h);
+            oracle_expert_mlp(xt, 1, H, I, wgu, wd, round_bf16, y, g, u, h);
             if (dprob) {
                 double s = 0.0;
                 for (int c = 0; c < H; c++) s += bf16_to_double(dot[c]) * y[c];

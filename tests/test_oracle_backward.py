@@ -21,12 +21,12 @@ def setup(T=5, H=16, I=8, E=3, k=2, seed=0):
 
 def loss(oracle_lib, w, x, logits_unused, wgu, wd, idx, prob, dout):
     """L = <dout, out> with out = sum_j p_j MLP_{e_j}(x_t), via the oracle's
-    forward pieces (round_h off, so L is smooth)."""
+    forward pieces (round_bf16 off, so L is smooth)."""
     out = np.zeros((w.T, w.H))
     for t in range(w.T):
         for j in range(w.k):
             e = idx[t, j]
-            y = oracle_lib.expert_mlp(x[t:t + 1], wgu[e], wd[e], round_h=False)
+            y = oracle_lib.expert_mlp(x[t:t + 1], wgu[e], wd[e], round_bf16=False)
             out[t] += float(prob[t, j]) * y[0]
     return float((oracle_lib.bits_to_float(dout) * out).sum())
 
@@ -62,7 +62,7 @@ def test_backward_matches_finite_differences(oracle_lib):
             arrs = {"x": x, "w_gate_up": wgu, "w_down": wd}
             arrs[name] = with_value(base, pos, c)
             g = oracle_lib.moe_backward(arrs["x"], idx, prob, arrs["w_gate_up"], arrs["w_down"],
-                                        dout, round_h=False)
+                                        dout, round_bf16=False)
             analytic = {"x": g["dx"], "w_gate_up": g["dw_gate_up"], "w_down": g["dw_down"]}[name][pos]
 
             def f(dl):
@@ -73,14 +73,14 @@ def test_backward_matches_finite_differences(oracle_lib):
             assert abs(numeric - analytic) <= 1e-6 + 1e-5 * abs(analytic), (name, pos, numeric, analytic)
             checked += 1
     # routing weights: fp32 inputs
-    g = oracle_lib.moe_backward(x, idx, prob, wgu, wd, dout, round_h=False)
+    g = oracle_lib.moe_backward(x, idx, prob, wgu, wd, dout, round_bf16=False)
     for t in range(w.T):
         for j in range(w.k):
             def f(dl):
                 p2 = prob.astype(np.float64).copy()
                 p2[t, j] += dl
                 out = 0.0
-                y = oracle_lib.expert_mlp(x[t:t + 1], wgu[idx[t, j]], wd[idx[t, j]], round_h=False)
+                y = oracle_lib.expert_mlp(x[t:t + 1], wgu[idx[t, j]], wd[idx[t, j]], round_bf16=False)
                 return float((oracle_lib.bits_to_float(dout[t]) * y[0]).sum() * p2[t, j])
             numeric = richardson(f, 1e-3)
             assert abs(numeric - g["dprob"][t, j]) <= 1e-9 + 1e-9 * abs(numeric)
@@ -88,8 +88,8 @@ def test_backward_matches_finite_differences(oracle_lib):
     assert checked == 36 + w.T * w.k
 
 
-@pytest.mark.parametrize("round_h", [False, True])
-def test_backward_matches_torch_autograd(oracle_lib, round_h):
+@pytest.mark.parametrize("round_bf16", [False, True])
+def test_backward_matches_torch_autograd(oracle_lib, round_bf16):
     w, d = setup(T=24, H=32, I=24, E=5, k=2, seed=3)
     bits = oracle_lib.bf16_bits
     r = oracle_lib.router_topk(d["logits"].numpy(), w.k)
@@ -104,12 +104,15 @@ def test_backward_matches_torch_autograd(oracle_lib, round_h):
         for j in range(w.k):
             e = int(idx[t, j])
             h = F.silu(x[t] @ wgu[e][:, :I]) * (x[t] @ wgu[e][:, I:])
-            if round_h:      # straight-through rounding: value rounded, gradient identity
+            if round_bf16:      # straight-through rounding: value rounded, gradient identity
                 h = h + (h.detach().float().to(torch.bfloat16).double() - h.detach())
-            out[t] = out[t] + prob[t, j] * (h @ wd[e])
+            y = h @ wd[e]
+            if round_bf16:
+                y = y + (y.detach().float().to(torch.bfloat16).double() - y.detach())
+            out[t] = out[t] + prob[t, j] * y
     (out * d["dout"].double()).sum().backward()
     g = oracle_lib.moe_backward(bits(d["x"]), r["topk_idx"], r["topk_prob"], bits(d["w_gate_up"]),
-                                bits(d["w_down"]), bits(d["dout"]), round_h=round_h)
+                                bits(d["w_down"]), bits(d["dout"]), round_bf16=round_bf16)
     np.testing.assert_allclose(g["dx"], x.grad.numpy(), rtol=1e-9, atol=1e-11)
     np.testing.assert_allclose(g["dw_gate_up"], wgu.grad.numpy(), rtol=1e-9, atol=1e-11)
     np.testing.assert_allclose(g["dw_down"], wd.grad.numpy(), rtol=1e-9, atol=1e-11)

@@ -20,29 +20,34 @@ def small(name="tiny", **kw):
     return w, d
 
 
-def dense_swiglu_torch(x, wgu, wd, round_h):
+def dense_swiglu_torch(x, wgu, wd, round_bf16):
     """A dense SwiGLU MLP from torch primitives, in fp64: the special case
     the layer reduces to with one expert."""
     x64, wgu64, wd64 = x.double(), wgu.double(), wd.double()
     I = wd.shape[0]
     h = F.silu(x64 @ wgu64[:, :I]) * (x64 @ wgu64[:, I:])
-    if round_h:
+    if round_bf16:
         h = h.float().to(torch.bfloat16).double()
-    return (h @ wd64).numpy()
+    y = h @ wd64
+    if round_bf16:
+        y = y.float().to(torch.bfloat16).double()
+    return y.numpy()
 
 
-@pytest.mark.parametrize("round_h", [False, True])
-def test_single_expert_is_a_dense_swiglu_mlp(oracle_lib, round_h):
+@pytest.mark.parametrize("round_bf16", [False, True])
+def test_single_expert_is_a_dense_swiglu_mlp(oracle_lib, round_bf16):
     # H != I != 2I, so a transposed operand or a swapped gate/up fails
     w, d = small(T=40, H=48, I=40, E=1, k=1)
     bits = oracle_lib.bf16_bits
     out = oracle_lib.moe_forward_tokens(bits(d["x"]), d["logits"].numpy(), bits(d["w_gate_up"]),
-                                        bits(d["w_down"]), 1, round_h=round_h)
-    ref = dense_swiglu_torch(d["x"], d["w_gate_up"][0], d["w_down"][0], round_h)
-    if round_h:
-        # torch rounds h through fp32; a rare double-rounding tie moves h by one
-        # bf16 ulp, so compare to a tolerance far below any real defect
-        np.testing.assert_allclose(out, ref, rtol=1e-3, atol=1e-4)
+                                        bits(d["w_down"]), 1, round_bf16=round_bf16)
+    ref = dense_swiglu_torch(d["x"], d["w_gate_up"][0], d["w_down"][0], round_bf16)
+    if round_bf16:
+        # torch rounds through fp32, so a rare double-rounding tie can move h or
+        # y by one bf16 ulp: almost every element is equal, and none is further
+        # than one ulp away
+        assert np.mean(out == ref) > 0.99
+        np.testing.assert_allclose(out, ref, rtol=2.0 ** -7, atol=1e-6)
     else:
         np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12)
 
@@ -54,7 +59,7 @@ def test_identical_experts_reduce_to_dense_mlp(oracle_lib):
     wd = d["w_down"][:1].expand(6, -1, -1).contiguous()
     bits = oracle_lib.bf16_bits
     out = oracle_lib.moe_forward_tokens(bits(d["x"]), d["logits"].numpy(), bits(wgu), bits(wd), 3,
-                                        round_h=False)
+                                        round_bf16=False)
     ref = dense_swiglu_torch(d["x"], wgu[0], wd[0], False)
     np.testing.assert_allclose(out, ref, rtol=1e-6, atol=1e-7)
 
@@ -62,7 +67,7 @@ def test_identical_experts_reduce_to_dense_mlp(oracle_lib):
 def test_shared_expert_adds_a_dense_mlp(oracle_lib):
     w, d = small("llama4_17bx16e", T=20, H=32, I=16, E=4)
     bits = oracle_lib.bf16_bits
-    kw = dict(score=w.score, renormalize=w.renormalize, round_h=False)
+    kw = dict(score=w.score, renormalize=w.renormalize, round_bf16=False)
     routed = oracle_lib.moe_forward_tokens(bits(d["x"]), d["logits"].numpy(), bits(d["w_gate_up"]),
                                            bits(d["w_down"]), 1, **kw)
     both = oracle_lib.moe_forward_tokens(bits(d["x"]), d["logits"].numpy(), bits(d["w_gate_up"]),
