@@ -1,0 +1,216 @@
+/*
+ * moe_b200.h -- C ABI of the single-GPU Mixture-of-Experts layer for B200
+ * (sm_100a): router -> dispatch (permute) -> grouped SwiGLU expert MLP ->
+ * combine, plus the backward of the grouped MLP.
+ *
+ * The stages follow the Transformer Engine documentation page "Mixture of
+ * Experts" (sections Introduction, Router, Token dispatch, Token combine,
+ * Token probabilities, Grouped GEMM, Grouped MLP and "Example: MoE layer on a
+ * single device"). The expert MLP is the SwiGLU of the te_mixtral.py example
+ * (_expert_ffn) and of torchtitan's GroupedExperts.
+ *
+ * Conventions, for every entry point:
+ *  - Pointers. Every tensor pointer is DEVICE memory that the caller
+ *    allocates and owns. Each must be 16-byte aligned, except routing_map.
+ *    The library never allocates, frees or synchronises on these calls.
+ *    Scratch memory is the caller's `workspace`; query its size with the
+ *    matching *_workspace_size function.
+ *  - Layouts are dense and row-major. bf16 tensors are passed as moe_bf16
+ *    (the 16-bit pattern of a bfloat16).
+ *  - Stream. Every call is asynchronous on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream). Results are valid once the stream reaches
+ *    them.
+ *  - Errors. Argument errors are reported before anything is launched, as
+ *    MOE_ERR_INVALID_ARG (bad sizes or NULL pointers), MOE_ERR_UNSUPPORTED (a
+ *    valid shape outside the kernels' limits) or MOE_ERR_WORKSPACE. A failed
+ *    launch gives MOE_ERR_CUDA. Kernels report problems that they detect (an
+ *    expert index outside [0,E), inconsistent offsets, a wait that timed out)
+ *    in a device-side error word, and skip the offending row instead of
+ *    trapping. moe_get_device_status reads and clears that word.
+ *  - Limits. 1 <= E <= 256; 1 <= k <= min(E, 16); H and I are multiples of 64;
+ *    T * k < 2^31.
+ *  - Dropless routing. A = T * k routed rows, a static size: buffers never
+ *    depend on the routing, so no device-to-host copy is needed (TE Token
+ *    dispatch: num_out_tokens known statically).
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t moe_bf16; /* bfloat16 bit pattern */
+
+typedef enum moe_status {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,
+    MOE_ERR_UNSUPPORTED = 2,
+    MOE_ERR_CUDA = 3,
+    MOE_ERR_WORKSPACE = 4,
+    MOE_ERR_DEVICE_CHECK = 5, /* a kernel found invalid data (index or offsets) */
+    MOE_ERR_TIMEOUT = 6       /* a kernel gave up on a bounded wait */
+} moe_status;
+
+typedef enum moe_score_fn {
+    MOE_SCORE_SOFTMAX = 0,
+    MOE_SCORE_SIGMOID = 1
+} moe_score_fn;
+
+/*
+ * Router options (TE "Mixture of Experts", Router):
+ *  score_fn     MOE_SCORE_SOFTMAX or MOE_SCORE_SIGMOID.
+ *  renormalize  softmax: 1 = softmax after top-k, so the k weights are a
+ *               softmax over the chosen logits and sum to one; 0 = softmax
+ *               over all E experts before top-k (use_pre_softmax).
+ *               sigmoid: 1 = divide the k sigmoids by their sum; 0 = raw.
+ *  scaling      multiplies every returned weight (scaling_factor); 1 = none.
+ *  expert_bias  NULL, or device fp32 [E]. It is added to the sigmoid score for
+ *               the choice of experts only, never to the weights (Load
+ *               balancing section). Valid with MOE_SCORE_SIGMOID only.
+ */
+typedef struct moe_router_opts {
+    int score_fn;
+    int renormalize;
+    float scaling;
+    const float* expert_bias;
+} moe_router_opts;
+
+/* Human-readable name of a status code (static storage). */
+const char* moe_status_string(moe_status status);
+
+/* Synchronises `stream`, then reads and clears the device-side error word.
+ * Returns MOE_OK, MOE_ERR_DEVICE_CHECK, MOE_ERR_TIMEOUT or MOE_ERR_CUDA. */
+moe_status moe_get_device_status(void* stream);
+
+/* ------------------------------------------------------------------ router
+ * moe_router_topk -- TE Router (fused_topk_with_score_function); te_mixtral.py
+ * TEMixtralSparseMoeBlock.forward (fp32 softmax, top-k, renormalise).
+ * All math runs in fp32. For each token t, the k experts with the largest
+ * score are chosen (softmax ranks the logits; sigmoid ranks
+ * sigmoid(logit) + expert_bias). Among equal scores the lower expert index
+ * wins, and NaN ranks below every number.
+ *  logits       in  fp32 [T, E]
+ *  topk_idx     out int32 [T, k]  chosen experts, best first
+ *  topk_prob    out fp32  [T, k]  routing weight of each chosen expert
+ *  routing_map  out uint8 [T, E]  1 at the chosen experts, else 0 (NULL: skip)
+ *  counts       out int32 [E]     tokens routed to each expert (column sums)
+ *  offsets      out int32 [E+1]   offsets[0] = 0, offsets[e+1] = offsets[e] +
+ *                                 counts[e]: the start of each expert block
+ *                                 ("offsets are the cumulative per-expert
+ *                                 counts", TE Expert parallelism, Receive buffer)
+ *  workspace    scratch of moe_router_workspace_size(T, E, k) bytes
+ * T = 0 is allowed: counts and offsets are zeroed. */
+size_t moe_router_workspace_size(int64_t T, int E, int k);
+moe_status moe_router_topk(const float* logits, int64_t T, int E, int k,
+                           const moe_router_opts* opts, int32_t* topk_idx, float* topk_prob,
+                           uint8_t* routing_map, int32_t* counts, int32_t* offsets,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* ----------------------------------------------------------------- dispatch
+ * moe_permute -- TE Token dispatch: the rows of all tokens routed to the same
+ * expert are stored back to back, in expert order. Inside an expert block,
+ * rows are in ascending token order: the assignment (t, j) with
+ * e = topk_idx[t, j] goes to row offsets[e] + #{t' < t routed to e}.
+ *  x            in  bf16 [T, H]
+ *  topk_idx     in  int32 [T, k]  (from moe_router_topk)
+ *  offsets      in  int32 [E+1]   (from moe_router_topk)
+ *  x_perm       out bf16 [T*k, H] expert-contiguous copy of the routed rows
+ *  sorted_token out int32 [T*k]   token of each permuted row
+ *  row_of       out int32 [T, k]  permuted row of each assignment (the map
+ *                                 that combine uses to restore token order)
+ *  workspace    scratch of moe_permute_workspace_size(T, E, k) bytes */
+size_t moe_permute_workspace_size(int64_t T, int E, int k);
+moe_status moe_permute(const moe_bf16* x, int64_t T, int H, const int32_t* topk_idx, int k,
+                       const int32_t* offsets, int E, moe_bf16* x_perm, int32_t* sorted_token,
+                       int32_t* row_of, void* workspace, size_t workspace_bytes, void* stream);
+
+/* -------------------------------------------------------------- grouped MLP
+ * moe_grouped_mlp -- TE Grouped GEMM (Y_i = X_i W_i^T per expert block,
+ * Y = concat(Y_i)) and Grouped MLP (FC1 with the activation fused, then FC2).
+ * For the rows r of expert e, [offsets[e], offsets[e+1]):
+ *   g = x_perm[r] . w_gate_up[e][:, 0:I]   u = x_perm[r] . w_gate_up[e][:, I:2I]
+ *   h[r] = bf16(silu(g) * u)               y_perm[r] = bf16(h[r] . w_down[e])
+ * in fp32 accumulation. Experts may have any number of rows, zero included.
+ *  x_perm       in  bf16 [A, H]
+ *  offsets      in  int32 [E+1]   offsets[E] <= A; rows past offsets[E] untouched
+ *  w_gate_up    in  bf16 [E, H, 2I]  (gate columns first, then up)
+ *  w_down       in  bf16 [E, I, H]
+ *  y_perm       out bf16 [A, H]
+ *  gu_save      out bf16 [A, 2I]  g and u, kept for the backward (NULL: skip)
+ *  h_save       out bf16 [A, I]   h (NULL: h goes to the workspace)
+ *  workspace    moe_grouped_mlp_workspace_size(A, E, H, I) bytes; 0 when
+ *               h_save is given */
+size_t moe_grouped_mlp_workspace_size(int64_t A, int E, int H, int I);
+moe_status moe_grouped_mlp(const moe_bf16* x_perm, int64_t A, const int32_t* offsets, int E,
+                           int H, int I, const moe_bf16* w_gate_up, const moe_bf16* w_down,
+                           moe_bf16* y_perm, moe_bf16* gu_save, moe_bf16* h_save,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------ combine
+ * moe_unpermute_combine -- TE Token combine with merging_probs:
+ *   out[t] = bf16( shared_out[t] + sum_{j<k} topk_prob[t,j] * y_perm[row_of[t,j]] )
+ * summed in fp32, j ascending. Each output row has one writer, so the result
+ * is deterministic. topk_prob NULL sums the rows unweighted. shared_out NULL
+ * means no shared expert. The routing weights must be applied exactly once (TE
+ * Token probabilities): pass NULL here if y_perm is already weighted.
+ *  y_perm in bf16 [A, H]; row_of in int32 [T, k]; topk_prob in fp32 [T, k];
+ *  shared_out in bf16 [T, H]; out out bf16 [T, H]. */
+moe_status moe_unpermute_combine(const moe_bf16* y_perm, const int32_t* row_of,
+                                 const float* topk_prob, int64_t T, int k, int H,
+                                 const moe_bf16* shared_out, moe_bf16* out, void* stream);
+
+/* ------------------------------------------------------------ fused layer
+ * moe_layer_forward -- the four stages on one stream (TE "Example: MoE layer
+ * on a single device"):
+ *   out[t] = shared(x[t]) + sum_j p[t,j] * MLP_{e[t,j]}(x[t])
+ * shared_gate_up [H, 2I] and shared_down [I, H] are the dense SwiGLU shared
+ * expert (torchtitan MoE.forward adds it to the routed output); pass NULL for
+ * none. The optional outputs below keep the forward state for
+ * moe_grouped_mlp_backward. Each may be NULL, in which case it lives in the
+ * workspace: topk_idx [T,k], topk_prob [T,k], counts [E], offsets [E+1],
+ * row_of [T,k], x_perm [A,H], gu [A,2I] (NULL: not computed), h [A,I],
+ * y_perm [A,H].
+ * The call records no device-to-host copy and no host synchronisation, so it
+ * can be captured in a CUDA graph. */
+size_t moe_layer_forward_workspace_size(int64_t T, int H, int I, int E, int k, int has_shared);
+moe_status moe_layer_forward(const float* logits, const moe_bf16* x, int64_t T, int H, int I,
+                             int E, int k, const moe_router_opts* opts,
+                             const moe_bf16* w_gate_up, const moe_bf16* w_down,
+                             const moe_bf16* shared_gate_up, const moe_bf16* shared_down,
+                             moe_bf16* out, int32_t* topk_idx, float* topk_prob, int32_t* counts,
+                             int32_t* offsets, int32_t* row_of, moe_bf16* x_perm, moe_bf16* gu,
+                             moe_bf16* h, moe_bf16* y_perm, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/* ----------------------------------------------------------------- backward
+ * moe_grouped_mlp_backward -- gradients of out[t] = sum_j p[t,j] MLP_e(x[t])
+ * with respect to x, w_gate_up, w_down and the routing weights p (TE Example:
+ * every stage is differentiable; the logits do not receive a gradient here):
+ *   dprob[t,j] = <dout[t], y_perm[row]>           dy[row] = p[t,j] * dout[t]
+ *   dh = dy . w_down[e]^T     du = dh * silu(g)    dg = dh * u * silu'(g)
+ *   dx_perm = [dg | du] . w_gate_up[e]^T           dx[t] = sum_j dx_perm[row_of[t,j]]
+ *   dw_down[e] = h_e^T . dy_e                      dw_gate_up[e] = x_e^T . [dg | du]_e
+ * with row = row_of[t,j] and the forward state saved by moe_layer_forward
+ * (gu must have been saved). Accumulation is fp32. An expert with no rows
+ * gets zero weight gradients.
+ *  dout in bf16 [T,H]; dx out bf16 [T,H]; dw_gate_up out bf16 [E,H,2I];
+ *  dw_down out bf16 [E,I,H]; dprob out fp32 [T,k];
+ *  workspace of moe_grouped_mlp_backward_workspace_size(T, H, I, E, k) bytes. */
+size_t moe_grouped_mlp_backward_workspace_size(int64_t T, int H, int I, int E, int k);
+moe_status moe_grouped_mlp_backward(const moe_bf16* dout, int64_t T, int H, int I, int E, int k,
+                                    const moe_bf16* w_gate_up, const moe_bf16* w_down,
+                                    const int32_t* row_of, const float* topk_prob,
+                                    const int32_t* offsets, const moe_bf16* x_perm,
+                                    const moe_bf16* gu, const moe_bf16* h, const moe_bf16* y_perm,
+                                    moe_bf16* dx, moe_bf16* dw_gate_up, moe_bf16* dw_down,
+                                    float* dprob, void* workspace, size_t workspace_bytes,
+                                    void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

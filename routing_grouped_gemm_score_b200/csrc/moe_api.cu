@@ -1,0 +1,419 @@
+// moe_api.cu -- the extern "C" entry points declared in include/moe_b200.h:
+// argument checks (before any CUDA call), workspace layout, the device error
+// word, and the stage order of the fused forward and of the backward.
+#include <cstring>
+#include <mutex>
+
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+__device__ unsigned g_device_error;
+
+constexpr int kMaxDevices = 64;
+
+int current_device() {
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess) return -1;
+    return d;
+}
+
+struct DeviceInfo {
+    std::once_flag once;
+    int sms = 148;
+    unsigned* err = nullptr;
+};
+DeviceInfo g_info[kMaxDevices];
+
+DeviceInfo* info() {
+    const int d = current_device();
+    if (d < 0 || d >= kMaxDevices) return nullptr;
+    DeviceInfo* di = &g_info[d];
+    std::call_once(di->once, [di, d] {
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, d) == cudaSuccess && sms > 0)
+            di->sms = sms;
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) == cudaSuccess)
+            di->err = static_cast<unsigned*>(p);
+    });
+    return di;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Bump allocator over the caller's workspace; every piece is 256-byte aligned.
+struct Carver {
+    char* base;
+    size_t used = 0;
+    explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+    template <class T>
+    T* take(size_t count) {
+        used = (used + 255) & ~size_t(255);
+        T* p = reinterpret_cast<T*>(base ? base + used : nullptr);
+        used += count * sizeof(T);
+        return p;
+    }
+    size_t bytes() const { return (used + 255) & ~size_t(255); }
+};
+
+bool shape_ok(int64_t T, int E, int k) {
+    return T >= 0 && E >= 1 && E <= 256 && k >= 1 && k <= 16 && k <= E &&
+           T * (int64_t)k < (int64_t(1) << 31);
+}
+
+bool dims_ok(int H, int I) { return H > 0 && I > 0 && H % 64 == 0 && I % 64 == 0; }
+
+moe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+moe_router_opts default_opts() {
+    moe_router_opts o;
+    o.score_fn = MOE_SCORE_SOFTMAX;
+    o.renormalize = 1;
+    o.scaling = 1.0f;
+    o.expert_bias = nullptr;
+    return o;
+}
+
+moe_status check_opts(const moe_router_opts& o) {
+    if (o.score_fn != MOE_SCORE_SOFTMAX && o.score_fn != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
+    if (o.expert_bias && o.score_fn != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
+    if (!(o.scaling == o.scaling)) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
+}
+
+// Layout of the fused forward's workspace. Pieces the caller supplies are
+// still reserved, so the size depends on the shape only.
+struct FwdLayout {
+    RouteScratch rs;
+    int32_t *topk_idx, *counts, *offsets, *row_of, *sorted_token;
+    float* topk_prob;
+    bf16 *x_perm, *h, *y_perm, *shared_h, *shared_out;
+    size_t bytes;
+};
+
+FwdLayout fwd_layout(void* ws, int64_t T, int H, int I, int E, int k, int has_shared) {
+    const int64_t A = T * k;
+    Carver c(ws);
+    FwdLayout L;
+    char* route = c.take<char>(route_scratch_bytes(T, E, k));
+    L.rs = carve_route_scratch(route, T, E, k);
+    L.topk_idx = c.take<int32_t>((size_t)A);
+    L.topk_prob = c.take<float>((size_t)A);
+    L.counts = c.take<int32_t>((size_t)E);
+    L.offsets = c.take<int32_t>((size_t)E + 1);
+    L.row_of = c.take<int32_t>((size_t)A);
+    L.sorted_token = c.take<int32_t>((size_t)A);
+    L.x_perm = c.take<bf16>((size_t)A * H);
+    L.h = c.take<bf16>((size_t)A * I);
+    L.y_perm = c.take<bf16>((size_t)A * H);
+    L.shared_h = has_shared ? c.take<bf16>((size_t)T * I) : nullptr;
+    L.shared_out = has_shared ? c.take<bf16>((size_t)T * H) : nullptr;
+    L.bytes = c.bytes();
+    return L;
+}
+
+struct BwdLayout {
+    bf16 *dy, *dgu, *dx_perm;
+    size_t bytes;
+};
+
+BwdLayout bwd_layout(void* ws, int64_t T, int H, int I, int k) {
+    const int64_t A = T * k;
+    Carver c(ws);
+    BwdLayout L;
+    L.dy = c.take<bf16>((size_t)A * H);
+    L.dgu = c.take<bf16>((size_t)A * 2 * I);
+    L.dx_perm = c.take<bf16>((size_t)A * H);
+    L.bytes = c.bytes();
+    return L;
+}
+
+}  // namespace
+
+unsigned* device_error_word() {
+    DeviceInfo* di = info();
+    return di ? di->err : nullptr;
+}
+
+int sm_count() {
+    DeviceInfo* di = info();
+    return di ? di->sms : 148;
+}
+
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: shape outside the kernels' limits";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA call or launch failed";
+        case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace too small or missing";
+        case MOE_ERR_DEVICE_CHECK: return "MOE_ERR_DEVICE_CHECK: a kernel found invalid routing data";
+        case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT: a kernel gave up on a bounded wait";
+    }
+    return "unknown moe_status";
+}
+
+moe_status moe_get_device_status(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+    unsigned* err = device_error_word();
+    if (!err) return MOE_ERR_CUDA;
+    unsigned v = 0;
+    if (cudaMemcpy(&v, err, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    if (v) {
+        const unsigned zero = 0;
+        if (cudaMemcpy(err, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
+    if (v & kErrTimeout) return MOE_ERR_TIMEOUT;
+    if (v & kErrDeviceCheck) return MOE_ERR_DEVICE_CHECK;
+    return MOE_OK;
+}
+
+size_t moe_router_workspace_size(int64_t T, int E, int k) {
+    if (!shape_ok(T, E, k)) return 0;
+    return route_scratch_bytes(T, E, k);
+}
+
+moe_status moe_router_topk(const float* logits, int64_t T, int E, int k,
+                           const moe_router_opts* opts_in, int32_t* topk_idx, float* topk_prob,
+                           uint8_t* routing_map, int32_t* counts, int32_t* offsets,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+    if (!shape_ok(T, E, k)) return MOE_ERR_INVALID_ARG;
+    const moe_router_opts opts = opts_in ? *opts_in : default_opts();
+    if (check_opts(opts) != MOE_OK) return MOE_ERR_INVALID_ARG;
+    if (!counts || !offsets || !aligned16(counts) || !aligned16(offsets)) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!logits || !topk_idx || !topk_prob || !aligned16(logits) ||
+                  !aligned16(topk_idx) || !aligned16(topk_prob)))
+        return MOE_ERR_INVALID_ARG;
+    if (opts.expert_bias && !aligned16(opts.expert_bias)) return MOE_ERR_INVALID_ARG;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, st) != cudaSuccess) return MOE_ERR_CUDA;
+        return from_cuda(cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), st));
+    }
+    if (!workspace || workspace_bytes < route_scratch_bytes(T, E, k)) return MOE_ERR_WORKSPACE;
+    unsigned* err = device_error_word();
+    if (!err) return MOE_ERR_CUDA;
+    const RouteScratch rs = carve_route_scratch(workspace, T, E, k);
+    cudaError_t e = launch_router_topk(logits, T, E, k, opts, topk_idx, topk_prob, routing_map, rs,
+                                       st, err);
+    if (e == cudaSuccess) e = launch_expert_scan(T, E, rs, counts, offsets, st);
+    return from_cuda(e);
+}
+
+size_t moe_permute_workspace_size(int64_t T, int E, int k) {
+    if (!shape_ok(T, E, k)) return 0;
+    return route_scratch_bytes(T, E, k);
+}
+
+moe_status moe_permute(const moe_bf16* x, int64_t T, int H, const int32_t* topk_idx, int k,
+                       const int32_t* offsets, int E, moe_bf16* x_perm, int32_t* sorted_token,
+                       int32_t* row_of, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!shape_ok(T, E, k) || H <= 0 || H % 8 != 0) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!x || !topk_idx || !offsets || !x_perm || !sorted_token || !row_of) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(x_perm) || !aligned16(topk_idx) || !aligned16(offsets) ||
+        !aligned16(sorted_token) || !aligned16(row_of))
+        return MOE_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < route_scratch_bytes(T, E, k)) return MOE_ERR_WORKSPACE;
+    unsigned* err = device_error_word();
+    if (!err) return MOE_ERR_CUDA;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const RouteScratch rs = carve_route_scratch(workspace, T, E, k);
+    cudaError_t e = launch_rank_from_indices(topk_idx, T, E, k, rs, st, err);
+    if (e == cudaSuccess) e = launch_expert_scan(T, E, rs, nullptr, nullptr, st);
+    if (e == cudaSuccess)
+        e = launch_permute(reinterpret_cast<const bf16*>(x), T, H, topk_idx, k, offsets, E, rs,
+                           reinterpret_cast<bf16*>(x_perm), sorted_token, row_of, st, err);
+    return from_cuda(e);
+}
+
+size_t moe_grouped_mlp_workspace_size(int64_t A, int E, int H, int I) {
+    if (A < 0 || E < 1 || E > 256 || !dims_ok(H, I)) return 0;
+    Carver c(nullptr);
+    c.take<bf16>((size_t)A * I);
+    return c.bytes();
+}
+
+moe_status moe_grouped_mlp(const moe_bf16* x_perm, int64_t A, const int32_t* offsets, int E,
+                           int H, int I, const moe_bf16* w_gate_up, const moe_bf16* w_down,
+                           moe_bf16* y_perm, moe_bf16* gu_save, moe_bf16* h_save,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+    if (A < 0 || A >= (int64_t(1) << 31) || E < 1 || E > 256) return MOE_ERR_INVALID_ARG;
+    if (H <= 0 || I <= 0) return MOE_ERR_INVALID_ARG;
+    if (!dims_ok(H, I)) return MOE_ERR_UNSUPPORTED;
+    if (A == 0) return MOE_OK;
+    if (!x_perm || !offsets || !w_gate_up || !w_down || !y_perm) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x_perm) || !aligned16(offsets) || !aligned16(w_gate_up) || !aligned16(w_down) ||
+        !aligned16(y_perm) || (gu_save && !aligned16(gu_save)) || (h_save && !aligned16(h_save)))
+        return MOE_ERR_INVALID_ARG;
+    bf16* h = reinterpret_cast<bf16*>(h_save);
+    if (!h) {
+        if (!workspace || workspace_bytes < moe_grouped_mlp_workspace_size(A, E, H, I))
+            return MOE_ERR_WORKSPACE;
+        h = Carver(workspace).take<bf16>((size_t)A * I);
+    }
+    unsigned* err = device_error_word();
+    if (!err) return MOE_ERR_CUDA;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = gemm_gate_up_swiglu(reinterpret_cast<const bf16*>(x_perm), A, offsets, E, H, I,
+                                        reinterpret_cast<const bf16*>(w_gate_up), h,
+                                        reinterpret_cast<bf16*>(gu_save), st, err);
+    if (e == cudaSuccess)
+        e = gemm_down(h, A, offsets, E, H, I, reinterpret_cast<const bf16*>(w_down),
+                      reinterpret_cast<bf16*>(y_perm), st, err);
+    return from_cuda(e);
+}
+
+moe_status moe_unpermute_combine(const moe_bf16* y_perm, const int32_t* row_of,
+                                 const float* topk_prob, int64_t T, int k, int H,
+                                 const moe_bf16* shared_out, moe_bf16* out, void* stream) {
+    if (T < 0 || k < 1 || k > 16 || H <= 0 || H % 8 != 0 || T * (int64_t)k >= (int64_t(1) << 31))
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    if (!y_perm || !row_of || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(y_perm) || !aligned16(row_of) || !aligned16(out) ||
+        (topk_prob && !aligned16(topk_prob)) || (shared_out && !aligned16(shared_out)))
+        return MOE_ERR_INVALID_ARG;
+    unsigned* err = device_error_word();
+    if (!err) return MOE_ERR_CUDA;
+    return from_cuda(launch_combine(reinterpret_cast<const bf16*>(y_perm), row_of, topk_prob, T, k,
+                                    H, T * k, reinterpret_cast<const bf16*>(shared_out),
+                                    reinterpret_cast<bf16*>(out), static_cast<cudaStream_t>(stream),
+                                    err));
+}
+
+size_t moe_layer_forward_workspace_size(int64_t T, int H, int I, int E, int k, int has_shared) {
+    if (!shape_ok(T, E, k) || !dims_ok(H, I)) return 0;
+    return fwd_layout(nullptr, T, H, I, E, k, has_shared).bytes;
+}
+
+moe_status moe_layer_forward(const float* logits, const moe_bf16* x, int64_t T, int H, int I,
+                             int E, int k, const moe_router_opts* opts_in,
+                             const moe_bf16* w_gate_up, const moe_bf16* w_down,
+                             const moe_bf16* shared_gate_up, const moe_bf16* shared_down,
+                             moe_bf16* out, int32_t* topk_idx, float* topk_prob, int32_t* counts,
+                             int32_t* offsets, int32_t* row_of, moe_bf16* x_perm, moe_bf16* gu,
+                             moe_bf16* h, moe_bf16* y_perm, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+    if (!shape_ok(T, E, k) || H <= 0 || I <= 0) return MOE_ERR_INVALID_ARG;
+    if (!dims_ok(H, I)) return MOE_ERR_UNSUPPORTED;
+    const moe_router_opts opts = opts_in ? *opts_in : default_opts();
+    if (check_opts(opts) != MOE_OK) return MOE_ERR_INVALID_ARG;
+    if ((shared_gate_up == nullptr) != (shared_down == nullptr)) return MOE_ERR_INVALID_ARG;
+    const void* must[] = {logits, x, w_gate_up, w_down, out};
+    for (const void* p : must)
+        if (T > 0 && (!p || !aligned16(p))) return MOE_ERR_INVALID_ARG;
+    const void* opt[] = {shared_gate_up, shared_down, topk_idx, topk_prob, counts, offsets,
+                         row_of, x_perm, gu, h, y_perm, opts.expert_bias};
+    for (const void* p : opt)
+        if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+    const int has_shared = shared_gate_up != nullptr;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        cudaError_t e = cudaSuccess;
+        if (counts) e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, st);
+        if (e == cudaSuccess && offsets) e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), st);
+        return from_cuda(e);
+    }
+    const FwdLayout L0 = fwd_layout(nullptr, T, H, I, E, k, has_shared);
+    if (!workspace || workspace_bytes < L0.bytes) return MOE_ERR_WORKSPACE;
+    unsigned* err = device_error_word();
+    if (!err) return MOE_ERR_CUDA;
+    FwdLayout L = fwd_layout(workspace, T, H, I, E, k, has_shared);
+    if (topk_idx) L.topk_idx = topk_idx;
+    if (topk_prob) L.topk_prob = topk_prob;
+    if (counts) L.counts = counts;
+    if (offsets) L.offsets = offsets;
+    if (row_of) L.row_of = row_of;
+    if (x_perm) L.x_perm = reinterpret_cast<bf16*>(x_perm);
+    if (h) L.h = reinterpret_cast<bf16*>(h);
+    if (y_perm) L.y_perm = reinterpret_cast<bf16*>(y_perm);
+    const int64_t A = T * k;
+    const bf16* xb = reinterpret_cast<const bf16*>(x);
+
+    cudaError_t e = launch_router_topk(logits, T, E, k, opts, L.topk_idx, L.topk_prob, nullptr,
+                                       L.rs, st, err);
+    if (e == cudaSuccess) e = launch_expert_scan(T, E, L.rs, L.counts, L.offsets, st);
+    if (e == cudaSuccess)
+        e = launch_permute(xb, T, H, L.topk_idx, k, L.offsets, E, L.rs, L.x_perm, L.sorted_token,
+                           L.row_of, st, err);
+    if (e == cudaSuccess)
+        e = gemm_gate_up_swiglu(L.x_perm, A, L.offsets, E, H, I,
+                                reinterpret_cast<const bf16*>(w_gate_up), L.h,
+                                reinterpret_cast<bf16*>(gu), st, err);
+    if (e == cudaSuccess)
+        e = gemm_down(L.h, A, L.offsets, E, H, I, reinterpret_cast<const bf16*>(w_down), L.y_perm,
+                      st, err);
+    if (e == cudaSuccess && has_shared) {
+        e = gemm_gate_up_swiglu(xb, T, nullptr, 1, H, I,
+                                reinterpret_cast<const bf16*>(shared_gate_up), L.shared_h, nullptr,
+                                st, err);
+        if (e == cudaSuccess)
+            e = gemm_down(L.shared_h, T, nullptr, 1, H, I,
+                          reinterpret_cast<const bf16*>(shared_down), L.shared_out, st, err);
+    }
+    if (e == cudaSuccess)
+        e = launch_combine(L.y_perm, L.row_of, L.topk_prob, T, k, H, A, L.shared_out,
+                           reinterpret_cast<bf16*>(out), st, err);
+    return from_cuda(e);
+}
+
+size_t moe_grouped_mlp_backward_workspace_size(int64_t T, int H, int I, int E, int k) {
+    if (!shape_ok(T, E, k) || !dims_ok(H, I)) return 0;
+    return bwd_layout(nullptr, T, H, I, k).bytes;
+}
+
+moe_status moe_grouped_mlp_backward(const moe_bf16* dout, int64_t T, int H, int I, int E, int k,
+                                    const moe_bf16* w_gate_up, const moe_bf16* w_down,
+                                    const int32_t* row_of, const float* topk_prob,
+                                    const int32_t* offsets, const moe_bf16* x_perm,
+                                    const moe_bf16* gu, const moe_bf16* h, const moe_bf16* y_perm,
+                                    moe_bf16* dx, moe_bf16* dw_gate_up, moe_bf16* dw_down,
+                                    float* dprob, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+    if (!shape_ok(T, E, k) || H <= 0 || I <= 0) return MOE_ERR_INVALID_ARG;
+    if (!dims_ok(H, I)) return MOE_ERR_UNSUPPORTED;
+    const void* must[] = {dout, w_gate_up, w_down, row_of, topk_prob, offsets, x_perm, gu, h,
+                          y_perm, dx, dw_gate_up, dw_down, dprob};
+    for (const void* p : must)
+        if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+    const BwdLayout L0 = bwd_layout(nullptr, T, H, I, k);
+    if (!workspace || workspace_bytes < L0.bytes) return MOE_ERR_WORKSPACE;
+    unsigned* err = device_error_word();
+    if (!err) return MOE_ERR_CUDA;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const BwdLayout L = bwd_layout(workspace, T, H, I, k);
+    const int64_t A = T * k;
+    auto B = [](const moe_bf16* p) { return reinterpret_cast<const bf16*>(p); };
+    cudaError_t e = cudaSuccess;
+    if (T > 0) {
+        e = launch_combine_backward(B(dout), B(y_perm), row_of, topk_prob, T, k, H, A, L.dy, dprob,
+                                    st, err);
+        if (e == cudaSuccess)
+            e = gemm_down_dgrad_swiglu(L.dy, A, offsets, E, H, I, B(w_down), B(gu), L.dgu, st, err);
+        if (e == cudaSuccess)
+            e = gemm_gate_up_dgrad(L.dgu, A, offsets, E, H, I, B(w_gate_up), L.dx_perm, st, err);
+        if (e == cudaSuccess)
+            e = launch_combine(L.dx_perm, row_of, nullptr, T, k, H, A, nullptr,
+                               reinterpret_cast<bf16*>(dx), st, err);
+    }
+    if (e == cudaSuccess)
+        e = gemm_wgrad(B(h), L.dy, A, offsets, E, I, H, reinterpret_cast<bf16*>(dw_down), st, err);
+    if (e == cudaSuccess)
+        e = gemm_wgrad(B(x_perm), L.dgu, A, offsets, E, H, 2 * I,
+                       reinterpret_cast<bf16*>(dw_gate_up), st, err);
+    return from_cuda(e);
+}
+
+}  // extern "C"

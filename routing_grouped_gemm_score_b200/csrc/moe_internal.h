@@ -1,0 +1,81 @@
+// moe_internal.h -- launchers shared between the kernel files and the C ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe_b200.h"
+
+namespace moe {
+
+using bf16 = __nv_bfloat16;
+
+// Tokens handled by one block of the router / rank kernels. Ranks inside an
+// expert block are counted per such token block, then offset by a scan.
+constexpr int kTokensPerRouteBlock = 64;
+
+inline int64_t route_blocks(int64_t T) {
+    return (T + kTokensPerRouteBlock - 1) / kTokensPerRouteBlock;
+}
+
+// Scratch of the routing path, carved from the caller's workspace.
+struct RouteScratch {
+    int32_t* block_base;  // [E][nb]: per-(expert, token block) counts, then exclusive prefix
+    int32_t* local_rank;  // [T][k]: rank of the assignment inside its token block
+    unsigned* ticket;     // last-block-done counter of the scan kernel
+};
+size_t route_scratch_bytes(int64_t T, int E, int k);
+RouteScratch carve_route_scratch(void* base, int64_t T, int E, int k);
+
+cudaError_t launch_router_topk(const float* logits, int64_t T, int E, int k,
+                               const moe_router_opts& opts, int32_t* topk_idx, float* topk_prob,
+                               uint8_t* routing_map, const RouteScratch& rs, cudaStream_t st,
+                               unsigned* err);
+cudaError_t launch_rank_from_indices(const int32_t* topk_idx, int64_t T, int E, int k,
+                                     const RouteScratch& rs, cudaStream_t st, unsigned* err);
+// Turns block counts into exclusive prefixes; writes counts/offsets if given.
+cudaError_t launch_expert_scan(int64_t T, int E, const RouteScratch& rs, int32_t* counts,
+                               int32_t* offsets, cudaStream_t st);
+cudaError_t launch_permute(const bf16* x, int64_t T, int H, const int32_t* topk_idx, int k,
+                           const int32_t* offsets, int E, const RouteScratch& rs, bf16* x_perm,
+                           int32_t* sorted_token, int32_t* row_of, cudaStream_t st, unsigned* err);
+
+cudaError_t launch_combine(const bf16* y_perm, const int32_t* row_of, const float* probs,
+                           int64_t T, int k, int H, int64_t A, const bf16* shared, bf16* out,
+                           cudaStream_t st, unsigned* err);
+cudaError_t launch_combine_backward(const bf16* dout, const bf16* y_perm, const int32_t* row_of,
+                                    const float* probs, int64_t T, int k, int H, int64_t A,
+                                    bf16* dy_perm, float* dprob, cudaStream_t st, unsigned* err);
+
+// ---------------------------------------------------------------- GEMMs
+// Grouped GEMMs on tcgen05. Each returns cudaErrorInvalidValue if a tensor
+// map cannot be encoded (bad alignment or extent).
+struct GemmStatus {
+    cudaError_t err;
+};
+// gate_up + SwiGLU: h[r] = silu(x[r] Wg[e]) * (x[r] Wu[e]); optionally gu[r] = [g | u].
+// offsets NULL: one group of `rows` rows using the weights of group 0.
+cudaError_t gemm_gate_up_swiglu(const bf16* x, int64_t rows, const int32_t* offsets, int E, int H,
+                                int I, const bf16* w_gate_up, bf16* h, bf16* gu_save,
+                                cudaStream_t st, unsigned* err);
+// down: y[r] = h[r] Wd[e]
+cudaError_t gemm_down(const bf16* h, int64_t rows, const int32_t* offsets, int E, int H, int I,
+                      const bf16* w_down, bf16* y, cudaStream_t st, unsigned* err);
+// dgrad of down with SwiGLU backward: dh = dy Wd[e]^T, then dgu = [dg | du]
+cudaError_t gemm_down_dgrad_swiglu(const bf16* dy, int64_t rows, const int32_t* offsets, int E,
+                                   int H, int I, const bf16* w_down, const bf16* gu, bf16* dgu,
+                                   cudaStream_t st, unsigned* err);
+// dgrad of gate_up: dx_perm = dgu Wgu[e]^T
+cudaError_t gemm_gate_up_dgrad(const bf16* dgu, int64_t rows, const int32_t* offsets, int E, int H,
+                               int I, const bf16* w_gate_up, bf16* dx_perm, cudaStream_t st,
+                               unsigned* err);
+// wgrad: dW[e] = X_e^T D_e over the rows of group e (ragged reduction);
+// X [rows, M], D [rows, N], dW [E, M, N]. Empty groups get dW[e] = 0.
+cudaError_t gemm_wgrad(const bf16* X, const bf16* D, int64_t rows, const int32_t* offsets, int E,
+                       int M, int N, bf16* dW, cudaStream_t st, unsigned* err);
+
+int sm_count();
+
+}  // namespace moe

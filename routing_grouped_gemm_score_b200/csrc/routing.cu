@@ -1,0 +1,423 @@
+// routing.cu -- router (score function + top-k + routing weights), rank and
+// expert-offset scan, and the permute (token dispatch) kernel.
+//
+// Transformer Engine "Mixture of Experts", sections Router and Token
+// dispatch; te_mixtral.py TEMixtralSparseMoeBlock.forward.
+//
+// Design: one warp per token. A lane holds the scores of experts lane,
+// lane+32, ... in registers. The k experts are picked in k rounds of a warp
+// arg-max over 64-bit keys (score ordered as an unsigned integer in the high
+// half, bit-inverted expert index in the low half), so a larger key means a
+// larger score, or the same score at a lower index. The choice is made on
+// the logit itself: softmax and sigmoid are increasing, so the ranking is
+// the same and no rounding of the score function can create a tie. Ranks
+// inside each expert are counted per block of 64 tokens in shared memory, in
+// token order, and an exclusive scan over the token blocks turns them into
+// global rows. Positions never come from atomics, so the permutation is the
+// same on every run.
+#include "moe_common.cuh"
+#include "moe_internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kRouteThreads = 256;  // 8 warps, 8 tokens each per block
+constexpr unsigned kFull = 0xFFFFFFFFu;
+
+// Order-preserving map of a float to uint32: a larger float gives a larger
+// key. NaN maps below -inf, and -0 maps like +0.
+__device__ __forceinline__ uint32_t float_order_key(float s) {
+    uint32_t b = __float_as_uint(s);
+    if ((b & 0x7FFFFFFFu) > 0x7F800000u) return 0u;  // NaN
+    if ((b & 0x7FFFFFFFu) == 0u) b = 0u;             // -0 -> +0
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        uint64_t o = __shfl_xor_sync(kFull, v, off);
+        v = o > v ? o : v;
+    }
+    return v;
+}
+
+struct RouterArgs {
+    const float* logits;
+    int64_t T;
+    int E, k;
+    int score_fn, renormalize;
+    float scaling;
+    const float* bias;
+    int32_t* topk_idx;
+    float* topk_prob;
+    uint8_t* routing_map;
+    int32_t* block_base;  // [E][nb]
+    int32_t* local_rank;  // [T][k]
+    unsigned* ticket;
+    int nb;
+};
+
+// After the token loop: thread e counts, in token order, the assignments of
+// the block's tokens to expert e. sel[tt][e] holds j+1 if token tt chose e as
+// its j-th expert, else 0.
+__device__ __forceinline__ void rank_block(const uint8_t (*sel)[256], int64_t t0, int64_t T,
+                                           int E, int k, int32_t* local_rank,
+                                           int32_t* block_base, int nb) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int cnt = 0;
+        for (int tt = 0; tt < kTokensPerRouteBlock; ++tt) {
+            int v = sel[tt][e];
+            if (v) {
+                local_rank[(t0 + tt) * k + (v - 1)] = cnt;
+                ++cnt;
+            }
+        }
+        block_base[(int64_t)e * nb + blockIdx.x] = cnt;
+    }
+}
+
+template <int SLOTS>
+__global__ void __launch_bounds__(kRouteThreads) router_topk_kernel(const RouterArgs a) {
+    __shared__ uint8_t sel[kTokensPerRouteBlock][256];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = a.E, k = a.k;
+    for (int i = threadIdx.x; i < kTokensPerRouteBlock * 256 / 16; i += blockDim.x)
+        reinterpret_cast<uint4*>(&sel[0][0])[i] = make_uint4(0, 0, 0, 0);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *a.ticket = 0u;
+    __syncthreads();
+    const int64_t t0 = (int64_t)blockIdx.x * kTokensPerRouteBlock;
+
+    for (int tt = warp; tt < kTokensPerRouteBlock; tt += kRouteThreads / 32) {
+        const int64_t t = t0 + tt;
+        if (t >= a.T) break;
+        const float* lrow = a.logits + t * E;
+        float lv[SLOTS];
+        uint64_t key[SLOTS];
+#pragma unroll
+        for (int s = 0; s < SLOTS; ++s) {
+            const int e = lane + 32 * s;
+            lv[s] = e < E ? __ldg(lrow + e) : 0.0f;
+        }
+#pragma unroll
+        for (int s = 0; s < SLOTS; ++s) {
+            const int e = lane + 32 * s;
+            float score = lv[s];
+            if (a.bias) score = 1.0f / (1.0f + expf(-lv[s])) + __ldg(a.bias + (e < E ? e : 0));
+            key[s] = e < E ? ((uint64_t)float_order_key(score) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)e)
+                           : 0ull;
+        }
+        uint64_t mine = 0;
+#pragma unroll
+        for (int s = 0; s < SLOTS; ++s) mine = key[s] > mine ? key[s] : mine;
+        unsigned taken = 0;   // bit s: slot s chosen
+        int my_e = -1;        // lane j < k keeps the j-th chosen expert
+        for (int j = 0; j < k; ++j) {
+            const uint64_t best = warp_max_u64(mine);
+            const int e = (int)(0xFFFFFFFFu - (uint32_t)best);
+            if (lane == j) my_e = e;
+            if (lane == (e & 31)) {
+                const int s_taken = e >> 5;
+                mine = 0;
+#pragma unroll
+                for (int s = 0; s < SLOTS; ++s) {
+                    if (s == s_taken) { key[s] = 0; taken |= 1u << s; }
+                    mine = key[s] > mine ? key[s] : mine;
+                }
+                sel[tt][e] = (uint8_t)(j + 1);
+            }
+        }
+        // routing weights (fp32), in the oracle's order of operations
+        float my_l = (lane < k) ? __ldg(lrow + my_e) : 0.0f;
+        float p = 0.0f;
+        if (a.score_fn == MOE_SCORE_SOFTMAX) {
+            if (a.renormalize) {
+                // max over the chosen, scanned in selection order
+                float m = __shfl_sync(kFull, my_l, 0);
+                for (int j = 1; j < k; ++j) {
+                    const float lj = __shfl_sync(kFull, my_l, j);
+                    if (lj > m) m = lj;
+                }
+                const float ex = (lane < k) ? expf(my_l - m) : 0.0f;
+                float sum = 0.0f;
+                for (int j = 0; j < k; ++j) sum += __shfl_sync(kFull, ex, j);
+                p = ex / sum;
+            } else {
+                // softmax over all experts: row max and sum scanned in expert order
+                float m = __shfl_sync(kFull, lv[0], 0);
+#pragma unroll
+                for (int s = 0; s < SLOTS; ++s)
+                    for (int src = 0; src < 32; ++src) {
+                        const float v = __shfl_sync(kFull, lv[s], src);
+                        if (src + 32 * s < E && v > m) m = v;
+                    }
+                float ex_all[SLOTS];
+#pragma unroll
+                for (int s = 0; s < SLOTS; ++s) ex_all[s] = expf(lv[s] - m);
+                float sum = 0.0f;
+#pragma unroll
+                for (int s = 0; s < SLOTS; ++s)
+                    for (int src = 0; src < 32; ++src) {
+                        const float v = __shfl_sync(kFull, ex_all[s], src);
+                        if (src + 32 * s < E) sum += v;
+                    }
+                p = (lane < k) ? expf(my_l - m) / sum : 0.0f;
+            }
+        } else {
+            const float sg = (lane < k) ? 1.0f / (1.0f + expf(-my_l)) : 0.0f;
+            if (a.renormalize) {
+                float sum = 0.0f;
+                for (int j = 0; j < k; ++j) sum += __shfl_sync(kFull, sg, j);
+                p = sg / sum;
+            } else {
+                p = sg;
+            }
+        }
+        p = p * a.scaling;
+        if (lane < k) {
+            a.topk_idx[t * k + lane] = my_e;
+            a.topk_prob[t * k + lane] = p;
+        }
+        if (a.routing_map) {
+            uint8_t* mrow = a.routing_map + t * E;
+#pragma unroll
+            for (int s = 0; s < SLOTS; ++s) {
+                const int e = lane + 32 * s;
+                if (e < E) mrow[e] = (taken >> s) & 1u;
+            }
+        }
+    }
+    __syncthreads();
+    rank_block(sel, t0, a.T, E, k, a.local_rank, a.block_base, a.nb);
+}
+
+// Rank pass for caller-supplied expert indices (moe_permute on its own).
+__global__ void __launch_bounds__(kRouteThreads)
+    rank_from_indices_kernel(const int32_t* __restrict__ topk_idx, int64_t T, int E, int k,
+                             int32_t* local_rank, int32_t* block_base, unsigned* ticket, int nb,
+                             unsigned* err) {
+    __shared__ uint8_t sel[kTokensPerRouteBlock][256];
+    for (int i = threadIdx.x; i < kTokensPerRouteBlock * 256 / 16; i += blockDim.x)
+        reinterpret_cast<uint4*>(&sel[0][0])[i] = make_uint4(0, 0, 0, 0);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0u;
+    __syncthreads();
+    const int64_t t0 = (int64_t)blockIdx.x * kTokensPerRouteBlock;
+    for (int tt = threadIdx.x; tt < kTokensPerRouteBlock; tt += blockDim.x) {
+        const int64_t t = t0 + tt;
+        if (t >= T) break;
+        for (int j = 0; j < k; ++j) {
+            const int e = topk_idx[t * k + j];
+            local_rank[t * k + j] = -1;  // stays -1 for an invalid or repeated expert
+            if (e < 0 || e >= E || sel[tt][e] != 0) {
+                raise_error(err, kErrDeviceCheck);
+                continue;
+            }
+            sel[tt][e] = (uint8_t)(j + 1);
+        }
+    }
+    __syncthreads();
+    rank_block(sel, t0, T, E, k, local_rank, block_base, nb);
+}
+
+// Inclusive scan over the block (blockDim.x a multiple of 32, <= 1024).
+__device__ __forceinline__ int block_inclusive_scan(int v, int* warp_tot, int& total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(kFull, v, off);
+        if (lane >= off) v += o;
+    }
+    if (lane == 31) warp_tot[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < nw ? warp_tot[lane] : 0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(kFull, w, off);
+            if (lane >= off) w += o;
+        }
+        if (lane < nw) warp_tot[lane] = w;
+    }
+    __syncthreads();
+    if (warp > 0) v += warp_tot[warp - 1];
+    total = warp_tot[nw - 1];
+    __syncthreads();
+    return v;
+}
+
+// One block per expert: exclusive scan of its per-token-block counts. The last
+// block to finish also writes offsets (exclusive scan of the expert counts).
+__global__ void __launch_bounds__(1024)
+    expert_scan_kernel(int32_t* block_base, int nb, int E, int32_t* counts, int32_t* offsets,
+                       unsigned* ticket) {
+    __shared__ int warp_tot[32];
+    __shared__ bool is_last;
+    const int e = blockIdx.x;
+    int32_t* row = block_base + (int64_t)e * nb;
+    int carry = 0;
+    for (int base = 0; base < nb; base += blockDim.x) {
+        const int i = base + threadIdx.x;
+        const int v = i < nb ? row[i] : 0;
+        int total;
+        const int incl = block_inclusive_scan(v, warp_tot, total);
+        if (i < nb) row[i] = carry + incl - v;
+        carry += total;
+    }
+    if (counts == nullptr) return;
+    if (threadIdx.x == 0) {
+        counts[e] = carry;
+        __threadfence();
+        const unsigned done = atomicAdd(ticket, 1u);
+        is_last = (done == (unsigned)E - 1);
+    }
+    __syncthreads();
+    if (is_last && threadIdx.x == 0) {
+        __threadfence();
+        const volatile int32_t* c = counts;
+        int acc = 0;
+        offsets[0] = 0;
+        for (int i = 0; i < E; ++i) {
+            acc += c[i];
+            offsets[i + 1] = acc;
+        }
+        *ticket = 0u;
+    }
+}
+
+// Token dispatch: one warp per token. Lane j < k computes the row of the
+// token's j-th assignment; then the warp copies the token's row (16-byte
+// vectors) to each of its k destinations.
+__global__ void __launch_bounds__(256)
+    permute_kernel(const uint4* __restrict__ x, int64_t T, int H8, const int32_t* __restrict__ topk_idx,
+                   int k, const int32_t* __restrict__ offsets, int E,
+                   const int32_t* __restrict__ block_base, int nb,
+                   const int32_t* __restrict__ local_rank, uint4* __restrict__ x_perm,
+                   int32_t* __restrict__ sorted_token, int32_t* __restrict__ row_of, int64_t A,
+                   unsigned* err) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T;
+         t += warps) {
+        int64_t row = -1;
+        if (lane < k) {
+            const int e = topk_idx[t * k + lane];
+            const int rank = local_rank[t * k + lane];
+            if (e >= 0 && e < E && rank >= 0) {
+                const int64_t r = (int64_t)offsets[e] +
+                                  block_base[(int64_t)e * nb + t / kTokensPerRouteBlock] + rank;
+                if (r >= offsets[e] && r < offsets[e + 1] && r < A) row = r;
+            }
+            if (row < 0) raise_error(err, kErrDeviceCheck);
+            row_of[t * k + lane] = (int32_t)row;
+            if (row >= 0) sorted_token[row] = (int32_t)t;
+        }
+        int64_t rows[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) rows[j] = (j < k) ? __shfl_sync(kFull, row, j) : -1;
+        const uint4* src = x + t * H8;
+        int c = lane;
+        for (; c + 32 < H8; c += 64) {  // two 16-byte loads in flight per lane
+            const uint4 v0 = __ldg(src + c);
+            const uint4 v1 = __ldg(src + c + 32);
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                if (rows[j] >= 0) {
+                    x_perm[rows[j] * H8 + c] = v0;
+                    x_perm[rows[j] * H8 + c + 32] = v1;
+                }
+        }
+        for (; c < H8; c += 32) {
+            const uint4 v0 = __ldg(src + c);
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                if (rows[j] >= 0) x_perm[rows[j] * H8 + c] = v0;
+        }
+    }
+}
+
+}  // namespace
+
+size_t route_scratch_bytes(int64_t T, int E, int k) {
+    const int64_t nb = route_blocks(T);
+    size_t b = (size_t)E * nb * 4;
+    b = (b + 255) & ~size_t(255);
+    b += (size_t)T * k * 4;
+    b = (b + 255) & ~size_t(255);
+    b += 256;
+    return b;
+}
+
+RouteScratch carve_route_scratch(void* base, int64_t T, int E, int k) {
+    const int64_t nb = route_blocks(T);
+    char* p = static_cast<char*>(base);
+    RouteScratch rs;
+    rs.block_base = reinterpret_cast<int32_t*>(p);
+    size_t off = ((size_t)E * nb * 4 + 255) & ~size_t(255);
+    rs.local_rank = reinterpret_cast<int32_t*>(p + off);
+    off = (off + (size_t)T * k * 4 + 255) & ~size_t(255);
+    rs.ticket = reinterpret_cast<unsigned*>(p + off);
+    return rs;
+}
+
+cudaError_t launch_router_topk(const float* logits, int64_t T, int E, int k,
+                               const moe_router_opts& opts, int32_t* topk_idx, float* topk_prob,
+                               uint8_t* routing_map, const RouteScratch& rs, cudaStream_t st,
+                               unsigned* err) {
+    RouterArgs a;
+    a.logits = logits;
+    a.T = T;
+    a.E = E;
+    a.k = k;
+    a.score_fn = opts.score_fn;
+    a.renormalize = opts.renormalize;
+    a.scaling = opts.scaling;
+    a.bias = opts.expert_bias;
+    a.topk_idx = topk_idx;
+    a.topk_prob = topk_prob;
+    a.routing_map = routing_map;
+    a.block_base = rs.block_base;
+    a.local_rank = rs.local_rank;
+    a.ticket = rs.ticket;
+    a.nb = (int)route_blocks(T);
+    const dim3 grid((unsigned)a.nb), block(kRouteThreads);
+    if (E <= 32) router_topk_kernel<1><<<grid, block, 0, st>>>(a);
+    else if (E <= 64) router_topk_kernel<2><<<grid, block, 0, st>>>(a);
+    else if (E <= 128) router_topk_kernel<4><<<grid, block, 0, st>>>(a);
+    else router_topk_kernel<8><<<grid, block, 0, st>>>(a);
+    (void)err;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_rank_from_indices(const int32_t* topk_idx, int64_t T, int E, int k,
+                                     const RouteScratch& rs, cudaStream_t st, unsigned* err) {
+    const int nb = (int)route_blocks(T);
+    rank_from_indices_kernel<<<nb, kRouteThreads, 0, st>>>(topk_idx, T, E, k, rs.local_rank,
+                                                          rs.block_base, rs.ticket, nb, err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_expert_scan(int64_t T, int E, const RouteScratch& rs, int32_t* counts,
+                               int32_t* offsets, cudaStream_t st) {
+    const int nb = (int)route_blocks(T);
+    int threads = 32;
+    while (threads < nb && threads < 1024) threads <<= 1;
+    expert_scan_kernel<<<E, threads, 0, st>>>(rs.block_base, nb, E, counts, offsets, rs.ticket);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_permute(const bf16* x, int64_t T, int H, const int32_t* topk_idx, int k,
+                           const int32_t* offsets, int E, const RouteScratch& rs, bf16* x_perm,
+                           int32_t* sorted_token, int32_t* row_of, cudaStream_t st, unsigned* err) {
+    const int nb = (int)route_blocks(T);
+    const int64_t warps_needed = T;
+    int64_t blocks = (warps_needed + 7) / 8;
+    const int64_t cap = (int64_t)sm_count() * 8;   // 8 resident 256-thread blocks per SM
+    if (blocks > cap) blocks = cap;
+    permute_kernel<<<(unsigned)blocks, 256, 0, st>>>(
+        reinterpret_cast<const uint4*>(x), T, H / 8, topk_idx, k, offsets, E, rs.block_base, nb,
+        rs.local_rank, reinterpret_cast<uint4*>(x_perm), sorted_token, row_of, T * k, err);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

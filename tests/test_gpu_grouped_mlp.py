@@ -1,0 +1,90 @@
+"""Grouped SwiGLU MLP parity on the GPU (Transformer Engine "Mixture of
+Experts", Grouped GEMM and Grouped MLP), through the C ABI, against the
+oracle's per-expert loop. Shapes span several 128x256 tiles, ragged expert
+blocks and empty experts."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as wl
+from helpers import assert_close, bits, require_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def grouped_case(T, H, I, E, k, seed, dead=(), skew=False):
+    w = wl.WORKLOADS["tiny"].scaled(T=T, H=H, I=I, E=E, k=k, seed=seed, skew=skew,
+                                     dead_experts=0)
+    d = wl.make_inputs(w, "cuda")
+    logits = d["logits"]
+    for e in dead:
+        logits[:, e] -= 1e4
+    import routing_grouped_gemm_score_b200 as m
+    r = m.moe_router_topk(logits, k)
+    p = m.moe_permute(d["x"], r["topk_idx"], r["offsets"])
+    return m, w, d, r, p
+
+
+@pytest.mark.parametrize("T,H,I,E,k,dead", [
+    (64, 128, 256, 8, 2, ()),            # the tiny workload's shape
+    (1000, 256, 384, 4, 2, (2,)),        # several M tiles per expert, a ragged tail, an empty expert
+    (300, 512, 192, 8, 2, (0, 7)),       # I not a multiple of 128: half-empty SwiGLU tile
+    (700, 320, 640, 16, 4, ()),          # H not a multiple of 256: ragged N tile in the down GEMM
+    (1, 128, 128, 8, 2, ()),             # a single token
+])
+def test_grouped_mlp_matches_expert_loop(T, H, I, E, k, dead):
+    m, w, d, r, p = grouped_case(T, H, I, E, k, seed=T + H + I, dead=dead)
+    out = m.moe_grouped_mlp(p["x_perm"], r["offsets"], d["w_gate_up"], d["w_down"], save=True)
+    torch.cuda.synchronize()
+    assert m.moe_get_device_status() == 0
+    offs = r["offsets"].cpu().numpy()
+    for e in dead:
+        assert offs[e + 1] == offs[e]
+    xp = bits(p["x_perm"])
+    wgu, wd = bits(d["w_gate_up"]), bits(d["w_down"])
+    y_ref = oracle.grouped_mlp(xp, offs, wgu, wd, round_bf16=True)
+    assert_close(out["y_perm"], y_ref, "y_perm")
+    # intermediates: g, u and h of every row
+    for e in range(E):
+        r0, r1 = offs[e], offs[e + 1]
+        if r1 == r0:
+            continue
+        y, g, u, h = oracle.expert_mlp(xp[r0:r1], wgu[e], wd[e], round_bf16=True, want_intermediates=True)
+        assert_close(out["gu"][r0:r1, :I], g, f"g of expert {e}")
+        assert_close(out["gu"][r0:r1, I:], u, f"u of expert {e}")
+        assert_close(out["h"][r0:r1], h, f"h of expert {e}")
+
+
+def test_grouped_mlp_is_deterministic():
+    m, w, d, r, p = grouped_case(512, 256, 256, 8, 2, seed=3)
+    a = m.moe_grouped_mlp(p["x_perm"], r["offsets"], d["w_gate_up"], d["w_down"])["y_perm"]
+    b = m.moe_grouped_mlp(p["x_perm"], r["offsets"], d["w_gate_up"], d["w_down"])["y_perm"]
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_rows_past_offsets_end_are_untouched():
+    """offsets[E] < A: rows after the last expert block are not written."""
+    import routing_grouped_gemm_score_b200 as m
+    E, H, I = 4, 128, 128
+    A = 300
+    offsets = torch.tensor([0, 50, 50, 170, 200], dtype=torch.int32, device="cuda")
+    g_ = torch.Generator(device="cuda").manual_seed(1)
+    x = torch.randn((A, H), generator=g_, device="cuda").to(torch.bfloat16)
+    wgu = (torch.randn((E, H, 2 * I), generator=g_, device="cuda") / H ** 0.5).to(torch.bfloat16)
+    wd = (torch.randn((E, I, H), generator=g_, device="cuda") / I ** 0.5).to(torch.bfloat16)
+    y = torch.full((A, H), 7.0, device="cuda").to(torch.bfloat16)
+    ws = torch.empty(m.lib().moe_grouped_mlp_workspace_size(A, E, H, I), dtype=torch.uint8, device="cuda")
+    rc = m.lib().moe_grouped_mlp(x.data_ptr(), A, offsets.data_ptr(), E, H, I, wgu.data_ptr(),
+                                 wd.data_ptr(), y.data_ptr(), None, None, ws.data_ptr(), ws.numel(),
+                                 torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert torch.all(y[200:].float() == 7.0)
+    ref = oracle.grouped_mlp(bits(x), offsets.cpu().numpy(), bits(wgu), bits(wd))
+    assert_close(y[:200], ref[:200], "y_perm")

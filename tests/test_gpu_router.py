@@ -1,0 +1,98 @@
+"""Router parity on the GPU: topk_idx, routing_map, counts and offsets
+bit-exact, routing weights within 1e-6 relative, against the oracle on the
+same seeded logits (Transformer Engine "Mixture of Experts", Router)."""
+import numpy as np
+import pytest
+import torch
+
+import workloads as wl
+from helpers import assert_equal, require_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def run_both(logits, k, score=0, renormalize=True, scaling=1.0, bias=None):
+    import oracle
+    import routing_grouped_gemm_score_b200 as m
+    opts = m.RouterOpts(score, renormalize, scaling, None if bias is None else bias.cuda())
+    g = m.moe_router_topk(logits.cuda(), k, opts, routing_map=True)
+    torch.cuda.synchronize()
+    assert m.moe_get_device_status() == 0
+    r = oracle.router_topk(logits.cpu().numpy(), k, score, renormalize, scaling,
+                           None if bias is None else bias.cpu().numpy())
+    return g, r
+
+
+def check(g, r):
+    assert_equal(g["topk_idx"], r["topk_idx"], "topk_idx")
+    assert_equal(g["routing_map"], r["routing_map"], "routing_map")
+    assert_equal(g["counts"], r["counts"], "counts")
+    assert_equal(g["offsets"], r["offsets"], "offsets")
+    np.testing.assert_allclose(g["topk_prob"].cpu().numpy(), r["topk_prob"], rtol=1e-6, atol=0)
+
+
+@pytest.mark.parametrize("name", ["tiny", "mixtral_8x7b", "qwen3_30b_a3b", "llama4_17bx16e",
+                                  "skew_t1", "skew_t8", "skew_t64", "skew_t16384", "tie_t64"])
+def test_router_workloads(name):
+    w = wl.WORKLOADS[name]
+    logits = wl.make_logits(w, "cuda")
+    g, r = run_both(logits, w.k, w.score, w.renormalize)
+    check(g, r)
+
+
+@pytest.mark.parametrize("E,k", [(1, 1), (7, 3), (31, 4), (32, 8), (33, 1), (64, 16), (100, 6),
+                                 (129, 8), (256, 16), (256, 1)])
+def test_router_shapes_ragged_token_blocks(E, k):
+    g_ = torch.Generator().manual_seed(E * 17 + k)
+    logits = torch.randn((193, E), generator=g_)      # 193 = three token blocks + a tail
+    g, r = run_both(logits, k)
+    check(g, r)
+
+
+def test_router_ties_and_degenerate_values():
+    g_ = torch.Generator().manual_seed(5)
+    logits = torch.round(torch.randn((300, 64), generator=g_) * 2) / 2
+    logits[0] = 0.0
+    logits[1, ::3] = float("-inf")
+    logits[2, 5] = float("nan")
+    logits[3] = -0.0
+    logits[3, 10] = 0.0
+    logits[4, :] = float("-inf")
+    logits[4, 7] = 1.0
+    g, r = run_both(logits, 8)
+    assert_equal(g["topk_idx"], r["topk_idx"], "topk_idx")
+    assert_equal(g["counts"], r["counts"], "counts")
+    gp, rp = g["topk_prob"].cpu().numpy(), r["topk_prob"]
+    finite = np.isfinite(rp)
+    np.testing.assert_allclose(gp[finite], rp[finite], rtol=1e-6, atol=0)
+    assert np.array_equal(np.isnan(gp), np.isnan(rp))
+
+
+def test_router_options():
+    g_ = torch.Generator().manual_seed(9)
+    logits = torch.randn((500, 48), generator=g_) * 2
+    check(*run_both(logits, 6, renormalize=False))                  # softmax before top-k
+    check(*run_both(logits, 6, score=1, renormalize=False))         # sigmoid
+    check(*run_both(logits, 6, score=1, renormalize=True))          # sigmoid, renormalised
+    check(*run_both(logits, 6, scaling=2.5))                        # scaling factor
+    bias = torch.randn(48, generator=g_) * 0.3
+    check(*run_both(logits, 6, score=1, renormalize=False, bias=bias))
+
+
+def test_router_empty_batch():
+    import routing_grouped_gemm_score_b200 as m
+    g = m.moe_router_topk(torch.empty((0, 16), device="cuda"), 2)
+    assert g["counts"].sum().item() == 0 and g["offsets"].abs().sum().item() == 0
+
+
+def test_router_large_sweep_invariants():
+    """T = 2^18 tokens at E=128, k=8: checked against the oracle on every row."""
+    g_ = torch.Generator().manual_seed(21)
+    logits = torch.randn((1 << 18, 128), generator=g_)
+    g, r = run_both(logits, 8)
+    check(g, r)
