@@ -373,21 +373,28 @@ int oracle_moe_forward_tokens(const uint16_t* x, const float* logits, int H, int
  * routing (topk_idx, topk_prob) and upstream gradient dout. It is the chain
  * rule applied to the forward above. [TE] Example: every stage is
  * differentiable. The routing weights are an input here, so nothing flows into
- * the logits. The bf16 rounding of h and y is treated as the identity.
+ * the logits.
  * Per assignment (t, j) with e = topk_idx[t,j] and p = topk_prob[t,j]:
  *   y = MLP_e(x_t);           dprob[t,j] = <dout_t, y>
  *   dy = p * dout_t;          dWd[e]   += h^T dy
  *   dh = dy . Wd[e]^T;        du = dh * silu(g);  dg = dh * u * silu'(g)
  *   silu'(g) = s + g s (1 - s),  s = 1 / (1 + e^-g)
  *   dWgu[e][:, 0:I] += x_t^T dg;   dWgu[e][:, I:2I] += x_t^T du
- *   dx_t += dg . Wgu[e][:, 0:I]^T + du . Wgu[e][:, I:2I]^T
- * All in fp64. only_expert >= 0 restricts the sums to that expert's
+ *   dxp = dg . Wgu[e][:, 0:I]^T + du . Wgu[e][:, I:2I]^T;   dx_t += dxp
+ * All in fp64. With round_bf16, every tensor that a bf16 pipeline stores
+ * between its stages is rounded to bf16, as in the forward: the saved FC1
+ * outputs g and u that the SwiGLU backward reads; the gradient dy of the
+ * bf16 expert output; the gradients dg, du of the bf16 FC1 output; and the
+ * gradient dxp of each bf16 permuted token row, which the unpermute then sums.
+ * The rounding functions themselves pass gradients through unchanged.
+ * With round_bf16 = 0, nothing is rounded, and the result is the exact
+ * derivative that the finite-difference pin checks.
+ * only_expert >= 0 restricts the sums to that expert's
  * assignments. token_list (NULL = all T tokens) restricts t, and dx / dprob
  * rows are then written in list order. With only_expert >= 0 the dw_* outputs
  * hold that one expert ([H,2I] and [I,H]), else all E. Output pointers may be
- * NULL. Every
- * non-NULL output is zeroed first, so an expert that gets no assignment has a
- * zero weight gradient.
+ * NULL. Every non-NULL output is zeroed first, so an expert that gets no
+ * assignment has a zero weight gradient.
  */
 int oracle_moe_backward(const uint16_t* x, int64_t T, int H, int I, int E, int k,
                         const int32_t* topk_idx, const float* topk_prob,
@@ -426,7 +433,15 @@ int oracle_moe_backward(const uint16_t* x, int64_t T, int H, int I, int E, int k
                 for (int c = 0; c < H; c++) s += bf16_to_double(dot[c]) * y[c];
                 dprob[n * k + j] = s;
             }
-            for (int c = 0; c < H; c++) dy[c] = p * bf16_to_double(dot[c]);
+            if (round_bf16)
+                for (int i = 0; i < I; i++) {
+                    g[i] = bf16_to_double(double_to_bf16(g[i]));
+                    u[i] = bf16_to_double(double_to_bf16(u[i]));
+                }
+            for (int c = 0; c < H; c++) {
+                dy[c] = p * bf16_to_double(dot[c]);
+                if (round_bf16) dy[c] = bf16_to_double(double_to_bf16(dy[c]));
+            }
             if (dw_down) {
                 double* dwd = dw_down + (only_expert >= 0 ? 0 : (int64_t)e * I * H);
                 for (int i = 0; i < I; i++)
@@ -442,6 +457,10 @@ int oracle_moe_backward(const uint16_t* x, int64_t T, int H, int I, int E, int k
                 double a = g[i] * sg;                      /* silu(g) */
                 du[i] = dh[i] * a;
                 dg[i] = dh[i] * u[i] * (sg + g[i] * sg * (1.0 - sg));
+                if (round_bf16) {
+                    du[i] = bf16_to_double(double_to_bf16(du[i]));
+                    dg[i] = bf16_to_double(double_to_bf16(dg[i]));
+                }
             }
             if (dw_gate_up) {
                 double* dw = dw_gate_up + (only_expert >= 0 ? 0 : (int64_t)e * H * 2 * I);
@@ -458,6 +477,7 @@ int oracle_moe_backward(const uint16_t* x, int64_t T, int H, int I, int E, int k
                     double s = 0.0;
                     for (int i = 0; i < I; i++)
                         s += dg[i] * bf16_to_double(row[i]) + du[i] * bf16_to_double(row[I + i]);
+                    if (round_bf16) s = bf16_to_double(double_to_bf16(s));
                     dxr[hh] += s;
                 }
             }

@@ -88,8 +88,38 @@ def test_backward_matches_finite_differences(oracle_lib):
     assert checked == 36 + w.T * w.k
 
 
+class _RoundValue(torch.autograd.Function):
+    """Forward: round to bf16. Backward: gradient passed through unchanged."""
+    @staticmethod
+    def forward(ctx, v):
+        return v.float().to(torch.bfloat16).double()
+
+    @staticmethod
+    def backward(ctx, g):
+        return g
+
+
+class _RoundGrad(torch.autograd.Function):
+    """Forward: identity. Backward: the gradient is rounded to bf16 (a stored
+    gradient tensor of a bf16 pipeline)."""
+    @staticmethod
+    def forward(ctx, v):
+        return v.clone()
+
+    @staticmethod
+    def backward(ctx, g):
+        return g.float().to(torch.bfloat16).double()
+
+
+def _round_both(v):
+    return _RoundGrad.apply(_RoundValue.apply(v))
+
+
 @pytest.mark.parametrize("round_bf16", [False, True])
 def test_backward_matches_torch_autograd(oracle_lib, round_bf16):
+    """torch autograd of the layer written with torch primitives. With
+    rounding: the stored tensors (g, u, h, y) round their values, and the
+    stored gradients (dy, dg, du, dx_perm) round theirs."""
     w, d = setup(T=24, H=32, I=24, E=5, k=2, seed=3)
     bits = oracle_lib.bf16_bits
     r = oracle_lib.router_topk(d["logits"].numpy(), w.k)
@@ -103,12 +133,17 @@ def test_backward_matches_torch_autograd(oracle_lib, round_bf16):
     for t in range(w.T):
         for j in range(w.k):
             e = int(idx[t, j])
-            h = F.silu(x[t] @ wgu[e][:, :I]) * (x[t] @ wgu[e][:, I:])
-            if round_bf16:      # straight-through rounding: value rounded, gradient identity
-                h = h + (h.detach().float().to(torch.bfloat16).double() - h.detach())
-            y = h @ wd[e]
+            xr = _RoundGrad.apply(x[t]) if round_bf16 else x[t]
+            g = xr @ wgu[e][:, :I]
+            u = xr @ wgu[e][:, I:]
             if round_bf16:
-                y = y + (y.detach().float().to(torch.bfloat16).double() - y.detach())
+                gb, ub = _round_both(g), _round_both(u)
+                # value from the unrounded g, u; gradient through the stored g, u
+                h = F.silu(gb) * ub + (F.silu(g) * u - F.silu(gb) * ub).detach()
+                h = _RoundValue.apply(h)
+                y = _round_both(h @ wd[e])
+            else:
+                y = (F.silu(g) * u) @ wd[e]
             out[t] = out[t] + prob[t, j] * y
     (out * d["dout"].double()).sum().backward()
     g = oracle_lib.moe_backward(bits(d["x"]), r["topk_idx"], r["topk_prob"], bits(d["w_gate_up"]),
