@@ -1,0 +1,460 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 MoE layer: tokens/s of the whole layer step and
+TFLOP/s of the grouped expert GEMMs, as a fraction of the measured peak.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+A step is one pass of the whole layer over one batch of seeded synthetic
+tokens: router -> permute -> grouped SwiGLU MLP -> combine (a forward pass,
+plus the grouped-MLP backward for workloads that train). It is one call of
+moe_layer_forward (and moe_grouped_mlp_backward) through the C ABI. Inputs
+are already resident in HBM when the timed region starts. The weights exceed
+L2 (126 MB), which keeps the steps L2-cold without a flush. Rank 0 prints one
+JSON line.
+
+With N > 1 (torchrun), each rank runs its own replica of the layer on its own
+tokens (data-parallel replicas; the forward has no exchange step). value =
+tokens of all ranks / the slowest rank's time. --impl reference times the CPU
+oracle (the plain restatement the tests compare against) on the host cores of
+rank 0, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer tokens/s and grouped-GEMM TFLOP/s (% of B200 bf16 peak), 1 GPU"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "mixtral_8x7b"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--T", type=int, default=None,
+                    help="override the token count (small cases for profiling)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.15)
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.tmp.flush()
+        self.tmp.seek(0)
+        rows = [r.strip().split(",") for r in self.tmp.read().splitlines() if r.strip()]
+        os.unlink(self.tmp.name)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [c.strip() for c in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ dist
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ CPU baseline
+class OracleRunner:
+    """The oracle's per-token layer (and, for training workloads, its
+    backward for dx and the routing-weight gradient) on host copies of the
+    workload's inputs."""
+
+    def __init__(self, w, inputs_cpu, threads):
+        import oracle
+        bits = oracle.bf16_bits
+        self.w, self.threads, self.oracle = w, threads, oracle
+        self.x = bits(inputs_cpu["x"])
+        self.logits = inputs_cpu["logits"].numpy()
+        self.wgu = bits(inputs_cpu["w_gate_up"])
+        self.wd = bits(inputs_cpu["w_down"])
+        sg, sd = inputs_cpu["shared_gate_up"], inputs_cpu["shared_down"]
+        self.sgu = None if sg is None else bits(sg[0])
+        self.sd = None if sd is None else bits(sd[0])
+        self.dout = bits(inputs_cpu["dout"]) if "dout" in inputs_cpu else None
+
+    def run(self, tokens):
+        w, o = self.w, self.oracle
+        o.moe_forward_tokens(self.x, self.logits, self.wgu, self.wd, w.k, tokens=tokens,
+                             score=w.score, renormalize=w.renormalize, shared_gu_bits=self.sgu,
+                             shared_d_bits=self.sd, threads=self.threads)
+        if self.dout is not None:
+            r = o.router_topk(self.logits[tokens], w.k, w.score, w.renormalize, with_map=False)
+            o.moe_backward(self.x[tokens], r["topk_idx"], r["topk_prob"], self.wgu, self.wd,
+                           self.dout[tokens], want=("dx", "dprob"))
+
+    def sample_for(self, budget_s):
+        """Tokens (spread over the batch) that take about budget_s seconds."""
+        import numpy as np
+        n = max(1, self.threads)
+        t0 = time.perf_counter()
+        self.run(np.arange(n))
+        dt = time.perf_counter() - t0
+        n2 = int(max(n, min(self.w.T, n * budget_s / max(dt, 1e-6))))
+        n2 = max(n, (n2 // n) * n)
+        return np.linspace(0, self.w.T - 1, n2).astype(np.int64)
+
+    def time(self, tokens):
+        t0 = time.perf_counter()
+        self.run(tokens)
+        return time.perf_counter() - t0
+
+
+def cpu_inputs(w, d):
+    """Host copies of the device inputs (the oracle reads exactly these bytes)."""
+    return {k: (None if v is None else v.detach().to("cpu")) for k, v in d.items()}
+
+
+def reference_arm(args, world, rank):
+    if rank != 0:
+        return 0
+    import torch
+
+    import workloads as wl
+    w = workload(args)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    d = wl.make_inputs(w, dev)
+    threads = os.cpu_count() or 1
+    runner = OracleRunner(w, cpu_inputs(w, d), threads)
+    tokens = runner.sample_for(0.5)
+    for _ in range(args.warmup):
+        runner.time(tokens)
+    elapsed = sum(runner.time(tokens) for _ in range(args.steps))
+    value = len(tokens) * args.steps / elapsed
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_dict(w, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{len(tokens)} of {w.T} tokens of the workload per step "
+                                   f"(plain C oracle, fp64 accumulation, {threads} host threads)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def workload(args):
+    import workloads as wl
+    w = wl.WORKLOADS[args.workload]
+    return w.scaled(T=args.T) if args.T else w
+
+
+def config_dict(w, args):
+    return {"workload": w.name, "T": w.T, "H": w.H, "I": w.I, "E": w.E, "top_k": w.k,
+            "score": "sigmoid" if w.score == 1 else "softmax",
+            "shared_expert": w.shared_expert, "pass": "fwd+bwd" if w.backward else "fwd",
+            "global_batch_tokens": w.T * max(1, args.gpus),
+            "l2": "inputs larger than L2 (weights exceed 126 MB); no flush",
+            "parallelism": f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"}
+
+
+def source_sha(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def traffic_for(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if the
+    kernel's source has not changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = t.get(kernel)
+    if not e:
+        return None
+    src = os.path.join(ROOT, e["source"])
+    if not os.path.exists(src) or source_sha(src) != e.get("source_sha"):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ our arm
+def our_arm(args, world, rank, local):
+    import torch
+
+    import routing_grouped_gemm_score_b200 as m
+    import workloads as wl
+    from routing_grouped_gemm_score_b200 import build as bld
+    bld.build()
+    torch.cuda.set_device(local)
+    w = workload(args)
+    # each rank its own tokens (seeded per rank), the same weights
+    d = wl.make_inputs(w, "cuda")
+    if rank:
+        wr = w.scaled(seed=w.seed + 1000 * rank)
+        d["logits"] = wl.make_logits(wr, "cuda")
+        d["x"] = wl.make_x(wr, "cuda")
+        if w.backward:
+            d["dout"] = wl.make_dout(wr, "cuda")
+    opts = m.RouterOpts(w.score, w.renormalize)
+    ws = m.LayerWorkspace(w.T, w.H, w.I, w.E, w.k, w.shared_expert, backward=w.backward)
+    out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device="cuda")
+    state = None
+    grads = None
+    if w.backward:
+        _, state = m.moe_layer_forward(d["logits"], d["x"], d["w_gate_up"], d["w_down"], w.k, opts,
+                                       save_for_backward=True, workspace=ws, out=out)
+        grads = m.moe_grouped_mlp_backward(d["dout"], state, d["w_gate_up"], d["w_down"], ws)
+
+    nfev = 7
+    def step(fev=None, bev=None):
+        if fev:
+            m.moe_trace_set(fev)
+        m.moe_layer_forward(d["logits"], d["x"], d["w_gate_up"], d["w_down"], w.k, opts,
+                            d["shared_gate_up"], d["shared_down"], save_for_backward=w.backward,
+                            workspace=ws, out=out, state=state)
+        if w.backward:
+            if bev:
+                m.moe_trace_set(bev)
+            m.moe_grouped_mlp_backward(d["dout"], state, d["w_gate_up"], d["w_down"], ws, grads)
+        if fev or bev:
+            m.moe_trace_set(None)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if m.moe_get_device_status() != 0:
+        raise RuntimeError("device status error after warm-up")
+
+    K = args.steps
+    fevs = [[torch.cuda.Event(enable_timing=True) for _ in range(nfev)] for _ in range(K)]
+    bevs = [[torch.cuda.Event(enable_timing=True) for _ in range(nfev)] for _ in range(K)] if w.backward else [None] * K
+    for evs in fevs + ([e for e in bevs if e] if w.backward else []):
+        for e in evs:
+            e.record()           # materialise the events before handing them to the library
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    start.record()
+    for i in range(K):
+        step(fevs[i], bevs[i])
+    end.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier(world)
+    ms = start.elapsed_time(end)
+    ms_max = max_over_ranks(ms, world)
+    if m.moe_get_device_status() != 0:
+        raise RuntimeError("device status error in the timed region")
+
+    def stage_ms(evsets, i):
+        return statistics.mean(evs[i].elapsed_time(evs[i + 1]) for evs in evsets)
+    fwd_stages = ["router", "permute", "gate_up_swiglu", "down", "shared_expert", "combine"]
+    stages = {f"fwd_{n}": stage_ms(fevs, i) for i, n in enumerate(fwd_stages)}
+    if w.backward:
+        bwd_stages = ["combine_bwd", "down_dgrad_swiglu_bwd", "gate_up_dgrad", "dx_token_sum",
+                      "down_wgrad", "gate_up_wgrad"]
+        stages.update({f"bwd_{n}": stage_ms(bevs, i) for i, n in enumerate(bwd_stages)})
+
+    tokens_total = w.T * world
+    value = tokens_total * K / (ms_max / 1e3)
+    peaks, peaks_src = load_peaks()
+    long_region = ms / 1e3 >= 1.0
+    peak_tf = peaks["bf16_tflops_sustained" if long_region else "bf16_tflops"]
+    A = w.A
+    gate_up_flop = 4.0 * A * w.H * w.I
+    gate_up_ms = stages["fwd_gate_up_swiglu"]
+    achieved = gate_up_flop / (gate_up_ms / 1e3) / 1e12
+    gemm_ms = stages["fwd_gate_up_swiglu"] + stages["fwd_down"] + (stages["fwd_shared_expert"] if w.shared_expert else 0.0)
+    gemm_flop = w.fwd_flops()
+    if w.backward:
+        gemm_ms += sum(stages[k] for k in ("bwd_down_dgrad_swiglu_bwd", "bwd_gate_up_dgrad",
+                                           "bwd_down_wgrad", "bwd_gate_up_wgrad"))
+        gemm_flop += w.bwd_flops()
+    gemm_tflops = gemm_flop / (gemm_ms / 1e3) / 1e12
+
+    launches_fwd = 6 + (2 if w.shared_expert else 0)
+    launches = K * (launches_fwd + (6 if w.backward else 0))
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_max / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_dict(w, args),
+        "grouped_gemm": {"tflops": gemm_tflops, "frac_of_peak": gemm_tflops / peak_tf,
+                         "peak_tflops": peak_tf, "flop_per_step": gemm_flop,
+                         "note": "expert GEMM FLOPs (6AHI fwd, 12AHI bwd) / device time of the GEMM stages"},
+        "roofline": {"bound": "tensor", "kernel": "grouped_gemm_kernel<SwiGLU> (gate_up)",
+                     "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": achieved / peak_tf,
+                     "traffic": traffic_for("gate_up_swiglu"),
+                     "peak_source": f"{peaks_src} {'sustained' if long_region else 'burst'} bf16",
+                     "flop_per_launch": gate_up_flop, "ms_per_launch": gate_up_ms},
+        "stages_ms": stages,
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+
+    if not args.no_e2e:
+        line["e2e"] = e2e_measure(args, w, d, m, opts, ws, world)
+    if not args.no_cpu_baseline and world == 1 and rank == 0:
+        threads = os.cpu_count() or 1
+        runner = OracleRunner(w, cpu_inputs(w, d), threads)
+        tokens = runner.sample_for(10.0)
+        n = len(tokens)
+        tps = n / runner.time(tokens)
+        line["cpu_baseline"] = {"value": tps, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": f"{n} of {w.T} tokens of the same workload"
+                                          f"{' (fwd + dx/dprob bwd)' if w.backward else ''}, "
+                                          f"plain C oracle, fp64 accumulation"}
+    if rank == 0:
+        print(json.dumps(line))
+    return 0
+
+
+def e2e_measure(args, w, d, m, opts, ws, world):
+    """Same metric through the public call with host buffers: every step
+    copies its inputs (logits, x) from pinned host memory to the device and
+    reads the layer output back, inside the timed region."""
+    import torch
+    h_logits = d["logits"].cpu().pin_memory()
+    h_x = d["x"].cpu().pin_memory()
+    h_out = torch.empty((w.T, w.H), dtype=torch.bfloat16).pin_memory()
+    dl = torch.empty_like(d["logits"])
+    dx = torch.empty_like(d["x"])
+    out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device="cuda")
+    K = max(1, min(args.steps, 50))
+
+    def step():
+        dl.copy_(h_logits, non_blocking=True)
+        dx.copy_(h_x, non_blocking=True)
+        m.moe_layer_forward(dl, dx, d["w_gate_up"], d["w_down"], w.k, opts, d["shared_gate_up"],
+                            d["shared_down"], workspace=ws, out=out)
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(K):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(s.elapsed_time(e), world)
+    return {"value": w.T * world * K / (ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": h_logits.numel() * 4 + h_x.numel() * 2,
+            "d2h_bytes_per_step": h_out.numel() * 2, "steps": K,
+            "pass": "fwd", "note": "weights resident on the device"}
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            return reference_arm(args, world, rank)
+        return our_arm(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -86,6 +86,20 @@ const char* moe_status_string(moe_status status);
  * Returns MOE_OK, MOE_ERR_DEVICE_CHECK, MOE_ERR_TIMEOUT or MOE_ERR_CUDA. */
 moe_status moe_get_device_status(void* stream);
 
+/* Stage tracing. `events` points to n_events cudaEvent_t handles that the
+ * caller created (with timing enabled) and owns; NULL or n_events = 0 turns
+ * tracing off. While set, moe_layer_forward records them on its stream at its
+ * stage boundaries, in this order:
+ *   [0] start  [1] router + offsets  [2] permute  [3] gate_up + SwiGLU
+ *   [4] down   [5] shared expert (recorded even without one)  [6] combine
+ * and moe_grouped_mlp_backward records:
+ *   [0] start  [1] combine backward  [2] down dgrad + SwiGLU backward
+ *   [3] gate_up dgrad  [4] token sum of dx  [5] down wgrad  [6] gate_up wgrad
+ * Events beyond n_events are skipped. The elapsed time between consecutive
+ * events is the device time of one stage. The setting is process-wide and
+ * not thread-safe. Returns MOE_ERR_INVALID_ARG if n_events < 0. */
+moe_status moe_trace_set(void* const* events, int n_events);
+
 /* ------------------------------------------------------------------ router
  * moe_router_topk -- TE Router (fused_topk_with_score_function); te_mixtral.py
  * TEMixtralSparseMoeBlock.forward (fp32 softmax, top-k, renormalise).

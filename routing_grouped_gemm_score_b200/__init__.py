@@ -25,7 +25,7 @@ __all__ = [
     "MoEError", "RouterOpts", "SCORE_SOFTMAX", "SCORE_SIGMOID", "library_path", "lib",
     "moe_status_string", "moe_get_device_status", "moe_router_topk", "moe_permute",
     "moe_grouped_mlp", "moe_unpermute_combine", "moe_layer_forward", "moe_grouped_mlp_backward",
-    "ABI_FUNCTIONS",
+    "moe_trace_set", "LayerWorkspace", "ABI_FUNCTIONS",
 ]
 
 SCORE_SOFTMAX = 0
@@ -73,6 +73,7 @@ P, I64, I32, F32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_f
 ABI_FUNCTIONS = {
     "moe_status_string": (ctypes.c_char_p, [I32]),
     "moe_get_device_status": (I32, [P]),
+    "moe_trace_set": (I32, [ctypes.POINTER(ctypes.c_void_p), I32]),
     "moe_router_workspace_size": (SZ, [I64, I32, I32]),
     "moe_router_topk": (I32, [P, I64, I32, I32, ctypes.POINTER(_RouterOptsC), P, P, P, P, P, P, SZ, P]),
     "moe_permute_workspace_size": (SZ, [I64, I32, I32]),
@@ -150,6 +151,17 @@ def moe_get_device_status() -> int:
     """Synchronise the current stream and return (and clear) the device error
     status: MOE_OK, or the code of the first problem a kernel recorded."""
     return int(lib().moe_get_device_status(_stream()))
+
+
+def moe_trace_set(events) -> None:
+    """Record the given torch.cuda.Event objects (timing enabled, already
+    recorded once so that they exist) at the stage boundaries of the next
+    calls; None turns tracing off. Order of stages: see include/moe_b200.h."""
+    if not events:
+        _check(lib().moe_trace_set(None, 0), "moe_trace_set")
+        return
+    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    _check(lib().moe_trace_set(arr, len(events)), "moe_trace_set")
 
 
 def moe_router_topk(logits: torch.Tensor, k: int, opts: Optional[RouterOpts] = None,

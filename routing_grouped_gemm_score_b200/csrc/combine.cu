@@ -26,6 +26,22 @@ __device__ __forceinline__ void add_scaled(float (&acc)[8], const uint4& v, floa
     }
 }
 
+// dot += <d, y> (in element order); s = p * d
+__device__ __forceinline__ void dot_and_scale(const uint4& d, const uint4& yv, float p, float& dot,
+                                              float (&s)[8]) {
+    const uint32_t dw[4] = {d.x, d.y, d.z, d.w};
+    const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 df = unpack_bf16x2(dw[i]);
+        const float2 yf = unpack_bf16x2(yw[i]);
+        dot += df.x * yf.x;
+        dot += df.y * yf.y;
+        s[2 * i] = p * df.x;
+        s[2 * i + 1] = p * df.y;
+    }
+}
+
 __device__ __forceinline__ uint4 pack8(const float (&acc)[8]) {
     return make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
                       pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
@@ -50,32 +66,29 @@ __global__ void __launch_bounds__(256)
                 raise_error(err, kErrDeviceCheck);
             }
         }
-        int64_t rows[16];
-        float ps[16];
+        // two 16-byte column chunks per lane and pass, so that 2k loads are in flight
+        for (int c0 = lane; c0 < H8; c0 += 64) {
+            const int c1 = c0 + 32;
+            const bool two = c1 < H8;
+            float a0[8], a1[8];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            rows[j] = (j < k) ? __shfl_sync(kFull, my_row, j) : -1;
-            ps[j] = (j < k) ? __shfl_sync(kFull, my_p, j) : 0.0f;
-        }
-        for (int c = lane; c < H8; c += 32) {
-            float acc[8];
+            for (int i = 0; i < 8; ++i) a0[i] = a1[i] = 0.0f;
             if (shared) {
-                const uint4 s = __ldg(shared + t * H8 + c);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-                add_scaled(acc, s, 1.0f);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+                add_scaled(a0, __ldg(shared + t * H8 + c0), 1.0f);
+                if (two) add_scaled(a1, __ldg(shared + t * H8 + c1), 1.0f);
             }
-            uint4 v[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-                if (rows[j] >= 0) v[j] = __ldg(y + rows[j] * H8 + c);
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-                if (rows[j] >= 0) add_scaled(acc, v[j], ps[j]);
-            out[t * H8 + c] = pack8(acc);
+#pragma unroll 4
+            for (int j = 0; j < k; ++j) {
+                const int64_t r = __shfl_sync(kFull, my_row, j);
+                const float pj = __shfl_sync(kFull, my_p, j);
+                if (r < 0) continue;
+                const uint4 v0 = __ldg(y + r * H8 + c0);
+                const uint4 v1 = two ? __ldg(y + r * H8 + c1) : make_uint4(0, 0, 0, 0);
+                add_scaled(a0, v0, pj);
+                add_scaled(a1, v1, pj);
+            }
+            out[t * H8 + c0] = pack8(a0);
+            if (two) out[t * H8 + c1] = pack8(a1);
         }
     }
 }
@@ -84,7 +97,8 @@ __global__ void __launch_bounds__(256)
 //   dy_perm[row_of[t,j]] = bf16(p[t,j] * dout[t])
 //   dprob[t,j] = sum_h dout[t,h] * y_perm[row_of[t,j], h]   (fp32)
 // Each lane sums its own columns in order; the warp then reduces in a fixed
-// butterfly, so dprob is the same on every run.
+// butterfly, so dprob is the same on every run. The dout row is read once per
+// assignment; after the first pass it comes from L1.
 __global__ void __launch_bounds__(256)
     combine_backward_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ y,
                             const int32_t* __restrict__ row_of, const float* __restrict__ probs,
@@ -102,48 +116,28 @@ __global__ void __launch_bounds__(256)
             else raise_error(err, kErrDeviceCheck);
             my_p = probs[t * k + lane];
         }
-        int64_t rows[16];
-        float ps[16], dot[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            rows[j] = (j < k) ? __shfl_sync(kFull, my_row, j) : -1;
-            ps[j] = (j < k) ? __shfl_sync(kFull, my_p, j) : 0.0f;
-            dot[j] = 0.0f;
-        }
-        for (int c = lane; c < H8; c += 32) {
-            const uint4 d = __ldg(dout + t * H8 + c);
-            const uint32_t dw[4] = {d.x, d.y, d.z, d.w};
-            float df[8];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float2 f = unpack_bf16x2(dw[i]);
-                df[2 * i] = f.x;
-                df[2 * i + 1] = f.y;
-            }
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                if (rows[j] < 0) continue;
-                const uint4 yv = __ldg(y + rows[j] * H8 + c);
-                const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float2 f = unpack_bf16x2(yw[i]);
-                    dot[j] += df[2 * i] * f.x;
-                    dot[j] += df[2 * i + 1] * f.y;
+        for (int j = 0; j < k; ++j) {
+            const int64_t r = __shfl_sync(kFull, my_row, j);
+            const float pj = __shfl_sync(kFull, my_p, j);
+            float dot = 0.0f;
+            if (r >= 0) {
+                for (int c0 = lane; c0 < H8; c0 += 64) {
+                    const int c1 = c0 + 32;
+                    const bool two = c1 < H8;
+                    const uint4 d0 = __ldg(dout + t * H8 + c0);
+                    const uint4 y0 = __ldg(y + r * H8 + c0);
+                    const uint4 d1 = two ? __ldg(dout + t * H8 + c1) : make_uint4(0, 0, 0, 0);
+                    const uint4 y1 = two ? __ldg(y + r * H8 + c1) : make_uint4(0, 0, 0, 0);
+                    float s0[8], s1[8];
+                    dot_and_scale(d0, y0, pj, dot, s0);
+                    dot_and_scale(d1, y1, pj, dot, s1);
+                    dy[r * H8 + c0] = pack8(s0);
+                    if (two) dy[r * H8 + c1] = pack8(s1);
                 }
-                float s[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) s[i] = ps[j] * df[i];
-                dy[rows[j] * H8 + c] = pack8(s);
             }
-        }
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            if (j >= k) break;
-            float v = dot[j];
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
-            if (lane == 0) dprob[t * k + j] = v;
+            for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(kFull, dot, off);
+            if (lane == 0) dprob[t * k + j] = dot;
         }
     }
 }

@@ -45,6 +45,16 @@ DeviceInfo* info() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Stage tracing (moe_trace_set): caller-owned events recorded at stage ends.
+constexpr int kMaxTraceEvents = 16;
+cudaEvent_t g_trace[kMaxTraceEvents];
+int g_trace_n = 0;
+
+cudaError_t trace_mark(int i, cudaStream_t st) {
+    if (i >= g_trace_n) return cudaSuccess;
+    return cudaEventRecord(g_trace[i], st);
+}
+
 // Bump allocator over the caller's workspace; every piece is 256-byte aligned.
 struct Carver {
     char* base;
@@ -176,6 +186,15 @@ moe_status moe_get_device_status(void* stream) {
     }
     if (v & kErrTimeout) return MOE_ERR_TIMEOUT;
     if (v & kErrDeviceCheck) return MOE_ERR_DEVICE_CHECK;
+    return MOE_OK;
+}
+
+moe_status moe_trace_set(void* const* events, int n_events) {
+    if (n_events < 0) return MOE_ERR_INVALID_ARG;
+    if (!events) n_events = 0;
+    if (n_events > kMaxTraceEvents) n_events = kMaxTraceEvents;
+    for (int i = 0; i < n_events; ++i) g_trace[i] = static_cast<cudaEvent_t>(events[i]);
+    g_trace_n = n_events;
     return MOE_OK;
 }
 
@@ -342,19 +361,25 @@ moe_status moe_layer_forward(const float* logits, const moe_bf16* x, int64_t T, 
     const int64_t A = T * k;
     const bf16* xb = reinterpret_cast<const bf16*>(x);
 
-    cudaError_t e = launch_router_topk(logits, T, E, k, opts, L.topk_idx, L.topk_prob, nullptr,
-                                       L.rs, st, err);
+    cudaError_t e = trace_mark(0, st);
+    if (e == cudaSuccess)
+        e = launch_router_topk(logits, T, E, k, opts, L.topk_idx, L.topk_prob, nullptr, L.rs, st,
+                               err);
     if (e == cudaSuccess) e = launch_expert_scan(T, E, L.rs, L.counts, L.offsets, st);
+    if (e == cudaSuccess) e = trace_mark(1, st);
     if (e == cudaSuccess)
         e = launch_permute(xb, T, H, L.topk_idx, k, L.offsets, E, L.rs, L.x_perm, L.sorted_token,
                            L.row_of, st, err);
+    if (e == cudaSuccess) e = trace_mark(2, st);
     if (e == cudaSuccess)
         e = gemm_gate_up_swiglu(L.x_perm, A, L.offsets, E, H, I,
                                 reinterpret_cast<const bf16*>(w_gate_up), L.h,
                                 reinterpret_cast<bf16*>(gu), st, err);
+    if (e == cudaSuccess) e = trace_mark(3, st);
     if (e == cudaSuccess)
         e = gemm_down(L.h, A, L.offsets, E, H, I, reinterpret_cast<const bf16*>(w_down), L.y_perm,
                       st, err);
+    if (e == cudaSuccess) e = trace_mark(4, st);
     if (e == cudaSuccess && has_shared) {
         e = gemm_gate_up_swiglu(xb, T, nullptr, 1, H, I,
                                 reinterpret_cast<const bf16*>(shared_gate_up), L.shared_h, nullptr,
@@ -363,9 +388,11 @@ moe_status moe_layer_forward(const float* logits, const moe_bf16* x, int64_t T, 
             e = gemm_down(L.shared_h, T, nullptr, 1, H, I,
                           reinterpret_cast<const bf16*>(shared_down), L.shared_out, st, err);
     }
+    if (e == cudaSuccess) e = trace_mark(5, st);
     if (e == cudaSuccess)
         e = launch_combine(L.y_perm, L.row_of, L.topk_prob, T, k, H, A, L.shared_out,
                            reinterpret_cast<bf16*>(out), st, err);
+    if (e == cudaSuccess) e = trace_mark(6, st);
     return from_cuda(e);
 }
 
@@ -396,23 +423,30 @@ moe_status moe_grouped_mlp_backward(const moe_bf16* dout, int64_t T, int H, int 
     const BwdLayout L = bwd_layout(workspace, T, H, I, k);
     const int64_t A = T * k;
     auto B = [](const moe_bf16* p) { return reinterpret_cast<const bf16*>(p); };
-    cudaError_t e = cudaSuccess;
+    cudaError_t e = trace_mark(0, st);
     if (T > 0) {
-        e = launch_combine_backward(B(dout), B(y_perm), row_of, topk_prob, T, k, H, A, L.dy, dprob,
-                                    st, err);
+        if (e == cudaSuccess)
+            e = launch_combine_backward(B(dout), B(y_perm), row_of, topk_prob, T, k, H, A, L.dy,
+                                        dprob, st, err);
+        if (e == cudaSuccess) e = trace_mark(1, st);
         if (e == cudaSuccess)
             e = gemm_down_dgrad_swiglu(L.dy, A, offsets, E, H, I, B(w_down), B(gu), L.dgu, st, err);
+        if (e == cudaSuccess) e = trace_mark(2, st);
         if (e == cudaSuccess)
             e = gemm_gate_up_dgrad(L.dgu, A, offsets, E, H, I, B(w_gate_up), L.dx_perm, st, err);
+        if (e == cudaSuccess) e = trace_mark(3, st);
         if (e == cudaSuccess)
             e = launch_combine(L.dx_perm, row_of, nullptr, T, k, H, A, nullptr,
                                reinterpret_cast<bf16*>(dx), st, err);
+        if (e == cudaSuccess) e = trace_mark(4, st);
     }
     if (e == cudaSuccess)
         e = gemm_wgrad(B(h), L.dy, A, offsets, E, I, H, reinterpret_cast<bf16*>(dw_down), st, err);
+    if (e == cudaSuccess) e = trace_mark(5, st);
     if (e == cudaSuccess)
         e = gemm_wgrad(B(x_perm), L.dgu, A, offsets, E, H, 2 * I,
                        reinterpret_cast<bf16*>(dw_gate_up), st, err);
+    if (e == cudaSuccess) e = trace_mark(6, st);
     return from_cuda(e);
 }
 

@@ -12,12 +12,22 @@ namespace moe {
 
 using bf16 = __nv_bfloat16;
 
-// Tokens handled by one block of the router / rank kernels. Ranks inside an
-// expert block are counted per such token block, then offset by a scan.
-constexpr int kTokensPerRouteBlock = 64;
+// Tokens handled by one block of the router / rank kernels (a power of two,
+// 8..64). Ranks inside an expert block are counted per such token block, then
+// offset by a scan. Small batches use small token blocks so that every SM gets
+// work; large ones use 64 to keep the per-block counts ([E][blocks]) small.
+constexpr int kMaxTokensPerRouteBlock = 64;
+
+inline int route_tokens_per_block(int64_t T) {
+    if (T <= 8192) return 8;
+    if (T <= 32768) return 16;
+    if (T <= 131072) return 32;
+    return 64;
+}
 
 inline int64_t route_blocks(int64_t T) {
-    return (T + kTokensPerRouteBlock - 1) / kTokensPerRouteBlock;
+    const int tpb = route_tokens_per_block(T);
+    return (T + tpb - 1) / tpb;
 }
 
 // Scratch of the routing path, carved from the caller's workspace.
@@ -52,9 +62,6 @@ cudaError_t launch_combine_backward(const bf16* dout, const bf16* y_perm, const 
 // ---------------------------------------------------------------- GEMMs
 // Grouped GEMMs on tcgen05. Each returns cudaErrorInvalidValue if a tensor
 // map cannot be encoded (bad alignment or extent).
-struct GemmStatus {
-    cudaError_t err;
-};
 // gate_up + SwiGLU: h[r] = silu(x[r] Wg[e]) * (x[r] Wu[e]); optionally gu[r] = [g | u].
 // offsets NULL: one group of `rows` rows using the weights of group 0.
 cudaError_t gemm_gate_up_swiglu(const bf16* x, int64_t rows, const int32_t* offsets, int E, int H,

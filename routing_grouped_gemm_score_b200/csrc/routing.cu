@@ -13,7 +13,7 @@
 // the same and no rounding of the score function can create a tie. Ranks
 // inside each expert are counted per block of 64 tokens in shared memory, in
 // token order, and an exclusive scan over the token blocks turns them into
-// global rows. Positions never come from atomics, so the permutation is the
+// global rows. A block holds 8 to 64 tokens (route_tokens_per_block). Positions never come from atomics, so the permutation is the
 // same on every run.
 #include "moe_common.cuh"
 #include "moe_internal.h"
@@ -22,7 +22,7 @@ namespace moe {
 
 namespace {
 
-constexpr int kRouteThreads = 256;  // 8 warps, 8 tokens each per block
+constexpr int kRouteThreads = 256;  // 8 warps; a token block has 8..64 tokens
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
 // Order-preserving map of a float to uint32: a larger float gives a larger
@@ -57,17 +57,18 @@ struct RouterArgs {
     int32_t* local_rank;  // [T][k]
     unsigned* ticket;
     int nb;
+    int tpb;   // tokens per block
 };
 
 // After the token loop: thread e counts, in token order, the assignments of
 // the block's tokens to expert e. sel[tt][e] holds j+1 if token tt chose e as
 // its j-th expert, else 0.
-__device__ __forceinline__ void rank_block(const uint8_t (*sel)[256], int64_t t0, int64_t T,
+__device__ __forceinline__ void rank_block(const uint8_t (*sel)[256], int64_t t0, int tpb,
                                            int E, int k, int32_t* local_rank,
                                            int32_t* block_base, int nb) {
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
         int cnt = 0;
-        for (int tt = 0; tt < kTokensPerRouteBlock; ++tt) {
+        for (int tt = 0; tt < tpb; ++tt) {
             int v = sel[tt][e];
             if (v) {
                 local_rank[(t0 + tt) * k + (v - 1)] = cnt;
@@ -80,16 +81,16 @@ __device__ __forceinline__ void rank_block(const uint8_t (*sel)[256], int64_t t0
 
 template <int SLOTS>
 __global__ void __launch_bounds__(kRouteThreads) router_topk_kernel(const RouterArgs a) {
-    __shared__ uint8_t sel[kTokensPerRouteBlock][256];
+    __shared__ uint8_t sel[kMaxTokensPerRouteBlock][256];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int E = a.E, k = a.k;
-    for (int i = threadIdx.x; i < kTokensPerRouteBlock * 256 / 16; i += blockDim.x)
+    const int E = a.E, k = a.k, tpb = a.tpb;
+    for (int i = threadIdx.x; i < tpb * 256 / 16; i += blockDim.x)
         reinterpret_cast<uint4*>(&sel[0][0])[i] = make_uint4(0, 0, 0, 0);
     if (blockIdx.x == 0 && threadIdx.x == 0) *a.ticket = 0u;
     __syncthreads();
-    const int64_t t0 = (int64_t)blockIdx.x * kTokensPerRouteBlock;
+    const int64_t t0 = (int64_t)blockIdx.x * tpb;
 
-    for (int tt = warp; tt < kTokensPerRouteBlock; tt += kRouteThreads / 32) {
+    for (int tt = warp; tt < tpb; tt += kRouteThreads / 32) {
         const int64_t t = t0 + tt;
         if (t >= a.T) break;
         const float* lrow = a.logits + t * E;
@@ -189,21 +190,21 @@ __global__ void __launch_bounds__(kRouteThreads) router_topk_kernel(const Router
         }
     }
     __syncthreads();
-    rank_block(sel, t0, a.T, E, k, a.local_rank, a.block_base, a.nb);
+    rank_block(sel, t0, tpb, E, k, a.local_rank, a.block_base, a.nb);
 }
 
 // Rank pass for caller-supplied expert indices (moe_permute on its own).
 __global__ void __launch_bounds__(kRouteThreads)
     rank_from_indices_kernel(const int32_t* __restrict__ topk_idx, int64_t T, int E, int k,
                              int32_t* local_rank, int32_t* block_base, unsigned* ticket, int nb,
-                             unsigned* err) {
-    __shared__ uint8_t sel[kTokensPerRouteBlock][256];
-    for (int i = threadIdx.x; i < kTokensPerRouteBlock * 256 / 16; i += blockDim.x)
+                             int tpb, unsigned* err) {
+    __shared__ uint8_t sel[kMaxTokensPerRouteBlock][256];
+    for (int i = threadIdx.x; i < tpb * 256 / 16; i += blockDim.x)
         reinterpret_cast<uint4*>(&sel[0][0])[i] = make_uint4(0, 0, 0, 0);
     if (blockIdx.x == 0 && threadIdx.x == 0) *ticket = 0u;
     __syncthreads();
-    const int64_t t0 = (int64_t)blockIdx.x * kTokensPerRouteBlock;
-    for (int tt = threadIdx.x; tt < kTokensPerRouteBlock; tt += blockDim.x) {
+    const int64_t t0 = (int64_t)blockIdx.x * tpb;
+    for (int tt = threadIdx.x; tt < tpb; tt += blockDim.x) {
         const int64_t t = t0 + tt;
         if (t >= T) break;
         for (int j = 0; j < k; ++j) {
@@ -217,7 +218,7 @@ __global__ void __launch_bounds__(kRouteThreads)
         }
     }
     __syncthreads();
-    rank_block(sel, t0, T, E, k, local_rank, block_base, nb);
+    rank_block(sel, t0, tpb, E, k, local_rank, block_base, nb);
 }
 
 // Inclusive scan over the block (blockDim.x a multiple of 32, <= 1024).
@@ -291,7 +292,7 @@ __global__ void __launch_bounds__(1024)
 __global__ void __launch_bounds__(256)
     permute_kernel(const uint4* __restrict__ x, int64_t T, int H8, const int32_t* __restrict__ topk_idx,
                    int k, const int32_t* __restrict__ offsets, int E,
-                   const int32_t* __restrict__ block_base, int nb,
+                   const int32_t* __restrict__ block_base, int nb, int tpb,
                    const int32_t* __restrict__ local_rank, uint4* __restrict__ x_perm,
                    int32_t* __restrict__ sorted_token, int32_t* __restrict__ row_of, int64_t A,
                    unsigned* err) {
@@ -305,7 +306,7 @@ __global__ void __launch_bounds__(256)
             const int rank = local_rank[t * k + lane];
             if (e >= 0 && e < E && rank >= 0) {
                 const int64_t r = (int64_t)offsets[e] +
-                                  block_base[(int64_t)e * nb + t / kTokensPerRouteBlock] + rank;
+                                  block_base[(int64_t)e * nb + t / tpb] + rank;
                 if (r >= offsets[e] && r < offsets[e + 1] && r < A) row = r;
             }
             if (row < 0) raise_error(err, kErrDeviceCheck);
@@ -380,6 +381,7 @@ cudaError_t launch_router_topk(const float* logits, int64_t T, int E, int k,
     a.local_rank = rs.local_rank;
     a.ticket = rs.ticket;
     a.nb = (int)route_blocks(T);
+    a.tpb = route_tokens_per_block(T);
     const dim3 grid((unsigned)a.nb), block(kRouteThreads);
     if (E <= 32) router_topk_kernel<1><<<grid, block, 0, st>>>(a);
     else if (E <= 64) router_topk_kernel<2><<<grid, block, 0, st>>>(a);
@@ -393,7 +395,8 @@ cudaError_t launch_rank_from_indices(const int32_t* topk_idx, int64_t T, int E, 
                                      const RouteScratch& rs, cudaStream_t st, unsigned* err) {
     const int nb = (int)route_blocks(T);
     rank_from_indices_kernel<<<nb, kRouteThreads, 0, st>>>(topk_idx, T, E, k, rs.local_rank,
-                                                          rs.block_base, rs.ticket, nb, err);
+                                                          rs.block_base, rs.ticket, nb,
+                                                          route_tokens_per_block(T), err);
     return cudaGetLastError();
 }
 
@@ -416,7 +419,8 @@ cudaError_t launch_permute(const bf16* x, int64_t T, int H, const int32_t* topk_
     if (blocks > cap) blocks = cap;
     permute_kernel<<<(unsigned)blocks, 256, 0, st>>>(
         reinterpret_cast<const uint4*>(x), T, H / 8, topk_idx, k, offsets, E, rs.block_base, nb,
-        rs.local_rank, reinterpret_cast<uint4*>(x_perm), sorted_token, row_of, T * k, err);
+        route_tokens_per_block(T), rs.local_rank, reinterpret_cast<uint4*>(x_perm), sorted_token,
+        row_of, T * k, err);
     return cudaGetLastError();
 }
 
