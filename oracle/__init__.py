@@ -50,6 +50,8 @@ def _load():
             i64, i32, f32 = ctypes.c_int64, ctypes.c_int, ctypes.c_float
             lib.oracle_round_bf16.argtypes = [ctypes.c_double]
             lib.oracle_round_bf16.restype = ctypes.c_uint16
+            lib.oracle_round_bf16_array.argtypes = [P, i64, P]
+            lib.oracle_round_bf16_array.restype = None
             lib.oracle_router_topk.argtypes = [P, i64, i32, i32, i32, i32, f32, P, P, P, P, P, P]
             lib.oracle_router_topk.restype = i32
             lib.oracle_dispatch.argtypes = [P, i64, i32, i32, P, P, P]
@@ -93,6 +95,14 @@ def bits_to_float(b: np.ndarray) -> np.ndarray:
 
 def round_bf16(v: float) -> int:
     return int(_load().oracle_round_bf16(float(v)))
+
+
+def round_bf16_array(v) -> np.ndarray:
+    """float64 array -> uint16 bf16 bit patterns (nearest, ties to even)."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    out = np.zeros(v.shape, np.uint16)
+    _load().oracle_round_bf16_array(_p(v), v.size, _p(out))
+    return out
 
 
 def router_topk(logits, k, score=0, renormalize=True, scaling=1.0, expert_bias=None,

@@ -76,6 +76,11 @@ static uint16_t double_to_bf16(double d)
 
 uint16_t oracle_round_bf16(double d) { return double_to_bf16(d); }
 
+void oracle_round_bf16_array(const double* v, int64_t n, uint16_t* out)
+{
+    for (int64_t i = 0; i < n; i++) out[i] = double_to_bf16(v[i]);
+}
+
 /* ------------------------------------------------------------- router --- */
 
 /* Selection key order: larger score first; among equal scores the lower
@@ -384,7 +389,8 @@ int oracle_moe_forward_tokens(const uint16_t* x, const float* logits, int H, int
  * All in fp64. With round_bf16, every tensor that a bf16 pipeline stores
  * between its stages is rounded to bf16, as in the forward: the saved FC1
  * outputs g and u that the SwiGLU backward reads; the gradient dy of the
- * bf16 expert output; the gradients dg, du of the bf16 FC1 output; and the
+ * bf16 expert output (p * dout taken in fp32, the kernel's precision, since
+ * the pages fix none for it); the gradients dg, du of the bf16 FC1 output; and the
  * gradient dxp of each bf16 permuted token row, which the unpermute then sums.
  * The rounding functions themselves pass gradients through unchanged.
  * With round_bf16 = 0, nothing is rounded, and the result is the exact
@@ -439,8 +445,16 @@ int oracle_moe_backward(const uint16_t* x, int64_t T, int H, int I, int E, int k
                     u[i] = bf16_to_double(double_to_bf16(u[i]));
                 }
             for (int c = 0; c < H; c++) {
-                dy[c] = p * bf16_to_double(dot[c]);
-                if (round_bf16) dy[c] = bf16_to_double(double_to_bf16(dy[c]));
+                if (round_bf16) {
+                    /* the stored dy is a bf16 rounding of p * dout; the pages fix
+                     * no precision for this product, so it is taken in the
+                     * kernel's (fp32), as a rounding decision must be */
+                    const float pf = topk_prob[t * k + j];
+                    const float v = pf * (float)bf16_to_double(dot[c]);
+                    dy[c] = bf16_to_double(double_to_bf16((double)v));
+                } else {
+                    dy[c] = p * bf16_to_double(dot[c]);
+                }
             }
             if (dw_down) {
                 double* dwd = dw_down + (only_expert >= 0 ? 0 : (int64_t)e * I * H);

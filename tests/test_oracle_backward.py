@@ -111,6 +111,21 @@ class _RoundGrad(torch.autograd.Function):
         return g.float().to(torch.bfloat16).double()
 
 
+class _WeightedGrad(torch.autograd.Function):
+    """Forward: p * y. Backward: dy = bf16(fp32(p) * fp32(dout)) and
+    dp = <dout, y>, as a bf16 pipeline stores the expert-output gradient."""
+    @staticmethod
+    def forward(ctx, y, p):
+        ctx.save_for_backward(y, p)
+        return p * y
+
+    @staticmethod
+    def backward(ctx, g):
+        y, p = ctx.saved_tensors
+        dy = (p.float() * g.float()).to(torch.bfloat16).double()
+        return dy, (g * y).sum()
+
+
 def _round_both(v):
     return _RoundGrad.apply(_RoundValue.apply(v))
 
@@ -141,10 +156,13 @@ def test_backward_matches_torch_autograd(oracle_lib, round_bf16):
                 # value from the unrounded g, u; gradient through the stored g, u
                 h = F.silu(gb) * ub + (F.silu(g) * u - F.silu(gb) * ub).detach()
                 h = _RoundValue.apply(h)
-                y = _round_both(h @ wd[e])
+                y = _RoundValue.apply(h @ wd[e])
+                # the stored gradient of y is bf16(p * dout) with the product in fp32
+                y = _WeightedGrad.apply(y, prob[t, j])
+                out[t] = out[t] + y
             else:
                 y = (F.silu(g) * u) @ wd[e]
-            out[t] = out[t] + prob[t, j] * y
+                out[t] = out[t] + prob[t, j] * y
     (out * d["dout"].double()).sum().backward()
     g = oracle_lib.moe_backward(bits(d["x"]), r["topk_idx"], r["topk_prob"], bits(d["w_gate_up"]),
                                 bits(d["w_down"]), bits(d["dout"]), round_bf16=round_bf16)
