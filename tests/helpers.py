@@ -148,3 +148,24 @@ def flip_terms(w, d, r, s):
     t_dx = dxp[row_of].sum(axis=1)
     t_dprob = np.abs(dout[:, None, :] * s["y"][row_of]).max(axis=2)
     return dict(dw_down=t_dwd, dw_gate_up=t_dwgu, dx=t_dx, dprob=t_dprob)
+
+
+def forward_terms(w, d, tokens, logits=None):
+    """Largest stored bf16 summand of each output element: out[t] is
+    shared[t] + sum_j p_j y_j with shared and y stored in bf16, so a flip of
+    one stored summand moves the element by at most 2^-7 of it."""
+    import oracle
+    bits_ = oracle.bf16_bits
+    x, wgu, wd = bits_(d["x"]), bits_(d["w_gate_up"]), bits_(d["w_down"])
+    logits = d["logits"].cpu().numpy() if logits is None else logits
+    r = oracle.router_topk(logits[tokens], w.k, w.score, w.renormalize, with_map=False)
+    term = np.zeros((len(tokens), w.H))
+    for n, t in enumerate(tokens):
+        if d.get("shared_gate_up") is not None:
+            s = oracle.expert_mlp(x[t:t + 1], bits_(d["shared_gate_up"][0]), bits_(d["shared_down"][0]))
+            term[n] = np.abs(s[0])
+        for j in range(w.k):
+            e = int(r["topk_idx"][n, j])
+            y = oracle.expert_mlp(x[t:t + 1], wgu[e], wd[e])
+            np.maximum(term[n], abs(float(r["topk_prob"][n, j])) * np.abs(y[0]), out=term[n])
+    return term

@@ -52,7 +52,8 @@ def test_layer_forward_matches_per_token_definition(name):
     w = SMALL[name]
     d = wl.make_inputs(w, "cuda")
     out = layer(w, d)
-    assert_close(out, oracle_out(w, d), f"{name}: out")
+    tokens = np.arange(w.T)
+    helpers.assert_close_flips(out, oracle_out(w, d), helpers.forward_terms(w, d, tokens), f"{name}: out")
 
 
 def test_layer_forward_saved_state_and_empty_batch():
