@@ -124,6 +124,29 @@ moe_status moe_router_topk(const float* logits, int64_t T, int E, int k,
                            uint8_t* routing_map, int32_t* counts, int32_t* offsets,
                            void* workspace, size_t workspace_bytes, void* stream);
 
+/* moe_router_topk_noalloc -- the same routing as moe_router_topk, with no
+ * workspace argument: for callers that cannot allocate device memory when they
+ * route, such as a runtime that hands out all device memory from its own
+ * pool before serving starts, or code running where allocation is forbidden.
+ * The pages have no counterpart to it; it is an interface of this library.
+ * Its scratch is one fixed array inside the library (a little over 3 MiB), which
+ * every GPU that loads the library keeps until the process exits. It is
+ * therefore limited to T <= MOE_NOALLOC_MAX_TOKENS and
+ * T * k <= MOE_NOALLOC_MAX_ASSIGNMENTS; larger sizes return
+ * MOE_ERR_UNSUPPORTED before anything is launched. Calls allocate nothing and
+ * share that one array: two calls whose kernels overlap on the GPU (for
+ * example on different streams without ordering) race and may return wrong
+ * results. Calls that are ordered on one stream are safe. The first call on
+ * a device looks up the array's device address once; make that first call
+ * before any stream capture. Arguments, outputs and errors are otherwise those
+ * of moe_router_topk. */
+#define MOE_NOALLOC_MAX_TOKENS 32768
+#define MOE_NOALLOC_MAX_ASSIGNMENTS 262144
+moe_status moe_router_topk_noalloc(const float* logits, int64_t T, int E, int k,
+                                   const moe_router_opts* opts, int32_t* topk_idx,
+                                   float* topk_prob, uint8_t* routing_map, int32_t* counts,
+                                   int32_t* offsets, void* stream);
+
 /* ----------------------------------------------------------------- dispatch
  * moe_permute -- TE Token dispatch: the rows of all tokens routed to the same
  * expert are stored back to back, in expert order. Inside an expert block,

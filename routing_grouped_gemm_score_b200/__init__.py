@@ -25,7 +25,7 @@ __all__ = [
     "MoEError", "RouterOpts", "SCORE_SOFTMAX", "SCORE_SIGMOID", "library_path", "lib",
     "moe_status_string", "moe_get_device_status", "moe_router_topk", "moe_permute",
     "moe_grouped_mlp", "moe_unpermute_combine", "moe_layer_forward", "moe_grouped_mlp_backward",
-    "moe_trace_set", "LayerWorkspace", "ABI_FUNCTIONS",
+    "moe_trace_set", "moe_router_topk_noalloc", "LayerWorkspace", "ABI_FUNCTIONS",
 ]
 
 SCORE_SOFTMAX = 0
@@ -76,6 +76,8 @@ ABI_FUNCTIONS = {
     "moe_trace_set": (I32, [ctypes.POINTER(ctypes.c_void_p), I32]),
     "moe_router_workspace_size": (SZ, [I64, I32, I32]),
     "moe_router_topk": (I32, [P, I64, I32, I32, ctypes.POINTER(_RouterOptsC), P, P, P, P, P, P, SZ, P]),
+    "moe_router_topk_noalloc": (I32, [P, I64, I32, I32, ctypes.POINTER(_RouterOptsC), P, P, P, P,
+                                       P, P]),
     "moe_permute_workspace_size": (SZ, [I64, I32, I32]),
     "moe_permute": (I32, [P, I64, I32, P, I32, P, I32, P, P, P, P, SZ, P]),
     "moe_grouped_mlp_workspace_size": (SZ, [I64, I32, I32, I32]),
@@ -184,6 +186,33 @@ def moe_router_topk(logits: torch.Tensor, k: int, opts: Optional[RouterOpts] = N
                                  _ptr(out["topk_prob"]), _ptr(out["routing_map"]), _ptr(out["counts"]),
                                  _ptr(out["offsets"]), _ptr(ws), ws.numel(), _stream()),
            "moe_router_topk")
+    return out
+
+
+def moe_router_topk_noalloc(logits: torch.Tensor, k: int, opts: Optional[RouterOpts] = None,
+                            routing_map: bool = False, out: Optional[dict] = None) -> dict:
+    """moe_router_topk through the entry point that takes no workspace. It is
+    for callers that cannot allocate device memory while routing. Pass `out`
+    with preallocated topk_idx, topk_prob, counts, offsets (and routing_map)
+    tensors to allocate nothing at all; the library's fixed scratch limits T
+    to 32768 and T * k to 262144."""
+    _need(logits, torch.float32, "logits")
+    T, E = logits.shape
+    dev = logits.device
+    if out is None:
+        out = {
+            "topk_idx": torch.empty((T, k), dtype=torch.int32, device=dev),
+            "topk_prob": torch.empty((T, k), dtype=torch.float32, device=dev),
+            "routing_map": torch.empty((T, E), dtype=torch.uint8, device=dev) if routing_map else None,
+            "counts": torch.empty(E, dtype=torch.int32, device=dev),
+            "offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+        }
+    oc = (opts or RouterOpts()).c()
+    _check(lib().moe_router_topk_noalloc(_ptr(logits), T, E, k, ctypes.byref(oc),
+                                         _ptr(out["topk_idx"]), _ptr(out["topk_prob"]),
+                                         _ptr(out.get("routing_map")), _ptr(out["counts"]),
+                                         _ptr(out["offsets"]), _stream()),
+           "moe_router_topk_noalloc")
     return out
 
 

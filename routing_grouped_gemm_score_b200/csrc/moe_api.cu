@@ -230,6 +230,40 @@ moe_status moe_router_topk(const float* logits, int64_t T, int E, int k,
     return from_cuda(e);
 }
 
+moe_status moe_router_topk_noalloc(const float* logits, int64_t T, int E, int k,
+                                   const moe_router_opts* opts_in, int32_t* topk_idx,
+                                   float* topk_prob, uint8_t* routing_map, int32_t* counts,
+                                   int32_t* offsets, void* stream) {
+    if (!shape_ok(T, E, k)) return MOE_ERR_INVALID_ARG;
+    const moe_router_opts opts = opts_in ? *opts_in : default_opts();
+    if (check_opts(opts) != MOE_OK) return MOE_ERR_INVALID_ARG;
+    if (!counts || !offsets || !aligned16(counts) || !aligned16(offsets)) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!logits || !topk_idx || !topk_prob || !aligned16(logits) ||
+                  !aligned16(topk_idx) || !aligned16(topk_prob)))
+        return MOE_ERR_INVALID_ARG;
+    if (opts.expert_bias && !aligned16(opts.expert_bias)) return MOE_ERR_INVALID_ARG;
+    if (T > MOE_NOALLOC_MAX_TOKENS || T * (int64_t)k > MOE_NOALLOC_MAX_ASSIGNMENTS ||
+        route_scratch_bytes(T, E, k) > router_noalloc_capacity())
+        return MOE_ERR_UNSUPPORTED;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, st) != cudaSuccess) return MOE_ERR_CUDA;
+        return from_cuda(cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (E + 1), st));
+    }
+    void* scratch = nullptr;
+    if (router_noalloc_scratch(&scratch) != cudaSuccess || !scratch) return MOE_ERR_CUDA;
+    unsigned* err = device_error_word();
+    if (!err) return MOE_ERR_CUDA;
+    // The router kernel resets the scan's ticket counter itself, and every
+    // other scratch word is written before it is read, so the previous call's
+    // contents need no clearing.
+    const RouteScratch rs = carve_route_scratch(scratch, T, E, k);
+    cudaError_t e = launch_router_topk(logits, T, E, k, opts, topk_idx, topk_prob, routing_map, rs,
+                                       st, err);
+    if (e == cudaSuccess) e = launch_expert_scan(T, E, rs, counts, offsets, st);
+    return from_cuda(e);
+}
+
 size_t moe_permute_workspace_size(int64_t T, int E, int k) {
     if (!shape_ok(T, E, k)) return 0;
     return route_scratch_bytes(T, E, k);

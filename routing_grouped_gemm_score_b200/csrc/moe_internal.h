@@ -52,6 +52,10 @@ cudaError_t launch_permute(const bf16* x, int64_t T, int H, const int32_t* topk_
                            const int32_t* offsets, int E, const RouteScratch& rs, bf16* x_perm,
                            int32_t* sorted_token, int32_t* row_of, cudaStream_t st, unsigned* err);
 
+// The fixed scratch array behind moe_router_topk_noalloc (routing.cu).
+size_t router_noalloc_capacity();
+cudaError_t router_noalloc_scratch(void** ptr);
+
 cudaError_t launch_combine(const bf16* y_perm, const int32_t* row_of, const float* probs,
                            int64_t T, int k, int H, int64_t A, const bf16* shared, bf16* out,
                            cudaStream_t st, unsigned* err);

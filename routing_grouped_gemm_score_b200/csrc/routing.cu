@@ -15,6 +15,8 @@
 // token order, and an exclusive scan over the token blocks turns them into
 // global rows. A block holds 8 to 64 tokens (route_tokens_per_block). Positions never come from atomics, so the permutation is the
 // same on every run.
+#include <mutex>
+
 #include "moe_common.cuh"
 #include "moe_internal.h"
 
@@ -337,6 +339,11 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// Scratch for moe_router_topk_noalloc: a fixed array in device memory, so the
+// call allocates nothing. Its size bounds the routing sizes that call accepts.
+constexpr size_t kNoAllocScratchBytes = (3u << 20) + 4096;
+static __device__ __align__(256) unsigned char g_router_noalloc_scratch[kNoAllocScratchBytes];
+
 }  // namespace
 
 size_t route_scratch_bytes(int64_t T, int E, int k) {
@@ -422,6 +429,29 @@ cudaError_t launch_permute(const bf16* x, int64_t T, int H, const int32_t* topk_
         route_tokens_per_block(T), rs.local_rank, reinterpret_cast<uint4*>(x_perm), sorted_token,
         row_of, T * k, err);
     return cudaGetLastError();
+}
+
+// Device address of g_router_noalloc_scratch on the current device. In host
+// code the array's name is only a host-side stand-in, so the address is taken
+// with cudaGetSymbolAddress, once per device, while that device is current.
+size_t router_noalloc_capacity() { return kNoAllocScratchBytes; }
+
+cudaError_t router_noalloc_scratch(void** ptr) {
+    constexpr int kMaxDev = 64;
+    static std::once_flag once[kMaxDev];
+    static void* addr[kMaxDev];
+    static cudaError_t status[kMaxDev];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+    std::call_once(once[dev], [dev] {
+        void* p = nullptr;
+        status[dev] = cudaGetSymbolAddress(&p, g_router_noalloc_scratch);
+        addr[dev] = (status[dev] == cudaSuccess) ? p : nullptr;
+    });
+    *ptr = addr[dev];
+    return status[dev];
 }
 
 }  // namespace moe
