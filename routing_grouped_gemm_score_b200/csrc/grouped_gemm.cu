@@ -1,4 +1,4 @@
-// grouped_gemm.cu -- persistent grouped GEMM on the sm_100a tensor cores
+// grouped_gemm.cu -- persistent grouped GEMMs on the sm_100a tensor cores
 // (tcgen05.mma, accumulators in tensor memory), fed by TMA.
 //
 // Transformer Engine "Mixture of Experts", section Grouped GEMM: for each
@@ -8,36 +8,43 @@
 // reads the intermediate from memory. The SwiGLU is that of te_mixtral.py
 // (_expert_ffn) and torchtitan GroupedExperts: silu(x Wg) * (x Wu).
 //
-// One CTA per SM runs a static round-robin over output tiles of 128 x 256.
-// Warp roles:
-//   warp 0   one thread issues the TMA loads of the A and B tiles of each
-//            64-deep K slice into a 4-stage shared-memory ring (128-byte
-//            swizzle).
-//   warp 1   allocates 512 TMEM columns (two 128 x 256 fp32 accumulators).
-//            One thread issues tcgen05.mma (M=128, N=256, K=16, bf16 in,
-//            fp32 accumulate) and tcgen05.commit, which frees a smem stage
-//            or publishes a finished accumulator.
-//   warps 2-5 epilogue: tcgen05.ld of the accumulator rows of their TMEM
-//            lane quarter, the fused element-wise work, and 16-byte stores.
-// The two accumulators let the epilogue of one tile overlap the MMAs of the
-// next.
+// Two kernels share the schedule and the epilogues. The forward and dgrad
+// GEMMs run on pair tiles when the average expert block is large (>= 2048 rows,
+// or a single dense group), else on single-CTA 128-row tiles, which round
+// ragged blocks up less (use_pair_tiles).
 //
-// Two schedules:
-//   group-M (forward and dgrad): expert e owns rows [off[e], off[e+1]) of
-//     A and of the output. Its tiles are ceil(rows/128) x n_blocks, in
-//     expert order, then N block, then M block, so the M blocks that share a
-//     weight tile run at about the same time and reuse it from L2. A tile
-//     that crosses into the next expert's rows computes them too, and the
-//     epilogue drops them. Past the end of A, TMA reads zeros. An expert
-//     with no rows has no tiles.
-//   group-K (weight gradients): dW[e] = X_e^T D_e. The reduction runs over
-//     the rows of expert e. In the last K slice, the rows that belong to the
-//     next expert are zeroed in shared memory before the MMA. An expert with
-//     no rows writes a zero tile.
+// gemm_pair_kernel (group-M: forward and dgrad). Clusters of two CTAs on two
+// SMs compute 256 x 256 output tiles with tcgen05.mma.cta_group::2 (M=256,
+// N=256, K=16). Each CTA loads 128 rows of A and 128 columns of B per
+// 64-deep K slice (32 KB) into a 6-stage shared-memory ring, so a weight tile
+// is read once per 256 rows. The leader CTA issues the MMAs. Its commits
+// free both CTAs' stages and publish both CTAs' accumulators
+// (tcgen05.commit ... multicast::cluster). The peer CTA's TMA loads complete
+// on the leader's full barrier. Expert e owns rows [off[e], off[e+1]) of A and
+// of the output. Its tiles are ceil(rows/256) x n_blocks, in expert order,
+// then N block, then M block. A tile that crosses into the next expert's rows
+// computes them too, and the epilogue drops them. Past the end of A, TMA reads
+// zeros. An expert with no rows has no tiles.
+//
+// gemm_1cta_kernel (group-M with small expert blocks, and group-K: weight
+// gradients, dW[e] = X_e^T D_e). One CTA
+// per 128 x 256 tile, a 4-stage ring of 48 KB, tcgen05.mma.cta_group::1. The
+// reduction runs over the rows of expert e. In the last K slice, the rows
+// that belong to the next expert are zeroed in shared memory before the MMA.
+// An expert with no rows writes a zero tile.
+//
+// Warp roles, in both: warp 0 issues TMA loads (one thread); warp 1 owns
+// TMEM (two 128 x 256 fp32 accumulators, 512 columns) and issues the MMAs
+// (one thread); warps 2-5 are the epilogue (tcgen05.ld of their TMEM lane
+// quarter, the fused element-wise work, then 32 x 32 bf16 chunks staged in
+// shared memory and written by TMA stores; a 32-row group that crosses an
+// expert boundary is stored directly with masks instead). The two
+// accumulators let the epilogue of one tile overlap the MMAs of the next.
 // Every wait is bounded (moe_common.cuh). On a timeout the kernel records an
 // error, every role leaves its loop, and TMEM is still freed.
 #include <cudaTypedefs.h>
 
+#include <cstdlib>
 #include <mutex>
 
 #include "moe_common.cuh"
@@ -47,14 +54,18 @@ namespace moe {
 
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BN = 256, BK = 64;
 constexpr int kThreads = 192;
-constexpr int kChunkBytes = 64 * BK * 2;       // one 64-wide swizzle chunk x 64 rows: 8 KB
-constexpr int kStageA = BM * BK * 2;           // 16 KB
-constexpr int kStageB = BN * BK * 2;           // 32 KB
-constexpr int kStageBytes = kStageA + kStageB;  // 48 KB
+constexpr int kChunkBytes = 64 * BK * 2;  // one 64-wide swizzle chunk x 64 rows: 8 KB
 constexpr int kTmemCols = 512;
 constexpr int kMaxGroups = 256;
+
+// single CTA: 128 x 256 tile, 4 stages of 16 + 32 KB
+constexpr int BM1 = 128, STAGES1 = 4;
+constexpr int kStageA1 = BM1 * BK * 2, kStageB1 = BN * BK * 2, kStage1 = kStageA1 + kStageB1;
+// CTA pair: 256 x 256 tile, each CTA 6 stages of 16 + 16 KB
+constexpr int BMP = 256, STAGESP = 6;
+constexpr int kStageAP = 128 * BK * 2, kStageBP = (BN / 2) * BK * 2, kStageP = kStageAP + kStageBP;
 
 enum Epi { kEpiStore = 0, kEpiSwiglu = 1, kEpiSwigluBwd = 2 };
 
@@ -78,8 +89,10 @@ struct Params {
     unsigned* err;
 };
 
+template <int STAGES, int STAGE_BYTES>
 struct __align__(1024) Smem {
-    uint8_t stage[STAGES][kStageBytes];
+    uint8_t stage[STAGES][STAGE_BYTES];
+    uint8_t epi[4][2][2048];   // per epilogue warp: two 32 x 32 bf16 staging buffers
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
     uint64_t acc_full[2];
@@ -91,7 +104,10 @@ struct __align__(1024) Smem {
     int tile_start[kMaxGroups + 1];
     int off[kMaxGroups + 1];
 };
-constexpr size_t kSmemBytes = sizeof(Smem) + 1024;  // + alignment slack
+using Smem1 = Smem<STAGES1, kStage1>;
+using SmemP = Smem<STAGESP, kStageP>;
+constexpr size_t kSmem1Bytes = sizeof(Smem1) + 1024;  // + alignment slack
+constexpr size_t kSmemPBytes = sizeof(SmemP) + 1024;
 
 // Shared-memory matrix descriptor: 128-byte swizzle, sm_100 version bit.
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -99,11 +115,11 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
            ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
-// Instruction descriptor: bf16 A and B, fp32 D, M=128, N=256, majors as given.
-template <bool A_MN, bool B_MN>
+// Instruction descriptor: bf16 A and B, fp32 D, the given M and N and majors.
+template <int M, int N, bool A_MN, bool B_MN>
 __device__ __forceinline__ constexpr uint32_t instr_desc() {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((A_MN ? 1u : 0u) << 15) |
-           ((B_MN ? 1u : 0u) << 16) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+           ((B_MN ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
@@ -115,8 +131,57 @@ struct Tile {
     int num_kb;
 };
 
-template <bool GROUP_K>
-__device__ __forceinline__ Tile decode_tile(const Smem& s, const Params& p, int id) {
+// Expert offsets and the exclusive prefix of tiles per expert, in shared
+// memory. Called by all threads of the CTA; ends with a __syncthreads.
+template <bool GROUP_K, class S>
+__device__ __forceinline__ void build_schedule(S& s, const Params& p, int bm) {
+    const int G = p.groups;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int g = threadIdx.x; g <= G; g += blockDim.x) {
+        int v;
+        if (p.offsets) v = __ldg(p.offsets + g);
+        else v = (g == 0) ? 0 : p.rows;
+        s.off[g] = min(max(v, 0), p.rows);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        int local[8];
+        int sum = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int g = lane * 8 + i;
+            int tiles = 0;
+            if (g < G) {
+                if (GROUP_K) {
+                    tiles = p.m_blocks * p.n_blocks;
+                } else {
+                    const int cnt = max(s.off[g + 1] - s.off[g], 0);
+                    tiles = ((cnt + bm - 1) / bm) * p.n_blocks;
+                }
+            }
+            local[i] = tiles;
+            sum += tiles;
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - sum;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int g = lane * 8 + i;
+            if (g <= G) s.tile_start[g] = run;
+            run += local[i];
+        }
+        if (lane == 31) s.total_tiles = incl;
+    }
+    __syncthreads();
+}
+
+template <bool GROUP_K, class S>
+__device__ __forceinline__ Tile decode_tile(const S& s, const Params& p, int id, int bm) {
     Tile t;
     if (GROUP_K) {
         const int per = p.m_blocks * p.n_blocks;
@@ -136,84 +201,393 @@ __device__ __forceinline__ Tile decode_tile(const Smem& s, const Params& p, int 
         }
         t.g = lo;
         const int cnt = max(s.off[t.g + 1] - s.off[t.g], 0);
-        const int mt = (cnt + BM - 1) / BM;
+        const int mt = (cnt + bm - 1) / bm;
         const int local = id - s.tile_start[t.g];
         t.n_blk = local / mt;
         t.m_blk = local - t.n_blk * mt;
-        t.row0 = s.off[t.g] + t.m_blk * BM;
-        t.rows = min(BM, cnt - t.m_blk * BM);
+        t.row0 = s.off[t.g] + t.m_blk * bm;
+        t.rows = min(bm, cnt - t.m_blk * bm);
         t.num_kb = (p.K + BK - 1) / BK;
     }
     return t;
 }
 
+// One epilogue warp's double-buffered staging area for TMA stores.
+struct Stager {
+    uint8_t* base;    // two 2 KB buffers, 1024-byte aligned
+    uint32_t count;   // TMA stores issued so far by this warp (lane 0)
+};
+
+// Stores 32 values of each lane's row (lane = row of the warp's 32-row group)
+// as bf16, through shared memory and one TMA store of a 32 x 32 box at
+// (x, y[, z]). The buffer layout matches the map's 64-byte swizzle: the
+// 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3). Warp-collective.
+template <int DIMS>
+__device__ __forceinline__ void staged_store(Stager& st, const CUtensorMap* map, const float* v,
+                                             int x, int y, int z, int lane) {
+    uint8_t* buf = st.base + (st.count & 1u) * 2048u;
+    if (st.count >= 2 && lane == 0) bulk_wait_group_read<1>();   // this buffer's last store has read it
+    __syncwarp();
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint4 w = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                   pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
+                                   pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+        *reinterpret_cast<uint4*>(buf + lane * 64 + ((q ^ ((lane >> 1) & 3)) * 16)) = w;
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        if (DIMS == 2) tma_store_2d(map, buf, x, y);
+        else tma_store_3d(map, buf, x, y, z);
+        bulk_commit_group();
+    }
+    st.count += 1;
+}
+
+// Masked direct stores of 32 values of this thread's row at `dst`.
+__device__ __forceinline__ void direct_store32(bf16* dst, const float* v) {
+    uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        d[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                          pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+}
+
+// SwiGLU backward for 32 columns: dg, du from dh and the saved bf16 g, u.
+__device__ __forceinline__ void swiglu_bwd32(const float* dh, const bf16* g_src, const bf16* u_src,
+                                             float* dg, float* du) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint4 gv = *reinterpret_cast<const uint4*>(g_src + 8 * q);
+        const uint4 uv = *reinterpret_cast<const uint4*>(u_src + 8 * q);
+        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+        const uint32_t uw[4] = {uv.x, uv.y, uv.z, uv.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 gf = unpack_bf16x2(gw[i]);
+            const float2 uf = unpack_bf16x2(uw[i]);
+            const int c = 8 * q + 2 * i;
+            const float s0 = 1.0f / (1.0f + expf(-gf.x));
+            const float s1 = 1.0f / (1.0f + expf(-gf.y));
+            du[c] = dh[c] * gf.x * s0;
+            du[c + 1] = dh[c + 1] * gf.y * s1;
+            dg[c] = dh[c] * uf.x * (s0 + gf.x * s0 * (1.0f - s0));
+            dg[c + 1] = dh[c + 1] * uf.y * (s1 + gf.y * s1 * (1.0f - s1));
+        }
+    }
+}
+
+// Epilogue of one tile for one epilogue warp. The warp owns rows
+// [warp_r0, warp_r0 + 32) of the tile; its lane `lane` reads TMEM lane row
+// t_row (the thread's accumulator row). For group-M the rows count from the
+// tile's first row; for group-K, from the first output row of the M block.
+// Groups of 32 rows that lie wholly inside the expert's block (always true for
+// group-K, whose 3-D output map clips at M) leave through TMA stores; the
+// others use masked direct stores, so no row of another expert is written.
+template <int EPI, bool GROUP_K>
+__device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, uint32_t t_row,
+                                              int warp_r0, int lane, int n_tile,
+                                              const CUtensorMap* tmO, const CUtensorMap* tmO2,
+                                              Stager& st) {
+    const int r = warp_r0 + lane;
+    if (EPI == kEpiSwiglu) {
+        const int n0 = t.n_blk * (n_tile / 2);
+        const bool valid = r < t.rows;
+        const bool staged = warp_r0 + 32 <= t.rows;
+        const int64_t grow = (int64_t)t.row0 + r;
+        const int yrow = t.row0 + warp_r0;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN / 2; c0 += 32) {
+            float g[32], u[32];
+            tmem_load_2x32(t_row + c0, t_row + BN / 2 + c0, g, u);
+            if (n0 + c0 >= p.N) continue;
+            float h[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) h[i] = silu_f(g[i]) * u[i];
+            if (staged) {
+                staged_store<2>(st, tmO, h, n0 + c0, yrow, 0, lane);
+                if (p.out2) {
+                    staged_store<2>(st, tmO2, g, n0 + c0, yrow, 0, lane);
+                    staged_store<2>(st, tmO2, u, p.I + n0 + c0, yrow, 0, lane);
+                }
+            } else if (valid) {
+                direct_store32(p.out + grow * p.ldo + n0 + c0, h);
+                if (p.out2) {
+                    direct_store32(p.out2 + grow * p.ldo2 + n0 + c0, g);
+                    direct_store32(p.out2 + grow * p.ldo2 + p.I + n0 + c0, u);
+                }
+            }
+        }
+    } else if (EPI == kEpiSwigluBwd) {
+        const int n0 = t.n_blk * n_tile;
+        const bool valid = r < t.rows;
+        const bool staged = warp_r0 + 32 <= t.rows;
+        const int64_t grow = (int64_t)t.row0 + r;
+        const int yrow = t.row0 + warp_r0;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 64) {
+            float dh[64];
+            tmem_load_2x32(t_row + c0, t_row + c0 + 32, *reinterpret_cast<float(*)[32]>(dh),
+                           *reinterpret_cast<float(*)[32]>(dh + 32));
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int col = n0 + c0 + 32 * half;
+                if (col >= p.N) continue;
+                float dg[32], du[32];
+                if (valid)
+                    swiglu_bwd32(dh + 32 * half, p.aux + grow * p.ld_aux + col,
+                                 p.aux + grow * p.ld_aux + p.I + col, dg, du);
+                if (staged) {
+                    staged_store<2>(st, tmO, dg, col, yrow, 0, lane);
+                    staged_store<2>(st, tmO, du, p.I + col, yrow, 0, lane);
+                } else if (valid) {
+                    direct_store32(p.out + grow * p.ldo + col, dg);
+                    direct_store32(p.out + grow * p.ldo + p.I + col, du);
+                }
+            }
+        }
+    } else {
+        const int n0 = t.n_blk * n_tile;
+        bool valid, staged;
+        bf16* orow;
+        int yrow;
+        if (GROUP_K) {
+            const int m0 = t.m_blk * BM1;
+            valid = m0 + r < p.M;
+            staged = true;
+            orow = p.out + (int64_t)t.g * p.out_group_stride + (int64_t)(m0 + r) * p.ldo;
+            yrow = m0 + warp_r0;
+        } else {
+            valid = r < t.rows;
+            staged = warp_r0 + 32 <= t.rows;
+            orow = p.out + ((int64_t)t.row0 + r) * p.ldo;
+            yrow = t.row0 + warp_r0;
+        }
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 64) {
+            float v[64];
+            if (t.num_kb > 0) {
+                tmem_load_2x32(t_row + c0, t_row + c0 + 32, *reinterpret_cast<float(*)[32]>(v),
+                               *reinterpret_cast<float(*)[32]>(v + 32));
+            } else {
+#pragma unroll
+                for (int i = 0; i < 64; ++i) v[i] = 0.0f;
+            }
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int col = n0 + c0 + 32 * half;
+                if (col >= p.N) continue;
+                if (staged) {
+                    if (GROUP_K) staged_store<3>(st, tmO, v + 32 * half, col, yrow, t.g, lane);
+                    else staged_store<2>(st, tmO, v + 32 * half, col, yrow, 0, lane);
+                } else if (valid) {
+                    direct_store32(orow + col, v + 32 * half);
+                }
+            }
+        }
+    }
+}
+
+// ===================================================================== pair
+template <int EPI, bool B_MN>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
+                     const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    SmemP& s = *reinterpret_cast<SmemP*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                         ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();      // 0: leader, 1: peer
+    const int cluster = blockIdx.x >> 1, clusters = gridDim.x >> 1;
+    volatile int* abort_flag = &s.abort;
+
+    build_schedule<false>(s, p, BMP);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGESP; ++i) {
+            mbar_init(&s.full[i], 1);
+            mbar_init(&s.empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s.acc_full[i], 1);
+            mbar_init(&s.acc_empty[i], 8);   // one arrival per epilogue warp of both CTAs
+        }
+        mbar_init(&s.drain, 1);
+        s.abort = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(&s.tmem_base, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync_all();        // barriers of both CTAs initialised, TMEM allocated
+    tc_fence_after();
+    const uint32_t tmem_base = s.tmem_base;
+    const int total = s.total_tiles;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            const uint64_t keep = l2_policy_evict_last();   // A panels are read by every N block
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued[STAGESP] = {0, 0, 0, 0, 0, 0};
+            bool ok = true;
+            for (int id = cluster; id < total && ok; id += clusters) {
+                const Tile t = decode_tile<false>(s, p, id, BMP);
+                for (int kb = 0; kb < t.num_kb; ++kb) {
+                    if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* a_s = s.stage[stage];
+                    uint8_t* b_s = s.stage[stage] + kStageAP;
+                    const uint32_t bar = mapa_shared(smem_u32(&s.full[stage]), 0);
+                    if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], 2 * kStageP);
+                    tma_load_2d_pair_hint(&tmA, bar, a_s, kb * BK, t.row0 + (int)rank * 128, keep);
+                    if (B_MN) {
+#pragma unroll
+                        for (int c = 0; c < 2; ++c) {
+                            int col;
+                            if (EPI == kEpiSwiglu) {
+                                const int n0 = t.n_blk * (BN / 2);
+                                col = (rank == 0 ? n0 : p.I + n0) + 64 * c;
+                            } else {
+                                col = t.n_blk * BN + (int)rank * 128 + 64 * c;
+                            }
+                            tma_load_3d_pair(&tmB, bar, b_s + c * kChunkBytes, col, kb * BK, t.g);
+                        }
+                    } else {
+                        tma_load_3d_pair(&tmB, bar, b_s, kb * BK, t.n_blk * BN + (int)rank * 128,
+                                         t.g);
+                    }
+                    issued[stage] += 1;
+                    if (++stage == STAGESP) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // the leader waits for every load it armed to land before it may exit
+            if (rank == 0)
+                for (int i = 0; i < STAGESP; ++i)
+                    if (issued[i]) mbar_wait(&s.full[i], (issued[i] - 1) & 1u, abort_flag, p.err);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer (leader)
+        if (rank == 0) {
+            constexpr uint32_t idesc = instr_desc<BMP, BN, false, B_MN>();
+            int stage = 0;
+            uint32_t phase = 0;
+            int local_tile = 0;
+            bool ok = true;
+            bool any_mma = false;
+            for (int id = cluster; id < total && ok; id += clusters, ++local_tile) {
+                const Tile t = decode_tile<false>(s, p, id, BMP);
+                const int buf = local_tile & 1;
+                const uint32_t use = (uint32_t)(local_tile >> 1);
+                if (!mbar_wait_cluster(&s.acc_empty[buf], (use & 1u) ^ 1u, abort_flag, p.err)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
+                for (int kb = 0; kb < t.num_kb; ++kb) {
+                    if (!mbar_wait(&s.full[stage], phase, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(s.stage[stage]);
+                    const uint32_t b_addr = a_addr + kStageAP;
+                    if (lane == 0) {
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            const uint64_t adesc = smem_desc(a_addr + kk * 32, 16, 1024);
+                            const uint64_t bdesc = B_MN ? smem_desc(b_addr + kk * 2048, kChunkBytes, 1024)
+                                                        : smem_desc(b_addr + kk * 32, 16, 1024);
+                            umma_bf16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        }
+                        umma_commit_pair_mc(&s.empty[stage], 0x3);
+                        any_mma = true;
+                    }
+                    __syncwarp();
+                    if (++stage == STAGESP) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                if (lane == 0) umma_commit_pair_mc(&s.acc_full[buf], 0x3);
+                __syncwarp();
+            }
+            if (lane == 0 && any_mma) {
+                umma_commit_pair_mc(&s.drain, 0x1);
+                mbar_wait(&s.drain, 0, abort_flag, p.err);
+            }
+            __syncwarp();
+        }
+    } else {
+        // ------------------------------------------------------ epilogue (both CTAs)
+        const int quarter = warp & 3;
+        const int warp_r0 = (int)rank * 128 + quarter * 32;    // first row of the 256-row tile
+        Stager st{s.epi[quarter][0], 0};
+        prefetch_tensormap(&tmO);
+        const uint32_t leader_acc_empty[2] = {mapa_shared(smem_u32(&s.acc_empty[0]), 0),
+                                              mapa_shared(smem_u32(&s.acc_empty[1]), 0)};
+        int local_tile = 0;
+        for (int id = cluster; id < total; id += clusters, ++local_tile) {
+            const Tile t = decode_tile<false>(s, p, id, BMP);
+            const int buf = local_tile & 1;
+            const uint32_t use = (uint32_t)(local_tile >> 1);
+            if (!mbar_wait(&s.acc_full[buf], use & 1u, abort_flag, p.err)) break;
+            tc_fence_after();
+            const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
+            epilogue_tile<EPI, false>(p, t, t_row, warp_r0, lane, BN, &tmO, &tmO2, st);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(leader_acc_empty[buf]);
+        }
+        if (lane == 0) bulk_wait_all();     // the last TMA stores have landed
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    cluster_sync_all();        // no MMA, load or remote arrival of either CTA is still pending
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, kTmemCols);
+    }
+}
+
+// ===================================================================== single CTA
 template <int EPI, bool A_MN, bool B_MN, bool GROUP_K>
 __global__ void __launch_bounds__(kThreads, 1)
-    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                        const __grid_constant__ CUtensorMap tmB, const Params p) {
+    gemm_1cta_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
+                     const Params p) {
     extern __shared__ uint8_t smem_raw[];
-    Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                       ~uintptr_t(1023));
+    Smem1& s = *reinterpret_cast<Smem1*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                         ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int* abort_flag = &s.abort;
 
-    // ---- schedule: expert offsets and the tile prefix, in shared memory
-    const int G = p.groups;
-    for (int g = threadIdx.x; g <= G; g += blockDim.x) {
-        int v;
-        if (p.offsets) v = __ldg(p.offsets + g);
-        else v = (g == 0) ? 0 : p.rows;
-        s.off[g] = min(max(v, 0), p.rows);
-    }
-    __syncthreads();
-    if (warp == 0) {
-        // tile_start = exclusive prefix of tiles per expert; 8 experts per lane
-        int local[8];
-        int sum = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int g = lane * 8 + i;
-            int tiles = 0;
-            if (g < G) {
-                if (GROUP_K) {
-                    tiles = p.m_blocks * p.n_blocks;
-                } else {
-                    const int cnt = max(s.off[g + 1] - s.off[g], 0);
-                    tiles = ((cnt + BM - 1) / BM) * p.n_blocks;
-                }
-            }
-            local[i] = tiles;
-            sum += tiles;
+    build_schedule<GROUP_K>(s, p, BM1);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < STAGES1; ++i) {
+            mbar_init(&s.full[i], 1);
+            mbar_init(&s.empty[i], 1);
         }
-        int incl = sum;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-            if (lane >= off) incl += o;
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s.acc_full[i], 1);
+            mbar_init(&s.acc_empty[i], 128);
         }
-        int run = incl - sum;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int g = lane * 8 + i;
-            if (g <= G) s.tile_start[g] = run;
-            run += local[i];
-        }
-        if (lane == 31) s.total_tiles = incl;
-        if (lane == 0) {
-            for (int i = 0; i < STAGES; ++i) {
-                mbar_init(&s.full[i], 1);
-                mbar_init(&s.empty[i], 1);
-            }
-            for (int i = 0; i < 2; ++i) {
-                mbar_init(&s.acc_full[i], 1);
-                mbar_init(&s.acc_empty[i], 128);
-            }
-            mbar_init(&s.drain, 1);
-            s.abort = 0;
-            fence_mbar_init();
-            prefetch_tensormap(&tmA);
-            prefetch_tensormap(&tmB);
-        }
+        mbar_init(&s.drain, 1);
+        s.abort = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmB);
     }
     if (warp == 1) {
         tmem_alloc(&s.tmem_base, kTmemCols);
@@ -228,31 +602,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
+            const uint64_t keep = l2_policy_evict_last();   // activation panels are read again
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t issued[STAGES] = {0, 0, 0, 0};
+            uint32_t issued[STAGES1] = {0, 0, 0, 0};
             bool ok = true;
             for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
-                const Tile t = decode_tile<GROUP_K>(s, p, id);
+                const Tile t = decode_tile<GROUP_K>(s, p, id, BM1);
                 for (int kb = 0; kb < t.num_kb; ++kb) {
                     if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag, p.err)) {
                         ok = false;
                         break;
                     }
                     uint8_t* a_s = s.stage[stage];
-                    uint8_t* b_s = s.stage[stage] + kStageA;
+                    uint8_t* b_s = s.stage[stage] + kStageA1;
                     uint64_t* bar = &s.full[stage];
-                    mbar_arrive_expect_tx(bar, kStageBytes);
+                    mbar_arrive_expect_tx(bar, kStage1);
                     if (GROUP_K) {
                         const int krow = t.row0 + kb * BK;
-                        const int m0 = t.m_blk * BM, n0 = t.n_blk * BN;
-                        tma_load_2d(&tmA, bar, a_s, m0, krow);
-                        tma_load_2d(&tmA, bar, a_s + kChunkBytes, m0 + 64, krow);
+                        const int m0 = t.m_blk * BM1, n0 = t.n_blk * BN;
+                        tma_load_2d_hint(&tmA, bar, a_s, m0, krow, keep);
+                        tma_load_2d_hint(&tmA, bar, a_s + kChunkBytes, m0 + 64, krow, keep);
 #pragma unroll
                         for (int c = 0; c < 4; ++c)
-                            tma_load_2d(&tmB, bar, b_s + c * kChunkBytes, n0 + 64 * c, krow);
+                            tma_load_2d_hint(&tmB, bar, b_s + c * kChunkBytes, n0 + 64 * c, krow, keep);
                     } else {
-                        tma_load_2d(&tmA, bar, a_s, kb * BK, t.row0);
+                        tma_load_2d_hint(&tmA, bar, a_s, kb * BK, t.row0, keep);
                         if (B_MN) {
 #pragma unroll
                             for (int c = 0; c < 4; ++c) {
@@ -270,26 +645,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     issued[stage] += 1;
-                    if (++stage == STAGES) {
+                    if (++stage == STAGES1) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
             // let every load still in flight land before the CTA may exit
-            for (int i = 0; i < STAGES; ++i)
+            for (int i = 0; i < STAGES1; ++i)
                 if (issued[i]) mbar_wait(&s.full[i], (issued[i] - 1) & 1u, abort_flag, p.err);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
-        constexpr uint32_t idesc = instr_desc<A_MN, B_MN>();
+        constexpr uint32_t idesc = instr_desc<BM1, BN, A_MN, B_MN>();
         int stage = 0;
         uint32_t phase = 0;
         int local_tile = 0;
         bool ok = true;
         bool any_mma = false;
         for (int id = blockIdx.x; id < total && ok; id += gridDim.x, ++local_tile) {
-            const Tile t = decode_tile<GROUP_K>(s, p, id);
+            const Tile t = decode_tile<GROUP_K>(s, p, id, BM1);
             const int buf = local_tile & 1;
             const uint32_t use = (uint32_t)(local_tile >> 1);
             if (!mbar_wait(&s.acc_empty[buf], (use & 1u) ^ 1u, abort_flag, p.err)) break;
@@ -307,7 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after();
                 const uint32_t a_addr = smem_u32(s.stage[stage]);
-                const uint32_t b_addr = a_addr + kStageA;
+                const uint32_t b_addr = a_addr + kStageA1;
                 if (GROUP_K) {
                     const int valid = t.rows - kb * BK;
                     if (valid < BK) {
@@ -316,9 +691,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int i = lane; i < nrows * 6 * 8; i += 32) {
                             const int chunk = i / (nrows * 8);
                             const int rem = i - chunk * nrows * 8;
-                            const int r = valid + rem / 8, q = rem % 8;
+                            const int rr = valid + rem / 8, q = rem % 8;
                             uint4* dst = reinterpret_cast<uint4*>(s.stage[stage] + chunk * kChunkBytes +
-                                                                  r * 128) + q;
+                                                                  rr * 128) + q;
                             *dst = make_uint4(0, 0, 0, 0);
                         }
                         fence_proxy_async_smem();
@@ -340,7 +715,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     any_mma = true;
                 }
                 __syncwarp();
-                if (++stage == STAGES) {
+                if (++stage == STAGES1) {
                     stage = 0;
                     phase ^= 1u;
                 }
@@ -358,127 +733,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------------ epilogue
         const int quarter = warp & 3;               // TMEM lanes 32*quarter .. +31
-        const int r = quarter * 32 + lane;          // row of the tile owned by this thread
+        const int warp_r0 = quarter * 32;           // first tile row of this warp
+        Stager st{s.epi[quarter][0], 0};
+        prefetch_tensormap(&tmO);
         int local_tile = 0;
         for (int id = blockIdx.x; id < total; id += gridDim.x, ++local_tile) {
-            const Tile t = decode_tile<GROUP_K>(s, p, id);
+            const Tile t = decode_tile<GROUP_K>(s, p, id, BM1);
             const int buf = local_tile & 1;
             const uint32_t use = (uint32_t)(local_tile >> 1);
             if (!mbar_wait(&s.acc_full[buf], use & 1u, abort_flag, p.err)) break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-            if (EPI == kEpiSwiglu) {
-                const int n0 = t.n_blk * (BN / 2);
-                const bool valid = r < t.rows;
-                const int64_t grow = (int64_t)t.row0 + r;
-#pragma unroll 1
-                for (int c0 = 0; c0 < BN / 2; c0 += 32) {
-                    float g[32], u[32];
-                    tmem_load_2x32(t_row + c0, t_row + BN / 2 + c0, g, u);
-                    if (valid && n0 + c0 < p.N) {
-                        uint32_t hv[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            hv[i] = pack_bf16x2(silu_f(g[2 * i]) * u[2 * i],
-                                                silu_f(g[2 * i + 1]) * u[2 * i + 1]);
-                        uint4* dst = reinterpret_cast<uint4*>(p.out + grow * p.ldo + n0 + c0);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            if (n0 + c0 + 8 * q < p.N)
-                                dst[q] = make_uint4(hv[4 * q], hv[4 * q + 1], hv[4 * q + 2], hv[4 * q + 3]);
-                        if (p.out2) {
-                            uint4* dg = reinterpret_cast<uint4*>(p.out2 + grow * p.ldo2 + n0 + c0);
-                            uint4* du = reinterpret_cast<uint4*>(p.out2 + grow * p.ldo2 + p.I + n0 + c0);
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                if (n0 + c0 + 8 * q >= p.N) continue;
-                                dg[q] = make_uint4(pack_bf16x2(g[8 * q], g[8 * q + 1]),
-                                                   pack_bf16x2(g[8 * q + 2], g[8 * q + 3]),
-                                                   pack_bf16x2(g[8 * q + 4], g[8 * q + 5]),
-                                                   pack_bf16x2(g[8 * q + 6], g[8 * q + 7]));
-                                du[q] = make_uint4(pack_bf16x2(u[8 * q], u[8 * q + 1]),
-                                                   pack_bf16x2(u[8 * q + 2], u[8 * q + 3]),
-                                                   pack_bf16x2(u[8 * q + 4], u[8 * q + 5]),
-                                                   pack_bf16x2(u[8 * q + 6], u[8 * q + 7]));
-                            }
-                        }
-                    }
-                }
-            } else if (EPI == kEpiSwigluBwd) {
-                const int n0 = t.n_blk * BN;
-                const bool valid = r < t.rows;
-                const int64_t grow = (int64_t)t.row0 + r;
-#pragma unroll 1
-                for (int c0 = 0; c0 < BN; c0 += 64) {
-                    float dh[64];
-                    tmem_load_2x32(t_row + c0, t_row + c0 + 32, *reinterpret_cast<float(*)[32]>(dh),
-                                   *reinterpret_cast<float(*)[32]>(dh + 32));
-                    if (!valid) continue;
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const int col = n0 + c0 + 8 * q;
-                        if (col >= p.N) continue;
-                        const uint4 gv = *reinterpret_cast<const uint4*>(p.aux + grow * p.ld_aux + col);
-                        const uint4 uv = *reinterpret_cast<const uint4*>(p.aux + grow * p.ld_aux + p.I + col);
-                        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-                        const uint32_t uw[4] = {uv.x, uv.y, uv.z, uv.w};
-                        uint32_t dgw[4], duw[4];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const float2 gf = unpack_bf16x2(gw[i]);
-                            const float2 uf = unpack_bf16x2(uw[i]);
-                            const float d0 = dh[8 * q + 2 * i], d1 = dh[8 * q + 2 * i + 1];
-                            const float s0 = 1.0f / (1.0f + expf(-gf.x));
-                            const float s1 = 1.0f / (1.0f + expf(-gf.y));
-                            const float du0 = d0 * gf.x * s0, du1 = d1 * gf.y * s1;
-                            const float dg0 = d0 * uf.x * (s0 + gf.x * s0 * (1.0f - s0));
-                            const float dg1 = d1 * uf.y * (s1 + gf.y * s1 * (1.0f - s1));
-                            dgw[i] = pack_bf16x2(dg0, dg1);
-                            duw[i] = pack_bf16x2(du0, du1);
-                        }
-                        *reinterpret_cast<uint4*>(p.out + grow * p.ldo + col) =
-                            make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]);
-                        *reinterpret_cast<uint4*>(p.out + grow * p.ldo + p.I + col) =
-                            make_uint4(duw[0], duw[1], duw[2], duw[3]);
-                    }
-                }
-            } else {
-                const int n0 = t.n_blk * BN;
-                bool valid;
-                bf16* orow;
-                if (GROUP_K) {
-                    const int m = t.m_blk * BM + r;
-                    valid = m < p.M;
-                    orow = p.out + (int64_t)t.g * p.out_group_stride + (int64_t)m * p.ldo;
-                } else {
-                    valid = r < t.rows;
-                    orow = p.out + ((int64_t)t.row0 + r) * p.ldo;
-                }
-#pragma unroll 1
-                for (int c0 = 0; c0 < BN; c0 += 64) {
-                    float v[64];
-                    if (t.num_kb > 0) {
-                        tmem_load_2x32(t_row + c0, t_row + c0 + 32, *reinterpret_cast<float(*)[32]>(v),
-                                       *reinterpret_cast<float(*)[32]>(v + 32));
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 64; ++i) v[i] = 0.0f;
-                    }
-                    if (!valid) continue;
-                    uint4* dst = reinterpret_cast<uint4*>(orow + n0 + c0);
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        if (n0 + c0 + 8 * q >= p.N) continue;
-                        dst[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]),
-                                            pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                                            pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
-                                            pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
-                    }
-                }
-            }
+            epilogue_tile<EPI, GROUP_K>(p, t, t_row, warp_r0, lane, BN, &tmO, &tmO2, st);
             tc_fence_before();
             mbar_arrive(&s.acc_empty[buf]);
         }
+        if (lane == 0) bulk_wait_all();     // the last TMA stores have landed
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -532,21 +803,76 @@ bool make_map_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int EPI, bool A_MN, bool B_MN, bool GROUP_K>
-cudaError_t launch(const CUtensorMap& a, const CUtensorMap& b, const Params& p, int64_t max_tiles,
-                   cudaStream_t st) {
-    auto kern = grouped_gemm_kernel<EPI, A_MN, B_MN, GROUP_K>;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
+// Output maps: 32 x 32 boxes with the 64-byte swizzle of the staging buffers.
+bool make_store_map_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t pitch) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {pitch * 2};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t es[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_store_map_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+    cuuint32_t box[3] = {32, 32, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <class K>
+cudaError_t set_smem_once(K kern, size_t bytes, std::once_flag& once, cudaError_t& status) {
     std::call_once(once, [&] {
-        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)kSmemBytes);
+        status = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     });
-    if (attr_err != cudaSuccess) return attr_err;
+    return status;
+}
+
+template <int EPI, bool B_MN>
+cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o,
+                        const CUtensorMap& o2, const Params& p, int64_t max_tiles, cudaStream_t st) {
+    auto kern = gemm_pair_kernel<EPI, B_MN>;
+    static std::once_flag once;
+    static cudaError_t attr = cudaSuccess;
+    if (set_smem_once(kern, kSmemPBytes, once, attr) != cudaSuccess) return attr;
+    if (max_tiles <= 0) return cudaSuccess;
+    int64_t clusters = sm_count() / 2;
+    if (clusters > max_tiles) clusters = max_tiles;
+    if (clusters < 1) clusters = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * clusters));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemPBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attrs[1];
+    attrs[0].id = cudaLaunchAttributeClusterDimension;
+    attrs[0].val.clusterDim.x = 2;
+    attrs[0].val.clusterDim.y = 1;
+    attrs[0].val.clusterDim.z = 1;
+    cfg.attrs = attrs;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a, b, o, o2, p);
+}
+
+template <int EPI, bool A_MN, bool B_MN, bool GROUP_K>
+cudaError_t launch_1cta(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o,
+                        const CUtensorMap& o2, const Params& p, int64_t max_tiles, cudaStream_t st) {
+    auto kern = gemm_1cta_kernel<EPI, A_MN, B_MN, GROUP_K>;
+    static std::once_flag once;
+    static cudaError_t attr = cudaSuccess;
+    if (set_smem_once(kern, kSmem1Bytes, once, attr) != cudaSuccess) return attr;
     if (max_tiles <= 0) return cudaSuccess;
     int64_t grid = sm_count();
     if (grid > max_tiles) grid = max_tiles;
-    kern<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(a, b, p);
+    kern<<<(unsigned)grid, kThreads, kSmem1Bytes, st>>>(a, b, o, o2, p);
     return cudaGetLastError();
 }
 
@@ -559,9 +885,39 @@ Params base_params(int groups, int64_t rows, const int32_t* offsets, unsigned* e
     return p;
 }
 
-// Upper bound of group-M tiles without reading the device counts.
-int64_t group_m_tile_bound(int64_t rows, int groups, int n_blocks) {
-    return ((rows + BM - 1) / BM + groups) * (int64_t)n_blocks;
+// Upper bound of group-M pair tiles without reading the device counts.
+int64_t pair_tile_bound(int64_t rows, int groups, int n_blocks) {
+    return ((rows + BMP - 1) / BMP + groups) * (int64_t)n_blocks;
+}
+
+int64_t single_tile_bound(int64_t rows, int groups, int n_blocks) {
+    return ((rows + BM1 - 1) / BM1 + groups) * (int64_t)n_blocks;
+}
+
+// Pair tiles (256 rows) halve each CTA's weight traffic but round every
+// expert block up to 256 rows; single tiles round up to 128. The expected
+// rounding waste is about half a tile per expert, so pair tiles pay off once
+// the average block is large compared with a tile.
+// MOE_GEMM_TILES=pair|single overrides the choice (used by the tests to run
+// both kernels on the same shapes).
+bool use_pair_tiles(int64_t rows, int groups) {
+    const char* force = getenv("MOE_GEMM_TILES");
+    if (force && force[0] == 'p') return true;
+    if (force && force[0] == 's') return false;
+    return groups == 1 || rows >= (int64_t)groups * 2048;
+}
+
+// Group-M GEMM on pair or single tiles. `tb_pair` and `tb_single` are the B
+// maps for each (their K-major boxes differ: 128 or 256 rows of N).
+template <int EPI, bool B_MN>
+cudaError_t launch_group_m(const CUtensorMap& ta, const CUtensorMap& tb_pair,
+                           const CUtensorMap& tb_single, const CUtensorMap& to,
+                           const CUtensorMap& to2, const Params& p, cudaStream_t st) {
+    if (use_pair_tiles(p.rows, p.groups))
+        return launch_pair<EPI, B_MN>(ta, tb_pair, to, to2, p,
+                                      pair_tile_bound(p.rows, p.groups, p.n_blocks), st);
+    return launch_1cta<EPI, false, B_MN, false>(ta, tb_single, to, to2, p,
+                                                single_tile_bound(p.rows, p.groups, p.n_blocks), st);
 }
 
 }  // namespace
@@ -571,7 +927,7 @@ cudaError_t gemm_gate_up_swiglu(const bf16* x, int64_t rows, const int32_t* offs
                                 cudaStream_t st, unsigned* err) {
     if (rows == 0) return cudaSuccess;
     CUtensorMap ta, tb;
-    if (!make_map_2d(&ta, x, H, rows, H, BK, BM)) return cudaErrorInvalidValue;
+    if (!make_map_2d(&ta, x, H, rows, H, BK, 128)) return cudaErrorInvalidValue;
     if (!make_map_3d(&tb, w_gate_up, 2 * (uint64_t)I, H, offsets ? E : 1, 64, BK))
         return cudaErrorInvalidValue;
     const int groups = offsets ? E : 1;
@@ -584,15 +940,22 @@ cudaError_t gemm_gate_up_swiglu(const bf16* x, int64_t rows, const int32_t* offs
     p.ldo = I;
     p.out2 = gu_save;
     p.ldo2 = 2 * (int64_t)I;
-    return launch<kEpiSwiglu, false, true, false>(ta, tb, p,
-                                                  group_m_tile_bound(rows, groups, p.n_blocks), st);
+    CUtensorMap to, to2;
+    if (!make_store_map_2d(&to, h, I, rows, I)) return cudaErrorInvalidValue;
+    if (gu_save) {
+        if (!make_store_map_2d(&to2, gu_save, 2 * (uint64_t)I, rows, 2 * (uint64_t)I))
+            return cudaErrorInvalidValue;
+    } else {
+        to2 = to;
+    }
+    return launch_group_m<kEpiSwiglu, true>(ta, tb, tb, to, to2, p, st);
 }
 
 cudaError_t gemm_down(const bf16* h, int64_t rows, const int32_t* offsets, int E, int H, int I,
                       const bf16* w_down, bf16* y, cudaStream_t st, unsigned* err) {
     if (rows == 0) return cudaSuccess;
     CUtensorMap ta, tb;
-    if (!make_map_2d(&ta, h, I, rows, I, BK, BM)) return cudaErrorInvalidValue;
+    if (!make_map_2d(&ta, h, I, rows, I, BK, 128)) return cudaErrorInvalidValue;
     if (!make_map_3d(&tb, w_down, H, I, offsets ? E : 1, 64, BK)) return cudaErrorInvalidValue;
     const int groups = offsets ? E : 1;
     Params p = base_params(groups, rows, offsets, err);
@@ -601,8 +964,9 @@ cudaError_t gemm_down(const bf16* h, int64_t rows, const int32_t* offsets, int E
     p.n_blocks = (H + BN - 1) / BN;
     p.out = y;
     p.ldo = H;
-    return launch<kEpiStore, false, true, false>(ta, tb, p,
-                                                 group_m_tile_bound(rows, groups, p.n_blocks), st);
+    CUtensorMap to;
+    if (!make_store_map_2d(&to, y, H, rows, H)) return cudaErrorInvalidValue;
+    return launch_group_m<kEpiStore, true>(ta, tb, tb, to, to, p, st);
 }
 
 cudaError_t gemm_down_dgrad_swiglu(const bf16* dy, int64_t rows, const int32_t* offsets, int E,
@@ -610,9 +974,12 @@ cudaError_t gemm_down_dgrad_swiglu(const bf16* dy, int64_t rows, const int32_t* 
                                    cudaStream_t st, unsigned* err) {
     if (rows == 0) return cudaSuccess;
     CUtensorMap ta, tb;
-    if (!make_map_2d(&ta, dy, H, rows, H, BK, BM)) return cudaErrorInvalidValue;
-    // B[n = i][k = h] = w_down[e][i][h]: K-major, box 64 (h) x 256 (i)
-    if (!make_map_3d(&tb, w_down, H, I, E, BK, BN)) return cudaErrorInvalidValue;
+    if (!make_map_2d(&ta, dy, H, rows, H, BK, 128)) return cudaErrorInvalidValue;
+    // B[n = i][k = h] = w_down[e][i][h]: K-major, box 64 (h) x 128 (i) per CTA of a
+    // pair, 64 x 256 for a single CTA
+    CUtensorMap tb1;
+    if (!make_map_3d(&tb, w_down, H, I, E, BK, BN / 2)) return cudaErrorInvalidValue;
+    if (!make_map_3d(&tb1, w_down, H, I, E, BK, BN)) return cudaErrorInvalidValue;
     Params p = base_params(E, rows, offsets, err);
     p.N = I;
     p.K = H;
@@ -622,8 +989,9 @@ cudaError_t gemm_down_dgrad_swiglu(const bf16* dy, int64_t rows, const int32_t* 
     p.ldo = 2 * (int64_t)I;
     p.aux = gu;
     p.ld_aux = 2 * (int64_t)I;
-    return launch<kEpiSwigluBwd, false, false, false>(ta, tb, p,
-                                                      group_m_tile_bound(rows, E, p.n_blocks), st);
+    CUtensorMap to;
+    if (!make_store_map_2d(&to, dgu, 2 * (uint64_t)I, rows, 2 * (uint64_t)I)) return cudaErrorInvalidValue;
+    return launch_group_m<kEpiSwigluBwd, false>(ta, tb, tb1, to, to, p, st);
 }
 
 cudaError_t gemm_gate_up_dgrad(const bf16* dgu, int64_t rows, const int32_t* offsets, int E, int H,
@@ -631,18 +999,22 @@ cudaError_t gemm_gate_up_dgrad(const bf16* dgu, int64_t rows, const int32_t* off
                                unsigned* err) {
     if (rows == 0) return cudaSuccess;
     CUtensorMap ta, tb;
-    if (!make_map_2d(&ta, dgu, 2 * (uint64_t)I, rows, 2 * (uint64_t)I, BK, BM))
+    if (!make_map_2d(&ta, dgu, 2 * (uint64_t)I, rows, 2 * (uint64_t)I, BK, 128))
         return cudaErrorInvalidValue;
-    // B[n = h][k = c] = w_gate_up[e][h][c]: K-major, box 64 (c) x 256 (h)
-    if (!make_map_3d(&tb, w_gate_up, 2 * (uint64_t)I, H, E, BK, BN)) return cudaErrorInvalidValue;
+    // B[n = h][k = c] = w_gate_up[e][h][c]: K-major, box 64 (c) x 128 (h) per CTA of a
+    // pair, 64 x 256 for a single CTA
+    CUtensorMap tb1;
+    if (!make_map_3d(&tb, w_gate_up, 2 * (uint64_t)I, H, E, BK, BN / 2)) return cudaErrorInvalidValue;
+    if (!make_map_3d(&tb1, w_gate_up, 2 * (uint64_t)I, H, E, BK, BN)) return cudaErrorInvalidValue;
     Params p = base_params(E, rows, offsets, err);
     p.N = H;
     p.K = 2 * I;
     p.n_blocks = (H + BN - 1) / BN;
     p.out = dx_perm;
     p.ldo = H;
-    return launch<kEpiStore, false, false, false>(ta, tb, p,
-                                                  group_m_tile_bound(rows, E, p.n_blocks), st);
+    CUtensorMap to;
+    if (!make_store_map_2d(&to, dx_perm, H, rows, H)) return cudaErrorInvalidValue;
+    return launch_group_m<kEpiStore, false>(ta, tb, tb1, to, to, p, st);
 }
 
 cudaError_t gemm_wgrad(const bf16* X, const bf16* D, int64_t rows, const int32_t* offsets, int E,
@@ -654,13 +1026,15 @@ cudaError_t gemm_wgrad(const bf16* X, const bf16* D, int64_t rows, const int32_t
     Params p = base_params(E, rows, offsets, err);
     p.M = M;
     p.N = N;
-    p.m_blocks = (M + BM - 1) / BM;
+    p.m_blocks = (M + BM1 - 1) / BM1;
     p.n_blocks = (N + BN - 1) / BN;
     p.out = dW;
     p.ldo = N;
     p.out_group_stride = (int64_t)M * N;
-    return launch<kEpiStore, true, true, true>(ta, tb, p,
-                                               (int64_t)E * p.m_blocks * p.n_blocks, st);
+    CUtensorMap to;
+    if (!make_store_map_3d(&to, dW, N, M, E)) return cudaErrorInvalidValue;
+    return launch_1cta<kEpiStore, true, true, true>(ta, tb, to, to, p,
+                                                   (int64_t)E * p.m_blocks * p.n_blocks, st);
 }
 
 }  // namespace moe

@@ -256,6 +256,7 @@ __global__ void __launch_bounds__(1024)
                        unsigned* ticket) {
     __shared__ int warp_tot[32];
     __shared__ bool is_last;
+    int carry_off = 0;
     const int e = blockIdx.x;
     int32_t* row = block_base + (int64_t)e * nb;
     int carry = 0;
@@ -275,17 +276,20 @@ __global__ void __launch_bounds__(1024)
         is_last = (done == (unsigned)E - 1);
     }
     __syncthreads();
-    if (is_last && threadIdx.x == 0) {
-        __threadfence();
-        const volatile int32_t* c = counts;
-        int acc = 0;
-        offsets[0] = 0;
-        for (int i = 0; i < E; ++i) {
-            acc += c[i];
-            offsets[i + 1] = acc;
-        }
-        *ticket = 0u;
+    if (!is_last) return;
+    // last block: offsets = exclusive scan of all experts' counts, loaded in
+    // parallel (L2, bypassing L1) and scanned across the block
+    __threadfence();
+    for (int base = 0; base < E; base += blockDim.x) {
+        const int i = base + threadIdx.x;
+        const int v = i < E ? __ldcg(counts + i) : 0;
+        int total;
+        const int incl = block_inclusive_scan(v, warp_tot, total);
+        if (i < E) offsets[i + 1] = carry_off + incl;
+        if (base == 0 && threadIdx.x == 0) offsets[0] = 0;
+        carry_off += total;
     }
+    if (threadIdx.x == 0) *ticket = 0u;
 }
 
 // Token dispatch: one warp per token. Lane j < k computes the row of the

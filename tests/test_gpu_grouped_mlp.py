@@ -31,14 +31,17 @@ def grouped_case(T, H, I, E, k, seed, dead=(), skew=False):
     return m, w, d, r, p
 
 
+@pytest.mark.parametrize("tiles", ["single", "pair"])
 @pytest.mark.parametrize("T,H,I,E,k,dead", [
     (64, 128, 256, 8, 2, ()),            # the tiny workload's shape
     (1000, 256, 384, 4, 2, (2,)),        # several M tiles per expert, a ragged tail, an empty expert
     (300, 512, 192, 8, 2, (0, 7)),       # I not a multiple of 128: half-empty SwiGLU tile
     (700, 320, 640, 16, 4, ()),          # H not a multiple of 256: ragged N tile in the down GEMM
     (1, 128, 128, 8, 2, ()),             # a single token
+    (4500, 256, 256, 4, 2, (1,)),        # large expert blocks (the default picks pair tiles)
 ])
-def test_grouped_mlp_matches_expert_loop(T, H, I, E, k, dead):
+def test_grouped_mlp_matches_expert_loop(T, H, I, E, k, dead, tiles, monkeypatch):
+    monkeypatch.setenv("MOE_GEMM_TILES", tiles)
     m, w, d, r, p = grouped_case(T, H, I, E, k, seed=T + H + I, dead=dead)
     out = m.moe_grouped_mlp(p["x_perm"], r["offsets"], d["w_gate_up"], d["w_down"], save=True)
     torch.cuda.synchronize()

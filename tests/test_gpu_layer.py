@@ -47,8 +47,10 @@ SMALL = {
 }
 
 
+@pytest.mark.parametrize("tiles", ["single", "pair"])
 @pytest.mark.parametrize("name", list(SMALL))
-def test_layer_forward_matches_per_token_definition(name):
+def test_layer_forward_matches_per_token_definition(name, tiles, monkeypatch):
+    monkeypatch.setenv("MOE_GEMM_TILES", tiles)
     w = SMALL[name]
     d = wl.make_inputs(w, "cuda")
     out = layer(w, d)
@@ -80,14 +82,16 @@ def _oracle_backward(w, d, r):
                                bits(d["w_down"]), bits(d["dout"]))
 
 
+@pytest.mark.parametrize("tiles", ["single", "pair"])
 @pytest.mark.parametrize("name", BWD)
-def test_backward_on_oracle_state(name):
+def test_backward_on_oracle_state(name, tiles, monkeypatch):
     """The backward kernels fed with the oracle's own saved forward state, so
     both sides read identical bf16 inputs. dW_down and dprob then differ only
     in accumulation order; dW_gate_up and dx also carry the bf16 rounding of
     dg, du and each token row's dx, whose fp32 and fp64 pre-images can round
     apart (assert_close_flips)."""
     import routing_grouped_gemm_score_b200 as m
+    monkeypatch.setenv("MOE_GEMM_TILES", tiles)
     w = SMALL[name]
     d = wl.make_inputs(w, "cuda", with_dout=True)
     r = oracle.router_topk(d["logits"].cpu().numpy(), w.k)
