@@ -29,16 +29,18 @@
 // gemm_1cta_kernel (group-M with small expert blocks, and group-K: weight
 // gradients, dW[e] = X_e^T D_e). One CTA
 // per 128 x 256 tile, a 4-stage ring of 48 KB, tcgen05.mma.cta_group::1. The
-// reduction runs over the rows of expert e. In the last K slice, the rows
-// that belong to the next expert are zeroed in shared memory before the MMA.
+// reduction runs over the rows of expert e. In the last K slice only the
+// 16-row K steps that hold rows of expert e are issued, and the few rows of the
+// last step that belong to the next expert are zeroed in shared memory first.
 // An expert with no rows writes a zero tile.
 //
 // Warp roles, in both: warp 0 issues TMA loads (one thread); warp 1 owns
 // TMEM (two 128 x 256 fp32 accumulators, 512 columns) and issues the MMAs
-// (one thread); warps 2-5 are the epilogue (tcgen05.ld of their TMEM lane
-// quarter, the fused element-wise work, then 32 x 32 bf16 chunks staged in
-// shared memory and written by TMA stores; a 32-row group that crosses an
-// expert boundary is stored directly with masks instead). The two
+// (one thread); warps 2-9 are the epilogue, two per TMEM lane quarter, each
+// on one half of the tile's columns (tcgen05.ld of their TMEM lane
+// quarter, the fused element-wise work, then a transpose through a per-warp
+// shared-memory buffer so that each store instruction writes whole 128- or
+// 64-byte row segments; rows outside the expert's block are masked). The two
 // accumulators let the epilogue of one tile overlap the MMAs of the next.
 // Every wait is bounded (moe_common.cuh). On a timeout the kernel records an
 // error, every role leaves its loop, and TMEM is still freed.
@@ -55,7 +57,8 @@ namespace moe {
 namespace {
 
 constexpr int BN = 256, BK = 64;
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;                  // two per TMEM lane quarter, one per column half
+constexpr int kThreads = 64 + 32 * kEpiWarps;   // warp 0 TMA, warp 1 MMA, warps 2.. epilogue
 constexpr int kChunkBytes = 64 * BK * 2;  // one 64-wide swizzle chunk x 64 rows: 8 KB
 constexpr int kTmemCols = 512;
 constexpr int kMaxGroups = 256;
@@ -92,7 +95,7 @@ struct Params {
 template <int STAGES, int STAGE_BYTES>
 struct __align__(1024) Smem {
     uint8_t stage[STAGES][STAGE_BYTES];
-    uint8_t epi[4][2][2048];   // per epilogue warp: two 32 x 32 bf16 staging buffers
+    uint8_t epi[kEpiWarps][32 * 80];  // per epilogue warp: 32 rows x 32 bf16, rows padded to 80 B
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
     uint64_t acc_full[2];
@@ -212,46 +215,33 @@ __device__ __forceinline__ Tile decode_tile(const S& s, const Params& p, int id,
     return t;
 }
 
-// One epilogue warp's double-buffered staging area for TMA stores.
-struct Stager {
-    uint8_t* base;    // two 2 KB buffers, 1024-byte aligned
-    uint32_t count;   // TMA stores issued so far by this warp (lane 0)
-};
-
-// Stores 32 values of each lane's row (lane = row of the warp's 32-row group)
-// as bf16, through shared memory and one TMA store of a 32 x 32 box at
-// (x, y[, z]). The buffer layout matches the map's 64-byte swizzle: the
-// 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3). Warp-collective.
-template <int DIMS>
-__device__ __forceinline__ void staged_store(Stager& st, const CUtensorMap* map, const float* v,
-                                             int x, int y, int z, int lane) {
-    uint8_t* buf = st.base + (st.count & 1u) * 2048u;
-    if (st.count >= 2 && lane == 0) bulk_wait_group_read<1>();   // this buffer's last store has read it
-    __syncwarp();
+// Writes NC (32 or 64) values of each lane's row -- lane = row of the warp's
+// 32-row group -- as bf16 to rows [0, nvalid) at dst (row stride ld elements),
+// through the warp's staging buffer: each lane writes its row into shared
+// memory, then the warp reads it back so that one store instruction covers
+// whole row segments of 128 (NC=64) or 64 (NC=32) contiguous bytes. Rows are
+// padded by 16 bytes, so neither phase has more than 2-way bank conflicts.
+// Warp-collective.
+template <int NC>
+__device__ __forceinline__ void store_rows(uint8_t* buf, bf16* dst, int64_t ld, int nvalid,
+                                           const float* v, int lane) {
+    constexpr int kChunks = NC / 8;              // 16-byte chunks per row
+    constexpr int kRowsPerPass = 32 / kChunks;   // rows one instruction covers
+    constexpr int kPitch = NC * 2 + 16;          // padded row pitch of the buffer
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const uint4 w = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                                   pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
-                                   pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
-        *reinterpret_cast<uint4*>(buf + lane * 64 + ((q ^ ((lane >> 1) & 3)) * 16)) = w;
-    }
-    fence_proxy_async_smem();
+    for (int q = 0; q < kChunks; ++q)
+        *reinterpret_cast<uint4*>(buf + lane * kPitch + q * 16) =
+            make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                       pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
     __syncwarp();
-    if (lane == 0) {
-        if (DIMS == 2) tma_store_2d(map, buf, x, y);
-        else tma_store_3d(map, buf, x, y, z);
-        bulk_commit_group();
-    }
-    st.count += 1;
-}
-
-// Masked direct stores of 32 values of this thread's row at `dst`.
-__device__ __forceinline__ void direct_store32(bf16* dst, const float* v) {
-    uint4* d = reinterpret_cast<uint4*>(dst);
+    const int chunk = lane % kChunks;
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-        d[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                          pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+    for (int pass = 0; pass < kChunks; ++pass) {
+        const int row = pass * kRowsPerPass + lane / kChunks;
+        const uint4 w = *reinterpret_cast<const uint4*>(buf + row * kPitch + chunk * 16);
+        if (row < nvalid) *reinterpret_cast<uint4*>(dst + (int64_t)row * ld + chunk * 8) = w;
+    }
+    __syncwarp();   // the buffer is free again
 }
 
 // SwiGLU backward for 32 columns: dg, du from dh and the saved bf16 g, u.
@@ -279,93 +269,68 @@ __device__ __forceinline__ void swiglu_bwd32(const float* dh, const bf16* g_src,
 }
 
 // Epilogue of one tile for one epilogue warp. The warp owns rows
-// [warp_r0, warp_r0 + 32) of the tile; its lane `lane` reads TMEM lane row
-// t_row (the thread's accumulator row). For group-M the rows count from the
-// tile's first row; for group-K, from the first output row of the M block.
-// Groups of 32 rows that lie wholly inside the expert's block (always true for
-// group-K, whose 3-D output map clips at M) leave through TMA stores; the
-// others use masked direct stores, so no row of another expert is written.
+// [warp_r0, warp_r0 + 32) of the tile and one half of its columns (col_half);
+// lane `lane` reads TMEM lane row t_row (its accumulator row). For group-M the
+// rows count from the tile's first row, and only rows inside the expert's
+// block are written. For group-K they count from the first output row of the
+// M block.
 template <int EPI, bool GROUP_K>
 __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, uint32_t t_row,
-                                              int warp_r0, int lane, int n_tile,
-                                              const CUtensorMap* tmO, const CUtensorMap* tmO2,
-                                              Stager& st) {
+                                              int warp_r0, int col_half, int lane, int n_tile,
+                                              uint8_t* buf) {
     const int r = warp_r0 + lane;
     if (EPI == kEpiSwiglu) {
+        // accumulator columns: gate [0, 128), up [128, 256); this warp: h columns
+        // [64 * col_half, 64 * col_half + 64) of the tile
         const int n0 = t.n_blk * (n_tile / 2);
-        const bool valid = r < t.rows;
-        const bool staged = warp_r0 + 32 <= t.rows;
-        const int64_t grow = (int64_t)t.row0 + r;
-        const int yrow = t.row0 + warp_r0;
+        const int nvalid = min(max(t.rows - warp_r0, 0), 32);
+        const int64_t row0 = (int64_t)t.row0 + warp_r0;
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN / 2; c0 += 32) {
+        for (int c0 = 64 * col_half; c0 < 64 * col_half + 64; c0 += 32) {
             float g[32], u[32];
             tmem_load_2x32(t_row + c0, t_row + BN / 2 + c0, g, u);
             if (n0 + c0 >= p.N) continue;
-            float h[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) h[i] = silu_f(g[i]) * u[i];
-            if (staged) {
-                staged_store<2>(st, tmO, h, n0 + c0, yrow, 0, lane);
-                if (p.out2) {
-                    staged_store<2>(st, tmO2, g, n0 + c0, yrow, 0, lane);
-                    staged_store<2>(st, tmO2, u, p.I + n0 + c0, yrow, 0, lane);
-                }
-            } else if (valid) {
-                direct_store32(p.out + grow * p.ldo + n0 + c0, h);
-                if (p.out2) {
-                    direct_store32(p.out2 + grow * p.ldo2 + n0 + c0, g);
-                    direct_store32(p.out2 + grow * p.ldo2 + p.I + n0 + c0, u);
-                }
+            if (p.out2) {
+                store_rows<32>(buf, p.out2 + row0 * p.ldo2 + n0 + c0, p.ldo2, nvalid, g, lane);
+                store_rows<32>(buf, p.out2 + row0 * p.ldo2 + p.I + n0 + c0, p.ldo2, nvalid, u, lane);
             }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i]) * u[i];     // h, in place
+            store_rows<32>(buf, p.out + row0 * p.ldo + n0 + c0, p.ldo, nvalid, g, lane);
         }
     } else if (EPI == kEpiSwigluBwd) {
         const int n0 = t.n_blk * n_tile;
         const bool valid = r < t.rows;
-        const bool staged = warp_r0 + 32 <= t.rows;
+        const int nvalid = min(max(t.rows - warp_r0, 0), 32);
         const int64_t grow = (int64_t)t.row0 + r;
-        const int yrow = t.row0 + warp_r0;
+        const int64_t row0 = (int64_t)t.row0 + warp_r0;
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 64) {
-            float dh[64];
-            tmem_load_2x32(t_row + c0, t_row + c0 + 32, *reinterpret_cast<float(*)[32]>(dh),
-                           *reinterpret_cast<float(*)[32]>(dh + 32));
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                const int col = n0 + c0 + 32 * half;
-                if (col >= p.N) continue;
-                float dg[32], du[32];
-                if (valid)
-                    swiglu_bwd32(dh + 32 * half, p.aux + grow * p.ld_aux + col,
-                                 p.aux + grow * p.ld_aux + p.I + col, dg, du);
-                if (staged) {
-                    staged_store<2>(st, tmO, dg, col, yrow, 0, lane);
-                    staged_store<2>(st, tmO, du, p.I + col, yrow, 0, lane);
-                } else if (valid) {
-                    direct_store32(p.out + grow * p.ldo + col, dg);
-                    direct_store32(p.out + grow * p.ldo + p.I + col, du);
-                }
-            }
+        for (int c0 = 128 * col_half; c0 < 128 * col_half + 128; c0 += 32) {
+            float dh[32];
+            tmem_load_32(t_row + c0, dh);
+            const int col = n0 + c0;
+            if (col >= p.N) continue;
+            float dg[32], du[32];
+            if (valid)
+                swiglu_bwd32(dh, p.aux + grow * p.ld_aux + col, p.aux + grow * p.ld_aux + p.I + col,
+                             dg, du);
+            store_rows<32>(buf, p.out + row0 * p.ldo + col, p.ldo, nvalid, dg, lane);
+            store_rows<32>(buf, p.out + row0 * p.ldo + p.I + col, p.ldo, nvalid, du, lane);
         }
     } else {
         const int n0 = t.n_blk * n_tile;
-        bool valid, staged;
-        bf16* orow;
-        int yrow;
+        int nvalid;
+        bf16* row0;
         if (GROUP_K) {
-            const int m0 = t.m_blk * BM1;
-            valid = m0 + r < p.M;
-            staged = true;
-            orow = p.out + (int64_t)t.g * p.out_group_stride + (int64_t)(m0 + r) * p.ldo;
-            yrow = m0 + warp_r0;
+            const int m0 = t.m_blk * BM1 + warp_r0;
+            nvalid = min(max(p.M - m0, 0), 32);
+            row0 = p.out + (int64_t)t.g * p.out_group_stride + (int64_t)m0 * p.ldo;
         } else {
-            valid = r < t.rows;
-            staged = warp_r0 + 32 <= t.rows;
-            orow = p.out + ((int64_t)t.row0 + r) * p.ldo;
-            yrow = t.row0 + warp_r0;
+            nvalid = min(max(t.rows - warp_r0, 0), 32);
+            row0 = p.out + ((int64_t)t.row0 + warp_r0) * p.ldo;
         }
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 64) {
+        for (int c0 = 128 * col_half; c0 < 128 * col_half + 128; c0 += 64) {
             float v[64];
             if (t.num_kb > 0) {
                 tmem_load_2x32(t_row + c0, t_row + c0 + 32, *reinterpret_cast<float(*)[32]>(v),
@@ -376,14 +341,8 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
             }
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                const int col = n0 + c0 + 32 * half;
-                if (col >= p.N) continue;
-                if (staged) {
-                    if (GROUP_K) staged_store<3>(st, tmO, v + 32 * half, col, yrow, t.g, lane);
-                    else staged_store<2>(st, tmO, v + 32 * half, col, yrow, 0, lane);
-                } else if (valid) {
-                    direct_store32(orow + col, v + 32 * half);
-                }
+                if (n0 + c0 + 32 * half >= p.N) continue;
+                store_rows<32>(buf, row0 + n0 + c0 + 32 * half, p.ldo, nvalid, v + 32 * half, lane);
             }
         }
     }
@@ -393,7 +352,6 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
 template <int EPI, bool B_MN>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
                      const Params p) {
     extern __shared__ uint8_t smem_raw[];
     SmemP& s = *reinterpret_cast<SmemP*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -411,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s.acc_full[i], 1);
-            mbar_init(&s.acc_empty[i], 8);   // one arrival per epilogue warp of both CTAs
+            mbar_init(&s.acc_empty[i], 2 * kEpiWarps);   // one arrival per epilogue warp of both CTAs
         }
         mbar_init(&s.drain, 1);
         s.abort = 0;
@@ -530,10 +488,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------ epilogue (both CTAs)
-        const int quarter = warp & 3;
+        const int quarter = warp & 3;                           // TMEM lanes 32*quarter .. +31
+        const int col_half = (warp - 2) / 4;
         const int warp_r0 = (int)rank * 128 + quarter * 32;    // first row of the 256-row tile
-        Stager st{s.epi[quarter][0], 0};
-        prefetch_tensormap(&tmO);
         const uint32_t leader_acc_empty[2] = {mapa_shared(smem_u32(&s.acc_empty[0]), 0),
                                               mapa_shared(smem_u32(&s.acc_empty[1]), 0)};
         int local_tile = 0;
@@ -544,13 +501,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(&s.acc_full[buf], use & 1u, abort_flag, p.err)) break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-            epilogue_tile<EPI, false>(p, t, t_row, warp_r0, lane, BN, &tmO, &tmO2, st);
+            epilogue_tile<EPI, false>(p, t, t_row, warp_r0, col_half, lane, BN, s.epi[warp - 2]);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_acc_empty[buf]);
         }
-        if (lane == 0) bulk_wait_all();     // the last TMA stores have landed
-        __syncwarp();
     }
 
     tc_fence_before();
@@ -565,7 +520,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int EPI, bool A_MN, bool B_MN, bool GROUP_K>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_1cta_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
                      const Params p) {
     extern __shared__ uint8_t smem_raw[];
     Smem1& s = *reinterpret_cast<Smem1*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -581,7 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s.acc_full[i], 1);
-            mbar_init(&s.acc_empty[i], 128);
+            mbar_init(&s.acc_empty[i], 32 * kEpiWarps);
         }
         mbar_init(&s.drain, 1);
         s.abort = 0;
@@ -683,11 +637,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const uint32_t a_addr = smem_u32(s.stage[stage]);
                 const uint32_t b_addr = a_addr + kStageA1;
+                int ksteps = BK / 16;
                 if (GROUP_K) {
                     const int valid = t.rows - kb * BK;
                     if (valid < BK) {
-                        // rows [valid, 64) of every chunk belong to the next expert: zero them
-                        const int nrows = BK - valid;
+                        // Rows [valid, 64) belong to the next expert. Only the 16-row
+                        // K steps that hold valid rows are issued, and the rows of the
+                        // last one past `valid` are zeroed in both operands, so no other
+                        // expert's data reaches this expert's gradient.
+                        ksteps = (valid + 15) / 16;
+                        const int nrows = ksteps * 16 - valid;
                         for (int i = lane; i < nrows * 6 * 8; i += 32) {
                             const int chunk = i / (nrows * 8);
                             const int rem = i - chunk * nrows * 8;
@@ -696,13 +655,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                                   rr * 128) + q;
                             *dst = make_uint4(0, 0, 0, 0);
                         }
-                        fence_proxy_async_smem();
+                        if (nrows > 0) fence_proxy_async_smem();
                         __syncwarp();
                     }
                 }
                 if (lane == 0) {
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
+                        if (kk >= ksteps) break;
                         const uint64_t adesc =
                             A_MN ? smem_desc(a_addr + kk * 2048, kChunkBytes, 1024)
                                  : smem_desc(a_addr + kk * 32, 16, 1024);
@@ -733,9 +693,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------------ epilogue
         const int quarter = warp & 3;               // TMEM lanes 32*quarter .. +31
+        const int col_half = (warp - 2) / 4;
         const int warp_r0 = quarter * 32;           // first tile row of this warp
-        Stager st{s.epi[quarter][0], 0};
-        prefetch_tensormap(&tmO);
         int local_tile = 0;
         for (int id = blockIdx.x; id < total; id += gridDim.x, ++local_tile) {
             const Tile t = decode_tile<GROUP_K>(s, p, id, BM1);
@@ -744,12 +703,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(&s.acc_full[buf], use & 1u, abort_flag, p.err)) break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-            epilogue_tile<EPI, GROUP_K>(p, t, t_row, warp_r0, lane, BN, &tmO, &tmO2, st);
+            epilogue_tile<EPI, GROUP_K>(p, t, t_row, warp_r0, col_half, lane, BN, s.epi[warp - 2]);
             tc_fence_before();
             mbar_arrive(&s.acc_empty[buf]);
         }
-        if (lane == 0) bulk_wait_all();     // the last TMA stores have landed
-        __syncwarp();
     }
 
     tc_fence_before();
@@ -803,31 +760,6 @@ bool make_map_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Output maps: 32 x 32 boxes with the 64-byte swizzle of the staging buffers.
-bool make_store_map_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t pitch) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {inner, outer};
-    cuuint64_t strides[1] = {pitch * 2};
-    cuuint32_t box[2] = {32, 32};
-    cuuint32_t es[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
-              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
-              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-bool make_store_map_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[3] = {d0, d1, d2};
-    cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
-    cuuint32_t box[3] = {32, 32, 1};
-    cuuint32_t es[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
-              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
-              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <class K>
 cudaError_t set_smem_once(K kern, size_t bytes, std::once_flag& once, cudaError_t& status) {
     std::call_once(once, [&] {
@@ -837,8 +769,8 @@ cudaError_t set_smem_once(K kern, size_t bytes, std::once_flag& once, cudaError_
 }
 
 template <int EPI, bool B_MN>
-cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o,
-                        const CUtensorMap& o2, const Params& p, int64_t max_tiles, cudaStream_t st) {
+cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const Params& p,
+                        int64_t max_tiles, cudaStream_t st) {
     auto kern = gemm_pair_kernel<EPI, B_MN>;
     static std::once_flag once;
     static cudaError_t attr = cudaSuccess;
@@ -859,12 +791,12 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtens
     attrs[0].val.clusterDim.z = 1;
     cfg.attrs = attrs;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, a, b, o, o2, p);
+    return cudaLaunchKernelEx(&cfg, kern, a, b, p);
 }
 
 template <int EPI, bool A_MN, bool B_MN, bool GROUP_K>
-cudaError_t launch_1cta(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o,
-                        const CUtensorMap& o2, const Params& p, int64_t max_tiles, cudaStream_t st) {
+cudaError_t launch_1cta(const CUtensorMap& a, const CUtensorMap& b, const Params& p,
+                        int64_t max_tiles, cudaStream_t st) {
     auto kern = gemm_1cta_kernel<EPI, A_MN, B_MN, GROUP_K>;
     static std::once_flag once;
     static cudaError_t attr = cudaSuccess;
@@ -872,7 +804,7 @@ cudaError_t launch_1cta(const CUtensorMap& a, const CUtensorMap& b, const CUtens
     if (max_tiles <= 0) return cudaSuccess;
     int64_t grid = sm_count();
     if (grid > max_tiles) grid = max_tiles;
-    kern<<<(unsigned)grid, kThreads, kSmem1Bytes, st>>>(a, b, o, o2, p);
+    kern<<<(unsigned)grid, kThreads, kSmem1Bytes, st>>>(a, b, p);
     return cudaGetLastError();
 }
 
@@ -911,12 +843,10 @@ bool use_pair_tiles(int64_t rows, int groups) {
 // maps for each (their K-major boxes differ: 128 or 256 rows of N).
 template <int EPI, bool B_MN>
 cudaError_t launch_group_m(const CUtensorMap& ta, const CUtensorMap& tb_pair,
-                           const CUtensorMap& tb_single, const CUtensorMap& to,
-                           const CUtensorMap& to2, const Params& p, cudaStream_t st) {
+                           const CUtensorMap& tb_single, const Params& p, cudaStream_t st) {
     if (use_pair_tiles(p.rows, p.groups))
-        return launch_pair<EPI, B_MN>(ta, tb_pair, to, to2, p,
-                                      pair_tile_bound(p.rows, p.groups, p.n_blocks), st);
-    return launch_1cta<EPI, false, B_MN, false>(ta, tb_single, to, to2, p,
+        return launch_pair<EPI, B_MN>(ta, tb_pair, p, pair_tile_bound(p.rows, p.groups, p.n_blocks), st);
+    return launch_1cta<EPI, false, B_MN, false>(ta, tb_single, p,
                                                 single_tile_bound(p.rows, p.groups, p.n_blocks), st);
 }
 
@@ -940,15 +870,7 @@ cudaError_t gemm_gate_up_swiglu(const bf16* x, int64_t rows, const int32_t* offs
     p.ldo = I;
     p.out2 = gu_save;
     p.ldo2 = 2 * (int64_t)I;
-    CUtensorMap to, to2;
-    if (!make_store_map_2d(&to, h, I, rows, I)) return cudaErrorInvalidValue;
-    if (gu_save) {
-        if (!make_store_map_2d(&to2, gu_save, 2 * (uint64_t)I, rows, 2 * (uint64_t)I))
-            return cudaErrorInvalidValue;
-    } else {
-        to2 = to;
-    }
-    return launch_group_m<kEpiSwiglu, true>(ta, tb, tb, to, to2, p, st);
+    return launch_group_m<kEpiSwiglu, true>(ta, tb, tb, p, st);
 }
 
 cudaError_t gemm_down(const bf16* h, int64_t rows, const int32_t* offsets, int E, int H, int I,
@@ -964,9 +886,7 @@ cudaError_t gemm_down(const bf16* h, int64_t rows, const int32_t* offsets, int E
     p.n_blocks = (H + BN - 1) / BN;
     p.out = y;
     p.ldo = H;
-    CUtensorMap to;
-    if (!make_store_map_2d(&to, y, H, rows, H)) return cudaErrorInvalidValue;
-    return launch_group_m<kEpiStore, true>(ta, tb, tb, to, to, p, st);
+    return launch_group_m<kEpiStore, true>(ta, tb, tb, p, st);
 }
 
 cudaError_t gemm_down_dgrad_swiglu(const bf16* dy, int64_t rows, const int32_t* offsets, int E,
@@ -989,9 +909,7 @@ cudaError_t gemm_down_dgrad_swiglu(const bf16* dy, int64_t rows, const int32_t* 
     p.ldo = 2 * (int64_t)I;
     p.aux = gu;
     p.ld_aux = 2 * (int64_t)I;
-    CUtensorMap to;
-    if (!make_store_map_2d(&to, dgu, 2 * (uint64_t)I, rows, 2 * (uint64_t)I)) return cudaErrorInvalidValue;
-    return launch_group_m<kEpiSwigluBwd, false>(ta, tb, tb1, to, to, p, st);
+    return launch_group_m<kEpiSwigluBwd, false>(ta, tb, tb1, p, st);
 }
 
 cudaError_t gemm_gate_up_dgrad(const bf16* dgu, int64_t rows, const int32_t* offsets, int E, int H,
@@ -1012,9 +930,7 @@ cudaError_t gemm_gate_up_dgrad(const bf16* dgu, int64_t rows, const int32_t* off
     p.n_blocks = (H + BN - 1) / BN;
     p.out = dx_perm;
     p.ldo = H;
-    CUtensorMap to;
-    if (!make_store_map_2d(&to, dx_perm, H, rows, H)) return cudaErrorInvalidValue;
-    return launch_group_m<kEpiStore, false>(ta, tb, tb1, to, to, p, st);
+    return launch_group_m<kEpiStore, false>(ta, tb, tb1, p, st);
 }
 
 cudaError_t gemm_wgrad(const bf16* X, const bf16* D, int64_t rows, const int32_t* offsets, int E,
@@ -1031,9 +947,7 @@ cudaError_t gemm_wgrad(const bf16* X, const bf16* D, int64_t rows, const int32_t
     p.out = dW;
     p.ldo = N;
     p.out_group_stride = (int64_t)M * N;
-    CUtensorMap to;
-    if (!make_store_map_3d(&to, dW, N, M, E)) return cudaErrorInvalidValue;
-    return launch_1cta<kEpiStore, true, true, true>(ta, tb, to, to, p,
+    return launch_1cta<kEpiStore, true, true, true>(ta, tb, p,
                                                    (int64_t)E * p.m_blocks * p.n_blocks, st);
 }
 
