@@ -52,6 +52,8 @@ def parse():
                     help="override the token count (small cases for profiling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--router-sweep", action="store_true",
+                    help="also time the router alone at E=128, k=8, T = 2^16 .. 2^20")
     return ap.parse_args()
 
 
@@ -372,6 +374,22 @@ def our_arm(args, world, rank, local):
         gemm_flop += w.bwd_flops()
     gemm_tflops = gemm_flop / (gemm_ms / 1e3) / 1e12
 
+    # algorithmic bytes of the bandwidth-bound stages
+    hbm = peaks["hbm_gbs"]
+    T, H, k, E = w.T, w.H, w.k, w.E
+    bw_bytes = {
+        "fwd_router": T * E * 4 + T * k * 8 + E * 8,
+        "fwd_permute": T * H * 2 + A * H * 2 + A * 4 + T * k * 4,
+        "fwd_combine": A * H * 2 + T * H * 2 + T * k * 8 + (T * H * 2 if w.shared_expert else 0),
+    }
+    if w.backward:
+        bw_bytes["bwd_combine_bwd"] = T * H * 2 + 2 * A * H * 2 + T * k * 12
+        bw_bytes["bwd_dx_token_sum"] = A * H * 2 + T * H * 2 + T * k * 4
+    bandwidth = {}
+    for key, nbytes in bw_bytes.items():
+        gbs = nbytes / (stages[key] / 1e3) / 1e9
+        bandwidth[key] = {"bytes": nbytes, "us": stages[key] * 1e3, "GB/s": gbs, "frac_of_hbm": gbs / hbm}
+
     launches_fwd = 6 + (2 if w.shared_expert else 0)
     launches = K * (launches_fwd + (6 if w.backward else 0))
 
@@ -391,12 +409,16 @@ def our_arm(args, world, rank, local):
                      "peak_source": f"{peaks_src} {'sustained' if long_region else 'burst'} bf16",
                      "flop_per_launch": gate_up_flop, "ms_per_launch": gate_up_ms},
         "stages_ms": stages,
+        "bandwidth_kernels": bandwidth,
+        "hbm_peak_gbs": hbm,
         "gpu_launches": launches,
         "clocks": clocks,
     }
 
     if not args.no_e2e:
         line["e2e"] = e2e_measure(args, w, d, m, opts, ws, world)
+    if args.router_sweep:
+        line["router_sweep"] = router_sweep(m, hbm)
     if not args.no_cpu_baseline and world == 1 and rank == 0:
         threads = os.cpu_count() or 1
         runner = OracleRunner(w, cpu_inputs(w, d), threads)
@@ -410,6 +432,44 @@ def our_arm(args, world, rank, local):
     if rank == 0:
         print(json.dumps(line))
     return 0
+
+
+def router_sweep(m, hbm):
+    """The router alone (score + top-k + weights + counts/offsets) at E=128,
+    k=8 on N(0,1) logits, large T, each launch L2-cold (logits > L2 from
+    T = 2^18 on; before every launch a 256 MB read evicts them)."""
+    import ctypes
+
+    import torch
+    out = []
+    # a 256 MB read evicts the logits from L2 and leaves only clean lines there
+    flush = torch.ones(64 << 20, dtype=torch.float32, device="cuda")
+    for logT in (16, 18, 20):
+        T, E, k = 1 << logT, 128, 8
+        g = torch.Generator(device="cuda").manual_seed(77 + logT)
+        logits = torch.randn((T, E), generator=g, device="cuda")
+        res = m.moe_router_topk(logits, k)
+        ws = torch.empty(m.lib().moe_router_workspace_size(T, E, k), dtype=torch.uint8, device="cuda")
+        times = []
+        for it in range(8):
+            flush.sum()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            oc = m.RouterOpts().c()
+            s.record()
+            m.lib().moe_router_topk(logits.data_ptr(), T, E, k, ctypes.byref(oc),
+                                    res["topk_idx"].data_ptr(), res["topk_prob"].data_ptr(), None,
+                                    res["counts"].data_ptr(), res["offsets"].data_ptr(),
+                                    ws.data_ptr(), ws.numel(), torch.cuda.current_stream().cuda_stream)
+            e.record()
+            torch.cuda.synchronize()
+            if it >= 2:
+                times.append(s.elapsed_time(e))
+        ms = statistics.median(times)
+        nbytes = T * E * 4 + T * k * 8 + E * 8
+        gbs = nbytes / (ms / 1e3) / 1e9
+        out.append({"T": T, "E": E, "k": k, "us": ms * 1e3, "GB/s": gbs, "frac_of_hbm": gbs / hbm})
+        del logits, res, ws
+    return out
 
 
 def e2e_measure(args, w, d, m, opts, ws, world):

@@ -3,10 +3,10 @@
 // Transformer Engine "Mixture of Experts", sections Token combine and Token
 // probabilities:
 //   out[t] = shared[t] + sum_j p[t,j] * y_perm[row_of[t,j]]
-// One warp owns one output row, so the sum has a single writer and a fixed
+// One block owns one output row, so the sum has a single writer and a fixed
 // order (shared first, then j ascending, fp32). The result is the same on
 // every run, unlike a scatter-add with atomics. Rows move as 16-byte vectors
-// of 8 bf16.
+// of 8 bf16, and each thread issues the k loads of its column chunk together.
 #include "moe_common.cuh"
 #include "moe_internal.h"
 
@@ -47,107 +47,151 @@ __device__ __forceinline__ uint4 pack8(const float (&acc)[8]) {
                       pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
 }
 
+// One block per output row. The first k threads fetch the row's permuted
+// rows and weights into shared memory; then each thread owns 16-byte column
+// chunks and issues the k row loads of a chunk together.
 __global__ void __launch_bounds__(256)
     combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ row_of,
                    const float* __restrict__ probs, int64_t T, int k, int H8, int64_t A,
                    const uint4* __restrict__ shared, uint4* __restrict__ out, unsigned* err) {
-    const int lane = threadIdx.x & 31;
-    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T;
-         t += warps) {
-        int64_t my_row = -1;
-        float my_p = 0.0f;
-        if (lane < k) {
-            const int32_t r = row_of[t * k + lane];
-            if (r >= 0 && r < A) {
-                my_row = r;
-                my_p = probs ? probs[t * k + lane] : 1.0f;
-            } else {
-                raise_error(err, kErrDeviceCheck);
-            }
+    __shared__ int64_t rows[16];
+    __shared__ float ps[16];
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        if (threadIdx.x < (unsigned)k) {
+            const int j = threadIdx.x;
+            const int32_t r = row_of[t * k + j];
+            const bool ok = r >= 0 && r < A;
+            if (!ok) raise_error(err, kErrDeviceCheck);
+            rows[j] = ok ? r : -1;
+            ps[j] = probs ? probs[t * k + j] : 1.0f;
         }
-        // two 16-byte column chunks per lane and pass, so that 2k loads are in flight
-        for (int c0 = lane; c0 < H8; c0 += 64) {
-            const int c1 = c0 + 32;
-            const bool two = c1 < H8;
-            float a0[8], a1[8];
+        __syncthreads();
+        if (k <= 4) {
+            // few rows per token: two column chunks per thread and pass
+            for (int c0 = threadIdx.x; c0 < H8; c0 += 2 * blockDim.x) {
+                const int c1 = c0 + blockDim.x;
+                const bool two = c1 < H8;
+                float a0[8], a1[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) a0[i] = a1[i] = 0.0f;
-            if (shared) {
-                add_scaled(a0, __ldg(shared + t * H8 + c0), 1.0f);
-                if (two) add_scaled(a1, __ldg(shared + t * H8 + c1), 1.0f);
+                for (int i = 0; i < 8; ++i) a0[i] = a1[i] = 0.0f;
+                if (shared) {
+                    add_scaled(a0, __ldg(shared + t * H8 + c0), 1.0f);
+                    if (two) add_scaled(a1, __ldg(shared + t * H8 + c1), 1.0f);
+                }
+                uint4 v0[4], v1[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (j < k && rows[j] >= 0) {
+                        v0[j] = __ldg(y + rows[j] * H8 + c0);
+                        if (two) v1[j] = __ldg(y + rows[j] * H8 + c1);
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (j < k && rows[j] >= 0) {
+                        add_scaled(a0, v0[j], ps[j]);
+                        if (two) add_scaled(a1, v1[j], ps[j]);
+                    }
+                }
+                out[t * H8 + c0] = pack8(a0);
+                if (two) out[t * H8 + c1] = pack8(a1);
             }
-#pragma unroll 4
-            for (int j = 0; j < k; ++j) {
-                const int64_t r = __shfl_sync(kFull, my_row, j);
-                const float pj = __shfl_sync(kFull, my_p, j);
-                if (r < 0) continue;
-                const uint4 v0 = __ldg(y + r * H8 + c0);
-                const uint4 v1 = two ? __ldg(y + r * H8 + c1) : make_uint4(0, 0, 0, 0);
-                add_scaled(a0, v0, pj);
-                add_scaled(a1, v1, pj);
+        } else {
+            for (int c = threadIdx.x; c < H8; c += blockDim.x) {
+                float acc[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+                if (shared) add_scaled(acc, __ldg(shared + t * H8 + c), 1.0f);
+                for (int j0 = 0; j0 < k; j0 += 8) {      // up to 8 row loads in flight
+                    uint4 v[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        if (j0 + j < k && rows[j0 + j] >= 0) v[j] = __ldg(y + rows[j0 + j] * H8 + c);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        if (j0 + j < k && rows[j0 + j] >= 0) add_scaled(acc, v[j], ps[j0 + j]);
+                }
+                out[t * H8 + c] = pack8(acc);
             }
-            out[t * H8 + c0] = pack8(a0);
-            if (two) out[t * H8 + c1] = pack8(a1);
         }
+        __syncthreads();   // rows/ps are rewritten for the next row
     }
 }
 
-// Backward of the weighted combine, one warp per token:
+// Backward of the weighted combine, one block per token:
 //   dy_perm[row_of[t,j]] = bf16(p[t,j] * dout[t])
 //   dprob[t,j] = sum_h dout[t,h] * y_perm[row_of[t,j], h]   (fp32)
-// Each lane sums its own columns in order; the warp then reduces in a fixed
-// butterfly, so dprob is the same on every run. The dout row is read once per
-// assignment; after the first pass it comes from L1.
+// Each thread keeps its dout chunk in registers and sums its products for
+// every j; the block then reduces the k partial sums in a fixed tree (warp
+// butterfly, then warps in order), so dprob is the same on every run.
 __global__ void __launch_bounds__(256)
     combine_backward_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ y,
                             const int32_t* __restrict__ row_of, const float* __restrict__ probs,
                             int64_t T, int k, int H8, int64_t A, uint4* __restrict__ dy,
                             float* __restrict__ dprob, unsigned* err) {
-    const int lane = threadIdx.x & 31;
-    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T;
-         t += warps) {
-        int64_t my_row = -1;
-        float my_p = 0.0f;
-        if (lane < k) {
-            const int32_t r = row_of[t * k + lane];
-            if (r >= 0 && r < A) my_row = r;
-            else raise_error(err, kErrDeviceCheck);
-            my_p = probs[t * k + lane];
+    __shared__ int64_t rows[16];
+    __shared__ float ps[16];
+    __shared__ float part[8][16];   // per warp, per j
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        if (threadIdx.x < (unsigned)k) {
+            const int j = threadIdx.x;
+            const int32_t r = row_of[t * k + j];
+            const bool ok = r >= 0 && r < A;
+            if (!ok) raise_error(err, kErrDeviceCheck);
+            rows[j] = ok ? r : -1;
+            ps[j] = probs[t * k + j];
         }
-        for (int j = 0; j < k; ++j) {
-            const int64_t r = __shfl_sync(kFull, my_row, j);
-            const float pj = __shfl_sync(kFull, my_p, j);
-            float dot = 0.0f;
-            if (r >= 0) {
-                for (int c0 = lane; c0 < H8; c0 += 64) {
-                    const int c1 = c0 + 32;
-                    const bool two = c1 < H8;
-                    const uint4 d0 = __ldg(dout + t * H8 + c0);
-                    const uint4 y0 = __ldg(y + r * H8 + c0);
-                    const uint4 d1 = two ? __ldg(dout + t * H8 + c1) : make_uint4(0, 0, 0, 0);
-                    const uint4 y1 = two ? __ldg(y + r * H8 + c1) : make_uint4(0, 0, 0, 0);
-                    float s0[8], s1[8];
-                    dot_and_scale(d0, y0, pj, dot, s0);
-                    dot_and_scale(d1, y1, pj, dot, s1);
-                    dy[r * H8 + c0] = pack8(s0);
-                    if (two) dy[r * H8 + c1] = pack8(s1);
+        __syncthreads();
+        float dot[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) dot[j] = 0.0f;
+        for (int c = threadIdx.x; c < H8; c += blockDim.x) {
+            const uint4 d = __ldg(dout + t * H8 + c);
+#pragma unroll
+            for (int j0 = 0; j0 < 16; j0 += 8) {      // up to 8 row loads in flight
+                if (j0 >= k) break;
+                uint4 v[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    if (j0 + j < k && rows[j0 + j] >= 0) v[j] = __ldg(y + rows[j0 + j] * H8 + c);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (j0 + j >= k || rows[j0 + j] < 0) continue;
+                    float sc[8];
+                    dot_and_scale(d, v[j], ps[j0 + j], dot[j0 + j], sc);
+                    dy[rows[j0 + j] * H8 + c] = pack8(sc);
                 }
             }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(kFull, dot, off);
-            if (lane == 0) dprob[t * k + j] = dot;
         }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            if (j >= k) break;
+            float v = dot[j];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
+            if (lane == 0) part[warp][j] = v;
+        }
+        __syncthreads();
+        if (threadIdx.x < (unsigned)k) {
+            float sum = 0.0f;
+            for (int w = 0; w < nw; ++w) sum += part[w][threadIdx.x];
+            dprob[t * k + threadIdx.x] = sum;
+        }
+        __syncthreads();
     }
 }
 
-int64_t grid_for_warps(int64_t warps) {
-    int64_t blocks = (warps + 7) / 8;
-    const int64_t cap = (int64_t)sm_count() * 8;
-    if (blocks > cap) blocks = cap;
-    if (blocks < 1) blocks = 1;
-    return blocks;
+// Threads per block for one row of H8 chunks: one chunk per thread up to 256.
+int row_threads(int H8) {
+    int th = 32;
+    while (th < H8 && th < 256) th <<= 1;
+    return th;
+}
+
+int64_t row_blocks(int64_t T) {
+    const int64_t cap = (int64_t)sm_count() * 64;   // enough to fill the GPU; rows loop beyond
+    return T < cap ? (T > 0 ? T : 1) : cap;
 }
 
 }  // namespace
@@ -155,7 +199,7 @@ int64_t grid_for_warps(int64_t warps) {
 cudaError_t launch_combine(const bf16* y_perm, const int32_t* row_of, const float* probs,
                            int64_t T, int k, int H, int64_t A, const bf16* shared, bf16* out,
                            cudaStream_t st, unsigned* err) {
-    combine_kernel<<<(unsigned)grid_for_warps(T), 256, 0, st>>>(
+    combine_kernel<<<(unsigned)row_blocks(T), row_threads(H / 8), 0, st>>>(
         reinterpret_cast<const uint4*>(y_perm), row_of, probs, T, k, H / 8, A,
         reinterpret_cast<const uint4*>(shared), reinterpret_cast<uint4*>(out), err);
     return cudaGetLastError();
@@ -164,7 +208,7 @@ cudaError_t launch_combine(const bf16* y_perm, const int32_t* row_of, const floa
 cudaError_t launch_combine_backward(const bf16* dout, const bf16* y_perm, const int32_t* row_of,
                                     const float* probs, int64_t T, int k, int H, int64_t A,
                                     bf16* dy_perm, float* dprob, cudaStream_t st, unsigned* err) {
-    combine_backward_kernel<<<(unsigned)grid_for_warps(T), 256, 0, st>>>(
+    combine_backward_kernel<<<(unsigned)row_blocks(T), row_threads(H / 8), 0, st>>>(
         reinterpret_cast<const uint4*>(dout), reinterpret_cast<const uint4*>(y_perm), row_of, probs,
         T, k, H / 8, A, reinterpret_cast<uint4*>(dy_perm), dprob, err);
     return cudaGetLastError();

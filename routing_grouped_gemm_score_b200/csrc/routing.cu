@@ -5,10 +5,11 @@
 // dispatch; te_mixtral.py TEMixtralSparseMoeBlock.forward.
 //
 // Design: one warp per token. A lane holds the scores of experts lane,
-// lane+32, ... in registers. The k experts are picked in k rounds of a warp
-// arg-max over 64-bit keys (score ordered as an unsigned integer in the high
-// half, bit-inverted expert index in the low half), so a larger key means a
-// larger score, or the same score at a lower index. The choice is made on
+// lane+32, ... in registers. The k experts are picked in k rounds; each round
+// is two single-instruction warp reductions: the largest order key (the score
+// mapped to an unsigned integer that sorts like the float), then the lowest
+// expert index among the lanes holding it, which breaks ties toward the lower
+// index. The choice is made on
 // the logit itself: softmax and sigmoid are increasing, so the ranking is
 // the same and no rounding of the score function can create a tie. Ranks
 // inside each expert are counted per block of 64 tokens in shared memory, in
@@ -34,15 +35,6 @@ __device__ __forceinline__ uint32_t float_order_key(float s) {
     if ((b & 0x7FFFFFFFu) > 0x7F800000u) return 0u;  // NaN
     if ((b & 0x7FFFFFFFu) == 0u) b = 0u;             // -0 -> +0
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
-
-__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        uint64_t o = __shfl_xor_sync(kFull, v, off);
-        v = o > v ? o : v;
-    }
-    return v;
 }
 
 struct RouterArgs {
@@ -97,39 +89,56 @@ __global__ void __launch_bounds__(kRouteThreads) router_topk_kernel(const Router
         if (t >= a.T) break;
         const float* lrow = a.logits + t * E;
         float lv[SLOTS];
-        uint64_t key[SLOTS];
 #pragma unroll
         for (int s = 0; s < SLOTS; ++s) {
             const int e = lane + 32 * s;
             lv[s] = e < E ? __ldg(lrow + e) : 0.0f;
         }
+        // Each lane sorts its slots once, best first (larger key, then lower
+        // index; slots beyond E last); a round then only looks at list heads.
+        constexpr uint32_t kNone = 0xFFFFFFFFu;
+        uint32_t so[SLOTS], se[SLOTS];
 #pragma unroll
         for (int s = 0; s < SLOTS; ++s) {
             const int e = lane + 32 * s;
             float score = lv[s];
             if (a.bias) score = 1.0f / (1.0f + expf(-lv[s])) + __ldg(a.bias + (e < E ? e : 0));
-            key[s] = e < E ? ((uint64_t)float_order_key(score) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)e)
-                           : 0ull;
+            so[s] = e < E ? float_order_key(score) : 0u;
+            se[s] = e < E ? (uint32_t)e : kNone;
         }
-        uint64_t mine = 0;
 #pragma unroll
-        for (int s = 0; s < SLOTS; ++s) mine = key[s] > mine ? key[s] : mine;
-        unsigned taken = 0;   // bit s: slot s chosen
+        for (int i = 1; i < SLOTS; ++i)
+#pragma unroll
+            for (int j = i; j > 0; --j) {
+                // move slot j ahead of slot j-1 if it ranks better
+                const bool better = se[j] != kNone &&
+                                    (se[j - 1] == kNone || so[j] > so[j - 1] ||
+                                     (so[j] == so[j - 1] && se[j] < se[j - 1]));
+                const uint32_t o0 = so[j - 1], e0 = se[j - 1];
+                so[j - 1] = better ? so[j] : o0;
+                se[j - 1] = better ? se[j] : e0;
+                so[j] = better ? o0 : so[j];
+                se[j] = better ? e0 : se[j];
+            }
+        unsigned taken = 0;   // bit s: slot s chosen (for the routing map)
         int my_e = -1;        // lane j < k keeps the j-th chosen expert
         for (int j = 0; j < k; ++j) {
-            const uint64_t best = warp_max_u64(mine);
-            const int e = (int)(0xFFFFFFFFu - (uint32_t)best);
+            // the largest head key of the warp, then the lowest expert index holding it
+            const uint32_t top = __reduce_max_sync(kFull, se[0] == kNone ? 0u : so[0]);
+            const int e = (int)__reduce_min_sync(kFull, se[0] != kNone && so[0] == top ? se[0] : kNone);
             if (lane == j) my_e = e;
-            if (lane == (e & 31)) {
-                const int s_taken = e >> 5;
-                mine = 0;
-#pragma unroll
-                for (int s = 0; s < SLOTS; ++s) {
-                    if (s == s_taken) { key[s] = 0; taken |= 1u << s; }
-                    mine = key[s] > mine ? key[s] : mine;
-                }
+            const bool win = lane == (e & 31);
+            if (win) {
+                taken |= 1u << (e >> 5);
                 sel[tt][e] = (uint8_t)(j + 1);
             }
+#pragma unroll
+            for (int s = 0; s + 1 < SLOTS; ++s) {     // the winner pops its head
+                so[s] = win ? so[s + 1] : so[s];
+                se[s] = win ? se[s + 1] : se[s];
+            }
+            so[SLOTS - 1] = win ? 0u : so[SLOTS - 1];
+            se[SLOTS - 1] = win ? kNone : se[SLOTS - 1];
         }
         // routing weights (fp32), in the oracle's order of operations
         float my_l = (lane < k) ? __ldg(lrow + my_e) : 0.0f;
@@ -292,9 +301,10 @@ __global__ void __launch_bounds__(1024)
     if (threadIdx.x == 0) *ticket = 0u;
 }
 
-// Token dispatch: one warp per token. Lane j < k computes the row of the
-// token's j-th assignment; then the warp copies the token's row (16-byte
-// vectors) to each of its k destinations.
+// Token dispatch: one block per token. The first k threads compute the rows
+// of the token's k assignments (expert offset + rank of the token block +
+// rank inside it) into shared memory; then each thread reads its 16-byte
+// column chunks of the token's row once and writes them to the k rows.
 __global__ void __launch_bounds__(256)
     permute_kernel(const uint4* __restrict__ x, int64_t T, int H8, const int32_t* __restrict__ topk_idx,
                    int k, const int32_t* __restrict__ offsets, int E,
@@ -302,44 +312,37 @@ __global__ void __launch_bounds__(256)
                    const int32_t* __restrict__ local_rank, uint4* __restrict__ x_perm,
                    int32_t* __restrict__ sorted_token, int32_t* __restrict__ row_of, int64_t A,
                    unsigned* err) {
-    const int lane = threadIdx.x & 31;
-    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T;
-         t += warps) {
-        int64_t row = -1;
-        if (lane < k) {
-            const int e = topk_idx[t * k + lane];
-            const int rank = local_rank[t * k + lane];
+    __shared__ int64_t rows[16];
+    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+        if (threadIdx.x < (unsigned)k) {
+            const int j = threadIdx.x;
+            int64_t row = -1;
+            const int e = topk_idx[t * k + j];
+            const int rank = local_rank[t * k + j];
             if (e >= 0 && e < E && rank >= 0) {
-                const int64_t r = (int64_t)offsets[e] +
-                                  block_base[(int64_t)e * nb + t / tpb] + rank;
+                const int64_t r = (int64_t)offsets[e] + block_base[(int64_t)e * nb + t / tpb] + rank;
                 if (r >= offsets[e] && r < offsets[e + 1] && r < A) row = r;
             }
             if (row < 0) raise_error(err, kErrDeviceCheck);
-            row_of[t * k + lane] = (int32_t)row;
+            row_of[t * k + j] = (int32_t)row;
             if (row >= 0) sorted_token[row] = (int32_t)t;
+            rows[j] = row;
         }
-        int64_t rows[16];
+        __syncthreads();
+        for (int c0 = threadIdx.x; c0 < H8; c0 += 2 * blockDim.x) {   // two loads in flight
+            const int c1 = c0 + blockDim.x;
+            const bool two = c1 < H8;
+            const uint4 v0 = __ldg(x + t * H8 + c0);
+            const uint4 v1 = two ? __ldg(x + t * H8 + c1) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) rows[j] = (j < k) ? __shfl_sync(kFull, row, j) : -1;
-        const uint4* src = x + t * H8;
-        int c = lane;
-        for (; c + 32 < H8; c += 64) {  // two 16-byte loads in flight per lane
-            const uint4 v0 = __ldg(src + c);
-            const uint4 v1 = __ldg(src + c + 32);
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-                if (rows[j] >= 0) {
-                    x_perm[rows[j] * H8 + c] = v0;
-                    x_perm[rows[j] * H8 + c + 32] = v1;
+            for (int j = 0; j < 16; ++j) {
+                if (j < k && rows[j] >= 0) {
+                    x_perm[rows[j] * H8 + c0] = v0;
+                    if (two) x_perm[rows[j] * H8 + c1] = v1;
                 }
+            }
         }
-        for (; c < H8; c += 32) {
-            const uint4 v0 = __ldg(src + c);
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-                if (rows[j] >= 0) x_perm[rows[j] * H8 + c] = v0;
-        }
+        __syncthreads();
     }
 }
 
@@ -424,12 +427,15 @@ cudaError_t launch_permute(const bf16* x, int64_t T, int H, const int32_t* topk_
                            const int32_t* offsets, int E, const RouteScratch& rs, bf16* x_perm,
                            int32_t* sorted_token, int32_t* row_of, cudaStream_t st, unsigned* err) {
     const int nb = (int)route_blocks(T);
-    const int64_t warps_needed = T;
-    int64_t blocks = (warps_needed + 7) / 8;
-    const int64_t cap = (int64_t)sm_count() * 8;   // 8 resident 256-thread blocks per SM
+    const int H8 = H / 8;
+    int threads = 32;
+    while (threads < H8 && threads < 256) threads <<= 1;
+    int64_t blocks = T;
+    const int64_t cap = (int64_t)sm_count() * 64;
     if (blocks > cap) blocks = cap;
-    permute_kernel<<<(unsigned)blocks, 256, 0, st>>>(
-        reinterpret_cast<const uint4*>(x), T, H / 8, topk_idx, k, offsets, E, rs.block_base, nb,
+    if (blocks < 1) blocks = 1;
+    permute_kernel<<<(unsigned)blocks, threads, 0, st>>>(
+        reinterpret_cast<const uint4*>(x), T, H8, topk_idx, k, offsets, E, rs.block_base, nb,
         route_tokens_per_block(T), rs.local_rank, reinterpret_cast<uint4*>(x_perm), sorted_token,
         row_of, T * k, err);
     return cudaGetLastError();
