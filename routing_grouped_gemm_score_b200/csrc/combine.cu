@@ -199,6 +199,9 @@ int64_t row_blocks(int64_t T) {
 cudaError_t launch_combine(const bf16* y_perm, const int32_t* row_of, const float* probs,
                            int64_t T, int k, int H, int64_t A, const bf16* shared, bf16* out,
                            cudaStream_t st, unsigned* err) {
+    cudaError_t res = cudaSuccess;
+    if (T == 0) return cudaSuccess;
+    if (rows_combine(y_perm, row_of, probs, T, k, H, A, shared, out, st, err, &res)) return res;
     combine_kernel<<<(unsigned)row_blocks(T), row_threads(H / 8), 0, st>>>(
         reinterpret_cast<const uint4*>(y_perm), row_of, probs, T, k, H / 8, A,
         reinterpret_cast<const uint4*>(shared), reinterpret_cast<uint4*>(out), err);
@@ -208,6 +211,9 @@ cudaError_t launch_combine(const bf16* y_perm, const int32_t* row_of, const floa
 cudaError_t launch_combine_backward(const bf16* dout, const bf16* y_perm, const int32_t* row_of,
                                     const float* probs, int64_t T, int k, int H, int64_t A,
                                     bf16* dy_perm, float* dprob, cudaStream_t st, unsigned* err) {
+    if (T == 0) return cudaSuccess;
+    // The register-path kernel below measured faster than the bulk-copy one
+    // (rows_combine_backward) at the Qwen3-30B-A3B shape, so it is the one used.
     combine_backward_kernel<<<(unsigned)row_blocks(T), row_threads(H / 8), 0, st>>>(
         reinterpret_cast<const uint4*>(dout), reinterpret_cast<const uint4*>(y_perm), row_of, probs,
         T, k, H / 8, A, reinterpret_cast<uint4*>(dy_perm), dprob, err);

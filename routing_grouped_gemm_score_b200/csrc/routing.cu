@@ -73,16 +73,60 @@ __device__ __forceinline__ void rank_block(const uint8_t (*sel)[256], int64_t t0
     }
 }
 
+// Inverse of float_order_key for a key that came from a logit: key 0 (NaN)
+// gives NaN, and -0 comes back as +0, which changes no routing weight.
+__device__ __forceinline__ float order_key_to_float(uint32_t key) {
+    if (key == 0u) return __uint_as_float(0x7FC00000u);
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+// Put slot j behind slot i unless j ranks strictly better (larger key, or the
+// same key and a lower expert index).
+__device__ __forceinline__ void order_pair(uint32_t& ki, uint32_t& ei, uint32_t& kj, uint32_t& ej) {
+    const bool swap = kj > ki || (kj == ki && ej < ei);
+    const uint32_t k0 = ki, e0 = ei;
+    ki = swap ? kj : ki;
+    ei = swap ? ej : ei;
+    kj = swap ? k0 : kj;
+    ej = swap ? e0 : ej;
+}
+
+// Sort a lane's slots best first. Networks: 1 pair for 2, 5 pairs for 4,
+// Batcher's odd-even merge (19 pairs) for 8.
 template <int SLOTS>
+__device__ __forceinline__ void sort_slots(uint32_t (&so)[SLOTS], uint32_t (&se)[SLOTS]) {
+    if constexpr (SLOTS == 2) {
+        order_pair(so[0], se[0], so[1], se[1]);
+    } else if constexpr (SLOTS == 4) {
+        constexpr int net[5][2] = {{0, 1}, {2, 3}, {0, 2}, {1, 3}, {1, 2}};
+#pragma unroll
+        for (int c = 0; c < 5; ++c) order_pair(so[net[c][0]], se[net[c][0]], so[net[c][1]], se[net[c][1]]);
+    } else if constexpr (SLOTS == 8) {
+        constexpr int net[19][2] = {{0, 1}, {2, 3}, {4, 5}, {6, 7}, {0, 2}, {1, 3}, {4, 6},
+                                    {5, 7}, {1, 2}, {5, 6}, {0, 4}, {1, 5}, {2, 6}, {3, 7},
+                                    {2, 4}, {3, 5}, {1, 2}, {3, 4}, {5, 6}};
+#pragma unroll
+        for (int c = 0; c < 19; ++c) order_pair(so[net[c][0]], se[net[c][0]], so[net[c][1]], se[net[c][1]]);
+    }
+}
+
+// Router, one warp per token. SLOTS = experts per lane (E <= 32*SLOTS). KC is
+// the number of picks when fixed at compile time, or 0 for any k <= 16 given
+// at run time.
+template <int SLOTS, int KC>
 __global__ void __launch_bounds__(kRouteThreads) router_topk_kernel(const RouterArgs a) {
     __shared__ uint8_t sel[kMaxTokensPerRouteBlock][256];
+    __shared__ __align__(16) float wbuf[kRouteThreads / 32][32 * SLOTS];   // per warp: values to sum in order
+    constexpr int KMAX = KC ? KC : 16;
+    constexpr uint32_t kNone = 0xFFFFFFFFu;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int E = a.E, k = a.k, tpb = a.tpb;
+    const int E = a.E, k = KC ? KC : a.k, tpb = a.tpb;
     for (int i = threadIdx.x; i < tpb * 256 / 16; i += blockDim.x)
         reinterpret_cast<uint4*>(&sel[0][0])[i] = make_uint4(0, 0, 0, 0);
     if (blockIdx.x == 0 && threadIdx.x == 0) *a.ticket = 0u;
     __syncthreads();
     const int64_t t0 = (int64_t)blockIdx.x * tpb;
+    float* wrow = wbuf[warp];
 
     for (int tt = warp; tt < tpb; tt += kRouteThreads / 32) {
         const int64_t t = t0 + tt;
@@ -94,9 +138,8 @@ __global__ void __launch_bounds__(kRouteThreads) router_topk_kernel(const Router
             const int e = lane + 32 * s;
             lv[s] = e < E ? __ldg(lrow + e) : 0.0f;
         }
-        // Each lane sorts its slots once, best first (larger key, then lower
-        // index; slots beyond E last); a round then only looks at list heads.
-        constexpr uint32_t kNone = 0xFFFFFFFFu;
+        // Selection keys; a slot beyond E has key 0 and index kNone, so it
+        // ranks below every expert, a NaN one (key 0, real index) included.
         uint32_t so[SLOTS], se[SLOTS];
 #pragma unroll
         for (int s = 0; s < SLOTS; ++s) {
@@ -106,88 +149,86 @@ __global__ void __launch_bounds__(kRouteThreads) router_topk_kernel(const Router
             so[s] = e < E ? float_order_key(score) : 0u;
             se[s] = e < E ? (uint32_t)e : kNone;
         }
+        sort_slots<SLOTS>(so, se);   // best first in each lane
+        // k rounds: the largest head key, then the lowest expert index holding
+        // it; the lane that owns the pick drops its head.
+        int my_e = 0;
+        uint32_t my_key = 0u, top0 = 0u;
 #pragma unroll
-        for (int i = 1; i < SLOTS; ++i)
+        for (int j = 0; j < KMAX; ++j) {
+            if (KC == 0 && j >= k) break;
+            const uint32_t top = __reduce_max_sync(kFull, so[0]);
+            const uint32_t e = __reduce_min_sync(kFull, so[0] == top ? se[0] : kNone);
+            if (j == 0) top0 = top;
+            my_e = lane == j ? (int)e : my_e;
+            my_key = lane == j ? top : my_key;
+            const bool win = lane == (int)(e & 31u);
 #pragma unroll
-            for (int j = i; j > 0; --j) {
-                // move slot j ahead of slot j-1 if it ranks better
-                const bool better = se[j] != kNone &&
-                                    (se[j - 1] == kNone || so[j] > so[j - 1] ||
-                                     (so[j] == so[j - 1] && se[j] < se[j - 1]));
-                const uint32_t o0 = so[j - 1], e0 = se[j - 1];
-                so[j - 1] = better ? so[j] : o0;
-                se[j - 1] = better ? se[j] : e0;
-                so[j] = better ? o0 : so[j];
-                se[j] = better ? e0 : se[j];
-            }
-        unsigned taken = 0;   // bit s: slot s chosen (for the routing map)
-        int my_e = -1;        // lane j < k keeps the j-th chosen expert
-        for (int j = 0; j < k; ++j) {
-            // the largest head key of the warp, then the lowest expert index holding it
-            const uint32_t top = __reduce_max_sync(kFull, se[0] == kNone ? 0u : so[0]);
-            const int e = (int)__reduce_min_sync(kFull, se[0] != kNone && so[0] == top ? se[0] : kNone);
-            if (lane == j) my_e = e;
-            const bool win = lane == (e & 31);
-            if (win) {
-                taken |= 1u << (e >> 5);
-                sel[tt][e] = (uint8_t)(j + 1);
-            }
-#pragma unroll
-            for (int s = 0; s + 1 < SLOTS; ++s) {     // the winner pops its head
+            for (int s = 0; s + 1 < SLOTS; ++s) {
                 so[s] = win ? so[s + 1] : so[s];
                 se[s] = win ? se[s + 1] : se[s];
             }
             so[SLOTS - 1] = win ? 0u : so[SLOTS - 1];
             se[SLOTS - 1] = win ? kNone : se[SLOTS - 1];
         }
-        // routing weights (fp32), in the oracle's order of operations
-        float my_l = (lane < k) ? __ldg(lrow + my_e) : 0.0f;
+        const bool picks = lane < k;                 // lane j holds the j-th pick
+        if (picks) sel[tt][my_e] = (uint8_t)(lane + 1);
+        // logit of the pick: the key inverted, or reread when a bias shaped the key
+        float my_l = 0.0f;
+        if (picks) my_l = a.bias ? __ldg(lrow + my_e) : order_key_to_float(my_key);
+
+        // routing weights (fp32), in the oracle's order of operations; sums
+        // run in order over a per-warp row of shared memory
+        __syncwarp();
         float p = 0.0f;
         if (a.score_fn == MOE_SCORE_SOFTMAX) {
             if (a.renormalize) {
-                // max over the chosen, scanned in selection order
-                float m = __shfl_sync(kFull, my_l, 0);
-                for (int j = 1; j < k; ++j) {
-                    const float lj = __shfl_sync(kFull, my_l, j);
-                    if (lj > m) m = lj;
-                }
-                const float ex = (lane < k) ? expf(my_l - m) : 0.0f;
+                // the first pick holds the largest logit of the picks (or NaN)
+                const float m = __shfl_sync(kFull, my_l, 0);
+                const float ex = picks ? expf(my_l - m) : 0.0f;
+                if (lane < KMAX) wrow[lane] = ex;
+                __syncwarp();
                 float sum = 0.0f;
-                for (int j = 0; j < k; ++j) sum += __shfl_sync(kFull, ex, j);
+#pragma unroll
+                for (int j = 0; j < KMAX; ++j) sum += (KC || j < k) ? wrow[j] : 0.0f;
                 p = ex / sum;
             } else {
-                // softmax over all experts: row max and sum scanned in expert order
-                float m = __shfl_sync(kFull, lv[0], 0);
+                // softmax over all experts: row maximum (NaN if expert 0 is
+                // NaN, as a scan from expert 0 gives), then the sum in expert order
+                const bool nan0 = isnan(__shfl_sync(kFull, lv[0], 0));
+                const float m = nan0 ? __uint_as_float(0x7FC00000u) : order_key_to_float(top0);
 #pragma unroll
-                for (int s = 0; s < SLOTS; ++s)
-                    for (int src = 0; src < 32; ++src) {
-                        const float v = __shfl_sync(kFull, lv[s], src);
-                        if (src + 32 * s < E && v > m) m = v;
-                    }
-                float ex_all[SLOTS];
-#pragma unroll
-                for (int s = 0; s < SLOTS; ++s) ex_all[s] = expf(lv[s] - m);
+                for (int s = 0; s < SLOTS; ++s) {
+                    const int e = lane + 32 * s;
+                    wrow[e] = e < E ? expf(lv[s] - m) : 0.0f;
+                }
+                __syncwarp();
                 float sum = 0.0f;
-#pragma unroll
-                for (int s = 0; s < SLOTS; ++s)
-                    for (int src = 0; src < 32; ++src) {
-                        const float v = __shfl_sync(kFull, ex_all[s], src);
-                        if (src + 32 * s < E) sum += v;
-                    }
-                p = (lane < k) ? expf(my_l - m) / sum : 0.0f;
+                const float4* w4 = reinterpret_cast<const float4*>(wrow);
+                for (int q = 0; q < (E + 3) / 4; ++q) {
+                    const float4 v = w4[q];
+                    sum += v.x;
+                    sum += v.y;
+                    sum += v.z;
+                    sum += v.w;
+                }
+                p = picks ? expf(my_l - m) / sum : 0.0f;
             }
         } else {
-            const float sg = (lane < k) ? 1.0f / (1.0f + expf(-my_l)) : 0.0f;
+            const float sg = picks ? 1.0f / (1.0f + expf(-my_l)) : 0.0f;
             if (a.renormalize) {
+                if (lane < KMAX) wrow[lane] = sg;
+                __syncwarp();
                 float sum = 0.0f;
-                for (int j = 0; j < k; ++j) sum += __shfl_sync(kFull, sg, j);
+#pragma unroll
+                for (int j = 0; j < KMAX; ++j) sum += (KC || j < k) ? wrow[j] : 0.0f;
                 p = sg / sum;
             } else {
                 p = sg;
             }
         }
         p = p * a.scaling;
-        if (lane < k) {
+        if (picks) {
             a.topk_idx[t * k + lane] = my_e;
             a.topk_prob[t * k + lane] = p;
         }
@@ -196,9 +237,10 @@ __global__ void __launch_bounds__(kRouteThreads) router_topk_kernel(const Router
 #pragma unroll
             for (int s = 0; s < SLOTS; ++s) {
                 const int e = lane + 32 * s;
-                if (e < E) mrow[e] = (taken >> s) & 1u;
+                if (e < E) mrow[e] = sel[tt][e] != 0 ? 1 : 0;
             }
         }
+        __syncwarp();   // wrow and this token's sel row are settled before the next token
     }
     __syncthreads();
     rank_block(sel, t0, tpb, E, k, a.local_rank, a.block_base, a.nb);
@@ -375,6 +417,18 @@ RouteScratch carve_route_scratch(void* base, int64_t T, int E, int k) {
     return rs;
 }
 
+template <int SLOTS>
+void launch_router_k(const RouterArgs& a, dim3 grid, dim3 block, cudaStream_t st) {
+    switch (a.k) {
+        case 1: router_topk_kernel<SLOTS, 1><<<grid, block, 0, st>>>(a); break;
+        case 2: router_topk_kernel<SLOTS, 2><<<grid, block, 0, st>>>(a); break;
+        case 4: router_topk_kernel<SLOTS, 4><<<grid, block, 0, st>>>(a); break;
+        case 6: router_topk_kernel<SLOTS, 6><<<grid, block, 0, st>>>(a); break;
+        case 8: router_topk_kernel<SLOTS, 8><<<grid, block, 0, st>>>(a); break;
+        default: router_topk_kernel<SLOTS, 0><<<grid, block, 0, st>>>(a); break;
+    }
+}
+
 cudaError_t launch_router_topk(const float* logits, int64_t T, int E, int k,
                                const moe_router_opts& opts, int32_t* topk_idx, float* topk_prob,
                                uint8_t* routing_map, const RouteScratch& rs, cudaStream_t st,
@@ -397,10 +451,10 @@ cudaError_t launch_router_topk(const float* logits, int64_t T, int E, int k,
     a.nb = (int)route_blocks(T);
     a.tpb = route_tokens_per_block(T);
     const dim3 grid((unsigned)a.nb), block(kRouteThreads);
-    if (E <= 32) router_topk_kernel<1><<<grid, block, 0, st>>>(a);
-    else if (E <= 64) router_topk_kernel<2><<<grid, block, 0, st>>>(a);
-    else if (E <= 128) router_topk_kernel<4><<<grid, block, 0, st>>>(a);
-    else router_topk_kernel<8><<<grid, block, 0, st>>>(a);
+    if (E <= 32) launch_router_k<1>(a, grid, block, st);
+    else if (E <= 64) launch_router_k<2>(a, grid, block, st);
+    else if (E <= 128) launch_router_k<4>(a, grid, block, st);
+    else launch_router_k<8>(a, grid, block, st);
     (void)err;
     return cudaGetLastError();
 }
@@ -427,6 +481,11 @@ cudaError_t launch_permute(const bf16* x, int64_t T, int H, const int32_t* topk_
                            const int32_t* offsets, int E, const RouteScratch& rs, bf16* x_perm,
                            int32_t* sorted_token, int32_t* row_of, cudaStream_t st, unsigned* err) {
     const int nb = (int)route_blocks(T);
+    if (T == 0) return cudaSuccess;
+    cudaError_t res = cudaSuccess;
+    if (rows_permute(x, T, H, topk_idx, k, offsets, E, rs.block_base, nb, route_tokens_per_block(T),
+                     rs.local_rank, x_perm, sorted_token, row_of, T * k, st, err, &res))
+        return res;
     const int H8 = H / 8;
     int threads = 32;
     while (threads < H8 && threads < 256) threads <<= 1;

@@ -73,6 +73,46 @@ def test_router_ties_and_degenerate_values():
     assert np.array_equal(np.isnan(gp), np.isnan(rp))
 
 
+MODES = {"softmax_renorm": (0, True), "softmax_all": (0, False), "sigmoid": (1, False),
+         "sigmoid_renorm": (1, True)}
+
+
+@pytest.mark.parametrize("mode", list(MODES))
+@pytest.mark.parametrize("k", [1, 2, 3, 4, 6, 8, 16])
+@pytest.mark.parametrize("E", [20, 64, 128, 256])
+def test_router_every_slot_count_and_k(E, k, mode):
+    """Each lane holds E/32 experts (1, 2, 4 or 8 slots) and k = 1, 2, 4, 6, 8
+    have kernels of their own, other k a generic one: every pairing, every
+    score function and weight mode."""
+    score, renorm = MODES[mode]
+    g_ = torch.Generator().manual_seed(E * 131 + k * 7 + score * 3 + renorm)
+    logits = torch.randn((97, E), generator=g_) * 3
+    check(*run_both(logits, k, score, renorm))
+
+
+@pytest.mark.parametrize("mode", list(MODES))
+def test_router_degenerate_values_every_mode(mode):
+    """NaN at expert 0 (the row maximum scan then yields NaN), a NaN elsewhere,
+    rows of -inf, signed zeros: indices exact, NaN where the oracle has NaN."""
+    score, renorm = MODES[mode]
+    g_ = torch.Generator().manual_seed(17)
+    logits = torch.randn((64, 128), generator=g_)
+    logits[0, 0] = float("nan")
+    logits[1, 77] = float("nan")
+    logits[2] = float("-inf")
+    logits[3] = -0.0
+    logits[3, 100] = 0.0
+    logits[4, :120] = float("nan")
+    g, r = run_both(logits, 8, score, renorm)
+    assert_equal(g["topk_idx"], r["topk_idx"], "topk_idx")
+    assert_equal(g["routing_map"], r["routing_map"], "routing_map")
+    assert_equal(g["counts"], r["counts"], "counts")
+    gp, rp = g["topk_prob"].cpu().numpy(), r["topk_prob"]
+    assert np.array_equal(np.isnan(gp), np.isnan(rp)), "NaN positions"
+    finite = np.isfinite(rp)
+    np.testing.assert_allclose(gp[finite], rp[finite], rtol=1e-6, atol=0)
+
+
 def test_router_options():
     g_ = torch.Generator().manual_seed(9)
     logits = torch.randn((500, 48), generator=g_) * 2
