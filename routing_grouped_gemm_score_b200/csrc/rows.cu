@@ -40,7 +40,7 @@ constexpr int kRowsThreads = 32 * (1 + kConsumerWarps);
 constexpr int kConsumerThreads = 32 * kConsumerWarps;
 constexpr int kMaxStages = 8;
 constexpr uint32_t kStageBudget = 16u * 1024;    // one stage: the row pieces of a unit
-constexpr uint32_t kBlockBudget = 100u * 1024;   // all stages of a block
+constexpr uint32_t kBlockBudget = 48u * 1024;    // all stages of a block: four blocks per SM
 constexpr int kMaxBlocksPerSm = 4;
 constexpr int kRouteEntries = 128;              // assignments per routing chunk
 
