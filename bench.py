@@ -405,7 +405,7 @@ def our_arm(args, world, rank, local):
         "roofline": {"bound": "tensor", "kernel": "grouped_gemm_kernel<SwiGLU> (gate_up)",
                      "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": achieved / peak_tf, "frac_of_burst_peak": achieved / burst_tf,
-                     "traffic": traffic_for("gate_up_swiglu"),
+                     "traffic": traffic_for(f"gate_up_swiglu/{w.name}"),
                      "peak_source": f"{peaks_src} {'sustained' if long_region else 'burst'} bf16",
                      "flop_per_launch": gate_up_flop, "ms_per_launch": gate_up_ms},
         "stages_ms": stages,
