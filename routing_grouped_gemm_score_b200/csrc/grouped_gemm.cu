@@ -277,7 +277,7 @@ __device__ __forceinline__ void swiglu_bwd32(const float* dh, const bf16* g_src,
 template <int EPI, bool GROUP_K>
 __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, uint32_t t_row,
                                               int warp_r0, int col_half, int lane, int n_tile,
-                                              uint8_t* buf) {
+                                              uint8_t* buf, const CUtensorMap* tmC) {
     const int r = warp_r0 + lane;
     if (EPI == kEpiSwiglu) {
         // accumulator columns: gate [0, 128), up [128, 256); this warp: h columns
@@ -316,6 +316,37 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
                              dg, du);
             store_rows<32>(buf, p.out + row0 * p.ldo + col, p.ldo, nvalid, dg, lane);
             store_rows<32>(buf, p.out + row0 * p.ldo + p.I + col, p.ldo, nvalid, du, lane);
+        }
+    } else if (GROUP_K) {
+        // weight gradient: each warp stages 32 rows x 32 columns in shared
+        // memory and one lane stores the block into dW[g] with a TMA store;
+        // the tensor map drops rows past M and columns past N.
+        const int n0 = t.n_blk * n_tile;
+        const int m0 = t.m_blk * BM1 + warp_r0;
+#pragma unroll 1
+        for (int c0 = 128 * col_half; c0 < 128 * col_half + 128; c0 += 32) {
+            float v[32];
+            if (t.num_kb > 0) {
+                tmem_load_32(t_row + c0, v);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+            }
+            if (n0 + c0 >= p.N || m0 >= p.M) continue;
+            if (lane == 0) bulk_wait_group_read0();   // the previous block has left the buffer
+            __syncwarp();
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                *reinterpret_cast<uint4*>(buf + lane * 64 + q * 16) =
+                    make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                               pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_3d(tmC, buf, n0 + c0, m0, t.g);
+                bulk_commit_group();
+            }
+            __syncwarp();
         }
     } else {
         const int n0 = t.n_blk * n_tile;
@@ -501,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(&s.acc_full[buf], use & 1u, abort_flag, p.err)) break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-            epilogue_tile<EPI, false>(p, t, t_row, warp_r0, col_half, lane, BN, s.epi[warp - 2]);
+            epilogue_tile<EPI, false>(p, t, t_row, warp_r0, col_half, lane, BN, s.epi[warp - 2], nullptr);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_acc_empty[buf]);
@@ -520,7 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int EPI, bool A_MN, bool B_MN, bool GROUP_K>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_1cta_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const Params p) {
+                     const __grid_constant__ CUtensorMap tmC, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     Smem1& s = *reinterpret_cast<Smem1*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                          ~uintptr_t(1023));
@@ -647,14 +678,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // expert's data reaches this expert's gradient.
                         ksteps = (valid + 15) / 16;
                         const int nrows = ksteps * 16 - valid;
-                        for (int i = lane; i < nrows * 6 * 8; i += 32) {
-                            const int chunk = i / (nrows * 8);
-                            const int rem = i - chunk * nrows * 8;
-                            const int rr = valid + rem / 8, q = rem % 8;
-                            uint4* dst = reinterpret_cast<uint4*>(s.stage[stage] + chunk * kChunkBytes +
-                                                                  rr * 128) + q;
-                            *dst = make_uint4(0, 0, 0, 0);
-                        }
+                        // lane: 16-byte column (lane & 7) of rows valid + (lane >> 3), +4, ...
+                        // of each of the 6 chunks (A: 2, B: 4), 128 bytes per row
+                        const int q = lane & 7;
+#pragma unroll
+                        for (int chunk = 0; chunk < 6; ++chunk)
+                            for (int rr = valid + (lane >> 3); rr < valid + nrows; rr += 4)
+                                *(reinterpret_cast<uint4*>(s.stage[stage] + chunk * kChunkBytes + rr * 128) +
+                                  q) = make_uint4(0, 0, 0, 0);
                         if (nrows > 0) fence_proxy_async_smem();
                         __syncwarp();
                     }
@@ -703,10 +734,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(&s.acc_full[buf], use & 1u, abort_flag, p.err)) break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-            epilogue_tile<EPI, GROUP_K>(p, t, t_row, warp_r0, col_half, lane, BN, s.epi[warp - 2]);
+            epilogue_tile<EPI, GROUP_K>(p, t, t_row, warp_r0, col_half, lane, BN, s.epi[warp - 2], &tmC);
             tc_fence_before();
             mbar_arrive(&s.acc_empty[buf]);
         }
+        if (GROUP_K && lane == 0) bulk_wait_group0();   // this warp's TMA stores have completed
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -748,7 +781,8 @@ bool make_map_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer
 
 // 3-D bf16 tensor [d2][d1][d0], densely packed.
 bool make_map_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2,
-                 uint32_t box0, uint32_t box1) {
+                 uint32_t box0, uint32_t box1,
+                 CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {d0, d1, d2};
@@ -756,7 +790,7 @@ bool make_map_3d(CUtensorMap* m, const void* ptr, uint64_t d0, uint64_t d1, uint
     cuuint32_t box[3] = {box0, box1, 1};
     cuuint32_t es[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
-              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -796,7 +830,7 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const Params
 
 template <int EPI, bool A_MN, bool B_MN, bool GROUP_K>
 cudaError_t launch_1cta(const CUtensorMap& a, const CUtensorMap& b, const Params& p,
-                        int64_t max_tiles, cudaStream_t st) {
+                        int64_t max_tiles, cudaStream_t st, const CUtensorMap* c = nullptr) {
     auto kern = gemm_1cta_kernel<EPI, A_MN, B_MN, GROUP_K>;
     static std::once_flag once;
     static cudaError_t attr = cudaSuccess;
@@ -804,7 +838,8 @@ cudaError_t launch_1cta(const CUtensorMap& a, const CUtensorMap& b, const Params
     if (max_tiles <= 0) return cudaSuccess;
     int64_t grid = sm_count();
     if (grid > max_tiles) grid = max_tiles;
-    kern<<<(unsigned)grid, kThreads, kSmem1Bytes, st>>>(a, b, p);
+    CUtensorMap unused{};   // the output map is read only by the group-K epilogue
+    kern<<<(unsigned)grid, kThreads, kSmem1Bytes, st>>>(a, b, c ? *c : unused, p);
     return cudaGetLastError();
 }
 
@@ -947,8 +982,11 @@ cudaError_t gemm_wgrad(const bf16* X, const bf16* D, int64_t rows, const int32_t
     p.out = dW;
     p.ldo = N;
     p.out_group_stride = (int64_t)M * N;
+    CUtensorMap tc;   // dW [E][M][N], stored in 32 x 32 blocks without swizzle
+    if (!make_map_3d(&tc, dW, N, M, E > 0 ? E : 1, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
     return launch_1cta<kEpiStore, true, true, true>(ta, tb, p,
-                                                   (int64_t)E * p.m_blocks * p.n_blocks, st);
+                                                   (int64_t)E * p.m_blocks * p.n_blocks, st, &tc);
 }
 
 }  // namespace moe
