@@ -89,6 +89,7 @@ struct Params {
     const bf16* aux;           // SwiGLU backward: the saved [g | u]
     int64_t ld_aux;
     int I;                     // SwiGLU: offset of the up half in [g | u]
+    int tma_out, tma_out2;     // single-CTA kernel: out / out2 have TMA store maps
     unsigned* err;
 };
 
@@ -244,6 +245,35 @@ __device__ __forceinline__ void store_rows(uint8_t* buf, bf16* dst, int64_t ld, 
     __syncwarp();   // the buffer is free again
 }
 
+// Writes a 32 x 32 block (lane = row) of bf16 at dst. With an output tensor
+// map and all 32 rows valid, the block goes through the warp's buffer to one
+// TMA store (x, y = its first column and row in the map); otherwise through
+// store_rows, which masks rows >= nvalid. The buffer is reused only after the
+// previous TMA store has read it.
+__device__ __forceinline__ void put_block32(uint8_t* buf, bf16* dst, int64_t ld, int nvalid, const float* v,
+                                            int lane, const CUtensorMap* map, int x, int y) {
+    if (map != nullptr) {
+        if (lane == 0) bulk_wait_group_read0();
+        __syncwarp();
+    }
+    if (map != nullptr && nvalid == 32) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(buf + lane * 64 + q * 16) =
+                make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                           pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(map, buf, x, y);
+            bulk_commit_group();
+        }
+        __syncwarp();
+    } else {
+        store_rows<32>(buf, dst, ld, nvalid, v, lane);
+    }
+}
+
 // SwiGLU backward for 32 columns: dg, du from dh and the saved bf16 g, u.
 __device__ __forceinline__ void swiglu_bwd32(const float* dh, const bf16* g_src, const bf16* u_src,
                                              float* dg, float* du) {
@@ -277,7 +307,8 @@ __device__ __forceinline__ void swiglu_bwd32(const float* dh, const bf16* g_src,
 template <int EPI, bool GROUP_K>
 __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, uint32_t t_row,
                                               int warp_r0, int col_half, int lane, int n_tile,
-                                              uint8_t* buf, const CUtensorMap* tmC) {
+                                              uint8_t* buf, const CUtensorMap* tmC,
+                                              const CUtensorMap* tmC2) {
     const int r = warp_r0 + lane;
     if (EPI == kEpiSwiglu) {
         // accumulator columns: gate [0, 128), up [128, 256); this warp: h columns
@@ -291,12 +322,14 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
             tmem_load_2x32(t_row + c0, t_row + BN / 2 + c0, g, u);
             if (n0 + c0 >= p.N) continue;
             if (p.out2) {
-                store_rows<32>(buf, p.out2 + row0 * p.ldo2 + n0 + c0, p.ldo2, nvalid, g, lane);
-                store_rows<32>(buf, p.out2 + row0 * p.ldo2 + p.I + n0 + c0, p.ldo2, nvalid, u, lane);
+                put_block32(buf, p.out2 + row0 * p.ldo2 + n0 + c0, p.ldo2, nvalid, g, lane, tmC2, n0 + c0,
+                            (int)row0);
+                put_block32(buf, p.out2 + row0 * p.ldo2 + p.I + n0 + c0, p.ldo2, nvalid, u, lane, tmC2,
+                            p.I + n0 + c0, (int)row0);
             }
 #pragma unroll
             for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i]) * u[i];     // h, in place
-            store_rows<32>(buf, p.out + row0 * p.ldo + n0 + c0, p.ldo, nvalid, g, lane);
+            put_block32(buf, p.out + row0 * p.ldo + n0 + c0, p.ldo, nvalid, g, lane, tmC, n0 + c0, (int)row0);
         }
     } else if (EPI == kEpiSwigluBwd) {
         const int n0 = t.n_blk * n_tile;
@@ -314,8 +347,9 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
             if (valid)
                 swiglu_bwd32(dh, p.aux + grow * p.ld_aux + col, p.aux + grow * p.ld_aux + p.I + col,
                              dg, du);
-            store_rows<32>(buf, p.out + row0 * p.ldo + col, p.ldo, nvalid, dg, lane);
-            store_rows<32>(buf, p.out + row0 * p.ldo + p.I + col, p.ldo, nvalid, du, lane);
+            put_block32(buf, p.out + row0 * p.ldo + col, p.ldo, nvalid, dg, lane, tmC, col, (int)row0);
+            put_block32(buf, p.out + row0 * p.ldo + p.I + col, p.ldo, nvalid, du, lane, tmC, p.I + col,
+                        (int)row0);
         }
     } else if (GROUP_K) {
         // weight gradient: each warp stages 32 rows x 32 columns in shared
@@ -373,7 +407,8 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 if (n0 + c0 + 32 * half >= p.N) continue;
-                store_rows<32>(buf, row0 + n0 + c0 + 32 * half, p.ldo, nvalid, v + 32 * half, lane);
+                put_block32(buf, row0 + n0 + c0 + 32 * half, p.ldo, nvalid, v + 32 * half, lane,
+                            GROUP_K ? nullptr : tmC, n0 + c0 + 32 * half, t.row0 + warp_r0);
             }
         }
     }
@@ -532,7 +567,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(&s.acc_full[buf], use & 1u, abort_flag, p.err)) break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-            epilogue_tile<EPI, false>(p, t, t_row, warp_r0, col_half, lane, BN, s.epi[warp - 2], nullptr);
+            epilogue_tile<EPI, false>(p, t, t_row, warp_r0, col_half, lane, BN, s.epi[warp - 2], nullptr,
+                                      nullptr);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_acc_empty[buf]);
@@ -551,7 +587,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int EPI, bool A_MN, bool B_MN, bool GROUP_K>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_1cta_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmC, const Params p) {
+                     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
+                     const Params p) {
     extern __shared__ uint8_t smem_raw[];
     Smem1& s = *reinterpret_cast<Smem1*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                          ~uintptr_t(1023));
@@ -734,11 +771,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(&s.acc_full[buf], use & 1u, abort_flag, p.err)) break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-            epilogue_tile<EPI, GROUP_K>(p, t, t_row, warp_r0, col_half, lane, BN, s.epi[warp - 2], &tmC);
+            epilogue_tile<EPI, GROUP_K>(p, t, t_row, warp_r0, col_half, lane, BN, s.epi[warp - 2],
+                                        p.tma_out ? &tmC : nullptr, p.tma_out2 ? &tmC2 : nullptr);
             tc_fence_before();
             mbar_arrive(&s.acc_empty[buf]);
         }
-        if (GROUP_K && lane == 0) bulk_wait_group0();   // this warp's TMA stores have completed
+        if (lane == 0) bulk_wait_group0();   // this warp's TMA stores have completed
         __syncwarp();
     }
 
@@ -767,7 +805,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // 2-D bf16 tensor [outer][inner] with row pitch `pitch` elements.
 bool make_map_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t pitch,
-                 uint32_t box_inner, uint32_t box_outer) {
+                 uint32_t box_inner, uint32_t box_outer,
+                 CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[2] = {inner, outer};
@@ -775,7 +814,7 @@ bool make_map_2d(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t es[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
-              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -830,7 +869,8 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const Params
 
 template <int EPI, bool A_MN, bool B_MN, bool GROUP_K>
 cudaError_t launch_1cta(const CUtensorMap& a, const CUtensorMap& b, const Params& p,
-                        int64_t max_tiles, cudaStream_t st, const CUtensorMap* c = nullptr) {
+                        int64_t max_tiles, cudaStream_t st, const CUtensorMap* c = nullptr,
+                        const CUtensorMap* c2 = nullptr) {
     auto kern = gemm_1cta_kernel<EPI, A_MN, B_MN, GROUP_K>;
     static std::once_flag once;
     static cudaError_t attr = cudaSuccess;
@@ -838,8 +878,11 @@ cudaError_t launch_1cta(const CUtensorMap& a, const CUtensorMap& b, const Params
     if (max_tiles <= 0) return cudaSuccess;
     int64_t grid = sm_count();
     if (grid > max_tiles) grid = max_tiles;
-    CUtensorMap unused{};   // the output map is read only by the group-K epilogue
-    kern<<<(unsigned)grid, kThreads, kSmem1Bytes, st>>>(a, b, c ? *c : unused, p);
+    CUtensorMap unused{};   // read only when p.tma_out / p.tma_out2 say so
+    Params q = p;
+    q.tma_out = c != nullptr;
+    q.tma_out2 = c2 != nullptr;
+    kern<<<(unsigned)grid, kThreads, kSmem1Bytes, st>>>(a, b, c ? *c : unused, c2 ? *c2 : unused, q);
     return cudaGetLastError();
 }
 
@@ -878,11 +921,18 @@ bool use_pair_tiles(int64_t rows, int groups) {
 // maps for each (their K-major boxes differ: 128 or 256 rows of N).
 template <int EPI, bool B_MN>
 cudaError_t launch_group_m(const CUtensorMap& ta, const CUtensorMap& tb_pair,
-                           const CUtensorMap& tb_single, const Params& p, cudaStream_t st) {
+                           const CUtensorMap& tb_single, const Params& p, cudaStream_t st,
+                           const CUtensorMap* out_map, const CUtensorMap* out2_map = nullptr) {
     if (use_pair_tiles(p.rows, p.groups))
         return launch_pair<EPI, B_MN>(ta, tb_pair, p, pair_tile_bound(p.rows, p.groups, p.n_blocks), st);
     return launch_1cta<EPI, false, B_MN, false>(ta, tb_single, p,
-                                                single_tile_bound(p.rows, p.groups, p.n_blocks), st);
+                                                single_tile_bound(p.rows, p.groups, p.n_blocks), st,
+                                                out_map, out2_map);
+}
+
+// TMA store map of a row-major bf16 output [rows][cols]: 32 x 32 blocks, no swizzle.
+bool make_out_map(CUtensorMap* m, const bf16* out, int64_t rows, uint64_t cols) {
+    return make_map_2d(m, out, cols, (uint64_t)rows, cols, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 }  // namespace
@@ -905,7 +955,10 @@ cudaError_t gemm_gate_up_swiglu(const bf16* x, int64_t rows, const int32_t* offs
     p.ldo = I;
     p.out2 = gu_save;
     p.ldo2 = 2 * (int64_t)I;
-    return launch_group_m<kEpiSwiglu, true>(ta, tb, tb, p, st);
+    CUtensorMap tc, tc2;
+    if (!make_out_map(&tc, h, rows, I)) return cudaErrorInvalidValue;
+    if (gu_save && !make_out_map(&tc2, gu_save, rows, 2 * (uint64_t)I)) return cudaErrorInvalidValue;
+    return launch_group_m<kEpiSwiglu, true>(ta, tb, tb, p, st, &tc, gu_save ? &tc2 : nullptr);
 }
 
 cudaError_t gemm_down(const bf16* h, int64_t rows, const int32_t* offsets, int E, int H, int I,
@@ -921,7 +974,9 @@ cudaError_t gemm_down(const bf16* h, int64_t rows, const int32_t* offsets, int E
     p.n_blocks = (H + BN - 1) / BN;
     p.out = y;
     p.ldo = H;
-    return launch_group_m<kEpiStore, true>(ta, tb, tb, p, st);
+    CUtensorMap tc;
+    if (!make_out_map(&tc, y, rows, H)) return cudaErrorInvalidValue;
+    return launch_group_m<kEpiStore, true>(ta, tb, tb, p, st, &tc);
 }
 
 cudaError_t gemm_down_dgrad_swiglu(const bf16* dy, int64_t rows, const int32_t* offsets, int E,
@@ -944,7 +999,9 @@ cudaError_t gemm_down_dgrad_swiglu(const bf16* dy, int64_t rows, const int32_t* 
     p.ldo = 2 * (int64_t)I;
     p.aux = gu;
     p.ld_aux = 2 * (int64_t)I;
-    return launch_group_m<kEpiSwigluBwd, false>(ta, tb, tb1, p, st);
+    CUtensorMap tc;
+    if (!make_out_map(&tc, dgu, rows, 2 * (uint64_t)I)) return cudaErrorInvalidValue;
+    return launch_group_m<kEpiSwigluBwd, false>(ta, tb, tb1, p, st, &tc);
 }
 
 cudaError_t gemm_gate_up_dgrad(const bf16* dgu, int64_t rows, const int32_t* offsets, int E, int H,
@@ -965,7 +1022,9 @@ cudaError_t gemm_gate_up_dgrad(const bf16* dgu, int64_t rows, const int32_t* off
     p.n_blocks = (H + BN - 1) / BN;
     p.out = dx_perm;
     p.ldo = H;
-    return launch_group_m<kEpiStore, false>(ta, tb, tb1, p, st);
+    CUtensorMap tc;
+    if (!make_out_map(&tc, dx_perm, rows, H)) return cudaErrorInvalidValue;
+    return launch_group_m<kEpiStore, false>(ta, tb, tb1, p, st, &tc);
 }
 
 cudaError_t gemm_wgrad(const bf16* X, const bf16* D, int64_t rows, const int32_t* offsets, int E,
