@@ -9,7 +9,7 @@
 // (_expert_ffn) and torchtitan GroupedExperts: silu(x Wg) * (x Wu).
 //
 // Two kernels share the schedule and the epilogues. The forward and dgrad
-// GEMMs run on pair tiles when the average expert block is large (>= 2048 rows,
+// GEMMs run on pair tiles when the average expert block is large (>= 1024 rows,
 // or a single dense group), else on single-CTA 128-row tiles, which round
 // ragged blocks up less (use_pair_tiles).
 //
@@ -418,6 +418,7 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
 template <int EPI, bool B_MN>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
                      const Params p) {
     extern __shared__ uint8_t smem_raw[];
     SmemP& s = *reinterpret_cast<SmemP*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -567,12 +568,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(&s.acc_full[buf], use & 1u, abort_flag, p.err)) break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-            epilogue_tile<EPI, false>(p, t, t_row, warp_r0, col_half, lane, BN, s.epi[warp - 2], nullptr,
-                                      nullptr);
+            epilogue_tile<EPI, false>(p, t, t_row, warp_r0, col_half, lane, BN, s.epi[warp - 2],
+                                      p.tma_out ? &tmC : nullptr, p.tma_out2 ? &tmC2 : nullptr);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_acc_empty[buf]);
         }
+        if (lane == 0) bulk_wait_group0();   // this warp's TMA stores have completed
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -843,7 +846,8 @@ cudaError_t set_smem_once(K kern, size_t bytes, std::once_flag& once, cudaError_
 
 template <int EPI, bool B_MN>
 cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const Params& p,
-                        int64_t max_tiles, cudaStream_t st) {
+                        int64_t max_tiles, cudaStream_t st, const CUtensorMap* c = nullptr,
+                        const CUtensorMap* c2 = nullptr) {
     auto kern = gemm_pair_kernel<EPI, B_MN>;
     static std::once_flag once;
     static cudaError_t attr = cudaSuccess;
@@ -864,7 +868,11 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const Params
     attrs[0].val.clusterDim.z = 1;
     cfg.attrs = attrs;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, a, b, p);
+    CUtensorMap unused{};   // read only when q.tma_out / q.tma_out2 say so
+    Params q = p;
+    q.tma_out = c != nullptr;
+    q.tma_out2 = c2 != nullptr;
+    return cudaLaunchKernelEx(&cfg, kern, a, b, c ? *c : unused, c2 ? *c2 : unused, q);
 }
 
 template <int EPI, bool A_MN, bool B_MN, bool GROUP_K>
@@ -907,14 +915,16 @@ int64_t single_tile_bound(int64_t rows, int groups, int n_blocks) {
 // Pair tiles (256 rows) halve each CTA's weight traffic but round every
 // expert block up to 256 rows; single tiles round up to 128. The expected
 // rounding waste is about half a tile per expert, so pair tiles pay off once
-// the average block is large compared with a tile.
+// the average block is large compared with a tile: measured on B200, they were
+// faster at 1024 rows per expert (Mixtral-8x7B shape) and slower at 256
+// (Qwen3-30B-A3B shape).
 // MOE_GEMM_TILES=pair|single overrides the choice (used by the tests to run
 // both kernels on the same shapes).
 bool use_pair_tiles(int64_t rows, int groups) {
     const char* force = getenv("MOE_GEMM_TILES");
     if (force && force[0] == 'p') return true;
     if (force && force[0] == 's') return false;
-    return groups == 1 || rows >= (int64_t)groups * 2048;
+    return groups == 1 || rows >= (int64_t)groups * 1024;
 }
 
 // Group-M GEMM on pair or single tiles. `tb_pair` and `tb_single` are the B
@@ -924,7 +934,8 @@ cudaError_t launch_group_m(const CUtensorMap& ta, const CUtensorMap& tb_pair,
                            const CUtensorMap& tb_single, const Params& p, cudaStream_t st,
                            const CUtensorMap* out_map, const CUtensorMap* out2_map = nullptr) {
     if (use_pair_tiles(p.rows, p.groups))
-        return launch_pair<EPI, B_MN>(ta, tb_pair, p, pair_tile_bound(p.rows, p.groups, p.n_blocks), st);
+        return launch_pair<EPI, B_MN>(ta, tb_pair, p, pair_tile_bound(p.rows, p.groups, p.n_blocks), st,
+                                      out_map, out2_map);
     return launch_1cta<EPI, false, B_MN, false>(ta, tb_single, p,
                                                 single_tile_bound(p.rows, p.groups, p.n_blocks), st,
                                                 out_map, out2_map);
