@@ -473,24 +473,40 @@ def router_sweep(m, hbm):
 
 
 def e2e_measure(args, w, d, m, opts, ws, world):
-    """Same metric through the public call with host buffers: every step
-    copies its inputs (logits, x) from pinned host memory to the device and
-    reads the layer output back, inside the timed region."""
+    """Same metric through the public calls with host buffers: every step
+    copies its inputs (logits, x, and dout for a training step) from pinned
+    host memory to the device and reads the step's result back (the layer
+    output, or dx for a training step), inside the timed region."""
     import torch
     h_logits = d["logits"].cpu().pin_memory()
     h_x = d["x"].cpu().pin_memory()
-    h_out = torch.empty((w.T, w.H), dtype=torch.bfloat16).pin_memory()
+    h_dout = d["dout"].cpu().pin_memory() if w.backward else None
+    h_res = torch.empty((w.T, w.H), dtype=torch.bfloat16).pin_memory()
     dl = torch.empty_like(d["logits"])
     dx = torch.empty_like(d["x"])
+    ddo = torch.empty_like(d["dout"]) if w.backward else None
     out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device="cuda")
     K = max(1, min(args.steps, 50))
+    state = None
+    grads = None
+    if w.backward:
+        _, state = m.moe_layer_forward(d["logits"], d["x"], d["w_gate_up"], d["w_down"], w.k, opts,
+                                       save_for_backward=True, workspace=ws, out=out)
+        grads = m.moe_grouped_mlp_backward(d["dout"], state, d["w_gate_up"], d["w_down"], ws)
 
     def step():
         dl.copy_(h_logits, non_blocking=True)
         dx.copy_(h_x, non_blocking=True)
+        if w.backward:
+            ddo.copy_(h_dout, non_blocking=True)
         m.moe_layer_forward(dl, dx, d["w_gate_up"], d["w_down"], w.k, opts, d["shared_gate_up"],
-                            d["shared_down"], workspace=ws, out=out)
-        h_out.copy_(out, non_blocking=True)
+                            d["shared_down"], save_for_backward=w.backward, workspace=ws, out=out,
+                            state=state)
+        if w.backward:
+            m.moe_grouped_mlp_backward(ddo, state, d["w_gate_up"], d["w_down"], ws, grads)
+            h_res.copy_(grads["dx"], non_blocking=True)
+        else:
+            h_res.copy_(out, non_blocking=True)
 
     for _ in range(2):
         step()
@@ -503,10 +519,12 @@ def e2e_measure(args, w, d, m, opts, ws, world):
     e.record()
     torch.cuda.synchronize()
     ms = max_over_ranks(s.elapsed_time(e), world)
+    h2d = h_logits.numel() * 4 + h_x.numel() * 2 + (h_dout.numel() * 2 if w.backward else 0)
     return {"value": w.T * world * K / (ms / 1e3), "unit": UNIT,
-            "h2d_bytes_per_step": h_logits.numel() * 4 + h_x.numel() * 2,
-            "d2h_bytes_per_step": h_out.numel() * 2, "steps": K,
-            "pass": "fwd", "note": "weights resident on the device"}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h_res.numel() * 2, "steps": K,
+            "pass": "fwd+bwd" if w.backward else "fwd",
+            "note": "weights resident on the device; the step's result read back is "
+                    + ("dx" if w.backward else "the layer output")}
 
 
 def main():

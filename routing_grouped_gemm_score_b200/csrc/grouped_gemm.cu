@@ -288,8 +288,10 @@ __device__ __forceinline__ void swiglu_bwd32(const float* dh, const bf16* g_src,
             const float2 gf = unpack_bf16x2(gw[i]);
             const float2 uf = unpack_bf16x2(uw[i]);
             const int c = 8 * q + 2 * i;
-            const float s0 = 1.0f / (1.0f + expf(-gf.x));
-            const float s1 = 1.0f / (1.0f + expf(-gf.y));
+            // 1/x rounded once: the correctly rounded reciprocal, the same value
+            // as the IEEE division 1.0f / x
+            const float s0 = __frcp_rn(1.0f + expf(-gf.x));
+            const float s1 = __frcp_rn(1.0f + expf(-gf.y));
             du[c] = dh[c] * gf.x * s0;
             du[c + 1] = dh[c + 1] * gf.y * s1;
             dg[c] = dh[c] * uf.x * (s0 + gf.x * s0 * (1.0f - s0));
