@@ -98,6 +98,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
+// Waits for the phase with the given parity for at most kWaitLimitNs,
+// whatever the abort flag says (used at exit, for copies still in flight).
+// Records kErrTimeout if it gives up.
+__device__ __forceinline__ void mbar_wait_bounded(uint64_t* bar, uint32_t parity, unsigned* err) {
+    if (mbar_try_wait(bar, parity)) return;
+    const unsigned long long start = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_timer_ns() - start > kWaitLimitNs) {
+            raise_error(err, kErrTimeout);
+            return;
+        }
+    }
+}
+
 // TMA tiled loads into shared memory, completing on an mbarrier.
 __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* dst,
                                             int x, int y) {

@@ -112,11 +112,41 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
     }
 }
 
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or about `ns` nanoseconds pass, instead of polling.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait that sleeps between checks (see mbar_wait for the bounds).
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                unsigned* err) {
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    const unsigned long long start = global_timer_ns();
+    for (;;) {
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+        if (*abort) return false;
+        if (global_timer_ns() - start > kWaitLimitNs) {
+            raise_error(err, kErrTimeout);
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
 // One lane waits (bounded), the warp follows its verdict.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           unsigned* err, int lane) {
     bool ok = true;
-    if (lane == 0) ok = mbar_wait(bar, parity, abort, err);
+    if (lane == 0) ok = mbar_wait_sleep(bar, parity, abort, err);
     ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
     __syncwarp();
     return ok;

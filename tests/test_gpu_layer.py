@@ -44,6 +44,9 @@ SMALL = {
     "skew_small": wl.WORKLOADS["skew_t64"].scaled(H=256, I=192),
     "tie_small": wl.WORKLOADS["tie_t64"].scaled(H=128, I=128),
     "mixtral_small": wl.WORKLOADS["mixtral_8x7b"].scaled(T=512, H=512, I=512),
+    # about 1000 rows per expert: the weight gradient streams B instead of
+    # keeping each expert's rows in shared memory (more than 320 rows)
+    "long_k": wl.WORKLOADS["mixtral_8x7b"].scaled(T=2048, H=256, I=192, E=4),
 }
 
 
@@ -74,7 +77,7 @@ def test_layer_forward_saved_state_and_empty_batch():
     assert empty.shape == (0, w.H)
 
 
-BWD = ["tiny", "qwen3_small", "skew_small", "mixtral_small"]
+BWD = ["tiny", "qwen3_small", "skew_small", "mixtral_small", "long_k"]
 
 
 def _oracle_backward(w, d, r):
@@ -82,9 +85,10 @@ def _oracle_backward(w, d, r):
                                bits(d["w_down"]), bits(d["dout"]))
 
 
+@pytest.mark.parametrize("wgrad", ["panel", "tiles"])
 @pytest.mark.parametrize("tiles", ["single", "pair"])
 @pytest.mark.parametrize("name", BWD)
-def test_backward_on_oracle_state(name, tiles, monkeypatch):
+def test_backward_on_oracle_state(name, tiles, wgrad, monkeypatch):
     """The backward kernels fed with the oracle's own saved forward state, so
     both sides read identical bf16 inputs. dW_down and dprob then differ only
     in accumulation order; dW_gate_up and dx also carry the bf16 rounding of
@@ -92,6 +96,7 @@ def test_backward_on_oracle_state(name, tiles, monkeypatch):
     apart (assert_close_flips)."""
     import routing_grouped_gemm_score_b200 as m
     monkeypatch.setenv("MOE_GEMM_TILES", tiles)
+    monkeypatch.setenv("MOE_WGRAD", wgrad)   # weight gradient: shared-memory B panel, or one tile per CTA
     w = SMALL[name]
     d = wl.make_inputs(w, "cuda", with_dout=True)
     r = oracle.router_topk(d["logits"].cpu().numpy(), w.k)
