@@ -277,15 +277,74 @@ __device__ __forceinline__ void put_block32(uint8_t* buf, bf16* dst, int64_t ld,
     }
 }
 
-// SwiGLU backward for 32 columns: dg, du from dh and the saved bf16 g, u.
-__device__ __forceinline__ void swiglu_bwd32(const float* dh, const bf16* g_src, const bf16* u_src,
-                                             float* dg, float* du) {
+// The saved bf16 g and u of one row for 32 columns (16-byte vectors).
+struct Aux32 {
+    uint4 g[4], u[4];
+};
+
+// Loads a row's g and u for columns [col, col + 32) of the saved [g | u];
+// does nothing when !ok. Issued a chunk ahead of use so that the loads'
+// latency overlaps other work.
+__device__ __forceinline__ void load_aux32(const Params& p, int64_t grow, int col, bool ok, Aux32& a) {
+    if (!ok) return;
+    const uint4* gs = reinterpret_cast<const uint4*>(p.aux + grow * p.ld_aux + col);
+    const uint4* us = reinterpret_cast<const uint4*>(p.aux + grow * p.ld_aux + p.I + col);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        const uint4 gv = *reinterpret_cast<const uint4*>(g_src + 8 * q);
-        const uint4 uv = *reinterpret_cast<const uint4*>(u_src + 8 * q);
-        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
-        const uint32_t uw[4] = {uv.x, uv.y, uv.z, uv.w};
+        a.g[q] = __ldg(gs + q);
+        a.u[q] = __ldg(us + q);
+    }
+}
+
+// store_rows<32> for values already packed as bf16 pairs (16 per lane).
+__device__ __forceinline__ void store_rows_packed32(uint8_t* buf, bf16* dst, int64_t ld, int nvalid,
+                                                    const uint32_t* w, int lane) {
+    constexpr int kPitch = 32 * 2 + 16;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4*>(buf + lane * kPitch + q * 16) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+    __syncwarp();
+    const int chunk = lane % 4;
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass) {
+        const int row = pass * 8 + lane / 4;
+        const uint4 v = *reinterpret_cast<const uint4*>(buf + row * kPitch + chunk * 16);
+        if (row < nvalid) *reinterpret_cast<uint4*>(dst + (int64_t)row * ld + chunk * 8) = v;
+    }
+    __syncwarp();
+}
+
+// put_block32 for values already packed as bf16 pairs.
+__device__ __forceinline__ void put_block32_packed(uint8_t* buf, bf16* dst, int64_t ld, int nvalid,
+                                                   const uint32_t* w, int lane, const CUtensorMap* map, int x,
+                                                   int y) {
+    if (map != nullptr) {
+        if (lane == 0) bulk_wait_group_read0();
+        __syncwarp();
+    }
+    if (map != nullptr && nvalid == 32) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(buf + lane * 64 + q * 16) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(map, buf, x, y);
+            bulk_commit_group();
+        }
+        __syncwarp();
+    } else {
+        store_rows_packed32(buf, dst, ld, nvalid, w, lane);
+    }
+}
+
+// SwiGLU backward for 32 columns: from dh and the saved g, u, the bf16 dg and
+// du, packed in pairs (dg in dgp, du in dup).
+__device__ __forceinline__ void swiglu_bwd32(const float* dh, const Aux32& a, uint32_t* dgp, uint32_t* dup) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint32_t gw[4] = {a.g[q].x, a.g[q].y, a.g[q].z, a.g[q].w};
+        const uint32_t uw[4] = {a.u[q].x, a.u[q].y, a.u[q].z, a.u[q].w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const float2 gf = unpack_bf16x2(gw[i]);
@@ -295,10 +354,9 @@ __device__ __forceinline__ void swiglu_bwd32(const float* dh, const bf16* g_src,
             // as the IEEE division 1.0f / x
             const float s0 = __frcp_rn(1.0f + expf(-gf.x));
             const float s1 = __frcp_rn(1.0f + expf(-gf.y));
-            du[c] = dh[c] * gf.x * s0;
-            du[c + 1] = dh[c + 1] * gf.y * s1;
-            dg[c] = dh[c] * uf.x * (s0 + gf.x * s0 * (1.0f - s0));
-            dg[c + 1] = dh[c + 1] * uf.y * (s1 + gf.y * s1 * (1.0f - s1));
+            dup[c / 2] = pack_bf16x2(dh[c] * gf.x * s0, dh[c + 1] * gf.y * s1);
+            dgp[c / 2] = pack_bf16x2(dh[c] * uf.x * (s0 + gf.x * s0 * (1.0f - s0)),
+                                     dh[c + 1] * uf.y * (s1 + gf.y * s1 * (1.0f - s1)));
         }
     }
 }
@@ -313,7 +371,7 @@ template <int EPI, bool GROUP_K>
 __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, uint32_t t_row,
                                               int warp_r0, int col_half, int lane, int n_tile,
                                               uint8_t* buf, const CUtensorMap* tmC,
-                                              const CUtensorMap* tmC2) {
+                                              const CUtensorMap* tmC2, Aux32* pre) {
     const int r = warp_r0 + lane;
     if (EPI == kEpiSwiglu) {
         // accumulator columns: gate [0, 128), up [128, 256); this warp: h columns
@@ -337,24 +395,32 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
             put_block32(buf, p.out + row0 * p.ldo + n0 + c0, p.ldo, nvalid, g, lane, tmC, n0 + c0, (int)row0);
         }
     } else if (EPI == kEpiSwigluBwd) {
+        // the first chunk's g and u were loaded before the accumulator was
+        // ready (`pre`); each later chunk's load while the one before is stored
         const int n0 = t.n_blk * n_tile;
         const bool valid = r < t.rows;
         const int nvalid = min(max(t.rows - warp_r0, 0), 32);
         const int64_t grow = (int64_t)t.row0 + r;
         const int64_t row0 = (int64_t)t.row0 + warp_r0;
+        Aux32& ax = *pre;   // reloaded in place for each later chunk
 #pragma unroll 1
         for (int c0 = 128 * col_half; c0 < 128 * col_half + 128; c0 += 32) {
+            const int col = n0 + c0;
             float dh[32];
             tmem_load_32(t_row + c0, dh);
-            const int col = n0 + c0;
             if (col >= p.N) continue;
-            float dg[32], du[32];
-            if (valid)
-                swiglu_bwd32(dh, p.aux + grow * p.ld_aux + col, p.aux + grow * p.ld_aux + p.I + col,
-                             dg, du);
-            put_block32(buf, p.out + row0 * p.ldo + col, p.ldo, nvalid, dg, lane, tmC, col, (int)row0);
-            put_block32(buf, p.out + row0 * p.ldo + p.I + col, p.ldo, nvalid, du, lane, tmC, p.I + col,
-                        (int)row0);
+            uint32_t dgp[16], dup[16];
+            if (valid) {
+                swiglu_bwd32(dh, ax, dgp, dup);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) dgp[i] = dup[i] = 0u;   // rows past the block: not stored
+            }
+            // the next chunk's g and u load while this chunk is stored
+            load_aux32(p, grow, col + 32, valid && c0 + 32 < 128 * col_half + 128 && col + 32 < p.N, ax);
+            put_block32_packed(buf, p.out + row0 * p.ldo + col, p.ldo, nvalid, dgp, lane, tmC, col, (int)row0);
+            put_block32_packed(buf, p.out + row0 * p.ldo + p.I + col, p.ldo, nvalid, dup, lane, tmC, p.I + col,
+                               (int)row0);
         }
     } else if (GROUP_K) {
         // weight gradient: each warp stages 32 rows x 32 columns in shared
@@ -570,11 +636,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const Tile t = decode_tile<false>(s, p, id, BMP);
             const int buf = local_tile & 1;
             const uint32_t use = (uint32_t)(local_tile >> 1);
+            Aux32 pre;
+            if (EPI == kEpiSwigluBwd) {
+                const int col = t.n_blk * BN + 128 * col_half;
+                load_aux32(p, (int64_t)t.row0 + warp_r0 + lane, col, warp_r0 + lane < t.rows && col < p.N, pre);
+            }
             if (!mbar_wait(&s.acc_full[buf], use & 1u, abort_flag, p.err)) break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
             epilogue_tile<EPI, false>(p, t, t_row, warp_r0, col_half, lane, BN, s.epi[warp - 2],
-                                      p.tma_out ? &tmC : nullptr, p.tma_out2 ? &tmC2 : nullptr);
+                                      p.tma_out ? &tmC : nullptr, p.tma_out2 ? &tmC2 : nullptr, &pre);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(leader_acc_empty[buf]);
@@ -764,11 +835,16 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
             const Tile t = decode_tile<GROUP_K>(s, p, id, BM1);
             const int buf = local_tile & 1;
             const uint32_t use = (uint32_t)(local_tile >> 1);
+            Aux32 pre;
+            if (EPI == kEpiSwigluBwd) {
+                const int col = t.n_blk * BN + 128 * col_half;
+                load_aux32(p, (int64_t)t.row0 + warp_r0 + lane, col, warp_r0 + lane < t.rows && col < p.N, pre);
+            }
             if (!mbar_wait(&s.acc_full[buf], use & 1u, abort_flag, p.err)) break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
             epilogue_tile<EPI, GROUP_K>(p, t, t_row, warp_r0, col_half, lane, BN, s.epi[warp - 2],
-                                        p.tma_out ? &tmC : nullptr, p.tma_out2 ? &tmC2 : nullptr);
+                                        p.tma_out ? &tmC : nullptr, p.tma_out2 ? &tmC2 : nullptr, &pre);
             tc_fence_before();
             mbar_arrive(&s.acc_empty[buf]);
         }
