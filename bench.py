@@ -51,6 +51,7 @@ def parse():
     ap.add_argument("--T", type=int, default=None,
                     help="override the token count (small cases for profiling)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--router-sweep", action="store_true",
                     help="also time the router alone at E=128, k=8, T = 2^16 .. 2^20")
@@ -352,6 +353,8 @@ def our_arm(args, world, rank, local):
                       "down_wgrad", "gate_up_wgrad"]
         stages.update({f"bwd_{n}": stage_ms(bevs, i) for i, n in enumerate(bwd_stages)})
 
+    graph = None if args.no_graph else graph_measure(args, step, w, world, m)
+
     tokens_total = w.T * world
     value = tokens_total * K / (ms_max / 1e3)
     peaks, peaks_src = load_peaks()
@@ -415,6 +418,8 @@ def our_arm(args, world, rank, local):
         "clocks": clocks,
     }
 
+    if graph:
+        line["cuda_graph"] = graph
     if not args.no_e2e:
         line["e2e"] = e2e_measure(args, w, d, m, opts, ws, world)
     if args.router_sweep:
@@ -470,6 +475,39 @@ def router_sweep(m, hbm):
         out.append({"T": T, "E": E, "k": k, "us": ms * 1e3, "GB/s": gbs, "frac_of_hbm": gbs / hbm})
         del logits, res, ws
     return out
+
+
+def graph_measure(args, step, w, world, m):
+    """The same step captured once in a CUDA graph and replayed: the device
+    time without per-launch host overhead (the calls allocate nothing and
+    never sync, so a whole step captures as is)."""
+    import torch
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    K = max(1, min(args.steps, 100))
+    barrier(world)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(K):
+        g.replay()
+    end.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(start.elapsed_time(end), world)
+    if m.moe_get_device_status() != 0:
+        raise RuntimeError("device status error in the graph replays")
+    del g
+    return {"value": w.T * world * K / (ms / 1e3), "unit": UNIT, "ms_per_step": ms / K, "steps": K,
+            "note": "one step captured in a CUDA graph, replayed back to back"}
 
 
 def e2e_measure(args, w, d, m, opts, ws, world):
