@@ -54,6 +54,8 @@ def _load():
             lib.oracle_round_bf16_array.restype = None
             lib.oracle_router_topk.argtypes = [P, i64, i32, i32, i32, i32, f32, P, P, P, P, P, P]
             lib.oracle_router_topk.restype = i32
+            lib.oracle_router_backward.argtypes = [P, i64, i32, i32, i32, i32, f32, P, P, P]
+            lib.oracle_router_backward.restype = i32
             lib.oracle_dispatch.argtypes = [P, i64, i32, i32, P, P, P]
             lib.oracle_dispatch.restype = i32
             lib.oracle_gather_rows.argtypes = [P, i32, P, i64, P]
@@ -121,6 +123,23 @@ def router_topk(logits, k, score=0, renormalize=True, scaling=1.0, expert_bias=N
     if rc:
         raise ValueError(f"oracle_router_topk rejected its arguments ({rc})")
     return dict(topk_idx=idx, topk_prob=prob, routing_map=rmap, counts=counts, offsets=offsets)
+
+
+def router_backward(logits, topk_idx, dprob, score=0, renormalize=True, scaling=1.0):
+    """dL/dlogits [T,E] (fp32) from dL/dtopk_prob, for the experts in topk_idx
+    (oracle_router_backward; fp64 inside)."""
+    lib = _load()
+    logits = _c(logits, np.float32)
+    topk_idx = _c(topk_idx, np.int32)
+    dprob = _c(dprob, np.float32)
+    T, E = logits.shape
+    k = topk_idx.shape[1]
+    dl = np.zeros((T, E), np.float32)
+    rc = lib.oracle_router_backward(_p(logits), T, E, k, score, int(renormalize), scaling, _p(topk_idx),
+                                    _p(dprob), _p(dl))
+    if rc:
+        raise ValueError(f"oracle_router_backward: invalid index ({rc})")
+    return dl
 
 
 def dispatch(topk_idx, offsets, E):

@@ -190,6 +190,69 @@ int oracle_router_topk(const float* logits, int64_t T, int E, int k, int score_f
     return 0;
 }
 
+/*
+ * oracle_router_backward -- [TE] Router: the gradient of the loss with
+ * respect to the logits, given dprob = dL/dp for the routing weights p[t,j]
+ * of the experts that oracle_router_topk chose (topk_idx). The selection is
+ * piecewise constant in the logits, so it contributes no gradient. With
+ * g_j = scaling * dprob[t,j] (p = scaling * q), in fp64:
+ *   softmax, renormalize=1: q_j = exp(l_j) / sum_{i in sel} exp(l_i);
+ *       dl[sel_j] = q_j (g_j - sum_i q_i g_i), 0 for experts not chosen.
+ *   softmax, renormalize=0: q_e = exp(l_e) / sum_{all e'} exp(l_e');
+ *       dl[e] = q_e (G_e - sum_j q_{sel_j} g_j), G_e = g_j if e = sel_j else 0.
+ *   sigmoid, renormalize=0: dl[sel_j] = g_j s_j (1 - s_j), s = sigmoid(l).
+ *   sigmoid, renormalize=1: r_j = s_j / S, S = sum_j s_j;
+ *       dl[sel_j] = ((g_j - sum_i r_i g_i) / S) s_j (1 - s_j).
+ * An expert bias only moves the selection, so it does not appear here.
+ * Writes dlogits[T,E]. Returns nonzero on an invalid index.
+ */
+int oracle_router_backward(const float* logits, int64_t T, int E, int k, int score_fn,
+                           int renormalize, float scaling, const int32_t* topk_idx,
+                           const float* dprob, float* dlogits)
+{
+    double* q = (double*)malloc(sizeof(double) * (size_t)(E > k ? E : k));
+    double* g = (double*)malloc(sizeof(double) * (size_t)k);
+    for (int64_t t = 0; t < T; t++) {
+        const float* l = logits + t * E;
+        const int32_t* sel = topk_idx + t * k;
+        float* dl = dlogits + t * E;
+        for (int e = 0; e < E; e++) dl[e] = 0.0f;
+        for (int j = 0; j < k; j++) {
+            if (sel[j] < 0 || sel[j] >= E) { free(q); free(g); return 1; }
+            g[j] = (double)scaling * (double)dprob[t * k + j];
+        }
+        if (score_fn == 0 && renormalize) {
+            double m = l[sel[0]], sum = 0.0, c = 0.0;
+            for (int j = 1; j < k; j++) if (l[sel[j]] > m) m = l[sel[j]];
+            for (int j = 0; j < k; j++) { q[j] = exp((double)l[sel[j]] - m); sum += q[j]; }
+            for (int j = 0; j < k; j++) { q[j] /= sum; c += q[j] * g[j]; }
+            for (int j = 0; j < k; j++) dl[sel[j]] = (float)(q[j] * (g[j] - c));
+        } else if (score_fn == 0) {
+            double m = l[0], sum = 0.0, c = 0.0;
+            for (int e = 1; e < E; e++) if (l[e] > m) m = l[e];
+            for (int e = 0; e < E; e++) { q[e] = exp((double)l[e] - m); sum += q[e]; }
+            for (int e = 0; e < E; e++) q[e] /= sum;
+            for (int j = 0; j < k; j++) c += q[sel[j]] * g[j];
+            for (int e = 0; e < E; e++) dl[e] = (float)(q[e] * (0.0 - c));
+            for (int j = 0; j < k; j++) dl[sel[j]] = (float)(q[sel[j]] * (g[j] - c));
+        } else {
+            double S = 0.0, c = 0.0;
+            for (int j = 0; j < k; j++) { q[j] = 1.0 / (1.0 + exp(-(double)l[sel[j]])); S += q[j]; }
+            for (int j = 0; j < k; j++) {
+                double ds = g[j];   /* dL/ds_j without renormalisation */
+                if (renormalize) {
+                    if (j == 0) for (int i = 0; i < k; i++) c += (q[i] / S) * g[i];
+                    ds = (g[j] - c) / S;
+                }
+                dl[sel[j]] = (float)(ds * q[j] * (1.0 - q[j]));
+            }
+        }
+    }
+    free(q);
+    free(g);
+    return 0;
+}
+
 /* ----------------------------------------------------------- dispatch --- */
 
 /*
