@@ -472,8 +472,27 @@ def router_sweep(m, hbm):
         ms = statistics.median(times)
         nbytes = T * E * 4 + T * k * 8 + E * 8
         gbs = nbytes / (ms / 1e3) / 1e9
-        out.append({"T": T, "E": E, "k": k, "us": ms * 1e3, "GB/s": gbs, "frac_of_hbm": gbs / hbm})
-        del logits, res, ws
+        entry = {"T": T, "E": E, "k": k, "us": ms * 1e3, "GB/s": gbs, "frac_of_hbm": gbs / hbm}
+        # the backward through the score function on the same routing:
+        # reads logits, topk_idx and dprob, writes dlogits
+        dprob = torch.randn((T, k), generator=g, device="cuda")
+        dl = torch.empty_like(logits)
+        btimes = []
+        for it in range(8):
+            flush.sum()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            m.moe_router_backward(logits, res["topk_idx"], dprob, out=dl)
+            e.record()
+            torch.cuda.synchronize()
+            if it >= 2:
+                btimes.append(s.elapsed_time(e))
+        bms = statistics.median(btimes)
+        bbytes = 2 * T * E * 4 + T * k * 8
+        entry["backward"] = {"us": bms * 1e3, "GB/s": bbytes / (bms / 1e3) / 1e9,
+                             "frac_of_hbm": bbytes / (bms / 1e3) / 1e9 / hbm}
+        out.append(entry)
+        del logits, res, ws, dprob, dl
     return out
 
 

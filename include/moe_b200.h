@@ -124,6 +124,28 @@ moe_status moe_router_topk(const float* logits, int64_t T, int E, int k,
                            uint8_t* routing_map, int32_t* counts, int32_t* offsets,
                            void* workspace, size_t workspace_bytes, void* stream);
 
+/* moe_router_backward -- TE Router, backward through the score function:
+ * dlogits = dL/dlogits from dprob = dL/dtopk_prob, for the experts the
+ * forward chose. The choice itself is piecewise constant in the logits and
+ * passes no gradient; an expert_bias only moves the choice and is ignored.
+ * With g_j = scaling * dprob[t,j], computed in fp32:
+ *   softmax, renormalize=1: q = softmax over the chosen logits;
+ *       dlogits[t, e_j] = q_j (g_j - sum_i q_i g_i), 0 at experts not chosen.
+ *   softmax, renormalize=0: q = softmax over all E logits;
+ *       dlogits[t, e] = q_e (G_e - sum_j q_{e_j} g_j), G_e = g_j at e = e_j, else 0.
+ *   sigmoid, renormalize=0: dlogits[t, e_j] = g_j s_j (1 - s_j), s = sigmoid(logit).
+ *   sigmoid, renormalize=1: r_j = s_j / S, S = sum_j s_j;
+ *       dlogits[t, e_j] = (g_j - sum_i r_i g_i) / S * s_j (1 - s_j).
+ *  logits    in  fp32 [T, E]   the forward's logits
+ *  topk_idx  in  int32 [T, k]  the forward's choice (moe_router_topk)
+ *  dprob     in  fp32 [T, k]
+ *  dlogits   out fp32 [T, E]   every element written
+ * opts as in the forward call. An index outside [0, E) is recorded as
+ * MOE_ERR_DEVICE_CHECK (moe_get_device_status) and contributes nothing. */
+moe_status moe_router_backward(const float* logits, int64_t T, int E, int k,
+                               const moe_router_opts* opts, const int32_t* topk_idx,
+                               const float* dprob, float* dlogits, void* stream);
+
 /* moe_router_topk_noalloc -- the same routing as moe_router_topk, with no
  * workspace argument: for callers that cannot allocate device memory when they
  * route, such as a runtime that hands out all device memory from its own

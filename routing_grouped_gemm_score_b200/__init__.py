@@ -10,7 +10,8 @@ there is no fallback.
 Stages (Transformer Engine "Mixture of Experts": Router, Token dispatch,
 Grouped MLP, Token combine):
     moe_router_topk -> moe_permute -> moe_grouped_mlp -> moe_unpermute_combine
-fused as moe_layer_forward, with moe_grouped_mlp_backward for training.
+fused as moe_layer_forward, with moe_grouped_mlp_backward for training and
+moe_router_backward for the gradient through the score function.
 """
 from __future__ import annotations
 
@@ -25,7 +26,7 @@ __all__ = [
     "MoEError", "RouterOpts", "SCORE_SOFTMAX", "SCORE_SIGMOID", "library_path", "lib",
     "moe_status_string", "moe_get_device_status", "moe_router_topk", "moe_permute",
     "moe_grouped_mlp", "moe_unpermute_combine", "moe_layer_forward", "moe_grouped_mlp_backward",
-    "moe_trace_set", "moe_router_topk_noalloc", "LayerWorkspace", "ABI_FUNCTIONS",
+    "moe_trace_set", "moe_router_topk_noalloc", "moe_router_backward", "LayerWorkspace", "ABI_FUNCTIONS",
 ]
 
 SCORE_SOFTMAX = 0
@@ -76,6 +77,7 @@ ABI_FUNCTIONS = {
     "moe_trace_set": (I32, [ctypes.POINTER(ctypes.c_void_p), I32]),
     "moe_router_workspace_size": (SZ, [I64, I32, I32]),
     "moe_router_topk": (I32, [P, I64, I32, I32, ctypes.POINTER(_RouterOptsC), P, P, P, P, P, P, SZ, P]),
+    "moe_router_backward": (I32, [P, I64, I32, I32, ctypes.POINTER(_RouterOptsC), P, P, P, P]),
     "moe_router_topk_noalloc": (I32, [P, I64, I32, I32, ctypes.POINTER(_RouterOptsC), P, P, P, P,
                                        P, P]),
     "moe_permute_workspace_size": (SZ, [I64, I32, I32]),
@@ -213,6 +215,23 @@ def moe_router_topk_noalloc(logits: torch.Tensor, k: int, opts: Optional[RouterO
                                          _ptr(out.get("routing_map")), _ptr(out["counts"]),
                                          _ptr(out["offsets"]), _stream()),
            "moe_router_topk_noalloc")
+    return out
+
+
+def moe_router_backward(logits: torch.Tensor, topk_idx: torch.Tensor, dprob: torch.Tensor,
+                        opts: Optional[RouterOpts] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """dL/dlogits [T,E] (fp32) from dL/dtopk_prob for the experts the forward
+    chose, through the score function and the weight normalisation."""
+    _need(logits, torch.float32, "logits")
+    _need(topk_idx, torch.int32, "topk_idx")
+    _need(dprob, torch.float32, "dprob")
+    T, E = logits.shape
+    k = topk_idx.shape[1]
+    if out is None:
+        out = torch.empty((T, E), dtype=torch.float32, device=logits.device)
+    oc = (opts or RouterOpts()).c()
+    _check(lib().moe_router_backward(_ptr(logits), T, E, k, ctypes.byref(oc), _ptr(topk_idx), _ptr(dprob),
+                                     _ptr(out), _stream()), "moe_router_backward")
     return out
 
 

@@ -230,6 +230,22 @@ moe_status moe_router_topk(const float* logits, int64_t T, int E, int k,
     return from_cuda(e);
 }
 
+moe_status moe_router_backward(const float* logits, int64_t T, int E, int k,
+                               const moe_router_opts* opts_in, const int32_t* topk_idx,
+                               const float* dprob, float* dlogits, void* stream) {
+    if (!shape_ok(T, E, k)) return MOE_ERR_INVALID_ARG;
+    const moe_router_opts opts = opts_in ? *opts_in : default_opts();
+    if (check_opts(opts) != MOE_OK) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!logits || !topk_idx || !dprob || !dlogits || !aligned16(logits) ||
+                  !aligned16(topk_idx) || !aligned16(dprob) || !aligned16(dlogits)))
+        return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    unsigned* err = device_error_word();
+    if (!err) return MOE_ERR_CUDA;
+    return from_cuda(launch_router_backward(logits, T, E, k, opts, topk_idx, dprob, dlogits,
+                                            static_cast<cudaStream_t>(stream), err));
+}
+
 moe_status moe_router_topk_noalloc(const float* logits, int64_t T, int E, int k,
                                    const moe_router_opts* opts_in, int32_t* topk_idx,
                                    float* topk_prob, uint8_t* routing_map, int32_t* counts,

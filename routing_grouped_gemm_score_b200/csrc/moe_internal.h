@@ -43,6 +43,9 @@ cudaError_t launch_router_topk(const float* logits, int64_t T, int E, int k,
                                const moe_router_opts& opts, int32_t* topk_idx, float* topk_prob,
                                uint8_t* routing_map, const RouteScratch& rs, cudaStream_t st,
                                unsigned* err);
+cudaError_t launch_router_backward(const float* logits, int64_t T, int E, int k, const moe_router_opts& opts,
+                                   const int32_t* topk_idx, const float* dprob, float* dlogits,
+                                   cudaStream_t st, unsigned* err);
 cudaError_t launch_rank_from_indices(const int32_t* topk_idx, int64_t T, int E, int k,
                                      const RouteScratch& rs, cudaStream_t st, unsigned* err);
 // Turns block counts into exclusive prefixes; writes counts/offsets if given.

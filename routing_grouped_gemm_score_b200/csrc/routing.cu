@@ -246,6 +246,109 @@ __global__ void __launch_bounds__(kRouteThreads) router_topk_kernel(const Router
     rank_block(sel, t0, tpb, E, k, a.local_rank, a.block_base, a.nb);
 }
 
+// Router backward: dL/dlogits from dL/dtopk_prob, one warp per token, fp32.
+// Lane j < k holds pick j: its expert, logit and g_j = scaling * dprob[t,j].
+// The formulas per mode are those of the forward's weights differentiated
+// with the selection held fixed (see moe_router_backward in the header).
+template <int SLOTS>
+__global__ void __launch_bounds__(kRouteThreads)
+    router_backward_kernel(const float* __restrict__ logits, int64_t T, int E, int k, int score_fn,
+                           int renormalize, float scaling, const int32_t* __restrict__ topk_idx,
+                           const float* __restrict__ dprob, float* __restrict__ dlogits, unsigned* err) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
+        const float* lrow = logits + t * E;
+        int sel = -1;
+        float g = 0.0f, lsel = 0.0f;
+        if (lane < k) {
+            sel = __ldg(topk_idx + t * k + lane);
+            if (sel < 0 || sel >= E) {
+                raise_error(err, kErrDeviceCheck);
+                sel = -1;
+            }
+            g = scaling * __ldg(dprob + t * k + lane);
+            if (sel >= 0) lsel = __ldg(lrow + sel);
+        }
+        const bool pick = sel >= 0;
+        float dsel = 0.0f;          // gradient at this lane's pick
+        float dall[SLOTS];          // softmax over all experts: gradient of every slot
+#pragma unroll
+        for (int s = 0; s < SLOTS; ++s) dall[s] = 0.0f;
+        if (score_fn == MOE_SCORE_SOFTMAX && renormalize) {
+            float m = pick ? lsel : -INFINITY;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+            const float ex = pick ? expf(lsel - m) : 0.0f;
+            float sum = ex;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(kFull, sum, off);
+            const float q = ex / sum;
+            float c = q * g;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(kFull, c, off);
+            dsel = q * (g - c);
+        } else if (score_fn == MOE_SCORE_SOFTMAX) {
+            float lv[SLOTS];
+            float m = -INFINITY;
+#pragma unroll
+            for (int s = 0; s < SLOTS; ++s) {
+                const int e = lane + 32 * s;
+                lv[s] = e < E ? __ldg(lrow + e) : -INFINITY;
+                m = fmaxf(m, lv[s]);
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, off));
+            float sum = 0.0f;
+#pragma unroll
+            for (int s = 0; s < SLOTS; ++s) {
+                lv[s] = lane + 32 * s < E ? expf(lv[s] - m) : 0.0f;   // exp, in place
+                sum += lv[s];
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(kFull, sum, off);
+            const float qsel = pick ? expf(lsel - m) / sum : 0.0f;
+            float c = qsel * g;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(kFull, c, off);
+#pragma unroll
+            for (int s = 0; s < SLOTS; ++s) dall[s] = (lv[s] / sum) * (0.0f - c);
+            dsel = qsel * (g - c);
+        } else {
+            const float sg = pick ? 1.0f / (1.0f + expf(-lsel)) : 0.0f;
+            float ds = g;
+            if (renormalize) {
+                float S = sg;
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) S += __shfl_xor_sync(kFull, S, off);
+                float c = (sg / S) * g;
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(kFull, c, off);
+                ds = (g - c) / S;
+            }
+            // s (1 - s) with 1 - s = sigmoid(-l), accurate where s is near 1
+            dsel = pick ? ds * sg * (1.0f / (1.0f + expf(lsel))) : 0.0f;
+        }
+        // the row: each slot's value, replaced by the pick's where it is a pick
+        float v[SLOTS];
+#pragma unroll
+        for (int s = 0; s < SLOTS; ++s) v[s] = dall[s];
+        for (int j = 0; j < k; ++j) {
+            const int sj = __shfl_sync(kFull, sel, j);
+            const float dj = __shfl_sync(kFull, dsel, j);
+#pragma unroll
+            for (int s = 0; s < SLOTS; ++s)
+                if (lane + 32 * s == sj) v[s] = dj;
+        }
+        float* drow = dlogits + t * E;
+#pragma unroll
+        for (int s = 0; s < SLOTS; ++s) {
+            const int e = lane + 32 * s;
+            if (e < E) drow[e] = v[s];
+        }
+    }
+}
+
 // Rank pass for caller-supplied expert indices (moe_permute on its own).
 __global__ void __launch_bounds__(kRouteThreads)
     rank_from_indices_kernel(const int32_t* __restrict__ topk_idx, int64_t T, int E, int k,
@@ -456,6 +559,26 @@ cudaError_t launch_router_topk(const float* logits, int64_t T, int E, int k,
     else if (E <= 128) launch_router_k<4>(a, grid, block, st);
     else launch_router_k<8>(a, grid, block, st);
     (void)err;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_router_backward(const float* logits, int64_t T, int E, int k, const moe_router_opts& opts,
+                                   const int32_t* topk_idx, const float* dprob, float* dlogits,
+                                   cudaStream_t st, unsigned* err) {
+    const int64_t warps_per_block = kRouteThreads / 32;
+    int64_t blocks = (T + warps_per_block - 1) / warps_per_block;
+    const int64_t cap = (int64_t)sm_count() * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) return cudaSuccess;
+    const dim3 grid((unsigned)blocks), block(kRouteThreads);
+#define MOE_ROUTER_BWD(S)                                                                              \
+    router_backward_kernel<S><<<grid, block, 0, st>>>(logits, T, E, k, opts.score_fn, opts.renormalize, \
+                                                      opts.scaling, topk_idx, dprob, dlogits, err)
+    if (E <= 32) MOE_ROUTER_BWD(1);
+    else if (E <= 64) MOE_ROUTER_BWD(2);
+    else if (E <= 128) MOE_ROUTER_BWD(4);
+    else MOE_ROUTER_BWD(8);
+#undef MOE_ROUTER_BWD
     return cudaGetLastError();
 }
 
