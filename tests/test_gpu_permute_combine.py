@@ -66,11 +66,18 @@ def test_permute_rejects_invalid_indices_on_the_device():
     assert m.moe_get_device_status() == 0          # the word was cleared
 
 
+@pytest.mark.parametrize("path", ["auto", "regs", "bulk"])
 @pytest.mark.parametrize("T,k,H,shared,probs", [(64, 2, 128, False, True), (1000, 8, 2048, False, True),
                                                  (333, 1, 5120, True, True), (257, 4, 64, False, False),
-                                                 (1, 8, 2048, True, True)])
-def test_combine_matches_weighted_sum(T, k, H, shared, probs):
+                                                 (1, 8, 2048, True, True), (3000, 16, 512, True, True),
+                                                 (4100, 2, 4096, False, True)])
+def test_combine_matches_weighted_sum(T, k, H, shared, probs, path, monkeypatch):
+    """Both combine kernels (register path for rows up to 4096 wide, bulk
+    copies) on every shape; the register path stages 2048 assignments at a
+    time, so T=3000 at k=16 spans several stages of one block."""
     import routing_grouped_gemm_score_b200 as m
+    if path != "auto":
+        monkeypatch.setenv("MOE_COMBINE", path)
     g_ = torch.Generator().manual_seed(T * 7 + k)
     A = T * k
     y = torch.randn((A, H), generator=g_).to(torch.bfloat16)
