@@ -16,6 +16,7 @@
 // token order, and an exclusive scan over the token blocks turns them into
 // global rows. A block holds 8 to 64 tokens (route_tokens_per_block). Positions never come from atomics, so the permutation is the
 // same on every run.
+#include <cstdlib>
 #include <mutex>
 
 #include "moe_common.cuh"
@@ -491,6 +492,64 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// Permute over contiguous token ranges, on plain 16-byte loads and stores. A
+// block owns tokens [t_begin, t_end). Its threads compute the destination rows
+// of kPermStage assignments at a time (offsets[e] + block_base[e][t / tpb] +
+// local_rank, checked against the expert's block; row_of and sorted_token are
+// written here) into shared memory. Then each thread owns one 16-byte column
+// chunk (blockDim = H/8 rounded up to a warp, H <= 4096), loads it for 4
+// tokens at once and stores each to the token's k rows.
+constexpr int kPermStage = 2048;
+
+__global__ void __launch_bounds__(512)
+    permute_tokens_kernel(const uint4* __restrict__ x, int64_t T, int H8, const int32_t* __restrict__ topk_idx,
+                          int k, const int32_t* __restrict__ offsets, int E, const int32_t* __restrict__ block_base,
+                          int nb, int tpb, const int32_t* __restrict__ local_rank, uint4* __restrict__ x_perm,
+                          int32_t* __restrict__ sorted_token, int32_t* __restrict__ row_of, int64_t A,
+                          int64_t per_block, unsigned* err) {
+    __shared__ int32_t s_row[kPermStage];
+    const int64_t t_begin = (int64_t)blockIdx.x * per_block;
+    const int64_t t_end = t_begin + per_block < T ? t_begin + per_block : T;
+    const int c = threadIdx.x;
+    const bool active = c < H8;
+    const int tok_per_stage = kPermStage / k;
+    for (int64_t s0 = t_begin; s0 < t_end; s0 += tok_per_stage) {
+        const int ntok = (int)(t_end - s0 < tok_per_stage ? t_end - s0 : tok_per_stage);
+        __syncthreads();   // the previous stage's rows are no longer read
+        for (int i = threadIdx.x; i < ntok * k; i += blockDim.x) {
+            const int64_t t = s0 + i / k;
+            const int e = __ldg(topk_idx + s0 * k + i);
+            const int rank = __ldg(local_rank + s0 * k + i);
+            int32_t row = -1;
+            if (e >= 0 && e < E && rank >= 0) {
+                const int64_t lo = __ldg(offsets + e), hi = __ldg(offsets + e + 1);
+                const int64_t r = lo + __ldg(block_base + (int64_t)e * nb + t / tpb) + rank;
+                if (r >= lo && r < hi && r < A) row = (int32_t)r;
+            }
+            if (row < 0) raise_error(err, kErrDeviceCheck);
+            s_row[i] = row;
+            row_of[s0 * k + i] = row;
+            if (row >= 0) sorted_token[row] = (int32_t)t;
+        }
+        __syncthreads();
+        if (!active) continue;
+        for (int tt0 = 0; tt0 < ntok; tt0 += 4) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (tt0 + u < ntok) v[u] = __ldg(x + (s0 + tt0 + u) * H8 + c);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                if (tt0 + u >= ntok) break;
+                for (int j = 0; j < k; ++j) {
+                    const int32_t r = s_row[(tt0 + u) * k + j];
+                    if (r >= 0) x_perm[(int64_t)r * H8 + c] = v[u];
+                }
+            }
+        }
+    }
+}
+
 // Scratch for moe_router_topk_noalloc: a fixed array in device memory, so the
 // call allocates nothing. Its size bounds the routing sizes that call accepts.
 constexpr size_t kNoAllocScratchBytes = (3u << 20) + 4096;
@@ -605,6 +664,26 @@ cudaError_t launch_permute(const bf16* x, int64_t T, int H, const int32_t* topk_
                            int32_t* sorted_token, int32_t* row_of, cudaStream_t st, unsigned* err) {
     const int nb = (int)route_blocks(T);
     if (T == 0) return cudaSuccess;
+    const int H8r = H / 8;
+    // Register path for few rows per token, bulk copies otherwise (the same
+    // rule as the combine); MOE_PERMUTE=bulk|regs overrides.
+    const char* force = getenv("MOE_PERMUTE");
+    const bool regs = force ? (force[0] == 'r' && H8r <= 512) : (k <= 2 && H8r <= 512);
+    if (regs) {
+        const int threads = (H8r + 31) / 32 * 32;
+        int per_sm = 1;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, permute_tokens_kernel, threads, 0) != cudaSuccess ||
+            per_sm < 1)
+            per_sm = 1;
+        const int64_t slots = (int64_t)sm_count() * per_sm;
+        const int64_t per_block = (T + slots - 1) / slots;
+        const int64_t blocks = (T + per_block - 1) / per_block;
+        permute_tokens_kernel<<<(unsigned)blocks, threads, 0, st>>>(
+            reinterpret_cast<const uint4*>(x), T, H8r, topk_idx, k, offsets, E, rs.block_base, nb,
+            route_tokens_per_block(T), rs.local_rank, reinterpret_cast<uint4*>(x_perm), sorted_token, row_of,
+            T * k, per_block, err);
+        return cudaGetLastError();
+    }
     cudaError_t res = cudaSuccess;
     if (rows_permute(x, T, H, topk_idx, k, offsets, E, rs.block_base, nb, route_tokens_per_block(T),
                      rs.local_rank, x_perm, sorted_token, row_of, T * k, st, err, &res))

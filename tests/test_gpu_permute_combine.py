@@ -28,8 +28,12 @@ def routed(w):
 @pytest.mark.parametrize("name,T,H", [("tiny", None, None), ("qwen3_30b_a3b", 4096, 2048),
                                       ("skew_t1", None, 256), ("skew_t8", None, 256),
                                       ("skew_t64", None, 2048), ("llama4_17bx16e", 1000, 5120),
-                                      ("tie_t64", None, 128)])
-def test_permute_matches_dispatch_definition(name, T, H):
+                                      ("tie_t64", None, 128), ("mixtral_8x7b", 3000, 4096)])
+@pytest.mark.parametrize("path", ["auto", "regs", "bulk"])
+def test_permute_matches_dispatch_definition(name, T, H, path, monkeypatch):
+    """Both permute kernels (register path for rows up to 4096 wide, bulk
+    copies) on every shape."""
+    monkeypatch.setenv("MOE_PERMUTE", path) if path != "auto" else None
     w = wl.WORKLOADS[name]
     if T is not None:
         w = w.scaled(T=T)
