@@ -96,7 +96,7 @@ def test_backward_on_oracle_state(name, tiles, wgrad, monkeypatch):
     apart (assert_close_flips)."""
     import routing_grouped_gemm_score_b200 as m
     monkeypatch.setenv("MOE_GEMM_TILES", tiles)
-    monkeypatch.setenv("MOE_WGRAD", wgrad)   # weight gradient: shared-memory B panel, or one tile per CTA
+    monkeypatch.setenv("MOE_WGRAD", wgrad)   # weight gradient: B panel in shared memory, or one tile per CTA
     w = SMALL[name]
     d = wl.make_inputs(w, "cuda", with_dout=True)
     r = oracle.router_topk(d["logits"].cpu().numpy(), w.k)
