@@ -56,6 +56,8 @@ def _load():
             lib.oracle_router_topk.restype = i32
             lib.oracle_router_backward.argtypes = [P, i64, i32, i32, i32, i32, f32, P, P, P]
             lib.oracle_router_backward.restype = i32
+            lib.oracle_expert_bias_update.argtypes = [P, i32, f32, P]
+            lib.oracle_expert_bias_update.restype = None
             lib.oracle_dispatch.argtypes = [P, i64, i32, i32, P, P, P]
             lib.oracle_dispatch.restype = i32
             lib.oracle_gather_rows.argtypes = [P, i32, P, i64, P]
@@ -140,6 +142,15 @@ def router_backward(logits, topk_idx, dprob, score=0, renormalize=True, scaling=
     if rc:
         raise ValueError(f"oracle_router_backward: invalid index ({rc})")
     return dl
+
+
+def expert_bias_update(counts, bias, coeff):
+    """The expert bias after one load-balancing update (returns a new array)."""
+    lib = _load()
+    counts = _c(counts, np.int32)
+    out = np.array(bias, np.float32, copy=True)
+    lib.oracle_expert_bias_update(_p(counts), len(counts), coeff, _p(out))
+    return out
 
 
 def dispatch(topk_idx, offsets, E):

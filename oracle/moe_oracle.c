@@ -253,6 +253,31 @@ int oracle_router_backward(const float* logits, int64_t T, int E, int k, int sco
     return 0;
 }
 
+/*
+ * oracle_expert_bias_update -- torchtitan pull request 1269, llama4 moe.py,
+ * MoE._update_expert_bias (auxiliary-loss-free load balancing): with the
+ * per-expert token counts c[E] of the last step,
+ *   delta_e = coeff * sign(mean(c) - c_e),  delta_e -= mean(delta),
+ *   bias_e += delta_e.
+ * sign(mean(c) - c_e) is decided exactly, as sign(sum(c) - E * c_e), and the
+ * mean of delta in double precision. bias is updated in place (fp32).
+ */
+void oracle_expert_bias_update(const int32_t* counts, int E, float coeff, float* bias)
+{
+    int64_t sum = 0;
+    for (int e = 0; e < E; e++) sum += counts[e];
+    double mean_delta = 0.0;
+    double* delta = (double*)malloc(sizeof(double) * (size_t)E);
+    for (int e = 0; e < E; e++) {
+        const int64_t d = sum - (int64_t)E * counts[e];
+        delta[e] = (double)coeff * (double)((d > 0) - (d < 0));
+        mean_delta += delta[e];
+    }
+    mean_delta /= E;
+    for (int e = 0; e < E; e++) bias[e] = (float)((double)bias[e] + (delta[e] - mean_delta));
+    free(delta);
+}
+
 /* ----------------------------------------------------------- dispatch --- */
 
 /*
