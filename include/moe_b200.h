@@ -146,6 +146,19 @@ moe_status moe_router_backward(const float* logits, int64_t T, int E, int k,
                                const moe_router_opts* opts, const int32_t* topk_idx,
                                const float* dprob, float* dlogits, void* stream);
 
+/* moe_expert_bias_update -- auxiliary-loss-free load balancing between steps
+ * (TE Router, Load balancing: lower the bias of overloaded experts, raise it
+ * for under-used ones; torchtitan MoE._update_expert_bias). With the counts of
+ * the last step (moe_router_topk's counts, on the device, no host sync):
+ *   delta_e = coeff * sign(mean(counts) - counts[e]), decided exactly in
+ *             integers; then delta_e -= mean(delta); expert_bias[e] += delta_e
+ * in fp32. The bias is then passed to the next moe_router_topk (sigmoid score).
+ *  counts       in     int32 [E]
+ *  expert_bias  in/out fp32  [E]
+ * E in [1, 256]. */
+moe_status moe_expert_bias_update(const int32_t* counts, int E, float coeff, float* expert_bias,
+                                  void* stream);
+
 /* moe_router_topk_noalloc -- the same routing as moe_router_topk, with no
  * workspace argument: for callers that cannot allocate device memory when they
  * route, such as a runtime that hands out all device memory from its own

@@ -26,7 +26,7 @@ __all__ = [
     "MoEError", "RouterOpts", "SCORE_SOFTMAX", "SCORE_SIGMOID", "library_path", "lib",
     "moe_status_string", "moe_get_device_status", "moe_router_topk", "moe_permute",
     "moe_grouped_mlp", "moe_unpermute_combine", "moe_layer_forward", "moe_grouped_mlp_backward",
-    "moe_trace_set", "moe_router_topk_noalloc", "moe_router_backward", "LayerWorkspace", "ABI_FUNCTIONS",
+    "moe_trace_set", "moe_router_topk_noalloc", "moe_router_backward", "moe_expert_bias_update", "LayerWorkspace", "ABI_FUNCTIONS",
 ]
 
 SCORE_SOFTMAX = 0
@@ -78,6 +78,7 @@ ABI_FUNCTIONS = {
     "moe_router_workspace_size": (SZ, [I64, I32, I32]),
     "moe_router_topk": (I32, [P, I64, I32, I32, ctypes.POINTER(_RouterOptsC), P, P, P, P, P, P, SZ, P]),
     "moe_router_backward": (I32, [P, I64, I32, I32, ctypes.POINTER(_RouterOptsC), P, P, P, P]),
+    "moe_expert_bias_update": (I32, [P, I32, ctypes.c_float, P, P]),
     "moe_router_topk_noalloc": (I32, [P, I64, I32, I32, ctypes.POINTER(_RouterOptsC), P, P, P, P,
                                        P, P]),
     "moe_permute_workspace_size": (SZ, [I64, I32, I32]),
@@ -233,6 +234,16 @@ def moe_router_backward(logits: torch.Tensor, topk_idx: torch.Tensor, dprob: tor
     _check(lib().moe_router_backward(_ptr(logits), T, E, k, ctypes.byref(oc), _ptr(topk_idx), _ptr(dprob),
                                      _ptr(out), _stream()), "moe_router_backward")
     return out
+
+
+def moe_expert_bias_update(counts: torch.Tensor, expert_bias: torch.Tensor, coeff: float) -> torch.Tensor:
+    """Aux-loss-free load balancing between steps: updates expert_bias in place
+    from the per-expert token counts of the last step, and returns it."""
+    _need(counts, torch.int32, "counts")
+    _need(expert_bias, torch.float32, "expert_bias")
+    _check(lib().moe_expert_bias_update(_ptr(counts), counts.numel(), float(coeff), _ptr(expert_bias), _stream()),
+           "moe_expert_bias_update")
+    return expert_bias
 
 
 def moe_permute(x: torch.Tensor, topk_idx: torch.Tensor, offsets: torch.Tensor) -> dict:

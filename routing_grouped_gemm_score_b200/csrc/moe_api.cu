@@ -246,6 +246,14 @@ moe_status moe_router_backward(const float* logits, int64_t T, int E, int k,
                                             static_cast<cudaStream_t>(stream), err));
 }
 
+moe_status moe_expert_bias_update(const int32_t* counts, int E, float coeff, float* expert_bias,
+                                  void* stream) {
+    if (E < 1 || E > 256 || !counts || !expert_bias || !aligned16(counts) || !aligned16(expert_bias))
+        return MOE_ERR_INVALID_ARG;
+    if (!(coeff == coeff)) return MOE_ERR_INVALID_ARG;
+    return from_cuda(launch_expert_bias_update(counts, E, coeff, expert_bias, static_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_router_topk_noalloc(const float* logits, int64_t T, int E, int k,
                                    const moe_router_opts* opts_in, int32_t* topk_idx,
                                    float* topk_prob, uint8_t* routing_map, int32_t* counts,

@@ -46,6 +46,7 @@ cudaError_t launch_router_topk(const float* logits, int64_t T, int E, int k,
 cudaError_t launch_router_backward(const float* logits, int64_t T, int E, int k, const moe_router_opts& opts,
                                    const int32_t* topk_idx, const float* dprob, float* dlogits,
                                    cudaStream_t st, unsigned* err);
+cudaError_t launch_expert_bias_update(const int32_t* counts, int E, float coeff, float* bias, cudaStream_t st);
 cudaError_t launch_rank_from_indices(const int32_t* topk_idx, int64_t T, int E, int k,
                                      const RouteScratch& rs, cudaStream_t st, unsigned* err);
 // Turns block counts into exclusive prefixes; writes counts/offsets if given.

@@ -350,6 +350,35 @@ __global__ void __launch_bounds__(kRouteThreads)
     }
 }
 
+// Expert-bias update (auxiliary-loss-free load balancing), one block of 256
+// threads: delta_e = coeff * sign(mean(c) - c_e), decided exactly as
+// sign(sum(c) - E c_e), then centred (mean of delta = coeff (n_below -
+// n_above) / E) and added to the bias.
+__global__ void __launch_bounds__(256)
+    expert_bias_update_kernel(const int32_t* __restrict__ counts, int E, float coeff, float* __restrict__ bias) {
+    __shared__ long long s_sum[8];
+    __shared__ int s_net[8];
+    const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
+    const int c = e < E ? counts[e] : 0;
+    long long sum = c;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(kFull, sum, off);
+    if (lane == 0) s_sum[warp] = sum;
+    __syncthreads();
+    long long total = 0;
+    for (int w = 0; w < 8; ++w) total += s_sum[w];
+    const long long d = total - (long long)E * c;
+    const int sgn = e < E ? (d > 0) - (d < 0) : 0;
+    int net = sgn;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) net += __shfl_xor_sync(kFull, net, off);
+    if (lane == 0) s_net[warp] = net;
+    __syncthreads();
+    int n = 0;
+    for (int w = 0; w < 8; ++w) n += s_net[w];
+    if (e < E) bias[e] = bias[e] + (coeff * (float)sgn - coeff * (float)n / (float)E);
+}
+
 // Rank pass for caller-supplied expert indices (moe_permute on its own).
 __global__ void __launch_bounds__(kRouteThreads)
     rank_from_indices_kernel(const int32_t* __restrict__ topk_idx, int64_t T, int E, int k,
@@ -638,6 +667,11 @@ cudaError_t launch_router_backward(const float* logits, int64_t T, int E, int k,
     else if (E <= 128) MOE_ROUTER_BWD(4);
     else MOE_ROUTER_BWD(8);
 #undef MOE_ROUTER_BWD
+    return cudaGetLastError();
+}
+
+cudaError_t launch_expert_bias_update(const int32_t* counts, int E, float coeff, float* bias, cudaStream_t st) {
+    expert_bias_update_kernel<<<1, 256, 0, st>>>(counts, E, coeff, bias);
     return cudaGetLastError();
 }
 

@@ -136,3 +136,25 @@ def test_router_large_sweep_invariants():
     logits = torch.randn((1 << 18, 128), generator=g_)
     g, r = run_both(logits, 8)
     check(g, r)
+
+
+@pytest.mark.parametrize("E", [1, 8, 100, 128, 256])
+def test_expert_bias_update_matches_oracle(E):
+    """Aux-loss-free load balancing: the bias update from the router's own
+    counts, on the device, against the oracle; then the next routing with the
+    new bias (sigmoid score)."""
+    import oracle
+    import routing_grouped_gemm_score_b200 as m
+    g_ = torch.Generator().manual_seed(E)
+    logits = torch.randn((777, E), generator=g_) * 2
+    k = min(E, 4)
+    bias = (torch.randn(E, generator=g_) * 0.1).cuda()
+    opts = m.RouterOpts(m.SCORE_SIGMOID, False, 1.0, bias)
+    r = m.moe_router_topk(logits.cuda(), k, opts)
+    before = bias.cpu().numpy().copy()
+    m.moe_expert_bias_update(r["counts"], bias, 1e-3)
+    torch.cuda.synchronize()
+    ref = oracle.expert_bias_update(r["counts"].cpu().numpy(), before, 1e-3)
+    np.testing.assert_allclose(bias.cpu().numpy(), ref, rtol=0, atol=1e-6 * 1e-3 + 1e-7 * np.abs(ref).max())
+    g, o = run_both(logits, k, 1, False, 1.0, bias.cpu())
+    check(g, o)
