@@ -49,77 +49,6 @@ __device__ __forceinline__ uint4 pack8(const float (&acc)[8]) {
                       pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
 }
 
-// One block per output row. The first k threads fetch the row's permuted
-// rows and weights into shared memory; then each thread owns 16-byte column
-// chunks and issues the k row loads of a chunk together.
-__global__ void __launch_bounds__(256)
-    combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ row_of,
-                   const float* __restrict__ probs, int64_t T, int k, int H8, int64_t A,
-                   const uint4* __restrict__ shared, uint4* __restrict__ out, unsigned* err) {
-    __shared__ int64_t rows[16];
-    __shared__ float ps[16];
-    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-        if (threadIdx.x < (unsigned)k) {
-            const int j = threadIdx.x;
-            const int32_t r = row_of[t * k + j];
-            const bool ok = r >= 0 && r < A;
-            if (!ok) raise_error(err, kErrDeviceCheck);
-            rows[j] = ok ? r : -1;
-            ps[j] = probs ? probs[t * k + j] : 1.0f;
-        }
-        __syncthreads();
-        if (k <= 4) {
-            // few rows per token: two column chunks per thread and pass
-            for (int c0 = threadIdx.x; c0 < H8; c0 += 2 * blockDim.x) {
-                const int c1 = c0 + blockDim.x;
-                const bool two = c1 < H8;
-                float a0[8], a1[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) a0[i] = a1[i] = 0.0f;
-                if (shared) {
-                    add_scaled(a0, __ldg(shared + t * H8 + c0), 1.0f);
-                    if (two) add_scaled(a1, __ldg(shared + t * H8 + c1), 1.0f);
-                }
-                uint4 v0[4], v1[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    if (j < k && rows[j] >= 0) {
-                        v0[j] = __ldg(y + rows[j] * H8 + c0);
-                        if (two) v1[j] = __ldg(y + rows[j] * H8 + c1);
-                    }
-                }
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    if (j < k && rows[j] >= 0) {
-                        add_scaled(a0, v0[j], ps[j]);
-                        if (two) add_scaled(a1, v1[j], ps[j]);
-                    }
-                }
-                out[t * H8 + c0] = pack8(a0);
-                if (two) out[t * H8 + c1] = pack8(a1);
-            }
-        } else {
-            for (int c = threadIdx.x; c < H8; c += blockDim.x) {
-                float acc[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-                if (shared) add_scaled(acc, __ldg(shared + t * H8 + c), 1.0f);
-                for (int j0 = 0; j0 < k; j0 += 8) {      // up to 8 row loads in flight
-                    uint4 v[8];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        if (j0 + j < k && rows[j0 + j] >= 0) v[j] = __ldg(y + rows[j0 + j] * H8 + c);
-#pragma unroll
-                    for (int j = 0; j < 8; ++j)
-                        if (j0 + j < k && rows[j0 + j] >= 0) add_scaled(acc, v[j], ps[j0 + j]);
-                }
-                out[t * H8 + c] = pack8(acc);
-            }
-        }
-        __syncthreads();   // rows/ps are rewritten for the next row
-    }
-}
-
 // Backward of the weighted combine, one block per token:
 //   dy_perm[row_of[t,j]] = bf16(p[t,j] * dout[t])
 //   dprob[t,j] = sum_h dout[t,h] * y_perm[row_of[t,j], h]   (fp32)
@@ -309,11 +238,8 @@ cudaError_t launch_combine(const bf16* y_perm, const int32_t* row_of, const floa
         return cudaGetLastError();
     }
     cudaError_t res = cudaSuccess;
-    if (rows_combine(y_perm, row_of, probs, T, k, H, A, shared, out, st, err, &res)) return res;
-    combine_kernel<<<(unsigned)row_blocks(T), row_threads(H / 8), 0, st>>>(
-        reinterpret_cast<const uint4*>(y_perm), row_of, probs, T, k, H / 8, A,
-        reinterpret_cast<const uint4*>(shared), reinterpret_cast<uint4*>(out), err);
-    return cudaGetLastError();
+    rows_combine(y_perm, row_of, probs, T, k, H, A, shared, out, st, err, &res);
+    return res;
 }
 
 cudaError_t launch_combine_backward(const bf16* dout, const bf16* y_perm, const int32_t* row_of,

@@ -476,51 +476,6 @@ __global__ void __launch_bounds__(1024)
     if (threadIdx.x == 0) *ticket = 0u;
 }
 
-// Token dispatch: one block per token. The first k threads compute the rows
-// of the token's k assignments (expert offset + rank of the token block +
-// rank inside it) into shared memory; then each thread reads its 16-byte
-// column chunks of the token's row once and writes them to the k rows.
-__global__ void __launch_bounds__(256)
-    permute_kernel(const uint4* __restrict__ x, int64_t T, int H8, const int32_t* __restrict__ topk_idx,
-                   int k, const int32_t* __restrict__ offsets, int E,
-                   const int32_t* __restrict__ block_base, int nb, int tpb,
-                   const int32_t* __restrict__ local_rank, uint4* __restrict__ x_perm,
-                   int32_t* __restrict__ sorted_token, int32_t* __restrict__ row_of, int64_t A,
-                   unsigned* err) {
-    __shared__ int64_t rows[16];
-    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-        if (threadIdx.x < (unsigned)k) {
-            const int j = threadIdx.x;
-            int64_t row = -1;
-            const int e = topk_idx[t * k + j];
-            const int rank = local_rank[t * k + j];
-            if (e >= 0 && e < E && rank >= 0) {
-                const int64_t r = (int64_t)offsets[e] + block_base[(int64_t)e * nb + t / tpb] + rank;
-                if (r >= offsets[e] && r < offsets[e + 1] && r < A) row = r;
-            }
-            if (row < 0) raise_error(err, kErrDeviceCheck);
-            row_of[t * k + j] = (int32_t)row;
-            if (row >= 0) sorted_token[row] = (int32_t)t;
-            rows[j] = row;
-        }
-        __syncthreads();
-        for (int c0 = threadIdx.x; c0 < H8; c0 += 2 * blockDim.x) {   // two loads in flight
-            const int c1 = c0 + blockDim.x;
-            const bool two = c1 < H8;
-            const uint4 v0 = __ldg(x + t * H8 + c0);
-            const uint4 v1 = two ? __ldg(x + t * H8 + c1) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                if (j < k && rows[j] >= 0) {
-                    x_perm[rows[j] * H8 + c0] = v0;
-                    if (two) x_perm[rows[j] * H8 + c1] = v1;
-                }
-            }
-        }
-        __syncthreads();
-    }
-}
-
 // Permute over contiguous token ranges, on plain 16-byte loads and stores. A
 // block owns tokens [t_begin, t_end). Its threads compute the destination rows
 // of kPermStage assignments at a time (offsets[e] + block_base[e][t / tpb] +
@@ -719,21 +674,9 @@ cudaError_t launch_permute(const bf16* x, int64_t T, int H, const int32_t* topk_
         return cudaGetLastError();
     }
     cudaError_t res = cudaSuccess;
-    if (rows_permute(x, T, H, topk_idx, k, offsets, E, rs.block_base, nb, route_tokens_per_block(T),
-                     rs.local_rank, x_perm, sorted_token, row_of, T * k, st, err, &res))
-        return res;
-    const int H8 = H / 8;
-    int threads = 32;
-    while (threads < H8 && threads < 256) threads <<= 1;
-    int64_t blocks = T;
-    const int64_t cap = (int64_t)sm_count() * 64;
-    if (blocks > cap) blocks = cap;
-    if (blocks < 1) blocks = 1;
-    permute_kernel<<<(unsigned)blocks, threads, 0, st>>>(
-        reinterpret_cast<const uint4*>(x), T, H8, topk_idx, k, offsets, E, rs.block_base, nb,
-        route_tokens_per_block(T), rs.local_rank, reinterpret_cast<uint4*>(x_perm), sorted_token,
-        row_of, T * k, err);
-    return cudaGetLastError();
+    rows_permute(x, T, H, topk_idx, k, offsets, E, rs.block_base, nb, route_tokens_per_block(T), rs.local_rank, x_perm,
+                 sorted_token, row_of, T * k, st, err, &res);
+    return res;
 }
 
 // Device address of g_router_noalloc_scratch on the current device. In host

@@ -1,26 +1,23 @@
 // rows.cu -- the row-moving kernels on bulk asynchronous copies: token
-// dispatch (permute), the weighted combine, its backward, and the token sum
-// of the backward's dx rows.
+// dispatch (permute), and the weighted combine (also the token sum of the
+// backward's dx rows, with weight 1).
 //
 // Transformer Engine "Mixture of Experts", sections Token dispatch, Token
 // combine and Token probabilities:
 //   permute:      x_perm[row(t,j)] = x[t]
 //   combine:      out[t] = shared[t] + sum_j p[t,j] * y_perm[row_of[t,j]]
-//   combine bwd:  dy_perm[row_of[t,j]] = bf16(p[t,j] * dout[t]),
-//                 dprob[t,j] = <dout[t], y_perm[row_of[t,j]]>
 //
-// Every one of them moves whole rows whose addresses come from a chain of
-// index loads. Each block has one producer warp and four consumer warps. The
-// producer fetches the routing of the unit after next while the current one
-// is in flight. It brings each unit's rows into a ring of shared-memory
-// stages with cp.async.bulk, which completes on the stage's mbarrier. The
-// consumers compute from shared memory and store 16-byte vectors to global
-// memory; permute writes its k copies of a row with bulk stores straight
-// from shared memory. A unit is a column piece of one token, sized so that a
-// stage holds about 16 KB; a block takes a token's pieces in order, so the
-// backward's dprob sums over the pieces in registers. Each output element has
-// a single writer and a fixed order of operations: shared first, then j
-// ascending, in fp32.
+// Both move whole rows whose addresses come from a chain of index loads.
+// Each block has one producer warp and four consumer warps (permute: one).
+// The producer reads the routing of its tokens a chunk ahead and brings each
+// unit's rows into a ring of shared-memory stages with cp.async.bulk, which
+// completes on the stage's mbarrier. Combine's consumers compute from shared
+// memory and store 16-byte vectors to global memory; permute writes its k
+// copies of a row with bulk stores straight from shared memory. A unit is a
+// column piece of one token, sized so that a stage holds about 16 KB; a block
+// takes a contiguous range of tokens and each token's pieces in order. Each
+// output element has a single writer and a fixed order of operations: shared
+// first, then j ascending, in fp32.
 //
 // Every wait is bounded (kWaitLimitNs). A timeout records MOE_ERR_TIMEOUT and
 // stops both roles. The producer then waits, again bounded, for the copies it
@@ -44,18 +41,17 @@ constexpr uint32_t kBlockBudget = 48u * 1024;    // all stages of a block: four 
 constexpr int kMaxBlocksPerSm = 4;
 constexpr int kRouteEntries = 128;              // assignments per routing chunk
 
-enum RowsMode { kPermute = 0, kCombine = 1, kCombineBwd = 2 };
+enum RowsMode { kPermute = 0, kCombine = 1 };
 
 struct RowsJob {
     int64_t T;
     int k, H;
     int64_t A;
-    const bf16* src;        // rows gathered by index (combine, combine bwd): y_perm [A,H]
-    const bf16* tok;        // the token-order row: shared (combine, may be null), x, dout
-    const int32_t* row_of;  // [T,k] (combine, combine bwd)
+    const bf16* src;        // rows gathered by index (combine): y_perm [A,H]
+    const bf16* tok;        // the token-order row: shared (combine, may be null) or x (permute)
+    const int32_t* row_of;  // [T,k] (combine)
     const float* probs;     // [T,k]; null: weight 1 (combine)
-    bf16* out;              // combine: out [T,H]; permute: x_perm [A,H]; bwd: dy_perm [A,H]
-    float* dprob;           // combine bwd: [T,k]
+    bf16* out;              // combine: out [T,H]; permute: x_perm [A,H]
     // permute: where each assignment goes
     const int32_t* topk_idx;
     const int32_t* offsets;
@@ -79,11 +75,10 @@ struct StageMeta {
 };
 static_assert(sizeof(StageMeta) == 256, "stage metadata is 256 bytes");
 
-// Shared memory: barriers and flags | per-stage metadata | dprob partials |
-// routing tables (2 x rows, 2 x weights) | expert offsets | data stages.
+// Shared memory: barriers and flags | per-stage metadata | routing tables
+// (2 x rows, 2 x weights) | expert offsets | data stages.
 constexpr uint32_t kMetaOffset = 256;
-constexpr uint32_t kPartOffset = kMetaOffset + kMaxStages * sizeof(StageMeta);
-constexpr uint32_t kRouteOffset = kPartOffset + kMaxStages * kConsumerWarps * 16 * 4;
+constexpr uint32_t kRouteOffset = kMetaOffset + kMaxStages * sizeof(StageMeta);
 constexpr uint32_t kOffsOffset = kRouteOffset + 4 * kRouteEntries * 4;
 constexpr uint32_t kDataOffset = (kOffsOffset + 260 * 4 + 127) & ~127u;
 
@@ -421,110 +416,42 @@ __device__ void permute_storer(const RowsJob& j, uint64_t* full, uint64_t* empty
     if (prev_s >= 0 && lane == 0) mbar_arrive(&empty[prev_s]);
 }
 
-template <int MODE>
-__device__ void rows_consumer(const RowsJob& j, uint64_t* full, uint64_t* empty, uint64_t* red,
-                              volatile int* abort, const StageMeta* meta, float* part_all,
-                              const uint8_t* data, int cw, int lane) {
+// Combine's consumer warps: shared + sum_j p_j y_j for each column chunk of
+// the stage, in fp32, j in order, then one 16-byte store.
+__device__ void rows_consumer(const RowsJob& j, uint64_t* full, uint64_t* empty, volatile int* abort,
+                              const StageMeta* meta, const uint8_t* data, int cw, int lane) {
     const int S = j.stages;
     const int ct = cw * 32 + lane;                 // 0 .. kConsumerThreads-1
     const int H8 = j.H / 8;
     const int k = j.k;
     const int slot16 = (int)(j.slot_bytes / 16);
     uint4* out = reinterpret_cast<uint4*>(j.out);
-    const int ts = (MODE == kCombineBwd || j.tok != nullptr) ? 1 : 0;   // slot of the first gathered row
+    const bool tok_row = j.tok != nullptr;
+    const int ts = tok_row ? 1 : 0;                // slot of the first gathered row
     int64_t t_begin, t_end;
     block_tokens(j, t_begin, t_end);
     int i = 0;
     for (int64_t t = t_begin; t < t_end; ++t) {
-        bool ok = true;
-        constexpr int kDots = MODE == kCombineBwd ? 16 : 1;
-        float dot[kDots];   // combine bwd: this thread's part of <dout, y_j> over all pieces
-#pragma unroll
-        for (int q = 0; q < kDots; ++q) dot[q] = 0.0f;
         for (int piece = 0; piece < j.pieces; ++piece, ++i) {
             const int col0 = piece * j.cols;
             const int w8 = min(j.cols, j.H - col0) / 8;
             const int s = i % S;
-            const uint32_t ph = (uint32_t)(i / S) & 1u;
-            if (!warp_wait(&full[s], ph, abort, j.err, lane)) {
-                ok = false;
-                break;
-            }
+            if (!warp_wait(&full[s], (uint32_t)(i / S) & 1u, abort, j.err, lane)) return;
             const StageMeta& m = meta[s];
             const uint32_t valid = m.valid;
             const uint4* st = reinterpret_cast<const uint4*>(data + (size_t)s * j.stage_bytes);
-            if constexpr (MODE == kCombine) {
-                const bool tok_row = j.tok != nullptr;
-                for (int c = ct; c < w8; c += kConsumerThreads) {
-                    float acc[8];
+            for (int c = ct; c < w8; c += kConsumerThreads) {
+                float acc[8];
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
-                    if (tok_row) add_scaled(acc, st[c], 1.0f);
-                    for (int jj = 0; jj < k; ++jj)
-                        if ((valid >> jj) & 1u) add_scaled(acc, st[(ts + jj) * slot16 + c], m.p[jj]);
-                    out[t * H8 + col0 / 8 + c] = pack8(acc);
-                }
-            } else if constexpr (MODE == kCombineBwd) {
-                for (int c = ct; c < w8; c += kConsumerThreads) {
-                    const uint4 d = st[c];
-                    const uint32_t dw[4] = {d.x, d.y, d.z, d.w};
-#pragma unroll
-                    for (int jj = 0; jj < 16; ++jj) {
-                        if (jj >= k) break;
-                        if (!((valid >> jj) & 1u)) continue;
-                        const uint4 yv = st[(ts + jj) * slot16 + c];
-                        const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
-                        const float pj = m.p[jj];
-                        float sc[8];
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const float2 df = unpack_bf16x2(dw[q]);
-                            const float2 yf = unpack_bf16x2(yw[q]);
-                            dot[jj] += df.x * yf.x;
-                            dot[jj] += df.y * yf.y;
-                            sc[2 * q] = pj * df.x;
-                            sc[2 * q + 1] = pj * df.y;
-                        }
-                        out[(int64_t)m.row[jj] * H8 + col0 / 8 + c] = pack8(sc);
-                    }
-                }
-            }
-            if constexpr (MODE == kCombineBwd) {
-                // dprob: warp butterfly, then the four warps in order. Every use
-                // of a stage arrives on its reduction barrier, so the barrier's
-                // phases follow the stage's; only a token's last piece carries
-                // partial sums, and warp 0 of the consumers reads them.
-                const bool last = piece + 1 == j.pieces;
-                float* part = part_all + s * (kConsumerWarps * 16);
-                if (last) {
-#pragma unroll
-                    for (int jj = 0; jj < 16; ++jj) {
-                        if (jj >= k) break;
-                        float v = dot[jj];
-#pragma unroll
-                        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(kFull, v, off);
-                        if (lane == 0) part[cw * 16 + jj] = v;
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&red[s]);
-                if (last && cw == 0) {
-                    if (!warp_wait(&red[s], ph, abort, j.err, lane)) {
-                        ok = false;
-                        break;
-                    }
-                    if (lane < k) {
-                        float sum = 0.0f;
-#pragma unroll
-                        for (int q = 0; q < kConsumerWarps; ++q) sum += part[q * 16 + lane];
-                        j.dprob[t * k + lane] = sum;
-                    }
-                }
+                for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
+                if (tok_row) add_scaled(acc, st[c], 1.0f);
+                for (int jj = 0; jj < k; ++jj)
+                    if ((valid >> jj) & 1u) add_scaled(acc, st[(ts + jj) * slot16 + c], m.p[jj]);
+                out[t * H8 + col0 / 8 + c] = pack8(acc);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
         }
-        if (!ok) break;
     }
 }
 
@@ -534,10 +461,8 @@ __global__ void __launch_bounds__(kRowsThreads) rows_kernel(const RowsJob j) {
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kMaxStages;
-    uint64_t* red = empty + kMaxStages;
-    volatile int* abort = reinterpret_cast<volatile int*>(red + kMaxStages);
+    volatile int* abort = reinterpret_cast<volatile int*>(empty + kMaxStages);
     StageMeta* meta = reinterpret_cast<StageMeta*>(smem + kMetaOffset);
-    float* part = reinterpret_cast<float*>(smem + kPartOffset);
     int32_t* rt_a = reinterpret_cast<int32_t*>(smem + kRouteOffset);
     float* rt_p = reinterpret_cast<float*>(smem + kRouteOffset + 2 * kRouteEntries * 4);
     int32_t* s_off = reinterpret_cast<int32_t*>(smem + kOffsOffset);
@@ -546,7 +471,6 @@ __global__ void __launch_bounds__(kRowsThreads) rows_kernel(const RowsJob j) {
         for (int s = 0; s < j.stages; ++s) {
             mbar_init(&full[s], 32);
             mbar_init(&empty[s], MODE == kPermute ? 1 : kConsumerWarps);
-            mbar_init(&red[s], kConsumerWarps);
         }
         *abort = 0;
         fence_mbar_init();
@@ -559,7 +483,7 @@ __global__ void __launch_bounds__(kRowsThreads) rows_kernel(const RowsJob j) {
         if constexpr (MODE == kPermute)
             permute_storer(j, full, empty, abort, meta, data, lane);   // launched with two warps
         else
-            rows_consumer<MODE>(j, full, empty, red, abort, meta, part, data, warp - 1, lane);
+            rows_consumer(j, full, empty, abort, meta, data, warp - 1, lane);
     }
 }
 
@@ -628,21 +552,6 @@ bool rows_combine(const bf16* y_perm, const int32_t* row_of, const float* probs,
     j.probs = probs;
     j.out = out;
     *res = rows_launch<kCombine>(j, st);
-    return true;
-}
-
-bool rows_combine_backward(const bf16* dout, const bf16* y_perm, const int32_t* row_of, const float* probs,
-                           int64_t T, int k, int H, int64_t A, bf16* dy_perm, float* dprob, cudaStream_t st,
-                           unsigned* err, cudaError_t* res) {
-    RowsJob j = base_job(T, k, H, A, err);
-    rows_geometry(j, k + 1);
-    j.src = y_perm;
-    j.tok = dout;
-    j.row_of = row_of;
-    j.probs = probs;
-    j.out = dy_perm;
-    j.dprob = dprob;
-    *res = rows_launch<kCombineBwd>(j, st);
     return true;
 }
 
