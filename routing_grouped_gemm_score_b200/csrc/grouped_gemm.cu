@@ -70,6 +70,9 @@ constexpr int kStageA1 = BM1 * BK * 2, kStageB1 = BN * BK * 2, kStage1 = kStageA
 // CTA pair: 256 x 256 tile, each CTA 6 stages of 16 + 16 KB
 constexpr int BMP = 256, STAGESP = 6;
 constexpr int kStageAP = 128 * BK * 2, kStageBP = (BN / 2) * BK * 2, kStageP = kStageAP + kStageBP;
+// CTA pair, 128-row tile (an expert block's last <= 128 rows): each CTA loads
+// 64 rows of A and its usual half of B
+constexpr int kStageHalfP = 64 * BK * 2 + kStageBP;
 
 enum Epi { kEpiStore = 0, kEpiSwiglu = 1, kEpiSwigluBwd = 2 };
 
@@ -219,6 +222,30 @@ __device__ __forceinline__ Tile decode_tile(const S& s, const Params& p, int id,
     return t;
 }
 
+// First column of chunk c (64 columns) of an N-major weight tile. The SwiGLU
+// forward takes a tile's gate columns and the matching up columns, so that one
+// accumulator holds both. Single CTA: chunks 0..3 of a 256-column tile. Pair,
+// 256-row tile: CTA 0 the 128 gate columns, CTA 1 the matching up columns;
+// 128-row tile: each CTA 64 gate columns and their up columns.
+template <int EPI>
+__device__ __forceinline__ int b_col_1cta(const Tile& t, const Params& p, int c) {
+    if (EPI == kEpiSwiglu) {
+        const int n0 = t.n_blk * (BN / 2);
+        return (c < 2) ? n0 + 64 * c : p.I + n0 + 64 * (c - 2);
+    }
+    return t.n_blk * BN + 64 * c;
+}
+
+template <int EPI>
+__device__ __forceinline__ int b_col_pair(const Tile& t, const Params& p, uint32_t rank, int c, bool half) {
+    if (EPI == kEpiSwiglu) {
+        const int n0 = t.n_blk * (BN / 2);
+        if (half) return (c == 0 ? 0 : p.I) + n0 + 64 * (int)rank;
+        return (rank == 0 ? n0 : p.I + n0) + 64 * c;
+    }
+    return t.n_blk * BN + (int)rank * 128 + 64 * c;
+}
+
 // Writes NC (32 or 64) values of each lane's row -- lane = row of the warp's
 // 32-row group -- as bf16 to rows [0, nvalid) at dst (row stride ld elements),
 // through the warp's staging buffer: each lane writes its row into shared
@@ -361,28 +388,60 @@ __device__ __forceinline__ void swiglu_bwd32(const float* dh, const Aux32& a, ui
     }
 }
 
-// Epilogue of one tile for one epilogue warp. The warp owns rows
-// [warp_r0, warp_r0 + 32) of the tile and one half of its columns (col_half);
-// lane `lane` reads TMEM lane row t_row (its accumulator row). For group-M the
-// rows count from the tile's first row, and only rows inside the expert's
-// block are written. For group-K they count from the first output row of the
-// M block.
+// The part of a tile's accumulator that one epilogue warp writes out: rows
+// [r0, r0 + 32) of the tile (lane = row) and `chunks` 32-column chunks from
+// tile column c_lo (SwiGLU forward: columns of h). Column c of the part sits
+// at TMEM column tm + (c - c_lo) of the warp's lane quarter; in the SwiGLU
+// forward the gate value sits there and the matching up value `up` columns
+// further on.
+struct EpiMap {
+    int r0, c_lo, chunks, tm, up;
+};
+
+// A 128-lane accumulator (single-CTA tiles, 256-row pair tiles): lane i holds
+// row i; the two warps of a lane quarter split the columns in halves. SwiGLU
+// forward: gate in columns [0, 128), up in [128, 256).
+template <int EPI>
+__device__ __forceinline__ EpiMap full_map(int warp_r0, int col_half) {
+    if (EPI == kEpiSwiglu) return EpiMap{warp_r0, 64 * col_half, 2, 64 * col_half, BN / 2};
+    return EpiMap{warp_r0, 128 * col_half, 4, 128 * col_half, 0};
+}
+
+// A 128-row pair tile (M = 128 across the two CTAs): each CTA's accumulator
+// holds its 64 rows twice over -- tile columns [0, 128) in lanes 0..63 and
+// [128, 256) in lanes 64..127, both at TMEM columns 0..127. Quarter q thus
+// holds rows 32 * (q & 1) .. +31 (from the CTA's first row) of column half
+// q >> 1. The SwiGLU forward loads its B columns as [gate 64 | up 64] per CTA,
+// so a lane holds 64 gate columns at TMEM 0..63 and their up values at 64..127.
+template <int EPI>
+__device__ __forceinline__ EpiMap half_map(uint32_t rank, int quarter, int col_half) {
+    const int r0 = 64 * (int)rank + 32 * (quarter & 1);
+    if (EPI == kEpiSwiglu) return EpiMap{r0, 64 * (quarter >> 1) + 32 * col_half, 1, 32 * col_half, 64};
+    return EpiMap{r0, 128 * (quarter >> 1) + 64 * col_half, 2, 64 * col_half, 0};
+}
+
+// Epilogue of one tile for one epilogue warp, on the part `em` of the
+// accumulator; t_row addresses TMEM column 0 of the tile's buffer in the warp's
+// lane quarter. For group-M the rows count from the tile's first row, and only
+// rows inside the expert's block are written. For group-K they count from the
+// first output row of the M block.
 template <int EPI, bool GROUP_K>
 __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, uint32_t t_row,
-                                              int warp_r0, int col_half, int lane, int n_tile,
+                                              const EpiMap& em, int lane, int n_tile,
                                               uint8_t* buf, const CUtensorMap* tmC,
                                               const CUtensorMap* tmC2, Aux32* pre) {
+    const int warp_r0 = em.r0;
     const int r = warp_r0 + lane;
     if (EPI == kEpiSwiglu) {
-        // accumulator columns: gate [0, 128), up [128, 256); this warp: h columns
-        // [64 * col_half, 64 * col_half + 64) of the tile
         const int n0 = t.n_blk * (n_tile / 2);
         const int nvalid = min(max(t.rows - warp_r0, 0), 32);
         const int64_t row0 = (int64_t)t.row0 + warp_r0;
 #pragma unroll 1
-        for (int c0 = 64 * col_half; c0 < 64 * col_half + 64; c0 += 32) {
+        for (int i = 0; i < em.chunks; ++i) {
+            const int c0 = em.c_lo + 32 * i;
+            const uint32_t tc = t_row + (uint32_t)(em.tm + 32 * i);
             float g[32], u[32];
-            tmem_load_2x32(t_row + c0, t_row + BN / 2 + c0, g, u);
+            tmem_load_2x32(tc, tc + (uint32_t)em.up, g, u);
             if (n0 + c0 >= p.N) continue;
             if (p.out2) {
                 put_block32(buf, p.out2 + row0 * p.ldo2 + n0 + c0, p.ldo2, nvalid, g, lane, tmC2, n0 + c0,
@@ -404,10 +463,10 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
         const int64_t row0 = (int64_t)t.row0 + warp_r0;
         Aux32& ax = *pre;   // reloaded in place for each later chunk
 #pragma unroll 1
-        for (int c0 = 128 * col_half; c0 < 128 * col_half + 128; c0 += 32) {
-            const int col = n0 + c0;
+        for (int ci = 0; ci < em.chunks; ++ci) {
+            const int col = n0 + em.c_lo + 32 * ci;
             float dh[32];
-            tmem_load_32(t_row + c0, dh);
+            tmem_load_32(t_row + (uint32_t)(em.tm + 32 * ci), dh);
             if (col >= p.N) continue;
             uint32_t dgp[16], dup[16];
             if (valid) {
@@ -417,7 +476,7 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
                 for (int i = 0; i < 16; ++i) dgp[i] = dup[i] = 0u;   // rows past the block: not stored
             }
             // the next chunk's g and u load while this chunk is stored
-            load_aux32(p, grow, col + 32, valid && c0 + 32 < 128 * col_half + 128 && col + 32 < p.N, ax);
+            load_aux32(p, grow, col + 32, valid && ci + 1 < em.chunks && col + 32 < p.N, ax);
             put_block32_packed(buf, p.out + row0 * p.ldo + col, p.ldo, nvalid, dgp, lane, tmC, col, (int)row0);
             put_block32_packed(buf, p.out + row0 * p.ldo + p.I + col, p.ldo, nvalid, dup, lane, tmC, p.I + col,
                                (int)row0);
@@ -429,10 +488,10 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
         const int n0 = t.n_blk * n_tile;
         const int m0 = t.m_blk * BM1 + warp_r0;
 #pragma unroll 1
-        for (int c0 = 128 * col_half; c0 < 128 * col_half + 128; c0 += 32) {
+        for (int c0 = em.c_lo; c0 < em.c_lo + 32 * em.chunks; c0 += 32) {
             float v[32];
             if (t.num_kb > 0) {
-                tmem_load_32(t_row + c0, v);
+                tmem_load_32(t_row + (uint32_t)(em.tm + c0 - em.c_lo), v);
             } else {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = 0.0f;
@@ -466,10 +525,11 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
             row0 = p.out + ((int64_t)t.row0 + warp_r0) * p.ldo;
         }
 #pragma unroll 1
-        for (int c0 = 128 * col_half; c0 < 128 * col_half + 128; c0 += 64) {
+        for (int c0 = em.c_lo; c0 < em.c_lo + 32 * em.chunks; c0 += 64) {
             float v[64];
             if (t.num_kb > 0) {
-                tmem_load_2x32(t_row + c0, t_row + c0 + 32, *reinterpret_cast<float(*)[32]>(v),
+                const uint32_t tc = t_row + (uint32_t)(em.tm + c0 - em.c_lo);
+                tmem_load_2x32(tc, tc + 32, *reinterpret_cast<float(*)[32]>(v),
                                *reinterpret_cast<float(*)[32]>(v + 32));
             } else {
 #pragma unroll
@@ -488,9 +548,10 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
 // ===================================================================== pair
 template <int EPI, bool B_MN>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmC2,
-                     const Params p) {
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA64,
+                     const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmC,
+                     const __grid_constant__ CUtensorMap tmC2, const Params p) {
+    static_assert(EPI != kEpiSwiglu || B_MN, "the SwiGLU forward reads its weight N-major");
     extern __shared__ uint8_t smem_raw[];
     SmemP& s = *reinterpret_cast<SmemP*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                          ~uintptr_t(1023));
@@ -513,6 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         s.abort = 0;
         fence_mbar_init();
         prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmA64);
         prefetch_tensormap(&tmB);
     }
     if (warp == 1) {
@@ -535,6 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int id = cluster; id < total && ok; id += clusters) {
                 const Tile t = decode_tile<false>(s, p, id, BMP);
+                const bool half = t.rows <= 128;   // M = 128 across the pair: 64 rows per CTA
                 for (int kb = 0; kb < t.num_kb; ++kb) {
                     if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag, p.err)) {
                         ok = false;
@@ -543,20 +606,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t* a_s = s.stage[stage];
                     uint8_t* b_s = s.stage[stage] + kStageAP;
                     const uint32_t bar = mapa_shared(smem_u32(&s.full[stage]), 0);
-                    if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], 2 * kStageP);
-                    tma_load_2d_pair_hint(&tmA, bar, a_s, kb * BK, t.row0 + (int)rank * 128, keep);
+                    if (rank == 0) mbar_arrive_expect_tx(&s.full[stage], 2 * (half ? kStageHalfP : kStageP));
+                    if (half)
+                        tma_load_2d_pair_hint(&tmA64, bar, a_s, kb * BK, t.row0 + (int)rank * 64, keep);
+                    else
+                        tma_load_2d_pair_hint(&tmA, bar, a_s, kb * BK, t.row0 + (int)rank * 128, keep);
                     if (B_MN) {
 #pragma unroll
-                        for (int c = 0; c < 2; ++c) {
-                            int col;
-                            if (EPI == kEpiSwiglu) {
-                                const int n0 = t.n_blk * (BN / 2);
-                                col = (rank == 0 ? n0 : p.I + n0) + 64 * c;
-                            } else {
-                                col = t.n_blk * BN + (int)rank * 128 + 64 * c;
-                            }
-                            tma_load_3d_pair(&tmB, bar, b_s + c * kChunkBytes, col, kb * BK, t.g);
-                        }
+                        for (int c = 0; c < 2; ++c)
+                            tma_load_3d_pair(&tmB, bar, b_s + c * kChunkBytes, b_col_pair<EPI>(t, p, rank, c, half),
+                                             kb * BK, t.g);
                     } else {
                         tma_load_3d_pair(&tmB, bar, b_s, kb * BK, t.n_blk * BN + (int)rank * 128,
                                          t.g);
@@ -576,7 +635,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer (leader)
         if (rank == 0) {
-            constexpr uint32_t idesc = instr_desc<BMP, BN, false, B_MN>();
+            constexpr uint32_t idesc_full = instr_desc<BMP, BN, false, B_MN>();
+            constexpr uint32_t idesc_half = instr_desc<128, BN, false, B_MN>();
             int stage = 0;
             uint32_t phase = 0;
             int local_tile = 0;
@@ -589,6 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!mbar_wait_cluster(&s.acc_empty[buf], (use & 1u) ^ 1u, abort_flag, p.err)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
+                const uint32_t idesc = t.rows <= 128 ? idesc_half : idesc_full;
                 for (int kb = 0; kb < t.num_kb; ++kb) {
                     if (!mbar_wait(&s.full[stage], phase, abort_flag, p.err)) {
                         ok = false;
@@ -628,7 +689,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------ epilogue (both CTAs)
         const int quarter = warp & 3;                           // TMEM lanes 32*quarter .. +31
         const int col_half = (warp - 2) / 4;
-        const int warp_r0 = (int)rank * 128 + quarter * 32;    // first row of the 256-row tile
+        const EpiMap em_full = full_map<EPI>((int)rank * 128 + quarter * 32, col_half);
+        const EpiMap em_half = half_map<EPI>(rank, quarter, col_half);
         const uint32_t leader_acc_empty[2] = {mapa_shared(smem_u32(&s.acc_empty[0]), 0),
                                               mapa_shared(smem_u32(&s.acc_empty[1]), 0)};
         int local_tile = 0;
@@ -636,15 +698,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const Tile t = decode_tile<false>(s, p, id, BMP);
             const int buf = local_tile & 1;
             const uint32_t use = (uint32_t)(local_tile >> 1);
+            const EpiMap& em = t.rows <= 128 ? em_half : em_full;
             Aux32 pre;
             if (EPI == kEpiSwigluBwd) {
-                const int col = t.n_blk * BN + 128 * col_half;
-                load_aux32(p, (int64_t)t.row0 + warp_r0 + lane, col, warp_r0 + lane < t.rows && col < p.N, pre);
+                const int col = t.n_blk * BN + em.c_lo;
+                load_aux32(p, (int64_t)t.row0 + em.r0 + lane, col, em.r0 + lane < t.rows && col < p.N, pre);
             }
             if (!mbar_wait(&s.acc_full[buf], use & 1u, abort_flag, p.err)) break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-            epilogue_tile<EPI, false>(p, t, t_row, warp_r0, col_half, lane, BN, s.epi[warp - 2],
+            epilogue_tile<EPI, false>(p, t, t_row, em, lane, BN, s.epi[warp - 2],
                                       p.tma_out ? &tmC : nullptr, p.tma_out2 ? &tmC2 : nullptr, &pre);
             tc_fence_before();
             __syncwarp();
@@ -732,16 +795,9 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
                         tma_load_2d_hint(&tmA, bar, a_s, kb * BK, t.row0, keep);
                         if (B_MN) {
 #pragma unroll
-                            for (int c = 0; c < 4; ++c) {
-                                int col;
-                                if (EPI == kEpiSwiglu) {
-                                    const int n0 = t.n_blk * (BN / 2);
-                                    col = (c < 2) ? n0 + 64 * c : p.I + n0 + 64 * (c - 2);
-                                } else {
-                                    col = t.n_blk * BN + 64 * c;
-                                }
-                                tma_load_3d(&tmB, bar, b_s + c * kChunkBytes, col, kb * BK, t.g);
-                            }
+                            for (int c = 0; c < 4; ++c)
+                                tma_load_3d(&tmB, bar, b_s + c * kChunkBytes, b_col_1cta<EPI>(t, p, c), kb * BK,
+                                            t.g);
                         } else {
                             tma_load_3d(&tmB, bar, b_s, kb * BK, t.n_blk * BN, t.g);
                         }
@@ -830,6 +886,7 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
         const int quarter = warp & 3;               // TMEM lanes 32*quarter .. +31
         const int col_half = (warp - 2) / 4;
         const int warp_r0 = quarter * 32;           // first tile row of this warp
+        const EpiMap em = full_map<EPI>(warp_r0, col_half);
         int local_tile = 0;
         for (int id = blockIdx.x; id < total; id += gridDim.x, ++local_tile) {
             const Tile t = decode_tile<GROUP_K>(s, p, id, BM1);
@@ -837,13 +894,13 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
             const uint32_t use = (uint32_t)(local_tile >> 1);
             Aux32 pre;
             if (EPI == kEpiSwigluBwd) {
-                const int col = t.n_blk * BN + 128 * col_half;
+                const int col = t.n_blk * BN + em.c_lo;
                 load_aux32(p, (int64_t)t.row0 + warp_r0 + lane, col, warp_r0 + lane < t.rows && col < p.N, pre);
             }
             if (!mbar_wait(&s.acc_full[buf], use & 1u, abort_flag, p.err)) break;
             tc_fence_after();
             const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-            epilogue_tile<EPI, GROUP_K>(p, t, t_row, warp_r0, col_half, lane, BN, s.epi[warp - 2],
+            epilogue_tile<EPI, GROUP_K>(p, t, t_row, em, lane, BN, s.epi[warp - 2],
                                         p.tma_out ? &tmC : nullptr, p.tma_out2 ? &tmC2 : nullptr, &pre);
             tc_fence_before();
             mbar_arrive(&s.acc_empty[buf]);
@@ -1299,7 +1356,7 @@ cudaError_t set_smem_once(K kern, size_t bytes, std::once_flag& once, cudaError_
 }
 
 template <int EPI, bool B_MN>
-cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const Params& p,
+cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& a64, const CUtensorMap& b, const Params& p,
                         int64_t max_tiles, cudaStream_t st, const CUtensorMap* c = nullptr,
                         const CUtensorMap* c2 = nullptr) {
     auto kern = gemm_pair_kernel<EPI, B_MN>;
@@ -1326,7 +1383,7 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const Params
     Params q = p;
     q.tma_out = c != nullptr;
     q.tma_out2 = c2 != nullptr;
-    return cudaLaunchKernelEx(&cfg, kern, a, b, c ? *c : unused, c2 ? *c2 : unused, q);
+    return cudaLaunchKernelEx(&cfg, kern, a, a64, b, c ? *c : unused, c2 ? *c2 : unused, q);
 }
 
 template <int EPI, bool A_MN, bool B_MN, bool GROUP_K>
@@ -1403,12 +1460,11 @@ int64_t single_tile_bound(int64_t rows, int groups, int n_blocks) {
     return ((rows + BM1 - 1) / BM1 + groups) * (int64_t)n_blocks;
 }
 
-// Pair tiles (256 rows) halve each CTA's weight traffic but round every
-// expert block up to 256 rows; single tiles round up to 128. The expected
-// rounding waste is about half a tile per expert, so pair tiles pay off once
-// the average block is large compared with a tile: measured on B200, they were
-// faster at 1024 rows per expert (Mixtral-8x7B shape) and slower at 256
-// (Qwen3-30B-A3B shape).
+// Pair tiles (256 rows) halve each CTA's weight traffic; an expert block's
+// last <= 128 rows run as a 128-row pair tile, so both kinds round a block up
+// to a multiple of 128 rows. Measured on B200, pair tiles were faster at 1024
+// rows per expert (Mixtral-8x7B shape) and slower at 256 (Qwen3-30B-A3B shape,
+// 259 against 242 us for gate_up).
 // MOE_GEMM_TILES=pair|single overrides the choice (used by the tests to run
 // both kernels on the same shapes).
 bool use_pair_tiles(int64_t rows, int groups) {
@@ -1418,14 +1474,16 @@ bool use_pair_tiles(int64_t rows, int groups) {
     return groups == 1 || rows >= (int64_t)groups * 1024;
 }
 
-// Group-M GEMM on pair or single tiles. `tb_pair` and `tb_single` are the B
-// maps for each (their K-major boxes differ: 128 or 256 rows of N).
+// Group-M GEMM on pair or single tiles. `ta` and `ta64` are A maps with
+// 128- and 64-row boxes (pair tiles of 256 and of 128 rows); `tb_pair` and
+// `tb_single` are the B maps for each kernel (their K-major boxes differ: 128
+// or 256 rows of N).
 template <int EPI, bool B_MN>
-cudaError_t launch_group_m(const CUtensorMap& ta, const CUtensorMap& tb_pair,
+cudaError_t launch_group_m(const CUtensorMap& ta, const CUtensorMap& ta64, const CUtensorMap& tb_pair,
                            const CUtensorMap& tb_single, const Params& p, cudaStream_t st,
                            const CUtensorMap* out_map, const CUtensorMap* out2_map = nullptr) {
     if (use_pair_tiles(p.rows, p.groups))
-        return launch_pair<EPI, B_MN>(ta, tb_pair, p, pair_tile_bound(p.rows, p.groups, p.n_blocks), st,
+        return launch_pair<EPI, B_MN>(ta, ta64, tb_pair, p, pair_tile_bound(p.rows, p.groups, p.n_blocks), st,
                                       out_map, out2_map);
     return launch_1cta<EPI, false, B_MN, false>(ta, tb_single, p,
                                                 single_tile_bound(p.rows, p.groups, p.n_blocks), st,
@@ -1443,8 +1501,9 @@ cudaError_t gemm_gate_up_swiglu(const bf16* x, int64_t rows, const int32_t* offs
                                 int I, const bf16* w_gate_up, bf16* h, bf16* gu_save,
                                 cudaStream_t st, unsigned* err) {
     if (rows == 0) return cudaSuccess;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, ta64, tb;
     if (!make_map_2d(&ta, x, H, rows, H, BK, 128)) return cudaErrorInvalidValue;
+    if (!make_map_2d(&ta64, x, H, rows, H, BK, 64)) return cudaErrorInvalidValue;
     if (!make_map_3d(&tb, w_gate_up, 2 * (uint64_t)I, H, offsets ? E : 1, 64, BK))
         return cudaErrorInvalidValue;
     const int groups = offsets ? E : 1;
@@ -1460,14 +1519,15 @@ cudaError_t gemm_gate_up_swiglu(const bf16* x, int64_t rows, const int32_t* offs
     CUtensorMap tc, tc2;
     if (!make_out_map(&tc, h, rows, I)) return cudaErrorInvalidValue;
     if (gu_save && !make_out_map(&tc2, gu_save, rows, 2 * (uint64_t)I)) return cudaErrorInvalidValue;
-    return launch_group_m<kEpiSwiglu, true>(ta, tb, tb, p, st, &tc, gu_save ? &tc2 : nullptr);
+    return launch_group_m<kEpiSwiglu, true>(ta, ta64, tb, tb, p, st, &tc, gu_save ? &tc2 : nullptr);
 }
 
 cudaError_t gemm_down(const bf16* h, int64_t rows, const int32_t* offsets, int E, int H, int I,
                       const bf16* w_down, bf16* y, cudaStream_t st, unsigned* err) {
     if (rows == 0) return cudaSuccess;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, ta64, tb;
     if (!make_map_2d(&ta, h, I, rows, I, BK, 128)) return cudaErrorInvalidValue;
+    if (!make_map_2d(&ta64, h, I, rows, I, BK, 64)) return cudaErrorInvalidValue;
     if (!make_map_3d(&tb, w_down, H, I, offsets ? E : 1, 64, BK)) return cudaErrorInvalidValue;
     const int groups = offsets ? E : 1;
     Params p = base_params(groups, rows, offsets, err);
@@ -1478,15 +1538,16 @@ cudaError_t gemm_down(const bf16* h, int64_t rows, const int32_t* offsets, int E
     p.ldo = H;
     CUtensorMap tc;
     if (!make_out_map(&tc, y, rows, H)) return cudaErrorInvalidValue;
-    return launch_group_m<kEpiStore, true>(ta, tb, tb, p, st, &tc);
+    return launch_group_m<kEpiStore, true>(ta, ta64, tb, tb, p, st, &tc);
 }
 
 cudaError_t gemm_down_dgrad_swiglu(const bf16* dy, int64_t rows, const int32_t* offsets, int E,
                                    int H, int I, const bf16* w_down, const bf16* gu, bf16* dgu,
                                    cudaStream_t st, unsigned* err) {
     if (rows == 0) return cudaSuccess;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, ta64, tb;
     if (!make_map_2d(&ta, dy, H, rows, H, BK, 128)) return cudaErrorInvalidValue;
+    if (!make_map_2d(&ta64, dy, H, rows, H, BK, 64)) return cudaErrorInvalidValue;
     // B[n = i][k = h] = w_down[e][i][h]: K-major, box 64 (h) x 128 (i) per CTA of a
     // pair, 64 x 256 for a single CTA
     CUtensorMap tb1;
@@ -1503,15 +1564,17 @@ cudaError_t gemm_down_dgrad_swiglu(const bf16* dy, int64_t rows, const int32_t* 
     p.ld_aux = 2 * (int64_t)I;
     CUtensorMap tc;
     if (!make_out_map(&tc, dgu, rows, 2 * (uint64_t)I)) return cudaErrorInvalidValue;
-    return launch_group_m<kEpiSwigluBwd, false>(ta, tb, tb1, p, st, &tc);
+    return launch_group_m<kEpiSwigluBwd, false>(ta, ta64, tb, tb1, p, st, &tc);
 }
 
 cudaError_t gemm_gate_up_dgrad(const bf16* dgu, int64_t rows, const int32_t* offsets, int E, int H,
                                int I, const bf16* w_gate_up, bf16* dx_perm, cudaStream_t st,
                                unsigned* err) {
     if (rows == 0) return cudaSuccess;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, ta64, tb;
     if (!make_map_2d(&ta, dgu, 2 * (uint64_t)I, rows, 2 * (uint64_t)I, BK, 128))
+        return cudaErrorInvalidValue;
+    if (!make_map_2d(&ta64, dgu, 2 * (uint64_t)I, rows, 2 * (uint64_t)I, BK, 64))
         return cudaErrorInvalidValue;
     // B[n = h][k = c] = w_gate_up[e][h][c]: K-major, box 64 (c) x 128 (h) per CTA of a
     // pair, 64 x 256 for a single CTA
@@ -1526,7 +1589,7 @@ cudaError_t gemm_gate_up_dgrad(const bf16* dgu, int64_t rows, const int32_t* off
     p.ldo = H;
     CUtensorMap tc;
     if (!make_out_map(&tc, dx_perm, rows, H)) return cudaErrorInvalidValue;
-    return launch_group_m<kEpiStore, false>(ta, tb, tb1, p, st, &tc);
+    return launch_group_m<kEpiStore, false>(ta, ta64, tb, tb1, p, st, &tc);
 }
 
 cudaError_t gemm_wgrad(const bf16* X, const bf16* D, int64_t rows, const int32_t* offsets, int E,

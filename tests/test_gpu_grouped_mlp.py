@@ -91,3 +91,34 @@ def test_rows_past_offsets_end_are_untouched():
     assert torch.all(y[200:].float() == 7.0)
     ref = oracle.grouped_mlp(bits(x), offsets.cpu().numpy(), bits(wgu), bits(wd))
     assert_close(y[:200], ref[:200], "y_perm")
+
+
+@pytest.mark.parametrize("tiles", ["single", "pair"])
+def test_block_sizes_around_tile_edges(tiles, monkeypatch):
+    """Expert blocks of 0, 1, 63, 64, 65, 127, 128, 129, 255, 256, 257 and
+    385 rows: every split of a block into 256-row pair tiles plus a last
+    128-row pair tile (one CTA's 64 rows empty or not), and into 128-row
+    single tiles, with g, u and h checked as well as y."""
+    import routing_grouped_gemm_score_b200 as m
+    monkeypatch.setenv("MOE_GEMM_TILES", tiles)
+    sizes = [0, 1, 63, 64, 65, 127, 128, 129, 255, 256, 257, 385]
+    E, H, I = len(sizes), 192, 320
+    offs = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    A = int(offs[-1])
+    g_ = torch.Generator(device="cuda").manual_seed(11)
+    x = torch.randn((A, H), generator=g_, device="cuda").to(torch.bfloat16)
+    wgu = (torch.randn((E, H, 2 * I), generator=g_, device="cuda") / H ** 0.5).to(torch.bfloat16)
+    wd = (torch.randn((E, I, H), generator=g_, device="cuda") / I ** 0.5).to(torch.bfloat16)
+    out = m.moe_grouped_mlp(x, torch.from_numpy(offs).cuda(), wgu, wd, save=True)
+    torch.cuda.synchronize()
+    assert m.moe_get_device_status() == 0
+    xb, wgub, wdb = bits(x), bits(wgu), bits(wd)
+    assert_close(out["y_perm"], oracle.grouped_mlp(xb, offs, wgub, wdb, round_bf16=True), "y_perm")
+    for e in range(E):
+        r0, r1 = offs[e], offs[e + 1]
+        if r1 == r0:
+            continue
+        y, g, u, h = oracle.expert_mlp(xb[r0:r1], wgub[e], wdb[e], round_bf16=True, want_intermediates=True)
+        assert_close(out["gu"][r0:r1, :I], g, f"g of expert {e}")
+        assert_close(out["gu"][r0:r1, I:], u, f"u of expert {e}")
+        assert_close(out["h"][r0:r1], h, f"h of expert {e}")
