@@ -533,53 +533,83 @@ def e2e_measure(args, w, d, m, opts, ws, world):
     """Same metric through the public calls with host buffers: every step
     copies its inputs (logits, x, and dout for a training step) from pinned
     host memory to the device and reads the step's result back (the layer
-    output, or dx for a training step), inside the timed region."""
+    output, or dx for a training step), inside the timed region.
+
+    The steps are pipelined the way a serving or training loop runs them: the
+    copy-in of step i+1 (one stream) and the read-back of step i-1 (another)
+    overlap the compute of step i, with two device slots for the inputs and
+    the result. Every step still moves all of its bytes inside the region."""
     import torch
     h_logits = d["logits"].cpu().pin_memory()
     h_x = d["x"].cpu().pin_memory()
     h_dout = d["dout"].cpu().pin_memory() if w.backward else None
-    h_res = torch.empty((w.T, w.H), dtype=torch.bfloat16).pin_memory()
-    dl = torch.empty_like(d["logits"])
-    dx = torch.empty_like(d["x"])
-    ddo = torch.empty_like(d["dout"]) if w.backward else None
-    out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device="cuda")
+    h_res = [torch.empty((w.T, w.H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    dl = [torch.empty_like(d["logits"]) for _ in range(2)]
+    dx = [torch.empty_like(d["x"]) for _ in range(2)]
+    ddo = [torch.empty_like(d["dout"]) for _ in range(2)] if w.backward else None
+    out = [torch.empty((w.T, w.H), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
     K = max(1, min(args.steps, 50))
     state = None
     grads = None
     if w.backward:
         _, state = m.moe_layer_forward(d["logits"], d["x"], d["w_gate_up"], d["w_down"], w.k, opts,
-                                       save_for_backward=True, workspace=ws, out=out)
-        grads = m.moe_grouped_mlp_backward(d["dout"], state, d["w_gate_up"], d["w_down"], ws)
+                                       save_for_backward=True, workspace=ws, out=out[0])
+        g0 = m.moe_grouped_mlp_backward(d["dout"], state, d["w_gate_up"], d["w_down"], ws)
+        # the weight gradients are consumed on the device; dx is read back, so it has two slots
+        grads = [dict(g0), dict(g0, dx=torch.empty_like(g0["dx"]))]
 
-    def step():
-        dl.copy_(h_logits, non_blocking=True)
-        dx.copy_(h_x, non_blocking=True)
-        if w.backward:
-            ddo.copy_(h_dout, non_blocking=True)
-        m.moe_layer_forward(dl, dx, d["w_gate_up"], d["w_down"], w.k, opts, d["shared_gate_up"],
-                            d["shared_down"], save_for_backward=w.backward, workspace=ws, out=out,
+    compute = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    in_ready = [ev(), ev()]      # the slot's inputs have landed
+    in_free = [ev(), ev()]       # the compute has finished reading the slot's inputs
+    res_ready = [ev(), ev()]     # the slot's result is complete
+    res_free = [ev(), ev()]      # the slot's result has been read back
+    for e in in_free + res_free:
+        e.record(compute)
+
+    def step(i):
+        b = i % 2
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(in_free[b])
+            dl[b].copy_(h_logits, non_blocking=True)
+            dx[b].copy_(h_x, non_blocking=True)
+            if w.backward:
+                ddo[b].copy_(h_dout, non_blocking=True)
+            in_ready[b].record(s_in)
+        compute.wait_event(in_ready[b])
+        compute.wait_event(res_free[b])
+        m.moe_layer_forward(dl[b], dx[b], d["w_gate_up"], d["w_down"], w.k, opts, d["shared_gate_up"],
+                            d["shared_down"], save_for_backward=w.backward, workspace=ws, out=out[b],
                             state=state)
         if w.backward:
-            m.moe_grouped_mlp_backward(ddo, state, d["w_gate_up"], d["w_down"], ws, grads)
-            h_res.copy_(grads["dx"], non_blocking=True)
-        else:
-            h_res.copy_(out, non_blocking=True)
+            m.moe_grouped_mlp_backward(ddo[b], state, d["w_gate_up"], d["w_down"], ws, grads[b])
+        in_free[b].record(compute)
+        res_ready[b].record(compute)
+        res = grads[b]["dx"] if w.backward else out[b]
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(res_ready[b])
+            h_res[b].copy_(res, non_blocking=True)
+            res_free[b].record(s_out)
 
-    for _ in range(2):
-        step()
+    for i in range(3):
+        step(i)
     torch.cuda.synchronize()
     barrier(world)
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record()
-    for _ in range(K):
-        step()
-    e.record()
+    s.record(compute)
+    s_in.wait_stream(compute)      # the first copy-in starts after the start event
+    for i in range(K):
+        step(i)
+    compute.wait_stream(s_out)     # the end event follows the last read-back
+    e.record(compute)
     torch.cuda.synchronize()
     ms = max_over_ranks(s.elapsed_time(e), world)
     h2d = h_logits.numel() * 4 + h_x.numel() * 2 + (h_dout.numel() * 2 if w.backward else 0)
     return {"value": w.T * world * K / (ms / 1e3), "unit": UNIT,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h_res.numel() * 2, "steps": K,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h_res[0].numel() * 2, "steps": K,
             "pass": "fwd+bwd" if w.backward else "fwd",
+            "pipelined": "copy-in of step i+1 and read-back of step i-1 overlap step i on two copy streams",
             "note": "weights resident on the device; the step's result read back is "
                     + ("dx" if w.backward else "the layer output")}
 
