@@ -46,6 +46,7 @@
 // error, every role leaves its loop, and TMEM is still freed.
 #include <cudaTypedefs.h>
 
+#include <cstddef>
 #include <cstdlib>
 #include <mutex>
 
@@ -101,7 +102,9 @@ struct Params {
 template <int STAGES, int STAGE_BYTES>
 struct __align__(1024) Smem {
     uint8_t stage[STAGES][STAGE_BYTES];
-    uint8_t epi[kEpiWarps][32 * 80];  // per epilogue warp: 32 rows x 32 bf16, rows padded to 80 B
+    // per epilogue warp: 32 rows x 32 bf16 (rows padded to 80 B for store_rows;
+    // a TMA block uses the first 2 KB), each on a 512-byte boundary
+    uint8_t epi[kEpiWarps][32 * 80];
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
     uint64_t ready[STAGES];   // group-K: the stage's ragged rows are zeroed
@@ -116,6 +119,8 @@ struct __align__(1024) Smem {
 };
 using Smem1 = Smem<STAGES1, kStage1>;
 using SmemP = Smem<STAGESP, kStageP>;
+static_assert(offsetof(Smem1, epi) % 512 == 0 && offsetof(SmemP, epi) % 512 == 0 && (32 * 80) % 512 == 0,
+              "64-byte-swizzled staging blocks start on 512-byte boundaries");
 constexpr size_t kSmem1Bytes = sizeof(Smem1) + 1024;  // + alignment slack
 constexpr size_t kSmemPBytes = sizeof(SmemP) + 1024;
 
@@ -246,6 +251,15 @@ __device__ __forceinline__ int b_col_pair(const Tile& t, const Params& p, uint32
     return t.n_blk * BN + (int)rank * 128 + 64 * c;
 }
 
+// Byte offset of 16-byte chunk q (0..3) of row r in a 32 x 64-byte staging
+// block that a TMA store reads through a 64-byte-swizzled tensor map: the
+// chunk index is XORed with address bits 7-8, (r >> 1) & 3 for a block on a
+// 512-byte boundary. The same permutation puts the eight rows that a
+// quarter-warp writes at once on eight different groups of four banks.
+__device__ __forceinline__ uint32_t stage64_off(int r, int q) {
+    return (uint32_t)(r * 64 + ((q ^ ((r >> 1) & 3)) << 4));
+}
+
 // Writes NC (32 or 64) values of each lane's row -- lane = row of the warp's
 // 32-row group -- as bf16 to rows [0, nvalid) at dst (row stride ld elements),
 // through the warp's staging buffer: each lane writes its row into shared
@@ -289,7 +303,7 @@ __device__ __forceinline__ void put_block32(uint8_t* buf, bf16* dst, int64_t ld,
     if (map != nullptr && nvalid == 32) {
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-            *reinterpret_cast<uint4*>(buf + lane * 64 + q * 16) =
+            *reinterpret_cast<uint4*>(buf + stage64_off(lane, q)) =
                 make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
                            pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
         fence_proxy_async_smem();
@@ -352,7 +366,7 @@ __device__ __forceinline__ void put_block32_packed(uint8_t* buf, bf16* dst, int6
     if (map != nullptr && nvalid == 32) {
 #pragma unroll
         for (int q = 0; q < 4; ++q)
-            *reinterpret_cast<uint4*>(buf + lane * 64 + q * 16) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+            *reinterpret_cast<uint4*>(buf + stage64_off(lane, q)) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
@@ -501,7 +515,7 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
             __syncwarp();
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-                *reinterpret_cast<uint4*>(buf + lane * 64 + q * 16) =
+                *reinterpret_cast<uint4*>(buf + stage64_off(lane, q)) =
                     make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
                                pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
             fence_proxy_async_smem();
@@ -988,6 +1002,7 @@ struct __align__(1024) SmemW {
 };
 constexpr size_t kSmemWBytes = sizeof(SmemW) + 1024;
 static_assert(kSmemWBytes <= 227 * 1024, "weight-gradient shared memory");
+static_assert(offsetof(SmemW, epi) % 512 == 0, "64-byte-swizzled staging blocks start on 512-byte boundaries");
 
 struct WgItem {
     int g, n_blk, m_begin, m_end;
@@ -1222,7 +1237,7 @@ __device__ void wg_epilogue(SmemW& s, const Params& p, int total, volatile int* 
                 __syncwarp();
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4*>(buf8 + lane * 64 + q * 16) = make_uint4(
+                    *reinterpret_cast<uint4*>(buf8 + stage64_off(lane, q)) = make_uint4(
                         pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
                         pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
                 fence_proxy_async_smem();
@@ -1492,7 +1507,7 @@ cudaError_t launch_group_m(const CUtensorMap& ta, const CUtensorMap& ta64, const
 
 // TMA store map of a row-major bf16 output [rows][cols]: 32 x 32 blocks, no swizzle.
 bool make_out_map(CUtensorMap* m, const bf16* out, int64_t rows, uint64_t cols) {
-    return make_map_2d(m, out, cols, (uint64_t)rows, cols, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE);
+    return make_map_2d(m, out, cols, (uint64_t)rows, cols, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 }  // namespace
@@ -1607,7 +1622,7 @@ cudaError_t gemm_wgrad(const bf16* X, const bf16* D, int64_t rows, const int32_t
     p.ldo = N;
     p.out_group_stride = (int64_t)M * N;
     CUtensorMap tc;   // dW [E][M][N], stored in 32 x 32 blocks without swizzle
-    if (!make_map_3d(&tc, dW, N, M, E > 0 ? E : 1, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (!make_map_3d(&tc, dW, N, M, E > 0 ? E : 1, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
     // One 128 x 256 tile per CTA at a time. MOE_WGRAD=panel runs the kernel
     // that keeps each expert's B rows in shared memory instead; on B200 it
