@@ -113,6 +113,155 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// Backward of the weighted combine, one warp per token (same definition as
+// above). The warp's lanes cover the row in 16-byte chunks, CH chunks per lane
+// per step, each with its k row loads issued together; the next token's
+// routing is loaded while the current token is processed. Each lane sums its
+// products for every j over its chunks in order, and a warp butterfly then
+// gives dprob; the order is fixed, so the result is the same on every run.
+template <int KB, int CH>
+__global__ void __launch_bounds__(128, KB > 8 ? 2 : 4)
+    combine_backward_warp_kernel(const uint4* __restrict__ dout, const uint4* __restrict__ y,
+                                 const int32_t* __restrict__ row_of, const float* __restrict__ probs,
+                                 int64_t T, int k, int H8, int64_t A, uint4* __restrict__ dy,
+                                 float* __restrict__ dprob, unsigned* err) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    int32_t r_next = -1;
+    float p_next = 0.0f;
+    if (t < T && lane < k) {
+        r_next = __ldg(row_of + t * k + lane);
+        p_next = __ldg(probs + t * k + lane);
+    }
+    for (; t < T; t += nwarps) {
+        int32_t r = r_next;
+        const float p = p_next;
+        if (lane < k && (r < 0 || r >= A)) {
+            raise_error(err, kErrDeviceCheck);
+            r = -1;
+        }
+        const int64_t tn = t + nwarps;   // the next token's routing, one token ahead
+        r_next = -1;
+        p_next = 0.0f;
+        if (tn < T && lane < k) {
+            r_next = __ldg(row_of + tn * k + lane);
+            p_next = __ldg(probs + tn * k + lane);
+        }
+        int64_t off[KB];   // first chunk of row j in y and dy; -1: no row
+        float ps[KB], dot[KB];
+#pragma unroll
+        for (int j = 0; j < KB; ++j) {
+            const int32_t rj = __shfl_sync(kFull, r, j);
+            off[j] = (j < k && rj >= 0) ? (int64_t)rj * H8 : -1;
+            ps[j] = __shfl_sync(kFull, p, j);
+            dot[j] = 0.0f;
+        }
+        const uint4* drow = dout + t * H8;
+        for (int c0 = 0; c0 < H8; c0 += 32 * CH) {
+            uint4 d[CH], v[CH][KB];
+#pragma unroll
+            for (int h = 0; h < CH; ++h) {
+                const int c = c0 + 32 * h + lane;
+                if (c < H8) d[h] = __ldg(drow + c);
+#pragma unroll
+                for (int j = 0; j < KB; ++j)
+                    if (off[j] >= 0 && c < H8) v[h][j] = __ldg(y + off[j] + c);
+            }
+#pragma unroll
+            for (int h = 0; h < CH; ++h) {
+                const int c = c0 + 32 * h + lane;
+                if (c >= H8) continue;
+#pragma unroll
+                for (int j = 0; j < KB; ++j) {
+                    if (off[j] < 0) continue;
+                    float sc[8];
+                    dot_and_scale(d[h], v[h][j], ps[j], dot[j], sc);
+                    dy[off[j] + c] = pack8(sc);
+                }
+            }
+        }
+        float mine = 0.0f;
+#pragma unroll
+        for (int j = 0; j < KB; ++j) {
+            float v = dot[j];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+            if (lane == j) mine = v;
+        }
+        if (lane < k) dprob[t * k + lane] = mine;
+    }
+}
+
+// Combine, one warp per token: the warp's lanes cover the output row in
+// 16-byte chunks, CH chunks per lane per step, each with its k row loads (and
+// the shared row's chunk) issued together; the next token's routing is loaded
+// while the current token is summed. The sum runs in the fixed order of the
+// other combine kernels: shared first, then j ascending, fp32.
+template <int KB, int CH>
+__global__ void __launch_bounds__(128, KB > 8 ? 2 : 4)
+    combine_warp_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ row_of,
+                        const float* __restrict__ probs, int64_t T, int k, int H8, int64_t A,
+                        const uint4* __restrict__ shared, uint4* __restrict__ out, unsigned* err) {
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    int32_t r_next = -1;
+    float p_next = 1.0f;
+    if (t < T && lane < k) {
+        r_next = __ldg(row_of + t * k + lane);
+        if (probs) p_next = __ldg(probs + t * k + lane);
+    }
+    for (; t < T; t += nwarps) {
+        int32_t r = r_next;
+        const float p = p_next;
+        if (lane < k && (r < 0 || r >= A)) {
+            raise_error(err, kErrDeviceCheck);
+            r = -1;
+        }
+        const int64_t tn = t + nwarps;   // the next token's routing, one token ahead
+        r_next = -1;
+        p_next = 1.0f;
+        if (tn < T && lane < k) {
+            r_next = __ldg(row_of + tn * k + lane);
+            if (probs) p_next = __ldg(probs + tn * k + lane);
+        }
+        int64_t off[KB];   // first chunk of row j in y; -1: no row
+        float ps[KB];
+#pragma unroll
+        for (int j = 0; j < KB; ++j) {
+            const int32_t rj = __shfl_sync(kFull, r, j);
+            off[j] = (j < k && rj >= 0) ? (int64_t)rj * H8 : -1;
+            ps[j] = __shfl_sync(kFull, p, j);
+        }
+        for (int c0 = 0; c0 < H8; c0 += 32 * CH) {
+            uint4 v[CH][KB], sh[CH];
+#pragma unroll
+            for (int h = 0; h < CH; ++h) {
+                const int c = c0 + 32 * h + lane;
+                if (c >= H8) continue;
+                if (shared) sh[h] = __ldg(shared + t * H8 + c);
+#pragma unroll
+                for (int j = 0; j < KB; ++j)
+                    if (off[j] >= 0) v[h][j] = __ldg(y + off[j] + c);
+            }
+#pragma unroll
+            for (int h = 0; h < CH; ++h) {
+                const int c = c0 + 32 * h + lane;
+                if (c >= H8) continue;
+                float acc[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
+                if (shared) add_scaled(acc, sh[h], 1.0f);
+#pragma unroll
+                for (int j = 0; j < KB; ++j)
+                    if (off[j] >= 0) add_scaled(acc, v[h][j], ps[j]);
+                out[t * H8 + c] = pack8(acc);
+            }
+        }
+    }
+}
+
 // Combine over contiguous token ranges, on plain 16-byte loads. A block owns
 // tokens [t_begin, t_end). Its threads stage the range's source rows and
 // weights in shared memory (kStageTokens at a time, one coalesced load), so no
@@ -215,11 +364,25 @@ cudaError_t launch_combine(const bf16* y_perm, const int32_t* row_of, const floa
                            cudaStream_t st, unsigned* err) {
     if (T == 0) return cudaSuccess;
     const int H8 = H / 8;
-    // Register path for few rows per token, bulk copies otherwise. Measured on
-    // B200 (isolated, fraction of HBM): k=2, H=4096: 0.75 here against 0.63;
-    // k=8, H=2048: 0.46 here against 0.66. MOE_COMBINE=bulk|regs overrides.
     const char* force = getenv("MOE_COMBINE");
-    const bool regs = force ? (force[0] == 'r' && H8 <= 512) : (k <= 2 && H8 <= 512);
+    if (!force || force[0] == 'w') {
+        auto kern = k <= 2 ? combine_warp_kernel<2, 4>
+                  : k <= 4 ? combine_warp_kernel<4, 2>
+                  : k <= 8 ? combine_warp_kernel<8, 2> : combine_warp_kernel<16, 1>;
+        constexpr int kThreadsW = 128;
+        int per_sm = 1;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreadsW, 0) != cudaSuccess || per_sm < 1)
+            per_sm = 1;
+        const int64_t cap = (int64_t)sm_count() * per_sm * (kThreadsW / 32);
+        const int64_t warps = T < cap ? T : cap;
+        const int64_t blocks = (warps + kThreadsW / 32 - 1) / (kThreadsW / 32);
+        kern<<<(unsigned)blocks, kThreadsW, 0, st>>>(reinterpret_cast<const uint4*>(y_perm), row_of, probs, T, k, H8,
+                                                    A, reinterpret_cast<const uint4*>(shared),
+                                                    reinterpret_cast<uint4*>(out), err);
+        return cudaGetLastError();
+    }
+    // MOE_COMBINE=regs|bulk: the token-range register kernel or the bulk-copy one
+    const bool regs = force[0] == 'r' && H8 <= 512;
     if (regs) {
         const int threads = (H8 + 31) / 32 * 32;
         // blocks resident per SM for this kernel and block size
@@ -246,9 +409,24 @@ cudaError_t launch_combine_backward(const bf16* dout, const bf16* y_perm, const 
                                     const float* probs, int64_t T, int k, int H, int64_t A,
                                     bf16* dy_perm, float* dprob, cudaStream_t st, unsigned* err) {
     if (T == 0) return cudaSuccess;
-    // The register-path kernel below measured faster than the bulk-copy one
-    // (rows_combine_backward) at the Qwen3-30B-A3B shape, so it is the one used.
-    combine_backward_kernel<<<(unsigned)row_blocks(T), row_threads(H / 8), 0, st>>>(
+    const char* force = getenv("MOE_COMBINE_BWD");
+    if (force && force[0] == 'b') {
+        combine_backward_kernel<<<(unsigned)row_blocks(T), row_threads(H / 8), 0, st>>>(
+            reinterpret_cast<const uint4*>(dout), reinterpret_cast<const uint4*>(y_perm), row_of, probs,
+            T, k, H / 8, A, reinterpret_cast<uint4*>(dy_perm), dprob, err);
+        return cudaGetLastError();
+    }
+    auto kern = k <= 2 ? combine_backward_warp_kernel<2, 2>
+              : k <= 4 ? combine_backward_warp_kernel<4, 2>
+              : k <= 8 ? combine_backward_warp_kernel<8, 2> : combine_backward_warp_kernel<16, 1>;
+    constexpr int kThreadsW = 128;
+    int per_sm = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreadsW, 0) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
+    const int64_t warps = (T < (int64_t)sm_count() * per_sm * (kThreadsW / 32)) ? T
+                                                                               : (int64_t)sm_count() * per_sm * (kThreadsW / 32);
+    const int64_t blocks = (warps + kThreadsW / 32 - 1) / (kThreadsW / 32);
+    kern<<<(unsigned)blocks, kThreadsW, 0, st>>>(
         reinterpret_cast<const uint4*>(dout), reinterpret_cast<const uint4*>(y_perm), row_of, probs,
         T, k, H / 8, A, reinterpret_cast<uint4*>(dy_perm), dprob, err);
     return cudaGetLastError();

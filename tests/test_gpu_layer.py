@@ -94,10 +94,31 @@ def test_backward_on_oracle_state(name, tiles, wgrad, monkeypatch):
     in accumulation order; dW_gate_up and dx also carry the bf16 rounding of
     dg, du and each token row's dx, whose fp32 and fp64 pre-images can round
     apart (assert_close_flips)."""
-    import routing_grouped_gemm_score_b200 as m
     monkeypatch.setenv("MOE_GEMM_TILES", tiles)
     monkeypatch.setenv("MOE_WGRAD", wgrad)   # weight gradient: B panel in shared memory, or one tile per CTA
-    w = SMALL[name]
+    _check_backward_on_oracle_state(name, SMALL[name])
+
+
+COMBINE_BWD = {
+    "k1": wl.WORKLOADS["qwen3_30b_a3b"].scaled(T=160, H=192, I=128, E=16, k=1),
+    "k3": wl.WORKLOADS["qwen3_30b_a3b"].scaled(T=150, H=192, I=128, E=8, k=3),
+    "k8": wl.WORKLOADS["qwen3_30b_a3b"].scaled(T=256, H=2112, I=128, E=32),
+    "k16": wl.WORKLOADS["qwen3_30b_a3b"].scaled(T=200, H=256, I=128, E=32, k=16),
+}
+
+
+@pytest.mark.parametrize("kernel", ["block", "warp"])
+@pytest.mark.parametrize("name", list(COMBINE_BWD))
+def test_backward_combine_kernels(name, kernel, monkeypatch):
+    """Both combine-backward kernels (a block per token, or a warp per token)
+    at k = 1, 3, 8 and 16; H = 2112 is not a multiple of the warp kernel's 64
+    chunks per step."""
+    monkeypatch.setenv("MOE_COMBINE_BWD", kernel)
+    _check_backward_on_oracle_state(name, COMBINE_BWD[name])
+
+
+def _check_backward_on_oracle_state(name, w):
+    import routing_grouped_gemm_score_b200 as m
     d = wl.make_inputs(w, "cuda", with_dout=True)
     r = oracle.router_topk(d["logits"].cpu().numpy(), w.k)
     s = helpers.oracle_saved_state(w, d, r)

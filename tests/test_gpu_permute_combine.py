@@ -76,9 +76,11 @@ def test_permute_rejects_invalid_indices_on_the_device():
                                                  (1, 8, 2048, True, True), (3000, 16, 512, True, True),
                                                  (4100, 2, 4096, False, True)])
 def test_combine_matches_weighted_sum(T, k, H, shared, probs, path, monkeypatch):
-    """Both combine kernels (register path for rows up to 4096 wide, bulk
-    copies) on every shape; the register path stages 2048 assignments at a
-    time, so T=3000 at k=16 spans several stages of one block."""
+    """Every combine kernel on every shape: the default warp-per-token kernel
+    ("auto"), the token-range register kernel (rows up to 4096 wide), and the
+    bulk-copy kernel. The register kernel stages 2048 assignments at a time,
+    so T=3000 at k=16 spans several stages of one block; H=64 leaves most
+    lanes of the warp kernel without a chunk."""
     import routing_grouped_gemm_score_b200 as m
     if path != "auto":
         monkeypatch.setenv("MOE_COMBINE", path)
