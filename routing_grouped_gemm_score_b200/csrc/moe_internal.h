@@ -67,16 +67,6 @@ cudaError_t launch_combine_backward(const bf16* dout, const bf16* y_perm, const 
                                     const float* probs, int64_t T, int k, int H, int64_t A,
                                     bf16* dy_perm, float* dprob, cudaStream_t st, unsigned* err);
 
-// Bulk-copy row kernels (rows.cu). Any shape fits: rows wider than a stage
-// are cut into column pieces. *res holds the launch status; the return value
-// is always true.
-bool rows_combine(const bf16* y_perm, const int32_t* row_of, const float* probs, int64_t T, int k, int H,
-                  int64_t A, const bf16* shared, bf16* out, cudaStream_t st, unsigned* err, cudaError_t* res);
-bool rows_permute(const bf16* x, int64_t T, int H, const int32_t* topk_idx, int k, const int32_t* offsets, int E,
-                  const int32_t* block_base, int nb, int tpb, const int32_t* local_rank, bf16* x_perm,
-                  int32_t* sorted_token, int32_t* row_of, int64_t A, cudaStream_t st, unsigned* err,
-                  cudaError_t* res);
-
 // ---------------------------------------------------------------- GEMMs
 // Grouped GEMMs on tcgen05. Each returns cudaErrorInvalidValue if a tensor
 // map cannot be encoded (bad alignment or extent).

@@ -107,13 +107,10 @@ COMBINE_BWD = {
 }
 
 
-@pytest.mark.parametrize("kernel", ["block", "warp"])
 @pytest.mark.parametrize("name", list(COMBINE_BWD))
-def test_backward_combine_kernels(name, kernel, monkeypatch):
-    """Both combine-backward kernels (a block per token, or a warp per token)
-    at k = 1, 3, 8 and 16; H = 2112 is not a multiple of the warp kernel's 64
-    chunks per step."""
-    monkeypatch.setenv("MOE_COMBINE_BWD", kernel)
+def test_backward_combine_kernels(name):
+    """The warp-per-token combine backward at k = 1, 3, 8 and 16; H = 2112 is
+    not a multiple of the 64 chunks a warp covers per step."""
     _check_backward_on_oracle_state(name, COMBINE_BWD[name])
 
 

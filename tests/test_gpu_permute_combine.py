@@ -29,10 +29,11 @@ def routed(w):
                                       ("skew_t1", None, 256), ("skew_t8", None, 256),
                                       ("skew_t64", None, 2048), ("llama4_17bx16e", 1000, 5120),
                                       ("tie_t64", None, 128), ("mixtral_8x7b", 3000, 4096)])
-@pytest.mark.parametrize("path", ["auto", "regs", "bulk"])
+@pytest.mark.parametrize("path", ["auto", "warp"])
 def test_permute_matches_dispatch_definition(name, T, H, path, monkeypatch):
-    """Both permute kernels (register path for rows up to 4096 wide, bulk
-    copies) on every shape."""
+    """Both permute kernels on every shape: the default choice (the
+    token-range register kernel for rows up to 4096 wide, else one warp per
+    token) and the warp-per-token kernel forced."""
     monkeypatch.setenv("MOE_PERMUTE", path) if path != "auto" else None
     w = wl.WORKLOADS[name]
     if T is not None:
@@ -50,10 +51,12 @@ def test_permute_matches_dispatch_definition(name, T, H, path, monkeypatch):
                  oracle.gather_rows(bits(x), st), "x_perm")
 
 
-def test_permute_rejects_invalid_indices_on_the_device():
+@pytest.mark.parametrize("path", ["auto", "warp"])
+def test_permute_rejects_invalid_indices_on_the_device(path, monkeypatch):
     """Bad expert indices made on the host: the kernel flags them, skips the
     rows, and the status call reports MOE_ERR_DEVICE_CHECK."""
     import routing_grouped_gemm_score_b200 as m
+    monkeypatch.setenv("MOE_PERMUTE", path) if path != "auto" else None
     T, E, k, H = 100, 8, 2, 64
     idx = torch.randint(0, E, (T, k), dtype=torch.int32)
     idx[:, 1] = (idx[:, 0] + 1) % E
@@ -70,20 +73,16 @@ def test_permute_rejects_invalid_indices_on_the_device():
     assert m.moe_get_device_status() == 0          # the word was cleared
 
 
-@pytest.mark.parametrize("path", ["auto", "regs", "bulk"])
 @pytest.mark.parametrize("T,k,H,shared,probs", [(64, 2, 128, False, True), (1000, 8, 2048, False, True),
                                                  (333, 1, 5120, True, True), (257, 4, 64, False, False),
                                                  (1, 8, 2048, True, True), (3000, 16, 512, True, True),
-                                                 (4100, 2, 4096, False, True)])
-def test_combine_matches_weighted_sum(T, k, H, shared, probs, path, monkeypatch):
-    """Every combine kernel on every shape: the default warp-per-token kernel
-    ("auto"), the token-range register kernel (rows up to 4096 wide), and the
-    bulk-copy kernel. The register kernel stages 2048 assignments at a time,
-    so T=3000 at k=16 spans several stages of one block; H=64 leaves most
-    lanes of the warp kernel without a chunk."""
+                                                 (4100, 2, 4096, False, True), (700, 8, 2112, True, True)])
+def test_combine_matches_weighted_sum(T, k, H, shared, probs):
+    """The warp-per-token combine on shapes from one token to 4100, k from 1
+    to 16, with and without a shared row and weights; H=64 leaves most lanes
+    without a chunk, and H=2112 (264 chunks) ends in a part step of the 64
+    chunks a warp covers per step at k=8."""
     import routing_grouped_gemm_score_b200 as m
-    if path != "auto":
-        monkeypatch.setenv("MOE_COMBINE", path)
     g_ = torch.Generator().manual_seed(T * 7 + k)
     A = T * k
     y = torch.randn((A, H), generator=g_).to(torch.bfloat16)
