@@ -58,6 +58,13 @@ def _load():
             lib.oracle_router_backward.restype = i32
             lib.oracle_expert_bias_update.argtypes = [P, i32, f32, P]
             lib.oracle_expert_bias_update.restype = None
+            f64 = ctypes.c_double
+            lib.oracle_aux_scores.argtypes = [P, i64, i32, i32, P]
+            lib.oracle_aux_scores.restype = None
+            lib.oracle_aux_loss.argtypes = [P, P, i64, i32, i32, f64]
+            lib.oracle_aux_loss.restype = f64
+            lib.oracle_aux_loss_backward.argtypes = [P, P, i64, i32, i32, i32, f64, f64, P]
+            lib.oracle_aux_loss_backward.restype = None
             lib.oracle_dispatch.argtypes = [P, i64, i32, i32, P, P, P]
             lib.oracle_dispatch.restype = i32
             lib.oracle_gather_rows.argtypes = [P, i32, P, i64, P]
@@ -150,6 +157,39 @@ def expert_bias_update(counts, bias, coeff):
     counts = _c(counts, np.int32)
     out = np.array(bias, np.float32, copy=True)
     lib.oracle_expert_bias_update(_p(counts), len(counts), coeff, _p(out))
+    return out
+
+
+def aux_scores(logits, score=0):
+    """Dense scores [T,E] (float64) for the auxiliary loss: softmax over all
+    experts (score 0) or the sigmoid of each logit (score 1)."""
+    lib = _load()
+    logits = _c(logits, np.float32)
+    T, E = logits.shape
+    out = np.zeros((T, E), np.float64)
+    lib.oracle_aux_scores(_p(logits), T, E, int(score), _p(out))
+    return out
+
+
+def aux_loss(logits, counts, k, coeff, score=0):
+    """The load-balancing loss (float) from the logits and per-expert counts
+    (oracle_aux_loss on oracle_aux_scores)."""
+    lib = _load()
+    s = aux_scores(logits, score)
+    counts = _c(counts, np.int32)
+    T, E = s.shape
+    return float(lib.oracle_aux_loss(_p(s), _p(counts), T, E, int(k), float(coeff)))
+
+
+def aux_loss_backward(logits, counts, k, coeff, score=0, grad_loss=1.0):
+    """d(grad_loss * loss)/dlogits [T,E] (float64), counts held fixed."""
+    lib = _load()
+    logits = _c(logits, np.float32)
+    counts = _c(counts, np.int32)
+    T, E = logits.shape
+    out = np.zeros((T, E), np.float64)
+    lib.oracle_aux_loss_backward(_p(logits), _p(counts), T, E, int(k), int(score), float(coeff),
+                                 float(grad_loss), _p(out))
     return out
 
 

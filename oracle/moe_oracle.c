@@ -278,6 +278,87 @@ void oracle_expert_bias_update(const int32_t* counts, int E, float coeff, float*
     free(delta);
 }
 
+/* ---------------------------------------------------------- aux loss --- */
+
+/*
+ * oracle_aux_scores -- [TE] Mixture of Experts, Load balancing: the dense
+ * routing scores that the auxiliary loss takes, one per expert rather than
+ * only for the chosen k: the softmax over all E experts (score_fn 0) or the
+ * sigmoid of each logit (score_fn 1), in fp64. The page's score helper
+ * ignores an expert bias, so none is applied. Writes scores[T,E].
+ */
+void oracle_aux_scores(const float* logits, int64_t T, int E, int score_fn, double* scores)
+{
+    for (int64_t t = 0; t < T; t++) {
+        const float* l = logits + t * E;
+        double* s = scores + t * E;
+        if (score_fn == 0) {
+            double m = l[0], sum = 0.0;
+            for (int e = 1; e < E; e++) if (l[e] > m) m = l[e];
+            for (int e = 0; e < E; e++) { s[e] = exp((double)l[e] - m); sum += s[e]; }
+            for (int e = 0; e < E; e++) s[e] /= sum;
+        } else {
+            for (int e = 0; e < E; e++) s[e] = 1.0 / (1.0 + exp(-(double)l[e]));
+        }
+    }
+}
+
+/*
+ * oracle_aux_loss -- [TE] Mixture of Experts, Load balancing
+ * (fused_moe_aux_loss). The page names the inputs -- the dense scores, the
+ * per-expert token counts c[E] taken from the router's routing map, the
+ * number of tokens T and of experts E, the top-k and a coefficient -- but
+ * prints no formula. Reading: the switch-style load-balancing loss
+ *   loss = coeff * E / (k * T^2) * sum_e (sum_t s[t,e]) * c_e
+ *        = coeff * E * sum_e f_e * P_e,
+ *   f_e = c_e / (k T) (share of assignments), P_e = (1/T) sum_t s[t,e].
+ * With every expert at T k / E assignments and a mean score of 1/E it is
+ * exactly coeff, and it grows as the counts gather where the scores are
+ * high. Sums run in fp64, t then e in order.
+ */
+double oracle_aux_loss(const double* scores, const int32_t* counts, int64_t T, int E, int k, double coeff)
+{
+    double total = 0.0;
+    for (int e = 0; e < E; e++) {
+        double P = 0.0;
+        for (int64_t t = 0; t < T; t++) P += scores[t * E + e];
+        total += P * (double)counts[e];
+    }
+    return coeff * (double)E / ((double)k * (double)T * (double)T) * total;
+}
+
+/*
+ * oracle_aux_loss_backward -- the gradient of grad_loss * loss with respect
+ * to the logits, the counts held fixed (they come from the discrete
+ * selection). dloss/ds[t,e] is the same for every token,
+ *   G_e = grad_loss * coeff * E * c_e / (k T^2),
+ * and the chain rule through the score function gives
+ *   softmax: dl[t,i] = s[t,i] * (G_i - sum_e s[t,e] G_e);
+ *   sigmoid: dl[t,i] = G_i * s[t,i] * (1 - s[t,i]).
+ * Writes dlogits[T,E] in fp64.
+ */
+void oracle_aux_loss_backward(const float* logits, const int32_t* counts, int64_t T, int E, int k,
+                              int score_fn, double coeff, double grad_loss, double* dlogits)
+{
+    double* s = (double*)malloc(sizeof(double) * (size_t)E);
+    double* G = (double*)malloc(sizeof(double) * (size_t)E);
+    for (int e = 0; e < E; e++)
+        G[e] = grad_loss * coeff * (double)E * (double)counts[e] / ((double)k * (double)T * (double)T);
+    for (int64_t t = 0; t < T; t++) {
+        oracle_aux_scores(logits + t * E, 1, E, score_fn, s);
+        double* dl = dlogits + t * E;
+        if (score_fn == 0) {
+            double c = 0.0;
+            for (int e = 0; e < E; e++) c += s[e] * G[e];
+            for (int e = 0; e < E; e++) dl[e] = s[e] * (G[e] - c);
+        } else {
+            for (int e = 0; e < E; e++) dl[e] = G[e] * s[e] * (1.0 - s[e]);
+        }
+    }
+    free(s);
+    free(G);
+}
+
 /* ----------------------------------------------------------- dispatch --- */
 
 /*
