@@ -491,8 +491,29 @@ def router_sweep(m, hbm):
         bbytes = 2 * T * E * 4 + T * k * 8
         entry["backward"] = {"us": bms * 1e3, "GB/s": bbytes / (bms / 1e3) / 1e9,
                              "frac_of_hbm": bbytes / (bms / 1e3) / 1e9 / hbm}
+        # the auxiliary load-balancing loss on the same logits and counts: the
+        # forward reads the logits once; its backward reads them and writes dlogits
+        aws = torch.empty(m.lib().moe_aux_loss_workspace_size(T, E), dtype=torch.uint8, device="cuda")
+        for name, call, nb in (
+                ("aux_loss", lambda: m.moe_aux_loss(logits, res["counts"], k, 1e-2, workspace=aws),
+                 T * E * 4 + E * 4),
+                ("aux_loss_backward", lambda: m.moe_aux_loss_backward(logits, res["counts"], k, 1e-2, dlogits=dl),
+                 2 * T * E * 4 + E * 4)):
+            atimes = []
+            for it in range(8):
+                flush.sum()
+                s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                s.record()
+                call()
+                e.record()
+                torch.cuda.synchronize()
+                if it >= 2:
+                    atimes.append(s.elapsed_time(e))
+            ams = statistics.median(atimes)
+            entry[name] = {"us": ams * 1e3, "GB/s": nb / (ams / 1e3) / 1e9,
+                           "frac_of_hbm": nb / (ams / 1e3) / 1e9 / hbm}
         out.append(entry)
-        del logits, res, ws, dprob, dl
+        del logits, res, ws, dprob, dl, aws
     return out
 
 

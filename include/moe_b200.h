@@ -159,6 +159,42 @@ moe_status moe_router_backward(const float* logits, int64_t T, int E, int k,
 moe_status moe_expert_bias_update(const int32_t* counts, int E, float coeff, float* expert_bias,
                                   void* stream);
 
+/* moe_aux_loss -- TE Mixture of Experts, Load balancing (fused_moe_aux_loss
+ * on the dense scores of fused_compute_score_for_moe_aux_loss): the auxiliary
+ * loss that penalises uneven token counts. The page names its inputs but
+ * prints no formula; the reading implemented is the switch-style loss
+ *   loss = coeff * E / (k T^2) * sum_e (sum_t s[t,e]) * counts[e],
+ * which equals coeff when every expert has T k / E assignments and a mean
+ * score of 1/E. The dense scores s are the softmax over all E logits
+ * (MOE_SCORE_SOFTMAX) or the sigmoid of each logit (MOE_SCORE_SIGMOID), with
+ * no expert bias, in fp32; the sums over tokens run in a fixed order (fp32
+ * within a block, fp64 across blocks), so the result is the same on every run
+ * on a given GPU.
+ *  logits  in  fp32 [T, E]   the router's logits
+ *  counts  in  int32 [E]     tokens per expert from the router's routing map
+ *                            (moe_router_topk's counts)
+ *  loss    out fp32 [1]      on the device
+ *  scores  out fp32 [T, E]   the dense scores (NULL: not written)
+ * T >= 1, E in [1, 256], 1 <= k <= min(E, 16). workspace of at least
+ * moe_aux_loss_workspace_size(T, E) bytes, 16-byte aligned. */
+size_t moe_aux_loss_workspace_size(int64_t T, int E);
+moe_status moe_aux_loss(const float* logits, int64_t T, int E, int k, int score_fn,
+                        const int32_t* counts, float coeff, float* loss, float* scores,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* moe_aux_loss_backward -- the gradient of grad_loss * loss (moe_aux_loss) with
+ * respect to the logits, the counts held fixed (they come from the discrete
+ * choice). With G_e = grad_loss * coeff * E * counts[e] / (k T^2):
+ *   softmax: dlogits[t,i] = s[t,i] (G_i - sum_e s[t,e] G_e)
+ *   sigmoid: dlogits[t,i] = G_i s[t,i] (1 - s[t,i])
+ *  grad_loss  in  fp32 [1] on the device (NULL: 1)
+ *  dlogits    out fp32 [T, E]; accumulate != 0 adds to it (for example to the
+ *             router's own gradient from moe_router_backward), 0 overwrites.
+ * Other arguments as in moe_aux_loss. */
+moe_status moe_aux_loss_backward(const float* logits, int64_t T, int E, int k, int score_fn,
+                                 const int32_t* counts, float coeff, const float* grad_loss,
+                                 float* dlogits, int accumulate, void* stream);
+
 /* moe_router_topk_noalloc -- the same routing as moe_router_topk, with no
  * workspace argument: for callers that cannot allocate device memory when they
  * route, such as a runtime that hands out all device memory from its own

@@ -79,6 +79,9 @@ ABI_FUNCTIONS = {
     "moe_router_topk": (I32, [P, I64, I32, I32, ctypes.POINTER(_RouterOptsC), P, P, P, P, P, P, SZ, P]),
     "moe_router_backward": (I32, [P, I64, I32, I32, ctypes.POINTER(_RouterOptsC), P, P, P, P]),
     "moe_expert_bias_update": (I32, [P, I32, ctypes.c_float, P, P]),
+    "moe_aux_loss_workspace_size": (SZ, [I64, I32]),
+    "moe_aux_loss": (I32, [P, I64, I32, I32, I32, P, F32, P, P, P, SZ, P]),
+    "moe_aux_loss_backward": (I32, [P, I64, I32, I32, I32, P, F32, P, P, I32, P]),
     "moe_router_topk_noalloc": (I32, [P, I64, I32, I32, ctypes.POINTER(_RouterOptsC), P, P, P, P,
                                        P, P]),
     "moe_permute_workspace_size": (SZ, [I64, I32, I32]),
@@ -244,6 +247,45 @@ def moe_expert_bias_update(counts: torch.Tensor, expert_bias: torch.Tensor, coef
     _check(lib().moe_expert_bias_update(_ptr(counts), counts.numel(), float(coeff), _ptr(expert_bias), _stream()),
            "moe_expert_bias_update")
     return expert_bias
+
+
+def moe_aux_loss(logits: torch.Tensor, counts: torch.Tensor, k: int, coeff: float,
+                 score_fn: int = 0, want_scores: bool = False,
+                 workspace: Optional[torch.Tensor] = None) -> tuple:
+    """Auxiliary load-balancing loss: (loss as a 0-d fp32 device tensor, the
+    dense scores [T,E] or None). counts: tokens per expert from the router."""
+    _need(logits, torch.float32, "logits")
+    _need(counts, torch.int32, "counts")
+    T, E = logits.shape
+    dev = logits.device
+    loss = torch.empty((), dtype=torch.float32, device=dev)
+    scores = torch.empty((T, E), dtype=torch.float32, device=dev) if want_scores else None
+    need = lib().moe_aux_loss_workspace_size(T, E)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    _check(lib().moe_aux_loss(_ptr(logits), T, E, int(k), int(score_fn), _ptr(counts), float(coeff), _ptr(loss),
+                              _ptr(scores), _ptr(workspace), workspace.numel(), _stream()), "moe_aux_loss")
+    return loss, scores
+
+
+def moe_aux_loss_backward(logits: torch.Tensor, counts: torch.Tensor, k: int, coeff: float,
+                          score_fn: int = 0, grad_loss: Optional[torch.Tensor] = None,
+                          dlogits: Optional[torch.Tensor] = None, accumulate: bool = False) -> torch.Tensor:
+    """d(grad_loss * aux loss)/dlogits [T,E] (fp32), counts held fixed. With
+    accumulate, adds to the given dlogits."""
+    _need(logits, torch.float32, "logits")
+    _need(counts, torch.int32, "counts")
+    T, E = logits.shape
+    if grad_loss is not None:
+        _need(grad_loss, torch.float32, "grad_loss")
+    if dlogits is None:
+        if accumulate:
+            raise ValueError("accumulate needs the dlogits to add to")
+        dlogits = torch.empty((T, E), dtype=torch.float32, device=logits.device)
+    _check(lib().moe_aux_loss_backward(_ptr(logits), T, E, int(k), int(score_fn), _ptr(counts), float(coeff),
+                                       _ptr(grad_loss), _ptr(dlogits), int(bool(accumulate)), _stream()),
+           "moe_aux_loss_backward")
+    return dlogits
 
 
 def moe_permute(x: torch.Tensor, topk_idx: torch.Tensor, offsets: torch.Tensor) -> dict:

@@ -254,6 +254,39 @@ moe_status moe_expert_bias_update(const int32_t* counts, int E, float coeff, flo
     return from_cuda(launch_expert_bias_update(counts, E, coeff, expert_bias, static_cast<cudaStream_t>(stream)));
 }
 
+size_t moe_aux_loss_workspace_size(int64_t T, int E) {
+    if (T < 1 || E < 1 || E > 256) return 0;
+    return aux_loss_workspace_bytes(T, E);
+}
+
+namespace {
+bool aux_args_ok(const float* logits, int64_t T, int E, int k, int score_fn, const int32_t* counts) {
+    return T >= 1 && shape_ok(T, E, k) && (score_fn == MOE_SCORE_SOFTMAX || score_fn == MOE_SCORE_SIGMOID) &&
+           logits && counts && aligned16(logits) && aligned16(counts);
+}
+}  // namespace
+
+moe_status moe_aux_loss(const float* logits, int64_t T, int E, int k, int score_fn,
+                        const int32_t* counts, float coeff, float* loss, float* scores,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+    if (!aux_args_ok(logits, T, E, k, score_fn, counts) || !loss || !(coeff == coeff))
+        return MOE_ERR_INVALID_ARG;
+    if (scores && !aligned16(scores)) return MOE_ERR_INVALID_ARG;
+    if (!workspace || !aligned16(workspace)) return MOE_ERR_INVALID_ARG;
+    if (workspace_bytes < aux_loss_workspace_bytes(T, E)) return MOE_ERR_WORKSPACE;
+    return from_cuda(launch_aux_loss(logits, T, E, k, score_fn, counts, coeff, loss, scores, workspace,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_aux_loss_backward(const float* logits, int64_t T, int E, int k, int score_fn,
+                                 const int32_t* counts, float coeff, const float* grad_loss,
+                                 float* dlogits, int accumulate, void* stream) {
+    if (!aux_args_ok(logits, T, E, k, score_fn, counts) || !dlogits || !aligned16(dlogits) || !(coeff == coeff))
+        return MOE_ERR_INVALID_ARG;
+    return from_cuda(launch_aux_loss_backward(logits, T, E, k, score_fn, counts, coeff, grad_loss, dlogits,
+                                              accumulate, static_cast<cudaStream_t>(stream)));
+}
+
 moe_status moe_router_topk_noalloc(const float* logits, int64_t T, int E, int k,
                                    const moe_router_opts* opts_in, int32_t* topk_idx,
                                    float* topk_prob, uint8_t* routing_map, int32_t* counts,

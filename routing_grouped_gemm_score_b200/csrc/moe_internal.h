@@ -47,6 +47,14 @@ cudaError_t launch_router_backward(const float* logits, int64_t T, int E, int k,
                                    const int32_t* topk_idx, const float* dprob, float* dlogits,
                                    cudaStream_t st, unsigned* err);
 cudaError_t launch_expert_bias_update(const int32_t* counts, int E, float coeff, float* bias, cudaStream_t st);
+
+// Auxiliary load-balancing loss (aux_loss.cu).
+size_t aux_loss_workspace_bytes(int64_t T, int E);
+cudaError_t launch_aux_loss(const float* logits, int64_t T, int E, int k, int score_fn, const int32_t* counts,
+                            float coeff, float* loss, float* scores, void* ws, cudaStream_t st);
+cudaError_t launch_aux_loss_backward(const float* logits, int64_t T, int E, int k, int score_fn,
+                                     const int32_t* counts, float coeff, const float* grad_loss, float* dlogits,
+                                     int accumulate, cudaStream_t st);
 cudaError_t launch_rank_from_indices(const int32_t* topk_idx, int64_t T, int E, int k,
                                      const RouteScratch& rs, cudaStream_t st, unsigned* err);
 // Turns block counts into exclusive prefixes; writes counts/offsets if given.

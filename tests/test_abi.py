@@ -90,6 +90,13 @@ def test_invalid_arguments_are_rejected_without_a_device(built):
     assert l.moe_layer_forward(fake, fake, 10, 128, 128, 8, 2, ctypes.byref(opts), fake, fake,
                                fake, None, fake, None, None, None, None, None, None, None, None,
                                None, fake, 1 << 30, None) == 1
+    # aux loss: T = 0 (the loss divides by T^2), an unknown score function, a
+    # workspace too small, no loss output
+    assert l.moe_aux_loss(fake, 0, 8, 2, 0, fake, ctypes.c_float(0.01), fake, None, fake, 1 << 20, None) == 1
+    assert l.moe_aux_loss(fake, 10, 8, 2, 7, fake, ctypes.c_float(0.01), fake, None, fake, 1 << 20, None) == 1
+    assert l.moe_aux_loss(fake, 10, 8, 2, 0, fake, ctypes.c_float(0.01), fake, None, fake, 16, None) == 4
+    assert l.moe_aux_loss(fake, 10, 8, 2, 0, fake, ctypes.c_float(0.01), None, None, fake, 1 << 20, None) == 1
+    assert l.moe_aux_loss_backward(fake, 10, 8, 9, 0, fake, ctypes.c_float(0.01), None, fake, 0, None) == 1
     # backward: a missing saved tensor
     assert l.moe_grouped_mlp_backward(fake, 10, 128, 128, 8, 2, fake, fake, fake, fake, fake, fake,
                                       None, fake, fake, fake, fake, fake, fake, fake, 1 << 30,
@@ -101,6 +108,11 @@ def test_workspace_sizes_are_consistent(built):
     l = m.lib()
     assert l.moe_router_workspace_size(4096, 128, 8) > 4096 * 8 * 4
     assert l.moe_router_workspace_size(10, 0, 1) == 0
+    # aux loss: E fp32 values per block (one block per 32 tokens, at most 1024
+    # blocks) and a ticket
+    assert l.moe_aux_loss_workspace_size(4096, 128) >= 128 * 128 * 4
+    assert l.moe_aux_loss_workspace_size(1 << 24, 256) <= 1024 * 256 * 4 + 512
+    assert l.moe_aux_loss_workspace_size(0, 8) == 0
     a = l.moe_layer_forward_workspace_size(4096, 2048, 768, 128, 8, 0)
     b = l.moe_layer_forward_workspace_size(4096, 2048, 768, 128, 8, 1)
     A = 4096 * 8
