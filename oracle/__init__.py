@@ -67,6 +67,8 @@ def _load():
             lib.oracle_aux_loss_backward.restype = None
             lib.oracle_dispatch.argtypes = [P, i64, i32, i32, P, P, P]
             lib.oracle_dispatch.restype = i32
+            lib.oracle_dispatch_padded.argtypes = [P, i64, i32, i32, P, i32, P, P, P]
+            lib.oracle_dispatch_padded.restype = i32
             lib.oracle_gather_rows.argtypes = [P, i32, P, i64, P]
             lib.oracle_gather_rows.restype = None
             lib.oracle_expert_mlp.argtypes = [P, i64, i32, i32, P, P, i32, P, P, P, P]
@@ -205,6 +207,25 @@ def dispatch(topk_idx, offsets, E):
     if rc:
         raise ValueError(f"oracle_dispatch: invalid routing ({rc})")
     return sorted_token, row_of
+
+
+def dispatch_padded(topk_idx, offsets, E, align):
+    """Padded dispatch: (padded_offsets [E+1], sorted_token [padded total] with
+    -1 in the pad rows, row_of [T,k]) (oracle_dispatch_padded)."""
+    lib = _load()
+    topk_idx = _c(topk_idx, np.int32)
+    offsets = _c(offsets, np.int32)
+    T, k = topk_idx.shape
+    counts = np.diff(offsets.astype(np.int64))
+    total = int(sum(-(-c // align) * align for c in counts)) if align >= 1 else 0
+    padded = np.zeros(E + 1, np.int32)
+    sorted_token = np.full(max(total, 1), -1, np.int32)
+    row_of = np.full((T, k), -1, np.int32)
+    rc = lib.oracle_dispatch_padded(_p(topk_idx), T, k, E, _p(offsets), int(align), _p(padded),
+                                    _p(sorted_token), _p(row_of))
+    if rc:
+        raise ValueError(f"oracle_dispatch_padded: invalid routing ({rc})")
+    return padded, sorted_token[:total], row_of
 
 
 def gather_rows(x_bits, sorted_token):

@@ -392,12 +392,45 @@ int oracle_dispatch(const int32_t* topk_idx, int64_t T, int k, int E,
     return rc;
 }
 
-/* x_perm[row] = x[sorted_token[row]]: a plain copy of bf16 rows. */
+/*
+ * oracle_dispatch_padded -- [TE] Mixture of Experts, Token permutation,
+ * Padding and alignment: each expert's block is rounded up to a multiple of
+ * align rows (an empty block stays empty), the blocks follow one another in
+ * expert order, and the rows past an expert's tokens are padding.
+ *   padded_offsets[0] = 0,
+ *   padded_offsets[e+1] = padded_offsets[e] + align * ceil(counts[e] / align),
+ * with counts[e] = offsets[e+1] - offsets[e]. Inside a block the tokens keep
+ * the unpadded order, so the assignment (t, j) lands in row
+ *   padded_offsets[e] + #{ t' < t : e is among the experts of t' },
+ * which is oracle_dispatch on the padded offsets. Writes padded_offsets[E+1],
+ * row_of[T,k] and sorted_token[padded_offsets[E]] (the token of each row; the
+ * caller fills the pad rows' entries with -1 beforehand). Returns nonzero on
+ * an invalid routing or align < 1.
+ */
+int oracle_dispatch_padded(const int32_t* topk_idx, int64_t T, int k, int E, const int32_t* offsets,
+                           int align, int32_t* padded_offsets, int32_t* sorted_token, int32_t* row_of)
+{
+    if (align < 1) return 4;
+    padded_offsets[0] = 0;
+    for (int e = 0; e < E; e++) {
+        const int64_t c = (int64_t)offsets[e + 1] - offsets[e];
+        if (c < 0) return 5;
+        padded_offsets[e + 1] = padded_offsets[e] + (int32_t)(((c + align - 1) / align) * align);
+    }
+    return oracle_dispatch(topk_idx, T, k, E, padded_offsets, sorted_token, row_of);
+}
+
+/* x_perm[row] = x[sorted_token[row]]: a plain copy of bf16 rows; a row whose
+ * sorted_token is negative (a pad row of the padded dispatch) is zeros. */
 void oracle_gather_rows(const uint16_t* x, int H, const int32_t* sorted_token,
                         int64_t A, uint16_t* x_perm)
 {
-    for (int64_t r = 0; r < A; r++)
-        memcpy(x_perm + r * H, x + (int64_t)sorted_token[r] * H, sizeof(uint16_t) * (size_t)H);
+    for (int64_t r = 0; r < A; r++) {
+        if (sorted_token[r] < 0)
+            memset(x_perm + r * H, 0, sizeof(uint16_t) * (size_t)H);
+        else
+            memcpy(x_perm + r * H, x + (int64_t)sorted_token[r] * H, sizeof(uint16_t) * (size_t)H);
+    }
 }
 
 /* ---------------------------------------------------------- expert MLP -- */

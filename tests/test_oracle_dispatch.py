@@ -121,3 +121,58 @@ def test_bf16_rounding(oracle_lib):
     f32 = (rng.standard_normal(5000) * 3).astype(np.float32)
     tb = torch.from_numpy(f32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     assert all(oracle_lib.round_bf16(float(a)) == int(b) for a, b in zip(f32, tb))
+
+
+# ------------------------------------------------------------ padded dispatch
+# Transformer Engine "Mixture of Experts", Token permutation, Padding and alignment.
+
+def test_padded_dispatch_pages_example(oracle_lib):
+    """The page's example: counts of 129 and 127 take 384 rows at an
+    alignment of 128, although only 256 tokens arrive."""
+    topk = np.array([[0]] * 129 + [[1]] * 127, np.int32)
+    offsets = np.array([0, 129, 256], np.int32)
+    padded, st, row_of = oracle_lib.dispatch_padded(topk, offsets, 2, 128)
+    assert padded.tolist() == [0, 256, 384]
+    assert len(st) == 384
+    assert np.all(st[129:256] == -1) and np.all(st[256 + 127:] == -1)
+    assert st[:129].tolist() == list(range(129)) and st[256:383].tolist() == list(range(129, 256))
+
+
+def test_padded_dispatch_with_align_one_is_the_dispatch(oracle_lib):
+    w, r = routed(oracle_lib, "qwen3_30b_a3b", 300)
+    st, row_of = oracle_lib.dispatch(r["topk_idx"], r["offsets"], w.E)
+    padded, st1, row_of1 = oracle_lib.dispatch_padded(r["topk_idx"], r["offsets"], w.E, 1)
+    assert np.array_equal(padded, r["offsets"]) and np.array_equal(st1, st) and np.array_equal(row_of1, row_of)
+
+
+@pytest.mark.parametrize("name,T,align", [("qwen3_30b_a3b", 500, 16), ("skew_t64", None, 128),
+                                          ("mixtral_8x7b", 700, 256), ("tiny", None, 3)])
+def test_padded_dispatch_invariants(oracle_lib, name, T, align):
+    w, r = routed(oracle_lib, name, T)
+    offsets = r["offsets"].astype(np.int64)
+    padded, st, row_of = oracle_lib.dispatch_padded(r["topk_idx"], r["offsets"], w.E, align)
+    padded = padded.astype(np.int64)
+    counts, pcounts = np.diff(offsets), np.diff(padded)
+    assert np.all(padded % align == 0)                       # every block starts aligned
+    assert np.all((pcounts - counts >= 0) & (pcounts - counts < align))
+    assert np.all((pcounts == 0) == (counts == 0))           # an empty block stays empty
+    # the pad rows are exactly the tail of each block
+    pad = np.zeros(len(st), bool)
+    for e in range(w.E):
+        pad[padded[e] + counts[e]:padded[e + 1]] = True
+    assert np.all((st < 0) == pad)
+    # row_of is a bijection onto the real rows, inverse to sorted_token, and keeps
+    # the unpadded order inside each block
+    rows = row_of.ravel()
+    assert len(np.unique(rows)) == rows.size and not np.any(pad[rows])
+    t_of = np.repeat(np.arange(w.T), w.k)
+    assert np.array_equal(st[rows], t_of)
+    _, row_plain = oracle_lib.dispatch(r["topk_idx"], r["offsets"], w.E)
+    e_of = r["topk_idx"].ravel()
+    assert np.array_equal(rows - padded[e_of], row_plain.ravel() - offsets[e_of])
+
+
+def test_gather_rows_zero_fills_pad_rows(oracle_lib):
+    x = np.arange(12, dtype=np.uint16).reshape(3, 4) + 1
+    out = oracle_lib.gather_rows(x, np.array([2, -1, 0, -1], np.int32))
+    assert out.tolist() == [[9, 10, 11, 12], [0, 0, 0, 0], [1, 2, 3, 4], [0, 0, 0, 0]]
