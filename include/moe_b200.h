@@ -236,6 +236,36 @@ moe_status moe_permute(const moe_bf16* x, int64_t T, int H, const int32_t* topk_
                        const int32_t* offsets, int E, moe_bf16* x_perm, int32_t* sorted_token,
                        int32_t* row_of, void* workspace, size_t workspace_bytes, void* stream);
 
+/* moe_permute_padded -- TE Token permutation, Padding and alignment
+ * (moe_permute_and_pad_with_probs): the dispatch of moe_permute with each
+ * expert's block rounded up to a multiple of align rows, for grouped GEMM
+ * back ends that want aligned blocks. An empty block stays empty; the tokens
+ * keep their moe_permute order inside a block, and the rows past an expert's
+ * tokens are padding:
+ *   padded_offsets[e+1] = padded_offsets[e] + align * ceil(counts[e] / align)
+ *   assignment (t, j), e = topk_idx[t,j]: row padded_offsets[e] + #{t' < t routed to e}
+ * Pad rows are zeros in x_perm, -1 in sorted_token and 0 in prob_perm. The
+ * combine needs no padding information: row_of points at the real rows.
+ *  x, topk_idx, k, E       as in moe_permute
+ *  offsets         in  int32 [E+1]  unpadded, from moe_router_topk
+ *  topk_prob       in  fp32 [T, k]  (needed only with prob_perm)
+ *  align           in  1 .. 65536
+ *  padded_offsets  out int32 [E+1]
+ *  x_perm          out bf16 [R, H]  R = moe_permute_padded_max_rows(T, E, k, align)
+ *                      = T*k + E*(align-1), the bound that needs no host sync;
+ *                      rows past padded_offsets[E] are untouched
+ *  prob_perm       out fp32 [R]     routing weight of each row (NULL: skip);
+ *                      the weights for moe_grouped_mlp_scaled
+ *  sorted_token    out int32 [R]
+ *  row_of          out int32 [T, k]
+ *  workspace       moe_permute_workspace_size(T, E, k) bytes */
+int64_t moe_permute_padded_max_rows(int64_t T, int E, int k, int align);
+moe_status moe_permute_padded(const moe_bf16* x, int64_t T, int H, const int32_t* topk_idx,
+                              const float* topk_prob, int k, const int32_t* offsets, int E, int align,
+                              int32_t* padded_offsets, moe_bf16* x_perm, float* prob_perm,
+                              int32_t* sorted_token, int32_t* row_of, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
 /* -------------------------------------------------------------- grouped MLP
  * moe_grouped_mlp -- TE Grouped GEMM (Y_i = X_i W_i^T per expert block,
  * Y = concat(Y_i)) and Grouped MLP (FC1 with the activation fused, then FC2).
@@ -258,6 +288,20 @@ moe_status moe_grouped_mlp(const moe_bf16* x_perm, int64_t A, const int32_t* off
                            moe_bf16* y_perm, moe_bf16* gu_save, moe_bf16* h_save,
                            void* workspace, size_t workspace_bytes, void* stream);
 
+/* moe_grouped_mlp_scaled -- TE Grouped MLP with ScaledSwiGLU: moe_grouped_mlp
+ * with the routing weight of each row applied to the activation before FC2,
+ *   h[r] = bf16(silu(g) * u * row_scale[r]),  y_perm[r] = bf16(h[r] . w_down[e]),
+ * so y_perm is already weighted ((p h) W2 = p (h W2), the page's identity for
+ * FC2 without bias) and moe_unpermute_combine must then run with topk_prob
+ * NULL. gu_save keeps the unscaled g and u. row_scale fp32 [A] (for example
+ * moe_permute_padded's prob_perm; NULL: 1). The backward of this variant is
+ * not provided: moe_grouped_mlp_backward differentiates the layer with the
+ * weights applied in combine. Other arguments as in moe_grouped_mlp. */
+moe_status moe_grouped_mlp_scaled(const moe_bf16* x_perm, int64_t A, const int32_t* offsets, int E,
+                                  int H, int I, const moe_bf16* w_gate_up, const moe_bf16* w_down,
+                                  const float* row_scale, moe_bf16* y_perm, moe_bf16* gu_save,
+                                  moe_bf16* h_save, void* workspace, size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------------------ combine
  * moe_unpermute_combine -- TE Token combine with merging_probs:
  *   out[t] = bf16( shared_out[t] + sum_{j<k} topk_prob[t,j] * y_perm[row_of[t,j]] )
@@ -270,6 +314,16 @@ moe_status moe_grouped_mlp(const moe_bf16* x_perm, int64_t A, const int32_t* off
 moe_status moe_unpermute_combine(const moe_bf16* y_perm, const int32_t* row_of,
                                  const float* topk_prob, int64_t T, int k, int H,
                                  const moe_bf16* shared_out, moe_bf16* out, void* stream);
+
+/* moe_unpermute_combine_rows -- moe_unpermute_combine for a y_perm of y_rows
+ * rows, such as the output of a padded dispatch (moe_permute_padded: rows
+ * T*k + E*(align-1) at most, with row_of pointing at the real rows, so the pad
+ * rows are never read). moe_unpermute_combine is this call with
+ * y_rows = T*k. A row_of entry outside [0, y_rows) is recorded as
+ * MOE_ERR_DEVICE_CHECK and skipped. */
+moe_status moe_unpermute_combine_rows(const moe_bf16* y_perm, int64_t y_rows, const int32_t* row_of,
+                                      const float* topk_prob, int64_t T, int k, int H,
+                                      const moe_bf16* shared_out, moe_bf16* out, void* stream);
 
 /* ------------------------------------------------------------ fused layer
  * moe_layer_forward -- the four stages on one stream (TE "Example: MoE layer

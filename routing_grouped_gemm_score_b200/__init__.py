@@ -86,9 +86,13 @@ ABI_FUNCTIONS = {
                                        P, P]),
     "moe_permute_workspace_size": (SZ, [I64, I32, I32]),
     "moe_permute": (I32, [P, I64, I32, P, I32, P, I32, P, P, P, P, SZ, P]),
+    "moe_permute_padded_max_rows": (I64, [I64, I32, I32, I32]),
+    "moe_permute_padded": (I32, [P, I64, I32, P, P, I32, P, I32, I32, P, P, P, P, P, P, SZ, P]),
     "moe_grouped_mlp_workspace_size": (SZ, [I64, I32, I32, I32]),
     "moe_grouped_mlp": (I32, [P, I64, P, I32, I32, I32, P, P, P, P, P, P, SZ, P]),
+    "moe_grouped_mlp_scaled": (I32, [P, I64, P, I32, I32, I32, P, P, P, P, P, P, P, SZ, P]),
     "moe_unpermute_combine": (I32, [P, P, P, I64, I32, I32, P, P, P]),
+    "moe_unpermute_combine_rows": (I32, [P, I64, P, P, I64, I32, I32, P, P, P]),
     "moe_layer_forward_workspace_size": (SZ, [I64, I32, I32, I32, I32, I32]),
     "moe_layer_forward": (I32, [P, P, I64, I32, I32, I32, I32, ctypes.POINTER(_RouterOptsC), P, P, P,
                                 P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]),
@@ -309,11 +313,50 @@ def moe_permute(x: torch.Tensor, topk_idx: torch.Tensor, offsets: torch.Tensor) 
     return out
 
 
+def moe_permute_padded_max_rows(T: int, E: int, k: int, align: int) -> int:
+    """Rows a padded dispatch may use, T*k + E*(align-1), with no host sync."""
+    return int(lib().moe_permute_padded_max_rows(T, E, k, int(align)))
+
+
+def moe_permute_padded(x: torch.Tensor, topk_idx: torch.Tensor, offsets: torch.Tensor, align: int,
+                       topk_prob: Optional[torch.Tensor] = None) -> dict:
+    """Token dispatch with each expert block rounded up to a multiple of align
+    rows (zero pad rows). x_perm, prob_perm and sorted_token have the dropless
+    bound T*k + E*(align-1) rows; padded_offsets[E] says how many are used."""
+    _need(x, torch.bfloat16, "x")
+    _need(topk_idx, torch.int32, "topk_idx")
+    _need(offsets, torch.int32, "offsets")
+    if topk_prob is not None:
+        _need(topk_prob, torch.float32, "topk_prob")
+    T, H = x.shape
+    k = topk_idx.shape[1]
+    E = offsets.numel() - 1
+    dev = x.device
+    R = max(moe_permute_padded_max_rows(T, E, k, align), 1)
+    out = {
+        "padded_offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+        "x_perm": torch.empty((R, H), dtype=torch.bfloat16, device=dev),
+        "prob_perm": torch.empty(R, dtype=torch.float32, device=dev) if topk_prob is not None else None,
+        "sorted_token": torch.empty(R, dtype=torch.int32, device=dev),
+        "row_of": torch.empty((T, k), dtype=torch.int32, device=dev),
+    }
+    ws = _workspace(lib().moe_permute_workspace_size(T, E, k), dev)
+    _check(lib().moe_permute_padded(_ptr(x), T, H, _ptr(topk_idx), _ptr(topk_prob), k, _ptr(offsets), E,
+                                    int(align), _ptr(out["padded_offsets"]), _ptr(out["x_perm"]),
+                                    _ptr(out["prob_perm"]), _ptr(out["sorted_token"]), _ptr(out["row_of"]),
+                                    _ptr(ws), ws.numel(), _stream()), "moe_permute_padded")
+    return out
+
+
 def moe_grouped_mlp(x_perm: torch.Tensor, offsets: torch.Tensor, w_gate_up: torch.Tensor,
-                    w_down: torch.Tensor, save: bool = False) -> dict:
-    """Grouped SwiGLU expert MLP over expert-contiguous rows."""
+                    w_down: torch.Tensor, save: bool = False, row_scale: Optional[torch.Tensor] = None) -> dict:
+    """Grouped SwiGLU expert MLP over expert-contiguous rows. With row_scale
+    (fp32 [A]) the activation of row r is multiplied by row_scale[r] before
+    FC2 (ScaledSwiGLU), and the combine must then run without weights."""
     for t, n in ((x_perm, "x_perm"), (w_gate_up, "w_gate_up"), (w_down, "w_down")):
         _need(t, torch.bfloat16, n)
+    if row_scale is not None:
+        _need(row_scale, torch.float32, "row_scale")
     _need(offsets, torch.int32, "offsets")
     A, H = x_perm.shape
     E, _, I2 = w_gate_up.shape
@@ -323,10 +366,17 @@ def moe_grouped_mlp(x_perm: torch.Tensor, offsets: torch.Tensor, w_gate_up: torc
            "gu": torch.empty((A, 2 * I), dtype=torch.bfloat16, device=dev) if save else None,
            "h": torch.empty((A, I), dtype=torch.bfloat16, device=dev) if save else None}
     ws = _workspace(0 if save else lib().moe_grouped_mlp_workspace_size(A, E, H, I), dev)
-    _check(lib().moe_grouped_mlp(_ptr(x_perm), A, _ptr(offsets), E, H, I, _ptr(w_gate_up),
-                                 _ptr(w_down), _ptr(out["y_perm"]), _ptr(out["gu"]), _ptr(out["h"]),
-                                 _ptr(ws), ws.numel(), _stream()), "moe_grouped_mlp")
+    _check(lib().moe_grouped_mlp_scaled(_ptr(x_perm), A, _ptr(offsets), E, H, I, _ptr(w_gate_up),
+                                        _ptr(w_down), _ptr(row_scale), _ptr(out["y_perm"]), _ptr(out["gu"]),
+                                        _ptr(out["h"]), _ptr(ws), ws.numel(), _stream()), "moe_grouped_mlp")
     return out
+
+
+def moe_grouped_mlp_scaled(x_perm: torch.Tensor, offsets: torch.Tensor, w_gate_up: torch.Tensor,
+                           w_down: torch.Tensor, row_scale: torch.Tensor, save: bool = False) -> dict:
+    """Grouped MLP with ScaledSwiGLU: the routing weight of each row applied to
+    the activation before FC2 (combine then runs without weights)."""
+    return moe_grouped_mlp(x_perm, offsets, w_gate_up, w_down, save=save, row_scale=row_scale)
 
 
 def moe_unpermute_combine(y_perm: torch.Tensor, row_of: torch.Tensor,
@@ -340,12 +390,21 @@ def moe_unpermute_combine(y_perm: torch.Tensor, row_of: torch.Tensor,
     if shared_out is not None:
         _need(shared_out, torch.bfloat16, "shared_out")
     T, k = row_of.shape
-    H = y_perm.shape[1]
+    A, H = y_perm.shape
     out = torch.empty((T, H), dtype=torch.bfloat16, device=y_perm.device)
-    _check(lib().moe_unpermute_combine(_ptr(y_perm), _ptr(row_of), _ptr(topk_prob), T, k, H,
-                                       _ptr(shared_out), _ptr(out), _stream()),
+    _check(lib().moe_unpermute_combine_rows(_ptr(y_perm), A, _ptr(row_of), _ptr(topk_prob), T, k, H,
+                                            _ptr(shared_out), _ptr(out), _stream()),
            "moe_unpermute_combine")
     return out
+
+
+def moe_unpermute_combine_rows(y_perm: torch.Tensor, row_of: torch.Tensor,
+                               topk_prob: Optional[torch.Tensor] = None,
+                               shared_out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """moe_unpermute_combine for a y_perm with any number of rows (for example
+    a padded dispatch's); the binding's moe_unpermute_combine already passes
+    y_perm's row count."""
+    return moe_unpermute_combine(y_perm, row_of, topk_prob, shared_out)
 
 
 class LayerWorkspace:

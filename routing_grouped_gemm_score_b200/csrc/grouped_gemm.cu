@@ -96,6 +96,7 @@ struct Params {
     int I;                     // SwiGLU: offset of the up half in [g | u]
     int tma_out, tma_out2;     // single-CTA kernel: out / out2 have TMA store maps
     int mb_item;               // weight gradient: M blocks per item
+    const float* row_scale;    // SwiGLU forward: h[r] *= row_scale[r] (NULL: 1)
     unsigned* err;
 };
 
@@ -450,6 +451,8 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
         const int n0 = t.n_blk * (n_tile / 2);
         const int nvalid = min(max(t.rows - warp_r0, 0), 32);
         const int64_t row0 = (int64_t)t.row0 + warp_r0;
+        // ScaledSwiGLU: the routing weight of the lane's row, applied before FC2
+        const float rs = (p.row_scale && lane < nvalid) ? __ldg(p.row_scale + row0 + lane) : 1.0f;
 #pragma unroll 1
         for (int i = 0; i < em.chunks; ++i) {
             const int c0 = em.c_lo + 32 * i;
@@ -464,7 +467,7 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
                             p.I + n0 + c0, (int)row0);
             }
 #pragma unroll
-            for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i]) * u[i];     // h, in place
+            for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i]) * u[i] * rs;     // h, in place
             put_block32(buf, p.out + row0 * p.ldo + n0 + c0, p.ldo, nvalid, g, lane, tmC, n0 + c0, (int)row0);
         }
     } else if (EPI == kEpiSwigluBwd) {
@@ -1514,7 +1517,7 @@ bool make_out_map(CUtensorMap* m, const bf16* out, int64_t rows, uint64_t cols) 
 
 cudaError_t gemm_gate_up_swiglu(const bf16* x, int64_t rows, const int32_t* offsets, int E, int H,
                                 int I, const bf16* w_gate_up, bf16* h, bf16* gu_save,
-                                cudaStream_t st, unsigned* err) {
+                                cudaStream_t st, unsigned* err, const float* row_scale) {
     if (rows == 0) return cudaSuccess;
     CUtensorMap ta, ta64, tb;
     if (!make_map_2d(&ta, x, H, rows, H, BK, 128)) return cudaErrorInvalidValue;
@@ -1531,6 +1534,7 @@ cudaError_t gemm_gate_up_swiglu(const bf16* x, int64_t rows, const int32_t* offs
     p.ldo = I;
     p.out2 = gu_save;
     p.ldo2 = 2 * (int64_t)I;
+    p.row_scale = row_scale;
     CUtensorMap tc, tc2;
     if (!make_out_map(&tc, h, rows, I)) return cudaErrorInvalidValue;
     if (gu_save && !make_out_map(&tc2, gu_save, rows, 2 * (uint64_t)I)) return cudaErrorInvalidValue;

@@ -348,6 +348,46 @@ moe_status moe_permute(const moe_bf16* x, int64_t T, int H, const int32_t* topk_
     return from_cuda(e);
 }
 
+int64_t moe_permute_padded_max_rows(int64_t T, int E, int k, int align) {
+    if (!shape_ok(T, E, k) || align < 1 || align > 65536) return 0;
+    const int64_t m = T * k + (int64_t)E * (align - 1);
+    return m < (int64_t(1) << 31) ? m : 0;
+}
+
+moe_status moe_permute_padded(const moe_bf16* x, int64_t T, int H, const int32_t* topk_idx,
+                              const float* topk_prob, int k, const int32_t* offsets, int E, int align,
+                              int32_t* padded_offsets, moe_bf16* x_perm, float* prob_perm,
+                              int32_t* sorted_token, int32_t* row_of, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+    if (!shape_ok(T, E, k) || H <= 0 || H % 8 != 0) return MOE_ERR_INVALID_ARG;
+    if (moe_permute_padded_max_rows(T, E, k, align) <= 0 && T > 0) return MOE_ERR_INVALID_ARG;
+    if (align < 1 || align > 65536 || !offsets || !padded_offsets || !aligned16(offsets) ||
+        !aligned16(padded_offsets))
+        return MOE_ERR_INVALID_ARG;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) return from_cuda(cudaMemsetAsync(padded_offsets, 0, sizeof(int32_t) * (E + 1), st));
+    if (!x || !topk_idx || !x_perm || !sorted_token || !row_of) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(x_perm) || !aligned16(topk_idx) || !aligned16(sorted_token) ||
+        !aligned16(row_of) || (prob_perm && (!topk_prob || !aligned16(prob_perm) || !aligned16(topk_prob))))
+        return MOE_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < route_scratch_bytes(T, E, k)) return MOE_ERR_WORKSPACE;
+    unsigned* err = device_error_word();
+    if (!err) return MOE_ERR_CUDA;
+    const RouteScratch rs = carve_route_scratch(workspace, T, E, k);
+    cudaError_t e = launch_pad_offsets(offsets, E, align, padded_offsets, st);
+    if (e == cudaSuccess) e = launch_rank_from_indices(topk_idx, T, E, k, rs, st, err);
+    if (e == cudaSuccess) e = launch_expert_scan(T, E, rs, nullptr, nullptr, st);
+    if (e == cudaSuccess)
+        e = launch_permute(reinterpret_cast<const bf16*>(x), T, H, topk_idx, k, padded_offsets, E, rs,
+                           reinterpret_cast<bf16*>(x_perm), sorted_token, row_of, st, err,
+                           moe_permute_padded_max_rows(T, E, k, align));
+    if (e == cudaSuccess)
+        e = launch_pad_fill(offsets, padded_offsets, E, H, reinterpret_cast<bf16*>(x_perm), sorted_token,
+                            prob_perm, st);
+    if (e == cudaSuccess && prob_perm) e = launch_prob_perm(topk_prob, row_of, T * k, prob_perm, st);
+    return from_cuda(e);
+}
+
 size_t moe_grouped_mlp_workspace_size(int64_t A, int E, int H, int I) {
     if (A < 0 || E < 1 || E > 256 || !dims_ok(H, I)) return 0;
     Carver c(nullptr);
@@ -359,6 +399,15 @@ moe_status moe_grouped_mlp(const moe_bf16* x_perm, int64_t A, const int32_t* off
                            int H, int I, const moe_bf16* w_gate_up, const moe_bf16* w_down,
                            moe_bf16* y_perm, moe_bf16* gu_save, moe_bf16* h_save,
                            void* workspace, size_t workspace_bytes, void* stream) {
+    return moe_grouped_mlp_scaled(x_perm, A, offsets, E, H, I, w_gate_up, w_down, nullptr, y_perm, gu_save,
+                                  h_save, workspace, workspace_bytes, stream);
+}
+
+moe_status moe_grouped_mlp_scaled(const moe_bf16* x_perm, int64_t A, const int32_t* offsets, int E,
+                                  int H, int I, const moe_bf16* w_gate_up, const moe_bf16* w_down,
+                                  const float* row_scale, moe_bf16* y_perm, moe_bf16* gu_save,
+                                  moe_bf16* h_save, void* workspace, size_t workspace_bytes, void* stream) {
+    if (row_scale && !aligned16(row_scale)) return MOE_ERR_INVALID_ARG;
     if (A < 0 || A >= (int64_t(1) << 31) || E < 1 || E > 256) return MOE_ERR_INVALID_ARG;
     if (H <= 0 || I <= 0) return MOE_ERR_INVALID_ARG;
     if (!dims_ok(H, I)) return MOE_ERR_UNSUPPORTED;
@@ -378,7 +427,7 @@ moe_status moe_grouped_mlp(const moe_bf16* x_perm, int64_t A, const int32_t* off
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = gemm_gate_up_swiglu(reinterpret_cast<const bf16*>(x_perm), A, offsets, E, H, I,
                                         reinterpret_cast<const bf16*>(w_gate_up), h,
-                                        reinterpret_cast<bf16*>(gu_save), st, err);
+                                        reinterpret_cast<bf16*>(gu_save), st, err, row_scale);
     if (e == cudaSuccess)
         e = gemm_down(h, A, offsets, E, H, I, reinterpret_cast<const bf16*>(w_down),
                       reinterpret_cast<bf16*>(y_perm), st, err);
@@ -388,8 +437,16 @@ moe_status moe_grouped_mlp(const moe_bf16* x_perm, int64_t A, const int32_t* off
 moe_status moe_unpermute_combine(const moe_bf16* y_perm, const int32_t* row_of,
                                  const float* topk_prob, int64_t T, int k, int H,
                                  const moe_bf16* shared_out, moe_bf16* out, void* stream) {
+    return moe_unpermute_combine_rows(y_perm, T * (int64_t)k, row_of, topk_prob, T, k, H, shared_out, out,
+                                      stream);
+}
+
+moe_status moe_unpermute_combine_rows(const moe_bf16* y_perm, int64_t y_rows, const int32_t* row_of,
+                                      const float* topk_prob, int64_t T, int k, int H,
+                                      const moe_bf16* shared_out, moe_bf16* out, void* stream) {
     if (T < 0 || k < 1 || k > 16 || H <= 0 || H % 8 != 0 || T * (int64_t)k >= (int64_t(1) << 31))
         return MOE_ERR_INVALID_ARG;
+    if (y_rows < 0 || y_rows >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     if (!y_perm || !row_of || !out) return MOE_ERR_INVALID_ARG;
     if (!aligned16(y_perm) || !aligned16(row_of) || !aligned16(out) ||
@@ -398,7 +455,7 @@ moe_status moe_unpermute_combine(const moe_bf16* y_perm, const int32_t* row_of,
     unsigned* err = device_error_word();
     if (!err) return MOE_ERR_CUDA;
     return from_cuda(launch_combine(reinterpret_cast<const bf16*>(y_perm), row_of, topk_prob, T, k,
-                                    H, T * k, reinterpret_cast<const bf16*>(shared_out),
+                                    H, y_rows, reinterpret_cast<const bf16*>(shared_out),
                                     reinterpret_cast<bf16*>(out), static_cast<cudaStream_t>(stream),
                                     err));
 }

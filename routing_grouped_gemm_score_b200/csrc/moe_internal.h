@@ -60,9 +60,17 @@ cudaError_t launch_rank_from_indices(const int32_t* topk_idx, int64_t T, int E, 
 // Turns block counts into exclusive prefixes; writes counts/offsets if given.
 cudaError_t launch_expert_scan(int64_t T, int E, const RouteScratch& rs, int32_t* counts,
                                int32_t* offsets, cudaStream_t st);
+// Padded dispatch (Token permutation, Padding and alignment).
+cudaError_t launch_pad_offsets(const int32_t* offsets, int E, int align, int32_t* padded_offsets, cudaStream_t st);
+cudaError_t launch_pad_fill(const int32_t* offsets, const int32_t* padded_offsets, int E, int H, bf16* x_perm,
+                            int32_t* sorted_token, float* prob_perm, cudaStream_t st);
+cudaError_t launch_prob_perm(const float* topk_prob, const int32_t* row_of, int64_t n, float* prob_perm,
+                             cudaStream_t st);
+// row_bound: rows of x_perm and sorted_token (<= 0: T*k, the unpadded dispatch)
 cudaError_t launch_permute(const bf16* x, int64_t T, int H, const int32_t* topk_idx, int k,
                            const int32_t* offsets, int E, const RouteScratch& rs, bf16* x_perm,
-                           int32_t* sorted_token, int32_t* row_of, cudaStream_t st, unsigned* err);
+                           int32_t* sorted_token, int32_t* row_of, cudaStream_t st, unsigned* err,
+                           int64_t row_bound = 0);
 
 // The fixed scratch array behind moe_router_topk_noalloc (routing.cu).
 size_t router_noalloc_capacity();
@@ -82,7 +90,7 @@ cudaError_t launch_combine_backward(const bf16* dout, const bf16* y_perm, const 
 // offsets NULL: one group of `rows` rows using the weights of group 0.
 cudaError_t gemm_gate_up_swiglu(const bf16* x, int64_t rows, const int32_t* offsets, int E, int H,
                                 int I, const bf16* w_gate_up, bf16* h, bf16* gu_save,
-                                cudaStream_t st, unsigned* err);
+                                cudaStream_t st, unsigned* err, const float* row_scale = nullptr);
 // down: y[r] = h[r] Wd[e]
 cudaError_t gemm_down(const bf16* h, int64_t rows, const int32_t* offsets, int E, int H, int I,
                       const bf16* w_down, bf16* y, cudaStream_t st, unsigned* err);

@@ -629,6 +629,63 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+// Padded dispatch (Transformer Engine "Mixture of Experts", Token permutation,
+// Padding and alignment): each expert's block is rounded up to a multiple of
+// align rows, an empty block stays empty, and the permute kernels then run on
+// the padded offsets, so the rows keep their unpadded order inside a block.
+// pad_offsets_kernel: one block, one thread per expert, an exclusive scan of
+// the rounded counts in expert order.
+__global__ void __launch_bounds__(256)
+    pad_offsets_kernel(const int32_t* __restrict__ offsets, int E, int align, int32_t* __restrict__ padded) {
+    __shared__ int32_t warp_sum[8];
+    const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
+    int32_t c = 0;
+    if (e < E) {
+        const int32_t cnt = __ldg(offsets + e + 1) - __ldg(offsets + e);
+        c = cnt > 0 ? (int32_t)(((int64_t)cnt + align - 1) / align * align) : 0;
+    }
+    int32_t incl = c;   // inclusive scan within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int32_t v = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) warp_sum[warp] = incl;
+    __syncthreads();
+    int32_t base = 0;
+    for (int w = 0; w < warp; ++w) base += warp_sum[w];
+    if (e < E) padded[e + 1] = base + incl;
+    if (e == 0) padded[0] = 0;
+}
+
+// Pad rows of expert e (blockIdx.x): [padded[e] + count, padded[e+1]). Their
+// x_perm rows become zeros, their sorted_token -1 and their weight 0.
+__global__ void __launch_bounds__(256)
+    pad_fill_kernel(const int32_t* __restrict__ offsets, const int32_t* __restrict__ padded, int H8,
+                    uint4* __restrict__ x_perm, int32_t* __restrict__ sorted_token, float* __restrict__ prob_perm) {
+    const int e = blockIdx.x;
+    const int64_t cnt = (int64_t)__ldg(offsets + e + 1) - __ldg(offsets + e);
+    const int64_t r0 = (int64_t)__ldg(padded + e) + (cnt > 0 ? cnt : 0);
+    const int64_t r1 = __ldg(padded + e + 1);
+    if (r1 <= r0) return;
+    const int64_t n = (r1 - r0) * H8;
+    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) x_perm[r0 * H8 + i] = make_uint4(0, 0, 0, 0);
+    for (int64_t r = r0 + threadIdx.x; r < r1; r += blockDim.x) {
+        sorted_token[r] = -1;
+        if (prob_perm) prob_perm[r] = 0.0f;
+    }
+}
+
+// prob_perm[row_of[i]] = topk_prob[i]: the routing weight of each permuted row.
+__global__ void __launch_bounds__(256)
+    prob_perm_kernel(const float* __restrict__ topk_prob, const int32_t* __restrict__ row_of, int64_t n,
+                     float* __restrict__ prob_perm) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int32_t r = __ldg(row_of + i);
+        if (r >= 0) prob_perm[r] = __ldg(topk_prob + i);
+    }
+}
+
 // Scratch for moe_router_topk_noalloc: a fixed array in device memory, so the
 // call allocates nothing. Its size bounds the routing sizes that call accepts.
 constexpr size_t kNoAllocScratchBytes = (3u << 20) + 4096;
@@ -743,9 +800,33 @@ cudaError_t launch_expert_scan(int64_t T, int E, const RouteScratch& rs, int32_t
     return cudaGetLastError();
 }
 
+cudaError_t launch_pad_offsets(const int32_t* offsets, int E, int align, int32_t* padded_offsets, cudaStream_t st) {
+    pad_offsets_kernel<<<1, 256, 0, st>>>(offsets, E, align, padded_offsets);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pad_fill(const int32_t* offsets, const int32_t* padded_offsets, int E, int H, bf16* x_perm,
+                            int32_t* sorted_token, float* prob_perm, cudaStream_t st) {
+    pad_fill_kernel<<<(unsigned)E, 256, 0, st>>>(offsets, padded_offsets, H / 8, reinterpret_cast<uint4*>(x_perm),
+                                                sorted_token, prob_perm);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prob_perm(const float* topk_prob, const int32_t* row_of, int64_t n, float* prob_perm,
+                             cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    int64_t blocks = (n + 255) / 256;
+    const int64_t cap = (int64_t)sm_count() * 8;
+    if (blocks > cap) blocks = cap;
+    prob_perm_kernel<<<(unsigned)blocks, 256, 0, st>>>(topk_prob, row_of, n, prob_perm);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_permute(const bf16* x, int64_t T, int H, const int32_t* topk_idx, int k,
                            const int32_t* offsets, int E, const RouteScratch& rs, bf16* x_perm,
-                           int32_t* sorted_token, int32_t* row_of, cudaStream_t st, unsigned* err) {
+                           int32_t* sorted_token, int32_t* row_of, cudaStream_t st, unsigned* err,
+                           int64_t row_bound) {
+    const int64_t A = row_bound > 0 ? row_bound : T * k;   // rows of x_perm and sorted_token
     const int nb = (int)route_blocks(T);
     if (T == 0) return cudaSuccess;
     const int H8r = H / 8;
@@ -768,7 +849,7 @@ cudaError_t launch_permute(const bf16* x, int64_t T, int H, const int32_t* topk_
         permute_tokens_kernel<<<(unsigned)blocks, threads, 0, st>>>(
             reinterpret_cast<const uint4*>(x), T, H8r, topk_idx, k, offsets, E, rs.block_base, nb,
             route_tokens_per_block(T), rs.local_rank, reinterpret_cast<uint4*>(x_perm), sorted_token, row_of,
-            T * k, per_block, err);
+            A, per_block, err);
         return cudaGetLastError();
     }
     if (E > kPermMaxExperts) return cudaErrorInvalidValue;
@@ -785,7 +866,7 @@ cudaError_t launch_permute(const bf16* x, int64_t T, int H, const int32_t* topk_
     kern<<<(unsigned)blocks, kThreadsW, 0, st>>>(
         reinterpret_cast<const uint4*>(x), T, H8r, topk_idx, k, offsets, E, rs.block_base, nb,
         route_tokens_per_block(T), rs.local_rank, reinterpret_cast<uint4*>(x_perm), sorted_token, row_of,
-        T * k, err);
+        A, err);
     return cudaGetLastError();
 }
 
