@@ -247,6 +247,201 @@ __global__ void __launch_bounds__(kRouteThreads) router_topk_kernel(const Router
     rank_block(sel, t0, tpb, E, k, a.local_rank, a.block_base, a.nb);
 }
 
+// ---------------------------------------------------------------------------
+// Router for large T, one lane per token. A block holds 256 tokens, a warp 32.
+// The warp stages its tokens' logits in shared memory 32 experts at a time
+// (one coalesced 16-byte load per lane per 4 rows); each lane then reads its
+// own token's row and keeps that token's best 8 experts in registers: every 8
+// experts are sorted with Batcher's network (19 compare-exchanges) and merged
+// into the running 8 with one bitonic step (8 pairs) and a bitonic clean
+// (12 pairs). Every compare-exchange uses the selection order of the warp
+// kernel above (larger key first, then the lower expert index), so the picks
+// are the same, and the weights are computed in the same order of
+// operations. The block's counts come from one bit per (expert, token) in
+// shared memory: a token's rank inside its rank block (tpb tokens, as in the
+// warp kernel) is a population count of the bits below it.
+// Restrictions: E a multiple of 32 (up to 256), k <= 8, softmax weights
+// renormalised over the picks or sigmoid weights; other cases use the warp
+// kernel.
+constexpr int kLaneTokens = 256;                 // tokens (threads) per block
+constexpr int64_t kLaneMinTokens = 32768;        // below this, the warp kernel (more blocks, lower latency)
+constexpr int kLaneChunk = 32;                   // experts staged per step
+constexpr int kLanePitch = kLaneChunk + 4;       // floats per staged row (conflict-free 16-byte reads)
+
+// A selection entry as one 64-bit value: the order key above, the complement
+// of the expert index below, so that a larger value ranks strictly better in
+// the selection order (larger key, then the lower index). A compare-exchange
+// is then a branch-free max/min. 0 ranks below every expert (key 0 with the
+// largest index).
+__device__ __forceinline__ uint64_t lane_entry(uint32_t key, uint32_t e) {
+    return ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - e);
+}
+__device__ __forceinline__ uint32_t lane_key(uint64_t v) { return (uint32_t)(v >> 32); }
+__device__ __forceinline__ uint32_t lane_expert(uint64_t v) { return 0xFFFFFFFFu - (uint32_t)v; }
+
+__device__ __forceinline__ void lane_cx(uint64_t& a, uint64_t& b) {   // a := better, b := worse
+    const uint64_t hi = a > b ? a : b, lo = a > b ? b : a;
+    a = hi;
+    b = lo;
+}
+
+__device__ __forceinline__ void lane_sort8(uint64_t (&v)[8]) {
+    constexpr int net[19][2] = {{0, 1}, {2, 3}, {4, 5}, {6, 7}, {0, 2}, {1, 3}, {4, 6},
+                                {5, 7}, {1, 2}, {5, 6}, {0, 4}, {1, 5}, {2, 6}, {3, 7},
+                                {2, 4}, {3, 5}, {1, 2}, {3, 4}, {5, 6}};
+#pragma unroll
+    for (int c = 0; c < 19; ++c) lane_cx(v[net[c][0]], v[net[c][1]]);
+}
+
+// top (best first) := the best 8 of top and g (both best first).
+__device__ __forceinline__ void lane_merge8(uint64_t (&t)[8], uint64_t (&g)[8]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) t[i] = t[i] > g[7 - i] ? t[i] : g[7 - i];   // bitonic, holds the best 8
+#pragma unroll
+    for (int i = 0; i < 4; ++i) lane_cx(t[i], t[i + 4]);
+#pragma unroll
+    for (int i = 0; i < 8; i += 4) {
+        lane_cx(t[i], t[i + 2]);
+        lane_cx(t[i + 1], t[i + 3]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) lane_cx(t[i], t[i + 1]);
+}
+
+// Tokens of [lo, hi) (block-local indices, hi <= 256) whose bit is set in m[0..7].
+__device__ __forceinline__ int lane_count(const uint32_t* m, int lo, int hi) {
+    int c = 0;
+    for (int w = lo >> 5; w <= (hi - 1) >> 5 && lo < hi; ++w) {
+        uint32_t bits = m[w];
+        const int b0 = w * 32;
+        if (lo > b0) bits &= ~0u << (lo - b0);
+        if (hi < b0 + 32) bits &= (hi - b0) > 0 ? (~0u >> (32 - (hi - b0))) : 0u;
+        c += __popc(bits);
+    }
+    return c;
+}
+
+template <int KC>
+__global__ void __launch_bounds__(kLaneTokens)
+    router_lane_kernel(const RouterArgs a) {
+    __shared__ __align__(16) float stage[kLaneTokens / 32][32][kLanePitch];   // 36 KB
+    __shared__ uint32_t mask[256][kLaneTokens / 32];                          // 8 KB
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = a.E;
+    const int64_t t0 = (int64_t)blockIdx.x * kLaneTokens;
+    const int64_t t = t0 + threadIdx.x;
+    const bool live = t < a.T;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *a.ticket = 0u;
+    for (int i = threadIdx.x; i < E * (kLaneTokens / 32); i += blockDim.x) (&mask[0][0])[i] = 0u;
+
+    uint64_t top[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) top[i] = 0u;   // below every expert
+    float(*st)[kLanePitch] = stage[warp];
+    const int64_t wrow0 = t0 + warp * 32;
+    for (int c0 = 0; c0 < E; c0 += kLaneChunk) {
+        // stage rows wrow0 .. +31, experts c0 .. c0+31: lane -> row 4i + lane/8, 4 experts
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int r = 4 * i + (lane >> 3), q = lane & 7;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (wrow0 + r < a.T) v = __ldg(reinterpret_cast<const float4*>(a.logits + (wrow0 + r) * E + c0) + q);
+            *reinterpret_cast<float4*>(&st[r][4 * q]) = v;
+        }
+        __syncwarp();
+#pragma unroll
+        for (int g = 0; g < kLaneChunk; g += 8) {
+            const float4 v0 = *reinterpret_cast<const float4*>(&st[lane][g]);
+            const float4 v1 = *reinterpret_cast<const float4*>(&st[lane][g + 4]);
+            const float l[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            uint64_t gv[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int e = c0 + g + q;
+                float score = l[q];
+                if (a.bias) score = 1.0f / (1.0f + expf(-l[q])) + __ldg(a.bias + e);
+                gv[q] = lane_entry(float_order_key(score), (uint32_t)e);
+            }
+            lane_sort8(gv);
+            lane_merge8(top, gv);
+        }
+        __syncwarp();   // the stage is read before the next chunk overwrites it
+    }
+
+    // routing weights, in the warp kernel's order of operations
+    const int k = KC;
+    uint32_t tk[8], te[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        tk[j] = lane_key(top[j]);
+        te[j] = lane_expert(top[j]);
+    }
+    float lsel[8], p[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        lsel[j] = 0.0f;
+        if (j < k && live) lsel[j] = a.bias ? __ldg(a.logits + t * E + te[j]) : order_key_to_float(tk[j]);
+    }
+    if (a.score_fn == MOE_SCORE_SOFTMAX) {
+        const float m = lsel[0];   // the first pick holds the largest logit of the picks (or NaN)
+        float ex[8], sum = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            ex[j] = j < k ? expf(lsel[j] - m) : 0.0f;
+            if (j < k) sum += ex[j];
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) p[j] = ex[j] / sum;
+    } else {
+        float sg[8], sum = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            sg[j] = j < k ? 1.0f / (1.0f + expf(-lsel[j])) : 0.0f;
+            if (j < k) sum += sg[j];
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) p[j] = a.renormalize ? sg[j] / sum : sg[j];
+    }
+    if (live) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if (j >= k) break;
+            a.topk_idx[t * k + j] = (int32_t)te[j];
+            a.topk_prob[t * k + j] = p[j] * a.scaling;
+        }
+        if (a.routing_map) {
+            uint4* mrow = reinterpret_cast<uint4*>(a.routing_map + t * E);
+            for (int i = 0; i < E / 16; ++i) mrow[i] = make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (j < k) a.routing_map[t * E + te[j]] = 1;
+        }
+    }
+
+    // counts and ranks per rank block of tpb tokens
+    __syncthreads();   // masks zeroed
+    if (live) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (j < k) atomicOr(&mask[te[j]][warp], 1u << lane);
+    }
+    __syncthreads();
+    const int tpb = a.tpb;
+    if (live) {
+        const int lo = (threadIdx.x / tpb) * tpb;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (j < k) a.local_rank[t * k + j] = lane_count(mask[te[j]], lo, threadIdx.x);
+    }
+    const int nsub = kLaneTokens / tpb;
+    const int64_t sb0 = t0 / tpb;
+    for (int i = threadIdx.x; i < E * nsub; i += blockDim.x) {
+        const int e = i / nsub, sb = i - e * nsub;
+        if (sb0 + sb >= a.nb) continue;
+        a.block_base[(int64_t)e * a.nb + sb0 + sb] = lane_count(mask[e], sb * tpb, (sb + 1) * tpb);
+    }
+}
+
 // Router backward: dL/dlogits from dL/dtopk_prob, one warp per token, fp32.
 // Lane j < k holds pick j: its expert, logit and g_j = scaling * dprob[t,j].
 // The formulas per mode are those of the forward's weights differentiated
@@ -748,6 +943,27 @@ cudaError_t launch_router_topk(const float* logits, int64_t T, int E, int k,
     a.ticket = rs.ticket;
     a.nb = (int)route_blocks(T);
     a.tpb = route_tokens_per_block(T);
+    // Large T: the lane-per-token kernel where it applies. MOE_ROUTER=lane|warp
+    // overrides the choice (the tests run both on the same inputs).
+    const char* force = getenv("MOE_ROUTER");
+    const bool lane_ok = E % 32 == 0 && E <= 256 && k <= 8 && kLaneTokens % a.tpb == 0 &&
+                         (opts.score_fn == MOE_SCORE_SIGMOID || opts.renormalize);
+    const bool use_lane = lane_ok && (force ? force[0] == 'l' : T >= kLaneMinTokens);
+    if (use_lane) {
+        const dim3 lgrid((unsigned)((T + kLaneTokens - 1) / kLaneTokens)), lblock(kLaneTokens);
+        switch (k) {
+            case 1: router_lane_kernel<1><<<lgrid, lblock, 0, st>>>(a); break;
+            case 2: router_lane_kernel<2><<<lgrid, lblock, 0, st>>>(a); break;
+            case 3: router_lane_kernel<3><<<lgrid, lblock, 0, st>>>(a); break;
+            case 4: router_lane_kernel<4><<<lgrid, lblock, 0, st>>>(a); break;
+            case 5: router_lane_kernel<5><<<lgrid, lblock, 0, st>>>(a); break;
+            case 6: router_lane_kernel<6><<<lgrid, lblock, 0, st>>>(a); break;
+            case 7: router_lane_kernel<7><<<lgrid, lblock, 0, st>>>(a); break;
+            default: router_lane_kernel<8><<<lgrid, lblock, 0, st>>>(a); break;
+        }
+        (void)err;
+        return cudaGetLastError();
+    }
     const dim3 grid((unsigned)a.nb), block(kRouteThreads);
     if (E <= 32) launch_router_k<1>(a, grid, block, st);
     else if (E <= 64) launch_router_k<2>(a, grid, block, st);

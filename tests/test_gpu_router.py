@@ -158,3 +158,69 @@ def test_expert_bias_update_matches_oracle(E):
     np.testing.assert_allclose(bias.cpu().numpy(), ref, rtol=0, atol=1e-6 * 1e-3 + 1e-7 * np.abs(ref).max())
     g, o = run_both(logits, k, 1, False, 1.0, bias.cpu())
     check(g, o)
+
+
+LANE_CASES = [(1, 32, 1, "softmax_renorm"), (255, 64, 2, "softmax_renorm"), (256, 128, 8, "softmax_renorm"),
+              (1000, 128, 8, "sigmoid"), (777, 256, 3, "sigmoid_renorm"), (513, 96, 6, "softmax_renorm"),
+              (40001, 128, 8, "softmax_renorm"), (9000, 160, 7, "sigmoid")]
+
+
+def _router_outputs(logits, k, score, renorm, kernel, monkeypatch, bias=None, scaling=1.0):
+    import routing_grouped_gemm_score_b200 as m
+    monkeypatch.setenv("MOE_ROUTER", kernel)
+    opts = m.RouterOpts(score, renorm, scaling, bias)
+    g = m.moe_router_topk(logits, k, opts, routing_map=True)
+    torch.cuda.synchronize()
+    assert m.moe_get_device_status() == 0
+    return {n: v.clone() for n, v in g.items() if v is not None}
+
+
+@pytest.mark.parametrize("T,E,k,mode", LANE_CASES)
+def test_lane_router_matches_warp_router_bit_for_bit(T, E, k, mode, monkeypatch):
+    """The lane-per-token kernel (large T) and the warp-per-token kernel give
+    the same bits in every output, on ragged T (not a multiple of the
+    256-token lane block), E = 32 .. 256 and k = 1 .. 8."""
+    score, renorm = MODES[mode]
+    g_ = torch.Generator().manual_seed(T * 3 + E + k)
+    logits = (torch.randn((T, E), generator=g_) * 2).cuda()
+    a = _router_outputs(logits, k, score, renorm, "lane", monkeypatch)
+    b = _router_outputs(logits, k, score, renorm, "warp", monkeypatch)
+    for n in b:
+        assert torch.equal(a[n].view(torch.uint8), b[n].view(torch.uint8)), n
+
+
+@pytest.mark.parametrize("mode", ["softmax_renorm", "sigmoid", "sigmoid_renorm"])
+def test_lane_router_degenerate_values_bias_and_scaling(mode, monkeypatch):
+    score, renorm = MODES[mode]
+    g_ = torch.Generator().manual_seed(41)
+    logits = torch.round(torch.randn((700, 128), generator=g_) * 2) / 2      # many exact ties
+    logits[0, 0] = float("nan")
+    logits[1, 77] = float("nan")
+    logits[2] = float("-inf")
+    logits[3] = -0.0
+    logits[3, 100] = 0.0
+    logits[4, :120] = float("nan")
+    logits = logits.cuda()
+    bias = (torch.randn(128, generator=g_) * 0.3).cuda() if score == 1 else None
+    a = _router_outputs(logits, 8, score, renorm, "lane", monkeypatch, bias=bias, scaling=1.5)
+    b = _router_outputs(logits, 8, score, renorm, "warp", monkeypatch, bias=bias, scaling=1.5)
+    for n in b:
+        assert torch.equal(a[n].view(torch.uint8), b[n].view(torch.uint8)), n
+
+
+def test_lane_router_ranks_drive_the_same_dispatch(monkeypatch):
+    """The fused layer permutes with the router's per-block ranks: the lane
+    kernel's ranks give the same permutation and output bits."""
+    import routing_grouped_gemm_score_b200 as m
+    w = wl.WORKLOADS["qwen3_30b_a3b"].scaled(T=1500, H=256, I=128, E=64)
+    d = wl.make_inputs(w, "cuda")
+    res = {}
+    for kernel in ("lane", "warp"):
+        monkeypatch.setenv("MOE_ROUTER", kernel)
+        out, st = m.moe_layer_forward(d["logits"], d["x"], d["w_gate_up"], d["w_down"], w.k,
+                                      save_for_backward=True)
+        torch.cuda.synchronize()
+        assert m.moe_get_device_status() == 0
+        res[kernel] = (out.clone(), st["row_of"].clone(), st["x_perm"].clone(), st["offsets"].clone())
+    for a, b in zip(res["lane"], res["warp"]):
+        assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
