@@ -1,21 +1,23 @@
 // routing.cu -- router (score function + top-k + routing weights), rank and
-// expert-offset scan, and the permute (token dispatch) kernel.
+// expert-offset scan, the router's backward, the expert-bias update, and the
+// permute (token dispatch) kernels, padded dispatch included.
 //
-// Transformer Engine "Mixture of Experts", sections Router and Token
-// dispatch; te_mixtral.py TEMixtralSparseMoeBlock.forward.
+// Transformer Engine "Mixture of Experts", sections Router, Token dispatch
+// and Padding and alignment; te_mixtral.py TEMixtralSparseMoeBlock.forward.
 //
 // Design: one warp per token. A lane holds the scores of experts lane,
 // lane+32, ... in registers. The k experts are picked in k rounds; each round
 // is two single-instruction warp reductions: the largest order key (the score
 // mapped to an unsigned integer that sorts like the float), then the lowest
 // expert index among the lanes holding it, which breaks ties toward the lower
-// index. The choice is made on
-// the logit itself: softmax and sigmoid are increasing, so the ranking is
-// the same and no rounding of the score function can create a tie. Ranks
-// inside each expert are counted per block of 64 tokens in shared memory, in
-// token order, and an exclusive scan over the token blocks turns them into
-// global rows. A block holds 8 to 64 tokens (route_tokens_per_block). Positions never come from atomics, so the permutation is the
-// same on every run.
+// index. The choice is made on the logit itself: softmax and sigmoid are
+// increasing, so the ranking is the same and no rounding of the score
+// function can create a tie. For large T a lane-per-token kernel makes the
+// same choice with sorting networks (router_lane_kernel). Ranks inside each
+// expert are counted per block of 8 to 64 tokens (route_tokens_per_block) in
+// shared memory, in token order, and an exclusive scan over the token blocks
+// turns them into global rows. Positions never come from atomics, so the
+// permutation is the same on every run.
 #include <cstdlib>
 #include <mutex>
 
@@ -1048,9 +1050,9 @@ cudaError_t launch_permute(const bf16* x, int64_t T, int H, const int32_t* topk_
     const int H8r = H / 8;
     // Token-range register kernel for rows up to 4096 wide, warp per token
     // otherwise. Measured inside the steps on B200 (fraction of HBM): k=8,
-    // H=2048: 0.73 against 0.67 (warp) and 0.68 (bulk copies, removed); k=2,
-    // H=4096: 0.67 against 0.64 and 0.57; H=5120: warp 0.76 against bulk
-    // 0.73. MOE_PERMUTE=warp selects the warp kernel for any width.
+    // H=2048: 0.73 against 0.67 for the warp kernel; k=2, H=4096: 0.67
+    // against 0.64; H=5120: warp 0.76. MOE_PERMUTE=warp selects the warp
+    // kernel for any width.
     const char* force = getenv("MOE_PERMUTE");
     const bool regs = H8r <= 512 && !(force && force[0] == 'w');
     if (regs) {
