@@ -252,42 +252,93 @@ __global__ void __launch_bounds__(kRouteThreads) router_topk_kernel(const Router
 // ---------------------------------------------------------------------------
 // Router for large T, one lane per token. A block holds 256 tokens, a warp 32.
 // The warp stages its tokens' logits in shared memory 32 experts at a time
-// (one coalesced 16-byte load per lane per 4 rows); each lane then reads its
-// own token's row and keeps that token's best 8 experts in registers: every 8
+// (one coalesced 16-byte load per lane per 4 rows; the next chunk's loads are
+// in flight while the current chunk is sorted); each lane then reads its own
+// token's row and keeps that token's best 8 experts in registers: every 8
 // experts are sorted with Batcher's network (19 compare-exchanges) and merged
 // into the running 8 with one bitonic step (8 pairs) and a bitonic clean
-// (12 pairs). Every compare-exchange uses the selection order of the warp
-// kernel above (larger key first, then the lower expert index), so the picks
-// are the same, and the weights are computed in the same order of
-// operations. The block's counts come from one bit per (expert, token) in
-// shared memory: a token's rank inside its rank block (tpb tokens, as in the
-// warp kernel) is a population count of the bits below it.
+// (12 pairs).
+//
+// The sorting runs on 32-bit entries: the top bits of the score's signed
+// order key, with the complement of the expert index in the low 7 bits (E <=
+// 128) or 8 bits, so a compare-exchange is one integer max and one min.
+// Between entries whose prefixes differ this is the exact selection order
+// (larger score, then the lower index); entries that share a prefix are
+// ordered by index alone, which is exact only when their scores are equal.
+// The kernel therefore also keeps the entry just after the picks (for k = 8
+// the best entry any merge dropped; for k < 8 the (k+1)-th of the running 8)
+// and checks the neighbours (+0 and -0 count as one prefix):
+//  - the last pick and that entry share a prefix, the best entry is +inf or
+//    above (a NaN with the sign bit clear), or that entry is -inf or below (a
+//    NaN with the sign bit set): the set of picks may be wrong, and the token
+//    is selected again on 64-bit entries (full key, index) over its row in
+//    global memory;
+//  - otherwise, two picks share a prefix: the set is right, and the picks are
+//    sorted again on full keys.
+// Either way the picks are those of the warp kernel above, and the weights
+// are computed from the picked logits in the same order of operations. The
+// block's counts come from one bit per (expert, token) in shared memory: a
+// token's rank inside its rank block (tpb tokens, as in the warp kernel) is a
+// population count of the bits below it.
 // Restrictions: E a multiple of 32 (up to 256), k <= 8, softmax weights
-// renormalised over the picks or sigmoid weights; other cases use the warp
-// kernel.
+// renormalised over the picks or sigmoid weights, 16-byte aligned logits;
+// other cases use the warp kernel.
 constexpr int kLaneTokens = 256;                 // tokens (threads) per block
 constexpr int64_t kLaneMinTokens = 32768;        // below this, the warp kernel (more blocks, lower latency)
 constexpr int kLaneChunk = 32;                   // experts staged per step
 constexpr int kLanePitch = kLaneChunk + 4;       // floats per staged row (conflict-free 16-byte reads)
 
-// A selection entry as one 64-bit value: the order key above, the complement
-// of the expert index below, so that a larger value ranks strictly better in
-// the selection order (larger key, then the lower index). A compare-exchange
-// is then a branch-free max/min. 0 ranks below every expert (key 0 with the
-// largest index).
+// An exact selection entry as one 64-bit value: the order key above, the
+// complement of the expert index below, so that a larger value ranks strictly
+// better in the selection order (larger key, then the lower index). 0 ranks
+// below every expert (key 0 with the largest index).
 __device__ __forceinline__ uint64_t lane_entry(uint32_t key, uint32_t e) {
     return ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - e);
 }
-__device__ __forceinline__ uint32_t lane_key(uint64_t v) { return (uint32_t)(v >> 32); }
 __device__ __forceinline__ uint32_t lane_expert(uint64_t v) { return 0xFFFFFFFFu - (uint32_t)v; }
 
-__device__ __forceinline__ void lane_cx(uint64_t& a, uint64_t& b) {   // a := better, b := worse
-    const uint64_t hi = a > b ? a : b, lo = a > b ? b : a;
+// Signed order key: a larger float gives a larger int. -0 sits one below +0,
+// NaNs with the sign bit clear lie above +inf and the others below -inf.
+__device__ __forceinline__ int32_t lane_skey(float s) {
+    const int32_t b = __float_as_int(s);
+    return b ^ ((b >> 31) & 0x7FFFFFFF);
+}
+// The 32-bit entry: the key's top 32 - ib bits, then the complement of the
+// expert index in the low ib bits (ib = 7 for E <= 128, else 8).
+struct LaneFmt {
+    int ib;            // index bits
+    int32_t hi_mask;   // ~((1 << ib) - 1)
+    int32_t cmax;      // (1 << ib) - 1
+};
+__device__ __forceinline__ int32_t lane_entry32(float s, int e, const LaneFmt& f) {
+    return (lane_skey(s) & f.hi_mask) | (f.cmax - e);
+}
+__device__ __forceinline__ int lane_expert32(int32_t v, const LaneFmt& f) { return f.cmax - (v & f.cmax); }
+constexpr int32_t kLaneNone = INT32_MIN;                          // below every entry of a score
+constexpr int32_t kLaneKeyPosInf = 0x7F800000;                    // signed order keys of +inf and -inf
+constexpr int32_t kLaneKeyNegInf = (int32_t)0x807FFFFFu;
+// Neighbours (a before b in the 32-bit order) whose exact order may differ:
+// the same prefix, or the prefixes of -0 and +0.
+__device__ __forceinline__ bool lane_close(int32_t a, int32_t b, int ib) {
+    const int32_t pa = a >> ib, pb = b >> ib;
+    return pa == pb || (pa == 0 && pb == -1);
+}
+
+// Larger / smaller of two entries: one integer max or min for 32-bit entries.
+__device__ __forceinline__ int32_t lane_hi(int32_t a, int32_t b) { return max(a, b); }
+__device__ __forceinline__ int32_t lane_lo(int32_t a, int32_t b) { return min(a, b); }
+__device__ __forceinline__ uint64_t lane_hi(uint64_t a, uint64_t b) { return a > b ? a : b; }
+__device__ __forceinline__ uint64_t lane_lo(uint64_t a, uint64_t b) { return a > b ? b : a; }
+
+template <typename V>
+__device__ __forceinline__ void lane_cx(V& a, V& b) {   // a := better, b := worse
+    const V hi = lane_hi(a, b), lo = lane_lo(a, b);
     a = hi;
     b = lo;
 }
 
-__device__ __forceinline__ void lane_sort8(uint64_t (&v)[8]) {
+template <typename V>
+__device__ __forceinline__ void lane_sort8(V (&v)[8]) {
     constexpr int net[19][2] = {{0, 1}, {2, 3}, {4, 5}, {6, 7}, {0, 2}, {1, 3}, {4, 6},
                                 {5, 7}, {1, 2}, {5, 6}, {0, 4}, {1, 5}, {2, 6}, {3, 7},
                                 {2, 4}, {3, 5}, {1, 2}, {3, 4}, {5, 6}};
@@ -295,10 +346,9 @@ __device__ __forceinline__ void lane_sort8(uint64_t (&v)[8]) {
     for (int c = 0; c < 19; ++c) lane_cx(v[net[c][0]], v[net[c][1]]);
 }
 
-// top (best first) := the best 8 of top and g (both best first).
-__device__ __forceinline__ void lane_merge8(uint64_t (&t)[8], uint64_t (&g)[8]) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) t[i] = t[i] > g[7 - i] ? t[i] : g[7 - i];   // bitonic, holds the best 8
+// Sorts a bitonic 8 best first (12 pairs).
+template <typename V>
+__device__ __forceinline__ void lane_clean8(V (&t)[8]) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) lane_cx(t[i], t[i + 4]);
 #pragma unroll
@@ -308,6 +358,25 @@ __device__ __forceinline__ void lane_merge8(uint64_t (&t)[8], uint64_t (&g)[8]) 
     }
 #pragma unroll
     for (int i = 0; i < 8; i += 2) lane_cx(t[i], t[i + 1]);
+}
+
+// t (best first) := the best 8 of t and g (both best first). With DROP, drop
+// also takes the best of the 8 entries left out.
+template <bool DROP, typename V>
+__device__ __forceinline__ void lane_merge8(V (&t)[8], const V (&g)[8], V& drop) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const V x = t[i], y = g[7 - i];
+        t[i] = lane_hi(x, y);     // bitonic, holds the best 8
+        if (DROP) drop = lane_hi(drop, lane_lo(x, y));
+    }
+    lane_clean8(t);
+}
+
+// The score that is ranked: the logit, or with an expert bias sigmoid(logit) + bias.
+template <bool BIAS>
+__device__ __forceinline__ float lane_score(float l, const float* bias, int e) {
+    return BIAS ? 1.0f / (1.0f + expf(-l)) + __ldg(bias + e) : l;
 }
 
 // Tokens of [lo, hi) (block-local indices, hi <= 256) whose bit is set in m[0..7].
@@ -323,8 +392,8 @@ __device__ __forceinline__ int lane_count(const uint32_t* m, int lo, int hi) {
     return c;
 }
 
-template <int KC>
-__global__ void __launch_bounds__(kLaneTokens)
+template <int KC, bool BIAS>
+__global__ void __launch_bounds__(kLaneTokens, 3)
     router_lane_kernel(const RouterArgs a) {
     __shared__ __align__(16) float stage[kLaneTokens / 32][32][kLanePitch];   // 36 KB
     __shared__ uint32_t mask[256][kLaneTokens / 32];                          // 8 KB
@@ -336,53 +405,112 @@ __global__ void __launch_bounds__(kLaneTokens)
     if (blockIdx.x == 0 && threadIdx.x == 0) *a.ticket = 0u;
     for (int i = threadIdx.x; i < E * (kLaneTokens / 32); i += blockDim.x) (&mask[0][0])[i] = 0u;
 
-    uint64_t top[8];
+    LaneFmt fmt;
+    fmt.ib = E <= 128 ? 7 : 8;
+    fmt.cmax = (1 << fmt.ib) - 1;
+    fmt.hi_mask = ~fmt.cmax;
+    int32_t top[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) top[i] = 0u;   // below every expert
+    for (int i = 0; i < 8; ++i) top[i] = kLaneNone;
+    int32_t drop = kLaneNone;
     float(*st)[kLanePitch] = stage[warp];
     const int64_t wrow0 = t0 + warp * 32;
-    for (int c0 = 0; c0 < E; c0 += kLaneChunk) {
-        // stage rows wrow0 .. +31, experts c0 .. c0+31: lane -> row 4i + lane/8, 4 experts
+    // lane -> rows 4i + lane/8 of the warp's 32, 16-byte column lane % 8 of the chunk
+    float4 pf[8];
+    auto load_chunk = [&](int c0) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const int r = 4 * i + (lane >> 3), q = lane & 7;
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (wrow0 + r < a.T) v = __ldg(reinterpret_cast<const float4*>(a.logits + (wrow0 + r) * E + c0) + q);
-            *reinterpret_cast<float4*>(&st[r][4 * q]) = v;
+            const int r = 4 * i + (lane >> 3);
+            pf[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (wrow0 + r < a.T)
+                pf[i] = __ldg(reinterpret_cast<const float4*>(a.logits + (wrow0 + r) * E + c0) + (lane & 7));
         }
+    };
+    load_chunk(0);
+    for (int c0 = 0; c0 < E; c0 += kLaneChunk) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            *reinterpret_cast<float4*>(&st[4 * i + (lane >> 3)][4 * (lane & 7)]) = pf[i];
         __syncwarp();
+        if (c0 + kLaneChunk < E) load_chunk(c0 + kLaneChunk);   // in flight while this chunk is sorted
 #pragma unroll
         for (int g = 0; g < kLaneChunk; g += 8) {
             const float4 v0 = *reinterpret_cast<const float4*>(&st[lane][g]);
             const float4 v1 = *reinterpret_cast<const float4*>(&st[lane][g + 4]);
             const float l[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-            uint64_t gv[8];
+            int32_t gv[8];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const int e = c0 + g + q;
-                float score = l[q];
-                if (a.bias) score = 1.0f / (1.0f + expf(-l[q])) + __ldg(a.bias + e);
-                gv[q] = lane_entry(float_order_key(score), (uint32_t)e);
-            }
+            for (int q = 0; q < 8; ++q) gv[q] = lane_entry32(lane_score<BIAS>(l[q], a.bias, c0 + g + q), c0 + g + q, fmt);
             lane_sort8(gv);
-            lane_merge8(top, gv);
+            if (c0 == 0 && g == 0) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) top[i] = gv[i];
+            } else {
+                lane_merge8<KC == 8>(top, gv, drop);
+            }
         }
         __syncwarp();   // the stage is read before the next chunk overwrites it
     }
 
-    // routing weights, in the warp kernel's order of operations
+    // Where the 32-bit order may differ from the exact one. At the edge (the
+    // last pick and the entry after it share a prefix, or an infinity or NaN
+    // sits at either end) the set of picks itself may differ: the row is
+    // selected again. Otherwise the picks are right and only neighbours that
+    // share a prefix may be out of order: the picks are sorted again on full keys.
     const int k = KC;
-    uint32_t tk[8], te[8];
+    const int32_t next = KC == 8 ? drop : top[KC < 8 ? KC : 7];
+    const bool edge = top[0] >= (kLaneKeyPosInf & fmt.hi_mask) || next <= (kLaneKeyNegInf | fmt.cmax) ||
+                      lane_close(top[k - 1], next, fmt.ib);
+    bool inner = false;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        tk[j] = lane_key(top[j]);
-        te[j] = lane_expert(top[j]);
+    for (int j = 0; j + 1 < KC; ++j) inner |= lane_close(top[j], top[j + 1], fmt.ib);
+    int te[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) te[j] = lane_expert32(top[j], fmt);
+    if (edge && live) {
+        // exact selection over the row in global memory
+        uint64_t x[8], none = 0u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = 0u;
+        const float* row = a.logits + t * E;
+        for (int c = 0; c < E; c += 8) {
+            const float4 v0 = __ldg(reinterpret_cast<const float4*>(row + c));
+            const float4 v1 = __ldg(reinterpret_cast<const float4*>(row + c) + 1);
+            const float l[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            uint64_t gv[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                gv[q] = lane_entry(float_order_key(lane_score<BIAS>(l[q], a.bias, c + q)), (uint32_t)(c + q));
+            lane_sort8(gv);
+            lane_merge8<false>(x, gv, none);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) te[j] = (int)lane_expert(x[j]);
+    } else if (inner && live) {
+        // the picks on full keys (entries past k rank below every pick)
+        uint64_t x[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            x[j] = j < k ? lane_entry(float_order_key(lane_score<BIAS>(__ldg(a.logits + t * E + te[j]), a.bias, te[j])),
+                                      (uint32_t)te[j])
+                         : 0u;
+        lane_sort8(x);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (j < k) te[j] = (int)lane_expert(x[j]);
     }
+
+    // routing weights from the picked logits, in the warp kernel's order of operations
     float lsel[8], p[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         lsel[j] = 0.0f;
-        if (j < k && live) lsel[j] = a.bias ? __ldg(a.logits + t * E + te[j]) : order_key_to_float(tk[j]);
+        if (j < k && live) {
+            const float l = __ldg(a.logits + t * E + te[j]);
+            // without a bias the warp kernel works from the key: NaN comes back
+            // as the canonical NaN and -0 as +0
+            lsel[j] = BIAS ? l : order_key_to_float(float_order_key(l));
+        }
     }
     if (a.score_fn == MOE_SCORE_SOFTMAX) {
         const float m = lsel[0];   // the first pick holds the largest logit of the picks (or NaN)
@@ -404,12 +532,23 @@ __global__ void __launch_bounds__(kLaneTokens)
 #pragma unroll
         for (int j = 0; j < 8; ++j) p[j] = a.renormalize ? sg[j] / sum : sg[j];
     }
+    const bool vec = KC == 8 &&
+                     ((((uintptr_t)a.topk_idx) | ((uintptr_t)a.topk_prob) | ((uintptr_t)a.local_rank)) & 15u) == 0;
     if (live) {
+        if (vec) {
+            int4* ip = reinterpret_cast<int4*>(a.topk_idx + t * 8);
+            float4* pp = reinterpret_cast<float4*>(a.topk_prob + t * 8);
+            ip[0] = make_int4(te[0], te[1], te[2], te[3]);
+            ip[1] = make_int4(te[4], te[5], te[6], te[7]);
+            pp[0] = make_float4(p[0] * a.scaling, p[1] * a.scaling, p[2] * a.scaling, p[3] * a.scaling);
+            pp[1] = make_float4(p[4] * a.scaling, p[5] * a.scaling, p[6] * a.scaling, p[7] * a.scaling);
+        } else {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            if (j >= k) break;
-            a.topk_idx[t * k + j] = (int32_t)te[j];
-            a.topk_prob[t * k + j] = p[j] * a.scaling;
+            for (int j = 0; j < 8; ++j) {
+                if (j >= k) break;
+                a.topk_idx[t * k + j] = te[j];
+                a.topk_prob[t * k + j] = p[j] * a.scaling;
+            }
         }
         if (a.routing_map) {
             uint4* mrow = reinterpret_cast<uint4*>(a.routing_map + t * E);
@@ -431,9 +570,18 @@ __global__ void __launch_bounds__(kLaneTokens)
     const int tpb = a.tpb;
     if (live) {
         const int lo = (threadIdx.x / tpb) * tpb;
+        int rk[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            if (j < k) a.local_rank[t * k + j] = lane_count(mask[te[j]], lo, threadIdx.x);
+        for (int j = 0; j < 8; ++j) rk[j] = j < k ? lane_count(mask[te[j]], lo, threadIdx.x) : 0;
+        if (vec) {
+            int4* rp = reinterpret_cast<int4*>(a.local_rank + t * 8);
+            rp[0] = make_int4(rk[0], rk[1], rk[2], rk[3]);
+            rp[1] = make_int4(rk[4], rk[5], rk[6], rk[7]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (j < k) a.local_rank[t * k + j] = rk[j];
+        }
     }
     const int nsub = kLaneTokens / tpb;
     const int64_t sb0 = t0 / tpb;
@@ -630,6 +778,11 @@ __device__ __forceinline__ int block_inclusive_scan(int v, int* warp_tot, int& t
     return v;
 }
 
+constexpr int kScanPerThread = 8;   // values a scan thread holds per pass
+// Shared-memory slot of value i of a pass: thread i / 8's run, one padding
+// word per run, so that a warp reading its runs hits 32 different banks.
+__device__ __forceinline__ int scan_slot(int i) { return (i / kScanPerThread) * (kScanPerThread + 1) + i % kScanPerThread; }
+
 // One block per expert: exclusive scan of its per-token-block counts. The last
 // block to finish also writes offsets (exclusive scan of the expert counts).
 __global__ void __launch_bounds__(1024)
@@ -640,14 +793,38 @@ __global__ void __launch_bounds__(1024)
     int carry_off = 0;
     const int e = blockIdx.x;
     int32_t* row = block_base + (int64_t)e * nb;
+    __shared__ int s_v[(kScanPerThread + 1) * 1024];   // a run of 8 per thread, padded by one word
     int carry = 0;
-    for (int base = 0; base < nb; base += blockDim.x) {
-        const int i = base + threadIdx.x;
-        const int v = i < nb ? row[i] : 0;
+    // kScanPerThread values per thread per pass: coalesced loads into shared
+    // memory (all in flight at once), a serial scan of each thread's run, one
+    // block scan of the run totals, coalesced stores
+    const int span = kScanPerThread * (int)blockDim.x;
+    for (int base = 0; base < nb; base += span) {
+        const int n = nb - base < span ? nb - base : span;
+#pragma unroll
+        for (int j = 0; j < kScanPerThread; ++j) {
+            const int i = j * (int)blockDim.x + threadIdx.x;
+            s_v[scan_slot(i)] = i < n ? row[base + i] : 0;
+        }
+        __syncthreads();
+        int run[kScanPerThread], sum = 0;
+#pragma unroll
+        for (int j = 0; j < kScanPerThread; ++j) {
+            run[j] = sum;
+            sum += s_v[threadIdx.x * (kScanPerThread + 1) + j];
+        }
         int total;
-        const int incl = block_inclusive_scan(v, warp_tot, total);
-        if (i < nb) row[i] = carry + incl - v;
+        const int excl = carry + block_inclusive_scan(sum, warp_tot, total) - sum;
+#pragma unroll
+        for (int j = 0; j < kScanPerThread; ++j) s_v[threadIdx.x * (kScanPerThread + 1) + j] = excl + run[j];
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < kScanPerThread; ++j) {
+            const int i = j * (int)blockDim.x + threadIdx.x;
+            if (i < n) row[base + i] = s_v[scan_slot(i)];
+        }
         carry += total;
+        __syncthreads();   // s_v is read before the next pass overwrites it
     }
     if (counts == nullptr) return;
     if (threadIdx.x == 0) {
@@ -949,20 +1126,26 @@ cudaError_t launch_router_topk(const float* logits, int64_t T, int E, int k,
     // overrides the choice (the tests run both on the same inputs).
     const char* force = getenv("MOE_ROUTER");
     const bool lane_ok = E % 32 == 0 && E <= 256 && k <= 8 && kLaneTokens % a.tpb == 0 &&
-                         (opts.score_fn == MOE_SCORE_SIGMOID || opts.renormalize);
+                         (opts.score_fn == MOE_SCORE_SIGMOID || opts.renormalize) &&
+                         ((uintptr_t)logits & 15u) == 0;
     const bool use_lane = lane_ok && (force ? force[0] == 'l' : T >= kLaneMinTokens);
     if (use_lane) {
         const dim3 lgrid((unsigned)((T + kLaneTokens - 1) / kLaneTokens)), lblock(kLaneTokens);
+        const bool bias = opts.expert_bias != nullptr;
+#define MOE_LANE(KC)                                                \
+    if (bias) router_lane_kernel<KC, true><<<lgrid, lblock, 0, st>>>(a); \
+    else router_lane_kernel<KC, false><<<lgrid, lblock, 0, st>>>(a)
         switch (k) {
-            case 1: router_lane_kernel<1><<<lgrid, lblock, 0, st>>>(a); break;
-            case 2: router_lane_kernel<2><<<lgrid, lblock, 0, st>>>(a); break;
-            case 3: router_lane_kernel<3><<<lgrid, lblock, 0, st>>>(a); break;
-            case 4: router_lane_kernel<4><<<lgrid, lblock, 0, st>>>(a); break;
-            case 5: router_lane_kernel<5><<<lgrid, lblock, 0, st>>>(a); break;
-            case 6: router_lane_kernel<6><<<lgrid, lblock, 0, st>>>(a); break;
-            case 7: router_lane_kernel<7><<<lgrid, lblock, 0, st>>>(a); break;
-            default: router_lane_kernel<8><<<lgrid, lblock, 0, st>>>(a); break;
+            case 1: MOE_LANE(1); break;
+            case 2: MOE_LANE(2); break;
+            case 3: MOE_LANE(3); break;
+            case 4: MOE_LANE(4); break;
+            case 5: MOE_LANE(5); break;
+            case 6: MOE_LANE(6); break;
+            case 7: MOE_LANE(7); break;
+            default: MOE_LANE(8); break;
         }
+#undef MOE_LANE
         (void)err;
         return cudaGetLastError();
     }
@@ -1013,7 +1196,7 @@ cudaError_t launch_expert_scan(int64_t T, int E, const RouteScratch& rs, int32_t
                                int32_t* offsets, cudaStream_t st) {
     const int nb = (int)route_blocks(T);
     int threads = 32;
-    while (threads < nb && threads < 1024) threads <<= 1;
+    while (threads * kScanPerThread < nb && threads < 1024) threads <<= 1;
     expert_scan_kernel<<<E, threads, 0, st>>>(rs.block_base, nb, E, counts, offsets, rs.ticket);
     return cudaGetLastError();
 }

@@ -189,6 +189,54 @@ def test_lane_router_matches_warp_router_bit_for_bit(T, E, k, mode, monkeypatch)
         assert torch.equal(a[n].view(torch.uint8), b[n].view(torch.uint8)), n
 
 
+def _near_tie_logits(T, E, seed):
+    """Rows where a dozen experts hold floats that differ only in the low 8
+    bits of their order key (one 24-bit prefix, different values), on both
+    signs and around the 8th largest, so that the picks and the first entry
+    after them fall inside one prefix; rows of +0, -0 and denormals on top;
+    rows with +inf on top of near-equal values; rows where only the first
+    three picks share a prefix (their order, not the set, is in question)."""
+    rng = np.random.default_rng(seed)
+    base = rng.standard_normal((T, E)).astype(np.float32)
+    bits = base.view(np.uint32)
+    for t in range(T):
+        cols = rng.choice(E, 12, replace=False)
+        kind = t % 6
+        if kind == 3:      # zeros of both signs and tiny denormals above the rest
+            base[t] -= 10.0
+            base[t, cols] = np.array([0.0, -0.0, 1e-45, -1e-45, 2e-45, -3e-45] * 2, np.float32)
+            continue
+        if kind == 1:      # negative, with the rest pushed below
+            base[t] -= 10.0
+        if kind == 5:      # three picks far above the rest, inside one prefix
+            cols = cols[:3]
+        b0 = {0: np.float32(3.0), 1: np.float32(-2.5), 2: np.sort(base[t])[-8], 4: np.float32(1.75),
+              5: np.float32(6.0)}[kind]
+        low = rng.integers(0, 256, len(cols)).astype(np.uint32)
+        bits[t, cols] = (np.float32(b0).view(np.uint32) & np.uint32(0xFFFFFF00)) | low
+        if kind == 4:      # +inf above them
+            base[t, cols[0]] = np.inf
+    return torch.from_numpy(base)
+
+
+@pytest.mark.parametrize("k,E", [(8, 128), (3, 128), (7, 128), (8, 256), (5, 160)])
+@pytest.mark.parametrize("mode", ["softmax_renorm", "sigmoid"])
+def test_lane_router_near_ties_take_the_exact_pass(k, E, mode, monkeypatch):
+    """Values that the lane kernel's 32-bit entries cannot tell apart (the same
+    top 24 bits of the order key) must still be picked in the exact order:
+    the kernel detects them and selects those tokens again on full keys."""
+    score, renorm = MODES[mode]
+    logits = _near_tie_logits(1500, E, seed=5 + k + E).cuda()
+    a = _router_outputs(logits, k, score, renorm, "lane", monkeypatch)
+    b = _router_outputs(logits, k, score, renorm, "warp", monkeypatch)
+    for n in b:
+        assert torch.equal(a[n].view(torch.uint8), b[n].view(torch.uint8)), n
+    # and against the oracle's picks
+    import oracle
+    r = oracle.router_topk(logits.cpu().numpy(), k, score, renorm)
+    assert np.array_equal(a["topk_idx"].cpu().numpy(), r["topk_idx"])
+
+
 @pytest.mark.parametrize("mode", ["softmax_renorm", "sigmoid", "sigmoid_renorm"])
 def test_lane_router_degenerate_values_bias_and_scaling(mode, monkeypatch):
     score, renorm = MODES[mode]
