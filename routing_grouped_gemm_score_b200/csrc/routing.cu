@@ -379,6 +379,84 @@ __device__ __forceinline__ float lane_score(float l, const float* bias, int e) {
     return BIAS ? 1.0f / (1.0f + expf(-l)) + __ldg(bias + e) : l;
 }
 
+// The exact picks of one token, best first: 64-bit entries over its row in
+// global memory, 32 experts (eight 16-byte loads) in flight at a time. Out of
+// line, so that the main loop's registers are not spent on this rare path.
+template <bool BIAS>
+__device__ __noinline__ void lane_exact_row(const float* __restrict__ row, int E, const float* __restrict__ bias,
+                                            int* te) {
+    uint64_t x[8], none = 0u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[i] = 0u;
+    for (int c0 = 0; c0 < E; c0 += 32) {
+        float4 v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = __ldg(reinterpret_cast<const float4*>(row + c0) + i);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+            const float l[8] = {v[2 * g].x, v[2 * g].y, v[2 * g].z, v[2 * g].w,
+                                v[2 * g + 1].x, v[2 * g + 1].y, v[2 * g + 1].z, v[2 * g + 1].w};
+            uint64_t gv[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int e = c0 + 8 * g + q;
+                gv[q] = lane_entry(float_order_key(lane_score<BIAS>(l[q], bias, e)), (uint32_t)e);
+            }
+            lane_sort8(gv);
+            lane_merge8<false>(x, gv, none);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) te[j] = (int)lane_expert(x[j]);
+}
+
+// A tie at the edge of the picks: the experts whose 32-bit prefix equals pb,
+// the prefix of the last pick, compete for picks n_sure..k-1 (the picks
+// before them have larger prefixes and stay). They are found in one pass over
+// the row and ranked on 64-bit entries; te[n_sure..k) receives the best.
+template <bool BIAS>
+__device__ __noinline__ void lane_edge_picks(const float* __restrict__ row, int E, int k, int n_sure,
+                                             const float* __restrict__ bias, LaneFmt fmt, int32_t pb, int* te) {
+    uint64_t x[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[i] = 0u;
+    for (int c0 = 0; c0 < E; c0 += 32) {
+        float4 v[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] = __ldg(reinterpret_cast<const float4*>(row + c0) + i);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const float4 w = v[i / 4];
+            const float l = (i & 3) == 0 ? w.x : (i & 3) == 1 ? w.y : (i & 3) == 2 ? w.z : w.w;
+            const int e = c0 + i;
+            const float sc = lane_score<BIAS>(l, bias, e);
+            if ((lane_entry32(sc, e, fmt) >> fmt.ib) == pb) {
+                uint64_t y = lane_entry(float_order_key(sc), (uint32_t)e);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) lane_cx(x[j], y);   // insert, keeping the best 8
+            }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        if (j >= n_sure && j < k) te[j] = (int)lane_expert(x[j - n_sure]);
+}
+
+// The k picks te[0..k) sorted again on full keys (the set is right).
+template <bool BIAS>
+__device__ __noinline__ void lane_exact_picks(const float* __restrict__ row, int k, const float* __restrict__ bias,
+                                              int* te) {
+    uint64_t x[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        x[j] = j < k ? lane_entry(float_order_key(lane_score<BIAS>(__ldg(row + te[j]), bias, te[j])), (uint32_t)te[j])
+                     : 0u;   // below every pick
+    lane_sort8(x);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        if (j < k) te[j] = (int)lane_expert(x[j]);
+}
+
 // Tokens of [lo, hi) (block-local indices, hi <= 256) whose bit is set in m[0..7].
 __device__ __forceinline__ int lane_count(const uint32_t* m, int lo, int hi) {
     int c = 0;
@@ -467,37 +545,29 @@ __global__ void __launch_bounds__(kLaneTokens, 3)
     int te[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) te[j] = lane_expert32(top[j], fmt);
-    if (edge && live) {
-        // exact selection over the row in global memory
-        uint64_t x[8], none = 0u;
+    if ((edge || inner) && live) {
+        int fix[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) x[i] = 0u;
+        for (int j = 0; j < 8; ++j) fix[j] = te[j];
         const float* row = a.logits + t * E;
-        for (int c = 0; c < E; c += 8) {
-            const float4 v0 = __ldg(reinterpret_cast<const float4*>(row + c));
-            const float4 v1 = __ldg(reinterpret_cast<const float4*>(row + c) + 1);
-            const float l[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-            uint64_t gv[8];
+        const int32_t pb = top[k - 1] >> fmt.ib;
+        // an infinity or NaN at either end, or the prefixes of -0 and +0 at the
+        // edge: the whole row again on full keys
+        const bool whole = top[0] >= (kLaneKeyPosInf & fmt.hi_mask) || next <= (kLaneKeyNegInf | fmt.cmax) ||
+                           (edge && (pb == 0 || pb == -1));
+        if (whole) {
+            lane_exact_row<BIAS>(row, E, a.bias, fix);
+        } else {
+            if (edge) {
+                int n_sure = 0;
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-                gv[q] = lane_entry(float_order_key(lane_score<BIAS>(l[q], a.bias, c + q)), (uint32_t)(c + q));
-            lane_sort8(gv);
-            lane_merge8<false>(x, gv, none);
+                for (int j = 0; j < 8; ++j) n_sure += (j < k && (top[j] >> fmt.ib) != pb) ? 1 : 0;
+                lane_edge_picks<BIAS>(row, E, k, n_sure, a.bias, fmt, pb, fix);
+            }
+            lane_exact_picks<BIAS>(row, k, a.bias, fix);
         }
 #pragma unroll
-        for (int j = 0; j < 8; ++j) te[j] = (int)lane_expert(x[j]);
-    } else if (inner && live) {
-        // the picks on full keys (entries past k rank below every pick)
-        uint64_t x[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            x[j] = j < k ? lane_entry(float_order_key(lane_score<BIAS>(__ldg(a.logits + t * E + te[j]), a.bias, te[j])),
-                                      (uint32_t)te[j])
-                         : 0u;
-        lane_sort8(x);
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            if (j < k) te[j] = (int)lane_expert(x[j]);
+        for (int j = 0; j < 8; ++j) te[j] = fix[j];
     }
 
     // routing weights from the picked logits, in the warp kernel's order of operations
