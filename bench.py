@@ -442,7 +442,9 @@ def our_arm(args, world, rank, local):
 def router_sweep(m, hbm):
     """The router alone (score + top-k + weights + counts/offsets) at E=128,
     k=8 on N(0,1) logits, large T, each launch L2-cold (logits > L2 from
-    T = 2^18 on; before every launch a 256 MB read evicts them)."""
+    T = 2^18 on; before every launch a 256 MB read evicts them). A short GPU
+    spin between the flush and the start event keeps the host's launch time
+    out of the measured interval."""
     import ctypes
 
     import torch
@@ -458,6 +460,7 @@ def router_sweep(m, hbm):
         times = []
         for it in range(8):
             flush.sum()
+            torch.cuda._sleep(200000)   # the GPU is busy while the call is issued: device time only
             s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             oc = m.RouterOpts().c()
             s.record()
@@ -480,6 +483,7 @@ def router_sweep(m, hbm):
         btimes = []
         for it in range(8):
             flush.sum()
+            torch.cuda._sleep(200000)   # the GPU is busy while the call is issued: device time only
             s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             s.record()
             m.moe_router_backward(logits, res["topk_idx"], dprob, out=dl)
@@ -502,6 +506,7 @@ def router_sweep(m, hbm):
             atimes = []
             for it in range(8):
                 flush.sum()
+                torch.cuda._sleep(200000)   # the GPU is busy while the call is issued: device time only
                 s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 s.record()
                 call()
