@@ -55,6 +55,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--router-sweep", action="store_true",
                     help="also time the router alone at E=128, k=8, T = 2^16 .. 2^20")
+    ap.add_argument("--gather-compare", action="store_true",
+                    help="also time the Qwen3-30B-A3B-shaped forward (no saved state) through x_perm and "
+                         "with the gate_up GEMM gathering its rows from x")
     return ap.parse_args()
 
 
@@ -424,6 +427,8 @@ def our_arm(args, world, rank, local):
         line["e2e"] = e2e_measure(args, w, d, m, opts, ws, world)
     if args.router_sweep:
         line["router_sweep"] = router_sweep(m, hbm)
+    if args.gather_compare:
+        line["gather_compare"] = gather_compare(m)
     if not args.no_cpu_baseline and world == 1 and rank == 0:
         threads = os.cpu_count() or 1
         runner = OracleRunner(w, cpu_inputs(w, d), threads)
@@ -520,6 +525,39 @@ def router_sweep(m, hbm):
         out.append(entry)
         del logits, res, ws, dprob, dl, aws
     return out
+
+
+def gather_compare(m):
+    """The forward of the Qwen3-30B-A3B-shaped layer (T=4096, H=2048, I=768,
+    E=128, k=8), no saved state, L2-flushed before each call: the permute
+    writes x_perm and the gate_up GEMM loads it with TMA tiles, against the
+    permute computing only the rows and the GEMM gathering its A rows from x
+    (MOE_GATHER=1). The outputs are bit-identical (tested)."""
+    import torch
+    import workloads as wl
+    w = wl.WORKLOADS["qwen3_30b_a3b"]
+    d = wl.make_inputs(w, "cuda", with_dout=False)
+    opts = m.RouterOpts(w.score, w.renormalize)
+    flush = torch.ones(64 << 20, dtype=torch.float32, device="cuda")
+    res = {"workload": "qwen3_30b_a3b forward, no saved state"}
+    for name, env in (("x_perm_us", "0"), ("gather_us", "1")):
+        os.environ["MOE_GATHER"] = env
+        times = []
+        for it in range(12):
+            flush.sum()
+            torch.cuda._sleep(200000)   # the GPU is busy while the call is issued: device time only
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            m.moe_layer_forward(d["logits"], d["x"], d["w_gate_up"], d["w_down"], w.k, opts)
+            e.record()
+            torch.cuda.synchronize()
+            if it >= 2:
+                times.append(s.elapsed_time(e) * 1e3)
+        res[name] = statistics.median(times)
+    os.environ.pop("MOE_GATHER", None)
+    if m.moe_get_device_status() != 0:
+        raise RuntimeError("device status after the gather comparison")
+    return res
 
 
 def graph_measure(args, step, w, world, m):

@@ -97,8 +97,25 @@ struct Params {
     int tma_out, tma_out2;     // single-CTA kernel: out / out2 have TMA store maps
     int mb_item;               // weight gradient: M blocks per item
     const float* row_scale;    // SwiGLU forward: h[r] *= row_scale[r] (NULL: 1)
+    // group-M, single CTA: A row r is row gather_tok[r] of gather_x [gather_T][K]
+    // (-1: a zero row) instead of a TMA tile of A (NULL: TMA)
+    const bf16* gather_x;
+    const int32_t* gather_tok;
+    int64_t gather_T;
     unsigned* err;
 };
+
+// 16-byte asynchronous copy global -> shared, zero-filled past src_bytes
+// (0 or 16), cached in L2 only.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Waits until at most N of this thread's committed groups are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 template <int STAGES, int STAGE_BYTES>
 struct __align__(1024) Smem {
@@ -755,9 +772,10 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
     volatile int* abort_flag = &s.abort;
 
     build_schedule<GROUP_K>(s, p, BM1);
+    const bool gather = !GROUP_K && p.gather_tok != nullptr;
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES1; ++i) {
-            mbar_init(&s.full[i], 1);
+            mbar_init(&s.full[i], gather ? 2 : 1);   // gather: the B load's arrival and the A copies'
             mbar_init(&s.empty[i], 1);
             mbar_init(&s.ready[i], 1);
         }
@@ -781,7 +799,106 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
     const uint32_t tmem_base = s.tmem_base;
     const int total = s.total_tiles;
 
-    if (warp == 0) {
+    if (warp == 0 && gather) {
+        // ------------------------------------------------- gathering producer
+        // Lane 0 loads the B tile with TMA; all 32 lanes copy the A tile's rows
+        // from gather_x with 16-byte cp.async (eight lanes per row, four rows per
+        // instruction) into the same 128-byte-swizzled
+        // K-major layout a TMA tile has (row r at r * 128, its 16-byte chunk c
+        // at c ^ (r % 8)). A stage's copies are one commit group; its second
+        // arrival (after the copies landed and a proxy fence made them visible
+        // to the tensor cores) comes kLag stages later, so kLag + 1 stages of
+        // copies are in flight.
+        constexpr int kLag = 2;
+        int stage = 0, oldest = 0, npend = 0;
+        uint32_t phase = 0;
+        uint32_t issued[STAGES1] = {0, 0, 0, 0};
+        bool ok = true;
+        for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
+            const Tile t = decode_tile<false>(s, p, id, BM1);
+            // this lane's rows lane + 32 i: their source rows (NULL: zeros)
+            const bf16* src[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int r = lane + 32 * i;
+                int64_t tok = -1;
+                if (r < t.rows) {
+                    tok = __ldg(p.gather_tok + t.row0 + r);
+                    if (tok >= p.gather_T) {
+                        raise_error(p.err, kErrDeviceCheck);
+                        tok = -1;
+                    }
+                }
+                src[i] = tok >= 0 ? p.gather_x + tok * p.K : nullptr;
+            }
+            for (int kb = 0; kb < t.num_kb; ++kb) {
+                bool got = true;
+                if (lane == 0) got = mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag, p.err);
+                got = __shfl_sync(0xFFFFFFFFu, got ? 1 : 0, 0) != 0;
+                if (!got) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* a_s = s.stage[stage];
+                uint8_t* b_s = s.stage[stage] + kStageA1;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&s.full[stage], kStageB1);
+                    if (B_MN) {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+                            tma_load_3d(&tmB, &s.full[stage], b_s + c * kChunkBytes, b_col_1cta<EPI>(t, p, c),
+                                        kb * BK, t.g);
+                    } else {
+                        tma_load_3d(&tmB, &s.full[stage], b_s, kb * BK, t.n_blk * BN, t.g);
+                    }
+                    issued[stage] += 1;
+                }
+                // copy j: lane -> 16-byte chunk lane % 8 of row 4 j + lane / 8, so one
+                // warp instruction reads four whole 128-byte row segments; the
+                // row's source comes from the lane that looked it up
+                const uint32_t a_base = smem_u32(a_s);
+                const int k0 = kb * BK;
+                const int c = lane & 7;
+                const bool col_ok = k0 + 8 * c < p.K;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int r = 4 * j + (lane >> 3);
+                    const bf16* row_src = reinterpret_cast<const bf16*>(
+                        __shfl_sync(0xFFFFFFFFu, reinterpret_cast<uintptr_t>(src[j >> 3]), r & 31));
+                    const bool have = row_src != nullptr && col_ok;
+                    cp_async_16(a_base + r * 128 + ((c ^ (r & 7)) << 4), have ? row_src + k0 + 8 * c : p.gather_x,
+                                have ? 16 : 0);
+                }
+                cp_async_commit();
+                if (++npend > kLag) {
+                    cp_async_wait<kLag>();   // the oldest stage's copies have landed
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s.full[oldest]);
+                    if (++oldest == STAGES1) oldest = 0;
+                    --npend;
+                }
+                if (++stage == STAGES1) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        // the copies still in flight, then their arrivals; then every B load
+        // lands before the CTA may exit
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            for (; npend > 0; --npend) {
+                mbar_arrive(&s.full[oldest]);
+                if (++oldest == STAGES1) oldest = 0;
+            }
+            for (int i = 0; i < STAGES1; ++i)
+                if (issued[i]) mbar_wait(&s.full[i], (issued[i] - 1) & 1u, abort_flag, p.err);
+        }
+        __syncwarp();
+    } else if (warp == 0) {
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
             const uint64_t keep = l2_policy_evict_last();   // activation panels are read again
@@ -1540,6 +1657,38 @@ cudaError_t gemm_gate_up_swiglu(const bf16* x, int64_t rows, const int32_t* offs
     if (gu_save && !make_out_map(&tc2, gu_save, rows, 2 * (uint64_t)I)) return cudaErrorInvalidValue;
     return launch_group_m<kEpiSwiglu, true>(ta, ta64, tb, tb, p, st, &tc, gu_save ? &tc2 : nullptr);
 }
+
+cudaError_t gemm_gate_up_swiglu_gather(const bf16* x, int64_t T, const int32_t* sorted_token, int64_t rows,
+                                       const int32_t* offsets, int E, int H, int I, const bf16* w_gate_up, bf16* h,
+                                       bf16* gu_save, cudaStream_t st, unsigned* err, const float* row_scale) {
+    if (rows == 0) return cudaSuccess;
+    if (H % 8 != 0 || (reinterpret_cast<uintptr_t>(x) & 15u) != 0 || !sorted_token || !offsets)
+        return cudaErrorInvalidValue;
+    CUtensorMap ta, tb;
+    // a valid map for the kernel's signature; the A rows are gathered, not loaded through it
+    if (!make_map_2d(&ta, x, H, T, H, BK, 128)) return cudaErrorInvalidValue;
+    if (!make_map_3d(&tb, w_gate_up, 2 * (uint64_t)I, H, E, 64, BK)) return cudaErrorInvalidValue;
+    Params p = base_params(E, rows, offsets, err);
+    p.N = I;
+    p.K = H;
+    p.I = I;
+    p.n_blocks = (I + BN / 2 - 1) / (BN / 2);
+    p.out = h;
+    p.ldo = I;
+    p.out2 = gu_save;
+    p.ldo2 = 2 * (int64_t)I;
+    p.row_scale = row_scale;
+    p.gather_x = x;
+    p.gather_tok = sorted_token;
+    p.gather_T = T;
+    CUtensorMap tc, tc2;
+    if (!make_out_map(&tc, h, rows, I)) return cudaErrorInvalidValue;
+    if (gu_save && !make_out_map(&tc2, gu_save, rows, 2 * (uint64_t)I)) return cudaErrorInvalidValue;
+    return launch_1cta<kEpiSwiglu, false, true, false>(ta, tb, p, single_tile_bound(rows, E, p.n_blocks), st, &tc,
+                                                       gu_save ? &tc2 : nullptr);
+}
+
+bool grouped_gemm_pair_tiles(int64_t rows, int groups) { return use_pair_tiles(rows, groups); }
 
 cudaError_t gemm_down(const bf16* h, int64_t rows, const int32_t* offsets, int E, int H, int I,
                       const bf16* w_down, bf16* y, cudaStream_t st, unsigned* err) {

@@ -515,14 +515,26 @@ moe_status moe_layer_forward(const float* logits, const moe_bf16* x, int64_t T, 
                                err);
     if (e == cudaSuccess) e = launch_expert_scan(T, E, L.rs, L.counts, L.offsets, st);
     if (e == cudaSuccess) e = trace_mark(1, st);
+    // MOE_GATHER=1: without a requested x_perm, on single-CTA tiles, the gate_up
+    // GEMM gathers its A rows from x by token (the permute computes the rows
+    // only), so the permuted copy of x is never written or read. Off by
+    // default: on B200 the cp.async row gather feeds the tensor cores more
+    // slowly than TMA tiles of x_perm (522 against 417 us for the Qwen3-30B-A3B
+    // forward), more than the permute's copy costs.
+    const char* gather_env = getenv("MOE_GATHER");
+    const bool gather = x_perm == nullptr && !grouped_gemm_pair_tiles(A, E) && (H % 8) == 0 && gather_env &&
+                        gather_env[0] == '1';
     if (e == cudaSuccess)
-        e = launch_permute(xb, T, H, L.topk_idx, k, L.offsets, E, L.rs, L.x_perm, L.sorted_token,
-                           L.row_of, st, err);
+        e = launch_permute(xb, T, H, L.topk_idx, k, L.offsets, E, L.rs, gather ? nullptr : L.x_perm,
+                           L.sorted_token, L.row_of, st, err);
     if (e == cudaSuccess) e = trace_mark(2, st);
     if (e == cudaSuccess)
-        e = gemm_gate_up_swiglu(L.x_perm, A, L.offsets, E, H, I,
-                                reinterpret_cast<const bf16*>(w_gate_up), L.h,
-                                reinterpret_cast<bf16*>(gu), st, err);
+        e = gather ? gemm_gate_up_swiglu_gather(xb, T, L.sorted_token, A, L.offsets, E, H, I,
+                                                reinterpret_cast<const bf16*>(w_gate_up), L.h,
+                                                reinterpret_cast<bf16*>(gu), st, err)
+                   : gemm_gate_up_swiglu(L.x_perm, A, L.offsets, E, H, I,
+                                         reinterpret_cast<const bf16*>(w_gate_up), L.h,
+                                         reinterpret_cast<bf16*>(gu), st, err);
     if (e == cudaSuccess) e = trace_mark(3, st);
     if (e == cudaSuccess)
         e = gemm_down(L.h, A, L.offsets, E, H, I, reinterpret_cast<const bf16*>(w_down), L.y_perm,

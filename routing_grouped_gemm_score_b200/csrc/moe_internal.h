@@ -91,6 +91,15 @@ cudaError_t launch_combine_backward(const bf16* dout, const bf16* y_perm, const 
 cudaError_t gemm_gate_up_swiglu(const bf16* x, int64_t rows, const int32_t* offsets, int E, int H,
                                 int I, const bf16* w_gate_up, bf16* h, bf16* gu_save,
                                 cudaStream_t st, unsigned* err, const float* row_scale = nullptr);
+// gate_up + SwiGLU with A row r gathered from x: row sorted_token[r] (-1: a
+// zero row) of x [T][H], so no permuted copy of x is needed. Single-CTA tiles
+// only; H a multiple of 8 and x 16-byte aligned.
+cudaError_t gemm_gate_up_swiglu_gather(const bf16* x, int64_t T, const int32_t* sorted_token, int64_t rows,
+                                       const int32_t* offsets, int E, int H, int I, const bf16* w_gate_up, bf16* h,
+                                       bf16* gu_save, cudaStream_t st, unsigned* err,
+                                       const float* row_scale = nullptr);
+// Whether the group-M GEMMs run on CTA-pair tiles for this many rows and groups.
+bool grouped_gemm_pair_tiles(int64_t rows, int groups);
 // down: y[r] = h[r] Wd[e]
 cudaError_t gemm_down(const bf16* h, int64_t rows, const int32_t* offsets, int E, int H, int I,
                       const bf16* w_down, bf16* y, cudaStream_t st, unsigned* err);

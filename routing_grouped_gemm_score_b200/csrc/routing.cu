@@ -960,7 +960,7 @@ __global__ void __launch_bounds__(512)
             if (row >= 0) sorted_token[row] = (int32_t)t;
         }
         __syncthreads();
-        if (!active) continue;
+        if (!active || x_perm == nullptr) continue;   // no x_perm: the rows only
         for (int tt0 = 0; tt0 < ntok; tt0 += 4) {
             uint4 v[4];
 #pragma unroll
@@ -1307,9 +1307,10 @@ cudaError_t launch_permute(const bf16* x, int64_t T, int H, const int32_t* topk_
     // against 0.64; H=5120: warp 0.76. MOE_PERMUTE=warp selects the warp
     // kernel for any width.
     const char* force = getenv("MOE_PERMUTE");
-    const bool regs = H8r <= 512 && !(force && force[0] == 'w');
+    const bool regs = x_perm == nullptr || (H8r <= 512 && !(force && force[0] == 'w'));
     if (regs) {
-        const int threads = (H8r + 31) / 32 * 32;
+        // without x_perm only the rows are computed: 256 threads whatever H
+        const int threads = x_perm == nullptr ? 256 : (H8r + 31) / 32 * 32;
         int per_sm = 1;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, permute_tokens_kernel, threads, 0) != cudaSuccess ||
             per_sm < 1)
