@@ -110,11 +110,10 @@ struct Params {
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, int src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-// Waits until at most N of this thread's committed groups are still in flight.
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+// One arrival on `bar` once this thread's cp.async copies issued so far have
+// landed (the arrival is counted in the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 template <int STAGES, int STAGE_BYTES>
@@ -775,7 +774,7 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
     const bool gather = !GROUP_K && p.gather_tok != nullptr;
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES1; ++i) {
-            mbar_init(&s.full[i], gather ? 2 : 1);   // gather: the B load's arrival and the A copies'
+            mbar_init(&s.full[i], gather ? 33 : 1);   // gather: the B load's arrival and one per copying lane
             mbar_init(&s.empty[i], 1);
             mbar_init(&s.ready[i], 1);
         }
@@ -805,12 +804,10 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
         // from gather_x with 16-byte cp.async (eight lanes per row, four rows per
         // instruction) into the same 128-byte-swizzled
         // K-major layout a TMA tile has (row r at r * 128, its 16-byte chunk c
-        // at c ^ (r % 8)). A stage's copies are one commit group; its second
-        // arrival (after the copies landed and a proxy fence made them visible
-        // to the tensor cores) comes kLag stages later, so kLag + 1 stages of
-        // copies are in flight.
-        constexpr int kLag = 2;
-        int stage = 0, oldest = 0, npend = 0;
+        // at c ^ (r % 8)). Each lane's arrival on the stage's full barrier fires
+        // when its copies have landed; the MMA thread fences the async proxy
+        // after its wait, before the tensor cores read the stage.
+        int stage = 0;
         uint32_t phase = 0;
         uint32_t issued[STAGES1] = {0, 0, 0, 0};
         bool ok = true;
@@ -869,31 +866,17 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
                     cp_async_16(a_base + r * 128 + ((c ^ (r & 7)) << 4), have ? row_src + k0 + 8 * c : p.gather_x,
                                 have ? 16 : 0);
                 }
-                cp_async_commit();
-                if (++npend > kLag) {
-                    cp_async_wait<kLag>();   // the oldest stage's copies have landed
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&s.full[oldest]);
-                    if (++oldest == STAGES1) oldest = 0;
-                    --npend;
-                }
+                cp_async_arrive_noinc(&s.full[stage]);
                 if (++stage == STAGES1) {
                     stage = 0;
                     phase ^= 1u;
                 }
             }
         }
-        // the copies still in flight, then their arrivals; then every B load
-        // lands before the CTA may exit
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
+        // every copy and every B load lands before the CTA may exit
+        asm volatile("cp.async.wait_all;" ::: "memory");
         __syncwarp();
         if (lane == 0) {
-            for (; npend > 0; --npend) {
-                mbar_arrive(&s.full[oldest]);
-                if (++oldest == STAGES1) oldest = 0;
-            }
             for (int i = 0; i < STAGES1; ++i)
                 if (issued[i]) mbar_wait(&s.full[i], (issued[i] - 1) & 1u, abort_flag, p.err);
         }
@@ -975,6 +958,7 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
                     break;
                 }
                 tc_fence_after();
+                if (gather) fence_proxy_async_smem();   // the A copies were written by cp.async
                 const uint32_t a_addr = smem_u32(s.stage[stage]);
                 const uint32_t b_addr = a_addr + kStageA1;
                 int ksteps = BK / 16;

@@ -519,7 +519,7 @@ moe_status moe_layer_forward(const float* logits, const moe_bf16* x, int64_t T, 
     // GEMM gathers its A rows from x by token (the permute computes the rows
     // only), so the permuted copy of x is never written or read. Off by
     // default: on B200 the cp.async row gather feeds the tensor cores more
-    // slowly than TMA tiles of x_perm (522 against 417 us for the Qwen3-30B-A3B
+    // slowly than TMA tiles of x_perm (508 against 412 us for the Qwen3-30B-A3B
     // forward), more than the permute's copy costs.
     const char* gather_env = getenv("MOE_GATHER");
     const bool gather = x_perm == nullptr && !grouped_gemm_pair_tiles(A, E) && (H % 8) == 0 && gather_env &&
