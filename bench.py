@@ -134,9 +134,13 @@ def dist_setup(args):
 
         import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=120)
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            # a host without GPUs (the reference arm, the multi-rank tests): gloo
+            dist.init_process_group("gloo", timeout=timeout)
     return world, rank, local
 
 
@@ -151,9 +155,16 @@ def max_over_ranks(v: float, world: int) -> float:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_value(tokens_per_rank: int, world: int, steps: int, ms_max: float) -> float:
+    """Tokens per second of the whole job: every rank's tokens over the slowest
+    rank's time (weak scaling: each rank runs the same per-rank workload)."""
+    return tokens_per_rank * world * steps / (ms_max / 1e3)
 
 
 # ------------------------------------------------------------------ CPU baseline
@@ -358,8 +369,7 @@ def our_arm(args, world, rank, local):
 
     graph = None if args.no_graph else graph_measure(args, step, w, world, m)
 
-    tokens_total = w.T * world
-    value = tokens_total * K / (ms_max / 1e3)
+    value = whole_job_value(w.T, world, K, ms_max)
     peaks, peaks_src = load_peaks()
     # Under dense tensor load the 1 kW part settles at its power cap within
     # about a hundred milliseconds, so a timed region of a quarter second or
