@@ -55,6 +55,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--router-sweep", action="store_true",
                     help="also time the router alone at E=128, k=8, T = 2^16 .. 2^20")
+    ap.add_argument("--router-calls", type=int, default=None, metavar="LOGT",
+                    help="only call the router three times at T = 2^LOGT, E=128, k=8 on N(0,1) logits "
+                         "(a small program for ncu captures of the router), then exit")
     ap.add_argument("--gather-compare", action="store_true",
                     help="also time the Qwen3-30B-A3B-shaped forward (no saved state) through x_perm and "
                          "with the gate_up GEMM gathering its rows from x")
@@ -688,8 +691,28 @@ def e2e_measure(args, w, d, m, opts, ws, world):
                     + ("dx" if w.backward else "the layer output")}
 
 
+def router_calls(log_t: int) -> int:
+    """Three router calls at T = 2^log_t, E=128, k=8 on seeded N(0,1) logits:
+    the program the router's ncu captures run."""
+    import torch
+
+    import routing_grouped_gemm_score_b200 as m
+    T = 1 << log_t
+    g = torch.Generator(device="cuda").manual_seed(77)
+    logits = torch.randn((T, 128), generator=g, device="cuda")
+    for _ in range(3):
+        m.moe_router_topk(logits, 8)
+    torch.cuda.synchronize()
+    if m.moe_get_device_status() != 0:
+        raise RuntimeError("device status after the router calls")
+    print(json.dumps({"router_calls": 3, "T": T, "E": 128, "k": 8}))
+    return 0
+
+
 def main():
     args = parse()
+    if args.router_calls is not None:
+        return router_calls(args.router_calls)
     world, rank, local = dist_setup(args)
     try:
         if args.impl == "reference":
