@@ -83,6 +83,9 @@ def _load():
             lib.oracle_moe_backward.argtypes = [P, i64, i32, i32, i32, i32, P, P, P, P, P, i32,
                                                 i32, P, i64, P, P, P, P]
             lib.oracle_moe_backward.restype = i32
+            lib.oracle_moe_backward_state.argtypes = [P, i64, i32, i32, i32, i32, P, P, P, P, P, i32,
+                                                      i32, P, i64, P, P, P, P, P, P, P, P]
+            lib.oracle_moe_backward_state.restype = i32
             _lib = lib
     return _lib
 
@@ -327,8 +330,29 @@ def moe_forward_tokens(x_bits, logits, w_gu_bits, w_d_bits, k, tokens=None, scor
 
 
 def moe_backward(x_bits, topk_idx, topk_prob, w_gu_bits, w_d_bits, dout_bits, round_bf16=True,
-                 only_expert=-1, tokens=None, want=("dx", "dw_gate_up", "dw_down", "dprob")):
-    """Gradients of the layer for a given routing (see moe_oracle.c)."""
+                 only_expert=-1, tokens=None, want=("dx", "dw_gate_up", "dw_down", "dprob"),
+                 threads=None, state=None):
+    """Gradients of the layer for a given routing (see moe_oracle.c).
+
+    state: None (the forward values are recomputed), or a saved forward state
+    dict(row_of [T,k] int32, gu [rows,2I], h [rows,I], y [rows,H] as bf16 bit
+    patterns) whose rows the chain rule reads instead
+    (oracle_moe_backward_state).
+
+    With a token list and only per-token outputs wanted (dx, dprob), the list
+    is split over `threads` host threads (default: all cores); each token's
+    rows are independent of the others, so the split changes nothing."""
+    if tokens is not None and not ({"dw_gate_up", "dw_down"} & set(want)):
+        tl = np.asarray(tokens, np.int64)
+        chunks = _chunks(tl, threads or os.cpu_count() or 1)
+        if len(chunks) > 1:
+            def one(c):
+                return moe_backward(x_bits, topk_idx, topk_prob, w_gu_bits, w_d_bits, dout_bits,
+                                    round_bf16, only_expert, c, want, threads=1, state=state)
+            with ThreadPoolExecutor(max_workers=len(chunks)) as ex:
+                parts = list(ex.map(one, chunks))
+            return {key: (None if parts[0][key] is None else np.concatenate([q[key] for q in parts]))
+                    for key in ("dx", "dw_gate_up", "dw_down", "dprob")}
     lib = _load()
     x_bits = _c(x_bits, np.uint16)
     topk_idx = _c(topk_idx, np.int32)
@@ -347,10 +371,19 @@ def moe_backward(x_bits, topk_idx, topk_prob, w_gu_bits, w_d_bits, dout_bits, ro
     dwgu = np.zeros((ne, H, I2)) if "dw_gate_up" in want else None
     dwd = np.zeros((ne, I, H)) if "dw_down" in want else None
     dprob = np.zeros((nt, k)) if "dprob" in want else None
-    rc = lib.oracle_moe_backward(_p(x_bits), T, H, I, E, k, _p(topk_idx), _p(topk_prob),
-                                 _p(w_gu_bits), _p(w_d_bits), _p(dout_bits), int(round_bf16),
-                                 only_expert, _p(tl), 0 if tl is None else len(tl),
-                                 _p(dx), _p(dwgu), _p(dwd), _p(dprob))
+    st = [None] * 4
+    if state is not None:
+        st = [_c(state["row_of"], np.int32), _c(state["gu"], np.uint16), _c(state["h"], np.uint16),
+              _c(state["y"], np.uint16)]
+        rows = st[1].shape[0]
+        if st[0].shape != (T, k) or st[2].shape != (rows, I) or st[3].shape != (rows, H) or \
+                st[1].shape != (rows, 2 * I) or (st[0].size and (st[0].min() < 0 or st[0].max() >= rows)):
+            raise ValueError("moe_backward: state shapes do not match")
+    rc = lib.oracle_moe_backward_state(_p(x_bits), T, H, I, E, k, _p(topk_idx), _p(topk_prob),
+                                       _p(w_gu_bits), _p(w_d_bits), _p(dout_bits), int(round_bf16),
+                                       only_expert, _p(tl), 0 if tl is None else len(tl),
+                                       _p(st[0]), _p(st[1]), _p(st[2]), _p(st[3]),
+                                       _p(dx), _p(dwgu), _p(dwd), _p(dprob))
     if rc:
         raise ValueError(f"oracle_moe_backward failed ({rc})")
     return dict(dx=dx, dw_gate_up=dwgu, dw_down=dwd, dprob=dprob)

@@ -33,8 +33,7 @@
  * Pins. Each function is checked in tests/ against something other than
  * itself: brute-force sorts, invariants, closed forms, a special case that
  * reduces to a dense SwiGLU MLP computed by torch, fp64 central finite
- * differences and torch autograd. Which test pins which function is listed in
- * the design doc.
+ * differences and torch autograd (tests/test_oracle_*.py, one file per part).
  */
 #include <stdint.h>
 #include <stdlib.h>
@@ -591,9 +590,13 @@ int oracle_moe_forward_tokens(const uint16_t* x, const float* logits, int H, int
  * All in fp64. With round_bf16, every tensor that a bf16 pipeline stores
  * between its stages is rounded to bf16, as in the forward: the saved FC1
  * outputs g and u that the SwiGLU backward reads; the gradient dy of the
- * bf16 expert output (p * dout taken in fp32, the kernel's precision, since
- * the pages fix none for it); the gradients dg, du of the bf16 FC1 output; and the
- * gradient dxp of each bf16 permuted token row, which the unpermute then sums.
+ * bf16 expert output, which is the fp32 product p * dout rounded to bf16
+ * ([TT] MoE.forward, patch "multiply scores in FP32 datatype": the bf16 expert
+ * output is cast to fp32, multiplied by the fp32 scores and cast back to
+ * bf16, so the chain rule through that product gives the bf16 rounding of the
+ * fp32 product of the score and the bf16 upstream gradient); the gradients
+ * dg, du of the bf16 FC1 output; and the gradient dxp of each bf16 permuted
+ * token row, which the unpermute then sums.
  * The rounding functions themselves pass gradients through unchanged.
  * With round_bf16 = 0, nothing is rounded, and the result is the exact
  * derivative that the finite-difference pin checks.
@@ -604,12 +607,46 @@ int oracle_moe_forward_tokens(const uint16_t* x, const float* logits, int H, int
  * NULL. Every non-NULL output is zeroed first, so an expert that gets no
  * assignment has a zero weight gradient.
  */
+int oracle_moe_backward_state(const uint16_t* x, int64_t T, int H, int I, int E, int k,
+                              const int32_t* topk_idx, const float* topk_prob,
+                              const uint16_t* w_gate_up, const uint16_t* w_down, const uint16_t* dout,
+                              int round_bf16, int only_expert, const int64_t* token_list,
+                              int64_t n_tokens, const int32_t* row_of, const uint16_t* st_gu,
+                              const uint16_t* st_h, const uint16_t* st_y,
+                              double* dx, double* dw_gate_up, double* dw_down, double* dprob);
+
 int oracle_moe_backward(const uint16_t* x, int64_t T, int H, int I, int E, int k,
                         const int32_t* topk_idx, const float* topk_prob,
                         const uint16_t* w_gate_up, const uint16_t* w_down, const uint16_t* dout,
                         int round_bf16, int only_expert, const int64_t* token_list, int64_t n_tokens,
                         double* dx, double* dw_gate_up, double* dw_down, double* dprob)
 {
+    return oracle_moe_backward_state(x, T, H, I, E, k, topk_idx, topk_prob, w_gate_up, w_down, dout,
+                                     round_bf16, only_expert, token_list, n_tokens, NULL, NULL, NULL,
+                                     NULL, dx, dw_gate_up, dw_down, dprob);
+}
+
+/*
+ * oracle_moe_backward_state -- oracle_moe_backward on a given saved forward
+ * state. [TE] Grouped MLP: the pipeline stores the FC1 output and the
+ * activation between its stages, and the backward of each stage reads what
+ * the forward stored; the combine's backward reads the stored expert outputs.
+ * With row_of != NULL, the forward values of assignment (t, j) are read from
+ * row r = row_of[t * k + j] of the stored bf16 tensors instead of being
+ * recomputed: g = st_gu[r][0:I], u = st_gu[r][I:2I], h = st_h[r], y = st_y[r]
+ * (st_gu [rows][2I], st_h [rows][I], st_y [rows][H]). Everything after that is
+ * the chain rule of oracle_moe_backward, unchanged. Given the oracle's own
+ * rounded forward values, it returns what oracle_moe_backward returns.
+ */
+int oracle_moe_backward_state(const uint16_t* x, int64_t T, int H, int I, int E, int k,
+                              const int32_t* topk_idx, const float* topk_prob,
+                              const uint16_t* w_gate_up, const uint16_t* w_down, const uint16_t* dout,
+                              int round_bf16, int only_expert, const int64_t* token_list,
+                              int64_t n_tokens, const int32_t* row_of, const uint16_t* st_gu,
+                              const uint16_t* st_h, const uint16_t* st_y,
+                              double* dx, double* dw_gate_up, double* dw_down, double* dprob)
+{
+    if (row_of && (!st_gu || !st_h || !st_y)) return 3;
     int64_t nt = token_list ? n_tokens : T;
     if (dx) memset(dx, 0, sizeof(double) * (size_t)(nt * H));
     if (dprob) memset(dprob, 0, sizeof(double) * (size_t)(nt * k));
@@ -635,7 +672,18 @@ int oracle_moe_backward(const uint16_t* x, int64_t T, int H, int I, int E, int k
             double p = (double)topk_prob[t * k + j];
             const uint16_t* wgu = w_gate_up + (int64_t)e * H * 2 * I;
             const uint16_t* wd = w_down + (int64_t)e * I * H;
-            oracle_expert_mlp(xt, 1, H, I, wgu, wd, round_bf16, y, g, u, h);
+            if (row_of) {
+                int64_t r = row_of[t * k + j];
+                if (r < 0) return 2;
+                for (int i = 0; i < I; i++) {
+                    g[i] = bf16_to_double(st_gu[r * 2 * I + i]);
+                    u[i] = bf16_to_double(st_gu[r * 2 * I + I + i]);
+                    h[i] = bf16_to_double(st_h[r * I + i]);
+                }
+                for (int c = 0; c < H; c++) y[c] = bf16_to_double(st_y[r * H + c]);
+            } else {
+                oracle_expert_mlp(xt, 1, H, I, wgu, wd, round_bf16, y, g, u, h);
+            }
             if (dprob) {
                 double s = 0.0;
                 for (int c = 0; c < H; c++) s += bf16_to_double(dot[c]) * y[c];
@@ -648,9 +696,10 @@ int oracle_moe_backward(const uint16_t* x, int64_t T, int H, int I, int E, int k
                 }
             for (int c = 0; c < H; c++) {
                 if (round_bf16) {
-                    /* the stored dy is a bf16 rounding of p * dout; the pages fix
-                     * no precision for this product, so it is taken in the
-                     * kernel's (fp32), as a rounding decision must be */
+                    /* the stored dy is the bf16 rounding of the fp32 product
+                     * p * dout ([TT] MoE.forward multiplies the expert output by
+                     * the scores in fp32 before the bf16 cast; its backward
+                     * takes the same product in fp32) */
                     const float pf = topk_prob[t * k + j];
                     const float v = pf * (float)bf16_to_double(dot[c]);
                     dy[c] = bf16_to_double(double_to_bf16((double)v));

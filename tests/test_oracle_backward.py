@@ -191,3 +191,95 @@ def test_backward_empty_expert_and_expert_filter(oracle_lib):
     gt = oracle_lib.moe_backward(*args, tokens=toks, want=("dx", "dprob"))
     np.testing.assert_array_equal(gt["dx"], g["dx"][toks])
     np.testing.assert_array_equal(gt["dprob"], g["dprob"][toks])
+
+
+def _own_state(oracle_lib, w, d, r):
+    """The oracle's own forward state in the layout a saved state has: one
+    row per permuted assignment, [g | u], h and y as bf16 bit patterns."""
+    bits = oracle_lib.bf16_bits
+    x, wgu, wd = bits(d["x"]), bits(d["w_gate_up"]), bits(d["w_down"])
+    st, row_of = oracle_lib.dispatch(r["topk_idx"], r["offsets"], w.E)
+    xp = oracle_lib.gather_rows(x, st)
+    A = len(st)
+    gu = np.zeros((A, 2 * w.I), np.uint16)
+    h = np.zeros((A, w.I), np.uint16)
+    y = np.zeros((A, w.H), np.uint16)
+    offs = r["offsets"]
+    for e in range(w.E):
+        a, b = offs[e], offs[e + 1]
+        if b > a:
+            ye, ge, ue, he = oracle_lib.expert_mlp(xp[a:b], wgu[e], wd[e], True, True)
+            gu[a:b, :w.I] = oracle_lib.round_bf16_array(ge)
+            gu[a:b, w.I:] = oracle_lib.round_bf16_array(ue)
+            h[a:b] = oracle_lib.round_bf16_array(he)
+            y[a:b] = oracle_lib.round_bf16_array(ye)
+    return {"row_of": row_of, "gu": gu, "h": h, "y": y}
+
+
+def test_backward_from_saved_state_equals_recomputed_forward(oracle_lib):
+    """Given the oracle's own rounded forward state, the saved-state mode
+    returns exactly what the mode that recomputes the forward returns."""
+    w, d = setup(T=12, H=24, I=16, E=4, k=2, seed=7)
+    r = oracle_lib.router_topk(d["logits"].numpy(), w.k)
+    bits = oracle_lib.bf16_bits
+    args = (bits(d["x"]), r["topk_idx"], r["topk_prob"], bits(d["w_gate_up"]), bits(d["w_down"]),
+            bits(d["dout"]))
+    a = oracle_lib.moe_backward(*args)
+    b = oracle_lib.moe_backward(*args, state=_own_state(oracle_lib, w, d, r))
+    for key in ("dx", "dw_gate_up", "dw_down", "dprob"):
+        np.testing.assert_array_equal(a[key], b[key], err_msg=key)
+
+
+def test_backward_reads_the_given_state(oracle_lib):
+    """The saved state is what the chain rule reads: a change of one stored
+    row moves exactly the gradients that row feeds. dprob of the assignment
+    stored in row r is <dout_t, y_r>, so changing y_r by delta moves it by
+    <dout_t, delta> and moves nothing else; changing h_r moves only
+    dW_down of its expert, by the outer product of the change with that
+    assignment's bf16(p * dout)."""
+    w, d = setup(T=10, H=16, I=8, E=3, k=2, seed=8)
+    r = oracle_lib.router_topk(d["logits"].numpy(), w.k)
+    bits = oracle_lib.bf16_bits
+    args = (bits(d["x"]), r["topk_idx"], r["topk_prob"], bits(d["w_gate_up"]), bits(d["w_down"]),
+            bits(d["dout"]))
+    s0 = _own_state(oracle_lib, w, d, r)
+    g0 = oracle_lib.moe_backward(*args, state=s0)
+    t, j = 3, 1
+    row = s0["row_of"][t, j]
+    e = r["topk_idx"][t, j]
+    dout = oracle_lib.bits_to_float(bits(d["dout"]))
+    # y: a new stored row
+    s1 = {k_: v.copy() for k_, v in s0.items()}
+    y_new = oracle_lib.round_bf16_array(np.linspace(-2.0, 2.0, w.H))
+    s1["y"][row] = y_new
+    g1 = oracle_lib.moe_backward(*args, state=s1)
+    delta = oracle_lib.bits_to_float(y_new) - oracle_lib.bits_to_float(s0["y"][row])
+    want = g0["dprob"].copy()
+    want[t, j] += float(dout[t] @ delta)
+    np.testing.assert_allclose(g1["dprob"], want, rtol=1e-12, atol=1e-12)
+    for key in ("dx", "dw_gate_up", "dw_down"):
+        np.testing.assert_array_equal(g1[key], g0[key], err_msg=key)
+    # h: a new stored row
+    s2 = {k_: v.copy() for k_, v in s0.items()}
+    h_new = oracle_lib.round_bf16_array(np.linspace(0.5, -0.5, w.I))
+    s2["h"][row] = h_new
+    g2 = oracle_lib.moe_backward(*args, state=s2)
+    dh = oracle_lib.bits_to_float(h_new) - oracle_lib.bits_to_float(s0["h"][row])
+    dy = oracle_lib.bits_to_float(oracle_lib.round_bf16_array(
+        (np.float32(r["topk_prob"][t, j]) * dout[t].astype(np.float32)).astype(np.float64)))
+    want = g0["dw_down"].copy()
+    want[e] += np.outer(dh, dy)
+    np.testing.assert_allclose(g2["dw_down"], want, rtol=1e-12, atol=1e-12)
+    for key in ("dx", "dw_gate_up", "dprob"):
+        np.testing.assert_array_equal(g2[key], g0[key], err_msg=key)
+
+
+def test_backward_state_shapes_are_checked(oracle_lib):
+    w, d = setup(T=6, H=16, I=8, E=3, k=2, seed=9)
+    r = oracle_lib.router_topk(d["logits"].numpy(), w.k)
+    bits = oracle_lib.bf16_bits
+    s = _own_state(oracle_lib, w, d, r)
+    s["h"] = s["h"][:, :4]
+    with pytest.raises(ValueError):
+        oracle_lib.moe_backward(bits(d["x"]), r["topk_idx"], r["topk_prob"], bits(d["w_gate_up"]),
+                                bits(d["w_down"]), bits(d["dout"]), state=s)
