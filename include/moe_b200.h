@@ -208,9 +208,10 @@ moe_status moe_aux_loss_backward(const float* logits, int64_t T, int E, int k, i
  * share that one array: two calls whose kernels overlap on the GPU (for
  * example on different streams without ordering) race and may return wrong
  * results. Calls that are ordered on one stream are safe. The first call on
- * a device looks up the array's device address once; make that first call
- * before any stream capture. Arguments, outputs and errors are otherwise those
- * of moe_router_topk. */
+ * a device looks up the array's device address and keeps it; make that first
+ * call before any stream capture. If the lookup fails, the call returns
+ * MOE_ERR_CUDA, nothing is kept, and the next call looks it up again.
+ * Arguments, outputs and errors are otherwise those of moe_router_topk. */
 #define MOE_NOALLOC_MAX_TOKENS 32768
 #define MOE_NOALLOC_MAX_ASSIGNMENTS 262144
 moe_status moe_router_topk_noalloc(const float* logits, int64_t T, int E, int k,
@@ -377,6 +378,48 @@ moe_status moe_grouped_mlp_backward(const moe_bf16* dout, int64_t T, int H, int 
                                     moe_bf16* dx, moe_bf16* dw_gate_up, moe_bf16* dw_down,
                                     float* dprob, void* workspace, size_t workspace_bytes,
                                     void* stream);
+
+/* ------------------------------------------------------------ testing hooks
+ * moe_testing_set_kernels -- forces one kernel variant for every later call in
+ * this process, so that tests can run each variant on the same inputs. It is
+ * not an operation of the pages. The variants compute identical results (the
+ * tests compare them bit for bit, or against the oracle) and differ only in
+ * speed; by default (MOE_TESTING_AUTO everywhere) the library chooses by the
+ * shapes alone.
+ *  gemm_tiles    group-M GEMMs on single-CTA 128-row tiles or CTA-pair tiles;
+ *                or the forward GEMMs on swap-AB tiles (weights as the 128-row
+ *                operand, 64 token rows per tile; the backward GEMMs then take
+ *                single-CTA tiles)
+ *  router        the warp-per-token or the lane-per-token router kernel (the
+ *                lane kernel where it applies: E a multiple of 32, k <= 8,
+ *                renormalised softmax or sigmoid)
+ *  permute       the token-range (rows up to 4096 wide) or the warp-per-token
+ *                permute kernel
+ *  fold_permute  1: moe_layer_forward without a requested x_perm gathers the
+ *                gate_up GEMM's A rows from x by token id (single-CTA tiles),
+ *                so the permuted copy of x is never written; it measures
+ *                slower on B200 than TMA tiles of x_perm
+ * Returns MOE_ERR_INVALID_ARG for a value out of range. Not synchronised with
+ * calls issued from other threads. */
+#define MOE_TESTING_AUTO 0
+#define MOE_TESTING_GEMM_SINGLE 1
+#define MOE_TESTING_GEMM_PAIR 2
+#define MOE_TESTING_GEMM_SWAP 3
+#define MOE_TESTING_ROUTER_WARP 1
+#define MOE_TESTING_ROUTER_LANE 2
+#define MOE_TESTING_PERMUTE_TOKENS 1
+#define MOE_TESTING_PERMUTE_WARP 2
+moe_status moe_testing_set_kernels(int gemm_tiles, int router, int permute, int fold_permute);
+
+/* moe_testing_wait_timeout -- launches one block whose thread waits, with the
+ * same bounded wait as the GEMM kernels' pipeline barriers but a limit of
+ * limit_ns nanoseconds (1 .. 1e9), on a shared-memory barrier that nothing
+ * arrives on. The wait runs out, the kernel records MOE_ERR_TIMEOUT in the
+ * device error word and returns, so the next moe_get_device_status returns
+ * MOE_ERR_TIMEOUT (and clears it) and the context stays usable. It tests
+ * failure detection without a GPU fault; it is not an operation of the pages.
+ * Returns MOE_ERR_INVALID_ARG for a limit out of range. */
+moe_status moe_testing_wait_timeout(int64_t limit_ns, void* stream);
 
 #ifdef __cplusplus
 }

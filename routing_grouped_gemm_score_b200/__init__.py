@@ -36,6 +36,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "_build", "libmoe_b200.so")
 
 MOE_OK = 0
+MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA = 1, 2, 3
+MOE_ERR_WORKSPACE, MOE_ERR_DEVICE_CHECK, MOE_ERR_TIMEOUT = 4, 5, 6
 _STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_CUDA",
                  4: "MOE_ERR_WORKSPACE", 5: "MOE_ERR_DEVICE_CHECK", 6: "MOE_ERR_TIMEOUT"}
 
@@ -99,6 +101,8 @@ ABI_FUNCTIONS = {
     "moe_grouped_mlp_backward_workspace_size": (SZ, [I64, I32, I32, I32, I32]),
     "moe_grouped_mlp_backward": (I32, [P, I64, I32, I32, I32, I32, P, P, P, P, P, P, P, P, P, P, P,
                                        P, P, P, SZ, P]),
+    "moe_testing_set_kernels": (I32, [I32, I32, I32, I32]),
+    "moe_testing_wait_timeout": (I32, [I64, P]),
 }
 
 _lib = None
@@ -174,6 +178,43 @@ def moe_trace_set(events) -> None:
         return
     arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
     _check(lib().moe_trace_set(arr, len(events)), "moe_trace_set")
+
+
+# kernel variants for moe_testing_set_kernels (include/moe_b200.h, testing hooks)
+TESTING_AUTO = 0
+GEMM_SINGLE, GEMM_PAIR, GEMM_SWAP = 1, 2, 3
+ROUTER_WARP, ROUTER_LANE = 1, 2
+PERMUTE_TOKENS, PERMUTE_WARP = 1, 2
+
+
+def moe_testing_set_kernels(gemm_tiles: int = 0, router: int = 0, permute: int = 0,
+                            fold_permute: int = 0) -> None:
+    """Force kernel variants for later calls in this process (tests compare
+    the variants on the same inputs); all zero restores the library's choice."""
+    _check(lib().moe_testing_set_kernels(int(gemm_tiles), int(router), int(permute), int(fold_permute)),
+           "moe_testing_set_kernels")
+
+
+def moe_testing_wait_timeout(limit_ns: int) -> None:
+    """Launch the bounded wait that runs out after limit_ns (1 .. 1e9) on the
+    current stream; the next moe_get_device_status returns MOE_ERR_TIMEOUT."""
+    _check(lib().moe_testing_wait_timeout(int(limit_ns), _stream()), "moe_testing_wait_timeout")
+
+
+class forced_kernels:
+    """Context manager around moe_testing_set_kernels that restores the
+    library's own choice on exit."""
+
+    def __init__(self, **kw):
+        self.kw = kw
+
+    def __enter__(self):
+        moe_testing_set_kernels(**self.kw)
+        return self
+
+    def __exit__(self, *exc):
+        moe_testing_set_kernels()
+        return False
 
 
 def moe_router_topk(logits: torch.Tensor, k: int, opts: Optional[RouterOpts] = None,
@@ -381,7 +422,8 @@ def moe_grouped_mlp_scaled(x_perm: torch.Tensor, offsets: torch.Tensor, w_gate_u
 
 def moe_unpermute_combine(y_perm: torch.Tensor, row_of: torch.Tensor,
                           topk_prob: Optional[torch.Tensor] = None,
-                          shared_out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                          shared_out: Optional[torch.Tensor] = None,
+                          out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Token combine: out[t] = shared[t] + sum_j p[t,j] y_perm[row_of[t,j]]."""
     _need(y_perm, torch.bfloat16, "y_perm")
     _need(row_of, torch.int32, "row_of")
@@ -391,7 +433,12 @@ def moe_unpermute_combine(y_perm: torch.Tensor, row_of: torch.Tensor,
         _need(shared_out, torch.bfloat16, "shared_out")
     T, k = row_of.shape
     A, H = y_perm.shape
-    out = torch.empty((T, H), dtype=torch.bfloat16, device=y_perm.device)
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=y_perm.device)
+    else:
+        _need(out, torch.bfloat16, "out")
+        if tuple(out.shape) != (T, H):
+            raise ValueError(f"out: expected shape {(T, H)}, got {tuple(out.shape)}")
     _check(lib().moe_unpermute_combine_rows(_ptr(y_perm), A, _ptr(row_of), _ptr(topk_prob), T, k, H,
                                             _ptr(shared_out), _ptr(out), _stream()),
            "moe_unpermute_combine")

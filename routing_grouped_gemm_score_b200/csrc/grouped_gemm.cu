@@ -8,10 +8,11 @@
 // reads the intermediate from memory. The SwiGLU is that of te_mixtral.py
 // (_expert_ffn) and torchtitan GroupedExperts: silu(x Wg) * (x Wu).
 //
-// Two kernels share the schedule and the epilogues. The forward and dgrad
-// GEMMs run on pair tiles when the average expert block is large (>= 1024 rows,
-// or a single dense group), else on single-CTA 128-row tiles, which round
-// ragged blocks up less (use_pair_tiles).
+// Three kernels share the schedule. The forward and dgrad GEMMs run on pair
+// tiles when the average expert block is large (>= 512 rows, or a single dense
+// group), else on single-CTA 128-row tiles, which round ragged blocks up less
+// (use_pair_tiles); the forward GEMMs of small batches (<= 16 rows per expert
+// on average) run on swap-AB tiles (gemm_swap_kernel, use_swap_tiles).
 //
 // gemm_pair_kernel (group-M: forward and dgrad). Clusters of two CTAs on two
 // SMs compute 256 x 256 output tiles with tcgen05.mma.cta_group::2 (M=256,
@@ -95,7 +96,6 @@ struct Params {
     int64_t ld_aux;
     int I;                     // SwiGLU: offset of the up half in [g | u]
     int tma_out, tma_out2;     // single-CTA kernel: out / out2 have TMA store maps
-    int mb_item;               // weight gradient: M blocks per item
     const float* row_scale;    // SwiGLU forward: h[r] *= row_scale[r] (NULL: 1)
     // group-M, single CTA: A row r is row gather_tok[r] of gather_x [gather_T][K]
     // (-1: a zero row) instead of a TMA tile of A (NULL: TMA)
@@ -1077,347 +1077,242 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
     }
 }
 
-// ------------------------------------------------- weight gradient, B resident
-// gemm_wgrad_kernel: dW[e] = X_e^T D_e with the B panel of an expert (its K_e
-// rows of D, 256 columns) kept in shared memory while several 128-row M
-// blocks run against it, so D is read once per item instead of once per tile.
-// An item is (expert e, N block, a run of up to mb_item M blocks). Experts with
-// more than 320 rows (kWgPanel slices) stream B with each K slice instead (the panel slots
-// double as the B half of the A ring). Roles: warp 0 TMA (one thread), warp 1
-// MMA (one thread, owns TMEM), warps 2-9 epilogue (TMA stores of 32 x 32
-// blocks), warp 10 fixup: zeroes the rows of a ragged last slice that belong
-// to the next expert, in both operands, so no other expert's data reaches
-// this expert's gradient, then passes the stage on. Every wait is bounded.
-constexpr int kWgStagesA = 3;                  // A ring: 128 M x 64 K per stage
-constexpr int kWgPanel = 5;                    // B panel: 5 K slices of 64 rows x 256 N (320 rows)
-constexpr int kWgThreads = kThreadsK;          // 352
+// ===================================================================== swap-AB
+// gemm_swap_kernel: the forward GEMMs for expert blocks of a few rows (small
+// batches). The roles of the operands are swapped: the weights are the
+// 128-row A operand, read MN-major straight from their [K][N] layout (128
+// output columns per tile), and the expert's token rows are the B operand
+// (N = 64 rows per tile, K-major). D = W^T X^T sits in TMEM with one output
+// column per lane and one token row per TMEM column. A tile is (expert,
+// 128-column block, 64-row block); a block of up to 64 rows therefore reads
+// each weight byte once, and a one-token expert costs no padded MMA rows.
+// Tiles of one expert run in column-block order, its row blocks side by side.
+//
+// SwiGLU forward: a tile's 128 columns are 64 gate columns and the matching
+// 64 up columns, so lanes 0..63 hold g and lanes 64..127 hold u of the same
+// h columns. The epilogue warps of the upper lane quarters pass u to those of
+// the lower quarters through shared memory (an mbarrier, bounded wait), which
+// compute h = silu(g) u (times the row scale) and store h (and [g | u]).
+// Store epilogue (down): each lane writes its output column of every valid row.
+// Warp roles as in gemm_1cta_kernel: warp 0 TMA producer, warp 1 TMEM owner
+// and MMA issuer, warps 2-9 epilogue (two per lane quarter, each on 32 of
+// the 64 token columns). Every wait is bounded.
+constexpr int BNS = 64, STAGESS = 6;
+constexpr int kStageAS = 128 * BK * 2;           // 128 weight columns x 64 K: two 64-column chunks
+constexpr int kStageBS = BNS * BK * 2;           // 64 token rows x 64 K
+constexpr int kStageS = kStageAS + kStageBS;     // 24 KB
+constexpr int kTmemColsS = 128;                  // two 128-lane x 64-column accumulators
 
-struct __align__(1024) SmemW {
-    uint8_t a[kWgStagesA][kStageA1];           // 48 KB
-    uint8_t b[kWgPanel][kStageB1];             // 160 KB
-    uint8_t epi[kEpiWarps][2048];              // 16 KB: 32 x 32 bf16 per epilogue warp
-    uint64_t a_full[kWgStagesA], a_ready[kWgStagesA], a_empty[kWgStagesA];
-    uint64_t b_full, b_ready, b_empty;
-    uint64_t acc_full[2], acc_empty[2];
+struct __align__(1024) SmemS {
+    uint8_t stage[STAGESS][kStageS];
+    float ubuf[2][64][BNS + 1];   // SwiGLU: the up values of a tile's 64 columns, per accumulator
+    uint64_t full[STAGESS];
+    uint64_t empty[STAGESS];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t xchg[2];             // SwiGLU: the up values of the accumulator's tile are in ubuf
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
+    int total_tiles;
+    int tile_start[kMaxGroups + 1];
     int off[kMaxGroups + 1];
 };
-constexpr size_t kSmemWBytes = sizeof(SmemW) + 1024;
-static_assert(kSmemWBytes <= 227 * 1024, "weight-gradient shared memory");
-static_assert(offsetof(SmemW, epi) % 512 == 0, "64-byte-swizzled staging blocks start on 512-byte boundaries");
+static_assert(kStageS % 1024 == 0 && kStageAS % 1024 == 0, "swizzled stages stay 1024-byte aligned");
+constexpr size_t kSmemSBytes = sizeof(SmemS) + 1024;
 
-struct WgItem {
-    int g, n_blk, m_begin, m_end;
-    int row0, rows, nkb;
-    bool resident;
-};
-
-__device__ __forceinline__ WgItem wg_item(const SmemW& s, const Params& p, int id) {
-    const int m_groups = (p.m_blocks + p.mb_item - 1) / p.mb_item;
-    const int per = p.n_blocks * m_groups;
-    WgItem it;
-    it.g = id / per;
-    const int rem = id - it.g * per;
-    it.n_blk = rem / m_groups;
-    const int mg = rem - it.n_blk * m_groups;
-    it.m_begin = mg * p.mb_item;
-    it.m_end = min(p.m_blocks, it.m_begin + p.mb_item);
-    it.row0 = s.off[it.g];
-    it.rows = max(s.off[it.g + 1] - s.off[it.g], 0);
-    it.nkb = (it.rows + BK - 1) / BK;
-    it.resident = it.nkb > 0 && it.nkb <= kWgPanel;
-    return it;
+// First weight column of chunk c (0, 1) of the tile's 128 columns.
+template <int EPI>
+__device__ __forceinline__ int w_col_swap(const Tile& t, const Params& p, int c) {
+    if (EPI == kEpiSwiglu) return (c == 0 ? 0 : p.I) + t.n_blk * 64;
+    return t.n_blk * 128 + 64 * c;
 }
 
-// Zeroes rows [valid, round_up(valid, 16)) of `chunks` 8 KB MN-major chunks
-// (128 bytes per K row) starting at `base`; warp-collective, then publishes the
-// zeros to the async proxy.
-__device__ __forceinline__ void wg_zero_tail(uint8_t* base, int chunks, int valid, int lane) {
-    const int nrows = ((valid + 15) / 16) * 16 - valid;
-    if (nrows == 0) return;
-    const int q = lane & 7;
-    for (int chunk = 0; chunk < chunks; ++chunk)
-        for (int rr = valid + (lane >> 3); rr < valid + nrows; rr += 4)
-            *(reinterpret_cast<uint4*>(base + chunk * kChunkBytes + rr * 128) + q) = make_uint4(0, 0, 0, 0);
-    fence_proxy_async_smem();
-}
-
-__device__ void wg_producer(SmemW& s, const Params& p, const CUtensorMap* tmA, const CUtensorMap* tmB,
-                            int total, volatile int* abort) {
-    const uint64_t keep = l2_policy_evict_last();   // X panels are read again for each N block
-    int stage = 0;
-    uint32_t phase = 0;
-    int a_issued[kWgStagesA] = {0, 0, 0};
-    int panel_items = 0, b_issued = 0;
-    bool ok = true;
-    for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
-        const WgItem it = wg_item(s, p, id);
-        if (it.nkb == 0) continue;
-        // the previous item's MMAs have finished reading the panel slots
-        if (panel_items > 0 && !mbar_wait(&s.b_empty, (uint32_t)(panel_items - 1) & 1u, abort, p.err)) break;
-        ++panel_items;
-        const int n0 = it.n_blk * BN;
-        if (it.resident) {
-            mbar_arrive_expect_tx(&s.b_full, (uint32_t)(it.nkb * kStageB1));
-            for (int kb = 0; kb < it.nkb; ++kb)
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    tma_load_2d(tmB, &s.b_full, s.b[kb] + c * kChunkBytes, n0 + 64 * c, it.row0 + kb * BK);
-            ++b_issued;
-        }
-        for (int m = it.m_begin; m < it.m_end && ok; ++m) {
-            for (int kb = 0; kb < it.nkb; ++kb) {
-                if (!mbar_wait(&s.a_empty[stage], phase ^ 1u, abort, p.err)) {
-                    ok = false;
-                    break;
-                }
-                uint64_t* bar = &s.a_full[stage];
-                mbar_arrive_expect_tx(bar, (uint32_t)(kStageA1 + (it.resident ? 0 : kStageB1)));
-                const int krow = it.row0 + kb * BK;
-                tma_load_2d_hint(tmA, bar, s.a[stage], m * BM1, krow, keep);
-                tma_load_2d_hint(tmA, bar, s.a[stage] + kChunkBytes, m * BM1 + 64, krow, keep);
-                if (!it.resident)
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        tma_load_2d(tmB, bar, s.b[stage] + c * kChunkBytes, n0 + 64 * c, krow);
-                ++a_issued[stage];
-                if (++stage == kWgStagesA) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
-        }
-    }
-    // let every load still in flight land before the CTA may exit
-    for (int i = 0; i < kWgStagesA; ++i)
-        if (a_issued[i]) mbar_wait_bounded(&s.a_full[i], (uint32_t)(a_issued[i] - 1) & 1u, p.err);
-    if (b_issued) mbar_wait_bounded(&s.b_full, (uint32_t)(b_issued - 1) & 1u, p.err);
-}
-
-__device__ void wg_fixup(SmemW& s, const Params& p, int total, volatile int* abort, int lane) {
-    int stage = 0;
-    uint32_t phase = 0;
-    int res_items = 0;
-    for (int id = blockIdx.x; id < total; id += gridDim.x) {
-        const WgItem it = wg_item(s, p, id);
-        if (it.nkb == 0) continue;
-        const int valid_last = it.rows - (it.nkb - 1) * BK;   // rows of the expert in its last slice
-        if (it.resident) {
-            bool got = true;
-            if (lane == 0) got = mbar_wait(&s.b_full, (uint32_t)res_items & 1u, abort, p.err);
-            got = __shfl_sync(0xFFFFFFFFu, got ? 1 : 0, 0) != 0;
-            __syncwarp();
-            if (!got) return;
-            ++res_items;
-            if (valid_last < BK) wg_zero_tail(s.b[it.nkb - 1], 4, valid_last, lane);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s.b_ready);
-        }
-        for (int m = it.m_begin; m < it.m_end; ++m) {
-            for (int kb = 0; kb < it.nkb; ++kb) {
-                bool got = true;
-                if (lane == 0) got = mbar_wait(&s.a_full[stage], phase, abort, p.err);
-                got = __shfl_sync(0xFFFFFFFFu, got ? 1 : 0, 0) != 0;
-                __syncwarp();
-                if (!got) return;
-                if (kb == it.nkb - 1 && valid_last < BK) {
-                    wg_zero_tail(s.a[stage], 2, valid_last, lane);
-                    if (!it.resident) wg_zero_tail(s.b[stage], 4, valid_last, lane);
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s.a_ready[stage]);
-                if (++stage == kWgStagesA) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
-        }
-    }
-}
-
-__device__ void wg_mma(SmemW& s, const Params& p, int total, volatile int* abort, uint32_t tmem_base, int lane) {
-    constexpr uint32_t idesc = instr_desc<BM1, BN, true, true>();
-    int stage = 0;
-    uint32_t phase = 0;
-    int local_tile = 0, res_items = 0;
-    bool ok = true, any_mma = false;
-    for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
-        const WgItem it = wg_item(s, p, id);
-        if (it.resident) {
-            if (!mbar_wait(&s.b_ready, (uint32_t)res_items & 1u, abort, p.err)) break;
-            ++res_items;
-            tc_fence_after();
-        }
-        for (int m = it.m_begin; m < it.m_end && ok; ++m, ++local_tile) {
-            const int buf = local_tile & 1;
-            const uint32_t use = (uint32_t)(local_tile >> 1);
-            if (!mbar_wait(&s.acc_empty[buf], (use & 1u) ^ 1u, abort, p.err)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
-            for (int kb = 0; kb < it.nkb; ++kb) {
-                if (!mbar_wait(&s.a_ready[stage], phase, abort, p.err)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const int valid = it.rows - kb * BK;
-                const int ksteps = valid < BK ? (valid + 15) / 16 : BK / 16;
-                if (lane == 0) {
-                    const uint32_t a_addr = smem_u32(s.a[stage]);
-                    const uint32_t b_addr = smem_u32(it.resident ? s.b[kb] : s.b[stage]);
-#pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        if (kk >= ksteps) break;
-                        umma_bf16(d_tmem, smem_desc(a_addr + kk * 2048, kChunkBytes, 1024),
-                                  smem_desc(b_addr + kk * 2048, kChunkBytes, 1024), idesc,
-                                  (kb | kk) != 0 ? 1u : 0u);
-                    }
-                    umma_commit(&s.a_empty[stage]);
-                    any_mma = true;
-                }
-                __syncwarp();
-                if (++stage == kWgStagesA) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
-            if (!ok) break;
-            // an expert with no rows: the epilogue writes zeros, nothing to wait for
-            if (lane == 0) {
-                if (it.nkb > 0) umma_commit(&s.acc_full[buf]);
-                else mbar_arrive(&s.acc_full[buf]);
-            }
-            __syncwarp();
-        }
-        if (ok && it.nkb > 0) {
-            if (lane == 0) umma_commit(&s.b_empty);   // the panel slots are free once these MMAs end
-            __syncwarp();
-        }
-    }
-    if (lane == 0 && any_mma) {
-        umma_commit(&s.drain);
-        mbar_wait(&s.drain, 0, abort, p.err);
-    }
-    __syncwarp();
-}
-
-__device__ void wg_epilogue(SmemW& s, const Params& p, int total, volatile int* abort, uint32_t tmem_base,
-                            const CUtensorMap* tmC, int warp, int lane) {
-    const int quarter = warp & 3;               // TMEM lanes 32*quarter .. +31
-    const int col_half = (warp - 2) / 4;
-    const int warp_r0 = quarter * 32;
-    uint8_t* buf8 = s.epi[warp - 2];
-    int local_tile = 0;
-    for (int id = blockIdx.x; id < total; id += gridDim.x) {
-        const WgItem it = wg_item(s, p, id);
-        bool ok = true;
-        for (int m = it.m_begin; m < it.m_end; ++m, ++local_tile) {
-            const int buf = local_tile & 1;
-            const uint32_t use = (uint32_t)(local_tile >> 1);
-            if (!mbar_wait(&s.acc_full[buf], use & 1u, abort, p.err)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const uint32_t t_row = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-            const int n0 = it.n_blk * BN;
-            const int m0 = m * BM1 + warp_r0;
-#pragma unroll 1
-            for (int c0 = 128 * col_half; c0 < 128 * col_half + 128; c0 += 32) {
-                float v[32];
-                if (it.nkb > 0) {
-                    tmem_load_32(t_row + c0, v);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = 0.0f;
-                }
-                if (n0 + c0 >= p.N || m0 >= p.M) continue;
-                if (lane == 0) bulk_wait_group_read0();   // the previous block has left the buffer
-                __syncwarp();
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    *reinterpret_cast<uint4*>(buf8 + stage64_off(lane, q)) = make_uint4(
-                        pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                        pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_3d(tmC, buf8, n0 + c0, m0, it.g);
-                    bulk_commit_group();
-                }
-                __syncwarp();
-            }
-            tc_fence_before();
-            mbar_arrive(&s.acc_empty[buf]);
-        }
-        if (!ok) break;
-    }
-    if (lane == 0) bulk_wait_group0();   // this warp's TMA stores have completed
-    __syncwarp();
-}
-
-__global__ void __launch_bounds__(kWgThreads, 1)
-    gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                      const __grid_constant__ CUtensorMap tmC, const Params p) {
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_swap_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                     const Params p) {
+    static_assert(EPI == kEpiSwiglu || EPI == kEpiStore, "forward GEMMs only");
     extern __shared__ uint8_t smem_raw[];
-    SmemW& s = *reinterpret_cast<SmemW*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    SmemS& s = *reinterpret_cast<SmemS*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                         ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int* abort_flag = &s.abort;
-    for (int g = threadIdx.x; g <= p.groups; g += blockDim.x) {
-        const int v = p.offsets ? __ldg(p.offsets + g) : (g == 0 ? 0 : p.rows);
-        s.off[g] = min(max(v, 0), p.rows);
-    }
+
+    build_schedule<false>(s, p, BNS);
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kWgStagesA; ++i) {
-            mbar_init(&s.a_full[i], 1);
-            mbar_init(&s.a_ready[i], 1);
-            mbar_init(&s.a_empty[i], 1);
+        for (int i = 0; i < STAGESS; ++i) {
+            mbar_init(&s.full[i], 1);
+            mbar_init(&s.empty[i], 1);
         }
-        mbar_init(&s.b_full, 1);
-        mbar_init(&s.b_ready, 1);
-        mbar_init(&s.b_empty, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&s.acc_full[i], 1);
-            mbar_init(&s.acc_empty[i], 32 * kEpiWarps);
+            mbar_init(&s.acc_empty[i], kEpiWarps);   // one arrival per epilogue warp
+            mbar_init(&s.xchg[i], kEpiWarps / 2);    // one per upper-quarter warp
         }
         mbar_init(&s.drain, 1);
         s.abort = 0;
         fence_mbar_init();
-        prefetch_tensormap(&tmA);
-        prefetch_tensormap(&tmB);
+        prefetch_tensormap(&tmX);
+        prefetch_tensormap(&tmW);
     }
     if (warp == 1) {
-        tmem_alloc(&s.tmem_base, kTmemCols);
+        tmem_alloc(&s.tmem_base, kTmemColsS);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = s.tmem_base;
-    const int m_groups = (p.m_blocks + p.mb_item - 1) / p.mb_item;
-    const int total = p.groups * p.n_blocks * m_groups;
+    const int total = s.total_tiles;
 
     if (warp == 0) {
-        if (lane == 0) wg_producer(s, p, &tmA, &tmB, total, abort_flag);
-        __syncwarp();
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued[STAGESS] = {0, 0, 0, 0, 0, 0};
+            bool ok = true;
+            for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
+                const Tile t = decode_tile<false>(s, p, id, BNS);
+                for (int kb = 0; kb < t.num_kb; ++kb) {
+                    if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* a_s = s.stage[stage];
+                    uint8_t* b_s = s.stage[stage] + kStageAS;
+                    uint64_t* bar = &s.full[stage];
+                    mbar_arrive_expect_tx(bar, kStageS);
+#pragma unroll
+                    for (int c = 0; c < 2; ++c)
+                        tma_load_3d(&tmW, bar, a_s + c * kChunkBytes, w_col_swap<EPI>(t, p, c), kb * BK, t.g);
+                    tma_load_2d(&tmX, bar, b_s, kb * BK, t.row0);
+                    issued[stage] += 1;
+                    if (++stage == STAGESS) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // let every load still in flight land before the CTA may exit
+            for (int i = 0; i < STAGESS; ++i)
+                if (issued[i]) mbar_wait(&s.full[i], (issued[i] - 1) & 1u, abort_flag, p.err);
+        }
     } else if (warp == 1) {
-        wg_mma(s, p, total, abort_flag, tmem_base, lane);
-    } else if (warp < 2 + kEpiWarps) {
-        wg_epilogue(s, p, total, abort_flag, tmem_base, &tmC, warp, lane);
+        // ------------------------------------------------------ MMA issuer
+        constexpr uint32_t idesc = instr_desc<128, BNS, true, false>();
+        int stage = 0;
+        uint32_t phase = 0;
+        int local_tile = 0;
+        bool ok = true;
+        bool any_mma = false;
+        for (int id = blockIdx.x; id < total && ok; id += gridDim.x, ++local_tile) {
+            const Tile t = decode_tile<false>(s, p, id, BNS);
+            const int buf = local_tile & 1;
+            const uint32_t use = (uint32_t)(local_tile >> 1);
+            if (!mbar_wait(&s.acc_empty[buf], (use & 1u) ^ 1u, abort_flag, p.err)) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BNS);
+            for (int kb = 0; kb < t.num_kb; ++kb) {
+                if (!mbar_wait(&s.full[stage], phase, abort_flag, p.err)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a_addr = smem_u32(s.stage[stage]);
+                const uint32_t b_addr = a_addr + kStageAS;
+                if (lane == 0) {
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t adesc = smem_desc(a_addr + kk * 2048, kChunkBytes, 1024);
+                        const uint64_t bdesc = smem_desc(b_addr + kk * 32, 16, 1024);
+                        umma_bf16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    umma_commit(&s.empty[stage]);
+                    any_mma = true;
+                }
+                __syncwarp();
+                if (++stage == STAGESS) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+            if (lane == 0) umma_commit(&s.acc_full[buf]);
+            __syncwarp();
+        }
+        if (lane == 0 && any_mma) {
+            umma_commit(&s.drain);
+            mbar_wait(&s.drain, 0, abort_flag, p.err);
+        }
+        __syncwarp();
     } else {
-        wg_fixup(s, p, total, abort_flag, lane);
+        // ------------------------------------------------------ epilogue
+        const int quarter = warp & 3;               // TMEM lanes 32*quarter .. +31
+        const int half = (warp - 2) / 4;            // token columns 32*half .. +31
+        int local_tile = 0;
+        for (int id = blockIdx.x; id < total; id += gridDim.x, ++local_tile) {
+            const Tile t = decode_tile<false>(s, p, id, BNS);
+            const int buf = local_tile & 1;
+            const uint32_t use = (uint32_t)(local_tile >> 1);
+            if (!mbar_wait(&s.acc_full[buf], use & 1u, abort_flag, p.err)) break;
+            tc_fence_after();
+            float v[32];
+            tmem_load_32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BNS + 32 * half), v);
+            const int j0 = 32 * half;                        // first token column of this warp
+            const int nvalid = min(max(t.rows - j0, 0), 32);
+            bool ok = true;
+            if (EPI == kEpiSwiglu) {
+                if (quarter >= 2) {
+                    // up values of columns 32 (quarter - 2) + lane
+                    float* row = s.ubuf[buf][32 * (quarter - 2) + lane] + j0;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) row[i] = v[i];
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&s.xchg[buf]);
+                } else {
+                    ok = mbar_wait(&s.xchg[buf], use & 1u, abort_flag, p.err);
+                    if (ok) {
+                        const int hc = t.n_blk * 64 + 32 * quarter + lane;   // column of h
+                        const float* urow = s.ubuf[buf][32 * quarter + lane] + j0;
+                        const int64_t r0 = (int64_t)t.row0 + j0;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            if (i >= nvalid) break;
+                            const float g = v[i], u = urow[i];
+                            const float rs = p.row_scale ? __ldg(p.row_scale + r0 + i) : 1.0f;
+                            if (p.out2) {
+                                p.out2[(r0 + i) * p.ldo2 + hc] = __float2bfloat16_rn(g);
+                                p.out2[(r0 + i) * p.ldo2 + p.I + hc] = __float2bfloat16_rn(u);
+                            }
+                            p.out[(r0 + i) * p.ldo + hc] = __float2bfloat16_rn(silu_f(g) * u * rs);
+                        }
+                    }
+                }
+            } else {
+                const int col = t.n_blk * 128 + 32 * quarter + lane;
+                const int64_t r0 = (int64_t)t.row0 + j0;
+                if (col < p.N) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        if (i >= nvalid) break;
+                        p.out[(r0 + i) * p.ldo + col] = __float2bfloat16_rn(v[i]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.acc_empty[buf]);
+            if (!ok) break;
+        }
     }
 
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kTmemCols);
+        tmem_dealloc(tmem_base, kTmemColsS);
     }
 }
 
@@ -1525,42 +1420,6 @@ cudaError_t launch_1cta(const CUtensorMap& a, const CUtensorMap& b, const Params
     return cudaGetLastError();
 }
 
-// M blocks per weight-gradient item: split each expert's M blocks into the
-// fewest equal runs whose items, dealt round-robin to one CTA per SM, keep the
-// CTAs at least 90 % busy (tiles done / tiles of the slowest CTA), so the
-// panel is reused as much as the balance allows.
-int wgrad_mb_item(int groups, int n_blocks, int m_blocks, int ctas) {
-    const int64_t tiles = (int64_t)groups * n_blocks * m_blocks;
-    int best = 1;
-    double best_eff = 0.0;
-    for (int mg = 1; mg <= m_blocks; ++mg) {
-        const int mb = (m_blocks + mg - 1) / mg;
-        const int64_t items = (int64_t)groups * n_blocks * ((m_blocks + mb - 1) / mb);
-        const int64_t slowest = ((items + ctas - 1) / ctas) * mb;
-        const double eff = (double)tiles / (double)(slowest * ctas);
-        if (eff >= 0.9) return mb;
-        if (eff > best_eff) {
-            best_eff = eff;
-            best = mb;
-        }
-    }
-    return best;
-}
-
-cudaError_t launch_wgrad(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c, Params p,
-                         cudaStream_t st) {
-    static std::once_flag once;
-    static cudaError_t attr = cudaSuccess;
-    if (set_smem_once(gemm_wgrad_kernel, kSmemWBytes, once, attr) != cudaSuccess) return attr;
-    const int ctas = sm_count();
-    p.mb_item = wgrad_mb_item(p.groups, p.n_blocks, p.m_blocks, ctas);
-    const int64_t items = (int64_t)p.groups * p.n_blocks * ((p.m_blocks + p.mb_item - 1) / p.mb_item);
-    if (items <= 0) return cudaSuccess;
-    const int64_t grid = items < ctas ? items : ctas;
-    gemm_wgrad_kernel<<<(unsigned)grid, kWgThreads, kSmemWBytes, st>>>(a, b, c, p);
-    return cudaGetLastError();
-}
-
 Params base_params(int groups, int64_t rows, const int32_t* offsets, unsigned* err) {
     Params p{};
     p.groups = groups;
@@ -1582,15 +1441,40 @@ int64_t single_tile_bound(int64_t rows, int groups, int n_blocks) {
 // Pair tiles (256 rows) halve each CTA's weight traffic; an expert block's
 // last <= 128 rows run as a 128-row pair tile, so both kinds round a block up
 // to a multiple of 128 rows. Measured on B200, pair tiles were faster at 1024
-// rows per expert (Mixtral-8x7B shape) and slower at 256 (Qwen3-30B-A3B shape,
-// 259 against 242 us for gate_up).
-// MOE_GEMM_TILES=pair|single overrides the choice (used by the tests to run
-// both kernels on the same shapes).
+// rows per expert (Mixtral-8x7B shape: gate_up 1675 against 1777 us) and at 512
+// (Llama-4-17Bx16E shape: 1377 against 1470 us), and slower at 256
+// (Qwen3-30B-A3B shape: 321 against 286 us). moe_testing_set_kernels can force
+// either kind (the tests run both kernels on the same shapes).
 bool use_pair_tiles(int64_t rows, int groups) {
-    const char* force = getenv("MOE_GEMM_TILES");
-    if (force && force[0] == 'p') return true;
-    if (force && force[0] == 's') return false;
-    return groups == 1 || rows >= (int64_t)groups * 1024;
+    const int forced = kernel_override().gemm_tiles;
+    if (forced == MOE_TESTING_GEMM_PAIR) return true;
+    if (forced == MOE_TESTING_GEMM_SINGLE || forced == MOE_TESTING_GEMM_SWAP) return false;
+    return groups == 1 || rows >= (int64_t)groups * 512;
+}
+
+// The forward GEMMs take swap-AB tiles (weights as the 128-row operand, 64
+// token rows per tile) when the expert blocks average at most 16 rows: a
+// small batch, where 128-row token tiles would be mostly padding and too few
+// to spread the weight reads over the SMs.
+bool use_swap_tiles(int64_t rows, int groups) {
+    const int forced = kernel_override().gemm_tiles;
+    if (forced != MOE_TESTING_AUTO) return forced == MOE_TESTING_GEMM_SWAP;
+    return rows <= (int64_t)groups * 16;
+}
+
+template <int EPI>
+cudaError_t launch_swap(const CUtensorMap& x64, const CUtensorMap& w, const Params& p, cudaStream_t st) {
+    auto kern = gemm_swap_kernel<EPI>;
+    static std::once_flag once;
+    static cudaError_t attr = cudaSuccess;
+    if (set_smem_once(kern, kSmemSBytes, once, attr) != cudaSuccess) return attr;
+    // upper bound of the tiles without reading the device counts
+    const int64_t bound = ((int64_t)p.rows / BNS + p.groups) * (int64_t)p.n_blocks;
+    if (bound <= 0) return cudaSuccess;
+    int64_t grid = sm_count();
+    if (grid > bound) grid = bound;
+    kern<<<(unsigned)grid, kThreads, kSmemSBytes, st>>>(x64, w, p);
+    return cudaGetLastError();
 }
 
 // Group-M GEMM on pair or single tiles. `ta` and `ta64` are A maps with
@@ -1636,6 +1520,10 @@ cudaError_t gemm_gate_up_swiglu(const bf16* x, int64_t rows, const int32_t* offs
     p.out2 = gu_save;
     p.ldo2 = 2 * (int64_t)I;
     p.row_scale = row_scale;
+    if (use_swap_tiles(rows, groups)) {
+        p.n_blocks = I / 64;   // 64 gate and the matching 64 up columns per tile
+        return launch_swap<kEpiSwiglu>(ta64, tb, p, st);
+    }
     CUtensorMap tc, tc2;
     if (!make_out_map(&tc, h, rows, I)) return cudaErrorInvalidValue;
     if (gu_save && !make_out_map(&tc2, gu_save, rows, 2 * (uint64_t)I)) return cudaErrorInvalidValue;
@@ -1672,7 +1560,9 @@ cudaError_t gemm_gate_up_swiglu_gather(const bf16* x, int64_t T, const int32_t* 
                                                        gu_save ? &tc2 : nullptr);
 }
 
-bool grouped_gemm_pair_tiles(int64_t rows, int groups) { return use_pair_tiles(rows, groups); }
+bool grouped_gemm_single_tiles(int64_t rows, int groups) {
+    return !use_pair_tiles(rows, groups) && !use_swap_tiles(rows, groups);
+}
 
 cudaError_t gemm_down(const bf16* h, int64_t rows, const int32_t* offsets, int E, int H, int I,
                       const bf16* w_down, bf16* y, cudaStream_t st, unsigned* err) {
@@ -1688,6 +1578,10 @@ cudaError_t gemm_down(const bf16* h, int64_t rows, const int32_t* offsets, int E
     p.n_blocks = (H + BN - 1) / BN;
     p.out = y;
     p.ldo = H;
+    if (use_swap_tiles(rows, groups)) {
+        p.n_blocks = (H + 127) / 128;   // 128 output columns per tile
+        return launch_swap<kEpiStore>(ta64, tb, p, st);
+    }
     CUtensorMap tc;
     if (!make_out_map(&tc, y, rows, H)) return cudaErrorInvalidValue;
     return launch_group_m<kEpiStore, true>(ta, ta64, tb, tb, p, st, &tc);
@@ -1761,13 +1655,10 @@ cudaError_t gemm_wgrad(const bf16* X, const bf16* D, int64_t rows, const int32_t
     CUtensorMap tc;   // dW [E][M][N], stored in 32 x 32 blocks without swizzle
     if (!make_map_3d(&tc, dW, N, M, E > 0 ? E : 1, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
-    // One 128 x 256 tile per CTA at a time. MOE_WGRAD=panel runs the kernel
-    // that keeps each expert's B rows in shared memory instead; on B200 it
-    // measured slower at the Qwen3-30B-A3B shape (313 against 288 us for the
-    // gate_up gradient): its A ring has 3 stages and each item waits for its
-    // whole panel. The tests run both.
-    const char* force = getenv("MOE_WGRAD");
-    if (force && force[0] == 'p') return launch_wgrad(ta, tb, tc, p, st);
+    // One 128 x 256 tile per CTA at a time. A kernel that kept each expert's
+    // B rows in shared memory across M blocks measured slower at the
+    // Qwen3-30B-A3B shape (313 against 288 us for the gate_up gradient): its
+    // A ring had 3 stages and each item waited for its whole panel.
     return launch_1cta<kEpiStore, true, true, true>(ta, tb, p, (int64_t)E * p.m_blocks * p.n_blocks, st,
                                                    &tc);
 }

@@ -154,6 +154,26 @@ int sm_count() {
     return di ? di->sms : 148;
 }
 
+KernelOverride g_override;
+
+// One thread waits, with the given limit, on an mbarrier that nothing arrives
+// on: the bounded wait of the GEMM kernels (mbar_wait_limit) running out.
+// It records kErrTimeout in the device error word and returns.
+__global__ void wait_on_nothing_kernel(unsigned long long limit_ns, unsigned* err) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait_limit(&bar, 0, &abort_flag, err, limit_ns);
+    __syncthreads();
+}
+
+const KernelOverride& kernel_override() { return g_override; }
+
 }  // namespace moe
 
 using namespace moe;
@@ -187,6 +207,26 @@ moe_status moe_get_device_status(void* stream) {
     if (v & kErrTimeout) return MOE_ERR_TIMEOUT;
     if (v & kErrDeviceCheck) return MOE_ERR_DEVICE_CHECK;
     return MOE_OK;
+}
+
+moe_status moe_testing_set_kernels(int gemm_tiles, int router, int permute, int fold_permute) {
+    if (gemm_tiles < 0 || gemm_tiles > 3 || router < 0 || router > 2 || permute < 0 || permute > 2 ||
+        fold_permute < 0 || fold_permute > 1)
+        return MOE_ERR_INVALID_ARG;
+    moe::g_override.gemm_tiles = gemm_tiles;
+    moe::g_override.router = router;
+    moe::g_override.permute = permute;
+    moe::g_override.fold_permute = fold_permute;
+    return MOE_OK;
+}
+
+moe_status moe_testing_wait_timeout(int64_t limit_ns, void* stream) {
+    if (limit_ns <= 0 || limit_ns > 1000000000) return MOE_ERR_INVALID_ARG;
+    unsigned* err = device_error_word();
+    if (!err) return MOE_ERR_CUDA;
+    moe::wait_on_nothing_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        (unsigned long long)limit_ns, err);
+    return from_cuda(cudaGetLastError());
 }
 
 moe_status moe_trace_set(void* const* events, int n_events) {
@@ -515,15 +555,14 @@ moe_status moe_layer_forward(const float* logits, const moe_bf16* x, int64_t T, 
                                err);
     if (e == cudaSuccess) e = launch_expert_scan(T, E, L.rs, L.counts, L.offsets, st);
     if (e == cudaSuccess) e = trace_mark(1, st);
-    // MOE_GATHER=1: without a requested x_perm, on single-CTA tiles, the gate_up
-    // GEMM gathers its A rows from x by token (the permute computes the rows
-    // only), so the permuted copy of x is never written or read. Off by
-    // default: on B200 the cp.async row gather feeds the tensor cores more
-    // slowly than TMA tiles of x_perm (508 against 412 us for the Qwen3-30B-A3B
-    // forward), more than the permute's copy costs.
-    const char* gather_env = getenv("MOE_GATHER");
-    const bool gather = x_perm == nullptr && !grouped_gemm_pair_tiles(A, E) && (H % 8) == 0 && gather_env &&
-                        gather_env[0] == '1';
+    // Folded permute (moe_testing_set_kernels): without a requested x_perm, on
+    // single-CTA tiles, the gate_up GEMM gathers its A rows from x by token
+    // (the permute computes the rows only), so the permuted copy of x is never
+    // written or read. Off by default: on B200 the cp.async row gather feeds
+    // the tensor cores more slowly than TMA tiles of x_perm (508 against 412 us
+    // for the Qwen3-30B-A3B forward), more than the permute's copy costs.
+    const bool gather = x_perm == nullptr && grouped_gemm_single_tiles(A, E) && (H % 8) == 0 &&
+                        kernel_override().fold_permute != 0;
     if (e == cudaSuccess)
         e = launch_permute(xb, T, H, L.topk_idx, k, L.offsets, E, L.rs, gather ? nullptr : L.x_perm,
                            L.sorted_token, L.row_of, st, err);

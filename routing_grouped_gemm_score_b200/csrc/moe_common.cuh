@@ -79,23 +79,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase of `bar` with the given parity to complete. Gives up
-// after kWaitLimitNs, or at once when *abort is set by another role. On a
+// after limit_ns, or at once when *abort is set by another role. On a
 // timeout it records kErrTimeout and sets *abort. Returns false if it gave up.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          unsigned* err) {
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                unsigned* err, unsigned long long limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     unsigned long long start = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 63u) == 0) {
             if (*abort) return false;
-            if (global_timer_ns() - start > kWaitLimitNs) {
+            if (global_timer_ns() - start > limit_ns) {
                 raise_error(err, kErrTimeout);
                 *abort = 1;
                 return false;
             }
         }
     }
+}
+
+// mbar_wait_limit with the kernels' limit, kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          unsigned* err) {
+    return mbar_wait_limit(bar, parity, abort, err, kWaitLimitNs);
 }
 
 // Waits for the phase with the given parity for at most kWaitLimitNs,

@@ -98,8 +98,9 @@ cudaError_t gemm_gate_up_swiglu_gather(const bf16* x, int64_t T, const int32_t* 
                                        const int32_t* offsets, int E, int H, int I, const bf16* w_gate_up, bf16* h,
                                        bf16* gu_save, cudaStream_t st, unsigned* err,
                                        const float* row_scale = nullptr);
-// Whether the group-M GEMMs run on CTA-pair tiles for this many rows and groups.
-bool grouped_gemm_pair_tiles(int64_t rows, int groups);
+// Whether the forward gate_up GEMM runs on single-CTA 128-row tiles (not CTA
+// pairs, not swap-AB tiles) for this many rows and groups.
+bool grouped_gemm_single_tiles(int64_t rows, int groups);
 // down: y[r] = h[r] Wd[e]
 cudaError_t gemm_down(const bf16* h, int64_t rows, const int32_t* offsets, int E, int H, int I,
                       const bf16* w_down, bf16* y, cudaStream_t st, unsigned* err);
@@ -117,5 +118,15 @@ cudaError_t gemm_wgrad(const bf16* X, const bf16* D, int64_t rows, const int32_t
                        int M, int N, bf16* dW, cudaStream_t st, unsigned* err);
 
 int sm_count();
+
+// Kernel variants forced by moe_testing_set_kernels (MOE_TESTING_AUTO: the
+// library's own choice by shape).
+struct KernelOverride {
+    int gemm_tiles = MOE_TESTING_AUTO;
+    int router = MOE_TESTING_AUTO;
+    int permute = MOE_TESTING_AUTO;
+    int fold_permute = 0;
+};
+const KernelOverride& kernel_override();
 
 }  // namespace moe

@@ -1192,13 +1192,14 @@ cudaError_t launch_router_topk(const float* logits, int64_t T, int E, int k,
     a.ticket = rs.ticket;
     a.nb = (int)route_blocks(T);
     a.tpb = route_tokens_per_block(T);
-    // Large T: the lane-per-token kernel where it applies. MOE_ROUTER=lane|warp
-    // overrides the choice (the tests run both on the same inputs).
-    const char* force = getenv("MOE_ROUTER");
+    // Large T: the lane-per-token kernel where it applies. moe_testing_set_kernels
+    // can force either kernel (the tests run both on the same inputs).
+    const int force = kernel_override().router;
     const bool lane_ok = E % 32 == 0 && E <= 256 && k <= 8 && kLaneTokens % a.tpb == 0 &&
                          (opts.score_fn == MOE_SCORE_SIGMOID || opts.renormalize) &&
                          ((uintptr_t)logits & 15u) == 0;
-    const bool use_lane = lane_ok && (force ? force[0] == 'l' : T >= kLaneMinTokens);
+    const bool use_lane = lane_ok && (force != MOE_TESTING_AUTO ? force == MOE_TESTING_ROUTER_LANE
+                                                                 : T >= kLaneMinTokens);
     if (use_lane) {
         const dim3 lgrid((unsigned)((T + kLaneTokens - 1) / kLaneTokens)), lblock(kLaneTokens);
         const bool bias = opts.expert_bias != nullptr;
@@ -1304,10 +1305,10 @@ cudaError_t launch_permute(const bf16* x, int64_t T, int H, const int32_t* topk_
     // Token-range register kernel for rows up to 4096 wide, warp per token
     // otherwise. Measured inside the steps on B200 (fraction of HBM): k=8,
     // H=2048: 0.73 against 0.67 for the warp kernel; k=2, H=4096: 0.67
-    // against 0.64; H=5120: warp 0.76. MOE_PERMUTE=warp selects the warp
-    // kernel for any width.
-    const char* force = getenv("MOE_PERMUTE");
-    const bool regs = x_perm == nullptr || (H8r <= 512 && !(force && force[0] == 'w'));
+    // against 0.64; H=5120: warp 0.76. moe_testing_set_kernels can select
+    // the warp kernel for any width.
+    const int force = kernel_override().permute;
+    const bool regs = x_perm == nullptr || (H8r <= 512 && force != MOE_TESTING_PERMUTE_WARP);
     if (regs) {
         // without x_perm only the rows are computed: 256 threads whatever H
         const int threads = x_perm == nullptr ? 256 : (H8r + 31) / 32 * 32;
@@ -1344,25 +1345,32 @@ cudaError_t launch_permute(const bf16* x, int64_t T, int H, const int32_t* topk_
 
 // Device address of g_router_noalloc_scratch on the current device. In host
 // code the array's name is only a host-side stand-in, so the address is taken
-// with cudaGetSymbolAddress, once per device, while that device is current.
+// with cudaGetSymbolAddress while that device is current. A successful lookup
+// is kept for the device; a failed one (for example a first call made while
+// the stream is being captured) is not, and the next call tries again.
 size_t router_noalloc_capacity() { return kNoAllocScratchBytes; }
 
 cudaError_t router_noalloc_scratch(void** ptr) {
     constexpr int kMaxDev = 64;
-    static std::once_flag once[kMaxDev];
+    static std::mutex mu;
     static void* addr[kMaxDev];
-    static cudaError_t status[kMaxDev];
+    *ptr = nullptr;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
-    std::call_once(once[dev], [dev] {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
         void* p = nullptr;
-        status[dev] = cudaGetSymbolAddress(&p, g_router_noalloc_scratch);
-        addr[dev] = (status[dev] == cudaSuccess) ? p : nullptr;
-    });
+        e = cudaGetSymbolAddress(&p, g_router_noalloc_scratch);
+        if (e != cudaSuccess) {
+            cudaGetLastError();   // the failed lookup's error is returned here, not left for a later call
+            return e;
+        }
+        addr[dev] = p;
+    }
     *ptr = addr[dev];
-    return status[dev];
+    return cudaSuccess;
 }
 
 }  // namespace moe

@@ -7,6 +7,7 @@ import pytest
 import torch
 
 import oracle
+import helpers
 import workloads as wl
 from helpers import assert_close, bits, require_gpu
 
@@ -31,7 +32,7 @@ def grouped_case(T, H, I, E, k, seed, dead=(), skew=False):
     return m, w, d, r, p
 
 
-@pytest.mark.parametrize("tiles", ["single", "pair"])
+@pytest.mark.parametrize("tiles", ["single", "pair", "swap"])
 @pytest.mark.parametrize("T,H,I,E,k,dead", [
     (64, 128, 256, 8, 2, ()),            # the tiny workload's shape
     (1000, 256, 384, 4, 2, (2,)),        # several M tiles per expert, a ragged tail, an empty expert
@@ -41,7 +42,7 @@ def grouped_case(T, H, I, E, k, seed, dead=(), skew=False):
     (4500, 256, 256, 4, 2, (1,)),        # large expert blocks (the default picks pair tiles)
 ])
 def test_grouped_mlp_matches_expert_loop(T, H, I, E, k, dead, tiles, monkeypatch):
-    monkeypatch.setenv("MOE_GEMM_TILES", tiles)
+    helpers.force_kernels(gemm_tiles=tiles)
     m, w, d, r, p = grouped_case(T, H, I, E, k, seed=T + H + I, dead=dead)
     out = m.moe_grouped_mlp(p["x_perm"], r["offsets"], d["w_gate_up"], d["w_down"], save=True)
     torch.cuda.synchronize()
@@ -71,9 +72,11 @@ def test_grouped_mlp_is_deterministic():
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
-def test_rows_past_offsets_end_are_untouched():
+@pytest.mark.parametrize("tiles", ["auto", "swap"])
+def test_rows_past_offsets_end_are_untouched(tiles):
     """offsets[E] < A: rows after the last expert block are not written."""
     import routing_grouped_gemm_score_b200 as m
+    helpers.force_kernels(gemm_tiles=tiles)
     E, H, I = 4, 128, 128
     A = 300
     offsets = torch.tensor([0, 50, 50, 170, 200], dtype=torch.int32, device="cuda")
@@ -93,14 +96,14 @@ def test_rows_past_offsets_end_are_untouched():
     assert_close(y[:200], ref[:200], "y_perm")
 
 
-@pytest.mark.parametrize("tiles", ["single", "pair"])
+@pytest.mark.parametrize("tiles", ["single", "pair", "swap"])
 def test_block_sizes_around_tile_edges(tiles, monkeypatch):
     """Expert blocks of 0, 1, 63, 64, 65, 127, 128, 129, 255, 256, 257 and
     385 rows: every split of a block into 256-row pair tiles plus a last
     128-row pair tile (one CTA's 64 rows empty or not), and into 128-row
     single tiles, with g, u and h checked as well as y."""
     import routing_grouped_gemm_score_b200 as m
-    monkeypatch.setenv("MOE_GEMM_TILES", tiles)
+    helpers.force_kernels(gemm_tiles=tiles)
     sizes = [0, 1, 63, 64, 65, 127, 128, 129, 255, 256, 257, 385]
     E, H, I = len(sizes), 192, 320
     offs = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)

@@ -50,15 +50,15 @@ SMALL = {
 }
 
 
-@pytest.mark.parametrize("tiles", ["single", "pair"])
+@pytest.mark.parametrize("tiles", ["single", "pair", "swap"])
 @pytest.mark.parametrize("name", list(SMALL))
 def test_layer_forward_matches_per_token_definition(name, tiles, monkeypatch):
-    monkeypatch.setenv("MOE_GEMM_TILES", tiles)
+    helpers.force_kernels(gemm_tiles=tiles)
     w = SMALL[name]
     d = wl.make_inputs(w, "cuda")
     out = layer(w, d)
     tokens = np.arange(w.T)
-    helpers.assert_close_flips(out, oracle_out(w, d), helpers.forward_terms(w, d, tokens), f"{name}: out")
+    helpers.assert_close_flips(out, oracle_out(w, d), helpers.lazy_forward_terms(w, d, tokens), f"{name}: out")
 
 
 def test_layer_forward_saved_state_and_empty_batch():
@@ -85,17 +85,15 @@ def _oracle_backward(w, d, r):
                                bits(d["w_down"]), bits(d["dout"]))
 
 
-@pytest.mark.parametrize("wgrad", ["panel", "tiles"])
 @pytest.mark.parametrize("tiles", ["single", "pair"])
 @pytest.mark.parametrize("name", BWD)
-def test_backward_on_oracle_state(name, tiles, wgrad, monkeypatch):
+def test_backward_on_oracle_state(name, tiles):
     """The backward kernels fed with the oracle's own saved forward state, so
     both sides read identical bf16 inputs. dW_down and dprob then differ only
     in accumulation order; dW_gate_up and dx also carry the bf16 rounding of
     dg, du and each token row's dx, whose fp32 and fp64 pre-images can round
     apart (assert_close_flips)."""
-    monkeypatch.setenv("MOE_GEMM_TILES", tiles)
-    monkeypatch.setenv("MOE_WGRAD", wgrad)   # weight gradient: B panel in shared memory, or one tile per CTA
+    helpers.force_kernels(gemm_tiles=tiles)
     _check_backward_on_oracle_state(name, SMALL[name])
 
 
@@ -139,9 +137,13 @@ def _check_backward_on_oracle_state(name, w):
 
 @pytest.mark.parametrize("name", BWD)
 def test_backward_end_to_end(name):
-    """Forward state from the GPU forward, then the GPU backward, against the
-    oracle's chain rule. The forward's stored h and y can also round apart
-    from the oracle's, so every gradient uses assert_close_flips."""
+    """The GPU forward, then the GPU backward on the state it saved. The saved
+    state ([g | u], h, y) is checked against the oracle's forward, strictly
+    within the bound; the gradients against the oracle's chain rule on that
+    same state (the inputs the backward call was given). dprob and dW_down
+    read only that state: strict. dx and dW_gate_up also carry the backward's
+    own bf16 roundings of [dg | du] and of each permuted row's dx, whose fp32
+    and fp64 pre-images can round apart (one-flip allowance, counted)."""
     import routing_grouped_gemm_score_b200 as m
     w = SMALL[name]
     d = wl.make_inputs(w, "cuda", with_dout=True)
@@ -151,10 +153,21 @@ def test_backward_end_to_end(name):
     assert m.moe_get_device_status() == 0
     r = oracle.router_topk(d["logits"].cpu().numpy(), w.k)
     assert_equal(st["topk_idx"], r["topk_idx"], "topk_idx")
-    ref = _oracle_backward(w, d, r)
-    terms = helpers.flip_terms(w, d, r, helpers.oracle_saved_state(w, d, r))
-    for key in ("dprob", "dx", "dw_down", "dw_gate_up"):
-        helpers.assert_close_flips(gr[key], ref[key], terms[key], f"{name}: {key}")
+    s = helpers.oracle_saved_state(w, d, r)
+    assert_equal(st["row_of"], s["row_of"], f"{name}: row_of")
+    assert_close(st["gu"][:, :w.I], s["g"], f"{name}: saved g")
+    assert_close(st["gu"][:, w.I:], s["u"], f"{name}: saved u")
+    assert_close(st["h"], s["h"], f"{name}: saved h")
+    assert_close(st["y_perm"], s["y"], f"{name}: saved y")
+    gpu_state = {"row_of": st["row_of"].cpu().numpy(), "gu": bits(st["gu"]), "h": bits(st["h"]),
+                 "y": bits(st["y_perm"])}
+    ref = oracle.moe_backward(bits(d["x"]), r["topk_idx"], r["topk_prob"], bits(d["w_gate_up"]),
+                              bits(d["w_down"]), bits(d["dout"]), state=gpu_state)
+    assert_close(gr["dprob"], ref["dprob"], f"{name}: dprob")
+    assert_close(gr["dw_down"], ref["dw_down"], f"{name}: dw_down")
+    terms = helpers.flip_terms(w, d, r, s)
+    helpers.assert_close_flips(gr["dw_gate_up"], ref["dw_gate_up"], terms["dw_gate_up"], f"{name}: dw_gate_up")
+    helpers.assert_close_flips(gr["dx"], ref["dx"], terms["dx"], f"{name}: dx")
     counts = st["counts"].cpu().numpy()
     for e in np.nonzero(counts == 0)[0]:
         assert torch.all(gr["dw_down"][e] == 0) and torch.all(gr["dw_gate_up"][e] == 0)

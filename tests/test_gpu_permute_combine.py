@@ -6,6 +6,7 @@ import pytest
 import torch
 
 import oracle
+import helpers
 import workloads as wl
 from helpers import assert_close, assert_equal, bits, require_gpu
 
@@ -34,7 +35,7 @@ def test_permute_matches_dispatch_definition(name, T, H, path, monkeypatch):
     """Both permute kernels on every shape: the default choice (the
     token-range register kernel for rows up to 4096 wide, else one warp per
     token) and the warp-per-token kernel forced."""
-    monkeypatch.setenv("MOE_PERMUTE", path) if path != "auto" else None
+    helpers.force_kernels(permute=path)
     w = wl.WORKLOADS[name]
     if T is not None:
         w = w.scaled(T=T)
@@ -56,7 +57,7 @@ def test_permute_rejects_invalid_indices_on_the_device(path, monkeypatch):
     """Bad expert indices made on the host: the kernel flags them, skips the
     rows, and the status call reports MOE_ERR_DEVICE_CHECK."""
     import routing_grouped_gemm_score_b200 as m
-    monkeypatch.setenv("MOE_PERMUTE", path) if path != "auto" else None
+    helpers.force_kernels(permute=path)
     T, E, k, H = 100, 8, 2, 64
     idx = torch.randint(0, E, (T, k), dtype=torch.int32)
     idx[:, 1] = (idx[:, 0] + 1) % E

@@ -5,6 +5,7 @@ import numpy as np
 import pytest
 import torch
 
+import helpers
 import workloads as wl
 from helpers import assert_equal, require_gpu
 
@@ -167,7 +168,7 @@ LANE_CASES = [(1, 32, 1, "softmax_renorm"), (255, 64, 2, "softmax_renorm"), (256
 
 def _router_outputs(logits, k, score, renorm, kernel, monkeypatch, bias=None, scaling=1.0):
     import routing_grouped_gemm_score_b200 as m
-    monkeypatch.setenv("MOE_ROUTER", kernel)
+    helpers.force_kernels(router=kernel)
     opts = m.RouterOpts(score, renorm, scaling, bias)
     g = m.moe_router_topk(logits, k, opts, routing_map=True)
     torch.cuda.synchronize()
@@ -264,7 +265,7 @@ def test_lane_router_ranks_drive_the_same_dispatch(monkeypatch):
     d = wl.make_inputs(w, "cuda")
     res = {}
     for kernel in ("lane", "warp"):
-        monkeypatch.setenv("MOE_ROUTER", kernel)
+        helpers.force_kernels(router=kernel)
         out, st = m.moe_layer_forward(d["logits"], d["x"], d["w_gate_up"], d["w_down"], w.k,
                                       save_for_backward=True)
         torch.cuda.synchronize()

@@ -71,6 +71,29 @@ def test_noalloc_router_matches_workspace_router_twice():
                                    rtol=1e-6, atol=0)
 
 
+def test_noalloc_router_at_its_limit():
+    """T = 32768 tokens at E = 256, k = 8: the largest call the fixed scratch
+    admits (T * k at its limit, the scratch filled to within a few KiB), on
+    the router kernel that large batches use. Bit-exact against the
+    workspace router; one token more is rejected before any launch."""
+    import routing_grouped_gemm_score_b200 as m
+    T, E, k = 32768, 256, 8
+    g = torch.Generator(device="cuda").manual_seed(4242)
+    logits = torch.randn((T, E), generator=g, device="cuda")
+    oc = m.RouterOpts().c()
+    ref = _route("moe_router_topk", logits, k, oc, True)
+    got = _route("moe_router_topk_noalloc", logits, k, oc, False)
+    for key in ("topk_idx", "routing_map", "counts", "offsets", "topk_prob"):
+        assert torch.equal(got[key], ref[key]), key
+    b = _buffers(1, E, k)
+    rc = m.lib().moe_router_topk_noalloc(logits.data_ptr(), T + 1, E, k, ctypes.byref(oc),
+                                         b["topk_idx"].data_ptr(), b["topk_prob"].data_ptr(), None,
+                                         b["counts"].data_ptr(), b["offsets"].data_ptr(),
+                                         torch.cuda.current_stream().cuda_stream)
+    assert rc == 2      # MOE_ERR_UNSUPPORTED
+    assert torch.all(b["counts"] == -7)
+
+
 def test_noalloc_router_rejects_sizes_beyond_its_scratch():
     import routing_grouped_gemm_score_b200 as m
     l = m.lib()
