@@ -13,6 +13,13 @@ are already resident in HBM when the timed region starts. The weights exceed
 L2 (126 MB), which keeps the steps L2-cold without a flush. Rank 0 prints one
 JSON line.
 
+The default workload is the largest single-GPU one, the Llama-4-17Bx16E-shaped
+forward with its shared expert. On one GPU the line also carries the other
+workloads under "workloads": the Mixtral-8x7B-shaped forward, the
+Qwen3-30B-A3B-shaped forward + backward, and the skewed sweep at T = 1, 8, 64
+and 16384 (each of these small batches timed with L2 flushed before every
+step, since their weights can fit in L2).
+
 With N > 1 (torchrun), each rank runs its own replica of the layer on its own
 tokens (data-parallel replicas; the forward has no exchange step). value =
 tokens of all ranks / the slowest rank's time. --impl reference times the CPU
@@ -37,7 +44,9 @@ if ROOT not in sys.path:
 
 METRIC = "MoE layer tokens/s and grouped-GEMM TFLOP/s (% of B200 bf16 peak), 1 GPU"
 UNIT = "tokens/s"
-DEFAULT_WORKLOAD = "mixtral_8x7b"
+DEFAULT_WORKLOAD = "llama4_17bx16e"
+NOMINAL_BF16_TFLOPS = 2250.0   # dense bf16 tensor peak of one B200 (vendor figure, no sparsity)
+EXTRA_WORKLOADS = ["mixtral_8x7b", "qwen3_30b_a3b", "skew_t1", "skew_t8", "skew_t64", "skew_t16384"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -53,6 +62,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="time only --workload (not the other workloads of the \"workloads\" key)")
     ap.add_argument("--router-sweep", action="store_true",
                     help="also time the router alone at E=128, k=8, T = 2^16 .. 2^20")
     ap.add_argument("--router-calls", type=int, default=None, metavar="LOGT",
@@ -290,6 +301,258 @@ def traffic_for(kernel: str):
 
 
 # ------------------------------------------------------------------ our arm
+FWD_STAGES = ["router", "permute", "gate_up_swiglu", "down", "shared_expert", "combine"]
+BWD_STAGES = ["combine_bwd", "down_dgrad_swiglu_bwd", "gate_up_dgrad", "dx_token_sum", "down_wgrad",
+              "gate_up_wgrad"]
+GEMM_STAGES = ["fwd_gate_up_swiglu", "fwd_down", "fwd_shared_expert", "bwd_down_dgrad_swiglu_bwd",
+               "bwd_gate_up_dgrad", "bwd_down_wgrad", "bwd_gate_up_wgrad"]
+
+
+def bandwidth_bytes(w):
+    """Algorithmic bytes of the bandwidth-bound stages: what each must read
+    and write once (bf16 rows 2 B per element, indices and weights 4 B)."""
+    T, H, k, E, A = w.T, w.H, w.k, w.E, w.A
+    b = {"fwd_router": T * E * 4 + T * k * 8 + E * 8,
+         "fwd_permute": T * H * 2 + A * H * 2 + A * 4 + T * k * 4,
+         "fwd_combine": A * H * 2 + T * H * 2 + T * k * 8 + (T * H * 2 if w.shared_expert else 0)}
+    if w.backward:
+        b["bwd_combine_bwd"] = T * H * 2 + 2 * A * H * 2 + T * k * 12
+        b["bwd_dx_token_sum"] = A * H * 2 + T * H * 2 + T * k * 4
+    return b
+
+
+class Layer:
+    """One workload's inputs, workspace and outputs on the device, and its
+    step (the fused forward, plus the grouped-MLP backward when it trains)."""
+
+    def __init__(self, m, w, d):
+        import torch
+        self.m, self.w, self.d = m, w, d
+        self.opts = m.RouterOpts(w.score, w.renormalize)
+        self.ws = m.LayerWorkspace(w.T, w.H, w.I, w.E, w.k, w.shared_expert, backward=w.backward)
+        self.out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device="cuda")
+        # the routing and saved state are kept so the combine can be timed alone
+        _, self.state = m.moe_layer_forward(d["logits"], d["x"], d["w_gate_up"], d["w_down"], w.k, self.opts,
+                                            d["shared_gate_up"], d["shared_down"], save_for_backward=True,
+                                            workspace=self.ws, out=self.out)
+        self.grads = None
+        if w.backward:
+            self.grads = m.moe_grouped_mlp_backward(d["dout"], self.state, d["w_gate_up"], d["w_down"], self.ws)
+        if not w.backward:   # the forward-only step saves nothing beyond the routing
+            self.state = {k_: self.state[k_] for k_ in ("topk_idx", "topk_prob", "counts", "offsets", "row_of",
+                                                        "y_perm")}
+            self.fwd_state = None
+        else:
+            self.fwd_state = self.state
+
+    def step(self, fev=None, bev=None):
+        m, w, d = self.m, self.w, self.d
+        if fev:
+            m.moe_trace_set(fev)
+        m.moe_layer_forward(d["logits"], d["x"], d["w_gate_up"], d["w_down"], w.k, self.opts,
+                            d["shared_gate_up"], d["shared_down"], save_for_backward=w.backward,
+                            workspace=self.ws, out=self.out, state=self.fwd_state)
+        if w.backward:
+            if bev:
+                m.moe_trace_set(bev)
+            m.moe_grouped_mlp_backward(d["dout"], self.state, d["w_gate_up"], d["w_down"], self.ws, self.grads)
+        if fev or bev:
+            m.moe_trace_set(None)
+
+    def launches(self):
+        return 6 + (2 if self.w.shared_expert else 0) + (6 if self.w.backward else 0)
+
+
+def _events(n):
+    import torch
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for e in evs:
+        e.record()           # materialise the events before handing them to the library
+    return evs
+
+
+def stage_medians(layer, fevs, bevs):
+    """Per-stage device time (ms), the median over the traced steps."""
+    st = {}
+    for i, n in enumerate(FWD_STAGES):
+        st[f"fwd_{n}"] = statistics.median(evs[i].elapsed_time(evs[i + 1]) for evs in fevs)
+    if layer.w.backward:
+        for i, n in enumerate(BWD_STAGES):
+            st[f"bwd_{n}"] = statistics.median(evs[i].elapsed_time(evs[i + 1]) for evs in bevs)
+    return st
+
+
+def gemm_summary(w, stages, peaks):
+    """Grouped-GEMM TFLOP/s over the GEMM stages' device time, against the
+    burst and sustained measured peaks and the nominal dense bf16 peak."""
+    ms = sum(stages.get(k_, 0.0) for k_ in GEMM_STAGES if k_ != "fwd_shared_expert" or w.shared_expert)
+    flop = w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0)
+    tf = flop / (ms / 1e3) / 1e12
+    return {"tflops": tf, "flop_per_step": flop, "gemm_ms": ms,
+            "frac_of_burst_peak": tf / peaks["bf16_tflops"],
+            "frac_of_sustained_peak": tf / peaks["bf16_tflops_sustained"],
+            "frac_of_nominal_peak": tf / NOMINAL_BF16_TFLOPS,
+            "note": "expert GEMM FLOPs (6AHI fwd incl. shared expert, 12AHI bwd) / device time of the GEMM stages"}
+
+
+def warm_bandwidth(w, stages, hbm):
+    out = {}
+    for key, nbytes in bandwidth_bytes(w).items():
+        gbs = nbytes / (stages[key] / 1e3) / 1e9
+        out[key] = {"bytes": nbytes, "warm_us": stages[key] * 1e3, "warm_frac_of_hbm": gbs / hbm}
+    return out
+
+
+def cold_bandwidth(layer, hbm, flush, reps=50, warm=10):
+    """The bandwidth-bound stages with L2 flushed (a 256 MB read) before each
+    timed call; median of `reps` after `warm`. The fused forward's router and
+    permute run first after the flush; the combine (and the backward's dx
+    token sum, the same kernel without weights) is timed as its own call on
+    the step's saved rows; the backward's combine-bwd runs first in its call."""
+    import torch
+    m, w, d, st = layer.m, layer.w, layer.d, layer.state
+    res = {"fwd_router": [], "fwd_permute": [], "fwd_combine": []}
+    if w.backward:
+        res.update({"bwd_combine_bwd": [], "bwd_dx_token_sum": []})
+    shared = None
+    if w.shared_expert:
+        shared = torch.zeros((w.T, w.H), dtype=torch.bfloat16, device="cuda")
+
+    def timed(fn):
+        flush.sum()
+        torch.cuda._sleep(200000)      # the GPU is busy while the call is issued: device time only
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        fn()
+        e.record()
+        return s, e
+
+    for it in range(warm + reps):
+        fev = _events(7)
+        flush.sum()
+        torch.cuda._sleep(200000)
+        m.moe_trace_set(fev)
+        m.moe_layer_forward(d["logits"], d["x"], d["w_gate_up"], d["w_down"], w.k, layer.opts,
+                            d["shared_gate_up"], d["shared_down"], save_for_backward=w.backward,
+                            workspace=layer.ws, out=layer.out, state=layer.fwd_state)
+        m.moe_trace_set(None)
+        c = timed(lambda: m.moe_unpermute_combine(st["y_perm"], st["row_of"], st["topk_prob"], shared,
+                                                  out=layer.out))
+        if w.backward:
+            bev = _events(7)
+            flush.sum()
+            torch.cuda._sleep(200000)
+            m.moe_trace_set(bev)
+            m.moe_grouped_mlp_backward(d["dout"], st, d["w_gate_up"], d["w_down"], layer.ws, layer.grads)
+            m.moe_trace_set(None)
+            dxs = timed(lambda: m.moe_unpermute_combine(st["y_perm"], st["row_of"], None, out=layer.out))
+        torch.cuda.synchronize()
+        if it < warm:
+            continue
+        res["fwd_router"].append(fev[0].elapsed_time(fev[1]))
+        res["fwd_permute"].append(fev[1].elapsed_time(fev[2]))
+        res["fwd_combine"].append(c[0].elapsed_time(c[1]))
+        if w.backward:
+            res["bwd_combine_bwd"].append(bev[0].elapsed_time(bev[1]))
+            res["bwd_dx_token_sum"].append(dxs[0].elapsed_time(dxs[1]))
+    nbytes = bandwidth_bytes(w)
+    out = {}
+    for key, v in res.items():
+        ms = statistics.median(v)
+        out[key] = {"cold_us": ms * 1e3, "cold_frac_of_hbm": nbytes[key] / (ms / 1e3) / 1e9 / hbm}
+    return out
+
+
+def bandwidth_report(layer, stages, hbm, flush):
+    bw = warm_bandwidth(layer.w, stages, hbm)
+    for key, v in cold_bandwidth(layer, hbm, flush).items():
+        bw[key].update(v)
+    return bw
+
+
+def nonempty_experts(layer):
+    return int((layer.state["counts"] > 0).sum().item())
+
+
+def measure_flushed(layer, steps, warmup, flush):
+    """Each step timed on its own after an L2 flush (for workloads whose
+    weights could stay in L2 between steps); median over the steps."""
+    import torch
+    totals, fevs, bevs = [], [], []
+    for it in range(warmup + steps):
+        fev = _events(7)
+        bev = _events(7) if layer.w.backward else None
+        flush.sum()
+        torch.cuda._sleep(200000)
+        layer.step(fev, bev)
+        torch.cuda.synchronize()
+        if it >= warmup:
+            fevs.append(fev)
+            bevs.append(bev)
+            totals.append(fev[0].elapsed_time((bev or fev)[6]))
+    return statistics.median(totals), fevs, bevs
+
+
+def measure_back_to_back(layer, steps, warmup):
+    """`steps` steps back to back between two events (no flush: the weights
+    exceed L2); per-stage events on every step."""
+    import torch
+    for _ in range(warmup):
+        layer.step()
+    torch.cuda.synchronize()
+    fevs = [_events(7) for _ in range(steps)]
+    bevs = [_events(7) for _ in range(steps)] if layer.w.backward else [None] * steps
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for i in range(steps):
+        layer.step(fevs[i], bevs[i])
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / steps, fevs, bevs
+
+
+def workload_entry(m, name, peaks, flush, steps=50, warmup=10):
+    """One extra workload: its median step time, tokens/s, grouped-GEMM
+    fractions, bandwidth stages (warm and L2-cold), and for the small batches
+    the HBM roofline of the non-empty experts' weights."""
+    import torch
+    import workloads as wl
+    w = wl.WORKLOADS[name]
+    d = wl.make_inputs(w, "cuda")
+    layer = Layer(m, w, d)
+    small = w.T <= 64
+    if small:
+        ms, fevs, bevs = measure_flushed(layer, steps, warmup, flush)
+    else:
+        ms, fevs, bevs = measure_back_to_back(layer, steps, warmup)
+    if m.moe_get_device_status() != 0:
+        raise RuntimeError(f"device status error in {name}")
+    stages = stage_medians(layer, fevs, bevs)
+    hbm = peaks["hbm_gbs"]
+    e = {"T": w.T, "H": w.H, "I": w.I, "E": w.E, "top_k": w.k, "pass": "fwd+bwd" if w.backward else "fwd",
+         "ms_per_step": ms, "tokens_per_s": w.T / (ms / 1e3),
+         "l2": "flushed (256 MB read) before each step" if small else "weights exceed L2; steps back to back",
+         "grouped_gemm": gemm_summary(w, stages, peaks),
+         "stages_us": {k_: v * 1e3 for k_, v in stages.items()}}
+    if small:
+        ne = nonempty_experts(layer)
+        wbytes = ne * 3 * w.H * w.I * 2
+        gemm_ms = stages["fwd_gate_up_swiglu"] + stages["fwd_down"]
+        e["roofline"] = {"bound": "hbm", "unit": "GB/s",
+                         "weight_bytes": wbytes, "nonempty_experts": ne,
+                         "gemm_us": gemm_ms * 1e3, "achieved": wbytes / (gemm_ms / 1e3) / 1e9, "peak": hbm,
+                         "frac": wbytes / (gemm_ms / 1e3) / 1e9 / hbm,
+                         "layer_frac": wbytes / (ms / 1e3) / 1e9 / hbm,
+                         "note": "bytes = the non-empty experts' weights (3 H I bf16 each), read once per step; "
+                                 "frac over the two GEMM stages, layer_frac over the whole step"}
+    else:
+        e["bandwidth_kernels"] = bandwidth_report(layer, stages, hbm, flush)
+    del layer, d
+    torch.cuda.empty_cache()
+    return e
+
+
 def our_arm(args, world, rank, local):
     import torch
 
@@ -307,42 +570,17 @@ def our_arm(args, world, rank, local):
         d["x"] = wl.make_x(wr, "cuda")
         if w.backward:
             d["dout"] = wl.make_dout(wr, "cuda")
-    opts = m.RouterOpts(w.score, w.renormalize)
-    ws = m.LayerWorkspace(w.T, w.H, w.I, w.E, w.k, w.shared_expert, backward=w.backward)
-    out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device="cuda")
-    state = None
-    grads = None
-    if w.backward:
-        _, state = m.moe_layer_forward(d["logits"], d["x"], d["w_gate_up"], d["w_down"], w.k, opts,
-                                       save_for_backward=True, workspace=ws, out=out)
-        grads = m.moe_grouped_mlp_backward(d["dout"], state, d["w_gate_up"], d["w_down"], ws)
-
-    nfev = 7
-    def step(fev=None, bev=None):
-        if fev:
-            m.moe_trace_set(fev)
-        m.moe_layer_forward(d["logits"], d["x"], d["w_gate_up"], d["w_down"], w.k, opts,
-                            d["shared_gate_up"], d["shared_down"], save_for_backward=w.backward,
-                            workspace=ws, out=out, state=state)
-        if w.backward:
-            if bev:
-                m.moe_trace_set(bev)
-            m.moe_grouped_mlp_backward(d["dout"], state, d["w_gate_up"], d["w_down"], ws, grads)
-        if fev or bev:
-            m.moe_trace_set(None)
+    layer = Layer(m, w, d)
 
     for _ in range(args.warmup):
-        step()
+        layer.step()
     torch.cuda.synchronize()
     if m.moe_get_device_status() != 0:
         raise RuntimeError("device status error after warm-up")
 
     K = args.steps
-    fevs = [[torch.cuda.Event(enable_timing=True) for _ in range(nfev)] for _ in range(K)]
-    bevs = [[torch.cuda.Event(enable_timing=True) for _ in range(nfev)] for _ in range(K)] if w.backward else [None] * K
-    for evs in fevs + ([e for e in bevs if e] if w.backward else []):
-        for e in evs:
-            e.record()           # materialise the events before handing them to the library
+    fevs = [_events(7) for _ in range(K)]
+    bevs = [_events(7) for _ in range(K)] if w.backward else [None] * K
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
@@ -351,7 +589,7 @@ def our_arm(args, world, rank, local):
     sampler.start()
     start.record()
     for i in range(K):
-        step(fevs[i], bevs[i])
+        layer.step(fevs[i], bevs[i])
     end.record()
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -360,17 +598,9 @@ def our_arm(args, world, rank, local):
     ms_max = max_over_ranks(ms, world)
     if m.moe_get_device_status() != 0:
         raise RuntimeError("device status error in the timed region")
+    stages = stage_medians(layer, fevs, bevs)
 
-    def stage_ms(evsets, i):
-        return statistics.mean(evs[i].elapsed_time(evs[i + 1]) for evs in evsets)
-    fwd_stages = ["router", "permute", "gate_up_swiglu", "down", "shared_expert", "combine"]
-    stages = {f"fwd_{n}": stage_ms(fevs, i) for i, n in enumerate(fwd_stages)}
-    if w.backward:
-        bwd_stages = ["combine_bwd", "down_dgrad_swiglu_bwd", "gate_up_dgrad", "dx_token_sum",
-                      "down_wgrad", "gate_up_wgrad"]
-        stages.update({f"bwd_{n}": stage_ms(bevs, i) for i, n in enumerate(bwd_stages)})
-
-    graph = None if args.no_graph else graph_measure(args, step, w, world, m)
+    graph = None if args.no_graph else graph_measure(args, layer.step, w, world, m)
 
     value = whole_job_value(w.T, world, K, ms_max)
     peaks, peaks_src = load_peaks()
@@ -381,63 +611,44 @@ def our_arm(args, world, rank, local):
     long_region = ms / 1e3 >= 0.25
     peak_tf = peaks["bf16_tflops_sustained" if long_region else "bf16_tflops"]
     burst_tf = peaks["bf16_tflops"]
-    A = w.A
-    gate_up_flop = 4.0 * A * w.H * w.I
+    gate_up_flop = 4.0 * w.A * w.H * w.I
     gate_up_ms = stages["fwd_gate_up_swiglu"]
     achieved = gate_up_flop / (gate_up_ms / 1e3) / 1e12
-    gemm_ms = stages["fwd_gate_up_swiglu"] + stages["fwd_down"] + (stages["fwd_shared_expert"] if w.shared_expert else 0.0)
-    gemm_flop = w.fwd_flops()
-    if w.backward:
-        gemm_ms += sum(stages[k] for k in ("bwd_down_dgrad_swiglu_bwd", "bwd_gate_up_dgrad",
-                                           "bwd_down_wgrad", "bwd_gate_up_wgrad"))
-        gemm_flop += w.bwd_flops()
-    gemm_tflops = gemm_flop / (gemm_ms / 1e3) / 1e12
-
-    # algorithmic bytes of the bandwidth-bound stages
+    gg = gemm_summary(w, stages, peaks)
+    gg["frac_of_peak"] = gg["tflops"] / peak_tf
+    gg["peak_tflops"] = peak_tf
     hbm = peaks["hbm_gbs"]
-    T, H, k, E = w.T, w.H, w.k, w.E
-    bw_bytes = {
-        "fwd_router": T * E * 4 + T * k * 8 + E * 8,
-        "fwd_permute": T * H * 2 + A * H * 2 + A * 4 + T * k * 4,
-        "fwd_combine": A * H * 2 + T * H * 2 + T * k * 8 + (T * H * 2 if w.shared_expert else 0),
-    }
-    if w.backward:
-        bw_bytes["bwd_combine_bwd"] = T * H * 2 + 2 * A * H * 2 + T * k * 12
-        bw_bytes["bwd_dx_token_sum"] = A * H * 2 + T * H * 2 + T * k * 4
-    bandwidth = {}
-    for key, nbytes in bw_bytes.items():
-        gbs = nbytes / (stages[key] / 1e3) / 1e9
-        bandwidth[key] = {"bytes": nbytes, "us": stages[key] * 1e3, "GB/s": gbs, "frac_of_hbm": gbs / hbm}
-
-    launches_fwd = 6 + (2 if w.shared_expert else 0)
-    launches = K * (launches_fwd + (6 if w.backward else 0))
+    flush = torch.ones(64 << 20, dtype=torch.float32, device="cuda")   # a 256 MB read evicts L2
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_max / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": config_dict(w, args),
-        "grouped_gemm": {"tflops": gemm_tflops, "frac_of_peak": gemm_tflops / peak_tf,
-                         "peak_tflops": peak_tf, "frac_of_burst_peak": gemm_tflops / burst_tf,
-                         "flop_per_step": gemm_flop,
-                         "note": "expert GEMM FLOPs (6AHI fwd, 12AHI bwd) / device time of the GEMM stages"},
-        "roofline": {"bound": "tensor", "kernel": "grouped_gemm_kernel<SwiGLU> (gate_up)",
+        "grouped_gemm": gg,
+        "roofline": {"bound": "tensor", "kernel": "gate_up + SwiGLU grouped GEMM (routed experts)",
                      "achieved": achieved, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": achieved / peak_tf, "frac_of_burst_peak": achieved / burst_tf,
+                     "frac_of_nominal_peak": achieved / NOMINAL_BF16_TFLOPS,
                      "traffic": traffic_for(f"gate_up_swiglu/{w.name}"),
                      "peak_source": f"{peaks_src} {'sustained' if long_region else 'burst'} bf16",
-                     "flop_per_launch": gate_up_flop, "ms_per_launch": gate_up_ms},
+                     "flop_per_launch": gate_up_flop, "ms_per_launch": gate_up_ms,
+                     "ms_per_launch_is": "median over the timed steps (CUDA events on the launching stream)"},
         "stages_ms": stages,
-        "bandwidth_kernels": bandwidth,
+        "bandwidth_kernels": bandwidth_report(layer, stages, hbm, flush),
         "hbm_peak_gbs": hbm,
-        "gpu_launches": launches,
+        "gpu_launches": K * layer.launches(),
         "clocks": clocks,
     }
 
     if graph:
         line["cuda_graph"] = graph
     if not args.no_e2e:
-        line["e2e"] = e2e_measure(args, w, d, m, opts, ws, world)
+        line["e2e"] = e2e_measure(args, w, d, m, layer.opts, layer.ws, world)
+    if world == 1 and not args.no_extra and args.T is None:
+        del layer
+        torch.cuda.empty_cache()
+        line["workloads"] = {n: workload_entry(m, n, peaks, flush) for n in EXTRA_WORKLOADS if n != w.name}
     if args.router_sweep:
         line["router_sweep"] = router_sweep(m, hbm)
     if args.gather_compare:
@@ -545,7 +756,8 @@ def gather_compare(m):
     E=128, k=8), no saved state, L2-flushed before each call: the permute
     writes x_perm and the gate_up GEMM loads it with TMA tiles, against the
     permute computing only the rows and the GEMM gathering its A rows from x
-    (MOE_GATHER=1). The outputs are bit-identical (tested)."""
+    (the folded permute of moe_testing_set_kernels). The outputs are
+    bit-identical (tested)."""
     import torch
     import workloads as wl
     w = wl.WORKLOADS["qwen3_30b_a3b"]
@@ -553,8 +765,8 @@ def gather_compare(m):
     opts = m.RouterOpts(w.score, w.renormalize)
     flush = torch.ones(64 << 20, dtype=torch.float32, device="cuda")
     res = {"workload": "qwen3_30b_a3b forward, no saved state"}
-    for name, env in (("x_perm_us", "0"), ("gather_us", "1")):
-        os.environ["MOE_GATHER"] = env
+    for name, fold in (("x_perm_us", 0), ("gather_us", 1)):
+        m.moe_testing_set_kernels(fold_permute=fold)
         times = []
         for it in range(12):
             flush.sum()
@@ -567,7 +779,7 @@ def gather_compare(m):
             if it >= 2:
                 times.append(s.elapsed_time(e) * 1e3)
         res[name] = statistics.median(times)
-    os.environ.pop("MOE_GATHER", None)
+    m.moe_testing_set_kernels()
     if m.moe_get_device_status() != 0:
         raise RuntimeError("device status after the gather comparison")
     return res
