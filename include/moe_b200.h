@@ -27,8 +27,9 @@
  *    expert index outside [0,E), inconsistent offsets, a wait that timed out)
  *    in a device-side error word, and skip the offending row instead of
  *    trapping. moe_get_device_status reads and clears that word.
- *  - Limits. 1 <= E <= 256; 1 <= k <= min(E, 16); H and I are multiples of 64;
- *    T * k < 2^31.
+ *  - Limits. 1 <= E <= 256; 1 <= k <= min(E, 16); H and I are multiples of 8
+ *    (rows of 16 bytes: the stride rule of the tensor-memory-access maps and of
+ *    the 16-byte vector loads); T * k < 2^31.
  *  - Dropless routing. A = T * k routed rows, a static size: buffers never
  *    depend on the routing, so no device-to-host copy is needed (TE Token
  *    dispatch: num_out_tokens known statically).

@@ -65,6 +65,8 @@ __global__ void __launch_bounds__(kWarpKernelThreads, KB > 8 ? 2 : 4)
                                  const int32_t* __restrict__ row_of, const float* __restrict__ probs,
                                  int64_t T, int k, int H8, int64_t A, uint4* __restrict__ dy,
                                  float* __restrict__ dprob, unsigned* err) {
+    pdl_wait();
+    pdl_launch_dependents();
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -143,6 +145,8 @@ __global__ void __launch_bounds__(kWarpKernelThreads, KB > 8 ? 2 : 4)
     combine_warp_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ row_of,
                         const float* __restrict__ probs, int64_t T, int k, int H8, int64_t A,
                         const uint4* __restrict__ shared, uint4* __restrict__ out, unsigned* err) {
+    pdl_wait();
+    pdl_launch_dependents();
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -226,10 +230,9 @@ cudaError_t launch_combine(const bf16* y_perm, const int32_t* row_of, const floa
               : k <= 4 ? combine_warp_kernel<4, 2>
               : k <= 8 ? combine_warp_kernel<8, 2> : combine_warp_kernel<16, 1>;
     const int64_t blocks = warp_kernel_blocks(kern, T);
-    kern<<<(unsigned)blocks, kWarpKernelThreads, 0, st>>>(reinterpret_cast<const uint4*>(y_perm), row_of, probs, T,
-                                                         k, H / 8, A, reinterpret_cast<const uint4*>(shared),
-                                                         reinterpret_cast<uint4*>(out), err);
-    return cudaGetLastError();
+    return launch_chained(kern, dim3((unsigned)blocks), dim3(kWarpKernelThreads), 0, st,
+                          reinterpret_cast<const uint4*>(y_perm), row_of, probs, T, k, H / 8, A,
+                          reinterpret_cast<const uint4*>(shared), reinterpret_cast<uint4*>(out), err);
 }
 
 cudaError_t launch_combine_backward(const bf16* dout, const bf16* y_perm, const int32_t* row_of,
@@ -240,10 +243,9 @@ cudaError_t launch_combine_backward(const bf16* dout, const bf16* y_perm, const 
               : k <= 4 ? combine_backward_warp_kernel<4, 2>
               : k <= 8 ? combine_backward_warp_kernel<8, 2> : combine_backward_warp_kernel<16, 1>;
     const int64_t blocks = warp_kernel_blocks(kern, T);
-    kern<<<(unsigned)blocks, kWarpKernelThreads, 0, st>>>(
-        reinterpret_cast<const uint4*>(dout), reinterpret_cast<const uint4*>(y_perm), row_of, probs,
-        T, k, H / 8, A, reinterpret_cast<uint4*>(dy_perm), dprob, err);
-    return cudaGetLastError();
+    return launch_chained(kern, dim3((unsigned)blocks), dim3(kWarpKernelThreads), 0, st,
+                          reinterpret_cast<const uint4*>(dout), reinterpret_cast<const uint4*>(y_perm), row_of,
+                          probs, T, k, H / 8, A, reinterpret_cast<uint4*>(dy_perm), dprob, err);
 }
 
 }  // namespace moe

@@ -9,7 +9,7 @@
 // (_expert_ffn) and torchtitan GroupedExperts: silu(x Wg) * (x Wu).
 //
 // Three kernels share the schedule. The forward and dgrad GEMMs run on pair
-// tiles when the average expert block is large (>= 512 rows, or a single dense
+// tiles when the average expert block is large (>= 1024 rows, or a single dense
 // group), else on single-CTA 128-row tiles, which round ragged blocks up less
 // (use_pair_tiles); the forward GEMMs of small batches (<= 16 rows per expert
 // on average) run on swap-AB tiles (gemm_swap_kernel, use_swap_tiles).
@@ -285,7 +285,7 @@ __device__ __forceinline__ uint32_t stage64_off(int r, int q) {
 // padded by 16 bytes, so neither phase has more than 2-way bank conflicts.
 // Warp-collective.
 template <int NC>
-__device__ __forceinline__ void store_rows(uint8_t* buf, bf16* dst, int64_t ld, int nvalid,
+__device__ __forceinline__ void store_rows(uint8_t* buf, bf16* dst, int64_t ld, int nvalid, int ncols,
                                            const float* v, int lane) {
     constexpr int kChunks = NC / 8;              // 16-byte chunks per row
     constexpr int kRowsPerPass = 32 / kChunks;   // rows one instruction covers
@@ -301,7 +301,7 @@ __device__ __forceinline__ void store_rows(uint8_t* buf, bf16* dst, int64_t ld, 
     for (int pass = 0; pass < kChunks; ++pass) {
         const int row = pass * kRowsPerPass + lane / kChunks;
         const uint4 w = *reinterpret_cast<const uint4*>(buf + row * kPitch + chunk * 16);
-        if (row < nvalid) *reinterpret_cast<uint4*>(dst + (int64_t)row * ld + chunk * 8) = w;
+        if (row < nvalid && chunk * 8 < ncols) *reinterpret_cast<uint4*>(dst + (int64_t)row * ld + chunk * 8) = w;
     }
     __syncwarp();   // the buffer is free again
 }
@@ -311,13 +311,13 @@ __device__ __forceinline__ void store_rows(uint8_t* buf, bf16* dst, int64_t ld, 
 // TMA store (x, y = its first column and row in the map); otherwise through
 // store_rows, which masks rows >= nvalid. The buffer is reused only after the
 // previous TMA store has read it.
-__device__ __forceinline__ void put_block32(uint8_t* buf, bf16* dst, int64_t ld, int nvalid, const float* v,
-                                            int lane, const CUtensorMap* map, int x, int y) {
+__device__ __forceinline__ void put_block32(uint8_t* buf, bf16* dst, int64_t ld, int nvalid, int ncols,
+                                            const float* v, int lane, const CUtensorMap* map, int x, int y) {
     if (map != nullptr) {
         if (lane == 0) bulk_wait_group_read0();
         __syncwarp();
     }
-    if (map != nullptr && nvalid == 32) {
+    if (map != nullptr && nvalid == 32 && ncols == 32) {
 #pragma unroll
         for (int q = 0; q < 4; ++q)
             *reinterpret_cast<uint4*>(buf + stage64_off(lane, q)) =
@@ -331,7 +331,7 @@ __device__ __forceinline__ void put_block32(uint8_t* buf, bf16* dst, int64_t ld,
         }
         __syncwarp();
     } else {
-        store_rows<32>(buf, dst, ld, nvalid, v, lane);
+        store_rows<32>(buf, dst, ld, nvalid, ncols, v, lane);
     }
 }
 
@@ -349,13 +349,14 @@ __device__ __forceinline__ void load_aux32(const Params& p, int64_t grow, int co
     const uint4* us = reinterpret_cast<const uint4*>(p.aux + grow * p.ld_aux + p.I + col);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        a.g[q] = __ldg(gs + q);
-        a.u[q] = __ldg(us + q);
+        const bool in = col + 8 * q < p.I;   // columns past I are not read (they are not stored either)
+        a.g[q] = in ? __ldg(gs + q) : make_uint4(0, 0, 0, 0);
+        a.u[q] = in ? __ldg(us + q) : make_uint4(0, 0, 0, 0);
     }
 }
 
 // store_rows<32> for values already packed as bf16 pairs (16 per lane).
-__device__ __forceinline__ void store_rows_packed32(uint8_t* buf, bf16* dst, int64_t ld, int nvalid,
+__device__ __forceinline__ void store_rows_packed32(uint8_t* buf, bf16* dst, int64_t ld, int nvalid, int ncols,
                                                     const uint32_t* w, int lane) {
     constexpr int kPitch = 32 * 2 + 16;
 #pragma unroll
@@ -367,20 +368,20 @@ __device__ __forceinline__ void store_rows_packed32(uint8_t* buf, bf16* dst, int
     for (int pass = 0; pass < 4; ++pass) {
         const int row = pass * 8 + lane / 4;
         const uint4 v = *reinterpret_cast<const uint4*>(buf + row * kPitch + chunk * 16);
-        if (row < nvalid) *reinterpret_cast<uint4*>(dst + (int64_t)row * ld + chunk * 8) = v;
+        if (row < nvalid && chunk * 8 < ncols) *reinterpret_cast<uint4*>(dst + (int64_t)row * ld + chunk * 8) = v;
     }
     __syncwarp();
 }
 
 // put_block32 for values already packed as bf16 pairs.
-__device__ __forceinline__ void put_block32_packed(uint8_t* buf, bf16* dst, int64_t ld, int nvalid,
+__device__ __forceinline__ void put_block32_packed(uint8_t* buf, bf16* dst, int64_t ld, int nvalid, int ncols,
                                                    const uint32_t* w, int lane, const CUtensorMap* map, int x,
                                                    int y) {
     if (map != nullptr) {
         if (lane == 0) bulk_wait_group_read0();
         __syncwarp();
     }
-    if (map != nullptr && nvalid == 32) {
+    if (map != nullptr && nvalid == 32 && ncols == 32) {
 #pragma unroll
         for (int q = 0; q < 4; ++q)
             *reinterpret_cast<uint4*>(buf + stage64_off(lane, q)) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
@@ -392,7 +393,7 @@ __device__ __forceinline__ void put_block32_packed(uint8_t* buf, bf16* dst, int6
         }
         __syncwarp();
     } else {
-        store_rows_packed32(buf, dst, ld, nvalid, w, lane);
+        store_rows_packed32(buf, dst, ld, nvalid, ncols, w, lane);
     }
 }
 
@@ -476,15 +477,18 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
             float g[32], u[32];
             tmem_load_2x32(tc, tc + (uint32_t)em.up, g, u);
             if (n0 + c0 >= p.N) continue;
+            // columns of the chunk inside the output (a multiple of 8): a partial chunk takes
+            // masked row stores, since a TMA store of the g part would spill into the u columns
+            const int ncols = min(32, p.N - (n0 + c0));
             if (p.out2) {
-                put_block32(buf, p.out2 + row0 * p.ldo2 + n0 + c0, p.ldo2, nvalid, g, lane, tmC2, n0 + c0,
+                put_block32(buf, p.out2 + row0 * p.ldo2 + n0 + c0, p.ldo2, nvalid, ncols, g, lane, tmC2, n0 + c0,
                             (int)row0);
-                put_block32(buf, p.out2 + row0 * p.ldo2 + p.I + n0 + c0, p.ldo2, nvalid, u, lane, tmC2,
+                put_block32(buf, p.out2 + row0 * p.ldo2 + p.I + n0 + c0, p.ldo2, nvalid, ncols, u, lane, tmC2,
                             p.I + n0 + c0, (int)row0);
             }
 #pragma unroll
             for (int i = 0; i < 32; ++i) g[i] = silu_f(g[i]) * u[i] * rs;     // h, in place
-            put_block32(buf, p.out + row0 * p.ldo + n0 + c0, p.ldo, nvalid, g, lane, tmC, n0 + c0, (int)row0);
+            put_block32(buf, p.out + row0 * p.ldo + n0 + c0, p.ldo, nvalid, ncols, g, lane, tmC, n0 + c0, (int)row0);
         }
     } else if (EPI == kEpiSwigluBwd) {
         // the first chunk's g and u were loaded before the accumulator was
@@ -501,6 +505,7 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
             float dh[32];
             tmem_load_32(t_row + (uint32_t)(em.tm + 32 * ci), dh);
             if (col >= p.N) continue;
+            const int ncols = min(32, p.N - col);
             uint32_t dgp[16], dup[16];
             if (valid) {
                 swiglu_bwd32(dh, ax, dgp, dup);
@@ -510,8 +515,9 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
             }
             // the next chunk's g and u load while this chunk is stored
             load_aux32(p, grow, col + 32, valid && ci + 1 < em.chunks && col + 32 < p.N, ax);
-            put_block32_packed(buf, p.out + row0 * p.ldo + col, p.ldo, nvalid, dgp, lane, tmC, col, (int)row0);
-            put_block32_packed(buf, p.out + row0 * p.ldo + p.I + col, p.ldo, nvalid, dup, lane, tmC, p.I + col,
+            put_block32_packed(buf, p.out + row0 * p.ldo + col, p.ldo, nvalid, ncols, dgp, lane, tmC, col,
+                               (int)row0);
+            put_block32_packed(buf, p.out + row0 * p.ldo + p.I + col, p.ldo, nvalid, ncols, dup, lane, tmC, p.I + col,
                                (int)row0);
         }
     } else if (GROUP_K) {
@@ -571,7 +577,8 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 if (n0 + c0 + 32 * half >= p.N) continue;
-                put_block32(buf, row0 + n0 + c0 + 32 * half, p.ldo, nvalid, v + 32 * half, lane,
+                put_block32(buf, row0 + n0 + c0 + 32 * half, p.ldo, nvalid, min(32, p.N - (n0 + c0 + 32 * half)),
+                            v + 32 * half, lane,
                             GROUP_K ? nullptr : tmC, n0 + c0 + 32 * half, t.row0 + warp_r0);
             }
         }
@@ -593,7 +600,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int cluster = blockIdx.x >> 1, clusters = gridDim.x >> 1;
     volatile int* abort_flag = &s.abort;
 
-    build_schedule<false>(s, p, BMP);
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGESP; ++i) {
             mbar_init(&s.full[i], 1);
@@ -614,6 +620,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc_pair(&s.tmem_base, kTmemCols);
         tmem_relinquish_pair();
     }
+    pdl_wait();                // the previous kernel's outputs (A, offsets) are complete
+    build_schedule<false>(s, p, BMP);
     tc_fence_before();
     cluster_sync_all();        // barriers of both CTAs initialised, TMEM allocated
     tc_fence_after();
@@ -750,6 +758,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     }
 
+    // Every role has left its loop: the next kernel of the call may be scheduled
+    // (not earlier, so that its blocks do not sit beside this kernel's CTAs).
+    pdl_launch_dependents();
     tc_fence_before();
     cluster_sync_all();        // no MMA, load or remote arrival of either CTA is still pending
     if (warp == 1) {
@@ -770,7 +781,6 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int* abort_flag = &s.abort;
 
-    build_schedule<GROUP_K>(s, p, BM1);
     const bool gather = !GROUP_K && p.gather_tok != nullptr;
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES1; ++i) {
@@ -792,6 +802,8 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
         tmem_alloc(&s.tmem_base, kTmemCols);
         tmem_relinquish();
     }
+    pdl_wait();                // the previous kernel's outputs (A, B, offsets) are complete
+    build_schedule<GROUP_K>(s, p, BM1);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1069,6 +1081,7 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
         }
     }
 
+    pdl_launch_dependents();   // every role has left its loop (see gemm_pair_kernel)
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -1139,7 +1152,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int* abort_flag = &s.abort;
 
-    build_schedule<false>(s, p, BNS);
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGESS; ++i) {
             mbar_init(&s.full[i], 1);
@@ -1160,6 +1172,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc(&s.tmem_base, kTmemColsS);
         tmem_relinquish();
     }
+    pdl_wait();                // the previous kernel's outputs (token rows, offsets) are complete
+    build_schedule<false>(s, p, BNS);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1279,7 +1293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int64_t r0 = (int64_t)t.row0 + j0;
 #pragma unroll
                         for (int i = 0; i < 32; ++i) {
-                            if (i >= nvalid) break;
+                            if (i >= nvalid || hc >= p.N) break;
                             const float g = v[i], u = urow[i];
                             const float rs = p.row_scale ? __ldg(p.row_scale + r0 + i) : 1.0f;
                             if (p.out2) {
@@ -1308,6 +1322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
 
+    pdl_launch_dependents();   // every role has left its loop (see gemm_pair_kernel)
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -1386,13 +1401,15 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& a64, const CUte
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kSmemPBytes;
     cfg.stream = st;
-    cudaLaunchAttribute attrs[1];
+    cudaLaunchAttribute attrs[2];
     attrs[0].id = cudaLaunchAttributeClusterDimension;
     attrs[0].val.clusterDim.x = 2;
     attrs[0].val.clusterDim.y = 1;
     attrs[0].val.clusterDim.z = 1;
+    attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see launch_chained
+    attrs[1].val.programmaticStreamSerializationAllowed = chained_launches() ? 1 : 0;
     cfg.attrs = attrs;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     CUtensorMap unused{};   // read only when q.tma_out / q.tma_out2 say so
     Params q = p;
     q.tma_out = c != nullptr;
@@ -1415,9 +1432,8 @@ cudaError_t launch_1cta(const CUtensorMap& a, const CUtensorMap& b, const Params
     Params q = p;
     q.tma_out = c != nullptr;
     q.tma_out2 = c2 != nullptr;
-    kern<<<(unsigned)grid, GROUP_K ? kThreadsK : kThreads, kSmem1Bytes, st>>>(a, b, c ? *c : unused,
-                                                                            c2 ? *c2 : unused, q);
-    return cudaGetLastError();
+    return launch_chained(kern, dim3((unsigned)grid), dim3(GROUP_K ? kThreadsK : kThreads), kSmem1Bytes, st, a, b,
+                          c ? *c : unused, c2 ? *c2 : unused, q);
 }
 
 Params base_params(int groups, int64_t rows, const int32_t* offsets, unsigned* err) {
@@ -1440,16 +1456,18 @@ int64_t single_tile_bound(int64_t rows, int groups, int n_blocks) {
 
 // Pair tiles (256 rows) halve each CTA's weight traffic; an expert block's
 // last <= 128 rows run as a 128-row pair tile, so both kinds round a block up
-// to a multiple of 128 rows. Measured on B200, pair tiles were faster at 1024
-// rows per expert (Mixtral-8x7B shape: gate_up 1675 against 1777 us) and at 512
-// (Llama-4-17Bx16E shape: 1377 against 1470 us), and slower at 256
-// (Qwen3-30B-A3B shape: 321 against 286 us). moe_testing_set_kernels can force
-// either kind (the tests run both kernels on the same shapes).
+// to a multiple of 128 rows. Measured on B200 with the two kinds interleaved
+// call by call: pair tiles are faster at 1024 rows per expert (Mixtral-8x7B
+// shape) and for one dense group (the Llama-4 shared expert: 1595 against
+// 1727 us), equal at 512 (Llama-4-17Bx16E routed gate_up: 1339 against
+// 1326 us), and slower at 256 (Qwen3-30B-A3B shape: 321 against 286 us).
+// moe_testing_set_kernels can force either kind (the tests run both kernels
+// on the same shapes).
 bool use_pair_tiles(int64_t rows, int groups) {
     const int forced = kernel_override().gemm_tiles;
     if (forced == MOE_TESTING_GEMM_PAIR) return true;
-    if (forced == MOE_TESTING_GEMM_SINGLE || forced == MOE_TESTING_GEMM_SWAP) return false;
-    return groups == 1 || rows >= (int64_t)groups * 512;
+    if (forced != MOE_TESTING_AUTO) return false;
+    return groups == 1 || rows >= (int64_t)groups * 1024;
 }
 
 // The forward GEMMs take swap-AB tiles (weights as the 128-row operand, 64
@@ -1473,8 +1491,7 @@ cudaError_t launch_swap(const CUtensorMap& x64, const CUtensorMap& w, const Para
     if (bound <= 0) return cudaSuccess;
     int64_t grid = sm_count();
     if (grid > bound) grid = bound;
-    kern<<<(unsigned)grid, kThreads, kSmemSBytes, st>>>(x64, w, p);
-    return cudaGetLastError();
+    return launch_chained(kern, dim3((unsigned)grid), dim3(kThreads), kSmemSBytes, st, x64, w, p);
 }
 
 // Group-M GEMM on pair or single tiles. `ta` and `ta64` are A maps with
@@ -1521,7 +1538,7 @@ cudaError_t gemm_gate_up_swiglu(const bf16* x, int64_t rows, const int32_t* offs
     p.ldo2 = 2 * (int64_t)I;
     p.row_scale = row_scale;
     if (use_swap_tiles(rows, groups)) {
-        p.n_blocks = I / 64;   // 64 gate and the matching 64 up columns per tile
+        p.n_blocks = (I + 63) / 64;   // 64 gate and the matching 64 up columns per tile
         return launch_swap<kEpiSwiglu>(ta64, tb, p, st);
     }
     CUtensorMap tc, tc2;

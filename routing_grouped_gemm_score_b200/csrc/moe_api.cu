@@ -75,7 +75,10 @@ bool shape_ok(int64_t T, int E, int k) {
            T * (int64_t)k < (int64_t(1) << 31);
 }
 
-bool dims_ok(int H, int I) { return H > 0 && I > 0 && H % 64 == 0 && I % 64 == 0; }
+// H and I multiples of 8: 16-byte rows, the stride rule of the TMA maps and of
+// the 16-byte vector loads and stores (pytorch/ao pull request 2600, the
+// alignment of grouped-GEMM operands).
+bool dims_ok(int H, int I) { return H > 0 && I > 0 && H % 8 == 0 && I % 8 == 0; }
 
 moe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
@@ -155,6 +158,11 @@ int sm_count() {
 }
 
 KernelOverride g_override;
+
+bool& chained_launches() {
+    thread_local bool on = false;
+    return on;
+}
 
 // One thread waits, with the given limit, on an mbarrier that nothing arrives
 // on: the bounded wait of the GEMM kernels (mbar_wait_limit) running out.
@@ -247,6 +255,7 @@ moe_status moe_router_topk(const float* logits, int64_t T, int E, int k,
                            const moe_router_opts* opts_in, int32_t* topk_idx, float* topk_prob,
                            uint8_t* routing_map, int32_t* counts, int32_t* offsets,
                            void* workspace, size_t workspace_bytes, void* stream) {
+    const ChainScope chain(T * (int64_t)k <= kChainMaxRows);
     if (!shape_ok(T, E, k)) return MOE_ERR_INVALID_ARG;
     const moe_router_opts opts = opts_in ? *opts_in : default_opts();
     if (check_opts(opts) != MOE_OK) return MOE_ERR_INVALID_ARG;
@@ -331,6 +340,7 @@ moe_status moe_router_topk_noalloc(const float* logits, int64_t T, int E, int k,
                                    const moe_router_opts* opts_in, int32_t* topk_idx,
                                    float* topk_prob, uint8_t* routing_map, int32_t* counts,
                                    int32_t* offsets, void* stream) {
+    const ChainScope chain(T * (int64_t)k <= kChainMaxRows);
     if (!shape_ok(T, E, k)) return MOE_ERR_INVALID_ARG;
     const moe_router_opts opts = opts_in ? *opts_in : default_opts();
     if (check_opts(opts) != MOE_OK) return MOE_ERR_INVALID_ARG;
@@ -369,6 +379,7 @@ size_t moe_permute_workspace_size(int64_t T, int E, int k) {
 moe_status moe_permute(const moe_bf16* x, int64_t T, int H, const int32_t* topk_idx, int k,
                        const int32_t* offsets, int E, moe_bf16* x_perm, int32_t* sorted_token,
                        int32_t* row_of, void* workspace, size_t workspace_bytes, void* stream) {
+    const ChainScope chain(T * (int64_t)k <= kChainMaxRows);
     if (!shape_ok(T, E, k) || H <= 0 || H % 8 != 0) return MOE_ERR_INVALID_ARG;
     if (T == 0) return MOE_OK;
     if (!x || !topk_idx || !offsets || !x_perm || !sorted_token || !row_of) return MOE_ERR_INVALID_ARG;
@@ -399,6 +410,7 @@ moe_status moe_permute_padded(const moe_bf16* x, int64_t T, int H, const int32_t
                               int32_t* padded_offsets, moe_bf16* x_perm, float* prob_perm,
                               int32_t* sorted_token, int32_t* row_of, void* workspace,
                               size_t workspace_bytes, void* stream) {
+    const ChainScope chain(T * (int64_t)k <= kChainMaxRows);
     if (!shape_ok(T, E, k) || H <= 0 || H % 8 != 0) return MOE_ERR_INVALID_ARG;
     if (moe_permute_padded_max_rows(T, E, k, align) <= 0 && T > 0) return MOE_ERR_INVALID_ARG;
     if (align < 1 || align > 65536 || !offsets || !padded_offsets || !aligned16(offsets) ||
@@ -447,6 +459,7 @@ moe_status moe_grouped_mlp_scaled(const moe_bf16* x_perm, int64_t A, const int32
                                   int H, int I, const moe_bf16* w_gate_up, const moe_bf16* w_down,
                                   const float* row_scale, moe_bf16* y_perm, moe_bf16* gu_save,
                                   moe_bf16* h_save, void* workspace, size_t workspace_bytes, void* stream) {
+    const ChainScope chain(A <= kChainMaxRows);
     if (row_scale && !aligned16(row_scale)) return MOE_ERR_INVALID_ARG;
     if (A < 0 || A >= (int64_t(1) << 31) || E < 1 || E > 256) return MOE_ERR_INVALID_ARG;
     if (H <= 0 || I <= 0) return MOE_ERR_INVALID_ARG;
@@ -484,6 +497,7 @@ moe_status moe_unpermute_combine(const moe_bf16* y_perm, const int32_t* row_of,
 moe_status moe_unpermute_combine_rows(const moe_bf16* y_perm, int64_t y_rows, const int32_t* row_of,
                                       const float* topk_prob, int64_t T, int k, int H,
                                       const moe_bf16* shared_out, moe_bf16* out, void* stream) {
+    const ChainScope chain(T * (int64_t)k <= kChainMaxRows);
     if (T < 0 || k < 1 || k > 16 || H <= 0 || H % 8 != 0 || T * (int64_t)k >= (int64_t(1) << 31))
         return MOE_ERR_INVALID_ARG;
     if (y_rows < 0 || y_rows >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;
@@ -513,6 +527,7 @@ moe_status moe_layer_forward(const float* logits, const moe_bf16* x, int64_t T, 
                              int32_t* offsets, int32_t* row_of, moe_bf16* x_perm, moe_bf16* gu,
                              moe_bf16* h, moe_bf16* y_perm, void* workspace,
                              size_t workspace_bytes, void* stream) {
+    const ChainScope chain(T * (int64_t)k <= kChainMaxRows);
     if (!shape_ok(T, E, k) || H <= 0 || I <= 0) return MOE_ERR_INVALID_ARG;
     if (!dims_ok(H, I)) return MOE_ERR_UNSUPPORTED;
     const moe_router_opts opts = opts_in ? *opts_in : default_opts();
@@ -608,6 +623,7 @@ moe_status moe_grouped_mlp_backward(const moe_bf16* dout, int64_t T, int H, int 
                                     moe_bf16* dx, moe_bf16* dw_gate_up, moe_bf16* dw_down,
                                     float* dprob, void* workspace, size_t workspace_bytes,
                                     void* stream) {
+    const ChainScope chain(T * (int64_t)k <= kChainMaxRows);
     if (!shape_ok(T, E, k) || H <= 0 || I <= 0) return MOE_ERR_INVALID_ARG;
     if (!dims_ok(H, I)) return MOE_ERR_UNSUPPORTED;
     const void* must[] = {dout, w_gate_up, w_down, row_of, topk_prob, offsets, x_perm, gu, h,

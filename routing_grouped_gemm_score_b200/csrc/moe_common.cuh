@@ -29,6 +29,16 @@ __device__ __forceinline__ unsigned long long global_timer_ns() {
     return t;
 }
 
+// Programmatic dependent launch. The kernels of a layer call are launched
+// with programmatic stream serialization, so a kernel can be scheduled, and
+// run its prologue, while the kernel before it in the stream finishes.
+// pdl_wait() blocks until that kernel has completed and its writes are
+// visible; each such kernel calls it before its first access to global memory
+// that another kernel writes or reads. Without a programmatic dependency it
+// returns at once. pdl_launch_dependents() lets the next kernel be scheduled.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void raise_error(unsigned* err, unsigned bit) {
     if (err) atomicOr(err, bit);
 }

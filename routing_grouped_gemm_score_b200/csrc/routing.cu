@@ -126,6 +126,8 @@ __global__ void __launch_bounds__(kRouteThreads) router_topk_kernel(const Router
     const int E = a.E, k = KC ? KC : a.k, tpb = a.tpb;
     for (int i = threadIdx.x; i < tpb * 256 / 16; i += blockDim.x)
         reinterpret_cast<uint4*>(&sel[0][0])[i] = make_uint4(0, 0, 0, 0);
+    pdl_wait();
+    pdl_launch_dependents();
     if (blockIdx.x == 0 && threadIdx.x == 0) *a.ticket = 0u;
     __syncthreads();
     const int64_t t0 = (int64_t)blockIdx.x * tpb;
@@ -480,6 +482,8 @@ __global__ void __launch_bounds__(kLaneTokens, 3)
     const int64_t t0 = (int64_t)blockIdx.x * kLaneTokens;
     const int64_t t = t0 + threadIdx.x;
     const bool live = t < a.T;
+    pdl_wait();
+    pdl_launch_dependents();
     if (blockIdx.x == 0 && threadIdx.x == 0) *a.ticket = 0u;
     for (int i = threadIdx.x; i < E * (kLaneTokens / 32); i += blockDim.x) (&mask[0][0])[i] = 0u;
 
@@ -858,6 +862,8 @@ __device__ __forceinline__ int scan_slot(int i) { return (i / kScanPerThread) * 
 __global__ void __launch_bounds__(1024)
     expert_scan_kernel(int32_t* block_base, int nb, int E, int32_t* counts, int32_t* offsets,
                        unsigned* ticket) {
+    pdl_wait();
+    pdl_launch_dependents();
     __shared__ int warp_tot[32];
     __shared__ bool is_last;
     int carry_off = 0;
@@ -936,6 +942,8 @@ __global__ void __launch_bounds__(512)
                           int32_t* __restrict__ sorted_token, int32_t* __restrict__ row_of, int64_t A,
                           int64_t per_block, unsigned* err) {
     __shared__ int32_t s_row[kPermStage];
+    pdl_wait();
+    pdl_launch_dependents();
     const int64_t t_begin = (int64_t)blockIdx.x * per_block;
     const int64_t t_end = t_begin + per_block < T ? t_begin + per_block : T;
     const int c = threadIdx.x;
@@ -994,6 +1002,8 @@ __global__ void __launch_bounds__(256)
                         int32_t* __restrict__ sorted_token, int32_t* __restrict__ row_of, int64_t A,
                         unsigned* err) {
     __shared__ int32_t s_off[kPermMaxExperts + 1];
+    pdl_wait();
+    pdl_launch_dependents();
     for (int e = threadIdx.x; e <= E; e += blockDim.x) s_off[e] = __ldg(offsets + e);
     __syncthreads();
     const int lane = threadIdx.x & 31;
@@ -1160,14 +1170,14 @@ RouteScratch carve_route_scratch(void* base, int64_t T, int E, int k) {
 }
 
 template <int SLOTS>
-void launch_router_k(const RouterArgs& a, dim3 grid, dim3 block, cudaStream_t st) {
+cudaError_t launch_router_k(const RouterArgs& a, dim3 grid, dim3 block, cudaStream_t st) {
     switch (a.k) {
-        case 1: router_topk_kernel<SLOTS, 1><<<grid, block, 0, st>>>(a); break;
-        case 2: router_topk_kernel<SLOTS, 2><<<grid, block, 0, st>>>(a); break;
-        case 4: router_topk_kernel<SLOTS, 4><<<grid, block, 0, st>>>(a); break;
-        case 6: router_topk_kernel<SLOTS, 6><<<grid, block, 0, st>>>(a); break;
-        case 8: router_topk_kernel<SLOTS, 8><<<grid, block, 0, st>>>(a); break;
-        default: router_topk_kernel<SLOTS, 0><<<grid, block, 0, st>>>(a); break;
+        case 1: return launch_chained(router_topk_kernel<SLOTS, 1>, grid, block, 0, st, a);
+        case 2: return launch_chained(router_topk_kernel<SLOTS, 2>, grid, block, 0, st, a);
+        case 4: return launch_chained(router_topk_kernel<SLOTS, 4>, grid, block, 0, st, a);
+        case 6: return launch_chained(router_topk_kernel<SLOTS, 6>, grid, block, 0, st, a);
+        case 8: return launch_chained(router_topk_kernel<SLOTS, 8>, grid, block, 0, st, a);
+        default: return launch_chained(router_topk_kernel<SLOTS, 0>, grid, block, 0, st, a);
     }
 }
 
@@ -1203,9 +1213,10 @@ cudaError_t launch_router_topk(const float* logits, int64_t T, int E, int k,
     if (use_lane) {
         const dim3 lgrid((unsigned)((T + kLaneTokens - 1) / kLaneTokens)), lblock(kLaneTokens);
         const bool bias = opts.expert_bias != nullptr;
-#define MOE_LANE(KC)                                                \
-    if (bias) router_lane_kernel<KC, true><<<lgrid, lblock, 0, st>>>(a); \
-    else router_lane_kernel<KC, false><<<lgrid, lblock, 0, st>>>(a)
+        cudaError_t e = cudaSuccess;
+#define MOE_LANE(KC)                                                                    \
+    e = bias ? launch_chained(router_lane_kernel<KC, true>, lgrid, lblock, 0, st, a)    \
+             : launch_chained(router_lane_kernel<KC, false>, lgrid, lblock, 0, st, a)
         switch (k) {
             case 1: MOE_LANE(1); break;
             case 2: MOE_LANE(2); break;
@@ -1218,15 +1229,14 @@ cudaError_t launch_router_topk(const float* logits, int64_t T, int E, int k,
         }
 #undef MOE_LANE
         (void)err;
-        return cudaGetLastError();
+        return e;
     }
     const dim3 grid((unsigned)a.nb), block(kRouteThreads);
-    if (E <= 32) launch_router_k<1>(a, grid, block, st);
-    else if (E <= 64) launch_router_k<2>(a, grid, block, st);
-    else if (E <= 128) launch_router_k<4>(a, grid, block, st);
-    else launch_router_k<8>(a, grid, block, st);
     (void)err;
-    return cudaGetLastError();
+    if (E <= 32) return launch_router_k<1>(a, grid, block, st);
+    if (E <= 64) return launch_router_k<2>(a, grid, block, st);
+    if (E <= 128) return launch_router_k<4>(a, grid, block, st);
+    return launch_router_k<8>(a, grid, block, st);
 }
 
 cudaError_t launch_router_backward(const float* logits, int64_t T, int E, int k, const moe_router_opts& opts,
@@ -1268,8 +1278,8 @@ cudaError_t launch_expert_scan(int64_t T, int E, const RouteScratch& rs, int32_t
     const int nb = (int)route_blocks(T);
     int threads = 32;
     while (threads * kScanPerThread < nb && threads < 1024) threads <<= 1;
-    expert_scan_kernel<<<E, threads, 0, st>>>(rs.block_base, nb, E, counts, offsets, rs.ticket);
-    return cudaGetLastError();
+    return launch_chained(expert_scan_kernel, dim3(E), dim3(threads), 0, st, rs.block_base, nb, E, counts, offsets,
+                          rs.ticket);
 }
 
 cudaError_t launch_pad_offsets(const int32_t* offsets, int E, int align, int32_t* padded_offsets, cudaStream_t st) {
@@ -1319,11 +1329,11 @@ cudaError_t launch_permute(const bf16* x, int64_t T, int H, const int32_t* topk_
         const int64_t slots = (int64_t)sm_count() * per_sm;
         const int64_t per_block = (T + slots - 1) / slots;
         const int64_t blocks = (T + per_block - 1) / per_block;
-        permute_tokens_kernel<<<(unsigned)blocks, threads, 0, st>>>(
-            reinterpret_cast<const uint4*>(x), T, H8r, topk_idx, k, offsets, E, rs.block_base, nb,
-            route_tokens_per_block(T), rs.local_rank, reinterpret_cast<uint4*>(x_perm), sorted_token, row_of,
-            A, per_block, err);
-        return cudaGetLastError();
+        return launch_chained(permute_tokens_kernel, dim3((unsigned)blocks), dim3(threads), 0, st,
+                              reinterpret_cast<const uint4*>(x), T, H8r, topk_idx, k, offsets, E,
+                              (const int32_t*)rs.block_base, nb, route_tokens_per_block(T),
+                              (const int32_t*)rs.local_rank, reinterpret_cast<uint4*>(x_perm), sorted_token, row_of,
+                              A, per_block, err);
     }
     if (E > kPermMaxExperts) return cudaErrorInvalidValue;
     constexpr int kThreadsW = 256;
@@ -1336,11 +1346,10 @@ cudaError_t launch_permute(const bf16* x, int64_t T, int H, const int32_t* topk_
     const int64_t cap = (int64_t)sm_count() * per_sm * (kThreadsW / 32);
     const int64_t warps = T < cap ? T : cap;
     const int64_t blocks = (warps + kThreadsW / 32 - 1) / (kThreadsW / 32);
-    kern<<<(unsigned)blocks, kThreadsW, 0, st>>>(
-        reinterpret_cast<const uint4*>(x), T, H8r, topk_idx, k, offsets, E, rs.block_base, nb,
-        route_tokens_per_block(T), rs.local_rank, reinterpret_cast<uint4*>(x_perm), sorted_token, row_of,
-        A, err);
-    return cudaGetLastError();
+    return launch_chained(kern, dim3((unsigned)blocks), dim3(kThreadsW), 0, st, reinterpret_cast<const uint4*>(x), T,
+                          H8r, topk_idx, k, offsets, E, (const int32_t*)rs.block_base, nb, route_tokens_per_block(T),
+                          (const int32_t*)rs.local_rank, reinterpret_cast<uint4*>(x_perm), sorted_token, row_of, A,
+                          err);
 }
 
 // Device address of g_router_noalloc_scratch on the current device. In host

@@ -73,8 +73,8 @@ def test_invalid_arguments_are_rejected_without_a_device(built):
     # workspace too small
     assert l.moe_router_topk(fake, 10, 8, 2, ctypes.byref(opts), fake, fake, None, fake, fake,
                              fake, 16, None) == 4
-    # grouped MLP: H or I not a multiple of 64 is outside the kernels' limits
-    assert l.moe_grouped_mlp(fake, 100, fake, 8, 96, 128, fake, fake, fake, None, None, fake,
+    # grouped MLP: H or I not a multiple of 8 is outside the kernels' limits
+    assert l.moe_grouped_mlp(fake, 100, fake, 8, 100, 128, fake, fake, fake, None, None, fake,
                              1 << 30, None) == 2
     assert l.moe_grouped_mlp(fake, 100, fake, 8, 128, 100, fake, fake, fake, None, None, fake,
                              1 << 30, None) == 2

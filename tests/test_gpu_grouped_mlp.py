@@ -40,6 +40,8 @@ def grouped_case(T, H, I, E, k, seed, dead=(), skew=False):
     (700, 320, 640, 16, 4, ()),          # H not a multiple of 256: ragged N tile in the down GEMM
     (1, 128, 128, 8, 2, ()),             # a single token
     (4500, 256, 256, 4, 2, (1,)),        # large expert blocks (the default picks pair tiles)
+    (600, 200, 136, 8, 2, (5,)),         # H and I multiples of 8 only: partial 8-column chunks
+    (300, 72, 40, 4, 2, ()),             # narrow rows: one partial K slice, a partial N block
 ])
 def test_grouped_mlp_matches_expert_loop(T, H, I, E, k, dead, tiles, monkeypatch):
     helpers.force_kernels(gemm_tiles=tiles)

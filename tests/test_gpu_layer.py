@@ -47,6 +47,8 @@ SMALL = {
     # about 1000 rows per expert: the weight gradient streams B instead of
     # keeping each expert's rows in shared memory (more than 320 rows)
     "long_k": wl.WORKLOADS["mixtral_8x7b"].scaled(T=2048, H=256, I=192, E=4),
+    # H and I multiples of 8 only (not of 32 or 64): partial column chunks everywhere
+    "odd_dims": wl.WORKLOADS["qwen3_30b_a3b"].scaled(T=300, H=200, I=136, E=16),
 }
 
 
@@ -77,7 +79,7 @@ def test_layer_forward_saved_state_and_empty_batch():
     assert empty.shape == (0, w.H)
 
 
-BWD = ["tiny", "qwen3_small", "skew_small", "mixtral_small", "long_k"]
+BWD = ["tiny", "qwen3_small", "skew_small", "mixtral_small", "long_k", "odd_dims"]
 
 
 def _oracle_backward(w, d, r):
