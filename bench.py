@@ -474,41 +474,58 @@ def nonempty_experts(layer):
     return int((layer.state["counts"] > 0).sum().item())
 
 
+def traced_pass(layer, steps, flush=None):
+    """Per-stage events on `steps` further steps (the stage boundaries break
+    the programmatic overlap of consecutive kernels, so the step times are
+    taken without them); with `flush`, L2 is flushed before each step."""
+    import torch
+    fevs, bevs = [], []
+    for _ in range(steps):
+        fev = _events(7)
+        bev = _events(7) if layer.w.backward else None
+        if flush is not None:
+            flush.sum()
+            torch.cuda._sleep(200000)
+        layer.step(fev, bev)
+        fevs.append(fev)
+        bevs.append(bev)
+    torch.cuda.synchronize()
+    return fevs, bevs
+
+
 def measure_flushed(layer, steps, warmup, flush):
     """Each step timed on its own after an L2 flush (for workloads whose
     weights could stay in L2 between steps); median over the steps."""
     import torch
-    totals, fevs, bevs = [], [], []
+    totals = []
     for it in range(warmup + steps):
-        fev = _events(7)
-        bev = _events(7) if layer.w.backward else None
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         flush.sum()
-        torch.cuda._sleep(200000)
-        layer.step(fev, bev)
+        torch.cuda._sleep(200000)   # the GPU is busy while the step is issued: device time only
+        s.record()
+        layer.step()
+        e.record()
         torch.cuda.synchronize()
         if it >= warmup:
-            fevs.append(fev)
-            bevs.append(bev)
-            totals.append(fev[0].elapsed_time((bev or fev)[6]))
+            totals.append(s.elapsed_time(e))
+    fevs, bevs = traced_pass(layer, steps, flush)
     return statistics.median(totals), fevs, bevs
 
 
 def measure_back_to_back(layer, steps, warmup):
     """`steps` steps back to back between two events (no flush: the weights
-    exceed L2); per-stage events on every step."""
+    exceed L2), then a traced pass for the stage times."""
     import torch
     for _ in range(warmup):
         layer.step()
     torch.cuda.synchronize()
-    fevs = [_events(7) for _ in range(steps)]
-    bevs = [_events(7) for _ in range(steps)] if layer.w.backward else [None] * steps
-    torch.cuda.synchronize()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s.record()
     for i in range(steps):
-        layer.step(fevs[i], bevs[i])
+        layer.step()
     e.record()
     torch.cuda.synchronize()
+    fevs, bevs = traced_pass(layer, steps)
     return s.elapsed_time(e) / steps, fevs, bevs
 
 
@@ -579,9 +596,6 @@ def our_arm(args, world, rank, local):
         raise RuntimeError("device status error after warm-up")
 
     K = args.steps
-    fevs = [_events(7) for _ in range(K)]
-    bevs = [_events(7) for _ in range(K)] if w.backward else [None] * K
-    torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
     barrier(world)
@@ -589,7 +603,7 @@ def our_arm(args, world, rank, local):
     sampler.start()
     start.record()
     for i in range(K):
-        layer.step(fevs[i], bevs[i])
+        layer.step()
     end.record()
     torch.cuda.synchronize()
     clocks = sampler.stop()
@@ -598,6 +612,9 @@ def our_arm(args, world, rank, local):
     ms_max = max_over_ranks(ms, world)
     if m.moe_get_device_status() != 0:
         raise RuntimeError("device status error in the timed region")
+    # stage times: a separate pass of K steps with an event at every stage
+    # boundary (events between kernels break their programmatic overlap)
+    fevs, bevs = traced_pass(layer, K)
     stages = stage_medians(layer, fevs, bevs)
 
     graph = None if args.no_graph else graph_measure(args, layer.step, w, world, m)
@@ -633,7 +650,7 @@ def our_arm(args, world, rank, local):
                      "traffic": traffic_for(f"gate_up_swiglu/{w.name}"),
                      "peak_source": f"{peaks_src} {'sustained' if long_region else 'burst'} bf16",
                      "flop_per_launch": gate_up_flop, "ms_per_launch": gate_up_ms,
-                     "ms_per_launch_is": "median over the timed steps (CUDA events on the launching stream)"},
+                     "ms_per_launch_is": "median over a traced pass of as many steps as the timed region, events on the launching stream"},
         "stages_ms": stages,
         "bandwidth_kernels": bandwidth_report(layer, stages, hbm, flush),
         "hbm_peak_gbs": hbm,
