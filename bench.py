@@ -529,27 +529,38 @@ def measure_back_to_back(layer, steps, warmup):
     return s.elapsed_time(e) / steps, fevs, bevs
 
 
-def workload_entry(m, name, peaks, flush, steps=50, warmup=10):
-    """One extra workload: its median step time, tokens/s, grouped-GEMM
-    fractions, bandwidth stages (warm and L2-cold), and for the small batches
-    the HBM roofline of the non-empty experts' weights."""
+def workload_entry(m, name, peaks, flush, steps, warmup, local):
+    """One extra workload, timed like the main line: after a one-second idle
+    (so each workload starts from the same power state), `warmup` steps,
+    then `steps` timed steps with the clocks sampled. Reports the median step
+    time, tokens/s, grouped-GEMM fractions, the warm bandwidth stages, and for
+    the small batches the HBM roofline of the non-empty experts' weights.
+    Returns (entry, layer); the L2-cold bandwidth stages are measured later
+    (cold_pass), so that their loops do not heat the GPU before the next
+    workload's timing."""
     import torch
     import workloads as wl
     w = wl.WORKLOADS[name]
     d = wl.make_inputs(w, "cuda")
     layer = Layer(m, w, d)
     small = w.T <= 64
+    torch.cuda.synchronize()
+    time.sleep(1.0)
+    sampler = ClockSampler(local)
+    sampler.start()
     if small:
         ms, fevs, bevs = measure_flushed(layer, steps, warmup, flush)
     else:
         ms, fevs, bevs = measure_back_to_back(layer, steps, warmup)
+    clocks = sampler.stop()
     if m.moe_get_device_status() != 0:
         raise RuntimeError(f"device status error in {name}")
     stages = stage_medians(layer, fevs, bevs)
     hbm = peaks["hbm_gbs"]
     e = {"T": w.T, "H": w.H, "I": w.I, "E": w.E, "top_k": w.k, "pass": "fwd+bwd" if w.backward else "fwd",
-         "ms_per_step": ms, "tokens_per_s": w.T / (ms / 1e3),
+         "steps": steps, "warmup": warmup, "ms_per_step": ms, "tokens_per_s": w.T / (ms / 1e3),
          "l2": "flushed (256 MB read) before each step" if small else "weights exceed L2; steps back to back",
+         "clocks": clocks,
          "grouped_gemm": gemm_summary(w, stages, peaks),
          "stages_us": {k_: v * 1e3 for k_, v in stages.items()}}
     if small:
@@ -563,11 +574,29 @@ def workload_entry(m, name, peaks, flush, steps=50, warmup=10):
                          "layer_frac": wbytes / (ms / 1e3) / 1e9 / hbm,
                          "note": "bytes = the non-empty experts' weights (3 H I bf16 each), read once per step; "
                                  "frac over the two GEMM stages, layer_frac over the whole step"}
-    else:
-        e["bandwidth_kernels"] = bandwidth_report(layer, stages, hbm, flush)
-    del layer, d
+        return e, None
+    e["bandwidth_kernels"] = warm_bandwidth(w, stages, hbm)
+    return e, layer
+
+
+def extra_workloads(m, args, peaks, flush, local, skip):
+    """Every other workload, timed one after another, then their L2-cold
+    bandwidth stages in a second pass."""
+    import torch
+    steps, warmup = max(args.steps, 20), max(args.warmup, 5)
+    out, layers = {}, {}
+    for n in EXTRA_WORKLOADS:
+        if n == skip:
+            continue
+        out[n], layers[n] = workload_entry(m, n, peaks, flush, steps, warmup, local)
+    for n, layer in layers.items():
+        if layer is None:
+            continue
+        for key, v in cold_bandwidth(layer, peaks["hbm_gbs"], flush).items():
+            out[n]["bandwidth_kernels"][key].update(v)
+    layers.clear()
     torch.cuda.empty_cache()
-    return e
+    return out
 
 
 def our_arm(args, world, rank, local):
@@ -665,7 +694,7 @@ def our_arm(args, world, rank, local):
     if world == 1 and not args.no_extra and args.T is None:
         del layer
         torch.cuda.empty_cache()
-        line["workloads"] = {n: workload_entry(m, n, peaks, flush) for n in EXTRA_WORKLOADS if n != w.name}
+        line["workloads"] = extra_workloads(m, args, peaks, flush, local, w.name)
     if args.router_sweep:
         line["router_sweep"] = router_sweep(m, hbm)
     if args.gather_compare:

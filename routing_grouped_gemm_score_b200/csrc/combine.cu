@@ -140,33 +140,43 @@ __global__ void __launch_bounds__(kWarpKernelThreads, KB > 8 ? 2 : 4)
 // the shared row's chunk) issued together; the next token's routing is loaded
 // while the current token is summed. The sum runs in a fixed order: shared
 // first, then j ascending, fp32.
+// A warp's unit of work is one 2^lg_parts-th of a token's row (the whole row
+// but for small batches, where one warp per token would leave the GPU idle);
+// each output element is summed the same way whatever the split.
 template <int KB, int CH>
 __global__ void __launch_bounds__(kWarpKernelThreads, KB > 8 ? 2 : 4)
     combine_warp_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ row_of,
                         const float* __restrict__ probs, int64_t T, int k, int H8, int64_t A,
-                        const uint4* __restrict__ shared, uint4* __restrict__ out, unsigned* err) {
+                        const uint4* __restrict__ shared, uint4* __restrict__ out, unsigned* err, int lg_parts) {
     pdl_wait();
     pdl_launch_dependents();
     const int lane = threadIdx.x & 31;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t units = T << lg_parts;
+    const int span = (H8 + (1 << lg_parts) - 1) >> lg_parts;   // chunks of a part
+    int64_t u = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     int32_t r_next = -1;
     float p_next = 1.0f;
-    if (t < T && lane < k) {
+    if (u < units && lane < k) {
+        const int64_t t = u >> lg_parts;
         r_next = __ldg(row_of + t * k + lane);
         if (probs) p_next = __ldg(probs + t * k + lane);
     }
-    for (; t < T; t += nwarps) {
+    for (; u < units; u += nwarps) {
+        const int64_t t = u >> lg_parts;
+        const int c_begin = (int)(u & ((1 << lg_parts) - 1)) * span;
+        const int c_end = min(H8, c_begin + span);
         int32_t r = r_next;
         const float p = p_next;
         if (lane < k && (r < 0 || r >= A)) {
             raise_error(err, kErrDeviceCheck);
             r = -1;
         }
-        const int64_t tn = t + nwarps;   // the next token's routing, one token ahead
+        const int64_t un = u + nwarps;   // the next unit's routing, one unit ahead
         r_next = -1;
         p_next = 1.0f;
-        if (tn < T && lane < k) {
+        if (un < units && lane < k) {
+            const int64_t tn = un >> lg_parts;
             r_next = __ldg(row_of + tn * k + lane);
             if (probs) p_next = __ldg(probs + tn * k + lane);
         }
@@ -178,12 +188,12 @@ __global__ void __launch_bounds__(kWarpKernelThreads, KB > 8 ? 2 : 4)
             off[j] = (j < k && rj >= 0) ? (int64_t)rj * H8 : -1;
             ps[j] = __shfl_sync(kFull, p, j);
         }
-        for (int c0 = 0; c0 < H8; c0 += 32 * CH) {
+        for (int c0 = c_begin; c0 < c_end; c0 += 32 * CH) {
             uint4 v[CH][KB], sh[CH];
 #pragma unroll
             for (int h = 0; h < CH; ++h) {
                 const int c = c0 + 32 * h + lane;
-                if (c >= H8) continue;
+                if (c >= c_end) continue;
                 if (shared) sh[h] = __ldg(shared + t * H8 + c);
 #pragma unroll
                 for (int j = 0; j < KB; ++j)
@@ -192,7 +202,7 @@ __global__ void __launch_bounds__(kWarpKernelThreads, KB > 8 ? 2 : 4)
 #pragma unroll
             for (int h = 0; h < CH; ++h) {
                 const int c = c0 + 32 * h + lane;
-                if (c >= H8) continue;
+                if (c >= c_end) continue;
                 float acc[8];
 #pragma unroll
                 for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
@@ -229,10 +239,16 @@ cudaError_t launch_combine(const bf16* y_perm, const int32_t* row_of, const floa
     auto kern = k <= 2 ? combine_warp_kernel<2, 4>
               : k <= 4 ? combine_warp_kernel<4, 2>
               : k <= 8 ? combine_warp_kernel<8, 2> : combine_warp_kernel<16, 1>;
-    const int64_t blocks = warp_kernel_blocks(kern, T);
+    // small batches: split each token's row over up to 8 warps (whole 16-byte
+    // chunks per lane step), so that more SMs share the few rows
+    const int H8 = H / 8;
+    const int64_t cap = warp_kernel_blocks(kern, (int64_t)1 << 40) * (kWarpKernelThreads / 32);
+    int lg = 0;
+    while (lg < 3 && (T << (lg + 1)) <= cap && (H8 >> (lg + 1)) >= 64) ++lg;
+    const int64_t blocks = warp_kernel_blocks(kern, T << lg);
     return launch_chained(kern, dim3((unsigned)blocks), dim3(kWarpKernelThreads), 0, st,
-                          reinterpret_cast<const uint4*>(y_perm), row_of, probs, T, k, H / 8, A,
-                          reinterpret_cast<const uint4*>(shared), reinterpret_cast<uint4*>(out), err);
+                          reinterpret_cast<const uint4*>(y_perm), row_of, probs, T, k, H8, A,
+                          reinterpret_cast<const uint4*>(shared), reinterpret_cast<uint4*>(out), err, lg);
 }
 
 cudaError_t launch_combine_backward(const bf16* dout, const bf16* y_perm, const int32_t* row_of,

@@ -536,6 +536,13 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
                 for (int i = 0; i < 32; ++i) v[i] = 0.0f;
             }
             if (n0 + c0 >= p.N || m0 >= p.M) continue;
+            if (tmC == nullptr) {
+                // row stores from the warp (16-byte vectors through its buffer):
+                // the SM's TMA unit then carries only the operand loads
+                store_rows<32>(buf, p.out + (int64_t)t.g * p.out_group_stride + (int64_t)m0 * p.ldo + n0 + c0, p.ldo,
+                               min(p.M - m0, 32), min(p.N - (n0 + c0), 32), v, lane);
+                continue;
+            }
             if (lane == 0) bulk_wait_group_read0();   // the previous block has left the buffer
             __syncwarp();
 #pragma unroll
@@ -1095,11 +1102,14 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
 // batches). The roles of the operands are swapped: the weights are the
 // 128-row A operand, read MN-major straight from their [K][N] layout (128
 // output columns per tile), and the expert's token rows are the B operand
-// (N = 64 rows per tile, K-major). D = W^T X^T sits in TMEM with one output
-// column per lane and one token row per TMEM column. A tile is (expert,
-// 128-column block, 64-row block); a block of up to 64 rows therefore reads
-// each weight byte once, and a one-token expert costs no padded MMA rows.
-// Tiles of one expert run in column-block order, its row blocks side by side.
+// (N = NR rows per tile, K-major; NR = 64, or 16 when no expert can have more
+// than 16 rows). D = W^T X^T sits in TMEM with one output column per lane and
+// one token row per TMEM column. A tile is (expert, 128-column block, NR-row
+// block); a block of up to NR rows therefore reads each weight byte once, and
+// a one-token expert costs no padded MMA rows. Tiles of one expert run in
+// column-block order, its row blocks side by side. With NR = 16 a stage holds
+// 2 KB of token rows instead of 8 KB, so the ring keeps 176 KB of weights in
+// flight instead of 96 KB.
 //
 // SwiGLU forward: a tile's 128 columns are 64 gate columns and the matching
 // 64 up columns, so lanes 0..63 hold g and lanes 64..127 hold u of the same
@@ -1108,19 +1118,25 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
 // compute h = silu(g) u (times the row scale) and store h (and [g | u]).
 // Store epilogue (down): each lane writes its output column of every valid row.
 // Warp roles as in gemm_1cta_kernel: warp 0 TMA producer, warp 1 TMEM owner
-// and MMA issuer, warps 2-9 epilogue (two per lane quarter, each on 32 of
-// the 64 token columns). Every wait is bounded.
-constexpr int BNS = 64, STAGESS = 6;
+// and MMA issuer, warps 2-9 epilogue (two per lane quarter, each on half of
+// the NR token columns). Every wait is bounded.
 constexpr int kStageAS = 128 * BK * 2;           // 128 weight columns x 64 K: two 64-column chunks
-constexpr int kStageBS = BNS * BK * 2;           // 64 token rows x 64 K
-constexpr int kStageS = kStageAS + kStageBS;     // 24 KB
-constexpr int kTmemColsS = 128;                  // two 128-lane x 64-column accumulators
 
+template <int NR>
+struct SwapCfg {
+    static constexpr int kStages = NR == 16 ? 11 : 6;
+    static constexpr int kStageB = NR * BK * 2;                 // NR token rows x 64 K
+    static constexpr int kStage = kStageAS + kStageB;           // 18 or 24 KB
+    static constexpr uint32_t kTmemCols = NR == 16 ? 32 : 128;  // two 128-lane x NR-column accumulators
+    static constexpr int kWarpCols = NR / 2;                    // token columns of one epilogue warp
+};
+
+template <int NR>
 struct __align__(1024) SmemS {
-    uint8_t stage[STAGESS][kStageS];
-    float ubuf[2][64][BNS + 1];   // SwiGLU: the up values of a tile's 64 columns, per accumulator
-    uint64_t full[STAGESS];
-    uint64_t empty[STAGESS];
+    uint8_t stage[SwapCfg<NR>::kStages][SwapCfg<NR>::kStage];
+    float ubuf[2][64][NR + 1];    // SwiGLU: the up values of a tile's 64 columns, per accumulator
+    uint64_t full[SwapCfg<NR>::kStages];
+    uint64_t empty[SwapCfg<NR>::kStages];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t xchg[2];             // SwiGLU: the up values of the accumulator's tile are in ubuf
@@ -1131,8 +1147,11 @@ struct __align__(1024) SmemS {
     int tile_start[kMaxGroups + 1];
     int off[kMaxGroups + 1];
 };
-static_assert(kStageS % 1024 == 0 && kStageAS % 1024 == 0, "swizzled stages stay 1024-byte aligned");
-constexpr size_t kSmemSBytes = sizeof(SmemS) + 1024;
+static_assert(SwapCfg<16>::kStage % 1024 == 0 && SwapCfg<64>::kStage % 1024 == 0 && kStageAS % 1024 == 0,
+              "swizzled stages stay 1024-byte aligned");
+template <int NR>
+constexpr size_t swap_smem_bytes() { return sizeof(SmemS<NR>) + 1024; }
+static_assert(sizeof(SmemS<16>) + 1024 <= 227 * 1024 && sizeof(SmemS<64>) + 1024 <= 227 * 1024, "swap smem");
 
 // First weight column of chunk c (0, 1) of the tile's 128 columns.
 template <int EPI>
@@ -1141,19 +1160,20 @@ __device__ __forceinline__ int w_col_swap(const Tile& t, const Params& p, int c)
     return t.n_blk * 128 + 64 * c;
 }
 
-template <int EPI>
+template <int EPI, int NR>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_swap_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                      const Params p) {
     static_assert(EPI == kEpiSwiglu || EPI == kEpiStore, "forward GEMMs only");
     extern __shared__ uint8_t smem_raw[];
-    SmemS& s = *reinterpret_cast<SmemS*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+    using Cfg = SwapCfg<NR>;
+    SmemS<NR>& s = *reinterpret_cast<SmemS<NR>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                          ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int* abort_flag = &s.abort;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < STAGESS; ++i) {
+        for (int i = 0; i < Cfg::kStages; ++i) {
             mbar_init(&s.full[i], 1);
             mbar_init(&s.empty[i], 1);
         }
@@ -1169,11 +1189,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tensormap(&tmW);
     }
     if (warp == 1) {
-        tmem_alloc(&s.tmem_base, kTmemColsS);
+        tmem_alloc(&s.tmem_base, Cfg::kTmemCols);
         tmem_relinquish();
     }
     pdl_wait();                // the previous kernel's outputs (token rows, offsets) are complete
-    build_schedule<false>(s, p, BNS);
+    build_schedule<false>(s, p, NR);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1185,10 +1205,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t issued[STAGESS] = {0, 0, 0, 0, 0, 0};
+            uint32_t issued[Cfg::kStages] = {};
             bool ok = true;
             for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
-                const Tile t = decode_tile<false>(s, p, id, BNS);
+                const Tile t = decode_tile<false>(s, p, id, NR);
                 for (int kb = 0; kb < t.num_kb; ++kb) {
                     if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag, p.err)) {
                         ok = false;
@@ -1197,37 +1217,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t* a_s = s.stage[stage];
                     uint8_t* b_s = s.stage[stage] + kStageAS;
                     uint64_t* bar = &s.full[stage];
-                    mbar_arrive_expect_tx(bar, kStageS);
+                    mbar_arrive_expect_tx(bar, Cfg::kStage);
 #pragma unroll
                     for (int c = 0; c < 2; ++c)
                         tma_load_3d(&tmW, bar, a_s + c * kChunkBytes, w_col_swap<EPI>(t, p, c), kb * BK, t.g);
                     tma_load_2d(&tmX, bar, b_s, kb * BK, t.row0);
                     issued[stage] += 1;
-                    if (++stage == STAGESS) {
+                    if (++stage == Cfg::kStages) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
             // let every load still in flight land before the CTA may exit
-            for (int i = 0; i < STAGESS; ++i)
+            for (int i = 0; i < Cfg::kStages; ++i)
                 if (issued[i]) mbar_wait(&s.full[i], (issued[i] - 1) & 1u, abort_flag, p.err);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
-        constexpr uint32_t idesc = instr_desc<128, BNS, true, false>();
+        constexpr uint32_t idesc = instr_desc<128, NR, true, false>();
         int stage = 0;
         uint32_t phase = 0;
         int local_tile = 0;
         bool ok = true;
         bool any_mma = false;
         for (int id = blockIdx.x; id < total && ok; id += gridDim.x, ++local_tile) {
-            const Tile t = decode_tile<false>(s, p, id, BNS);
+            const Tile t = decode_tile<false>(s, p, id, NR);
             const int buf = local_tile & 1;
             const uint32_t use = (uint32_t)(local_tile >> 1);
             if (!mbar_wait(&s.acc_empty[buf], (use & 1u) ^ 1u, abort_flag, p.err)) break;
             tc_fence_after();
-            const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BNS);
+            const uint32_t d_tmem = tmem_base + (uint32_t)(buf * NR);
             for (int kb = 0; kb < t.num_kb; ++kb) {
                 if (!mbar_wait(&s.full[stage], phase, abort_flag, p.err)) {
                     ok = false;
@@ -1247,7 +1267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     any_mma = true;
                 }
                 __syncwarp();
-                if (++stage == STAGESS) {
+                if (++stage == Cfg::kStages) {
                     stage = 0;
                     phase ^= 1u;
                 }
@@ -1264,25 +1284,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------------ epilogue
         const int quarter = warp & 3;               // TMEM lanes 32*quarter .. +31
-        const int half = (warp - 2) / 4;            // token columns 32*half .. +31
+        const int half = (warp - 2) / 4;            // token columns kWarpCols*half ..
         int local_tile = 0;
         for (int id = blockIdx.x; id < total; id += gridDim.x, ++local_tile) {
-            const Tile t = decode_tile<false>(s, p, id, BNS);
+            const Tile t = decode_tile<false>(s, p, id, NR);
             const int buf = local_tile & 1;
             const uint32_t use = (uint32_t)(local_tile >> 1);
             if (!mbar_wait(&s.acc_full[buf], use & 1u, abort_flag, p.err)) break;
             tc_fence_after();
-            float v[32];
-            tmem_load_32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BNS + 32 * half), v);
-            const int j0 = 32 * half;                        // first token column of this warp
-            const int nvalid = min(max(t.rows - j0, 0), 32);
+            constexpr int kWC = Cfg::kWarpCols;
+            float v[kWC];
+            const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * NR + kWC * half);
+            if constexpr (kWC == 32) tmem_load_32(taddr, v);
+            else tmem_load_8(taddr, v);
+            const int j0 = kWC * half;                       // first token column of this warp
+            const int nvalid = min(max(t.rows - j0, 0), kWC);
             bool ok = true;
             if (EPI == kEpiSwiglu) {
                 if (quarter >= 2) {
                     // up values of columns 32 (quarter - 2) + lane
                     float* row = s.ubuf[buf][32 * (quarter - 2) + lane] + j0;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) row[i] = v[i];
+                    for (int i = 0; i < kWC; ++i) row[i] = v[i];
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&s.xchg[buf]);
                 } else {
@@ -1292,7 +1315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float* urow = s.ubuf[buf][32 * quarter + lane] + j0;
                         const int64_t r0 = (int64_t)t.row0 + j0;
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
+                        for (int i = 0; i < kWC; ++i) {
                             if (i >= nvalid || hc >= p.N) break;
                             const float g = v[i], u = urow[i];
                             const float rs = p.row_scale ? __ldg(p.row_scale + r0 + i) : 1.0f;
@@ -1309,7 +1332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int64_t r0 = (int64_t)t.row0 + j0;
                 if (col < p.N) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
+                    for (int i = 0; i < kWC; ++i) {
                         if (i >= nvalid) break;
                         p.out[(r0 + i) * p.ldo + col] = __float2bfloat16_rn(v[i]);
                     }
@@ -1327,7 +1350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kTmemColsS);
+        tmem_dealloc(tmem_base, Cfg::kTmemCols);
     }
 }
 
@@ -1480,18 +1503,32 @@ bool use_swap_tiles(int64_t rows, int groups) {
     return rows <= (int64_t)groups * 16;
 }
 
-template <int EPI>
-cudaError_t launch_swap(const CUtensorMap& x64, const CUtensorMap& w, const Params& p, cudaStream_t st) {
-    auto kern = gemm_swap_kernel<EPI>;
+template <int EPI, int NR>
+cudaError_t launch_swap(const CUtensorMap& x_rows, const CUtensorMap& w, const Params& p, cudaStream_t st) {
+    auto kern = gemm_swap_kernel<EPI, NR>;
     static std::once_flag once;
     static cudaError_t attr = cudaSuccess;
-    if (set_smem_once(kern, kSmemSBytes, once, attr) != cudaSuccess) return attr;
+    if (set_smem_once(kern, swap_smem_bytes<NR>(), once, attr) != cudaSuccess) return attr;
     // upper bound of the tiles without reading the device counts
-    const int64_t bound = ((int64_t)p.rows / BNS + p.groups) * (int64_t)p.n_blocks;
+    const int64_t bound = ((int64_t)p.rows / NR + p.groups) * (int64_t)p.n_blocks;
     if (bound <= 0) return cudaSuccess;
     int64_t grid = sm_count();
     if (grid > bound) grid = bound;
-    return launch_chained(kern, dim3((unsigned)grid), dim3(kThreads), kSmemSBytes, st, x64, w, p);
+    return launch_chained(kern, dim3((unsigned)grid), dim3(kThreads), swap_smem_bytes<NR>(), st, x_rows, w, p);
+}
+
+// Swap-AB launch with 16 token rows per tile when no group can hold more than
+// 16 rows (max_group_rows), else 64. x is the token-row matrix [rows][K].
+template <int EPI>
+cudaError_t launch_swap_rows(const bf16* x, int64_t rows, int K, int64_t max_group_rows, const CUtensorMap& w,
+                             const Params& p, cudaStream_t st) {
+    CUtensorMap xm;
+    if (max_group_rows <= 16) {
+        if (!make_map_2d(&xm, x, K, rows, K, BK, 16)) return cudaErrorInvalidValue;
+        return launch_swap<EPI, 16>(xm, w, p, st);
+    }
+    if (!make_map_2d(&xm, x, K, rows, K, BK, 64)) return cudaErrorInvalidValue;
+    return launch_swap<EPI, 64>(xm, w, p, st);
 }
 
 // Group-M GEMM on pair or single tiles. `ta` and `ta64` are A maps with
@@ -1519,7 +1556,8 @@ bool make_out_map(CUtensorMap* m, const bf16* out, int64_t rows, uint64_t cols) 
 
 cudaError_t gemm_gate_up_swiglu(const bf16* x, int64_t rows, const int32_t* offsets, int E, int H,
                                 int I, const bf16* w_gate_up, bf16* h, bf16* gu_save,
-                                cudaStream_t st, unsigned* err, const float* row_scale) {
+                                cudaStream_t st, unsigned* err, const float* row_scale, int64_t max_group_rows) {
+    if (max_group_rows <= 0 || max_group_rows > rows) max_group_rows = rows;
     if (rows == 0) return cudaSuccess;
     CUtensorMap ta, ta64, tb;
     if (!make_map_2d(&ta, x, H, rows, H, BK, 128)) return cudaErrorInvalidValue;
@@ -1539,7 +1577,7 @@ cudaError_t gemm_gate_up_swiglu(const bf16* x, int64_t rows, const int32_t* offs
     p.row_scale = row_scale;
     if (use_swap_tiles(rows, groups)) {
         p.n_blocks = (I + 63) / 64;   // 64 gate and the matching 64 up columns per tile
-        return launch_swap<kEpiSwiglu>(ta64, tb, p, st);
+        return launch_swap_rows<kEpiSwiglu>(x, rows, H, max_group_rows, tb, p, st);
     }
     CUtensorMap tc, tc2;
     if (!make_out_map(&tc, h, rows, I)) return cudaErrorInvalidValue;
@@ -1582,7 +1620,8 @@ bool grouped_gemm_single_tiles(int64_t rows, int groups) {
 }
 
 cudaError_t gemm_down(const bf16* h, int64_t rows, const int32_t* offsets, int E, int H, int I,
-                      const bf16* w_down, bf16* y, cudaStream_t st, unsigned* err) {
+                      const bf16* w_down, bf16* y, cudaStream_t st, unsigned* err, int64_t max_group_rows) {
+    if (max_group_rows <= 0 || max_group_rows > rows) max_group_rows = rows;
     if (rows == 0) return cudaSuccess;
     CUtensorMap ta, ta64, tb;
     if (!make_map_2d(&ta, h, I, rows, I, BK, 128)) return cudaErrorInvalidValue;
@@ -1597,7 +1636,7 @@ cudaError_t gemm_down(const bf16* h, int64_t rows, const int32_t* offsets, int E
     p.ldo = H;
     if (use_swap_tiles(rows, groups)) {
         p.n_blocks = (H + 127) / 128;   // 128 output columns per tile
-        return launch_swap<kEpiStore>(ta64, tb, p, st);
+        return launch_swap_rows<kEpiStore>(h, rows, I, max_group_rows, tb, p, st);
     }
     CUtensorMap tc;
     if (!make_out_map(&tc, y, rows, H)) return cudaErrorInvalidValue;

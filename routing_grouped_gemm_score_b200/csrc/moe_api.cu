@@ -588,11 +588,11 @@ moe_status moe_layer_forward(const float* logits, const moe_bf16* x, int64_t T, 
                                                 reinterpret_cast<bf16*>(gu), st, err)
                    : gemm_gate_up_swiglu(L.x_perm, A, L.offsets, E, H, I,
                                          reinterpret_cast<const bf16*>(w_gate_up), L.h,
-                                         reinterpret_cast<bf16*>(gu), st, err);
+                                         reinterpret_cast<bf16*>(gu), st, err, nullptr, T);
     if (e == cudaSuccess) e = trace_mark(3, st);
     if (e == cudaSuccess)
         e = gemm_down(L.h, A, L.offsets, E, H, I, reinterpret_cast<const bf16*>(w_down), L.y_perm,
-                      st, err);
+                      st, err, T);   // an expert gets at most T rows
     if (e == cudaSuccess) e = trace_mark(4, st);
     if (e == cudaSuccess && has_shared) {
         e = gemm_gate_up_swiglu(xb, T, nullptr, 1, H, I,

@@ -255,6 +255,20 @@ __device__ __forceinline__ void tmem_load_32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Loads 8 consecutive fp32 columns of this thread's TMEM lane and waits for
+// them. Warp-collective.
+__device__ __forceinline__ void tmem_load_8(uint32_t taddr, float (&v)[8]) {
+    uint32_t r[8];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 // Loads 32 consecutive fp32 columns of this thread's TMEM lane from each of
 // two column addresses, then waits for the loads. Loads and wait sit in one
 // asm statement, so no use of the registers can be scheduled before the wait.

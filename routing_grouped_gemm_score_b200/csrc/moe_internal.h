@@ -122,9 +122,13 @@ cudaError_t launch_combine_backward(const bf16* dout, const bf16* y_perm, const 
 // map cannot be encoded (bad alignment or extent).
 // gate_up + SwiGLU: h[r] = silu(x[r] Wg[e]) * (x[r] Wu[e]); optionally gu[r] = [g | u].
 // offsets NULL: one group of `rows` rows using the weights of group 0.
+// max_group_rows: an upper bound on the rows of any group (0: rows), which
+// lets small batches take narrower swap-AB tiles (a layer call passes T: a
+// token is routed to an expert at most once).
 cudaError_t gemm_gate_up_swiglu(const bf16* x, int64_t rows, const int32_t* offsets, int E, int H,
                                 int I, const bf16* w_gate_up, bf16* h, bf16* gu_save,
-                                cudaStream_t st, unsigned* err, const float* row_scale = nullptr);
+                                cudaStream_t st, unsigned* err, const float* row_scale = nullptr,
+                                int64_t max_group_rows = 0);
 // gate_up + SwiGLU with A row r gathered from x: row sorted_token[r] (-1: a
 // zero row) of x [T][H], so no permuted copy of x is needed. Single-CTA tiles
 // only; H a multiple of 8 and x 16-byte aligned.
@@ -137,7 +141,7 @@ cudaError_t gemm_gate_up_swiglu_gather(const bf16* x, int64_t T, const int32_t* 
 bool grouped_gemm_single_tiles(int64_t rows, int groups);
 // down: y[r] = h[r] Wd[e]
 cudaError_t gemm_down(const bf16* h, int64_t rows, const int32_t* offsets, int E, int H, int I,
-                      const bf16* w_down, bf16* y, cudaStream_t st, unsigned* err);
+                      const bf16* w_down, bf16* y, cudaStream_t st, unsigned* err, int64_t max_group_rows = 0);
 // dgrad of down with SwiGLU backward: dh = dy Wd[e]^T, then dgu = [dg | du]
 cudaError_t gemm_down_dgrad_swiglu(const bf16* dy, int64_t rows, const int32_t* offsets, int E,
                                    int H, int I, const bf16* w_down, const bf16* gu, bf16* dgu,

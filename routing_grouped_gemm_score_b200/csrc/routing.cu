@@ -926,6 +926,45 @@ __global__ void __launch_bounds__(1024)
     if (threadIdx.x == 0) *ticket = 0u;
 }
 
+// The same scan for at most 32 token blocks (T <= 256 at 8 tokens a block), in
+// one block and without the ticket: warp w scans the block counts of experts
+// w, w + 32, ... with one value per lane, then the block scans the expert
+// counts into the offsets. A small batch then pays for one block instead of E.
+constexpr int kScanSmallBlocks = 32;
+__global__ void __launch_bounds__(1024)
+    expert_scan_small_kernel(int32_t* block_base, int nb, int E, int32_t* counts, int32_t* offsets) {
+    pdl_wait();
+    pdl_launch_dependents();
+    __shared__ int cnt[256];
+    __shared__ int warp_tot[32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    for (int e = warp; e < E; e += nw) {
+        int32_t* row = block_base + (int64_t)e * nb;
+        const int v = lane < nb ? row[lane] : 0;
+        int incl = v;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(kFull, incl, off);
+            if (lane >= off) incl += o;
+        }
+        if (lane < nb) row[lane] = incl - v;
+        if (lane == 31) cnt[e] = incl;
+    }
+    __syncthreads();
+    if (counts == nullptr) return;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) counts[e] = cnt[e];
+    int carry = 0;
+    for (int base = 0; base < E; base += blockDim.x) {   // E <= 256 < blockDim: one pass
+        const int i = base + threadIdx.x;
+        const int v = i < E ? cnt[i] : 0;
+        int total;
+        const int incl = block_inclusive_scan(v, warp_tot, total);
+        if (i < E) offsets[i + 1] = carry + incl;
+        if (base == 0 && threadIdx.x == 0) offsets[0] = 0;
+        carry += total;
+    }
+}
+
 // Permute over contiguous token ranges, on plain 16-byte loads and stores. A
 // block owns tokens [t_begin, t_end). Its threads compute the destination rows
 // of kPermStage assignments at a time (offsets[e] + block_base[e][t / tpb] +
@@ -1276,6 +1315,9 @@ cudaError_t launch_rank_from_indices(const int32_t* topk_idx, int64_t T, int E, 
 cudaError_t launch_expert_scan(int64_t T, int E, const RouteScratch& rs, int32_t* counts,
                                int32_t* offsets, cudaStream_t st) {
     const int nb = (int)route_blocks(T);
+    if (nb <= kScanSmallBlocks)
+        return launch_chained(expert_scan_small_kernel, dim3(1), dim3(1024), 0, st, rs.block_base, nb, E, counts,
+                              offsets);
     int threads = 32;
     while (threads * kScanPerThread < nb && threads < 1024) threads <<= 1;
     return launch_chained(expert_scan_kernel, dim3(E), dim3(threads), 0, st, rs.block_base, nb, E, counts, offsets,

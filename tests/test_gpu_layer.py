@@ -49,6 +49,9 @@ SMALL = {
     "long_k": wl.WORKLOADS["mixtral_8x7b"].scaled(T=2048, H=256, I=192, E=4),
     # H and I multiples of 8 only (not of 32 or 64): partial column chunks everywhere
     "odd_dims": wl.WORKLOADS["qwen3_30b_a3b"].scaled(T=300, H=200, I=136, E=16),
+    # at most 16 rows per expert: the swap-AB tiles of 16 token rows
+    "t12": wl.WORKLOADS["tiny"].scaled(T=12),
+    "odd_t12": wl.WORKLOADS["qwen3_30b_a3b"].scaled(T=12, H=200, I=136, E=16),
 }
 
 
@@ -79,7 +82,7 @@ def test_layer_forward_saved_state_and_empty_batch():
     assert empty.shape == (0, w.H)
 
 
-BWD = ["tiny", "qwen3_small", "skew_small", "mixtral_small", "long_k", "odd_dims"]
+BWD = ["tiny", "qwen3_small", "skew_small", "mixtral_small", "long_k", "odd_dims", "odd_t12"]
 
 
 def _oracle_backward(w, d, r):
