@@ -536,13 +536,6 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
                 for (int i = 0; i < 32; ++i) v[i] = 0.0f;
             }
             if (n0 + c0 >= p.N || m0 >= p.M) continue;
-            if (tmC == nullptr) {
-                // row stores from the warp (16-byte vectors through its buffer):
-                // the SM's TMA unit then carries only the operand loads
-                store_rows<32>(buf, p.out + (int64_t)t.g * p.out_group_stride + (int64_t)m0 * p.ldo + n0 + c0, p.ldo,
-                               min(p.M - m0, 32), min(p.N - (n0 + c0), 32), v, lane);
-                continue;
-            }
             if (lane == 0) bulk_wait_group_read0();   // the previous block has left the buffer
             __syncwarp();
 #pragma unroll
