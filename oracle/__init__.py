@@ -86,6 +86,9 @@ def _load():
             lib.oracle_moe_backward_state.argtypes = [P, i64, i32, i32, i32, i32, P, P, P, P, P, i32,
                                                       i32, P, i64, P, P, P, P, P, P, P, P]
             lib.oracle_moe_backward_state.restype = i32
+            lib.oracle_moe_backward_scaled.argtypes = [P, i64, i32, i32, i32, i32, P, P, P, P, P, i32,
+                                                       i32, P, i64, P, P, P, P, P, P, P]
+            lib.oracle_moe_backward_scaled.restype = i32
             _lib = lib
     return _lib
 
@@ -331,8 +334,12 @@ def moe_forward_tokens(x_bits, logits, w_gu_bits, w_d_bits, k, tokens=None, scor
 
 def moe_backward(x_bits, topk_idx, topk_prob, w_gu_bits, w_d_bits, dout_bits, round_bf16=True,
                  only_expert=-1, tokens=None, want=("dx", "dw_gate_up", "dw_down", "dprob"),
-                 threads=None, state=None):
+                 threads=None, state=None, scaled=False):
     """Gradients of the layer for a given routing (see moe_oracle.c).
+
+    scaled: the ScaledSwiGLU layer, with the routing weight applied to the
+    SwiGLU output before FC2 and an unweighted combine
+    (oracle_moe_backward_scaled); its saved state needs no y.
 
     state: None (the forward values are recomputed), or a saved forward state
     dict(row_of [T,k] int32, gu [rows,2I], h [rows,I], y [rows,H] as bf16 bit
@@ -348,7 +355,7 @@ def moe_backward(x_bits, topk_idx, topk_prob, w_gu_bits, w_d_bits, dout_bits, ro
         if len(chunks) > 1:
             def one(c):
                 return moe_backward(x_bits, topk_idx, topk_prob, w_gu_bits, w_d_bits, dout_bits,
-                                    round_bf16, only_expert, c, want, threads=1, state=state)
+                                    round_bf16, only_expert, c, want, threads=1, state=state, scaled=scaled)
             with ThreadPoolExecutor(max_workers=len(chunks)) as ex:
                 parts = list(ex.map(one, chunks))
             return {key: (None if parts[0][key] is None else np.concatenate([q[key] for q in parts]))
@@ -374,11 +381,20 @@ def moe_backward(x_bits, topk_idx, topk_prob, w_gu_bits, w_d_bits, dout_bits, ro
     st = [None] * 4
     if state is not None:
         st = [_c(state["row_of"], np.int32), _c(state["gu"], np.uint16), _c(state["h"], np.uint16),
-              _c(state["y"], np.uint16)]
+              None if scaled else _c(state["y"], np.uint16)]
         rows = st[1].shape[0]
-        if st[0].shape != (T, k) or st[2].shape != (rows, I) or st[3].shape != (rows, H) or \
+        if st[0].shape != (T, k) or st[2].shape != (rows, I) or (not scaled and st[3].shape != (rows, H)) or \
                 st[1].shape != (rows, 2 * I) or (st[0].size and (st[0].min() < 0 or st[0].max() >= rows)):
             raise ValueError("moe_backward: state shapes do not match")
+    if scaled:
+        rc = lib.oracle_moe_backward_scaled(_p(x_bits), T, H, I, E, k, _p(topk_idx), _p(topk_prob),
+                                            _p(w_gu_bits), _p(w_d_bits), _p(dout_bits), int(round_bf16),
+                                            only_expert, _p(tl), 0 if tl is None else len(tl),
+                                            _p(st[0]), _p(st[1]), _p(st[2]),
+                                            _p(dx), _p(dwgu), _p(dwd), _p(dprob))
+        if rc:
+            raise ValueError(f"oracle_moe_backward_scaled failed ({rc})")
+        return dict(dx=dx, dw_gate_up=dwgu, dw_down=dwd, dprob=dprob)
     rc = lib.oracle_moe_backward_state(_p(x_bits), T, H, I, E, k, _p(topk_idx), _p(topk_prob),
                                        _p(w_gu_bits), _p(w_d_bits), _p(dout_bits), int(round_bf16),
                                        only_expert, _p(tl), 0 if tl is None else len(tl),

@@ -751,3 +751,130 @@ int oracle_moe_backward_state(const uint16_t* x, int64_t T, int H, int I, int E,
     free(g); free(u); free(h); free(y); free(dy); free(dh); free(dg); free(du);
     return 0;
 }
+
+/*
+ * oracle_moe_backward_scaled -- the gradients of the ScaledSwiGLU layer
+ * ([TE] Grouped MLP, scale_bias: the routing weight p multiplies the SwiGLU
+ * output before FC2, and the combine adds the expert outputs unweighted):
+ *   out_t = sum_j MLP'_{e_j}(x_t; p_j),  MLP'(x; p) = (p * silu(g) * u) . Wd.
+ * Per assignment (t, j), with s = silu(g) * u:
+ *   dy = dout_t;                dWd[e] += h^T dy   (h = p * s, as stored)
+ *   dh = dy . Wd[e]^T;          dprob[t,j] = <dh, s>
+ *   ds = p * dh;                dg = ds * u * silu'(g);  du = ds * silu(g)
+ *   dWgu[e][:, 0:I] += x_t^T dg;  dWgu[e][:, I:2I] += x_t^T du
+ *   dxp = dg . Wgu[e][:, 0:I]^T + du . Wgu[e][:, I:2I]^T;   dx_t += dxp
+ * All in fp64. With round_bf16, the stored tensors are bf16 as in
+ * oracle_moe_backward: h = bf16(p * s) from the forward's exact g and u; the
+ * backward reads g and u rounded to bf16 (so s in dprob and ds is formed from
+ * them); dg, du and each permuted row's dxp are rounded; dy = dout is bf16
+ * already. Unrounded, the layer equals the one with the weight applied in the
+ * combine (p (s . Wd) = (p s) . Wd), and so do all four gradients. A saved
+ * state (row_of != NULL) gives g, u and the stored h of each assignment's row,
+ * as in oracle_moe_backward_state. Other arguments as there.
+ */
+int oracle_moe_backward_scaled(const uint16_t* x, int64_t T, int H, int I, int E, int k,
+                               const int32_t* topk_idx, const float* topk_prob,
+                               const uint16_t* w_gate_up, const uint16_t* w_down, const uint16_t* dout,
+                               int round_bf16, int only_expert, const int64_t* token_list,
+                               int64_t n_tokens, const int32_t* row_of, const uint16_t* st_gu,
+                               const uint16_t* st_h,
+                               double* dx, double* dw_gate_up, double* dw_down, double* dprob)
+{
+    if (row_of && (!st_gu || !st_h)) return 3;
+    int64_t nt = token_list ? n_tokens : T;
+    if (dx) memset(dx, 0, sizeof(double) * (size_t)(nt * H));
+    if (dprob) memset(dprob, 0, sizeof(double) * (size_t)(nt * k));
+    int64_t n_dw = only_expert >= 0 ? 1 : E;
+    if (dw_gate_up) memset(dw_gate_up, 0, sizeof(double) * (size_t)(n_dw * H * 2 * I));
+    if (dw_down) memset(dw_down, 0, sizeof(double) * (size_t)(n_dw * I * H));
+    double* g = (double*)malloc(sizeof(double) * (size_t)I);
+    double* u = (double*)malloc(sizeof(double) * (size_t)I);
+    double* h = (double*)malloc(sizeof(double) * (size_t)I);
+    double* y = (double*)malloc(sizeof(double) * (size_t)H);
+    double* dy = (double*)malloc(sizeof(double) * (size_t)H);
+    double* dh = (double*)malloc(sizeof(double) * (size_t)I);
+    double* dg = (double*)malloc(sizeof(double) * (size_t)I);
+    double* du = (double*)malloc(sizeof(double) * (size_t)I);
+    int rc = 0;
+    for (int64_t n = 0; n < nt && rc == 0; n++) {
+        int64_t t = token_list ? token_list[n] : n;
+        const uint16_t* xt = x + t * H;
+        const uint16_t* dot = dout + t * H;
+        for (int j = 0; j < k; j++) {
+            int e = topk_idx[t * k + j];
+            if (e < 0 || e >= E) { rc = 2; break; }
+            if (only_expert >= 0 && e != only_expert) continue;
+            double p = (double)topk_prob[t * k + j];
+            const uint16_t* wgu = w_gate_up + (int64_t)e * H * 2 * I;
+            const uint16_t* wd = w_down + (int64_t)e * I * H;
+            if (row_of) {
+                int64_t r = row_of[t * k + j];
+                if (r < 0) { rc = 2; break; }
+                for (int i = 0; i < I; i++) {
+                    g[i] = bf16_to_double(st_gu[r * 2 * I + i]);
+                    u[i] = bf16_to_double(st_gu[r * 2 * I + I + i]);
+                    h[i] = bf16_to_double(st_h[r * I + i]);
+                }
+            } else {
+                /* the forward's exact g and u; the stored h is p * silu(g) * u */
+                oracle_expert_mlp(xt, 1, H, I, wgu, wd, 0, y, g, u, NULL);
+                for (int i = 0; i < I; i++) {
+                    double v = p * silu(g[i]) * u[i];
+                    h[i] = round_bf16 ? bf16_to_double(double_to_bf16(v)) : v;
+                }
+                if (round_bf16)
+                    for (int i = 0; i < I; i++) {
+                        g[i] = bf16_to_double(double_to_bf16(g[i]));
+                        u[i] = bf16_to_double(double_to_bf16(u[i]));
+                    }
+            }
+            for (int c = 0; c < H; c++) dy[c] = bf16_to_double(dot[c]);
+            if (dw_down) {
+                double* dwd = dw_down + (only_expert >= 0 ? 0 : (int64_t)e * I * H);
+                for (int i = 0; i < I; i++)
+                    for (int c = 0; c < H; c++) dwd[(int64_t)i * H + c] += h[i] * dy[c];
+            }
+            for (int i = 0; i < I; i++) {
+                double sum = 0.0;
+                for (int c = 0; c < H; c++) sum += bf16_to_double(wd[(int64_t)i * H + c]) * dy[c];
+                dh[i] = sum;
+            }
+            double dp = 0.0;
+            for (int i = 0; i < I; i++) {
+                double sg = 1.0 / (1.0 + exp(-g[i]));
+                double a = g[i] * sg;                      /* silu(g) */
+                dp += dh[i] * a * u[i];
+                double ds = p * dh[i];
+                du[i] = ds * a;
+                dg[i] = ds * u[i] * (sg + g[i] * sg * (1.0 - sg));
+                if (round_bf16) {
+                    du[i] = bf16_to_double(double_to_bf16(du[i]));
+                    dg[i] = bf16_to_double(double_to_bf16(dg[i]));
+                }
+            }
+            if (dprob) dprob[n * k + j] = dp;
+            if (dw_gate_up) {
+                double* dw = dw_gate_up + (only_expert >= 0 ? 0 : (int64_t)e * H * 2 * I);
+                for (int hh = 0; hh < H; hh++) {
+                    double xv = bf16_to_double(xt[hh]);
+                    double* row = dw + (int64_t)hh * 2 * I;
+                    for (int i = 0; i < I; i++) { row[i] += xv * dg[i]; row[I + i] += xv * du[i]; }
+                }
+            }
+            if (dx) {
+                double* dxr = dx + n * H;
+                for (int hh = 0; hh < H; hh++) {
+                    const uint16_t* row = wgu + (int64_t)hh * 2 * I;
+                    double sum = 0.0;
+                    for (int i = 0; i < I; i++)
+                        sum += dg[i] * bf16_to_double(row[i]) + du[i] * bf16_to_double(row[I + i]);
+                    if (round_bf16) sum = bf16_to_double(double_to_bf16(sum));
+                    dxr[hh] += sum;
+                }
+            }
+        }
+    }
+    free(g); free(u); free(h); free(y); free(dy); free(dh); free(dg); free(du);
+    return rc;
+}
+

@@ -283,3 +283,83 @@ def test_backward_state_shapes_are_checked(oracle_lib):
     with pytest.raises(ValueError):
         oracle_lib.moe_backward(bits(d["x"]), r["topk_idx"], r["topk_prob"], bits(d["w_gate_up"]),
                                 bits(d["w_down"]), bits(d["dout"]), state=s)
+
+
+def test_scaled_backward_equals_weighting_in_the_combine_when_exact(oracle_lib):
+    """ScaledSwiGLU (Transformer Engine Grouped MLP: the weight multiplies the
+    SwiGLU output before FC2, the combine is unweighted) is the same layer
+    as the weight applied in the combine, since FC2 is linear: p (s Wd) =
+    (p s) Wd. Without the bf16 roundings, its four gradients therefore equal
+    those of the weights-in-combine backward (itself pinned by finite
+    differences above)."""
+    w, d = setup(T=9, H=24, I=16, E=4, k=2, seed=11)
+    r = oracle_lib.router_topk(d["logits"].numpy(), w.k)
+    bits = oracle_lib.bf16_bits
+    args = (bits(d["x"]), r["topk_idx"], r["topk_prob"], bits(d["w_gate_up"]), bits(d["w_down"]),
+            bits(d["dout"]))
+    a = oracle_lib.moe_backward(*args, round_bf16=False)
+    b = oracle_lib.moe_backward(*args, round_bf16=False, scaled=True)
+    for key in ("dx", "dw_gate_up", "dw_down", "dprob"):
+        np.testing.assert_allclose(b[key], a[key], rtol=1e-10, atol=1e-12, err_msg=key)
+
+
+def test_scaled_backward_weight_gradient_by_finite_differences(oracle_lib):
+    """d out / d p of the ScaledSwiGLU layer: central differences in fp64 of
+    the layer restated with the weight on the SwiGLU output (torch
+    primitives on the exact bf16 inputs) against the oracle's dprob."""
+    w, d = setup(T=5, H=16, I=8, E=3, k=2, seed=12)
+    r = oracle_lib.router_topk(d["logits"].numpy(), w.k)
+    bits = oracle_lib.bf16_bits
+    x = d["x"].double()
+    wgu, wd, dout = d["w_gate_up"].double(), d["w_down"].double(), d["dout"].double()
+    idx = torch.from_numpy(r["topk_idx"]).long()
+
+    def loss(prob):
+        out = torch.zeros((w.T, w.H), dtype=torch.float64)
+        for t in range(w.T):
+            for j in range(w.k):
+                e = idx[t, j]
+                g = x[t] @ wgu[e][:, :w.I]
+                u = x[t] @ wgu[e][:, w.I:]
+                out[t] += (prob[t, j] * F.silu(g) * u) @ wd[e]
+        return float((dout * out).sum())
+
+    g = oracle_lib.moe_backward(bits(d["x"]), r["topk_idx"], r["topk_prob"], bits(d["w_gate_up"]),
+                                bits(d["w_down"]), bits(d["dout"]), round_bf16=False, scaled=True)
+    prob = torch.from_numpy(r["topk_prob"].astype(np.float64))
+    for t in range(w.T):
+        for j in range(w.k):
+            def f(delta):
+                q = prob.clone()
+                q[t, j] += delta
+                return loss(q)
+            fd = richardson(f, 1e-3)
+            assert abs(fd - g["dprob"][t, j]) <= 1e-8 * (1 + abs(fd)), (t, j, fd, g["dprob"][t, j])
+
+
+def test_scaled_backward_from_saved_state(oracle_lib):
+    """Given its own rounded scaled state (h = bf16(p silu(g) u) per row),
+    the saved-state mode of the scaled backward returns what the recomputing
+    mode returns."""
+    w, d = setup(T=12, H=24, I=16, E=4, k=2, seed=13)
+    r = oracle_lib.router_topk(d["logits"].numpy(), w.k)
+    bits = oracle_lib.bf16_bits
+    args = (bits(d["x"]), r["topk_idx"], r["topk_prob"], bits(d["w_gate_up"]), bits(d["w_down"]),
+            bits(d["dout"]))
+    s0 = _own_state(oracle_lib, w, d, r)
+    x, wgu = bits(d["x"]), bits(d["w_gate_up"])
+    st, row_of = oracle_lib.dispatch(r["topk_idx"], r["offsets"], w.E)
+    p_row = np.zeros(len(st))
+    p_row[row_of.ravel()] = r["topk_prob"].ravel()
+    offs = r["offsets"]
+    xp = oracle_lib.gather_rows(x, st)
+    for e in range(w.E):
+        a_, b_ = offs[e], offs[e + 1]
+        if b_ > a_:
+            _, ge, ue, _ = oracle_lib.expert_mlp(xp[a_:b_], wgu[e], bits(d["w_down"])[e], True, True)
+            sv = ge / (1 + np.exp(-ge)) * ue
+            s0["h"][a_:b_] = oracle_lib.round_bf16_array(p_row[a_:b_, None] * sv)
+    a = oracle_lib.moe_backward(*args, scaled=True)
+    b = oracle_lib.moe_backward(*args, scaled=True, state={"row_of": s0["row_of"], "gu": s0["gu"], "h": s0["h"]})
+    for key in ("dx", "dw_gate_up", "dw_down", "dprob"):
+        np.testing.assert_array_equal(a[key], b[key], err_msg=key)
