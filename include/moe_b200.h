@@ -296,9 +296,8 @@ moe_status moe_grouped_mlp(const moe_bf16* x_perm, int64_t A, const int32_t* off
  * so y_perm is already weighted ((p h) W2 = p (h W2), the page's identity for
  * FC2 without bias) and moe_unpermute_combine must then run with topk_prob
  * NULL. gu_save keeps the unscaled g and u. row_scale fp32 [A] (for example
- * moe_permute_padded's prob_perm; NULL: 1). The backward of this variant is
- * not provided: moe_grouped_mlp_backward differentiates the layer with the
- * weights applied in combine. Other arguments as in moe_grouped_mlp. */
+ * moe_permute_padded's prob_perm; NULL: 1). moe_grouped_mlp_scaled_backward
+ * is its backward. Other arguments as in moe_grouped_mlp. */
 moe_status moe_grouped_mlp_scaled(const moe_bf16* x_perm, int64_t A, const int32_t* offsets, int E,
                                   int H, int I, const moe_bf16* w_gate_up, const moe_bf16* w_down,
                                   const float* row_scale, moe_bf16* y_perm, moe_bf16* gu_save,
@@ -379,6 +378,43 @@ moe_status moe_grouped_mlp_backward(const moe_bf16* dout, int64_t T, int H, int 
                                     moe_bf16* dx, moe_bf16* dw_gate_up, moe_bf16* dw_down,
                                     float* dprob, void* workspace, size_t workspace_bytes,
                                     void* stream);
+
+/* moe_grouped_mlp_scaled_backward -- gradients of the ScaledSwiGLU layer (TE
+ * Grouped MLP, the routing weight applied to the activation before FC2):
+ *   out[t] = sum_j y_perm[row_of[t,j]],  y_perm[r] = bf16(p_r silu(g_r) u_r) . w_down[e]
+ * i.e. moe_grouped_mlp_scaled followed by moe_unpermute_combine with
+ * topk_prob NULL, with respect to x, w_gate_up, w_down and p:
+ *   dy[r] = dout[t]   (r = row_of[t,j]; a pad row: 0)
+ *   dh = dy . w_down[e]^T          dprob[t,j] = <dh, silu(g) * u>   (row r)
+ *   ds = p_r * dh                  du = ds * silu(g)    dg = ds * u * silu'(g)
+ *   dx_perm = [dg | du] . w_gate_up[e]^T       dx[t] = sum_j dx_perm[row_of[t,j]]
+ *   dw_down[e] = h_e^T . dy_e                  dw_gate_up[e] = x_e^T . [dg | du]_e
+ * The rows are those of the forward's dispatch, padded (moe_permute_padded)
+ * or not (moe_permute), A of them with offsets (padded_offsets) [E+1].
+ * Accumulation is fp32; dprob sums each 64-column group of dh * silu(g) * u
+ * in column order, then the groups in order, so it is the same on every run.
+ * An expert with no rows gets zero weight gradients.
+ *  dout          in  bf16 [T,H]
+ *  row_of        in  int32 [T,k]   row of each assignment
+ *  sorted_token  in  int32 [A]     token of each row, -1 for a pad row
+ *  row_scale     in  fp32 [A]      p of each row (prob_perm; 0 on pad rows)
+ *  x_perm        in  bf16 [A,H]    the forward's rows (pad rows zero)
+ *  gu            in  bf16 [A,2I]   the forward's unscaled g and u (gu_save)
+ *  h             in  bf16 [A,I]    the forward's scaled h (h_save)
+ *  dx out bf16 [T,H]; dw_gate_up out bf16 [E,H,2I]; dw_down out bf16 [E,I,H];
+ *  dprob out fp32 [T,k], the gradient of the routing weights (it reaches the
+ *  logits through the router's softmax or sigmoid, which is not done here);
+ *  workspace of moe_grouped_mlp_scaled_backward_workspace_size(A, H, I) bytes.
+ * A row index or token outside its range is recorded as MOE_ERR_DEVICE_CHECK. */
+size_t moe_grouped_mlp_scaled_backward_workspace_size(int64_t A, int H, int I);
+moe_status moe_grouped_mlp_scaled_backward(const moe_bf16* dout, int64_t T, int H, int I, int E, int k,
+                                           const moe_bf16* w_gate_up, const moe_bf16* w_down,
+                                           const int32_t* row_of, const int32_t* sorted_token,
+                                           const float* row_scale, const int32_t* offsets, int64_t A,
+                                           const moe_bf16* x_perm, const moe_bf16* gu, const moe_bf16* h,
+                                           moe_bf16* dx, moe_bf16* dw_gate_up, moe_bf16* dw_down,
+                                           float* dprob, void* workspace, size_t workspace_bytes,
+                                           void* stream);
 
 /* ------------------------------------------------------------ testing hooks
  * moe_testing_set_kernels -- forces one kernel variant for every later call in

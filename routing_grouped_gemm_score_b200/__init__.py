@@ -26,6 +26,7 @@ __all__ = [
     "MoEError", "RouterOpts", "SCORE_SOFTMAX", "SCORE_SIGMOID", "library_path", "lib",
     "moe_status_string", "moe_get_device_status", "moe_router_topk", "moe_permute",
     "moe_grouped_mlp", "moe_unpermute_combine", "moe_layer_forward", "moe_grouped_mlp_backward",
+    "moe_grouped_mlp_scaled_backward",
     "moe_trace_set", "moe_router_topk_noalloc", "moe_router_backward", "moe_expert_bias_update", "LayerWorkspace", "ABI_FUNCTIONS",
 ]
 
@@ -101,6 +102,9 @@ ABI_FUNCTIONS = {
     "moe_grouped_mlp_backward_workspace_size": (SZ, [I64, I32, I32, I32, I32]),
     "moe_grouped_mlp_backward": (I32, [P, I64, I32, I32, I32, I32, P, P, P, P, P, P, P, P, P, P, P,
                                        P, P, P, SZ, P]),
+    "moe_grouped_mlp_scaled_backward_workspace_size": (SZ, [I64, I32, I32]),
+    "moe_grouped_mlp_scaled_backward": (I32, [P, I64, I32, I32, I32, I32, P, P, P, P, P, P, I64, P, P, P,
+                                              P, P, P, P, P, SZ, P]),
     "moe_testing_set_kernels": (I32, [I32, I32, I32, I32]),
     "moe_testing_wait_timeout": (I32, [I64, P]),
 }
@@ -541,4 +545,45 @@ def moe_grouped_mlp_backward(dout: torch.Tensor, state: dict, w_gate_up: torch.T
         _ptr(s["topk_prob"]), _ptr(s["offsets"]), _ptr(s["x_perm"]), _ptr(s["gu"]), _ptr(s["h"]),
         _ptr(s["y_perm"]), _ptr(grads["dx"]), _ptr(grads["dw_gate_up"]), _ptr(grads["dw_down"]),
         _ptr(grads["dprob"]), _ptr(ws), ws.numel(), _stream()), "moe_grouped_mlp_backward")
+    return grads
+
+
+def moe_grouped_mlp_scaled_backward(dout: torch.Tensor, row_of: torch.Tensor, sorted_token: torch.Tensor,
+                                    row_scale: torch.Tensor, offsets: torch.Tensor, x_perm: torch.Tensor,
+                                    gu: torch.Tensor, h: torch.Tensor, w_gate_up: torch.Tensor,
+                                    w_down: torch.Tensor, grads: Optional[dict] = None,
+                                    workspace: Optional[torch.Tensor] = None) -> dict:
+    """Gradients of the ScaledSwiGLU layer (moe_grouped_mlp_scaled, then an
+    unweighted combine) with respect to x, w_gate_up, w_down and the routing
+    weights, from the forward's rows: x_perm, gu and h [A, ...] with their
+    sorted_token [A], row_scale [A] and offsets [E+1] (a padded dispatch's or
+    not), and row_of [T, k]."""
+    _need(dout, torch.bfloat16, "dout")
+    _need(row_of, torch.int32, "row_of")
+    _need(sorted_token, torch.int32, "sorted_token")
+    _need(row_scale, torch.float32, "row_scale")
+    _need(offsets, torch.int32, "offsets")
+    for t, n in ((x_perm, "x_perm"), (gu, "gu"), (h, "h"), (w_gate_up, "w_gate_up"), (w_down, "w_down")):
+        _need(t, torch.bfloat16, n)
+    T, H = dout.shape
+    E, _, I2 = w_gate_up.shape
+    I = I2 // 2
+    k = row_of.shape[1]
+    A = x_perm.shape[0]
+    dev = dout.device
+    if grads is None:
+        grads = {
+            "dx": torch.empty((T, H), dtype=torch.bfloat16, device=dev),
+            "dw_gate_up": torch.empty_like(w_gate_up),
+            "dw_down": torch.empty_like(w_down),
+            "dprob": torch.empty((T, k), dtype=torch.float32, device=dev),
+        }
+    ws = workspace
+    if ws is None:
+        ws = _workspace(lib().moe_grouped_mlp_scaled_backward_workspace_size(A, H, I), dev)
+    _check(lib().moe_grouped_mlp_scaled_backward(
+        _ptr(dout), T, H, I, E, k, _ptr(w_gate_up), _ptr(w_down), _ptr(row_of), _ptr(sorted_token),
+        _ptr(row_scale), _ptr(offsets), A, _ptr(x_perm), _ptr(gu), _ptr(h), _ptr(grads["dx"]),
+        _ptr(grads["dw_gate_up"]), _ptr(grads["dw_down"]), _ptr(grads["dprob"]), _ptr(ws), ws.numel(),
+        _stream()), "moe_grouped_mlp_scaled_backward")
     return grads

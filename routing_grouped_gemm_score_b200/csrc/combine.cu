@@ -9,7 +9,9 @@
 // writer and a fixed order of operations (shared first, then j ascending,
 // fp32). The results are the same on every run, unlike a scatter-add with
 // atomics. Rows move as 16-byte vectors of 8 bf16; a lane issues the k loads
-// of its column chunks together.
+// of its column chunks together. Also the two steps of the ScaledSwiGLU
+// backward around its GEMMs: the row gather of the output gradient and the
+// sum of the routing-weight gradient's partials.
 #include <cstdlib>
 
 #include "moe_common.cuh"
@@ -230,7 +232,78 @@ int64_t warp_kernel_blocks(K kern, int64_t T) {
     return (warps + kWarpKernelThreads / 32 - 1) / (kWarpKernelThreads / 32);
 }
 
+// ScaledSwiGLU backward, the combine's gradient: the combine adds the rows
+// unweighted, so each row's gradient is its token's output gradient,
+// dy[r] = dout[sorted_token[r]], and a pad row (sorted_token -1) gets zeros.
+// One warp per row, rows [0, offsets[E]) -- one writer per row, in row order.
+__global__ void __launch_bounds__(kWarpKernelThreads)
+    gather_rows_kernel(const uint4* __restrict__ dout, const int32_t* __restrict__ sorted_token, int64_t T,
+                       const int32_t* __restrict__ offsets, int E, int64_t A, int H8, uint4* __restrict__ dy,
+                       unsigned* err) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    int64_t rows = __ldg(offsets + E);
+    if (rows > A || rows < 0) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) raise_error(err, kErrDeviceCheck);
+        rows = rows < 0 ? 0 : A;
+    }
+    for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows; r += nwarps) {
+        int64_t t = __ldg(sorted_token + r);
+        if (t >= T) {
+            if (lane == 0) raise_error(err, kErrDeviceCheck);
+            t = -1;
+        }
+        for (int c = lane; c < H8; c += 32)
+            dy[r * H8 + c] = t >= 0 ? __ldg(dout + t * H8 + c) : make_uint4(0, 0, 0, 0);
+    }
+}
+
+// dprob[i] = sum_q row_dot[row_of[i] * nq + q], q ascending: the gradient of
+// each routing weight from the per-64-column partial sums that the ScaledSwiGLU
+// backward epilogue wrote. One thread per assignment; a fixed order, so the
+// result is the same on every run.
+__global__ void __launch_bounds__(256)
+    row_dot_sum_kernel(const float* __restrict__ row_dot, int nq, const int32_t* __restrict__ row_of, int64_t n,
+                       int64_t A, float* __restrict__ dprob, unsigned* err) {
+    pdl_wait();
+    pdl_launch_dependents();
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = __ldg(row_of + i);
+        if (r < 0 || r >= A) {
+            raise_error(err, kErrDeviceCheck);
+            dprob[i] = 0.0f;
+            continue;
+        }
+        const float* src = row_dot + r * nq;
+        float sum = 0.0f;
+#pragma unroll 8
+        for (int q = 0; q < nq; ++q) sum += __ldg(src + q);
+        dprob[i] = sum;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_gather_rows(const bf16* dout, const int32_t* sorted_token, int64_t T, const int32_t* offsets,
+                               int E, int64_t A, int H, bf16* dy, cudaStream_t st, unsigned* err) {
+    if (A == 0) return cudaSuccess;
+    const int64_t blocks = warp_kernel_blocks(gather_rows_kernel, A);
+    return launch_chained(gather_rows_kernel, dim3((unsigned)blocks), dim3(kWarpKernelThreads), 0, st,
+                          reinterpret_cast<const uint4*>(dout), sorted_token, T, offsets, E, A, H / 8,
+                          reinterpret_cast<uint4*>(dy), err);
+}
+
+cudaError_t launch_row_dot_sum(const float* row_dot, int nq, const int32_t* row_of, int64_t n, int64_t A,
+                               float* dprob, cudaStream_t st, unsigned* err) {
+    if (n == 0) return cudaSuccess;
+    int64_t blocks = (n + 255) / 256;
+    const int64_t cap = (int64_t)sm_count() * 8;
+    if (blocks > cap) blocks = cap;
+    return launch_chained(row_dot_sum_kernel, dim3((unsigned)blocks), dim3(256), 0, st, row_dot, nq, row_of, n, A,
+                          dprob, err);
+}
 
 cudaError_t launch_combine(const bf16* y_perm, const int32_t* row_of, const float* probs,
                            int64_t T, int k, int H, int64_t A, const bf16* shared, bf16* out,

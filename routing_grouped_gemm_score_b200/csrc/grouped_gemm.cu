@@ -96,7 +96,11 @@ struct Params {
     int64_t ld_aux;
     int I;                     // SwiGLU: offset of the up half in [g | u]
     int tma_out, tma_out2;     // single-CTA kernel: out / out2 have TMA store maps
-    const float* row_scale;    // SwiGLU forward: h[r] *= row_scale[r] (NULL: 1)
+    const float* row_scale;    // SwiGLU forward: h[r] *= row_scale[r]; backward: ds = row_scale[r] * dh (NULL: 1)
+    // SwiGLU backward with row_scale: row_dot[r * ld_row_dot + c / 64] = the sum
+    // over the 64 columns c.. of dh * silu(g) * u, in column order (NULL: skip)
+    float* row_dot;
+    int64_t ld_row_dot;
     // group-M, single CTA: A row r is row gather_tok[r] of gather_x [gather_T][K]
     // (-1: a zero row) instead of a TMA tile of A (NULL: TMA)
     const bf16* gather_x;
@@ -398,8 +402,13 @@ __device__ __forceinline__ void put_block32_packed(uint8_t* buf, bf16* dst, int6
 }
 
 // SwiGLU backward for 32 columns: from dh and the saved g, u, the bf16 dg and
-// du, packed in pairs (dg in dgp, du in dup).
-__device__ __forceinline__ void swiglu_bwd32(const float* dh, const Aux32& a, uint32_t* dgp, uint32_t* dup) {
+// du, packed in pairs (dg in dgp, du in dup). SCALED (ScaledSwiGLU, where the
+// forward stored h = p * silu(g) * u): the gradient reaching silu(g) * u is
+// ds = p * dh, and dot gains sum_c dh[c] * silu(g[c]) * u[c] (the gradient of
+// p), in column order.
+template <bool SCALED>
+__device__ __forceinline__ void swiglu_bwd32(const float* dh, const Aux32& a, float p, float& dot, uint32_t* dgp,
+                                             uint32_t* dup) {
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const uint32_t gw[4] = {a.g[q].x, a.g[q].y, a.g[q].z, a.g[q].w};
@@ -413,9 +422,16 @@ __device__ __forceinline__ void swiglu_bwd32(const float* dh, const Aux32& a, ui
             // as the IEEE division 1.0f / x
             const float s0 = __frcp_rn(1.0f + expf(-gf.x));
             const float s1 = __frcp_rn(1.0f + expf(-gf.y));
-            dup[c / 2] = pack_bf16x2(dh[c] * gf.x * s0, dh[c + 1] * gf.y * s1);
-            dgp[c / 2] = pack_bf16x2(dh[c] * uf.x * (s0 + gf.x * s0 * (1.0f - s0)),
-                                     dh[c + 1] * uf.y * (s1 + gf.y * s1 * (1.0f - s1)));
+            float d0 = dh[c], d1 = dh[c + 1];
+            if (SCALED) {
+                dot += d0 * (gf.x * s0 * uf.x);
+                dot += d1 * (gf.y * s1 * uf.y);
+                d0 *= p;
+                d1 *= p;
+            }
+            dup[c / 2] = pack_bf16x2(d0 * gf.x * s0, d1 * gf.y * s1);
+            dgp[c / 2] = pack_bf16x2(d0 * uf.x * (s0 + gf.x * s0 * (1.0f - s0)),
+                                     d1 * uf.y * (s1 + gf.y * s1 * (1.0f - s1)));
         }
     }
 }
@@ -499,6 +515,10 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
         const int64_t grow = (int64_t)t.row0 + r;
         const int64_t row0 = (int64_t)t.row0 + warp_r0;
         Aux32& ax = *pre;   // reloaded in place for each later chunk
+        // ScaledSwiGLU: the row's routing weight, and the partial gradient of
+        // it over each 64-column group (em.c_lo is a multiple of 64)
+        const float ps = (p.row_scale && valid) ? __ldg(p.row_scale + grow) : 1.0f;
+        float dot = 0.0f;
 #pragma unroll 1
         for (int ci = 0; ci < em.chunks; ++ci) {
             const int col = n0 + em.c_lo + 32 * ci;
@@ -508,7 +528,15 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
             const int ncols = min(32, p.N - col);
             uint32_t dgp[16], dup[16];
             if (valid) {
-                swiglu_bwd32(dh, ax, dgp, dup);
+                if (p.row_dot) {
+                    swiglu_bwd32<true>(dh, ax, ps, dot, dgp, dup);
+                    if ((ci & 1) || col + 32 >= p.N) {   // the group's last chunk
+                        p.row_dot[grow * p.ld_row_dot + (col >> 6)] = dot;
+                        dot = 0.0f;
+                    }
+                } else {
+                    swiglu_bwd32<false>(dh, ax, 1.0f, dot, dgp, dup);
+                }
             } else {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) dgp[i] = dup[i] = 0u;   // rows past the block: not stored
@@ -1638,7 +1666,7 @@ cudaError_t gemm_down(const bf16* h, int64_t rows, const int32_t* offsets, int E
 
 cudaError_t gemm_down_dgrad_swiglu(const bf16* dy, int64_t rows, const int32_t* offsets, int E,
                                    int H, int I, const bf16* w_down, const bf16* gu, bf16* dgu,
-                                   cudaStream_t st, unsigned* err) {
+                                   cudaStream_t st, unsigned* err, const float* row_scale, float* row_dot) {
     if (rows == 0) return cudaSuccess;
     CUtensorMap ta, ta64, tb;
     if (!make_map_2d(&ta, dy, H, rows, H, BK, 128)) return cudaErrorInvalidValue;
@@ -1657,6 +1685,11 @@ cudaError_t gemm_down_dgrad_swiglu(const bf16* dy, int64_t rows, const int32_t* 
     p.ldo = 2 * (int64_t)I;
     p.aux = gu;
     p.ld_aux = 2 * (int64_t)I;
+    if (row_dot) {
+        p.row_scale = row_scale;
+        p.row_dot = row_dot;
+        p.ld_row_dot = (I + 63) / 64;
+    }
     CUtensorMap tc;
     if (!make_out_map(&tc, dgu, rows, 2 * (uint64_t)I)) return cudaErrorInvalidValue;
     return launch_group_m<kEpiSwigluBwd, false>(ta, ta64, tb, tb1, p, st, &tc);

@@ -145,6 +145,23 @@ BwdLayout bwd_layout(void* ws, int64_t T, int H, int I, int k) {
     return L;
 }
 
+struct ScaledBwdLayout {
+    bf16 *dy, *dgu, *dx_perm;
+    float* row_dot;
+    size_t bytes;
+};
+
+ScaledBwdLayout scaled_bwd_layout(void* ws, int64_t A, int H, int I) {
+    Carver c(ws);
+    ScaledBwdLayout L;
+    L.dy = c.take<bf16>((size_t)A * H);
+    L.dgu = c.take<bf16>((size_t)A * 2 * I);
+    L.dx_perm = c.take<bf16>((size_t)A * H);
+    L.row_dot = c.take<float>((size_t)A * ((I + 63) / 64));
+    L.bytes = c.bytes();
+    return L;
+}
+
 }  // namespace
 
 unsigned* device_error_word() {
@@ -661,6 +678,62 @@ moe_status moe_grouped_mlp_backward(const moe_bf16* dout, int64_t T, int H, int 
     if (e == cudaSuccess)
         e = gemm_wgrad(B(x_perm), L.dgu, A, offsets, E, H, 2 * I,
                        reinterpret_cast<bf16*>(dw_gate_up), st, err);
+    if (e == cudaSuccess) e = trace_mark(6, st);
+    return from_cuda(e);
+}
+
+size_t moe_grouped_mlp_scaled_backward_workspace_size(int64_t A, int H, int I) {
+    if (A < 0 || A >= (int64_t(1) << 31) || !dims_ok(H, I)) return 0;
+    return scaled_bwd_layout(nullptr, A, H, I).bytes;
+}
+
+moe_status moe_grouped_mlp_scaled_backward(const moe_bf16* dout, int64_t T, int H, int I, int E, int k,
+                                           const moe_bf16* w_gate_up, const moe_bf16* w_down,
+                                           const int32_t* row_of, const int32_t* sorted_token,
+                                           const float* row_scale, const int32_t* offsets, int64_t A,
+                                           const moe_bf16* x_perm, const moe_bf16* gu, const moe_bf16* h,
+                                           moe_bf16* dx, moe_bf16* dw_gate_up, moe_bf16* dw_down,
+                                           float* dprob, void* workspace, size_t workspace_bytes,
+                                           void* stream) {
+    const ChainScope chain(A <= kChainMaxRows);
+    if (!shape_ok(T, E, k) || H <= 0 || I <= 0) return MOE_ERR_INVALID_ARG;
+    if (A < T * (int64_t)k || A >= (int64_t(1) << 31)) return MOE_ERR_INVALID_ARG;   // each assignment has a row
+    if (!dims_ok(H, I)) return MOE_ERR_UNSUPPORTED;
+    const void* must[] = {dout, w_gate_up, w_down, row_of, sorted_token, row_scale, offsets, x_perm, gu, h,
+                          dx, dw_gate_up, dw_down, dprob};
+    for (const void* p : must)
+        if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+    const ScaledBwdLayout L0 = scaled_bwd_layout(nullptr, A, H, I);
+    if (!workspace || workspace_bytes < L0.bytes) return MOE_ERR_WORKSPACE;
+    unsigned* err = device_error_word();
+    if (!err) return MOE_ERR_CUDA;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const ScaledBwdLayout L = scaled_bwd_layout(workspace, A, H, I);
+    auto B = [](const moe_bf16* p) { return reinterpret_cast<const bf16*>(p); };
+    cudaError_t e = trace_mark(0, st);
+    if (A > 0) {
+        if (e == cudaSuccess)
+            e = launch_gather_rows(B(dout), sorted_token, T, offsets, E, A, H, L.dy, st, err);
+        if (e == cudaSuccess) e = trace_mark(1, st);
+        if (e == cudaSuccess)
+            e = gemm_down_dgrad_swiglu(L.dy, A, offsets, E, H, I, B(w_down), B(gu), L.dgu, st, err, row_scale,
+                                       L.row_dot);
+        if (e == cudaSuccess)
+            e = launch_row_dot_sum(L.row_dot, (I + 63) / 64, row_of, T * (int64_t)k, A, dprob, st, err);
+        if (e == cudaSuccess) e = trace_mark(2, st);
+        if (e == cudaSuccess)
+            e = gemm_gate_up_dgrad(L.dgu, A, offsets, E, H, I, B(w_gate_up), L.dx_perm, st, err);
+        if (e == cudaSuccess) e = trace_mark(3, st);
+        if (e == cudaSuccess && T > 0)
+            e = launch_combine(L.dx_perm, row_of, nullptr, T, k, H, A, nullptr, reinterpret_cast<bf16*>(dx), st,
+                               err);
+        if (e == cudaSuccess) e = trace_mark(4, st);
+    }
+    if (e == cudaSuccess)
+        e = gemm_wgrad(B(h), L.dy, A, offsets, E, I, H, reinterpret_cast<bf16*>(dw_down), st, err);
+    if (e == cudaSuccess) e = trace_mark(5, st);
+    if (e == cudaSuccess)
+        e = gemm_wgrad(B(x_perm), L.dgu, A, offsets, E, H, 2 * I, reinterpret_cast<bf16*>(dw_gate_up), st, err);
     if (e == cudaSuccess) e = trace_mark(6, st);
     return from_cuda(e);
 }

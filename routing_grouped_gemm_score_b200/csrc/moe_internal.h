@@ -116,6 +116,12 @@ cudaError_t launch_combine(const bf16* y_perm, const int32_t* row_of, const floa
 cudaError_t launch_combine_backward(const bf16* dout, const bf16* y_perm, const int32_t* row_of,
                                     const float* probs, int64_t T, int k, int H, int64_t A,
                                     bf16* dy_perm, float* dprob, cudaStream_t st, unsigned* err);
+// dy[r] = dout[sorted_token[r]] for r < offsets[E] (-1: a zero row).
+cudaError_t launch_gather_rows(const bf16* dout, const int32_t* sorted_token, int64_t T, const int32_t* offsets,
+                               int E, int64_t A, int H, bf16* dy, cudaStream_t st, unsigned* err);
+// dprob[i] = sum_{q < nq} row_dot[row_of[i] * nq + q], q ascending.
+cudaError_t launch_row_dot_sum(const float* row_dot, int nq, const int32_t* row_of, int64_t n, int64_t A,
+                               float* dprob, cudaStream_t st, unsigned* err);
 
 // ---------------------------------------------------------------- GEMMs
 // Grouped GEMMs on tcgen05. Each returns cudaErrorInvalidValue if a tensor
@@ -142,10 +148,15 @@ bool grouped_gemm_single_tiles(int64_t rows, int groups);
 // down: y[r] = h[r] Wd[e]
 cudaError_t gemm_down(const bf16* h, int64_t rows, const int32_t* offsets, int E, int H, int I,
                       const bf16* w_down, bf16* y, cudaStream_t st, unsigned* err, int64_t max_group_rows = 0);
-// dgrad of down with SwiGLU backward: dh = dy Wd[e]^T, then dgu = [dg | du]
+// dgrad of down with SwiGLU backward: dh = dy Wd[e]^T, then dgu = [dg | du].
+// ScaledSwiGLU (row_dot non-NULL): the forward's h[r] was scaled by
+// row_scale[r], so [dg | du] is taken from row_scale[r] * dh, and
+// row_dot [rows][ceil(I/64)] gets each 64-column group's sum of
+// dh * silu(g) * u (the routing weight's gradient, in parts).
 cudaError_t gemm_down_dgrad_swiglu(const bf16* dy, int64_t rows, const int32_t* offsets, int E,
                                    int H, int I, const bf16* w_down, const bf16* gu, bf16* dgu,
-                                   cudaStream_t st, unsigned* err);
+                                   cudaStream_t st, unsigned* err, const float* row_scale = nullptr,
+                                   float* row_dot = nullptr);
 // dgrad of gate_up: dx_perm = dgu Wgu[e]^T
 cudaError_t gemm_gate_up_dgrad(const bf16* dgu, int64_t rows, const int32_t* offsets, int E, int H,
                                int I, const bf16* w_gate_up, bf16* dx_perm, cudaStream_t st,

@@ -101,6 +101,17 @@ def test_invalid_arguments_are_rejected_without_a_device(built):
     assert l.moe_grouped_mlp_backward(fake, 10, 128, 128, 8, 2, fake, fake, fake, fake, fake, fake,
                                       None, fake, fake, fake, fake, fake, fake, fake, 1 << 30,
                                       None) == 1
+    # ScaledSwiGLU backward: fewer rows than assignments, a missing sorted_token,
+    # a workspace too small, I not a multiple of 8
+    sb = l.moe_grouped_mlp_scaled_backward
+    assert sb(fake, 10, 128, 128, 8, 2, fake, fake, fake, fake, fake, fake, 19, fake, fake, fake,
+              fake, fake, fake, fake, fake, 1 << 30, None) == 1
+    assert sb(fake, 10, 128, 128, 8, 2, fake, fake, fake, None, fake, fake, 20, fake, fake, fake,
+              fake, fake, fake, fake, fake, 1 << 30, None) == 1
+    assert sb(fake, 10, 128, 128, 8, 2, fake, fake, fake, fake, fake, fake, 20, fake, fake, fake,
+              fake, fake, fake, fake, fake, 16, None) == 4
+    assert sb(fake, 10, 128, 100, 8, 2, fake, fake, fake, fake, fake, fake, 20, fake, fake, fake,
+              fake, fake, fake, fake, fake, 1 << 30, None) == 2
 
 
 def test_workspace_sizes_are_consistent(built):
@@ -119,3 +130,6 @@ def test_workspace_sizes_are_consistent(built):
     assert a >= A * 2048 * 2 * 2 + A * 768 * 2
     assert b > a
     assert l.moe_grouped_mlp_backward_workspace_size(4096, 2048, 768, 128, 8) >= A * (2048 * 4 + 1536 * 2)
+    # dy, dgu, dx_perm and the fp32 partials of dprob (one per 64 columns of I)
+    assert l.moe_grouped_mlp_scaled_backward_workspace_size(A, 2048, 768) >= A * (2048 * 4 + 1536 * 2 + 12 * 4)
+    assert l.moe_grouped_mlp_scaled_backward_workspace_size(A, 2048, 100) == 0
