@@ -123,9 +123,9 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
 template <int STAGES, int STAGE_BYTES>
 struct __align__(1024) Smem {
     uint8_t stage[STAGES][STAGE_BYTES];
-    // per epilogue warp: 32 rows x 32 bf16 (rows padded to 80 B for store_rows;
-    // a TMA block uses the first 2 KB), each on a 512-byte boundary
-    uint8_t epi[kEpiWarps][32 * 80];
+    // per epilogue warp: 32 rows x 32 bf16 in the 64-byte swizzle of stage64_off
+    // (row stores and TMA stores alike), each on a 512-byte boundary
+    uint8_t epi[kEpiWarps][32 * 64];
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
     uint64_t ready[STAGES];   // group-K: the stage's ragged rows are zeroed
@@ -140,10 +140,11 @@ struct __align__(1024) Smem {
 };
 using Smem1 = Smem<STAGES1, kStage1>;
 using SmemP = Smem<STAGESP, kStageP>;
-static_assert(offsetof(Smem1, epi) % 512 == 0 && offsetof(SmemP, epi) % 512 == 0 && (32 * 80) % 512 == 0,
+static_assert(offsetof(Smem1, epi) % 512 == 0 && offsetof(SmemP, epi) % 512 == 0 && (32 * 64) % 512 == 0,
               "64-byte-swizzled staging blocks start on 512-byte boundaries");
 constexpr size_t kSmem1Bytes = sizeof(Smem1) + 1024;  // + alignment slack
 constexpr size_t kSmemPBytes = sizeof(SmemP) + 1024;
+static_assert(kSmem1Bytes <= 227 * 1024 && kSmemPBytes <= 227 * 1024, "shared memory per CTA");
 
 // Shared-memory matrix descriptor: 128-byte swizzle, sm_100 version bit.
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -250,9 +251,10 @@ __device__ __forceinline__ Tile decode_tile(const S& s, const Params& p, int id,
 
 // First column of chunk c (64 columns) of an N-major weight tile. The SwiGLU
 // forward takes a tile's gate columns and the matching up columns, so that one
-// accumulator holds both. Single CTA: chunks 0..3 of a 256-column tile. Pair,
-// 256-row tile: CTA 0 the 128 gate columns, CTA 1 the matching up columns;
-// 128-row tile: each CTA 64 gate columns and their up columns.
+// accumulator holds both. Single CTA: chunks 0..3 of a 256-column tile (128
+// gate columns, then their up columns). Pair: each CTA 64 gate columns and
+// their up columns (CTA 0 the tile's first 64 columns of h, CTA 1 the next),
+// for 256-row and 128-row tiles alike.
 template <int EPI>
 __device__ __forceinline__ int b_col_1cta(const Tile& t, const Params& p, int c) {
     if (EPI == kEpiSwiglu) {
@@ -263,12 +265,8 @@ __device__ __forceinline__ int b_col_1cta(const Tile& t, const Params& p, int c)
 }
 
 template <int EPI>
-__device__ __forceinline__ int b_col_pair(const Tile& t, const Params& p, uint32_t rank, int c, bool half) {
-    if (EPI == kEpiSwiglu) {
-        const int n0 = t.n_blk * (BN / 2);
-        if (half) return (c == 0 ? 0 : p.I) + n0 + 64 * (int)rank;
-        return (rank == 0 ? n0 : p.I + n0) + 64 * c;
-    }
+__device__ __forceinline__ int b_col_pair(const Tile& t, const Params& p, uint32_t rank, int c) {
+    if (EPI == kEpiSwiglu) return (c == 0 ? 0 : p.I) + t.n_blk * (BN / 2) + 64 * (int)rank;
     return t.n_blk * BN + (int)rank * 128 + 64 * c;
 }
 
@@ -281,33 +279,39 @@ __device__ __forceinline__ uint32_t stage64_off(int r, int q) {
     return (uint32_t)(r * 64 + ((q ^ ((r >> 1) & 3)) << 4));
 }
 
-// Writes NC (32 or 64) values of each lane's row -- lane = row of the warp's
-// 32-row group -- as bf16 to rows [0, nvalid) at dst (row stride ld elements),
-// through the warp's staging buffer: each lane writes its row into shared
-// memory, then the warp reads it back so that one store instruction covers
-// whole row segments of 128 (NC=64) or 64 (NC=32) contiguous bytes. Rows are
-// padded by 16 bytes, so neither phase has more than 2-way bank conflicts.
-// Warp-collective.
-template <int NC>
-__device__ __forceinline__ void store_rows(uint8_t* buf, bf16* dst, int64_t ld, int nvalid, int ncols,
-                                           const float* v, int lane) {
-    constexpr int kChunks = NC / 8;              // 16-byte chunks per row
-    constexpr int kRowsPerPass = 32 / kChunks;   // rows one instruction covers
-    constexpr int kPitch = NC * 2 + 16;          // padded row pitch of the buffer
+// Writes the 32 values of each lane's row, packed as bf16 pairs (16 words) --
+// lane = row of the warp's 32-row group -- to rows [0, nvalid) and columns
+// [0, ncols) at dst (row stride ld elements), through the warp's 2 KB staging
+// block: each lane writes its row into shared memory, then the warp reads it
+// back so that one store instruction covers whole 64-byte row segments. The
+// block uses the 64-byte swizzle of stage64_off, so neither phase has bank
+// conflicts. Warp-collective.
+__device__ __forceinline__ void store_rows_packed32(uint8_t* buf, bf16* dst, int64_t ld, int nvalid, int ncols,
+                                                    const uint32_t* w, int lane) {
 #pragma unroll
-    for (int q = 0; q < kChunks; ++q)
-        *reinterpret_cast<uint4*>(buf + lane * kPitch + q * 16) =
-            make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                       pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+    for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4*>(buf + stage64_off(lane, q)) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
     __syncwarp();
-    const int chunk = lane % kChunks;
+    // rows lane / 4 + 8 * pass: the same swizzle term ((row >> 1) & 3) in every pass
+    const int chunk = lane % 4;
+    const uint8_t* src = buf + stage64_off(lane / 4, chunk);
+    bf16* out = dst + (int64_t)(lane / 4) * ld + chunk * 8;
+    const bool col_ok = chunk * 8 < ncols;
 #pragma unroll
-    for (int pass = 0; pass < kChunks; ++pass) {
-        const int row = pass * kRowsPerPass + lane / kChunks;
-        const uint4 w = *reinterpret_cast<const uint4*>(buf + row * kPitch + chunk * 16);
-        if (row < nvalid && chunk * 8 < ncols) *reinterpret_cast<uint4*>(dst + (int64_t)row * ld + chunk * 8) = w;
+    for (int pass = 0; pass < 4; ++pass) {
+        const uint4 v = *reinterpret_cast<const uint4*>(src + pass * 8 * 64);
+        if (pass * 8 + lane / 4 < nvalid && col_ok) *reinterpret_cast<uint4*>(out + (int64_t)pass * 8 * ld) = v;
     }
     __syncwarp();   // the buffer is free again
+}
+
+// store_rows_packed32 for fp32 values (rounded to bf16).
+__device__ __forceinline__ void store_rows32(uint8_t* buf, bf16* dst, int64_t ld, int nvalid, int ncols,
+                                             const float* v, int lane) {
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+    store_rows_packed32(buf, dst, ld, nvalid, ncols, w, lane);
 }
 
 // Writes a 32 x 32 block (lane = row) of bf16 at dst. With an output tensor
@@ -335,7 +339,7 @@ __device__ __forceinline__ void put_block32(uint8_t* buf, bf16* dst, int64_t ld,
         }
         __syncwarp();
     } else {
-        store_rows<32>(buf, dst, ld, nvalid, ncols, v, lane);
+        store_rows32(buf, dst, ld, nvalid, ncols, v, lane);
     }
 }
 
@@ -357,24 +361,6 @@ __device__ __forceinline__ void load_aux32(const Params& p, int64_t grow, int co
         a.g[q] = in ? __ldg(gs + q) : make_uint4(0, 0, 0, 0);
         a.u[q] = in ? __ldg(us + q) : make_uint4(0, 0, 0, 0);
     }
-}
-
-// store_rows<32> for values already packed as bf16 pairs (16 per lane).
-__device__ __forceinline__ void store_rows_packed32(uint8_t* buf, bf16* dst, int64_t ld, int nvalid, int ncols,
-                                                    const uint32_t* w, int lane) {
-    constexpr int kPitch = 32 * 2 + 16;
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4*>(buf + lane * kPitch + q * 16) = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-    __syncwarp();
-    const int chunk = lane % 4;
-#pragma unroll
-    for (int pass = 0; pass < 4; ++pass) {
-        const int row = pass * 8 + lane / 4;
-        const uint4 v = *reinterpret_cast<const uint4*>(buf + row * kPitch + chunk * 16);
-        if (row < nvalid && chunk * 8 < ncols) *reinterpret_cast<uint4*>(dst + (int64_t)row * ld + chunk * 8) = v;
-    }
-    __syncwarp();
 }
 
 // put_block32 for values already packed as bf16 pairs.
@@ -453,6 +439,15 @@ template <int EPI>
 __device__ __forceinline__ EpiMap full_map(int warp_r0, int col_half) {
     if (EPI == kEpiSwiglu) return EpiMap{warp_r0, 64 * col_half, 2, 64 * col_half, BN / 2};
     return EpiMap{warp_r0, 128 * col_half, 4, 128 * col_half, 0};
+}
+
+// full_map for a 256-row pair tile: its SwiGLU accumulator holds
+// [g 64 | u 64] of the tile's first 64 columns of h (CTA 0's weights), then
+// the same for the next 64 (CTA 1's).
+template <int EPI>
+__device__ __forceinline__ EpiMap pair_full_map(int warp_r0, int col_half) {
+    if (EPI == kEpiSwiglu) return EpiMap{warp_r0, 64 * col_half, 2, 128 * col_half, 64};
+    return full_map<EPI>(warp_r0, col_half);
 }
 
 // A 128-row pair tile (M = 128 across the two CTAs): each CTA's accumulator
@@ -662,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t keep = l2_policy_evict_last();   // A panels are read by every N block
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t issued[STAGESP] = {0, 0, 0, 0, 0, 0};
+            uint32_t loads = 0;   // stage loads issued; load j used stage j % STAGESP
             bool ok = true;
             for (int id = cluster; id < total && ok; id += clusters) {
                 const Tile t = decode_tile<false>(s, p, id, BMP);
@@ -683,13 +678,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (B_MN) {
 #pragma unroll
                         for (int c = 0; c < 2; ++c)
-                            tma_load_3d_pair(&tmB, bar, b_s + c * kChunkBytes, b_col_pair<EPI>(t, p, rank, c, half),
+                            tma_load_3d_pair(&tmB, bar, b_s + c * kChunkBytes, b_col_pair<EPI>(t, p, rank, c),
                                              kb * BK, t.g);
                     } else {
                         tma_load_3d_pair(&tmB, bar, b_s, kb * BK, t.n_blk * BN + (int)rank * 128,
                                          t.g);
                     }
-                    issued[stage] += 1;
+                    ++loads;
                     if (++stage == STAGESP) {
                         stage = 0;
                         phase ^= 1u;
@@ -699,7 +694,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // the leader waits for every load it armed to land before it may exit
             if (rank == 0)
                 for (int i = 0; i < STAGESP; ++i)
-                    if (issued[i]) mbar_wait(&s.full[i], (issued[i] - 1) & 1u, abort_flag, p.err);
+                    if (loads > (uint32_t)i)   // the stage's last load is its ((loads - 1 - i) / S)-th use
+                        mbar_wait(&s.full[i], ((loads - 1 - (uint32_t)i) / STAGESP) & 1u, abort_flag, p.err);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer (leader)
@@ -758,16 +754,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------ epilogue (both CTAs)
         const int quarter = warp & 3;                           // TMEM lanes 32*quarter .. +31
         const int col_half = (warp - 2) / 4;
-        const EpiMap em_full = full_map<EPI>((int)rank * 128 + quarter * 32, col_half);
+        const EpiMap em_full = pair_full_map<EPI>((int)rank * 128 + quarter * 32, col_half);
         const EpiMap em_half = half_map<EPI>(rank, quarter, col_half);
-        const uint32_t leader_acc_empty[2] = {mapa_shared(smem_u32(&s.acc_empty[0]), 0),
-                                              mapa_shared(smem_u32(&s.acc_empty[1]), 0)};
+        // the leader's barrier of buffer b (computed, not indexed, so that it stays in registers)
+        auto leader_acc_empty = [&](int b) { return mapa_shared(smem_u32(&s.acc_empty[b]), 0); };
         int local_tile = 0;
         for (int id = cluster; id < total; id += clusters, ++local_tile) {
             const Tile t = decode_tile<false>(s, p, id, BMP);
             const int buf = local_tile & 1;
             const uint32_t use = (uint32_t)(local_tile >> 1);
-            const EpiMap& em = t.rows <= 128 ? em_half : em_full;
+            const EpiMap em = t.rows <= 128 ? em_half : em_full;   // a copy: a reference would need memory
             Aux32 pre;
             if (EPI == kEpiSwigluBwd) {
                 const int col = t.n_blk * BN + em.c_lo;
@@ -780,7 +776,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                       p.tma_out ? &tmC : nullptr, p.tma_out2 ? &tmC2 : nullptr, &pre);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(leader_acc_empty[buf]);
+            if (lane == 0) mbar_arrive_cluster(leader_acc_empty(buf));
         }
         if (lane == 0) bulk_wait_group0();   // this warp's TMA stores have completed
         __syncwarp();
@@ -849,7 +845,7 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
         // after its wait, before the tensor cores read the stage.
         int stage = 0;
         uint32_t phase = 0;
-        uint32_t issued[STAGES1] = {0, 0, 0, 0};
+        uint32_t loads = 0;   // stage loads issued; load j used stage j % STAGES1
         bool ok = true;
         for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
             const Tile t = decode_tile<false>(s, p, id, BM1);
@@ -888,7 +884,7 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
                     } else {
                         tma_load_3d(&tmB, &s.full[stage], b_s, kb * BK, t.n_blk * BN, t.g);
                     }
-                    issued[stage] += 1;
+                    ++loads;
                 }
                 // copy j: lane -> 16-byte chunk lane % 8 of row 4 j + lane / 8, so one
                 // warp instruction reads four whole 128-byte row segments; the
@@ -918,7 +914,8 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
         __syncwarp();
         if (lane == 0) {
             for (int i = 0; i < STAGES1; ++i)
-                if (issued[i]) mbar_wait(&s.full[i], (issued[i] - 1) & 1u, abort_flag, p.err);
+                if (loads > (uint32_t)i)   // the stage's last load is its ((loads - 1 - i) / S)-th use
+                    mbar_wait(&s.full[i], ((loads - 1 - (uint32_t)i) / STAGES1) & 1u, abort_flag, p.err);
         }
         __syncwarp();
     } else if (warp == 0) {
@@ -927,7 +924,7 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
             const uint64_t keep = l2_policy_evict_last();   // activation panels are read again
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t issued[STAGES1] = {0, 0, 0, 0};
+            uint32_t loads = 0;   // stage loads issued; load j used stage j % STAGES1
             bool ok = true;
             for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
                 const Tile t = decode_tile<GROUP_K>(s, p, id, BM1);
@@ -959,7 +956,7 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
                             tma_load_3d(&tmB, bar, b_s, kb * BK, t.n_blk * BN, t.g);
                         }
                     }
-                    issued[stage] += 1;
+                    ++loads;
                     if (++stage == STAGES1) {
                         stage = 0;
                         phase ^= 1u;
@@ -968,7 +965,8 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
             }
             // let every load still in flight land before the CTA may exit
             for (int i = 0; i < STAGES1; ++i)
-                if (issued[i]) mbar_wait(&s.full[i], (issued[i] - 1) & 1u, abort_flag, p.err);
+                if (loads > (uint32_t)i)   // the stage's last load is its ((loads - 1 - i) / S)-th use
+                    mbar_wait(&s.full[i], ((loads - 1 - (uint32_t)i) / STAGES1) & 1u, abort_flag, p.err);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer
@@ -1226,7 +1224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t issued[Cfg::kStages] = {};
+            uint32_t loads = 0;   // stage loads issued; load j used stage j % kStages
             bool ok = true;
             for (int id = blockIdx.x; id < total && ok; id += gridDim.x) {
                 const Tile t = decode_tile<false>(s, p, id, NR);
@@ -1243,7 +1241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int c = 0; c < 2; ++c)
                         tma_load_3d(&tmW, bar, a_s + c * kChunkBytes, w_col_swap<EPI>(t, p, c), kb * BK, t.g);
                     tma_load_2d(&tmX, bar, b_s, kb * BK, t.row0);
-                    issued[stage] += 1;
+                    ++loads;
                     if (++stage == Cfg::kStages) {
                         stage = 0;
                         phase ^= 1u;
@@ -1252,7 +1250,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // let every load still in flight land before the CTA may exit
             for (int i = 0; i < Cfg::kStages; ++i)
-                if (issued[i]) mbar_wait(&s.full[i], (issued[i] - 1) & 1u, abort_flag, p.err);
+                if (loads > (uint32_t)i)   // the stage's last load is its ((loads - 1 - i) / S)-th use
+                    mbar_wait(&s.full[i], ((loads - 1 - (uint32_t)i) / Cfg::kStages) & 1u, abort_flag, p.err);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------ MMA issuer

@@ -98,22 +98,54 @@ def test_rows_past_offsets_end_are_untouched(tiles):
     assert_close(y[:200], ref[:200], "y_perm")
 
 
-@pytest.mark.parametrize("tiles", ["single", "pair", "swap"])
-def test_block_sizes_around_tile_edges(tiles, monkeypatch):
-    """Expert blocks of 0, 1, 63, 64, 65, 127, 128, 129, 255, 256, 257 and
-    385 rows: every split of a block into 256-row pair tiles plus a last
-    128-row pair tile (one CTA's 64 rows empty or not), and into 128-row
-    single tiles, with g, u and h checked as well as y."""
-    import routing_grouped_gemm_score_b200 as m
-    helpers.force_kernels(gemm_tiles=tiles)
-    sizes = [0, 1, 63, 64, 65, 127, 128, 129, 255, 256, 257, 385]
-    E, H, I = len(sizes), 192, 320
+TILE_EDGE_SIZES = [0, 1, 63, 64, 65, 127, 128, 129, 255, 256, 257, 270, 288, 289, 300, 385, 513, 544, 545]
+
+
+def edge_case_inputs(sizes, H, I, seed):
+    E = len(sizes)
     offs = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
     A = int(offs[-1])
-    g_ = torch.Generator(device="cuda").manual_seed(11)
+    g_ = torch.Generator(device="cuda").manual_seed(seed)
     x = torch.randn((A, H), generator=g_, device="cuda").to(torch.bfloat16)
     wgu = (torch.randn((E, H, 2 * I), generator=g_, device="cuda") / H ** 0.5).to(torch.bfloat16)
     wd = (torch.randn((E, I, H), generator=g_, device="cuda") / I ** 0.5).to(torch.bfloat16)
+    scale = torch.rand((A,), generator=g_, device="cuda") + 0.5
+    return offs, x, wgu, wd, scale
+
+
+def test_tile_kinds_agree_bit_for_bit_on_tails():
+    """Single-CTA, CTA-pair and swap-AB tiles give identical bits for y,
+    [g | u] and h, with and without a row scale, on blocks whose last tile is
+    short: each output element is the same fp32 sum over K in the same order,
+    whichever tile holds it and whichever operand the weights are."""
+    import routing_grouped_gemm_score_b200 as m
+    offs, x, wgu, wd, scale = edge_case_inputs(TILE_EDGE_SIZES, 192, 320, 12)
+    offs_t = torch.from_numpy(offs).cuda()
+    for rs in (None, scale):
+        outs = {}
+        for tiles in ("single", "pair", "swap"):
+            helpers.force_kernels(gemm_tiles=tiles)
+            o = m.moe_grouped_mlp(x, offs_t, wgu, wd, save=True, row_scale=rs)
+            torch.cuda.synchronize()
+            outs[tiles] = {k: v.view(torch.int16).clone() for k, v in o.items()}
+        assert m.moe_get_device_status() == 0
+        for tiles in ("pair", "swap"):
+            for key in ("y_perm", "gu", "h"):
+                assert torch.equal(outs["single"][key], outs[tiles][key]), (tiles, key, rs is not None)
+
+
+@pytest.mark.parametrize("tiles", ["single", "pair", "swap"])
+def test_block_sizes_around_tile_edges(tiles, monkeypatch):
+    """Expert blocks of 0 to 545 rows: every split of a block into 256-row
+    pair tiles plus a last 128-row or 256-row pair tile (one CTA's 64 rows
+    empty or not; a remainder of 1 to 33 rows: 257, 270, 288, 289, 513, 544,
+    545), and into 128-row single tiles, with g, u and h checked as well as
+    y."""
+    import routing_grouped_gemm_score_b200 as m
+    helpers.force_kernels(gemm_tiles=tiles)
+    sizes = TILE_EDGE_SIZES
+    E, H, I = len(sizes), 192, 320
+    offs, x, wgu, wd, _ = edge_case_inputs(sizes, H, I, 11)
     out = m.moe_grouped_mlp(x, torch.from_numpy(offs).cuda(), wgu, wd, save=True)
     torch.cuda.synchronize()
     assert m.moe_get_device_status() == 0

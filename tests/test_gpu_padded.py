@@ -59,7 +59,7 @@ def test_padded_dispatch_matches_the_oracle(name):
     assert n <= m.moe_permute_padded_max_rows(w.T, w.E, w.k, align)
 
 
-@pytest.mark.parametrize("tiles", ["auto", "swap"])
+@pytest.mark.parametrize("tiles", ["auto", "pair", "swap"])
 @pytest.mark.parametrize("scaled", [False, True])
 @pytest.mark.parametrize("name", ["qwen3_a16", "mixtral_a256", "tiny_a3"])
 def test_layer_through_padded_blocks(name, scaled, tiles):
