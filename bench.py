@@ -69,6 +69,9 @@ def parse():
     ap.add_argument("--router-calls", type=int, default=None, metavar="LOGT",
                     help="only call the router three times at T = 2^LOGT, E=128, k=8 on N(0,1) logits "
                          "(a small program for ncu captures of the router), then exit")
+    ap.add_argument("--scaled-compare", action="store_true",
+                    help="also time the Qwen3-30B-A3B fwd+bwd with the routing weights applied "
+                         "before FC2 (ScaledSwiGLU) on a padded dispatch, beside the default layer")
     ap.add_argument("--gather-compare", action="store_true",
                     help="also time the Qwen3-30B-A3B-shaped forward (no saved state) through x_perm and "
                          "with the gate_up GEMM gathering its rows from x")
@@ -699,6 +702,8 @@ def our_arm(args, world, rank, local):
         line["router_sweep"] = router_sweep(m, hbm)
     if args.gather_compare:
         line["gather_compare"] = gather_compare(m)
+    if args.scaled_compare:
+        line["scaled_compare"] = scaled_compare(m)
     if not args.no_cpu_baseline and world == 1 and rank == 0:
         threads = os.cpu_count() or 1
         runner = OracleRunner(w, cpu_inputs(w, d), threads)
@@ -795,6 +800,74 @@ def router_sweep(m, hbm):
         out.append(entry)
         del logits, res, ws, dprob, dl, aws
     return out
+
+
+def scaled_compare(m):
+    """The Qwen3-30B-A3B-shaped training step (T=4096, H=2048, I=768, E=128,
+    k=8, forward and backward) three ways, each L2-flushed before the step
+    and timed by CUDA events on the device (median of 10 after 3):
+    - the default layer: moe_layer_forward (weights applied in combine) and
+      moe_grouped_mlp_backward;
+    - ScaledSwiGLU on a padded dispatch (align 16 and 128):
+      moe_permute_padded -> moe_grouped_mlp_scaled (h = p silu(g) u) ->
+      unweighted moe_unpermute_combine_rows, then
+      moe_grouped_mlp_scaled_backward on the saved rows.
+    The router runs in every step. GEMM rates count the real rows only (the
+    pad rows' products are zeros)."""
+    import torch
+    import workloads as wl
+    w = wl.WORKLOADS["qwen3_30b_a3b"]
+    d = wl.make_inputs(w, "cuda", with_dout=True)
+    opts = m.RouterOpts(w.score, w.renormalize)
+    flush = torch.ones(64 << 20, dtype=torch.float32, device="cuda")
+    flops = 2.0 * w.T * w.k * w.H * 3 * w.I * 3   # forward and backward grouped GEMMs
+
+    ws = m.LayerWorkspace(w.T, w.H, w.I, w.E, w.k, w.shared_expert, backward=True)
+    out = torch.empty((w.T, w.H), dtype=torch.bfloat16, device="cuda")
+    _, state = m.moe_layer_forward(d["logits"], d["x"], d["w_gate_up"], d["w_down"], w.k, opts,
+                                   save_for_backward=True, workspace=ws, out=out)
+    grads = m.moe_grouped_mlp_backward(d["dout"], state, d["w_gate_up"], d["w_down"], ws)
+
+    def layer_step():
+        m.moe_layer_forward(d["logits"], d["x"], d["w_gate_up"], d["w_down"], w.k, opts, save_for_backward=True,
+                            workspace=ws, out=out, state=state)
+        m.moe_grouped_mlp_backward(d["dout"], state, d["w_gate_up"], d["w_down"], ws, grads)
+
+    def scaled_step(align):
+        def step():
+            r = m.moe_router_topk(d["logits"], w.k, opts)
+            p = m.moe_permute_padded(d["x"], r["topk_idx"], r["offsets"], align, r["topk_prob"])
+            mlp = m.moe_grouped_mlp_scaled(p["x_perm"], p["padded_offsets"], d["w_gate_up"], d["w_down"],
+                                           p["prob_perm"], save=True)
+            m.moe_unpermute_combine(mlp["y_perm"], p["row_of"], None)
+            m.moe_grouped_mlp_scaled_backward(d["dout"], p["row_of"], p["sorted_token"], p["prob_perm"],
+                                              p["padded_offsets"], p["x_perm"], mlp["gu"], mlp["h"],
+                                              d["w_gate_up"], d["w_down"])
+        return step
+
+    res = {"workload": "qwen3_30b_a3b fwd+bwd (T=4096), L2 flushed before each step"}
+    for name, step in (("default_layer", layer_step), ("scaled_align16", scaled_step(16)),
+                       ("scaled_align128", scaled_step(128))):
+        times = []
+        for it in range(13):
+            flush.sum()
+            torch.cuda._sleep(200000)   # the GPU is busy while the calls are issued: device time only
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            step()
+            e.record()
+            torch.cuda.synchronize()
+            if it >= 3:
+                times.append(s.elapsed_time(e))
+        ms = statistics.median(times)
+        res[name] = {"ms_per_step": ms, "tokens_per_s": w.T / (ms / 1e3),
+                     "gemm_tflop_per_step_time": flops / (ms / 1e3) / 1e12}
+    if m.moe_get_device_status() != 0:
+        raise RuntimeError("device status after the ScaledSwiGLU comparison")
+    res["note"] = ("gemm_tflop_per_step_time divides the grouped GEMMs' FLOPs by the whole step's time "
+                   "(router, permute and combine included); the padded steps also allocate their outputs "
+                   "through torch's caching allocator inside the timed region")
+    return res
 
 
 def gather_compare(m):
