@@ -363,7 +363,10 @@ class Layer:
             m.moe_trace_set(None)
 
     def launches(self):
-        return 6 + (2 if self.w.shared_expert else 0) + (6 if self.w.backward else 0)
+        # router, scan, permute, gate_up, down, combine; the shared expert's two
+        # GEMMs (the combine then folded into the second, above 16 tokens); the backward's six
+        return (6 + (2 if self.w.shared_expert else 0) - (1 if combine_folded(self.w) else 0)
+                + (6 if self.w.backward else 0))
 
 
 def _events(n):
@@ -398,9 +401,21 @@ def gemm_summary(w, stages, peaks):
             "note": "expert GEMM FLOPs (6AHI fwd incl. shared expert, 12AHI bwd) / device time of the GEMM stages"}
 
 
+def combine_folded(w):
+    """Whether moe_layer_forward runs the combine in the shared expert's down
+    GEMM epilogue (a shared expert on CTA-pair tiles: more than 16 tokens),
+    so that the step has no combine kernel (its traced combine stage is empty)."""
+    return w.shared_expert and w.T > 16
+
+
 def warm_bandwidth(w, stages, hbm):
     out = {}
     for key, nbytes in bandwidth_bytes(w).items():
+        if key == "fwd_combine" and combine_folded(w):
+            out[key] = {"bytes": nbytes, "warm_us": None, "warm_frac_of_hbm": None,
+                        "in_step": "folded into the shared expert's down GEMM epilogue; the cold figures "
+                                   "time the combine kernel alone on the step's stored rows"}
+            continue
         gbs = nbytes / (stages[key] / 1e3) / 1e9
         out[key] = {"bytes": nbytes, "warm_us": stages[key] * 1e3, "warm_frac_of_hbm": gbs / hbm}
     return out
@@ -684,6 +699,8 @@ def our_arm(args, world, rank, local):
                      "flop_per_launch": gate_up_flop, "ms_per_launch": gate_up_ms,
                      "ms_per_launch_is": "median over a traced pass of as many steps as the timed region, events on the launching stream"},
         "stages_ms": stages,
+        "stages_note": ("the combine runs in the shared expert's down GEMM epilogue: fwd_shared_expert holds it "
+                        "and fwd_combine is empty") if combine_folded(w) else None,
         "bandwidth_kernels": bandwidth_report(layer, stages, hbm, flush),
         "hbm_peak_gbs": hbm,
         "gpu_launches": K * layer.launches(),

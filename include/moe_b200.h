@@ -93,7 +93,9 @@ moe_status moe_get_device_status(void* stream);
  * stage boundaries, in this order:
  *   [0] start  [1] router + offsets  [2] permute  [3] gate_up + SwiGLU
  *   [4] down   [5] shared expert (recorded even without one)  [6] combine
- * and moe_grouped_mlp_backward records:
+ * (with the combine folded into the shared expert's down GEMM, see
+ * moe_layer_forward, the stage [5]..[6] is empty and [4]..[5] holds it);
+ * moe_grouped_mlp_backward and moe_grouped_mlp_scaled_backward record:
  *   [0] start  [1] combine backward  [2] down dgrad + SwiGLU backward
  *   [3] gate_up dgrad  [4] token sum of dx  [5] down wgrad  [6] gate_up wgrad
  * Events beyond n_events are skipped. The elapsed time between consecutive
@@ -337,12 +339,19 @@ moe_status moe_unpermute_combine_rows(const moe_bf16* y_perm, int64_t y_rows, co
  * workspace: topk_idx [T,k], topk_prob [T,k], counts [E], offsets [E+1],
  * row_of [T,k], x_perm [A,H], gu [A,2I] (NULL: not computed), h [A,I],
  * y_perm [A,H].
- * With the environment variable MOE_GATHER=1, x_perm NULL and single-CTA GEMM
- * tiles (experts averaging under 1024 rows), the permutation is folded into the
+ * With the folded permute forced (moe_testing_set_kernels, fold_permute = 1),
+ * x_perm NULL and single-CTA GEMM tiles (experts averaging under 1024 rows, at
+ * least 16), the permutation is folded into the
  * gate_up GEMM (TE Token permutation): its A rows are gathered from x by token,
  * and no permuted copy of x is written (x_perm in the workspace is left
  * unwritten). The result is bit-identical to the default path, which
  * measures faster on B200.
+ * With a shared expert whose GEMMs run on CTA-pair tiles (T > 16), the
+ * combine is done in the shared expert's down GEMM epilogue: each output row
+ * (one token) is the shared expert's fp32 result plus its k routed rows,
+ * weighted, j ascending, rounded to bf16 once (TE Token combine; the shared
+ * expert's output is then not stored as bf16 before the sum). Otherwise the
+ * combine kernel adds the stored bf16 shared output.
  * The call records no device-to-host copy and no host synchronisation, so it
  * can be captured in a CUDA graph. */
 size_t moe_layer_forward_workspace_size(int64_t T, int H, int I, int E, int k, int has_shared);

@@ -76,7 +76,9 @@ constexpr int kStageAP = 128 * BK * 2, kStageBP = (BN / 2) * BK * 2, kStageP = k
 // 64 rows of A and its usual half of B
 constexpr int kStageHalfP = 64 * BK * 2 + kStageBP;
 
-enum Epi { kEpiStore = 0, kEpiSwiglu = 1, kEpiSwigluBwd = 2 };
+// kEpiStoreAdd: the store with the token combine folded in (the shared
+// expert's down GEMM, whose output rows are the tokens in order).
+enum Epi { kEpiStore = 0, kEpiSwiglu = 1, kEpiSwigluBwd = 2, kEpiStoreAdd = 3 };
 
 struct Params {
     int groups;           // number of experts
@@ -106,6 +108,14 @@ struct Params {
     const bf16* gather_x;
     const int32_t* gather_tok;
     int64_t gather_T;
+    // kEpiStoreAdd: output row r also gets sum_{j < add_k} add_prob[r * add_k + j]
+    // * add_rows[add_row_of[r * add_k + j]], after the accumulator, j ascending, in
+    // fp32 (a row index outside [0, add_nrows) is a device-check error and adds nothing)
+    const bf16* add_rows;
+    const int32_t* add_row_of;
+    const float* add_prob;
+    int add_k;
+    int64_t add_nrows;
     unsigned* err;
 };
 
@@ -596,6 +606,31 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const Tile& t, ui
             } else {
 #pragma unroll
                 for (int i = 0; i < 64; ++i) v[i] = 0.0f;
+            }
+            if (EPI == kEpiStoreAdd && r < t.rows) {
+                // the token's routed rows, weighted, j ascending (16-byte loads of 8 columns)
+                const int64_t tok = (int64_t)t.row0 + r;
+                for (int j = 0; j < p.add_k; ++j) {
+                    const int64_t row = __ldg(p.add_row_of + tok * p.add_k + j);
+                    const float pj = __ldg(p.add_prob + tok * p.add_k + j);
+                    if (row < 0 || row >= p.add_nrows) {
+                        raise_error(p.err, kErrDeviceCheck);
+                        continue;
+                    }
+                    const bf16* src = p.add_rows + row * p.ldo + n0 + c0;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        if (n0 + c0 + 8 * q >= p.N) break;
+                        const uint4 w = __ldg(reinterpret_cast<const uint4*>(src) + q);
+                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const float2 f = unpack_bf16x2(ws[i]);
+                            v[8 * q + 2 * i] += pj * f.x;
+                            v[8 * q + 2 * i + 1] += pj * f.y;
+                        }
+                    }
+                }
             }
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
@@ -1661,6 +1696,35 @@ cudaError_t gemm_down(const bf16* h, int64_t rows, const int32_t* offsets, int E
     CUtensorMap tc;
     if (!make_out_map(&tc, y, rows, H)) return cudaErrorInvalidValue;
     return launch_group_m<kEpiStore, true>(ta, ta64, tb, tb, p, st, &tc);
+}
+
+bool grouped_gemm_pair_tiles(int64_t rows, int groups) {
+    return use_pair_tiles(rows, groups) && !use_swap_tiles(rows, groups);
+}
+
+cudaError_t gemm_down_combine(const bf16* h, int64_t T, int H, int I, const bf16* w_down, const bf16* y_perm,
+                              int64_t y_rows, const int32_t* row_of, const float* probs, int k, bf16* out,
+                              cudaStream_t st, unsigned* err) {
+    if (T == 0) return cudaSuccess;
+    if (!grouped_gemm_pair_tiles(T, 1)) return cudaErrorNotSupported;
+    CUtensorMap ta, ta64, tb;
+    if (!make_map_2d(&ta, h, I, T, I, BK, 128)) return cudaErrorInvalidValue;
+    if (!make_map_2d(&ta64, h, I, T, I, BK, 64)) return cudaErrorInvalidValue;
+    if (!make_map_3d(&tb, w_down, H, I, 1, 64, BK)) return cudaErrorInvalidValue;
+    Params p = base_params(1, T, nullptr, err);
+    p.N = H;
+    p.K = I;
+    p.n_blocks = (H + BN - 1) / BN;
+    p.out = out;
+    p.ldo = H;
+    p.add_rows = y_perm;
+    p.add_row_of = row_of;
+    p.add_prob = probs;
+    p.add_k = k;
+    p.add_nrows = y_rows;
+    CUtensorMap tc;
+    if (!make_out_map(&tc, out, T, H)) return cudaErrorInvalidValue;
+    return launch_pair<kEpiStoreAdd, true>(ta, ta64, tb, p, pair_tile_bound(T, 1, p.n_blocks), st, &tc);
 }
 
 cudaError_t gemm_down_dgrad_swiglu(const bf16* dy, int64_t rows, const int32_t* offsets, int E,

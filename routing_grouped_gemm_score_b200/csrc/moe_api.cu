@@ -611,16 +611,24 @@ moe_status moe_layer_forward(const float* logits, const moe_bf16* x, int64_t T, 
         e = gemm_down(L.h, A, L.offsets, E, H, I, reinterpret_cast<const bf16*>(w_down), L.y_perm,
                       st, err, T);   // an expert gets at most T rows
     if (e == cudaSuccess) e = trace_mark(4, st);
+    // With a shared expert on CTA-pair tiles, the combine runs in its down
+    // GEMM's epilogue: that GEMM's rows are the tokens in order, so each output
+    // row adds its token's k routed rows (j ascending) to the shared expert's
+    // fp32 result and is written once; the combine stage is then empty.
+    const bool fused = has_shared && grouped_gemm_pair_tiles(T, 1);
     if (e == cudaSuccess && has_shared) {
         e = gemm_gate_up_swiglu(xb, T, nullptr, 1, H, I,
                                 reinterpret_cast<const bf16*>(shared_gate_up), L.shared_h, nullptr,
                                 st, err);
-        if (e == cudaSuccess)
+        if (e == cudaSuccess && fused)
+            e = gemm_down_combine(L.shared_h, T, H, I, reinterpret_cast<const bf16*>(shared_down), L.y_perm, A,
+                                  L.row_of, L.topk_prob, k, reinterpret_cast<bf16*>(out), st, err);
+        else if (e == cudaSuccess)
             e = gemm_down(L.shared_h, T, nullptr, 1, H, I,
                           reinterpret_cast<const bf16*>(shared_down), L.shared_out, st, err);
     }
     if (e == cudaSuccess) e = trace_mark(5, st);
-    if (e == cudaSuccess)
+    if (e == cudaSuccess && !fused)
         e = launch_combine(L.y_perm, L.row_of, L.topk_prob, T, k, H, A, L.shared_out,
                            reinterpret_cast<bf16*>(out), st, err);
     if (e == cudaSuccess) e = trace_mark(6, st);

@@ -145,6 +145,15 @@ cudaError_t gemm_gate_up_swiglu_gather(const bf16* x, int64_t T, const int32_t* 
 // Whether the forward gate_up GEMM runs on single-CTA 128-row tiles (not CTA
 // pairs, not swap-AB tiles) for this many rows and groups.
 bool grouped_gemm_single_tiles(int64_t rows, int groups);
+// Whether a group-M GEMM of this many rows and groups runs on CTA-pair tiles.
+bool grouped_gemm_pair_tiles(int64_t rows, int groups);
+// The shared expert's down GEMM with the token combine folded into its
+// epilogue: out[t] = bf16(h[t] Wd + sum_j probs[t,j] y_perm[row_of[t,j]]), the
+// sum in fp32 after the product, j ascending. CTA-pair tiles only
+// (cudaErrorNotSupported when grouped_gemm_pair_tiles(T, 1) is false).
+cudaError_t gemm_down_combine(const bf16* h, int64_t T, int H, int I, const bf16* w_down, const bf16* y_perm,
+                              int64_t y_rows, const int32_t* row_of, const float* probs, int k, bf16* out,
+                              cudaStream_t st, unsigned* err);
 // down: y[r] = h[r] Wd[e]
 cudaError_t gemm_down(const bf16* h, int64_t rows, const int32_t* offsets, int E, int H, int I,
                       const bf16* w_down, bf16* y, cudaStream_t st, unsigned* err, int64_t max_group_rows = 0);

@@ -55,7 +55,7 @@ SMALL = {
 }
 
 
-@pytest.mark.parametrize("tiles", ["single", "pair", "swap"])
+@pytest.mark.parametrize("tiles", ["auto", "single", "pair", "swap"])
 @pytest.mark.parametrize("name", list(SMALL))
 def test_layer_forward_matches_per_token_definition(name, tiles, monkeypatch):
     helpers.force_kernels(gemm_tiles=tiles)
@@ -64,6 +64,39 @@ def test_layer_forward_matches_per_token_definition(name, tiles, monkeypatch):
     out = layer(w, d)
     tokens = np.arange(w.T)
     helpers.assert_close_flips(out, oracle_out(w, d), helpers.lazy_forward_terms(w, d, tokens), f"{name}: out")
+
+
+SHARED = {
+    "llama4_small": SMALL["llama4_small"],
+    "k4_shared": SMALL["qwen3_small"].scaled(k=4, shared_expert=True),
+    "odd_dims_shared": SMALL["odd_dims"].scaled(shared_expert=True),
+}
+
+
+@pytest.mark.parametrize("name", list(SHARED))
+def test_combine_in_the_shared_expert_gemm(name):
+    """With a shared expert on CTA-pair tiles the combine runs in that
+    GEMM's epilogue: out[t] = bf16(s[t] + sum_j p[t,j] y[row_of[t,j]]), the
+    shared output s in fp32. Checked against the oracle's shared expert (h
+    rounded to bf16 as stored, its product unrounded) plus the GPU's stored
+    routed rows, strictly; and the combine kernel's path (single tiles, s
+    stored in bf16 first) against the same reference."""
+    w = SHARED[name]
+    helpers.force_kernels(gemm_tiles="auto")
+    d = wl.make_inputs(w, "cuda")
+    out, st = layer(w, d, save=True)
+    f = oracle.bits_to_float
+    sgu, sd = bits(d["shared_gate_up"][0]), bits(d["shared_down"][0])
+    _, _, _, hs = oracle.expert_mlp(bits(d["x"]), sgu, sd, round_bf16=True, want_intermediates=True)
+    shared = hs @ f(sd)
+    y = f(bits(st["y_perm"]))
+    row_of = st["row_of"].cpu().numpy()
+    p = st["topk_prob"].cpu().numpy().astype(np.float64)
+    ref = shared + sum(p[:, j:j + 1] * y[row_of[:, j]] for j in range(w.k))
+    assert_close(out, ref, f"{name}: out, combine in the shared expert's GEMM")
+    helpers.force_kernels(gemm_tiles="single")
+    out2 = layer(w, d)
+    assert_close(out2, ref, f"{name}: out, combine kernel after the stored shared output")
 
 
 def test_layer_forward_saved_state_and_empty_batch():
