@@ -70,6 +70,8 @@ SHARED = {
     "llama4_small": SMALL["llama4_small"],
     "k4_shared": SMALL["qwen3_small"].scaled(k=4, shared_expert=True),
     "odd_dims_shared": SMALL["odd_dims"].scaled(shared_expert=True),
+    # 12 tokens: the shared expert on swap-AB tiles, so the combine kernel runs
+    "t12_shared": SMALL["odd_t12"].scaled(shared_expert=True),
 }
 
 
