@@ -660,8 +660,14 @@ def our_arm(args, world, rank, local):
     if m.moe_get_device_status() != 0:
         raise RuntimeError("device status error in the timed region")
     # stage times: a separate pass of K steps with an event at every stage
-    # boundary (events between kernels break their programmatic overlap)
+    # boundary (events between kernels break their programmatic overlap),
+    # after a second of idle so that it starts from the timed region's power
+    # state rather than from the end of it; its clocks are reported with it
+    time.sleep(1.0)
+    tsampler = ClockSampler(local)
+    tsampler.start()
     fevs, bevs = traced_pass(layer, K)
+    traced_clocks = tsampler.stop()
     stages = stage_medians(layer, fevs, bevs)
 
     graph = None if args.no_graph else graph_measure(args, layer.step, w, world, m)
@@ -697,7 +703,8 @@ def our_arm(args, world, rank, local):
                      "traffic": traffic_for(f"gate_up_swiglu/{w.name}"),
                      "peak_source": f"{peaks_src} {'sustained' if long_region else 'burst'} bf16",
                      "flop_per_launch": gate_up_flop, "ms_per_launch": gate_up_ms,
-                     "ms_per_launch_is": "median over a traced pass of as many steps as the timed region, events on the launching stream"},
+                     "ms_per_launch_is": "median over a traced pass of as many steps as the timed region, events on the launching stream",
+                     "clocks_traced_pass": traced_clocks},
         "stages_ms": stages,
         "stages_note": ("the combine runs in the shared expert's down GEMM epilogue: fwd_shared_expert holds it "
                         "and fwd_combine is empty") if combine_folded(w) else None,
