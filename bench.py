@@ -363,10 +363,11 @@ class Layer:
             m.moe_trace_set(None)
 
     def launches(self):
-        # router, scan, permute, gate_up, down, combine; the shared expert's two
-        # GEMMs (the combine then folded into the second, above 16 tokens); the backward's six
-        return (6 + (2 if self.w.shared_expert else 0) - (1 if combine_folded(self.w) else 0)
-                + (6 if self.w.backward else 0))
+        # router, scan (done by the router itself for one token block, T <= 8),
+        # permute, gate_up, down, combine; the shared expert's two GEMMs (the
+        # combine then folded into the second, above 16 tokens); the backward's six
+        return (6 - (1 if self.w.T <= 8 else 0) + (2 if self.w.shared_expert else 0)
+                - (1 if combine_folded(self.w) else 0) + (6 if self.w.backward else 0))
 
 
 def _events(n):

@@ -290,9 +290,10 @@ moe_status moe_router_topk(const float* logits, int64_t T, int E, int k,
     unsigned* err = device_error_word();
     if (!err) return MOE_ERR_CUDA;
     const RouteScratch rs = carve_route_scratch(workspace, T, E, k);
+    bool scanned = false;
     cudaError_t e = launch_router_topk(logits, T, E, k, opts, topk_idx, topk_prob, routing_map, rs,
-                                       st, err);
-    if (e == cudaSuccess) e = launch_expert_scan(T, E, rs, counts, offsets, st);
+                                       st, err, counts, offsets, &scanned);
+    if (e == cudaSuccess && !scanned) e = launch_expert_scan(T, E, rs, counts, offsets, st);
     return from_cuda(e);
 }
 
@@ -382,9 +383,10 @@ moe_status moe_router_topk_noalloc(const float* logits, int64_t T, int E, int k,
     // other scratch word is written before it is read, so the previous call's
     // contents need no clearing.
     const RouteScratch rs = carve_route_scratch(scratch, T, E, k);
+    bool scanned = false;
     cudaError_t e = launch_router_topk(logits, T, E, k, opts, topk_idx, topk_prob, routing_map, rs,
-                                       st, err);
-    if (e == cudaSuccess) e = launch_expert_scan(T, E, rs, counts, offsets, st);
+                                       st, err, counts, offsets, &scanned);
+    if (e == cudaSuccess && !scanned) e = launch_expert_scan(T, E, rs, counts, offsets, st);
     return from_cuda(e);
 }
 
@@ -582,10 +584,11 @@ moe_status moe_layer_forward(const float* logits, const moe_bf16* x, int64_t T, 
     const bf16* xb = reinterpret_cast<const bf16*>(x);
 
     cudaError_t e = trace_mark(0, st);
+    bool scanned = false;
     if (e == cudaSuccess)
         e = launch_router_topk(logits, T, E, k, opts, L.topk_idx, L.topk_prob, nullptr, L.rs, st,
-                               err);
-    if (e == cudaSuccess) e = launch_expert_scan(T, E, L.rs, L.counts, L.offsets, st);
+                               err, L.counts, L.offsets, &scanned);
+    if (e == cudaSuccess && !scanned) e = launch_expert_scan(T, E, L.rs, L.counts, L.offsets, st);
     if (e == cudaSuccess) e = trace_mark(1, st);
     // Folded permute (moe_testing_set_kernels): without a requested x_perm, on
     // single-CTA tiles, the gate_up GEMM gathers its A rows from x by token

@@ -73,10 +73,14 @@ struct RouteScratch {
 size_t route_scratch_bytes(int64_t T, int E, int k);
 RouteScratch carve_route_scratch(void* base, int64_t T, int E, int k);
 
+// With counts and offsets given and a single token block (T <= 8 tokens), the
+// router also writes the counts and offsets and sets *scanned; otherwise
+// launch_expert_scan must follow.
 cudaError_t launch_router_topk(const float* logits, int64_t T, int E, int k,
                                const moe_router_opts& opts, int32_t* topk_idx, float* topk_prob,
                                uint8_t* routing_map, const RouteScratch& rs, cudaStream_t st,
-                               unsigned* err);
+                               unsigned* err, int32_t* counts = nullptr, int32_t* offsets = nullptr,
+                               bool* scanned = nullptr);
 cudaError_t launch_router_backward(const float* logits, int64_t T, int E, int k, const moe_router_opts& opts,
                                    const int32_t* topk_idx, const float* dprob, float* dlogits,
                                    cudaStream_t st, unsigned* err);

@@ -55,6 +55,10 @@ struct RouterArgs {
     unsigned* ticket;
     int nb;
     int tpb;   // tokens per block
+    // a single token block (nb == 1) may also write the experts' counts and
+    // offsets, so that no scan kernel follows (NULL: the scan kernel does)
+    int32_t* counts;
+    int32_t* offsets;
 };
 
 // After the token loop: thread e counts, in token order, the assignments of
@@ -111,6 +115,32 @@ __device__ __forceinline__ void sort_slots(uint32_t (&so)[SLOTS], uint32_t (&se)
 #pragma unroll
         for (int c = 0; c < 19; ++c) order_pair(so[net[c][0]], se[net[c][0]], so[net[c][1]], se[net[c][1]]);
     }
+}
+
+// Inclusive scan over the block (blockDim.x a multiple of 32, <= 1024).
+__device__ __forceinline__ int block_inclusive_scan(int v, int* warp_tot, int& total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(kFull, v, off);
+        if (lane >= off) v += o;
+    }
+    if (lane == 31) warp_tot[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < nw ? warp_tot[lane] : 0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(kFull, w, off);
+            if (lane >= off) w += o;
+        }
+        if (lane < nw) warp_tot[lane] = w;
+    }
+    __syncthreads();
+    if (warp > 0) v += warp_tot[warp - 1];
+    total = warp_tot[nw - 1];
+    __syncthreads();
+    return v;
 }
 
 // Router, one warp per token. SLOTS = experts per lane (E <= 32*SLOTS). KC is
@@ -249,6 +279,22 @@ __global__ void __launch_bounds__(kRouteThreads) router_topk_kernel(const Router
     }
     __syncthreads();
     rank_block(sel, t0, tpb, E, k, a.local_rank, a.block_base, a.nb);
+    if (a.counts != nullptr) {
+        // the only token block: its counts are the experts' counts (thread e
+        // wrote expert e's in rank_block; E <= blockDim), the block's base rank
+        // in each expert is 0, and the offsets are the counts' exclusive scan
+        __shared__ int warp_tot[kRouteThreads / 32];
+        const int e = threadIdx.x;
+        const int cnt = e < E ? a.block_base[e] : 0;
+        if (e < E) {
+            a.counts[e] = cnt;
+            a.block_base[e] = 0;
+        }
+        int total;
+        const int incl = block_inclusive_scan(cnt, warp_tot, total);
+        if (e < E) a.offsets[e + 1] = incl;
+        if (e == 0) a.offsets[0] = 0;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -826,31 +872,6 @@ __global__ void __launch_bounds__(kRouteThreads)
     rank_block(sel, t0, tpb, E, k, local_rank, block_base, nb);
 }
 
-// Inclusive scan over the block (blockDim.x a multiple of 32, <= 1024).
-__device__ __forceinline__ int block_inclusive_scan(int v, int* warp_tot, int& total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int o = __shfl_up_sync(kFull, v, off);
-        if (lane >= off) v += o;
-    }
-    if (lane == 31) warp_tot[warp] = v;
-    __syncthreads();
-    if (warp == 0) {
-        int w = lane < nw ? warp_tot[lane] : 0;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int o = __shfl_up_sync(kFull, w, off);
-            if (lane >= off) w += o;
-        }
-        if (lane < nw) warp_tot[lane] = w;
-    }
-    __syncthreads();
-    if (warp > 0) v += warp_tot[warp - 1];
-    total = warp_tot[nw - 1];
-    __syncthreads();
-    return v;
-}
 
 constexpr int kScanPerThread = 8;   // values a scan thread holds per pass
 // Shared-memory slot of value i of a pass: thread i / 8's run, one padding
@@ -1223,7 +1244,8 @@ cudaError_t launch_router_k(const RouterArgs& a, dim3 grid, dim3 block, cudaStre
 cudaError_t launch_router_topk(const float* logits, int64_t T, int E, int k,
                                const moe_router_opts& opts, int32_t* topk_idx, float* topk_prob,
                                uint8_t* routing_map, const RouteScratch& rs, cudaStream_t st,
-                               unsigned* err) {
+                               unsigned* err, int32_t* counts, int32_t* offsets, bool* scanned) {
+    if (scanned) *scanned = false;
     RouterArgs a;
     a.logits = logits;
     a.T = T;
@@ -1241,6 +1263,8 @@ cudaError_t launch_router_topk(const float* logits, int64_t T, int E, int k,
     a.ticket = rs.ticket;
     a.nb = (int)route_blocks(T);
     a.tpb = route_tokens_per_block(T);
+    a.counts = nullptr;
+    a.offsets = nullptr;
     // Large T: the lane-per-token kernel where it applies. moe_testing_set_kernels
     // can force either kernel (the tests run both on the same inputs).
     const int force = kernel_override().router;
@@ -1272,6 +1296,11 @@ cudaError_t launch_router_topk(const float* logits, int64_t T, int E, int k,
     }
     const dim3 grid((unsigned)a.nb), block(kRouteThreads);
     (void)err;
+    if (a.nb == 1 && counts != nullptr && offsets != nullptr) {   // one token block: no scan kernel
+        a.counts = counts;
+        a.offsets = offsets;
+        if (scanned) *scanned = true;
+    }
     if (E <= 32) return launch_router_k<1>(a, grid, block, st);
     if (E <= 64) return launch_router_k<2>(a, grid, block, st);
     if (E <= 128) return launch_router_k<4>(a, grid, block, st);
