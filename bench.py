@@ -364,10 +364,18 @@ class Layer:
 
     def launches(self):
         # router, scan (done by the router itself for one token block, T <= 8),
-        # permute, gate_up, down, combine; the shared expert's two GEMMs (the
-        # combine then folded into the second, above 16 tokens); the backward's six
-        return (6 - (1 if self.w.T <= 8 else 0) + (2 if self.w.shared_expert else 0)
-                - (1 if combine_folded(self.w) else 0) + (6 if self.w.backward else 0))
+        # permute, gate_up, down (one launch with gate_up when every expert has
+        # at most T <= 64 rows on swap-AB tiles and the experts that can hold
+        # rows have at least one gate_up tile per SM), combine; the shared expert's
+        # two GEMMs (the combine then folded into the second, above 16 tokens);
+        # the backward's six
+        import torch
+        w = self.w
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+        fused_mlp = (w.T <= 64 and w.T * w.k <= 16 * w.E and w.E <= 256
+                     and min(w.E, w.T * w.k) * -(-w.I // 64) >= sms)
+        return (6 - (1 if w.T <= 8 else 0) - (1 if fused_mlp else 0) + (2 if w.shared_expert else 0)
+                - (1 if combine_folded(w) else 0) + (6 if w.backward else 0))
 
 
 def _events(n):

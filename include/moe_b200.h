@@ -94,7 +94,8 @@ moe_status moe_get_device_status(void* stream);
  *   [0] start  [1] router + offsets  [2] permute  [3] gate_up + SwiGLU
  *   [4] down   [5] shared expert (recorded even without one)  [6] combine
  * (with the combine folded into the shared expert's down GEMM, see
- * moe_layer_forward, the stage [5]..[6] is empty and [4]..[5] holds it);
+ * moe_layer_forward, the stage [5]..[6] is empty and [4]..[5] holds it; with
+ * gate_up and down in one launch, [3]..[4] is empty and [2]..[3] holds both);
  * moe_grouped_mlp_backward and moe_grouped_mlp_scaled_backward record:
  *   [0] start  [1] combine backward  [2] down dgrad + SwiGLU backward
  *   [3] gate_up dgrad  [4] token sum of dx  [5] down wgrad  [6] gate_up wgrad
@@ -352,6 +353,11 @@ moe_status moe_unpermute_combine_rows(const moe_bf16* y_perm, int64_t y_rows, co
  * weighted, j ascending, rounded to bf16 once (TE Token combine; the shared
  * expert's output is then not stored as bf16 before the sum). Otherwise the
  * combine kernel adds the stored bf16 shared output.
+ * With at most T <= 64 rows per expert on swap-AB tiles, where the experts
+ * that can hold rows (min(E, T k)) have at least one gate_up tile (64 columns
+ * of h) per SM, the gate_up and down GEMMs run as one launch: a down tile
+ * loads its weights first and waits (bounded) on a device counter until its
+ * expert's h is stored. The results are bit-identical to two launches.
  * The call records no device-to-host copy and no host synchronisation, so it
  * can be captured in a CUDA graph. */
 size_t moe_layer_forward_workspace_size(int64_t T, int H, int I, int E, int k, int has_shared);
@@ -435,7 +441,10 @@ moe_status moe_grouped_mlp_scaled_backward(const moe_bf16* dout, int64_t T, int 
  *  gemm_tiles    group-M GEMMs on single-CTA 128-row tiles or CTA-pair tiles;
  *                or the forward GEMMs on swap-AB tiles (weights as the 128-row
  *                operand, 64 token rows per tile; the backward GEMMs then take
- *                single-CTA tiles)
+ *                single-CTA tiles); SWAP_UNFUSED: swap-AB tiles with the
+ *                layer's gate_up and down GEMMs as two launches even where
+ *                every expert holds at most 64 rows (by default one launch
+ *                then computes both)
  *  router        the warp-per-token or the lane-per-token router kernel (the
  *                lane kernel where it applies: E a multiple of 32, k <= 8,
  *                renormalised softmax or sigmoid)
@@ -451,6 +460,7 @@ moe_status moe_grouped_mlp_scaled_backward(const moe_bf16* dout, int64_t T, int 
 #define MOE_TESTING_GEMM_SINGLE 1
 #define MOE_TESTING_GEMM_PAIR 2
 #define MOE_TESTING_GEMM_SWAP 3
+#define MOE_TESTING_GEMM_SWAP_UNFUSED 4
 #define MOE_TESTING_ROUTER_WARP 1
 #define MOE_TESTING_ROUTER_LANE 2
 #define MOE_TESTING_PERMUTE_TOKENS 1

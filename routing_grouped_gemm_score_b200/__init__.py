@@ -186,7 +186,7 @@ def moe_trace_set(events) -> None:
 
 # kernel variants for moe_testing_set_kernels (include/moe_b200.h, testing hooks)
 TESTING_AUTO = 0
-GEMM_SINGLE, GEMM_PAIR, GEMM_SWAP = 1, 2, 3
+GEMM_SINGLE, GEMM_PAIR, GEMM_SWAP, GEMM_SWAP_UNFUSED = 1, 2, 3, 4
 ROUTER_WARP, ROUTER_LANE = 1, 2
 PERMUTE_TOKENS, PERMUTE_WARP = 1, 2
 

@@ -116,6 +116,16 @@ struct Params {
     const float* add_prob;
     int add_k;
     int64_t add_nrows;
+    // fused swap-AB expert MLP (gemm_swap_mlp_kernel): the down GEMM's tiles
+    // follow the gate_up tiles in one launch; y [rows][N2] = h W_down, n_blocks2
+    // tiles of 128 columns per expert, K = I. sched[0] hands out the tiles and
+    // sched[1 + g] counts the epilogue warps that have stored their part of
+    // expert g's h; all are zero before the launch
+    bf16* y;
+    int64_t ldy;
+    int N2;
+    int n_blocks2;
+    int32_t* sched;
     unsigned* err;
 };
 
@@ -1176,6 +1186,8 @@ __global__ void __launch_bounds__(GROUP_K ? kThreadsK : kThreads, 1)
 // the NR token columns). Every wait is bounded.
 constexpr int kStageAS = 128 * BK * 2;           // 128 weight columns x 64 K: two 64-column chunks
 
+constexpr int kTileQ = 4;   // tile ids the fused kernel's producer may run ahead by
+
 template <int NR>
 struct SwapCfg {
     static constexpr int kStages = NR == 16 ? 11 : 6;
@@ -1195,6 +1207,10 @@ struct __align__(1024) SmemS {
     uint64_t acc_empty[2];
     uint64_t xchg[2];             // SwiGLU: the up values of the accumulator's tile are in ubuf
     uint64_t drain;
+    // gemm_swap_mlp_kernel: the producer's tile ids for the other roles
+    uint64_t tq_full[kTileQ];
+    uint64_t tq_empty[kTileQ];
+    int tile_q[kTileQ];
     uint32_t tmem_base;
     int abort;
     int total_tiles;
@@ -1212,6 +1228,62 @@ template <int EPI>
 __device__ __forceinline__ int w_col_swap(const Tile& t, const Params& p, int c) {
     if (EPI == kEpiSwiglu) return (c == 0 ? 0 : p.I) + t.n_blk * 64;
     return t.n_blk * 128 + 64 * c;
+}
+
+// Epilogue of a swap-AB SwiGLU tile for one warp: v holds the warp's kWC token
+// columns (j0 ..) of its lane's weight column. The warps of the upper lane
+// quarters (u) hand their values to those of the lower quarters (g) through
+// ubuf, which store h = silu(g) u (times the row scale) and [g | u]. Returns
+// false if the hand-over wait gave up.
+template <int NR>
+__device__ __forceinline__ bool swap_epi_swiglu(SmemS<NR>& s, const Params& p, const Tile& t, int buf,
+                                                uint32_t use, int quarter, int j0, int lane,
+                                                const float (&v)[SwapCfg<NR>::kWarpCols], volatile int* abort_flag) {
+    constexpr int kWC = SwapCfg<NR>::kWarpCols;
+    const int nvalid = min(max(t.rows - j0, 0), kWC);
+    if (quarter >= 2) {
+        // up values of columns 32 (quarter - 2) + lane
+        float* row = s.ubuf[buf][32 * (quarter - 2) + lane] + j0;
+#pragma unroll
+        for (int i = 0; i < kWC; ++i) row[i] = v[i];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.xchg[buf]);
+        return true;
+    }
+    if (!mbar_wait(&s.xchg[buf], use & 1u, abort_flag, p.err)) return false;
+    const int hc = t.n_blk * 64 + 32 * quarter + lane;   // column of h
+    const float* urow = s.ubuf[buf][32 * quarter + lane] + j0;
+    const int64_t r0 = (int64_t)t.row0 + j0;
+#pragma unroll
+    for (int i = 0; i < kWC; ++i) {
+        if (i >= nvalid || hc >= p.N) break;
+        const float g = v[i], u = urow[i];
+        const float rs = p.row_scale ? __ldg(p.row_scale + r0 + i) : 1.0f;
+        if (p.out2) {
+            p.out2[(r0 + i) * p.ldo2 + hc] = __float2bfloat16_rn(g);
+            p.out2[(r0 + i) * p.ldo2 + p.I + hc] = __float2bfloat16_rn(u);
+        }
+        p.out[(r0 + i) * p.ldo + hc] = __float2bfloat16_rn(silu_f(g) * u * rs);
+    }
+    return true;
+}
+
+// Store epilogue of a swap-AB tile for one warp: its lane's output column of
+// every valid token row, into out [rows][ld] (columns < n).
+template <int NR>
+__device__ __forceinline__ void swap_epi_store(bf16* out, int64_t ld, int n, const Tile& t, int quarter, int j0,
+                                               int lane, const float (&v)[SwapCfg<NR>::kWarpCols]) {
+    constexpr int kWC = SwapCfg<NR>::kWarpCols;
+    const int nvalid = min(max(t.rows - j0, 0), kWC);
+    const int col = t.n_blk * 128 + 32 * quarter + lane;
+    const int64_t r0 = (int64_t)t.row0 + j0;
+    if (col < n) {
+#pragma unroll
+        for (int i = 0; i < kWC; ++i) {
+            if (i >= nvalid) break;
+            out[(r0 + i) * ld + col] = __float2bfloat16_rn(v[i]);
+        }
+    }
 }
 
 template <int EPI, int NR>
@@ -1353,45 +1425,266 @@ __global__ void __launch_bounds__(kThreads, 1)
             if constexpr (kWC == 32) tmem_load_32(taddr, v);
             else tmem_load_8(taddr, v);
             const int j0 = kWC * half;                       // first token column of this warp
-            const int nvalid = min(max(t.rows - j0, 0), kWC);
             bool ok = true;
-            if (EPI == kEpiSwiglu) {
-                if (quarter >= 2) {
-                    // up values of columns 32 (quarter - 2) + lane
-                    float* row = s.ubuf[buf][32 * (quarter - 2) + lane] + j0;
-#pragma unroll
-                    for (int i = 0; i < kWC; ++i) row[i] = v[i];
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&s.xchg[buf]);
-                } else {
-                    ok = mbar_wait(&s.xchg[buf], use & 1u, abort_flag, p.err);
-                    if (ok) {
-                        const int hc = t.n_blk * 64 + 32 * quarter + lane;   // column of h
-                        const float* urow = s.ubuf[buf][32 * quarter + lane] + j0;
-                        const int64_t r0 = (int64_t)t.row0 + j0;
-#pragma unroll
-                        for (int i = 0; i < kWC; ++i) {
-                            if (i >= nvalid || hc >= p.N) break;
-                            const float g = v[i], u = urow[i];
-                            const float rs = p.row_scale ? __ldg(p.row_scale + r0 + i) : 1.0f;
-                            if (p.out2) {
-                                p.out2[(r0 + i) * p.ldo2 + hc] = __float2bfloat16_rn(g);
-                                p.out2[(r0 + i) * p.ldo2 + p.I + hc] = __float2bfloat16_rn(u);
-                            }
-                            p.out[(r0 + i) * p.ldo + hc] = __float2bfloat16_rn(silu_f(g) * u * rs);
-                        }
+            if (EPI == kEpiSwiglu) ok = swap_epi_swiglu<NR>(s, p, t, buf, use, quarter, j0, lane, v, abort_flag);
+            else swap_epi_store<NR>(p.out, p.ldo, p.N, t, quarter, j0, lane, v);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.acc_empty[buf]);
+            if (!ok) break;
+        }
+    }
+
+    pdl_launch_dependents();   // every role has left its loop (see gemm_pair_kernel)
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, Cfg::kTmemCols);
+    }
+}
+
+// ================================================================ fused MLP
+// gemm_swap_mlp_kernel: the expert MLP of a small batch in one launch, on the
+// swap-AB tiles of gemm_swap_kernel: first the gate_up + SwiGLU tiles of every
+// expert (h, and [g | u] when saved), then the down tiles (y = h W_down).
+// The producer takes each tile id from one device-wide counter (sched[0]) and
+// hands it to the MMA and epilogue warps through a small queue in shared
+// memory. Ids are taken in increasing order across the grid, so every gate_up
+// tile has been taken by a running CTA before any down tile is: a down tile
+// waits only on work already in progress, whichever CTAs are resident.
+// A down tile's producer first issues the weight loads of up to a ring's worth
+// of its K slices (the weights do not depend on h), then waits (bounded) until
+// the epilogue warps of all gate_up tiles of its expert have stored their
+// part of h and counted themselves in sched[1 + g], and then issues the loads
+// of h. Each expert must hold at most NR rows (one row block); otherwise the
+// launch records a device-check error and computes nothing.
+template <int NR>
+__device__ __forceinline__ Tile decode_mlp_tile(const SmemS<NR>& s, const Params& p, int id, int total1,
+                                                bool& down) {
+    down = id >= total1;
+    if (!down) return decode_tile<false>(s, p, id, NR);
+    const int local = id - total1;
+    const int q = local / p.n_blocks2;                      // q-th expert with rows
+    Tile t = decode_tile<false>(s, p, q * p.n_blocks, NR);  // its (only) row block
+    t.n_blk = local - q * p.n_blocks2;
+    t.num_kb = (p.I + BK - 1) / BK;
+    return t;
+}
+
+template <int NR>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_swap_mlp_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmWgu,
+                         const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmWd,
+                         const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    using Cfg = SwapCfg<NR>;
+    SmemS<NR>& s = *reinterpret_cast<SmemS<NR>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                         ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int* abort_flag = &s.abort;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < Cfg::kStages; ++i) {
+            mbar_init(&s.full[i], 1);
+            mbar_init(&s.empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s.acc_full[i], 1);
+            mbar_init(&s.acc_empty[i], kEpiWarps);
+            mbar_init(&s.xchg[i], kEpiWarps / 2);
+        }
+        for (int i = 0; i < kTileQ; ++i) {
+            mbar_init(&s.tq_full[i], 1);
+            mbar_init(&s.tq_empty[i], 1 + kEpiWarps);   // the MMA warp and each epilogue warp
+        }
+        mbar_init(&s.drain, 1);
+        s.abort = 0;
+        fence_mbar_init();
+        prefetch_tensormap(&tmX);
+        prefetch_tensormap(&tmWgu);
+        prefetch_tensormap(&tmH);
+        prefetch_tensormap(&tmWd);
+    }
+    if (warp == 1) {
+        tmem_alloc(&s.tmem_base, Cfg::kTmemCols);
+        tmem_relinquish();
+    }
+    pdl_wait();                // the previous kernels' outputs (token rows, offsets, zeroed counters) are complete
+    build_schedule<false>(s, p, NR);
+    bool bad = false;
+    for (int g = threadIdx.x; g < p.groups; g += blockDim.x) bad = bad || s.off[g + 1] - s.off[g] > NR;
+    bad = __syncthreads_or(bad) != 0;
+    if (bad && blockIdx.x == 0 && threadIdx.x == 0) raise_error(p.err, kErrDeviceCheck);
+    const int total1 = bad ? 0 : s.total_tiles;                              // gate_up tiles
+    const int total = total1 + (total1 / max(p.n_blocks, 1)) * p.n_blocks2;  // and the down tiles
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = s.tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t loads = 0;   // stage loads issued; load j used stage j % kStages
+            bool ok = true;
+            for (int j = 0;; ++j) {
+                const int slot = j % kTileQ;
+                if (!mbar_wait(&s.tq_empty[slot], ((uint32_t)(j / kTileQ) & 1u) ^ 1u, abort_flag, p.err)) break;
+                int id = atomicAdd(p.sched, 1);
+                if (id >= total) id = -1;
+                s.tile_q[slot] = id;
+                mbar_arrive(&s.tq_full[slot]);
+                if (id < 0) break;
+                bool down;
+                const Tile t = decode_mlp_tile(s, p, id, total1, down);
+                const CUtensorMap* mw = down ? &tmWd : &tmWgu;
+                const CUtensorMap* mx = down ? &tmH : &tmX;
+                // down tiles: the weight loads of the first `pre` K slices go out before h is ready
+                const int pre = down ? min(t.num_kb, Cfg::kStages) : 0;
+                const int stage0 = stage;
+                int early = 0;   // early stages issued whose h loads are still to be issued
+                // h of expert g is complete once every gate_up tile's 4 writer warps have
+                // counted; then the early stages get their h loads (issued after a failed
+                // wait too, so that every issued stage completes; the error is recorded)
+                auto load_h_early = [&](bool wait) {
+                    if (early == 0) return;
+                    if (wait) ok = wait_count(p.sched + 1 + t.g, 4 * p.n_blocks, abort_flag, p.err);
+                    fence_proxy_async_global();
+                    int st2 = stage0;
+                    for (int k2 = 0; k2 < early; ++k2) {
+                        tma_load_2d(mx, &s.full[st2], s.stage[st2] + kStageAS, k2 * BK, t.row0);
+                        if (++st2 == Cfg::kStages) st2 = 0;
                     }
+                    early = 0;
+                };
+                for (int kb = 0; kb < t.num_kb; ++kb) {
+                    if (kb == pre) load_h_early(true);
+                    if (!ok) break;
+                    if (!mbar_wait(&s.empty[stage], phase ^ 1u, abort_flag, p.err)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* a_s = s.stage[stage];
+                    uint64_t* bar = &s.full[stage];
+                    mbar_arrive_expect_tx(bar, Cfg::kStage);   // weights and token rows
+#pragma unroll
+                    for (int c = 0; c < 2; ++c)
+                        tma_load_3d(mw, bar, a_s + c * kChunkBytes,
+                                    down ? w_col_swap<kEpiStore>(t, p, c) : w_col_swap<kEpiSwiglu>(t, p, c),
+                                    kb * BK, t.g);
+                    if (kb >= pre) tma_load_2d(mx, bar, a_s + kStageAS, kb * BK, t.row0);
+                    else ++early;
+                    ++loads;
+                    if (++stage == Cfg::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                load_h_early(ok);   // every K slice was an early one, or a wait gave up
+                if (!ok) break;
+            }
+            // every issued stage completes (its h load was issued too): wait for each
+            // stage's last load, whatever the abort flag says, before the CTA may exit
+            for (int i = 0; i < Cfg::kStages; ++i)
+                if (loads > (uint32_t)i)
+                    mbar_wait_bounded(&s.full[i], ((loads - 1 - (uint32_t)i) / Cfg::kStages) & 1u, p.err);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------ MMA issuer
+        constexpr uint32_t idesc = instr_desc<128, NR, true, false>();
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        bool any_mma = false;
+        for (int j = 0; ok; ++j) {
+            const int slot = j % kTileQ;
+            if (!mbar_wait(&s.tq_full[slot], (uint32_t)(j / kTileQ) & 1u, abort_flag, p.err)) break;
+            const int id = s.tile_q[slot];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.tq_empty[slot]);
+            if (id < 0) break;
+            bool down;
+            const Tile t = decode_mlp_tile(s, p, id, total1, down);
+            const int buf = j & 1;
+            const uint32_t use = (uint32_t)(j >> 1);
+            if (!mbar_wait(&s.acc_empty[buf], (use & 1u) ^ 1u, abort_flag, p.err)) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + (uint32_t)(buf * NR);
+            for (int kb = 0; kb < t.num_kb; ++kb) {
+                if (!mbar_wait(&s.full[stage], phase, abort_flag, p.err)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a_addr = smem_u32(s.stage[stage]);
+                const uint32_t b_addr = a_addr + kStageAS;
+                if (lane == 0) {
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t adesc = smem_desc(a_addr + kk * 2048, kChunkBytes, 1024);
+                        const uint64_t bdesc = smem_desc(b_addr + kk * 32, 16, 1024);
+                        umma_bf16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    umma_commit(&s.empty[stage]);
+                    any_mma = true;
+                }
+                __syncwarp();
+                if (++stage == Cfg::kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            if (!ok) break;
+            if (lane == 0) umma_commit(&s.acc_full[buf]);
+            __syncwarp();
+        }
+        if (lane == 0 && any_mma) {
+            umma_commit(&s.drain);
+            mbar_wait_bounded(&s.drain, 0, p.err);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------ epilogue
+        const int quarter = warp & 3;               // TMEM lanes 32*quarter .. +31
+        const int half = (warp - 2) / 4;            // token columns kWarpCols*half ..
+        constexpr int kWC = Cfg::kWarpCols;
+        // A CTA's ids increase, so its gate_up tiles come before its down tiles:
+        // the hand-over barrier xchg[buf] is used by tiles j = buf, buf + 2, ...
+        // of the gate_up run only, and its parity follows j >> 1.
+        for (int j = 0;; ++j) {
+            const int slot = j % kTileQ;
+            if (!mbar_wait(&s.tq_full[slot], (uint32_t)(j / kTileQ) & 1u, abort_flag, p.err)) break;
+            const int id = s.tile_q[slot];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s.tq_empty[slot]);
+            if (id < 0) break;
+            bool down;
+            const Tile t = decode_mlp_tile(s, p, id, total1, down);
+            const int buf = j & 1;
+            const uint32_t use = (uint32_t)(j >> 1);
+            if (!mbar_wait(&s.acc_full[buf], use & 1u, abort_flag, p.err)) break;
+            tc_fence_after();
+            float v[kWC];
+            const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * NR + kWC * half);
+            if constexpr (kWC == 32) tmem_load_32(taddr, v);
+            else tmem_load_8(taddr, v);
+            const int j0 = kWC * half;
+            bool ok = true;
+            if (!down) {
+                ok = swap_epi_swiglu<NR>(s, p, t, buf, use, quarter, j0, lane, v, abort_flag);
+                if (ok && quarter < 2) {
+                    // this warp's part of expert g's h is stored: make it visible to
+                    // other CTAs' TMA loads, then count it
+                    __threadfence();
+                    fence_proxy_async_global();
+                    __syncwarp();
+                    if (lane == 0) atomicAdd(p.sched + 1 + t.g, 1);
                 }
             } else {
-                const int col = t.n_blk * 128 + 32 * quarter + lane;
-                const int64_t r0 = (int64_t)t.row0 + j0;
-                if (col < p.N) {
-#pragma unroll
-                    for (int i = 0; i < kWC; ++i) {
-                        if (i >= nvalid) break;
-                        p.out[(r0 + i) * p.ldo + col] = __float2bfloat16_rn(v[i]);
-                    }
-                }
+                swap_epi_store<NR>(p.y, p.ldy, p.N2, t, quarter, j0, lane, v);
             }
             tc_fence_before();
             __syncwarp();
@@ -1554,8 +1847,19 @@ bool use_pair_tiles(int64_t rows, int groups) {
 // to spread the weight reads over the SMs.
 bool use_swap_tiles(int64_t rows, int groups) {
     const int forced = kernel_override().gemm_tiles;
-    if (forced != MOE_TESTING_AUTO) return forced == MOE_TESTING_GEMM_SWAP;
+    if (forced != MOE_TESTING_AUTO) return forced == MOE_TESTING_GEMM_SWAP || forced == MOE_TESTING_GEMM_SWAP_UNFUSED;
     return rows <= (int64_t)groups * 16;
+}
+
+template <int NR>
+cudaError_t launch_mlp(const CUtensorMap& x_rows, const CUtensorMap& w_gate_up, const CUtensorMap& h_rows,
+                       const CUtensorMap& w_down, const Params& p, int64_t grid, cudaStream_t st) {
+    auto kern = gemm_swap_mlp_kernel<NR>;
+    static std::once_flag once;
+    static cudaError_t attr = cudaSuccess;
+    if (set_smem_once(kern, swap_smem_bytes<NR>(), once, attr) != cudaSuccess) return attr;
+    return launch_chained(kern, dim3((unsigned)grid), dim3(kThreads), swap_smem_bytes<NR>(), st, x_rows, w_gate_up,
+                          h_rows, w_down, p);
 }
 
 template <int EPI, int NR>
@@ -1668,6 +1972,53 @@ cudaError_t gemm_gate_up_swiglu_gather(const bf16* x, int64_t T, const int32_t* 
     if (gu_save && !make_out_map(&tc2, gu_save, rows, 2 * (uint64_t)I)) return cudaErrorInvalidValue;
     return launch_1cta<kEpiSwiglu, false, true, false>(ta, tb, p, single_tile_bound(rows, E, p.n_blocks), st, &tc,
                                                        gu_save ? &tc2 : nullptr);
+}
+
+bool use_fused_mlp(int64_t rows, int groups, int64_t max_group_rows, int I) {
+    if (kernel_override().gemm_tiles == MOE_TESTING_GEMM_SWAP_UNFUSED) return false;
+    if (!use_swap_tiles(rows, groups) || max_group_rows <= 0 || max_group_rows > 64 || groups > kMaxGroups)
+        return false;
+    if (kernel_override().gemm_tiles == MOE_TESTING_GEMM_SWAP) return true;
+    // With fewer gate_up tiles than SMs, the SMs without one can stage only a
+    // ring's worth of down weights before h is ready, and the rest of the down
+    // tiles queue behind the gate_up tiles on the busy SMs: two launches, the
+    // second on every SM, measured faster there (T = 1, Qwen3-30B-A3B shape:
+    // 34.9 against 35.8 us a step).
+    const int64_t experts = rows < groups ? rows : groups;   // at most this many hold rows
+    return experts * ((I + 63) / 64) >= sm_count();
+}
+
+cudaError_t gemm_expert_mlp_fused(const bf16* x, int64_t rows, const int32_t* offsets, int E, int H, int I,
+                                  const bf16* w_gate_up, const bf16* w_down, bf16* h, bf16* gu_save, bf16* y,
+                                  int32_t* sched, int64_t max_group_rows, cudaStream_t st, unsigned* err) {
+    if (rows == 0) return cudaSuccess;
+    if (!offsets || !sched || max_group_rows <= 0 || max_group_rows > 64 || E > kMaxGroups)
+        return cudaErrorInvalidValue;
+    const int nr = max_group_rows <= 16 ? 16 : 64;
+    CUtensorMap tx, th, twgu, twd;
+    if (!make_map_2d(&tx, x, H, rows, H, BK, nr)) return cudaErrorInvalidValue;
+    if (!make_map_2d(&th, h, I, rows, I, BK, nr)) return cudaErrorInvalidValue;
+    if (!make_map_3d(&twgu, w_gate_up, 2 * (uint64_t)I, H, E, 64, BK)) return cudaErrorInvalidValue;
+    if (!make_map_3d(&twd, w_down, H, I, E, 64, BK)) return cudaErrorInvalidValue;
+    Params p = base_params(E, rows, offsets, err);
+    p.N = I;
+    p.K = H;
+    p.I = I;
+    p.n_blocks = (I + 63) / 64;   // gate_up: 64 gate and the matching 64 up columns per tile
+    p.out = h;
+    p.ldo = I;
+    p.out2 = gu_save;
+    p.ldo2 = 2 * (int64_t)I;
+    p.y = y;
+    p.ldy = H;
+    p.N2 = H;
+    p.n_blocks2 = (H + 127) / 128;   // down: 128 output columns per tile
+    p.sched = sched;
+    // at most min(E, rows) experts hold rows, each one row block
+    const int64_t experts = rows < E ? rows : E;
+    int64_t grid = experts * (p.n_blocks + p.n_blocks2);
+    if (grid > sm_count()) grid = sm_count();
+    return nr == 16 ? launch_mlp<16>(tx, twgu, th, twd, p, grid, st) : launch_mlp<64>(tx, twgu, th, twd, p, grid, st);
 }
 
 bool grouped_gemm_single_tiles(int64_t rows, int groups) {

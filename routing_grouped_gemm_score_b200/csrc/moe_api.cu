@@ -103,6 +103,7 @@ moe_status check_opts(const moe_router_opts& o) {
 struct FwdLayout {
     RouteScratch rs;
     int32_t *topk_idx, *counts, *offsets, *row_of, *sorted_token;
+    int32_t* sched;   // [E + 1]: the fused small-batch MLP's tile counter and per-expert h counts
     float* topk_prob;
     bf16 *x_perm, *h, *y_perm, *shared_h, *shared_out;
     size_t bytes;
@@ -118,6 +119,7 @@ FwdLayout fwd_layout(void* ws, int64_t T, int H, int I, int E, int k, int has_sh
     L.topk_prob = c.take<float>((size_t)A);
     L.counts = c.take<int32_t>((size_t)E);
     L.offsets = c.take<int32_t>((size_t)E + 1);
+    L.sched = c.take<int32_t>((size_t)E + 1);
     L.row_of = c.take<int32_t>((size_t)A);
     L.sorted_token = c.take<int32_t>((size_t)A);
     L.x_perm = c.take<bf16>((size_t)A * H);
@@ -235,7 +237,7 @@ moe_status moe_get_device_status(void* stream) {
 }
 
 moe_status moe_testing_set_kernels(int gemm_tiles, int router, int permute, int fold_permute) {
-    if (gemm_tiles < 0 || gemm_tiles > 3 || router < 0 || router > 2 || permute < 0 || permute > 2 ||
+    if (gemm_tiles < 0 || gemm_tiles > 4 || router < 0 || router > 2 || permute < 0 || permute > 2 ||
         fold_permute < 0 || fold_permute > 1)
         return MOE_ERR_INVALID_ARG;
     moe::g_override.gemm_tiles = gemm_tiles;
@@ -583,13 +585,6 @@ moe_status moe_layer_forward(const float* logits, const moe_bf16* x, int64_t T, 
     const int64_t A = T * k;
     const bf16* xb = reinterpret_cast<const bf16*>(x);
 
-    cudaError_t e = trace_mark(0, st);
-    bool scanned = false;
-    if (e == cudaSuccess)
-        e = launch_router_topk(logits, T, E, k, opts, L.topk_idx, L.topk_prob, nullptr, L.rs, st,
-                               err, L.counts, L.offsets, &scanned);
-    if (e == cudaSuccess && !scanned) e = launch_expert_scan(T, E, L.rs, L.counts, L.offsets, st);
-    if (e == cudaSuccess) e = trace_mark(1, st);
     // Folded permute (moe_testing_set_kernels): without a requested x_perm, on
     // single-CTA tiles, the gate_up GEMM gathers its A rows from x by token
     // (the permute computes the rows only), so the permuted copy of x is never
@@ -598,11 +593,29 @@ moe_status moe_layer_forward(const float* logits, const moe_bf16* x, int64_t T, 
     // for the Qwen3-30B-A3B forward), more than the permute's copy costs.
     const bool gather = x_perm == nullptr && grouped_gemm_single_tiles(A, E) && (H % 8) == 0 &&
                         kernel_override().fold_permute != 0;
+    // A small batch (an expert gets at most T <= 64 rows, and the experts that
+    // can hold rows have as many gate_up tiles as there are SMs) runs gate_up
+    // and down as one launch; the router or the scan zeroes its counters.
+    const bool fused_mlp = !gather && use_fused_mlp(A, E, T, I);
+    int32_t* zero = fused_mlp ? L.sched : nullptr;
+    const int n_zero = fused_mlp ? E + 1 : 0;
+
+    cudaError_t e = trace_mark(0, st);
+    bool scanned = false;
+    if (e == cudaSuccess)
+        e = launch_router_topk(logits, T, E, k, opts, L.topk_idx, L.topk_prob, nullptr, L.rs, st,
+                               err, L.counts, L.offsets, &scanned, zero, n_zero);
+    if (e == cudaSuccess && !scanned) e = launch_expert_scan(T, E, L.rs, L.counts, L.offsets, st, zero, n_zero);
+    if (e == cudaSuccess) e = trace_mark(1, st);
     if (e == cudaSuccess)
         e = launch_permute(xb, T, H, L.topk_idx, k, L.offsets, E, L.rs, gather ? nullptr : L.x_perm,
                            L.sorted_token, L.row_of, st, err);
     if (e == cudaSuccess) e = trace_mark(2, st);
-    if (e == cudaSuccess)
+    if (e == cudaSuccess && fused_mlp)
+        e = gemm_expert_mlp_fused(L.x_perm, A, L.offsets, E, H, I, reinterpret_cast<const bf16*>(w_gate_up),
+                                  reinterpret_cast<const bf16*>(w_down), L.h, reinterpret_cast<bf16*>(gu), L.y_perm,
+                                  L.sched, T, st, err);   // the down stage's trace mark follows at once
+    else if (e == cudaSuccess)
         e = gather ? gemm_gate_up_swiglu_gather(xb, T, L.sorted_token, A, L.offsets, E, H, I,
                                                 reinterpret_cast<const bf16*>(w_gate_up), L.h,
                                                 reinterpret_cast<bf16*>(gu), st, err)
@@ -610,7 +623,7 @@ moe_status moe_layer_forward(const float* logits, const moe_bf16* x, int64_t T, 
                                          reinterpret_cast<const bf16*>(w_gate_up), L.h,
                                          reinterpret_cast<bf16*>(gu), st, err, nullptr, T);
     if (e == cudaSuccess) e = trace_mark(3, st);
-    if (e == cudaSuccess)
+    if (e == cudaSuccess && !fused_mlp)
         e = gemm_down(L.h, A, L.offsets, E, H, I, reinterpret_cast<const bf16*>(w_down), L.y_perm,
                       st, err, T);   // an expert gets at most T rows
     if (e == cudaSuccess) e = trace_mark(4, st);

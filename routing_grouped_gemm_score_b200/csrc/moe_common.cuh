@@ -173,6 +173,38 @@ __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// The same ordering between generic-proxy accesses of global memory and later
+// TMA accesses of it.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int32_t* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Waits until the counter *c (written by other CTAs) reaches `target`, with
+// acquire semantics. Gives up after kWaitLimitNs, or at once when *abort is
+// set; on a timeout it records kErrTimeout and sets *abort. Returns false if
+// it gave up.
+__device__ __forceinline__ bool wait_count(const int32_t* c, int target, volatile int* abort, unsigned* err) {
+    if (ld_acquire_gpu(c) >= target) return true;
+    const unsigned long long start = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        __nanosleep(64);
+        if (ld_acquire_gpu(c) >= target) return true;
+        if ((it & 15u) == 0) {
+            if (*abort) return false;
+            if (global_timer_ns() - start > kWaitLimitNs) {
+                raise_error(err, kErrTimeout);
+                *abort = 1;
+                return false;
+            }
+        }
+    }
+}
 
 // TMA tiled store from shared memory (bulk group), its commit and waits.
 // Elements of the box outside the tensor's extent are not written.

@@ -75,12 +75,13 @@ RouteScratch carve_route_scratch(void* base, int64_t T, int E, int k);
 
 // With counts and offsets given and a single token block (T <= 8 tokens), the
 // router also writes the counts and offsets and sets *scanned; otherwise
-// launch_expert_scan must follow.
+// launch_expert_scan must follow. Whichever writes the offsets also sets
+// zero[0 .. n_zero) to 0 (the fused expert MLP's schedule counters; NULL: none).
 cudaError_t launch_router_topk(const float* logits, int64_t T, int E, int k,
                                const moe_router_opts& opts, int32_t* topk_idx, float* topk_prob,
                                uint8_t* routing_map, const RouteScratch& rs, cudaStream_t st,
                                unsigned* err, int32_t* counts = nullptr, int32_t* offsets = nullptr,
-                               bool* scanned = nullptr);
+                               bool* scanned = nullptr, int32_t* zero = nullptr, int n_zero = 0);
 cudaError_t launch_router_backward(const float* logits, int64_t T, int E, int k, const moe_router_opts& opts,
                                    const int32_t* topk_idx, const float* dprob, float* dlogits,
                                    cudaStream_t st, unsigned* err);
@@ -95,9 +96,10 @@ cudaError_t launch_aux_loss_backward(const float* logits, int64_t T, int E, int 
                                      int accumulate, cudaStream_t st);
 cudaError_t launch_rank_from_indices(const int32_t* topk_idx, int64_t T, int E, int k,
                                      const RouteScratch& rs, cudaStream_t st, unsigned* err);
-// Turns block counts into exclusive prefixes; writes counts/offsets if given.
+// Turns block counts into exclusive prefixes; writes counts/offsets if given,
+// and then sets zero[0 .. n_zero) to 0 (NULL: none).
 cudaError_t launch_expert_scan(int64_t T, int E, const RouteScratch& rs, int32_t* counts,
-                               int32_t* offsets, cudaStream_t st);
+                               int32_t* offsets, cudaStream_t st, int32_t* zero = nullptr, int n_zero = 0);
 // Padded dispatch (Token permutation, Padding and alignment).
 cudaError_t launch_pad_offsets(const int32_t* offsets, int E, int align, int32_t* padded_offsets, cudaStream_t st);
 cudaError_t launch_pad_fill(const int32_t* offsets, const int32_t* padded_offsets, int E, int H, bf16* x_perm,
@@ -146,6 +148,16 @@ cudaError_t gemm_gate_up_swiglu_gather(const bf16* x, int64_t T, const int32_t* 
                                        const int32_t* offsets, int E, int H, int I, const bf16* w_gate_up, bf16* h,
                                        bf16* gu_save, cudaStream_t st, unsigned* err,
                                        const float* row_scale = nullptr);
+// The expert MLP of a small batch in one launch (gemm_swap_mlp_kernel):
+// h = SwiGLU(x W_gate_up) (and gu = [g | u] if gu_save), then y = h W_down,
+// on swap-AB tiles. Every expert must hold at most max_group_rows <= 64 rows
+// (a layer call passes T). sched: E + 1 int32 that are zero when the launch
+// starts (the router or the scan zeroes them). use_fused_mlp says whether a
+// call of this many rows, groups and columns of h takes it.
+bool use_fused_mlp(int64_t rows, int groups, int64_t max_group_rows, int I);
+cudaError_t gemm_expert_mlp_fused(const bf16* x, int64_t rows, const int32_t* offsets, int E, int H, int I,
+                                  const bf16* w_gate_up, const bf16* w_down, bf16* h, bf16* gu_save, bf16* y,
+                                  int32_t* sched, int64_t max_group_rows, cudaStream_t st, unsigned* err);
 // Whether the forward gate_up GEMM runs on single-CTA 128-row tiles (not CTA
 // pairs, not swap-AB tiles) for this many rows and groups.
 bool grouped_gemm_single_tiles(int64_t rows, int groups);

@@ -59,6 +59,8 @@ struct RouterArgs {
     // offsets, so that no scan kernel follows (NULL: the scan kernel does)
     int32_t* counts;
     int32_t* offsets;
+    int32_t* zero;   // with counts: zero[0 .. n_zero) is set to 0 as well
+    int n_zero;
 };
 
 // After the token loop: thread e counts, in token order, the assignments of
@@ -294,6 +296,7 @@ __global__ void __launch_bounds__(kRouteThreads) router_topk_kernel(const Router
         const int incl = block_inclusive_scan(cnt, warp_tot, total);
         if (e < E) a.offsets[e + 1] = incl;
         if (e == 0) a.offsets[0] = 0;
+        for (int i = threadIdx.x; i < a.n_zero; i += blockDim.x) a.zero[i] = 0;
     }
 }
 
@@ -882,7 +885,7 @@ __device__ __forceinline__ int scan_slot(int i) { return (i / kScanPerThread) * 
 // block to finish also writes offsets (exclusive scan of the expert counts).
 __global__ void __launch_bounds__(1024)
     expert_scan_kernel(int32_t* block_base, int nb, int E, int32_t* counts, int32_t* offsets,
-                       unsigned* ticket) {
+                       unsigned* ticket, int32_t* zero, int n_zero) {
     pdl_wait();
     pdl_launch_dependents();
     __shared__ int warp_tot[32];
@@ -944,6 +947,7 @@ __global__ void __launch_bounds__(1024)
         if (base == 0 && threadIdx.x == 0) offsets[0] = 0;
         carry_off += total;
     }
+    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero[i] = 0;
     if (threadIdx.x == 0) *ticket = 0u;
 }
 
@@ -953,7 +957,8 @@ __global__ void __launch_bounds__(1024)
 // counts into the offsets. A small batch then pays for one block instead of E.
 constexpr int kScanSmallBlocks = 32;
 __global__ void __launch_bounds__(1024)
-    expert_scan_small_kernel(int32_t* block_base, int nb, int E, int32_t* counts, int32_t* offsets) {
+    expert_scan_small_kernel(int32_t* block_base, int nb, int E, int32_t* counts, int32_t* offsets, int32_t* zero,
+                             int n_zero) {
     pdl_wait();
     pdl_launch_dependents();
     __shared__ int cnt[256];
@@ -984,6 +989,7 @@ __global__ void __launch_bounds__(1024)
         if (base == 0 && threadIdx.x == 0) offsets[0] = 0;
         carry += total;
     }
+    for (int i = threadIdx.x; i < n_zero; i += blockDim.x) zero[i] = 0;
 }
 
 // Permute over contiguous token ranges, on plain 16-byte loads and stores. A
@@ -1244,7 +1250,8 @@ cudaError_t launch_router_k(const RouterArgs& a, dim3 grid, dim3 block, cudaStre
 cudaError_t launch_router_topk(const float* logits, int64_t T, int E, int k,
                                const moe_router_opts& opts, int32_t* topk_idx, float* topk_prob,
                                uint8_t* routing_map, const RouteScratch& rs, cudaStream_t st,
-                               unsigned* err, int32_t* counts, int32_t* offsets, bool* scanned) {
+                               unsigned* err, int32_t* counts, int32_t* offsets, bool* scanned, int32_t* zero,
+                               int n_zero) {
     if (scanned) *scanned = false;
     RouterArgs a;
     a.logits = logits;
@@ -1265,6 +1272,8 @@ cudaError_t launch_router_topk(const float* logits, int64_t T, int E, int k,
     a.tpb = route_tokens_per_block(T);
     a.counts = nullptr;
     a.offsets = nullptr;
+    a.zero = nullptr;
+    a.n_zero = 0;
     // Large T: the lane-per-token kernel where it applies. moe_testing_set_kernels
     // can force either kernel (the tests run both on the same inputs).
     const int force = kernel_override().router;
@@ -1299,6 +1308,8 @@ cudaError_t launch_router_topk(const float* logits, int64_t T, int E, int k,
     if (a.nb == 1 && counts != nullptr && offsets != nullptr) {   // one token block: no scan kernel
         a.counts = counts;
         a.offsets = offsets;
+        a.zero = zero;
+        a.n_zero = zero ? n_zero : 0;
         if (scanned) *scanned = true;
     }
     if (E <= 32) return launch_router_k<1>(a, grid, block, st);
@@ -1342,15 +1353,17 @@ cudaError_t launch_rank_from_indices(const int32_t* topk_idx, int64_t T, int E, 
 }
 
 cudaError_t launch_expert_scan(int64_t T, int E, const RouteScratch& rs, int32_t* counts,
-                               int32_t* offsets, cudaStream_t st) {
+                               int32_t* offsets, cudaStream_t st, int32_t* zero, int n_zero) {
     const int nb = (int)route_blocks(T);
+    if (!counts) zero = nullptr;   // the kernels return before the offsets without counts
+    if (!zero) n_zero = 0;
     if (nb <= kScanSmallBlocks)
         return launch_chained(expert_scan_small_kernel, dim3(1), dim3(1024), 0, st, rs.block_base, nb, E, counts,
-                              offsets);
+                              offsets, zero, n_zero);
     int threads = 32;
     while (threads * kScanPerThread < nb && threads < 1024) threads <<= 1;
     return launch_chained(expert_scan_kernel, dim3(E), dim3(threads), 0, st, rs.block_base, nb, E, counts, offsets,
-                          rs.ticket);
+                          rs.ticket, zero, n_zero);
 }
 
 cudaError_t launch_pad_offsets(const int32_t* offsets, int E, int align, int32_t* padded_offsets, cudaStream_t st) {

@@ -223,10 +223,12 @@ def force_kernels(gemm_tiles=None, router=None, permute=None, fold_permute=None)
     (moe_testing_set_kernels) for the rest of the current test; conftest.py
     restores the library's own choice after each test. Values: gemm_tiles
     "single" | "pair", router "warp" | "lane", permute "tokens" | "warp",
-    fold_permute True | False ("swap": the forward GEMMs on swap-AB tiles);
+    fold_permute True | False ("swap": the forward GEMMs on swap-AB tiles,
+    "swap_unfused": the same with a layer's gate_up and down as two launches);
     "auto" or None leaves a setting as it is."""
     import routing_grouped_gemm_score_b200 as m
-    names = {"gemm_tiles": {"auto": 0, "single": m.GEMM_SINGLE, "pair": m.GEMM_PAIR, "swap": m.GEMM_SWAP},
+    names = {"gemm_tiles": {"auto": 0, "single": m.GEMM_SINGLE, "pair": m.GEMM_PAIR, "swap": m.GEMM_SWAP,
+                            "swap_unfused": m.GEMM_SWAP_UNFUSED},
              "router": {"auto": 0, "warp": m.ROUTER_WARP, "lane": m.ROUTER_LANE},
              "permute": {"auto": 0, "tokens": m.PERMUTE_TOKENS, "warp": m.PERMUTE_WARP}}
     for key, val in (("gemm_tiles", gemm_tiles), ("router", router), ("permute", permute)):

@@ -55,7 +55,7 @@ SMALL = {
 }
 
 
-@pytest.mark.parametrize("tiles", ["auto", "single", "pair", "swap"])
+@pytest.mark.parametrize("tiles", ["auto", "single", "pair", "swap", "swap_unfused"])
 @pytest.mark.parametrize("name", list(SMALL))
 def test_layer_forward_matches_per_token_definition(name, tiles, monkeypatch):
     helpers.force_kernels(gemm_tiles=tiles)
@@ -64,6 +64,45 @@ def test_layer_forward_matches_per_token_definition(name, tiles, monkeypatch):
     out = layer(w, d)
     tokens = np.arange(w.T)
     helpers.assert_close_flips(out, oracle_out(w, d), helpers.lazy_forward_terms(w, d, tokens), f"{name}: out")
+
+
+# every expert at most 64 rows (T <= 64): gate_up and down in one launch
+FUSED_MLP = {
+    "tiny": SMALL["tiny"],                       # 64-row token tiles, E = 8
+    "skew_small": SMALL["skew_small"],           # T = 64 over 128 experts, 16 dead
+    "t12": SMALL["t12"],                         # 16-row token tiles
+    "odd_t12": SMALL["odd_t12"],                 # H = 200, I = 136: partial tiles
+    "t1": wl.WORKLOADS["skew_t1"].scaled(H=256, I=192),
+    "t8_shared": wl.WORKLOADS["skew_t8"].scaled(H=256, I=320, shared_expert=True),
+}
+
+
+@pytest.mark.parametrize("name", list(FUSED_MLP))
+def test_fused_small_batch_mlp_is_bit_identical_to_two_launches(name):
+    """For a small batch the layer can compute gate_up + SwiGLU and down in
+    one launch (the down tiles wait for their expert's h through a device
+    counter; forced here with "swap", which the library otherwise takes only
+    when the gate_up tiles can fill the SMs). Each output element comes from
+    the same tile arithmetic as on the two-launch path, so the output and the
+    saved state agree bit for bit; the result is then also checked against
+    the oracle."""
+    w = FUSED_MLP[name]
+    d = wl.make_inputs(w, "cuda")
+    runs = []
+    for tiles in ("swap", "swap_unfused", "swap", "auto"):
+        helpers.force_kernels(gemm_tiles=tiles)
+        out, st = layer(w, d, save=True)
+        runs.append((out.clone(), {key: v.clone() for key, v in st.items()}))
+    for out, st in runs[1:]:
+        assert torch.equal(out.view(torch.int16), runs[0][0].view(torch.int16)), f"{name}: out"
+        for key, v in st.items():
+            a = runs[0][1][key]
+            as_int = a.view(torch.int16) if a.dtype == torch.bfloat16 else a.view(torch.int32)
+            other = v.view(torch.int16) if v.dtype == torch.bfloat16 else v.view(torch.int32)
+            assert torch.equal(as_int, other), f"{name}: {key}"
+    tokens = np.arange(w.T)
+    helpers.assert_close_flips(runs[0][0], oracle_out(w, d), helpers.lazy_forward_terms(w, d, tokens),
+                               f"{name}: out (one launch)")
 
 
 SHARED = {
