@@ -16,9 +16,10 @@ JSON line.
 The default workload is the largest single-GPU one, the Llama-4-17Bx16E-shaped
 forward with its shared expert. On one GPU the line also carries the other
 workloads under "workloads": the Mixtral-8x7B-shaped forward, the
-Qwen3-30B-A3B-shaped forward + backward, and the skewed sweep at T = 1, 8, 64
-and 16384 (each of these small batches timed with L2 flushed before every
-step, since their weights can fit in L2).
+Qwen3-30B-A3B-shaped forward + backward, the skewed sweep at T = 1, 8, 64
+and 16384, and the 64-token tie case, whose near-tied logits spread the
+batch over most experts (each batch of at most 64 tokens timed with L2
+flushed before every step, since their weights can fit in L2).
 
 With N > 1 (torchrun), each rank runs its own replica of the layer on its own
 tokens (data-parallel replicas; the forward has no exchange step). value =
@@ -46,7 +47,7 @@ METRIC = "MoE layer tokens/s and grouped-GEMM TFLOP/s (% of B200 bf16 peak), 1 G
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "llama4_17bx16e"
 NOMINAL_BF16_TFLOPS = 2250.0   # dense bf16 tensor peak of one B200 (vendor figure, no sparsity)
-EXTRA_WORKLOADS = ["mixtral_8x7b", "qwen3_30b_a3b", "skew_t1", "skew_t8", "skew_t64", "skew_t16384"]
+EXTRA_WORKLOADS = ["mixtral_8x7b", "qwen3_30b_a3b", "skew_t1", "skew_t8", "skew_t64", "skew_t16384", "tie_t64"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
