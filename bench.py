@@ -365,7 +365,7 @@ class Layer:
 
     def launches(self):
         # router, scan (done by the router itself for one token block, T <= 8),
-        # permute, gate_up, down (one launch with gate_up when every expert has
+        # permute (also done by the router there for at most 64 KB of rows), gate_up, down (one launch with gate_up when every expert has
         # at most T <= 64 rows on swap-AB tiles and the experts that can hold
         # rows have at least one gate_up tile per SM), combine; the shared expert's
         # two GEMMs (the combine then folded into the second, above 16 tokens);
@@ -375,8 +375,10 @@ class Layer:
         sms = torch.cuda.get_device_properties(0).multi_processor_count
         fused_mlp = (w.T <= 64 and w.T * w.k <= 16 * w.E and w.E <= 256
                      and min(w.E, w.T * w.k) * -(-w.I // 64) >= sms)
-        return (6 - (1 if w.T <= 8 else 0) - (1 if fused_mlp else 0) + (2 if w.shared_expert else 0)
-                - (1 if combine_folded(w) else 0) + (6 if w.backward else 0))
+        # the router's one token block (T <= 8) also permutes up to 64 KB of rows
+        router_permutes = w.T <= 8 and w.T * w.k * w.H * 2 <= 65536
+        return (6 - (1 if w.T <= 8 else 0) - (1 if router_permutes else 0) - (1 if fused_mlp else 0)
+                + (2 if w.shared_expert else 0) - (1 if combine_folded(w) else 0) + (6 if w.backward else 0))
 
 
 def _events(n):

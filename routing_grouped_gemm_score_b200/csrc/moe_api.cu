@@ -601,13 +601,17 @@ moe_status moe_layer_forward(const float* logits, const moe_bf16* x, int64_t T, 
     const int n_zero = fused_mlp ? E + 1 : 0;
 
     cudaError_t e = trace_mark(0, st);
-    bool scanned = false;
+    bool scanned = false, permuted = false;
+    // one token block (T <= 8): the router also writes the counts and offsets
+    // (no scan launch), and for at most 64 KB of rows the permuted rows too (no
+    // permute launch)
     if (e == cudaSuccess)
         e = launch_router_topk(logits, T, E, k, opts, L.topk_idx, L.topk_prob, nullptr, L.rs, st,
-                               err, L.counts, L.offsets, &scanned, zero, n_zero);
+                               err, L.counts, L.offsets, &scanned, zero, n_zero, xb, H, gather ? nullptr : L.x_perm,
+                               L.sorted_token, L.row_of, gather ? nullptr : &permuted);
     if (e == cudaSuccess && !scanned) e = launch_expert_scan(T, E, L.rs, L.counts, L.offsets, st, zero, n_zero);
     if (e == cudaSuccess) e = trace_mark(1, st);
-    if (e == cudaSuccess)
+    if (e == cudaSuccess && !permuted)
         e = launch_permute(xb, T, H, L.topk_idx, k, L.offsets, E, L.rs, gather ? nullptr : L.x_perm,
                            L.sorted_token, L.row_of, st, err);
     if (e == cudaSuccess) e = trace_mark(2, st);

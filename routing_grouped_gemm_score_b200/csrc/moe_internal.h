@@ -77,11 +77,17 @@ RouteScratch carve_route_scratch(void* base, int64_t T, int E, int k);
 // router also writes the counts and offsets and sets *scanned; otherwise
 // launch_expert_scan must follow. Whichever writes the offsets also sets
 // zero[0 .. n_zero) to 0 (the fused expert MLP's schedule counters; NULL: none).
+// When the router writes them, x, x_perm, sorted_token, row_of and permuted
+// are given and the permuted rows take at most 64 KB, it also does the permute
+// (x [T][H] into x_perm [T k][H]) and sets *permuted; otherwise
+// launch_permute must follow.
 cudaError_t launch_router_topk(const float* logits, int64_t T, int E, int k,
                                const moe_router_opts& opts, int32_t* topk_idx, float* topk_prob,
                                uint8_t* routing_map, const RouteScratch& rs, cudaStream_t st,
                                unsigned* err, int32_t* counts = nullptr, int32_t* offsets = nullptr,
-                               bool* scanned = nullptr, int32_t* zero = nullptr, int n_zero = 0);
+                               bool* scanned = nullptr, int32_t* zero = nullptr, int n_zero = 0,
+                               const bf16* x = nullptr, int H = 0, bf16* x_perm = nullptr,
+                               int32_t* sorted_token = nullptr, int32_t* row_of = nullptr, bool* permuted = nullptr);
 cudaError_t launch_router_backward(const float* logits, int64_t T, int E, int k, const moe_router_opts& opts,
                                    const int32_t* topk_idx, const float* dprob, float* dlogits,
                                    cudaStream_t st, unsigned* err);

@@ -140,9 +140,18 @@ def test_combine_in_the_shared_expert_gemm(name):
     assert_close(out2, ref, f"{name}: out, combine kernel after the stored shared output")
 
 
-def test_layer_forward_saved_state_and_empty_batch():
+# T <= 8 is one token block: the router kernel also writes the offsets (no
+# scan launch), and up to 64 KB of permuted rows (no permute launch; t8 has
+# 8 x 8 rows of 512 B, t1_odd 8 rows of 400 B)
+STATE = {"qwen3_small": SMALL["qwen3_small"],
+         "t8": SMALL["qwen3_small"].scaled(T=8),
+         "t1_odd": SMALL["odd_dims"].scaled(T=1)}
+
+
+@pytest.mark.parametrize("name", list(STATE))
+def test_layer_forward_saved_state_and_empty_batch(name):
     import routing_grouped_gemm_score_b200 as m
-    w = SMALL["qwen3_small"]
+    w = STATE[name]
     d = wl.make_inputs(w, "cuda")
     out, st = layer(w, d, save=True)
     r = oracle.router_topk(d["logits"].cpu().numpy(), w.k)
