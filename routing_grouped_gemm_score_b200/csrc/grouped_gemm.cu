@@ -12,7 +12,9 @@
 // tiles when the average expert block is large (>= 1024 rows, or a single dense
 // group), else on single-CTA 128-row tiles, which round ragged blocks up less
 // (use_pair_tiles); the forward GEMMs of small batches (<= 16 rows per expert
-// on average) run on swap-AB tiles (gemm_swap_kernel, use_swap_tiles).
+// on average) run on swap-AB tiles (gemm_swap_kernel, use_swap_tiles), and a
+// layer's gate_up and down GEMMs for at most 64 rows per expert can run as
+// one launch of such tiles (gemm_swap_mlp_kernel, use_fused_mlp).
 //
 // gemm_pair_kernel (group-M: forward and dgrad). Clusters of two CTAs on two
 // SMs compute 256 x 256 output tiles with tcgen05.mma.cta_group::2 (M=256,
