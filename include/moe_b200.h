@@ -353,6 +353,9 @@ moe_status moe_unpermute_combine_rows(const moe_bf16* y_perm, int64_t y_rows, co
  * weighted, j ascending, rounded to bf16 once (TE Token combine; the shared
  * expert's output is then not stored as bf16 before the sum). Otherwise the
  * combine kernel adds the stored bf16 shared output.
+ * For one token block (T <= 8) the router kernel also writes the counts and
+ * offsets, and, when the permuted rows take at most 64 KB, the rows
+ * themselves (no scan or permute launch).
  * With at most T <= 64 rows per expert on swap-AB tiles, where the experts
  * that can hold rows (min(E, T k)) have at least one gate_up tile (64 columns
  * of h) per SM, the gate_up and down GEMMs run as one launch: a down tile
