@@ -95,7 +95,8 @@ moe_status moe_get_device_status(void* stream);
  *   [4] down   [5] shared expert (recorded even without one)  [6] combine
  * (with the combine folded into the shared expert's down GEMM, see
  * moe_layer_forward, the stage [5]..[6] is empty and [4]..[5] holds it; with
- * gate_up and down in one launch, [3]..[4] is empty and [2]..[3] holds both);
+ * gate_up and down in one launch, [3]..[4] is empty and [2]..[3] holds both;
+ * with the permute done by the router kernel, [1]..[2] is empty);
  * moe_grouped_mlp_backward and moe_grouped_mlp_scaled_backward record:
  *   [0] start  [1] combine backward  [2] down dgrad + SwiGLU backward
  *   [3] gate_up dgrad  [4] token sum of dx  [5] down wgrad  [6] gate_up wgrad
