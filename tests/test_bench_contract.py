@@ -40,3 +40,17 @@ def test_reference_line_has_every_key():
                            "d2h_bytes_per_step": 0}
     cfg = line["config"]
     assert cfg["workload"] == "tiny" and cfg["parallelism"] == "single GPU"
+
+
+def test_every_extra_workload_is_defined_and_small_batches_are_flushed():
+    """The workloads the GPU line carries under "workloads" exist, and each
+    batch of at most 64 tokens (whose weights can fit in L2) is one that the
+    bench times with L2 flushed before every step."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as wl
+    assert bench.DEFAULT_WORKLOAD not in bench.EXTRA_WORKLOADS
+    for name in bench.EXTRA_WORKLOADS:
+        assert name in wl.WORKLOADS, name
+    small = [n for n in bench.EXTRA_WORKLOADS if wl.WORKLOADS[n].T <= 64]
+    assert {"skew_t1", "skew_t8", "skew_t64", "tie_t64"} <= set(small)
